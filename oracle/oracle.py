@@ -1,0 +1,278 @@
+"""Python face of the CPU oracle (bsq_oracle.c).
+
+TEST INFRASTRUCTURE ONLY: imported by tests/, by ``__graft_entry__.smoke()``
+and by the CPU-baseline leg of ``bench.py``.  The library in fp8_math_b200/
+never imports this module, and this module imports nothing from it.
+
+The C file is compiled on first use (gcc, ``-O2 -ffp-contract=off
+-fno-fast-math``) into ``oracle/liboracle.so``; ``build()`` does the same
+ahead of time.  Arrays are numpy; bf16 tensors travel as ``uint16`` bit
+patterns.  Each wrapper names the C function whose header comment cites the
+page and section it follows.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "bsq_oracle.c")
+_SO = os.path.join(_HERE, "liboracle.so")
+_CFLAGS = ["-std=c11", "-O2", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared"]
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle into oracle/liboracle.so (if missing or stale)."""
+    if force or not os.path.exists(_SO) or os.path.getmtime(_SO) < os.path.getmtime(_SRC):
+        tmp = _SO + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", *_CFLAGS, "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _SO)
+    return _SO
+
+
+_u8p = np.ctypeslib.ndpointer(np.uint8, flags="C_CONTIGUOUS")
+_u16p = np.ctypeslib.ndpointer(np.uint16, flags="C_CONTIGUOUS")
+_i32p = np.ctypeslib.ndpointer(np.int32, flags="C_CONTIGUOUS")
+_i64p = np.ctypeslib.ndpointer(np.int64, flags="C_CONTIGUOUS")
+_f32p = np.ctypeslib.ndpointer(np.float32, flags="C_CONTIGUOUS")
+_f64p = np.ctypeslib.ndpointer(np.float64, flags="C_CONTIGUOUS")
+_u32p = np.ctypeslib.ndpointer(np.uint32, flags="C_CONTIGUOUS")
+_i64 = C.c_int64
+
+
+def lib():
+    global _lib
+    with _lock:
+        if _lib is None:
+            L = C.CDLL(build())
+            sig = {
+                "ora_bf16_to_f32": (C.c_float, [C.c_uint16]),
+                "ora_f32_to_bf16": (C.c_uint16, [C.c_float]),
+                "ora_e2m1_value": (C.c_float, [C.c_uint8]),
+                "ora_e2m1_rne_sat": (C.c_uint8, [C.c_float]),
+                "ora_e4m3_value": (C.c_float, [C.c_uint8]),
+                "ora_e4m3_rne_sat": (C.c_uint8, [C.c_float]),
+                "ora_e8m0_value": (C.c_float, [C.c_uint8]),
+                "ora_e4m3_sr": (C.c_uint8, [C.c_float, C.c_uint16]),
+                "ora_philox4x32_10": (None, [_u32p, _u32p, _u32p]),
+                "ora_sr_draw": (C.c_uint16, [C.c_uint64, C.c_uint32, C.c_uint64]),
+                "ora_rht_sign_mask": (C.c_uint16, [C.c_uint64]),
+                "ora_rht16": (None, [_f32p, C.c_uint16, _f32p]),
+                "ora_rht_bf16": (C.c_int, [_u16p, _u16p, _i64, _i64, _i64, C.c_uint16]),
+                "ora_amax": (C.c_float, [_u16p, _i64, _i64, _i64, C.c_int, C.c_uint16, C.c_void_p]),
+                "ora_nvfp4_global_scale": (C.c_float, [C.c_float]),
+                "ora_quant_nvfp4": (C.c_int, [_u16p, _i64, _i64, _i64, C.c_int, C.c_int, C.c_int,
+                                              C.c_uint16, C.c_void_p, C.c_void_p, _f32p, _u8p, _u8p]),
+                "ora_quant_mxfp8": (C.c_int, [_u16p, _i64, _i64, _i64, C.c_int, C.c_int,
+                                              C.c_uint64, C.c_uint32, _u8p, _u8p]),
+                "ora_requant_transpose": (C.c_int, [_u8p, _u8p, _i64, _i64, C.c_int, C.c_uint64,
+                                                    C.c_uint32, _u8p, _u8p]),
+                "ora_sf_swizzled_bytes": (_i64, [_i64, _i64]),
+                "ora_sf_offset": (_i64, [_i64, _i64, _i64]),
+                "ora_sf_swizzle": (None, [_u8p, _i64, _i64, _u8p]),
+                "ora_sf_unswizzle": (None, [_u8p, _i64, _i64, _u8p]),
+                "ora_dequant": (None, [C.c_int, _u8p, _u8p, C.c_float, _i64, _i64, _f64p]),
+                "ora_gemm_f64": (None, [_f64p, _f64p, _i64, _i64, _i64, _f64p, _f64p]),
+                "ora_gemm_points": (None, [C.c_int, _u8p, _u8p, C.c_float, _u8p, _u8p, C.c_float,
+                                           _i64, _i64, _i64p, _i64p, _f64p, _f64p]),
+            }
+            for name, (res, args) in sig.items():
+                f = getattr(L, name)
+                f.restype = res
+                f.argtypes = args
+            _lib = L
+    return _lib
+
+
+def _c(a, dtype):
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(C.c_void_p)
+
+
+# ---------------------------------------------------------------- formats
+def bf16_to_f32(b):
+    b = _c(b, np.uint16)
+    return (b.astype(np.uint32) << 16).view(np.float32)
+
+
+def f32_to_bf16(f):
+    return np.array([lib().ora_f32_to_bf16(float(v)) for v in np.ravel(f)], np.uint16).reshape(np.shape(f))
+
+
+def e2m1_value(code):
+    return lib().ora_e2m1_value(int(code))
+
+
+def e2m1_rne_sat(v):
+    return lib().ora_e2m1_rne_sat(float(np.float32(v)))
+
+
+def e4m3_value(code):
+    return lib().ora_e4m3_value(int(code))
+
+
+def e4m3_rne_sat(v):
+    return lib().ora_e4m3_rne_sat(float(np.float32(v)))
+
+
+def e8m0_value(code):
+    return lib().ora_e8m0_value(int(code))
+
+
+def e4m3_sr(v, r16):
+    return lib().ora_e4m3_sr(float(np.float32(v)), int(r16))
+
+
+# ---------------------------------------------------------------- random
+def philox4x32_10(ctr, key):
+    out = np.zeros(4, np.uint32)
+    lib().ora_philox4x32_10(_c(ctr, np.uint32), _c(key, np.uint32), out)
+    return out
+
+
+def sr_draw(seed, stream_id, idx):
+    return lib().ora_sr_draw(int(seed), int(stream_id), int(idx))
+
+
+def rht_sign_mask(seed):
+    return lib().ora_rht_sign_mask(int(seed))
+
+
+# ---------------------------------------------------------------- transforms
+def rht16(x16, mask):
+    y = np.zeros(16, np.float32)
+    lib().ora_rht16(_c(x16, np.float32), int(mask), y)
+    return y
+
+
+def rht_bf16(x, mask):
+    x = _c(x, np.uint16)
+    M, K = x.shape
+    y = np.zeros_like(x)
+    if lib().ora_rht_bf16(x, y, M, K, K, int(mask)):
+        raise ValueError("K must be a multiple of 16")
+    return y
+
+
+def amax(x, rht_mask=None, row_index=None):
+    x = _c(x, np.uint16)
+    M, K = x.shape
+    ri = None if row_index is None else _c(row_index, np.int32)
+    rows = M if ri is None else ri.shape[0]
+    return lib().ora_amax(x, rows, K, K, int(rht_mask is not None), int(rht_mask or 0), _ptr(ri))
+
+
+def nvfp4_global_scale(a):
+    return lib().ora_nvfp4_global_scale(float(a))
+
+
+def quant_nvfp4(x, block_2d=False, four_over_six=False, rht_mask=None, row_index=None, amax_in=None):
+    """NVFP4 quantize (ora_quant_nvfp4).  Returns (codes [R,K/2] u8, sf [R,K/16] u8, s_g)."""
+    x = _c(x, np.uint16)
+    M, K = x.shape
+    ri = None if row_index is None else _c(row_index, np.int32)
+    R = M if ri is None else ri.shape[0]
+    codes = np.zeros((R, K // 2), np.uint8)
+    sf = np.zeros((R, K // 16), np.uint8)
+    sg = np.zeros(1, np.float32)
+    am = None if amax_in is None else np.array([amax_in], np.float32)
+    rc = lib().ora_quant_nvfp4(x, R, K, K, int(block_2d), int(four_over_six), int(rht_mask is not None),
+                               int(rht_mask or 0), _ptr(ri), _ptr(am), sg, codes, sf)
+    if rc:
+        raise ValueError("unsupported NVFP4 shape/options")
+    return codes, sf, float(sg[0])
+
+
+def quant_mxfp8(x, colwise=False, sr=False, seed=0, stream_id=0):
+    """MXFP8 quantize (ora_quant_mxfp8).  Returns (codes, sf) in the output orientation."""
+    x = _c(x, np.uint16)
+    M, K = x.shape
+    R, Cc = (K, M) if colwise else (M, K)
+    codes = np.zeros((R, Cc), np.uint8)
+    sf = np.zeros((R, Cc // 32), np.uint8)
+    if lib().ora_quant_mxfp8(x, M, K, K, int(colwise), int(sr), int(seed), int(stream_id), codes, sf):
+        raise ValueError("unsupported MXFP8 shape")
+    return codes, sf
+
+
+def requant_transpose(codes, sf, sr=True, seed=0, stream_id=1):
+    codes = _c(codes, np.uint8)
+    sf = _c(sf, np.uint8)
+    M, K = codes.shape
+    cc = np.zeros((K, M), np.uint8)
+    sc = np.zeros((K, M // 32), np.uint8)
+    if lib().ora_requant_transpose(codes, sf, M, K, int(sr), int(seed), int(stream_id), cc, sc):
+        raise ValueError("unsupported requant shape")
+    return cc, sc
+
+
+# ---------------------------------------------------------------- layout
+def sf_swizzled_bytes(rows, nblk):
+    return lib().ora_sf_swizzled_bytes(rows, nblk)
+
+
+def sf_offset(r, b, nblk):
+    return lib().ora_sf_offset(r, b, nblk)
+
+
+def sf_swizzle(sf):
+    sf = _c(sf, np.uint8)
+    rows, nblk = sf.shape
+    out = np.zeros(sf_swizzled_bytes(rows, nblk), np.uint8)
+    lib().ora_sf_swizzle(sf, rows, nblk, out)
+    return out
+
+
+def sf_unswizzle(buf, rows, nblk):
+    out = np.zeros((rows, nblk), np.uint8)
+    lib().ora_sf_unswizzle(_c(buf, np.uint8), rows, nblk, out)
+    return out
+
+
+# ---------------------------------------------------------------- GEMM
+NVFP4, MXFP8 = 0, 1
+
+
+def dequant(fmt, codes, sf, s_g=1.0):
+    codes = _c(codes, np.uint8)
+    sf = _c(sf, np.uint8)
+    R = codes.shape[0]
+    K = codes.shape[1] * (2 if fmt == NVFP4 else 1)
+    out = np.zeros((R, K), np.float64)
+    lib().ora_dequant(int(fmt), codes, sf, float(s_g), R, K, out)
+    return out
+
+
+def gemm_f64(A, B):
+    """C = A B^T and sum |A||B| in binary64 (ora_gemm_f64)."""
+    A = _c(A, np.float64)
+    B = _c(B, np.float64)
+    M, K = A.shape
+    N = B.shape[0]
+    Cm = np.zeros((M, N), np.float64)
+    Ra = np.zeros((M, N), np.float64)
+    lib().ora_gemm_f64(A, B, M, N, K, Cm, Ra)
+    return Cm, Ra
+
+
+def gemm_points(fmt, qa, qb, K, pm, pn):
+    """C and sum|.| at points (pm[i], pn[i]); qa/qb = (codes, sf, s_g)."""
+    ca, sa, ga = qa
+    cb, sb, gb = qb
+    pm = _c(pm, np.int64)
+    pn = _c(pn, np.int64)
+    Cm = np.zeros(pm.shape[0], np.float64)
+    Ra = np.zeros(pm.shape[0], np.float64)
+    lib().ora_gemm_points(int(fmt), _c(ca, np.uint8), _c(sa, np.uint8), float(ga),
+                          _c(cb, np.uint8), _c(sb, np.uint8), float(gb), int(K),
+                          pm.shape[0], pm, pn, Cm, Ra)
+    return Cm, Ra

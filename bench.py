@@ -1,0 +1,336 @@
+"""Benchmark: one step of the NVFP4 linear with RHT (8192x14336x4096) on B200.
+
+A step is the whole hot path for that workload, in the library's kernels:
+  amax(RHT(A)) -> NVFP4 1x16 quantize of RHT(A)          (bsq_quant_nvfp4)
+  amax(RHT(W)) -> NVFP4 16x16 quantize of RHT(W)         (bsq_quant_nvfp4)
+  C = A W^T, tcgen05 block-scaled GEMM, bf16 output       (bsq_gemm_blockscaled)
+value = 2*M*N*K / step time (TFLOP/s, whole job over all ranks).  Inputs (A
+and W in bf16, 176 MiB) are larger than L2, so no flush is needed.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+With N > 1 it runs under torchrun, one independent replica per GPU (weak
+scaling, no collective on the data path); rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+M, N, K = 8192, 14336, 4096
+RHT_SEED = 2
+METRIC = "NVFP4 GEMM TFLOPS (% of 9 PF FP4); quantize GB/s (% of HBM peak), 1×B200"
+WORKLOAD = "nvfp4_linear_rht: A 8192x4096 N(0,1) w/ 0.5% channels x100, W 14336x4096 N(0,0.02), 16x16 RHT seed 2"
+NOMINAL_FP4_OVER_BF16 = 4.0   # 9 PF / 2.25 PF dense (B200 table on the pages)
+FALLBACK_HBM, FALLBACK_BF16 = 6650.0, 1590.0
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+    return FALLBACK_HBM, FALLBACK_BF16, "fallback"
+
+
+# ---------------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML every ~2 ms."""
+
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4, "hw_slowdown": 0x8,
+        "sync_boost": 0x10, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+        "hw_power_brake_slowdown": 0x80, "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, index):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nv = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for name, bit in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self.nv:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self.nv:
+            self.t.join()
+
+    def summary(self):
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons - {"gpu_idle"}),
+                "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------- oracle
+def cpu_oracle_step(rows_a=1024, rows_w=2048):
+    """The oracle on a bounded sample of the workload: the first rows_a rows of
+    A and rows_w rows of W quantized (amax + RHT + NVFP4), then their GEMM in
+    binary64.  Returns (seconds, flops of the sample)."""
+    import numpy as np
+    from fp8_math_b200 import workloads as W
+    from oracle import oracle as ora
+    A, Wt, seed = W.nvfp4_linear_rht(M=rows_a, N=rows_w, K=K)
+    mask = ora.rht_sign_mask(seed)
+    xa, xw = W.bf16_bits(A), W.bf16_bits(Wt)
+    t0 = time.perf_counter()
+    qa = ora.quant_nvfp4(xa, rht_mask=mask)
+    qw = ora.quant_nvfp4(xw, block_2d=True, rht_mask=mask)
+    ora.gemm_f64(ora.dequant(0, *qa), ora.dequant(0, *qw))
+    dt = time.perf_counter() - t0
+    del np
+    return dt, 2.0 * rows_a * rows_w * K
+
+
+def reference_arm(args, rank):
+    if rank != 0:
+        return
+    sys.path.insert(0, ROOT)
+    from oracle import oracle as ora
+    ora.build()
+    for _ in range(args.warmup):
+        cpu_oracle_step(rows_a=32, rows_w=64)
+    times, flops = [], 0.0
+    for _ in range(args.steps):
+        dt, fl = cpu_oracle_step(rows_a=32, rows_w=64)
+        times.append(dt)
+        flops = fl
+    tot = sum(times)
+    value = flops * args.steps / tot / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "M": M, "N": N, "K": K},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
+                         "sample": "per step: amax+RHT+NVFP4 quantize of 32 rows of A and 64 rows of W (K=4096), "
+                                   "then their 32x64x4096 binary64 GEMM; single-threaded C oracle"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------- ours
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        return reference_arm(args, rank)
+
+    import torch
+    import torch.distributed as dist
+
+    from fp8_math_b200 import api, bsq
+    from fp8_math_b200 import workloads as W
+
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+
+    # ---- inputs (seeded, resident in HBM before timing)
+    A_h, W_h, seed = W.nvfp4_linear_rht()
+    mask = bsq.bsq_rht_sign_mask(seed)
+    A = A_h.cuda()
+    Wd = W_h.cuda()
+    dev = A.device
+    KB = K // 16
+    ca = torch.empty(M, K // 2, dtype=torch.uint8, device=dev)
+    sa = torch.zeros(bsq.bsq_sf_bytes(M, KB), dtype=torch.uint8, device=dev)
+    ga = torch.empty(1, dtype=torch.float32, device=dev)
+    cw = torch.empty(N, K // 2, dtype=torch.uint8, device=dev)
+    sw = torch.zeros(bsq.bsq_sf_bytes(N, KB), dtype=torch.uint8, device=dev)
+    gw = torch.empty(1, dtype=torch.float32, device=dev)
+    Cm = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream()
+    s_ptr = stream.cuda_stream
+
+    def q_a():
+        bsq.bsq_quant_nvfp4(A, M, K, K, 0, 0, 1, mask, None, 0, None, None, None, ga, ca, sa, s_ptr)
+
+    def q_w():
+        bsq.bsq_quant_nvfp4(Wd, N, K, K, 1, 0, 1, mask, None, 0, None, None, None, gw, cw, sw, s_ptr)
+
+    def gemm():
+        bsq.bsq_gemm_blockscaled(bsq.BSQ_NVFP4, ca, sa, ga, cw, sw, gw, M, N, K, Cm, N, bsq.BSQ_OUT_BF16, s_ptr)
+
+    def step():
+        q_a()
+        q_w()
+        gemm()
+
+    launches_per_step = 7  # per operand: amax, quantize, finalize; plus the GEMM
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st = bsq.bsq_check()
+    if st != bsq.BSQ_OK:
+        raise RuntimeError("device error in warm-up: " + bsq.status_str(st))
+
+    # ---- per-kernel breakdown (events on the launching stream)
+    def time_fn(fn, reps):
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+        for e0, e1 in evs:
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        return [e0.elapsed_time(e1) for e0, e1 in evs]
+
+    # ---- the timed region
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    gemm_ms, qa_ms, qw_ms = [], [], []
+    with ClockSampler(local) as clk:
+        t0.record(stream)
+        for _ in range(args.steps):
+            step()
+        t1.record(stream)
+        torch.cuda.synchronize()
+        # breakdown pass (same calls, one event pair each; not part of ms_per_step)
+        reps = max(10, min(args.steps, 50))
+        qa_ms = time_fn(q_a, reps)
+        qw_ms = time_fn(q_w, reps)
+        gemm_ms = time_fn(gemm, reps)
+    if world > 1:
+        dist.barrier()
+    ms = t0.elapsed_time(t1) / args.steps
+    st = bsq.bsq_check()
+    if st != bsq.BSQ_OK:
+        raise RuntimeError("device error in timed region: " + bsq.status_str(st))
+    if world > 1:
+        tt = torch.tensor([ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+
+    flops = 2.0 * M * N * K
+    value = world * flops / (ms * 1e-3) / 1e12
+
+    # ---- end to end through the C ABI with host buffers (pinned), copies timed
+    A_pin = A_h.pin_memory()
+    W_pin = W_h.pin_memory()
+    C_pin = torch.empty(M, N, dtype=torch.bfloat16).pin_memory()
+    e2e_steps = max(3, min(args.steps, 10))
+
+    def e2e_step():
+        A.copy_(A_pin, non_blocking=True)
+        Wd.copy_(W_pin, non_blocking=True)
+        step()
+        C_pin.copy_(Cm, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    if world > 1:
+        tt = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tt.item())
+
+    hbm, bf16, src = peaks()
+    fp4_peak = bf16 * NOMINAL_FP4_OVER_BF16
+    g_ms = statistics.mean(gemm_ms)
+    gemm_tflops = flops / (g_ms * 1e-3) / 1e12
+    # algorithmic bytes of a quantize call (amax pass + quantize pass): 2 B read
+    # for the amax, then 2 B read + 0.5 B codes + 1/16 B scales per element
+    qa_bytes = M * K * (2 + 2 + 0.5 + 1 / 16)
+    qw_bytes = N * K * (2 + 2 + 0.5 + 1 / 16)
+    qa_gbs = qa_bytes / (statistics.mean(qa_ms) * 1e-3) / 1e9
+    qw_gbs = qw_bytes / (statistics.mean(qw_ms) * 1e-3) / 1e9
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        from oracle import oracle as ora
+        ora.build()
+        dt, fl = cpu_oracle_step()
+        cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
+               "sample": "amax+RHT+NVFP4 quantize of the first 1024 rows of A and 2048 rows of W (K=4096), then "
+                         "their 1024x2048x4096 binary64 GEMM; single-threaded C oracle",
+               "seconds": dt}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "nvfp4", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "M": M, "N": N, "K": K, "out": "bf16",
+                       "l2": "inputs larger than L2 (A+W bf16 = 176 MiB > 126 MB); no flush",
+                       "parallelism": f"replicas x{world}"},
+            "roofline": {"bound": "tensor", "achieved": gemm_tflops, "peak": fp4_peak, "unit": "TFLOP/s",
+                         "frac": gemm_tflops / fp4_peak, "traffic": None,
+                         "kernel": "gemm_bs_kernel (NVFP4 8192x14336x4096)",
+                         "peak_source": f"{src} bf16 burst {bf16} x {NOMINAL_FP4_OVER_BF16} (nominal FP4/BF16)"},
+            "breakdown": {
+                "gemm_ms": g_ms, "gemm_tflops": gemm_tflops, "gemm_frac_of_9pf": gemm_tflops / 9000.0,
+                "quant_A_ms": statistics.mean(qa_ms), "quant_A_gbs": qa_gbs,
+                "quant_W_ms": statistics.mean(qw_ms), "quant_W_gbs": qw_gbs,
+                "quant_frac_of_hbm": {"A": qa_gbs / hbm, "W": qw_gbs / hbm, "hbm_gbs": hbm, "source": src},
+            },
+            "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": (M + N) * K * 2, "d2h_bytes_per_step": M * N * 2,
+                    "ms_per_step": e2e_ms},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clk.summary(),
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,97 @@
+"""Allocating convenience wrappers over the C ABI (torch tensors in and out).
+
+Each helper allocates its output tensors on the input's device with
+``torch.empty`` and calls one libbsq entry point through ``fp8_math_b200.bsq``;
+all arithmetic runs in the library's CUDA kernels.  Shapes and layouts are
+those of include/bsq.h.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import bsq
+
+
+def sf_bytes(rows: int, nblocks: int) -> int:
+    return bsq.bsq_sf_bytes(rows, nblocks)
+
+
+def _ld(x: torch.Tensor) -> int:
+    assert x.dim() == 2 and x.stride(1) == 1, "row-major 2-D tensor expected"
+    return x.stride(0)
+
+
+def amax(x, rht_mask=None, row_index=None, out=None):
+    M = x.shape[0] if row_index is None else row_index.shape[0]
+    out = torch.empty(1, dtype=torch.float32, device=x.device) if out is None else out
+    bsq.bsq_amax(x, M, x.shape[1], _ld(x), rht_mask is not None, rht_mask or 0, row_index, out)
+    return out
+
+
+def quant_nvfp4(x, block_2d=False, four_over_six=False, rht_mask=None, row_index=None, groups=None,
+                amax_in=None, out=None):
+    """Returns (codes [R, K/2] uint8, sf swizzled uint8, global_scale [1] fp32).
+    groups = (row_offsets int32 [G+1], sf_row_offsets int32 [G+1], sf_rows)."""
+    K = x.shape[1]
+    R = x.shape[0] if row_index is None else row_index.shape[0]
+    G, ro, so = 0, None, None
+    sf_rows = R
+    if groups is not None:
+        ro, so, sf_rows = groups
+        G = ro.shape[0] - 1
+    if out is None:
+        codes = torch.empty(R, K // 2, dtype=torch.uint8, device=x.device)
+        sf = torch.zeros(sf_bytes(sf_rows, K // 16), dtype=torch.uint8, device=x.device)
+        gs = torch.empty(1, dtype=torch.float32, device=x.device)
+    else:
+        codes, sf, gs = out
+    bsq.bsq_quant_nvfp4(x, R, K, _ld(x), block_2d, four_over_six, rht_mask is not None, rht_mask or 0, row_index,
+                        G, ro, so, amax_in, gs, codes, sf)
+    return codes, sf, gs
+
+
+def quant_mxfp8(x, colwise=False, sr=False, seed=0, stream_id=0, out=None):
+    """Returns (codes, sf swizzled) in the output orientation ([M,K] or [K,M])."""
+    M, K = x.shape
+    R, Cc = (K, M) if colwise else (M, K)
+    if out is None:
+        codes = torch.empty(R, Cc, dtype=torch.uint8, device=x.device)
+        sf = torch.zeros(sf_bytes(R, Cc // 32), dtype=torch.uint8, device=x.device)
+    else:
+        codes, sf = out
+    bsq.bsq_quant_mxfp8(x, M, K, _ld(x), colwise, bsq.BSQ_SR if sr else bsq.BSQ_RNE, seed, stream_id, codes, sf)
+    return codes, sf
+
+
+def rht(x, mask, out=None):
+    y = torch.empty_like(x) if out is None else out
+    bsq.bsq_rht(x, y, x.shape[0], x.shape[1], _ld(x), _ld(y), mask)
+    return y
+
+
+def requant_transpose(codes_row, sf_row, sr=True, seed=0, stream_id=1, out=None):
+    M, K = codes_row.shape
+    if out is None:
+        cc = torch.empty(K, M, dtype=torch.uint8, device=codes_row.device)
+        sc = torch.zeros(sf_bytes(K, M // 32), dtype=torch.uint8, device=codes_row.device)
+    else:
+        cc, sc = out
+    bsq.bsq_requant_transpose(codes_row, sf_row, M, K, bsq.BSQ_SR if sr else bsq.BSQ_RNE, seed, stream_id, cc, sc)
+    return cc, sc
+
+
+def gemm(fmt, A, sfA, B, sfB, M, N, K, gsA=None, gsB=None, out_dtype=torch.bfloat16, out=None):
+    C_out = torch.empty(M, N, dtype=out_dtype, device=A.device) if out is None else out
+    ot = bsq.BSQ_OUT_BF16 if C_out.dtype == torch.bfloat16 else bsq.BSQ_OUT_F32
+    bsq.bsq_gemm_blockscaled(fmt, A, sfA, gsA, B, sfB, gsB, M, N, K, C_out, C_out.stride(0), ot)
+    return C_out
+
+
+def grouped_gemm(fmt, row_offsets, sf_row_offsets, A, sfA, B, sfB, M_total, N, K, gsA=None, gsB=None,
+                 out_dtype=torch.bfloat16, out=None):
+    G = row_offsets.shape[0] - 1
+    C_out = torch.empty(M_total, N, dtype=out_dtype, device=A.device) if out is None else out
+    ot = bsq.BSQ_OUT_BF16 if C_out.dtype == torch.bfloat16 else bsq.BSQ_OUT_F32
+    bsq.bsq_grouped_gemm(fmt, G, row_offsets, sf_row_offsets, M_total, A, sfA, gsA, B, sfB, gsB, N, K, C_out,
+                         C_out.stride(0), ot)
+    return C_out

@@ -1,0 +1,242 @@
+// api.cu -- the C entry points of libbsq (include/bsq.h): argument
+// validation, per-device state (SM count, error word), kernel launches.
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "common.cuh"
+#include "gemm.cuh"
+#include "quant.cuh"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceState {
+    bool ready = false;
+    int num_sms = 0;
+    unsigned int *err = nullptr;  // device error word
+};
+
+std::mutex g_mu;
+DeviceState g_dev[kMaxDevices];
+
+// Per-device state for the current device; created on first use.
+int device_state(DeviceState **out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return BSQ_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_mu);
+    DeviceState &d = g_dev[dev];
+    if (!d.ready) {
+        if (cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return BSQ_ERR_CUDA;
+        if (cudaMalloc(&d.err, sizeof(unsigned int)) != cudaSuccess) return BSQ_ERR_CUDA;
+        if (cudaMemset(d.err, 0, sizeof(unsigned int)) != cudaSuccess) return BSQ_ERR_CUDA;
+        d.ready = true;
+    }
+    *out = &d;
+    return BSQ_OK;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int launch_status() { return cudaGetLastError() == cudaSuccess ? BSQ_OK : BSQ_ERR_CUDA; }
+
+// Philox4x32-10 on the host (Salmon et al., SC'11).
+void philox_host(uint32_t c[4], uint32_t k0, uint32_t k1) {
+    for (int r = 0; r < 10; r++) {
+        if (r) {
+            k0 += 0x9E3779B9u;
+            k1 += 0xBB67AE85u;
+        }
+        uint64_t p0 = (uint64_t)0xD2511F53u * c[0];
+        uint64_t p1 = (uint64_t)0xCD9E8D57u * c[2];
+        uint32_t n0 = (uint32_t)(p1 >> 32) ^ c[1] ^ k0, n1 = (uint32_t)p1;
+        uint32_t n2 = (uint32_t)(p0 >> 32) ^ c[3] ^ k1, n3 = (uint32_t)p0;
+        c[0] = n0; c[1] = n1; c[2] = n2; c[3] = n3;
+    }
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *bsq_status_str(int status) {
+    switch (status) {
+        case BSQ_OK: return "ok";
+        case BSQ_ERR_INVALID: return "invalid argument";
+        case BSQ_ERR_ALIGN: return "misaligned pointer or leading dimension";
+        case BSQ_ERR_UNSUPPORTED: return "unsupported request";
+        case BSQ_ERR_CUDA: return "CUDA error";
+        case BSQ_ERR_TIMEOUT: return "device-side wait timed out";
+        default: return "unknown status";
+    }
+}
+
+size_t bsq_sf_bytes(int64_t rows, int64_t nblocks) {
+    if (rows < 0 || nblocks < 0) return 0;
+    return (size_t)((rows + 127) / 128 * 128) * (size_t)((nblocks + 3) / 4 * 4);
+}
+
+uint16_t bsq_rht_sign_mask(uint64_t seed) {
+    uint32_t c[4] = {0u, 0u, 0u, 0u};
+    philox_host(c, (uint32_t)seed, (uint32_t)(seed >> 32));
+    return (uint16_t)(c[0] & 0xFFFFu);
+}
+
+int bsq_amax(const void *x, int64_t M, int64_t K, int64_t ldx, int rht_enable, uint16_t mask,
+             const int32_t *row_index, float *amax_dev, void *stream) {
+    if (!x || !amax_dev || M < 0 || K < 0 || K % 16 || ldx < K) return BSQ_ERR_INVALID;
+    if (!aligned16(x) || ldx % 8 || (reinterpret_cast<uintptr_t>(amax_dev) & 3u)) return BSQ_ERR_ALIGN;
+    DeviceState *d;
+    if (int st = device_state(&d)) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(amax_dev, 0, sizeof(float), s) != cudaSuccess) return BSQ_ERR_CUDA;
+    if (M == 0 || K == 0) return BSQ_OK;
+    bsq::launch_amax(static_cast<const uint16_t *>(x), M, K, ldx, rht_enable != 0, mask, row_index,
+                     reinterpret_cast<unsigned int *>(amax_dev), d->num_sms, s);
+    return launch_status();
+}
+
+int bsq_quant_nvfp4(const void *x, int64_t M, int64_t K, int64_t ldx, int block_2d, int four_over_six,
+                    int rht_enable, uint16_t mask, const int32_t *row_index, int G, const int32_t *row_off,
+                    const int32_t *sf_off, const float *amax_in, float *gs, uint8_t *codes, uint8_t *sf,
+                    void *stream) {
+    if (!x || !gs || !codes || !sf || M < 0 || K < 0 || K % 16 || ldx < K || G < 0) return BSQ_ERR_INVALID;
+    if (block_2d && (M % 16 || four_over_six || G > 0)) return BSQ_ERR_INVALID;
+    if (G > 0 && (!row_off || !sf_off)) return BSQ_ERR_INVALID;
+    if (!aligned16(x) || !aligned16(codes) || !aligned16(sf) || ldx % 8 ||
+        (reinterpret_cast<uintptr_t>(gs) & 3u) || (amax_in && (reinterpret_cast<uintptr_t>(amax_in) & 3u)))
+        return BSQ_ERR_ALIGN;
+    DeviceState *d;
+    if (int st = device_state(&d)) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const uint16_t *xx = static_cast<const uint16_t *>(x);
+    // Without an amax from the caller, the amax is accumulated in *gs, read
+    // by the quantize kernel, and finally replaced by s_g in place.
+    const bool in_place = (amax_in == nullptr) || (amax_in == gs);
+    if (amax_in == nullptr) {
+        if (cudaMemsetAsync(gs, 0, sizeof(float), s) != cudaSuccess) return BSQ_ERR_CUDA;
+        if (M > 0 && K > 0)
+            bsq::launch_amax(xx, M, K, ldx, rht_enable != 0, mask, row_index, reinterpret_cast<unsigned int *>(gs),
+                             d->num_sms, s);
+    }
+    const float *amax_ptr = amax_in ? amax_in : gs;
+    if (M > 0 && K > 0)
+        bsq::launch_quant_nvfp4(xx, M, K, ldx, block_2d != 0, four_over_six != 0, rht_enable != 0, mask, row_index,
+                                G, row_off, sf_off, amax_ptr, gs, !in_place, codes, sf, d->num_sms, s);
+    if (in_place || M == 0 || K == 0) bsq::launch_finalize_global_scale(gs, s);
+    return launch_status();
+}
+
+int bsq_quant_mxfp8(const void *x, int64_t M, int64_t K, int64_t ldx, int colwise, int rounding, uint64_t seed,
+                    uint32_t stream_id, uint8_t *codes, uint8_t *sf, void *stream) {
+    if (!x || !codes || !sf || M < 0 || K < 0 || ldx < K || (rounding != BSQ_RNE && rounding != BSQ_SR))
+        return BSQ_ERR_INVALID;
+    if (colwise ? (M % 32 || K % 8) : (K % 32)) return BSQ_ERR_INVALID;
+    if (!aligned16(x) || !aligned16(codes) || !aligned16(sf) || ldx % 8) return BSQ_ERR_ALIGN;
+    if (colwise && M % 16) return BSQ_ERR_ALIGN;
+    DeviceState *d;
+    if (int st = device_state(&d)) return st;
+    if (M == 0 || K == 0) return BSQ_OK;
+    bsq::launch_quant_mxfp8(static_cast<const uint16_t *>(x), M, K, ldx, colwise != 0, rounding == BSQ_SR, seed,
+                            stream_id, codes, sf, d->num_sms, static_cast<cudaStream_t>(stream));
+    return launch_status();
+}
+
+int bsq_rht(const void *x, void *y, int64_t M, int64_t K, int64_t ldx, int64_t ldy, uint16_t mask, void *stream) {
+    if (!x || !y || M < 0 || K < 0 || K % 16 || ldx < K || ldy < K) return BSQ_ERR_INVALID;
+    if (!aligned16(x) || !aligned16(y) || ldx % 8 || ldy % 8) return BSQ_ERR_ALIGN;
+    if (x == y && ldx != ldy) return BSQ_ERR_INVALID;
+    DeviceState *d;
+    if (int st = device_state(&d)) return st;
+    if (M == 0 || K == 0) return BSQ_OK;
+    bsq::launch_rht(static_cast<const uint16_t *>(x), static_cast<uint16_t *>(y), M, K, ldx, ldy, mask, d->num_sms,
+                    static_cast<cudaStream_t>(stream));
+    return launch_status();
+}
+
+int bsq_requant_transpose(const uint8_t *codes_row, const uint8_t *sf_row, int64_t M, int64_t K, int rounding,
+                          uint64_t seed, uint32_t stream_id, uint8_t *codes_col, uint8_t *sf_col, void *stream) {
+    if (!codes_row || !sf_row || !codes_col || !sf_col || M < 0 || K < 0 || M % 32 || K % 32 ||
+        (rounding != BSQ_RNE && rounding != BSQ_SR))
+        return BSQ_ERR_INVALID;
+    if (!aligned16(codes_row) || !aligned16(sf_row) || !aligned16(codes_col) || !aligned16(sf_col))
+        return BSQ_ERR_ALIGN;
+    DeviceState *d;
+    if (int st = device_state(&d)) return st;
+    if (M == 0 || K == 0) return BSQ_OK;
+    bsq::launch_requant_transpose(codes_row, sf_row, M, K, rounding == BSQ_SR, seed, stream_id, codes_col, sf_col,
+                                  d->num_sms, static_cast<cudaStream_t>(stream));
+    return launch_status();
+}
+
+int bsq_gemm_blockscaled(int fmt, const uint8_t *A, const uint8_t *sfA, const float *gsA, const uint8_t *B,
+                         const uint8_t *sfB, const float *gsB, int64_t M, int64_t N, int64_t K, void *C, int64_t ldc,
+                         int out_type, void *stream) {
+    if ((fmt != BSQ_NVFP4 && fmt != BSQ_MXFP8) || (out_type != BSQ_OUT_F32 && out_type != BSQ_OUT_BF16))
+        return BSQ_ERR_INVALID;
+    if (!A || !sfA || !B || !sfB || !C || M < 1 || N < 1 || K < 128 || K % 128 || ldc < N) return BSQ_ERR_INVALID;
+    if (M > (1LL << 31) - 1 || N > (1LL << 31) - 1 || K > (1LL << 31) - 1) return BSQ_ERR_UNSUPPORTED;
+    if (!aligned16(A) || !aligned16(B) || !aligned16(sfA) || !aligned16(sfB) || !aligned16(C) ||
+        (ldc * (out_type == BSQ_OUT_F32 ? 4 : 2)) % 16)
+        return BSQ_ERR_ALIGN;
+    DeviceState *d;
+    if (int st = device_state(&d)) return st;
+    bsq::GemmArgs g{};
+    g.fmt = fmt;
+    g.A = A; g.sfA = sfA; g.B = B; g.sfB = sfB; g.gsA = gsA; g.gsB = gsB;
+    g.M = M; g.N = N; g.K = K; g.C = C; g.ldc = ldc; g.out_bf16 = out_type == BSQ_OUT_BF16;
+    g.G = 0;
+    g.err = d->err;
+    g.num_sms = d->num_sms;
+    return bsq::launch_gemm(g, static_cast<cudaStream_t>(stream));
+}
+
+int bsq_grouped_gemm(int fmt, int G, const int32_t *row_off, const int32_t *sf_row_off, int64_t M_total,
+                     const uint8_t *A, const uint8_t *sfA, const float *gsA, const uint8_t *B, const uint8_t *sfB,
+                     const float *gsB, int64_t N, int64_t K, void *C, int64_t ldc, int out_type, void *stream) {
+    if ((fmt != BSQ_NVFP4 && fmt != BSQ_MXFP8) || (out_type != BSQ_OUT_F32 && out_type != BSQ_OUT_BF16))
+        return BSQ_ERR_INVALID;
+    if (G < 1 || !row_off || !sf_row_off || !A || !sfA || !B || !sfB || !C || M_total < 0 || N < 1 || K < 128 ||
+        K % 128 || ldc < N)
+        return BSQ_ERR_INVALID;
+    if (G > 1024) return BSQ_ERR_UNSUPPORTED;
+    if (!aligned16(A) || !aligned16(B) || !aligned16(sfA) || !aligned16(sfB) || !aligned16(C) ||
+        (ldc * (out_type == BSQ_OUT_F32 ? 4 : 2)) % 16)
+        return BSQ_ERR_ALIGN;
+    DeviceState *d;
+    if (int st = device_state(&d)) return st;
+    if (M_total == 0) return BSQ_OK;
+    bsq::GemmArgs g{};
+    g.fmt = fmt;
+    g.A = A; g.sfA = sfA; g.B = B; g.sfB = sfB; g.gsA = gsA; g.gsB = gsB;
+    g.M = M_total; g.N = N; g.K = K; g.C = C; g.ldc = ldc; g.out_bf16 = out_type == BSQ_OUT_BF16;
+    g.G = G; g.row_off = row_off; g.sf_row_off = sf_row_off;
+    g.err = d->err;
+    g.num_sms = d->num_sms;
+    return bsq::launch_gemm(g, static_cast<cudaStream_t>(stream));
+}
+
+int bsq_check(void *stream) {
+    DeviceState *d;
+    if (int st = device_state(&d)) return st;
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return BSQ_ERR_CUDA;
+    unsigned int w = 0;
+    if (cudaMemcpy(&w, d->err, sizeof w, cudaMemcpyDeviceToHost) != cudaSuccess) return BSQ_ERR_CUDA;
+    if (w) {
+        if (cudaMemset(d->err, 0, sizeof w) != cudaSuccess) return BSQ_ERR_CUDA;
+        return BSQ_ERR_TIMEOUT;
+    }
+    return BSQ_OK;
+}
+
+int bsq_debug_timeout_probe(uint64_t timeout_ns, void *stream) {
+    if (timeout_ns == 0 || timeout_ns > 10000000000ull) return BSQ_ERR_INVALID;
+    DeviceState *d;
+    if (int st = device_state(&d)) return st;
+    bsq::launch_timeout_probe(timeout_ns, d->err, static_cast<cudaStream_t>(stream));
+    return launch_status();
+}
+
+}  // extern "C"

@@ -1,0 +1,185 @@
+// common.cuh -- device helpers shared by the libbsq kernels: number-format
+// conversions (hand-written PTX cvt), Philox4x32-10, the MMA scale-factor
+// layout, the per-device error word.  Every floating-point step that decides
+// a code uses an explicit round-to-nearest intrinsic so that the compiler
+// cannot contract or reorder it.
+#pragma once
+#include <cstdint>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+
+#include "../../include/bsq.h"
+
+#define BSQ_DEV __device__ __forceinline__
+
+namespace bsq {
+
+// ---------------------------------------------------------------- error word
+// One 32-bit word per device: bit 0 set by a bounded wait that ran out, bits
+// 8..15 hold the site id of the first such wait.
+struct ErrWord {
+    unsigned int *ptr;
+};
+
+BSQ_DEV void report_timeout(unsigned int *err, unsigned int site) {
+    if (err) atomicOr(err, 1u | ((site & 0xFFu) << 8));
+}
+
+BSQ_DEV uint64_t globaltimer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// ---------------------------------------------------------------- bf16
+BSQ_DEV float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+BSQ_DEV float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// 16-byte streaming load of 8 bf16 -> 8 fp32
+BSQ_DEV void load8_bf16(const uint16_t *p, float v[8]) {
+    uint4 q = __ldg(reinterpret_cast<const uint4 *>(p));
+    v[0] = bf16_lo(q.x); v[1] = bf16_hi(q.x);
+    v[2] = bf16_lo(q.y); v[3] = bf16_hi(q.y);
+    v[4] = bf16_lo(q.z); v[5] = bf16_hi(q.z);
+    v[6] = bf16_lo(q.w); v[7] = bf16_hi(q.w);
+}
+
+// ---------------------------------------------------------------- E4M3 / E2M1
+// cvt.rn.satfinite.e4m3x2.f32: the first source lands in the upper byte.
+BSQ_DEV uint32_t cvt_e4m3x2(float lo, float hi) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+BSQ_DEV uint32_t e4m3_rne(float v) { return cvt_e4m3x2(v, 0.0f) & 0xFFu; }
+
+// E4M3 byte -> fp32 (exact), via cvt.rn.f16x2.e4m3x2 (low byte -> low half).
+BSQ_DEV float e4m3_to_f32(uint32_t code) {
+    uint32_t h2;
+    uint16_t in = (uint16_t)(code & 0xFFu);
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(in));
+    __half_raw hr;
+    hr.x = (unsigned short)(h2 & 0xFFFFu);
+    return __half2float(__half(hr));
+}
+
+// Two E4M3 bytes (low, high of a 16-bit word) -> two fp32.
+BSQ_DEV void e4m3x2_to_f32(uint32_t two, float &lo, float &hi) {
+    uint32_t h2;
+    uint16_t in = (uint16_t)(two & 0xFFFFu);
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(in));
+    __half_raw a, b;
+    a.x = (unsigned short)(h2 & 0xFFFFu);
+    b.x = (unsigned short)(h2 >> 16);
+    lo = __half2float(__half(a));
+    hi = __half2float(__half(b));
+}
+
+// 8 fp32 -> 8 E2M1 nibbles, element 2j in the low nibble of byte j.
+// cvt.rn.satfinite.e2m1x2.f32 d, a, b puts a in the upper nibble.
+BSQ_DEV uint32_t cvt_e2m1x8(const float q[8]) {
+    uint32_t out;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+        : "=r"(out)
+        : "f"(q[0]), "f"(q[1]), "f"(q[2]), "f"(q[3]), "f"(q[4]), "f"(q[5]), "f"(q[6]), "f"(q[7]));
+    return out;
+}
+
+// E2M1 nibble -> fp32 from the S E E M layout (bias 1; E = 0 is M * 0.5).
+BSQ_DEV float e2m1_to_f32(uint32_t code) {
+    uint32_t mag = code & 7u;
+    uint32_t bits = (mag >= 2u) ? ((((mag >> 1) + 126u) << 23) | ((mag & 1u) << 22))
+                                : (mag ? 0x3F000000u : 0u);
+    return __uint_as_float(bits | ((code & 8u) << 28));
+}
+
+// floor(log2 a) for a finite a > 0 (normal or subnormal binary32).
+BSQ_DEV int floor_log2(float a) {
+    uint32_t b = __float_as_uint(a) & 0x7FFFFFFFu;
+    int e = (int)(b >> 23);
+    if (e) return e - 127;
+    return (31 - __clz((int)b)) - 149;
+}
+
+// 2^k as a binary32 for k in [-149, 127].
+BSQ_DEV float exp2i(int k) {
+    if (k >= -126) return __uint_as_float((uint32_t)(k + 127) << 23);
+    return __uint_as_float(1u << (k + 149));
+}
+
+// ---------------------------------------------------------------- Philox
+// Philox4x32-10 (Salmon, Moraes, Dror, Shaw, SC'11).
+BSQ_DEV uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1) {
+#pragma unroll
+    for (int r = 0; r < 10; r++) {
+        if (r) {
+            k0 += 0x9E3779B9u;
+            k1 += 0xBB67AE85u;
+        }
+        uint32_t hi0 = __umulhi(0xD2511F53u, c.x), lo0 = 0xD2511F53u * c.x;
+        uint32_t hi1 = __umulhi(0xCD9E8D57u, c.z), lo1 = 0xCD9E8D57u * c.z;
+        c = make_uint4(hi1 ^ c.y ^ k0, lo1, hi0 ^ c.w ^ k1, lo0);
+    }
+    return c;
+}
+
+// Stochastic rounding of v (already clamped to +-448) to E4M3, with the
+// 16-bit draw r16: round the magnitude up to the next E4M3 value iff
+// r16 * 2^-16 < (|v| - lo) / ulp.
+BSQ_DEV uint32_t e4m3_sr(float v, uint32_t r16) {
+    uint32_t sgn = (__float_as_uint(v) >> 24) & 0x80u;
+    float a = fabsf(v);
+    if (a == 0.0f) return sgn;
+    int fl = floor_log2(a);
+    int ue = (fl > -6 ? fl : -6) - 3;
+    float inv = exp2i(-ue), ulp = exp2i(ue);
+    float lo = __fmul_rn(floorf(__fmul_rn(a, inv)), ulp);
+    float frac = __fmul_rn(__fsub_rn(a, lo), inv);
+    float u = __fmul_rn((float)r16, 1.0f / 65536.0f);
+    float mag = (u < frac) ? __fadd_rn(lo, ulp) : lo;
+    return sgn | e4m3_rne(mag);
+}
+
+// ---------------------------------------------------------------- RHT
+// In-place 16-point transform y = 1/4 * H16 * diag(s) * x; butterflies of
+// stride 1, 2, 4, 8 (Sylvester order).
+BSQ_DEV void rht16(float v[16], uint32_t mask) {
+#pragma unroll
+    for (int i = 0; i < 16; i++)
+        if ((mask >> i) & 1u) v[i] = -v[i];
+#pragma unroll
+    for (int h = 1; h < 16; h <<= 1) {
+#pragma unroll
+        for (int base = 0; base < 16; base += 2 * h) {
+#pragma unroll
+            for (int i = base; i < base + h; i++) {
+                float a = v[i], b = v[i + h];
+                v[i] = __fadd_rn(a, b);
+                v[i + h] = __fsub_rn(a, b);
+            }
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < 16; i++) v[i] = __fmul_rn(0.25f, v[i]);
+}
+
+// ---------------------------------------------------------------- SF layout
+// Byte offset of (row r, block b) in a swizzled SF buffer whose rows hold
+// nblk blocks: 512-byte atoms of 128 rows x 4 blocks, row-tile major.
+BSQ_DEV int64_t sf_offset(int64_t r, int64_t b, int64_t nblk) {
+    int64_t bt = (nblk + 3) >> 2;
+    return (((r >> 7) * bt + (b >> 2)) << 9) + ((r & 31) << 4) + (((r >> 5) & 3) << 2) + (b & 3);
+}
+// Offset of the 4-byte word holding blocks 4j..4j+3 of row r.
+BSQ_DEV int64_t sf_word_offset(int64_t r, int64_t b4, int64_t nblk) {
+    int64_t bt = (nblk + 3) >> 2;
+    return (((r >> 7) * bt + b4) << 9) + ((r & 31) << 4) + (((r >> 5) & 3) << 2);
+}
+
+}  // namespace bsq

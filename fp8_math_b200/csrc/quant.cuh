@@ -1,0 +1,24 @@
+// quant.cuh -- host-side launchers of the codec kernels (quant.cu).
+#pragma once
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace bsq {
+
+void launch_amax(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, bool rht, uint32_t mask,
+                 const int32_t *row_index, unsigned int *amax_bits, int num_sms, cudaStream_t s);
+void launch_finalize_global_scale(float *gs, cudaStream_t s);
+void launch_quant_nvfp4(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, bool block_2d, bool fos,
+                        bool rht, uint32_t mask, const int32_t *row_index, int G, const int32_t *row_off,
+                        const int32_t *sf_off, const float *amax_ptr, float *gs_out, bool write_gs,
+                        uint8_t *codes, uint8_t *sf, int num_sms, cudaStream_t s);
+void launch_quant_mxfp8(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, bool colwise, bool sr,
+                        uint64_t seed, uint32_t stream_id, uint8_t *codes, uint8_t *sf, int num_sms,
+                        cudaStream_t s);
+void launch_requant_transpose(const uint8_t *codes_row, const uint8_t *sf_row, int64_t M, int64_t K, bool sr,
+                              uint64_t seed, uint32_t stream_id, uint8_t *codes_col, uint8_t *sf_col,
+                              int num_sms, cudaStream_t s);
+void launch_rht(const uint16_t *x, uint16_t *y, int64_t M, int64_t K, int64_t ldx, int64_t ldy, uint32_t mask,
+                int num_sms, cudaStream_t s);
+
+}  // namespace bsq

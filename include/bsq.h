@@ -1,0 +1,196 @@
+/*
+ * bsq.h -- libbsq: block-scaled quantization (NVFP4, MXFP8), the 16-point
+ * random Hadamard transform and block-scaled GEMMs for NVIDIA B200
+ * (sm_100a).  Plain C ABI: device pointers, sizes, a stream handle.
+ *
+ * Formats (web pages cited by title and section):
+ *  - NVFP4 -- "Microscaling (MX) and block-scaled 4-bit formats", section
+ *    "NVFP4"; "08 -- FP4, MXFP4, NVFP4: The Blackwell Frontier", table "The
+ *    two Blackwell formats": E2M1 elements in blocks of 16, one E4M3 scale
+ *    per block, one FP32 per-tensor scale.  Codes are packed two per byte,
+ *    element 2j in the low nibble of byte j.
+ *  - MXFP8 -- "LMSYS and humans& ... low-precision recipes", section "Recipe
+ *    1: End-to-end MXFP8": 32 consecutive E4M3 share one E8M0 scale.
+ *  - Scale-factor ("SF") buffers are written in the layout the Blackwell
+ *    block-scaled MMA reads ("Microscaling ...", section "Hardware and
+ *    kernels": a block-scaled GEMM needs a particular scale-factor layout):
+ *    128-row x 4-block atoms of 512 bytes; row r, block b of an atom sits at
+ *    byte (r % 32) * 16 + (r / 32) * 4 + b; atoms are ordered row-tile major,
+ *    then block tile; rows pad to 128 and blocks to 4.  bsq_sf_bytes() gives
+ *    the size.  Padding bytes are never written by the quantizers.
+ *
+ * Conventions for every entry point:
+ *  - Pointers named *_dev, and all tensor pointers, are DEVICE pointers on
+ *    the current device, allocated and owned by the caller; none is retained
+ *    after the call returns.  Tensor pointers must be 16-byte aligned.
+ *  - bf16 matrices are row-major with a leading dimension in elements (ld*),
+ *    which must be a multiple of 8.
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream).  Every call
+ *    only enqueues work on it: it never synchronizes and returns a bsq status
+ *    from host-side argument validation alone (an invalid call launches
+ *    nothing).  Faults found on the device (a bounded wait that ran out) are
+ *    recorded in a per-device error word that bsq_check() reads.
+ *  - The library allocates no device memory on these paths except, once per
+ *    device, the 4-byte error word (created on first use).
+ *  - Inputs must be finite; nonzero magnitudes below 2^-100 are outside the
+ *    supported range for NVFP4 (codes there are unspecified).
+ */
+#ifndef BSQ_H
+#define BSQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define BSQ_API __attribute__((visibility("default")))
+#else
+#define BSQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum {
+    BSQ_OK = 0,
+    BSQ_ERR_INVALID = 1,     /* bad size, null pointer or option mix */
+    BSQ_ERR_ALIGN = 2,       /* pointer or leading dimension misaligned */
+    BSQ_ERR_UNSUPPORTED = 3, /* valid request this build does not handle */
+    BSQ_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed */
+    BSQ_ERR_TIMEOUT = 5      /* a device-side bounded wait ran out */
+};
+
+enum { BSQ_RNE = 0, BSQ_SR = 1 };          /* rounding for MXFP8 outputs */
+enum { BSQ_NVFP4 = 0, BSQ_MXFP8 = 1 };     /* GEMM operand format */
+enum { BSQ_OUT_F32 = 0, BSQ_OUT_BF16 = 1 }; /* GEMM output type */
+
+/* Human-readable name of a status code (static string). */
+BSQ_API const char *bsq_status_str(int status);
+
+/* Bytes of a swizzled scale-factor buffer for `rows` rows of `nblocks`
+ * blocks: roundup(rows,128) * roundup(nblocks,4).  Host-only helper. */
+BSQ_API size_t bsq_sf_bytes(int64_t rows, int64_t nblocks);
+
+/* RHT sign vector for a seed: bits 0..15 of word 0 of Philox4x32-10 with
+ * counter 0 and key (lo32(seed), hi32(seed)) (Salmon et al., SC'11); bit i
+ * set means s_i = -1.  Host-only helper, no device work. */
+BSQ_API uint16_t bsq_rht_sign_mask(uint64_t seed);
+
+/* Tensor amax: *amax_dev = max |x| over the M x K bf16 matrix x (rows
+ * selected through row_index[0..M) when it is not NULL), after the 16-point
+ * RHT along K when rht_enable != 0 (see bsq_rht).  This is the first level of
+ * NVFP4's two-level scale ("Microscaling ...", section "NVFP4").
+ * K % 16 == 0.  *amax_dev is overwritten (zeroed on the stream first). */
+BSQ_API int bsq_amax(const void *x_bf16, int64_t M, int64_t K, int64_t ldx,
+             int rht_enable, uint16_t rht_sign_mask, const int32_t *row_index_dev,
+             float *amax_dev, void *stream);
+
+/* NVFP4 quantize ("Microscaling ...", section "NVFP4"; "Thinking Machines
+ * ... Inkling 2 Small", section "A precision choice for each stage" for Four
+ * Over Six).  Output row i is input row row_index[i] (or i when row_index is
+ * NULL); with rht_enable the 16-point RHT along K is applied first (fp32).
+ *   s_g = amax / 2688 (amax = 0 gives s_g = 1); amax is *amax_in_dev, or is
+ *         computed here when amax_in_dev is NULL (the amax is then
+ *         accumulated in *global_scale_dev, which finally holds s_g);
+ *   per block (1x16 along K, or a 16x16 tile with block_2d):
+ *         s_b = E4M3_RNE((block_amax / 6) / s_g), r = 1 / (s_b * s_g),
+ *         code = E2M1_RNE_sat(x * r); s_b == 0 gives all-zero codes;
+ *   four_over_six (1x16 only): also try block_amax / 4 and keep it when its
+ *         squared error (pairwise fp32 sum over the 16 elements) is lower.
+ * Outputs: *global_scale_dev = s_g; codes [M][K/2] bytes (row stride K/2);
+ * sf swizzled.  With G > 0 the rows form G groups (MoE experts): group e
+ * owns output rows [row_offsets[e], row_offsets[e+1]) and its SF rows start
+ * at sf_row_offsets[e] (a multiple of 128); both arrays are device int32
+ * [G+1], and sf must hold sf_row_offsets[G] SF rows.
+ * Requirements: K % 16 == 0; block_2d needs M % 16 == 0 and excludes
+ * four_over_six and groups. */
+BSQ_API int bsq_quant_nvfp4(const void *x_bf16, int64_t M, int64_t K, int64_t ldx,
+                    int block_2d, int four_over_six, int rht_enable, uint16_t rht_sign_mask,
+                    const int32_t *row_index_dev,
+                    int G, const int32_t *row_offsets_dev, const int32_t *sf_row_offsets_dev,
+                    const float *amax_in_dev, float *global_scale_dev,
+                    uint8_t *codes_dev, uint8_t *sf_dev, void *stream);
+
+/* MXFP8 quantize ("LMSYS and humans& ...", section "Recipe 1"; stochastic
+ * rounding per "Microscaling ...", section "Words on this page", and
+ * "Thinking Machines ...", section "A precision choice for each stage").
+ * Per block of 32: E = clamp(floor(log2 block_amax) - 8, -127, 127), scale
+ * code E + 127 (an all-zero block has code 0); element x * 2^-E clamped to
+ * +-448, then E4M3 by nearest-even (BSQ_RNE) or stochastic rounding
+ * (BSQ_SR) with 16-bit draws from Philox4x32-10: the output element with
+ * row-major index idx (in the OUTPUT shape) uses counter (lo32(idx>>3),
+ * hi32(idx>>3), stream_id, 0), key (lo32(seed), hi32(seed)), and the low
+ * (idx even) or high (idx odd) half of word (idx>>1)&3; it rounds up iff
+ * draw * 2^-16 < the fractional position between the two neighbours.
+ * colwise == 0: blocks along K, codes [M][K], sf for M rows x K/32 blocks.
+ * colwise == 1: the quantization of x^T -- codes [K][M] (row stride M), sf
+ * for K rows x M/32 blocks.  K % 32 == 0 (row-wise); M % 32 == 0 and
+ * K % 8 == 0 (column-wise). */
+BSQ_API int bsq_quant_mxfp8(const void *x_bf16, int64_t M, int64_t K, int64_t ldx, int colwise,
+                    int rounding, uint64_t seed, uint32_t stream_id,
+                    uint8_t *codes_dev, uint8_t *sf_dev, void *stream);
+
+/* 16-point random Hadamard transform along K ("Microscaling ...", section
+ * "NVFP4"; "Thinking Machines ...", section "Why communication became the
+ * next bottleneck"): per group of 16, y = 1/4 * H16 * diag(s) * x with H16
+ * the Sylvester Hadamard matrix, computed in fp32 by butterflies of stride
+ * 1, 2, 4, 8 and rounded to bf16 (nearest-even).  K % 16 == 0.  x and y may
+ * not overlap unless they are the same buffer with the same ld. */
+BSQ_API int bsq_rht(const void *x_bf16, void *y_bf16, int64_t M, int64_t K, int64_t ldx, int64_t ldy,
+            uint16_t rht_sign_mask, void *stream);
+
+/* Dequantize -> transpose -> requantize ("Thinking Machines ...", section
+ * "A precision choice for each stage"): the row-wise MXFP8 tensor (codes
+ * [M][K], swizzled sf for M x K/32) is decoded exactly (E4M3 x 2^E, fp32),
+ * transposed, and quantized again as in bsq_quant_mxfp8 with blocks of 32
+ * along the old M: codes_col [K][M], sf_col for K rows x M/32 blocks.
+ * M % 128 == 0 and K % 32 == 0 (so the input SF has no partial atom). */
+BSQ_API int bsq_requant_transpose(const uint8_t *codes_row_dev, const uint8_t *sf_row_dev,
+                          int64_t M, int64_t K, int rounding, uint64_t seed, uint32_t stream_id,
+                          uint8_t *codes_col_dev, uint8_t *sf_col_dev, void *stream);
+
+/* Block-scaled GEMM ("Microscaling ...", section "Hardware and kernels":
+ * the tensor core applies the block scales inside the matrix instruction):
+ *   C[m][n] = alpha * sum_k decA[m][k] * decB[n][k],
+ * A [M][K] and B [N][K] both K-major (codes row-major, as the quantizers
+ * write them), with their swizzled SF buffers.  NVFP4: alpha =
+ * (*gsA_dev) * (*gsB_dev) (each may be NULL for 1); MXFP8: alpha = 1 and
+ * gs* are ignored.  Accumulation is fp32 in tensor memory; C is fp32 or
+ * bf16 (nearest-even), row-major with leading dimension ldc (elements).
+ * Requirements: K % 128 == 0; M, N >= 1. */
+BSQ_API int bsq_gemm_blockscaled(int fmt, const uint8_t *A_dev, const uint8_t *sfA_dev, const float *gsA_dev,
+                         const uint8_t *B_dev, const uint8_t *sfB_dev, const float *gsB_dev,
+                         int64_t M, int64_t N, int64_t K, void *C_dev, int64_t ldc, int out_type,
+                         void *stream);
+
+/* Grouped block-scaled GEMM for MoE experts ("Thinking Machines ...",
+ * section "A precision choice for each stage": NVFP4 forward in the
+ * expert layers).  For each group e with rows [row_offsets[e],
+ * row_offsets[e+1]) of A (M_total rows in all):
+ *   C[m][n] = alpha_e * sum_k decA[m][k] * decB_e[n][k],
+ * alpha_e = (*gsA_dev) * gsB_dev[e] for NVFP4 (either may be NULL for 1).
+ * A's SF rows of group e start at sf_row_offsets[e] (as bsq_quant_nvfp4
+ * writes them with groups); B is [G][N][K] codes with G consecutive SF
+ * buffers of bsq_sf_bytes(N, K/vec) bytes each.  Offsets are device int32
+ * [G+1]; the row counts may be anything (zero included).  K % 128 == 0. */
+BSQ_API int bsq_grouped_gemm(int fmt, int G, const int32_t *row_offsets_dev, const int32_t *sf_row_offsets_dev,
+                     int64_t M_total, const uint8_t *A_dev, const uint8_t *sfA_dev, const float *gsA_dev,
+                     const uint8_t *B_dev, const uint8_t *sfB_dev, const float *gsB_dev,
+                     int64_t N, int64_t K, void *C_dev, int64_t ldc, int out_type, void *stream);
+
+/* Synchronize `stream`, then read and clear this device's error word.
+ * Returns BSQ_OK, BSQ_ERR_TIMEOUT (a kernel's bounded wait ran out; the
+ * kernel returned early and its outputs are undefined) or BSQ_ERR_CUDA. */
+BSQ_API int bsq_check(void *stream);
+
+/* Test hook for the bounded-wait path: launches one CTA that waits on a
+ * shared-memory barrier nobody arrives at, giving up after timeout_ns
+ * nanoseconds (device clock) and recording BSQ_ERR_TIMEOUT.  The context
+ * stays usable.  timeout_ns must be in (0, 10^10]. */
+BSQ_API int bsq_debug_timeout_probe(uint64_t timeout_ns, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BSQ_H */

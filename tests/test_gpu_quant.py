@@ -1,0 +1,225 @@
+"""GPU parity of the codec kernels against the CPU oracle (bit-exact).
+
+Inputs are the seeded workloads at sizes the oracle finishes in seconds, plus
+edge tensors (zero blocks, exact E2M1 midpoints, saturating blocks, negative
+values that round to zero, ragged shapes), and the full-size workloads where
+the oracle still runs in seconds.  Codes, scale factors (unswizzled with the
+oracle's layout function) and the global scale must match exactly.
+"""
+import numpy as np
+import pytest
+import torch
+
+from fp8_math_b200 import api, bsq
+from fp8_math_b200 import workloads as W
+from gpu_util import assert_codes_equal, bits, dev, host_u8, sf_canonical
+
+pytestmark = pytest.mark.gpu
+
+
+def edge_tensor(M, K, seed=0):
+    """N(0,1) plus: an all-zero block, tiny negatives beside a large value,
+    exact E2M1 midpoints under a power-of-two global scale (amax = 2688),
+    a saturating column and a block of subnormal-range values."""
+    g = torch.Generator().manual_seed(seed)
+    x = torch.randn(M, K, generator=g)
+    x[0, :16] = 0.0
+    if M > 1:
+        x[1, 16:32] = -1e-6
+        if K >= 32:
+            x[1, 20] = 3.0
+    mids = torch.tensor([6.0, 2.5, 0.25, 0.75, 1.25, 1.75, 3.5, 5.0, -2.5, -0.25, -0.75, -1.25, -1.75, -3.5, -5.0, 1.0])
+    for r in range(2, min(M, 10)):
+        x[r, :16] = mids * (2.0 ** (r - 6))
+    x[M - 1, K - 1] = 2688.0
+    if K > 48:
+        x[:, 47] *= 1000.0
+        x[M - 1, K - 1] = float(x.abs().max()) * 1.0
+    if M > 12 and K >= 32:
+        x[12, 16:32] = 1e-30
+    return x.to(torch.bfloat16)
+
+
+def _nvfp4_check(ora, x, block_2d=False, fos=False, rht=None, row_index=None, groups=None, amax_in=None, what=""):
+    xd = dev(x)
+    ri = None if row_index is None else dev(torch.from_numpy(row_index))
+    gr = None
+    if groups is not None:
+        ro, so = groups
+        gr = (dev(torch.from_numpy(ro)), dev(torch.from_numpy(so)), int(so[-1]))
+    am = None if amax_in is None else dev(torch.tensor([amax_in], dtype=torch.float32))
+    codes, sf, gs = api.quant_nvfp4(xd, block_2d=block_2d, four_over_six=fos, rht_mask=rht, row_index=ri,
+                                    groups=gr, amax_in=am)
+    assert bsq.bsq_check() == 0
+    oc, osf, og = ora.quant_nvfp4(bits(x), block_2d=block_2d, four_over_six=fos, rht_mask=rht,
+                                  row_index=row_index, amax_in=amax_in)
+    R, K = oc.shape[0], x.shape[1]
+    assert np.float32(gs.item()) == np.float32(og), (what, gs.item(), og)
+    assert_codes_equal(host_u8(codes), oc, what + " codes")
+    if groups is None:
+        assert_codes_equal(sf_canonical(ora, sf, R, K // 16), osf, what + " sf")
+    else:
+        ro, so = groups
+        can = ora.sf_unswizzle(host_u8(sf), int(so[-1]), K // 16)
+        for e in range(len(ro) - 1):
+            n = ro[e + 1] - ro[e]
+            assert_codes_equal(can[so[e]:so[e] + n], osf[ro[e]:ro[e + 1]], f"{what} sf group {e}")
+
+
+# ------------------------------------------------------------------ NVFP4
+@pytest.mark.parametrize("M,K", [(128, 256), (1, 16), (3, 48), (37, 80), (256, 512), (130, 1024)])
+def test_nvfp4_1d_parity(ora, M, K):
+    x = edge_tensor(M, K, seed=M + K)
+    _nvfp4_check(ora, x, what=f"nvfp4 1d {M}x{K}")
+
+
+def test_nvfp4_small_linear_workload(ora):
+    A, Wt = W.nvfp4_linear_small()
+    _nvfp4_check(ora, A, what="A 1x16")
+    _nvfp4_check(ora, Wt, block_2d=True, what="W 16x16")
+
+
+@pytest.mark.parametrize("M,K", [(16, 16), (32, 48), (256, 256), (48, 1040), (160, 4096)])
+def test_nvfp4_2d_parity(ora, M, K):
+    x = edge_tensor(M, K, seed=3 * M + K)
+    _nvfp4_check(ora, x, block_2d=True, what=f"nvfp4 2d {M}x{K}")
+
+
+@pytest.mark.parametrize("block_2d", [False, True])
+def test_nvfp4_rht_parity(ora, block_2d):
+    A, Wt, seed = W.nvfp4_linear_rht(M=256, N=272, K=512)
+    mask = ora.rht_sign_mask(seed)
+    assert bsq.bsq_rht_sign_mask(seed) == mask
+    _nvfp4_check(ora, A if not block_2d else Wt, block_2d=block_2d, rht=mask, what="rht")
+
+
+@pytest.mark.parametrize("M,K", [(64, 256), (200, 1536), (5, 32)])
+def test_nvfp4_four_over_six_parity(ora, M, K):
+    x = edge_tensor(M, K, seed=7 * M)
+    _nvfp4_check(ora, x, fos=True, what="4/6")
+    _nvfp4_check(ora, x, fos=True, rht=0x5A5A, what="4/6 + rht")
+
+
+def test_nvfp4_given_amax_and_zero_tensor(ora):
+    x = edge_tensor(64, 128, seed=5)
+    _nvfp4_check(ora, x, amax_in=float(x.float().abs().max()) * 2.0, what="given amax")
+    _nvfp4_check(ora, torch.zeros(32, 64, dtype=torch.bfloat16), what="zeros")
+    _nvfp4_check(ora, torch.zeros(32, 64, dtype=torch.bfloat16), block_2d=True, what="zeros 2d")
+
+
+def test_nvfp4_moe_gather_groups_parity(ora):
+    """MoE activations: gather by routing, Four Over Six, per-expert SF rows
+    padded to 128 (small version of the MoE workload's shapes)."""
+    moe = W.moe_forward(T=512, H=256, E=8, F=128, weights=False)
+    _nvfp4_check(ora, moe.X, fos=True, row_index=moe.row_index,
+                 groups=(moe.row_offsets, moe.sf_row_offsets), what="moe gather")
+
+
+def test_amax_parity(ora):
+    x = edge_tensor(96, 160, seed=11)
+    xd = dev(x)
+    for rht in (None, 0xBEEF):
+        for ri in (None, np.array([5, 0, 95, 5, 17], np.int32)):
+            a = api.amax(xd, rht_mask=rht, row_index=None if ri is None else dev(torch.from_numpy(ri)))
+            want = ora.amax(bits(x), rht_mask=rht, row_index=ri)
+            assert np.float32(a.item()) == np.float32(want)
+
+
+# ------------------------------------------------------------------ RHT
+@pytest.mark.parametrize("M,K", [(1, 16), (64, 256), (33, 4096)])
+def test_rht_bf16_parity(ora, M, K):
+    x = edge_tensor(M, K, seed=M)
+    mask = ora.rht_sign_mask(2)
+    y = api.rht(dev(x), mask)
+    assert_codes_equal(y.cpu().view(torch.int16).numpy().view(np.uint16), ora.rht_bf16(bits(x), mask), "rht")
+
+
+# ------------------------------------------------------------------ MXFP8
+def mx_edge_tensor(M, K, seed=0):
+    g = torch.Generator().manual_seed(seed)
+    x = W.student_t((M, K), 3, g)
+    x[0, :32] = 0.0
+    if M > 1:
+        x[1, :32] = torch.linspace(-1, 1, 32) * 1e-38  # subnormal range, includes -0 outcomes
+    if M > 2:
+        x[2, :32] = 480.0  # (448, 512) x 2^0 saturates
+        x[2, 5] = 300.0
+    if M > 3:
+        x[3, :32] = -1e-3
+    return x.to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("sr", [False, True])
+@pytest.mark.parametrize("M,K", [(64, 128), (3, 32), (100, 96), (256, 4096)])
+def test_mxfp8_rowwise_parity(ora, M, K, sr):
+    x = mx_edge_tensor(M, K, seed=M * 3 + K)
+    c, s = api.quant_mxfp8(dev(x), sr=sr, seed=1, stream_id=0)
+    oc, osf = ora.quant_mxfp8(bits(x), sr=sr, seed=1, stream_id=0)
+    assert_codes_equal(host_u8(c), oc, "mx row codes")
+    assert_codes_equal(sf_canonical(ora, s, M, K // 32), osf, "mx row sf")
+
+
+@pytest.mark.parametrize("sr", [False, True])
+@pytest.mark.parametrize("M,K", [(128, 64), (32, 8), (96, 200), (512, 256), (160, 40)])
+def test_mxfp8_colwise_parity(ora, M, K, sr):
+    x = mx_edge_tensor(M, K, seed=M + 5 * K)
+    c, s = api.quant_mxfp8(dev(x), colwise=True, sr=sr, seed=4, stream_id=3)
+    oc, osf = ora.quant_mxfp8(bits(x), colwise=True, sr=sr, seed=4, stream_id=3)
+    assert_codes_equal(host_u8(c), oc, "mx col codes")
+    assert_codes_equal(sf_canonical(ora, s, K, M // 32), osf, "mx col sf")
+
+
+@pytest.mark.parametrize("sr", [False, True])
+@pytest.mark.parametrize("M,K", [(128, 64), (32, 32), (96, 160), (256, 512)])
+def test_requant_transpose_parity(ora, M, K, sr):
+    x = mx_edge_tensor(M, K, seed=M + K)
+    oc, osf = ora.quant_mxfp8(bits(x), sr=True, seed=1, stream_id=0)
+    # the oracle's row-wise output is the input of both sides
+    codes = dev(torch.from_numpy(oc))
+    sf = dev(torch.from_numpy(ora.sf_swizzle(osf)))
+    cc, sc = api.requant_transpose(codes, sf, sr=sr, seed=1, stream_id=1)
+    wc, ws = ora.requant_transpose(oc, osf, sr=sr, seed=1, stream_id=1)
+    assert_codes_equal(host_u8(cc), wc, "requant codes")
+    assert_codes_equal(sf_canonical(ora, sc, K, M // 32), ws, "requant sf")
+
+
+def test_mxfp8_requant_workload_full_size(ora):
+    """The Student-t 4096x4096 workload at full size: RNE, SR, then the
+    requant-transpose of the SR output -- all bit-exact."""
+    x = W.mxfp8_requant()
+    xb = bits(x)
+    xd = dev(x)
+    for sr in (False, True):
+        c, s = api.quant_mxfp8(xd, sr=sr, seed=1, stream_id=0)
+        oc, osf = ora.quant_mxfp8(xb, sr=sr, seed=1, stream_id=0)
+        assert_codes_equal(host_u8(c), oc, f"cfg1 sr={sr} codes")
+        assert_codes_equal(sf_canonical(ora, s, 4096, 128), osf, f"cfg1 sr={sr} sf")
+    cc, sc = api.requant_transpose(c, s, sr=True, seed=1, stream_id=1)
+    wc, ws = ora.requant_transpose(oc, osf, sr=True, seed=1, stream_id=1)
+    assert_codes_equal(host_u8(cc), wc, "cfg1 requant codes")
+    assert_codes_equal(sf_canonical(ora, sc, 4096, 128), ws, "cfg1 requant sf")
+
+
+# ------------------------------------------------------------------ errors
+def test_invalid_arguments_launch_nothing():
+    x = torch.zeros(16, 24, dtype=torch.bfloat16, device="cuda")
+    codes = torch.empty(16, 12, dtype=torch.uint8, device="cuda")
+    sf = torch.empty(4096, dtype=torch.uint8, device="cuda")
+    gs = torch.empty(1, dtype=torch.float32, device="cuda")
+    with pytest.raises(bsq.BsqError) as e:
+        bsq.bsq_quant_nvfp4(x, 16, 24, 24, 0, 0, 0, 0, None, 0, None, None, None, gs, codes, sf)
+    assert e.value.status == bsq.BSQ_ERR_INVALID
+    with pytest.raises(bsq.BsqError) as e:
+        bsq.bsq_quant_nvfp4(x, 16, 16, 24, 1, 1, 0, 0, None, 0, None, None, None, gs, codes, sf)
+    assert e.value.status == bsq.BSQ_ERR_INVALID
+    assert bsq.bsq_check() == bsq.BSQ_OK
+
+
+def test_bounded_wait_times_out_and_context_survives():
+    """A device wait on a barrier nobody arrives at runs out (short limit),
+    reports BSQ_ERR_TIMEOUT through bsq_check, and the context stays usable."""
+    bsq.bsq_debug_timeout_probe(50_000_000)  # 50 ms
+    assert bsq.bsq_check() == bsq.BSQ_ERR_TIMEOUT
+    assert bsq.bsq_check() == bsq.BSQ_OK  # the word was cleared
+    y = torch.ones(4, device="cuda") * 2
+    assert float(y.sum()) == 8.0

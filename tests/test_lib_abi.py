@@ -1,0 +1,68 @@
+"""CPU checks of the C-ABI library: it loads, exports every entry point that
+include/bsq.h declares, and its host-only helpers and argument validation
+behave (no device work is issued by these calls)."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from fp8_math_b200 import bsq
+    if not os.path.exists(bsq.LIB_PATH):
+        from fp8_math_b200 import build
+        build.build()
+    return bsq
+
+
+def declared_symbols():
+    with open(os.path.join(ROOT, "include", "bsq.h")) as f:
+        text = f.read()
+    return sorted(set(re.findall(r"BSQ_API[^;(]*?\b(bsq_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_symbols()
+    for n in ["bsq_amax", "bsq_quant_nvfp4", "bsq_quant_mxfp8", "bsq_rht", "bsq_requant_transpose",
+              "bsq_gemm_blockscaled", "bsq_grouped_gemm", "bsq_check"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    L = C.CDLL(lib.LIB_PATH)
+    for n in declared_symbols():
+        assert hasattr(L, n), n
+
+
+def test_sf_bytes_matches_oracle_layout(lib, ora):
+    for rows, nb in [(1, 1), (128, 16), (8192, 256), (131, 3), (0, 5)]:
+        assert lib.bsq_sf_bytes(rows, nb) == ora.sf_swizzled_bytes(rows, nb)
+
+
+def test_rht_sign_mask_matches_oracle(lib, ora):
+    for seed in [0, 1, 2, 3, 4, 2**40 + 17, 2**64 - 1]:
+        assert lib.bsq_rht_sign_mask(seed) == ora.rht_sign_mask(seed)
+
+
+def test_validation_rejects_before_any_device_work(lib):
+    L = lib.lib()
+    # NULL / misaligned pointers and bad shapes are refused on the host
+    assert L.bsq_quant_nvfp4(None, 16, 16, 16, 0, 0, 0, 0, None, 0, None, None, None, None, None, None,
+                             None) == lib.BSQ_ERR_INVALID
+    assert L.bsq_quant_nvfp4(16, 16, 24, 24, 0, 0, 0, 0, None, 0, None, None, None, 64, 64, 64,
+                             None) == lib.BSQ_ERR_INVALID  # K % 16
+    assert L.bsq_quant_nvfp4(16, 16, 32, 32, 1, 1, 0, 0, None, 0, None, None, None, 64, 64, 64,
+                             None) == lib.BSQ_ERR_INVALID  # 2-D with Four Over Six
+    assert L.bsq_quant_nvfp4(8, 16, 32, 32, 0, 0, 0, 0, None, 0, None, None, None, 64, 64, 64,
+                             None) == lib.BSQ_ERR_ALIGN    # x not 16-byte aligned
+    assert L.bsq_quant_mxfp8(16, 4, 48, 48, 0, 0, 0, 0, 64, 64, None) == lib.BSQ_ERR_INVALID  # K % 32
+    assert L.bsq_quant_mxfp8(16, 4, 64, 64, 0, 7, 0, 0, 64, 64, None) == lib.BSQ_ERR_INVALID  # rounding
+    assert L.bsq_gemm_blockscaled(0, 16, 16, None, 16, 16, None, 4, 4, 96, 16, 4, 0, None) == lib.BSQ_ERR_INVALID
+    assert L.bsq_gemm_blockscaled(5, 16, 16, None, 16, 16, None, 4, 4, 128, 16, 4, 0, None) == lib.BSQ_ERR_INVALID
+    assert L.bsq_requant_transpose(16, 16, 48, 32, 0, 0, 0, 16, 16, None) == lib.BSQ_ERR_INVALID  # M % 32
+    assert L.bsq_debug_timeout_probe(0, None) == lib.BSQ_ERR_INVALID
+    assert lib.status_str(lib.BSQ_ERR_TIMEOUT) == "device-side wait timed out"

@@ -80,8 +80,16 @@ def requant_transpose(codes_row, sf_row, sr=True, seed=0, stream_id=1, out=None)
     return cc, sc
 
 
+def _out(M, N, dtype, device):
+    """[M, N] output whose row stride is a multiple of 16 bytes (a view of a
+    padded buffer when N needs it)."""
+    per = 16 // torch.tensor([], dtype=dtype).element_size()
+    ld = -(-N // per) * per
+    return torch.empty(M, ld, dtype=dtype, device=device)[:, :N]
+
+
 def gemm(fmt, A, sfA, B, sfB, M, N, K, gsA=None, gsB=None, out_dtype=torch.bfloat16, out=None):
-    C_out = torch.empty(M, N, dtype=out_dtype, device=A.device) if out is None else out
+    C_out = _out(M, N, out_dtype, A.device) if out is None else out
     ot = bsq.BSQ_OUT_BF16 if C_out.dtype == torch.bfloat16 else bsq.BSQ_OUT_F32
     bsq.bsq_gemm_blockscaled(fmt, A, sfA, gsA, B, sfB, gsB, M, N, K, C_out, C_out.stride(0), ot)
     return C_out
@@ -90,7 +98,7 @@ def gemm(fmt, A, sfA, B, sfB, M, N, K, gsA=None, gsB=None, out_dtype=torch.bfloa
 def grouped_gemm(fmt, row_offsets, sf_row_offsets, A, sfA, B, sfB, M_total, N, K, gsA=None, gsB=None,
                  out_dtype=torch.bfloat16, out=None):
     G = row_offsets.shape[0] - 1
-    C_out = torch.empty(M_total, N, dtype=out_dtype, device=A.device) if out is None else out
+    C_out = _out(M_total, N, out_dtype, A.device) if out is None else out
     ot = bsq.BSQ_OUT_BF16 if C_out.dtype == torch.bfloat16 else bsq.BSQ_OUT_F32
     bsq.bsq_grouped_gemm(fmt, G, row_offsets, sf_row_offsets, M_total, A, sfA, gsA, B, sfB, gsB, N, K, C_out,
                          C_out.stride(0), ot)

@@ -12,25 +12,42 @@
 namespace bsq {
 
 // ===================================================================== amax
+// Work mapping shared by the row-oriented kernels: a CTA of 256 threads
+// covers (256 >> lpr_shift) rows per step; lanes_per_row = 1 << lpr_shift
+// threads walk a row's units, so no index needs an integer division.
+struct RowMap {
+    int lpr_shift;  // log2(lanes per row)
+};
+
+static int lpr_shift_for(int64_t units_per_row) {
+    int sh = 0;
+    while (sh < 8 && (int64_t(1) << sh) < units_per_row) sh++;
+    return sh;
+}
+
 template <bool RHT, bool GATHER>
 __global__ void __launch_bounds__(256) amax_kernel(const uint16_t *__restrict__ x, int64_t M, int64_t K,
                                                    int64_t ldx, uint32_t mask,
                                                    const int32_t *__restrict__ row_index,
-                                                   unsigned int *amax_bits) {
+                                                   unsigned int *amax_bits, RowMap map) {
     const int64_t KB = K >> 4;
-    const int64_t units = M * KB;
+    const int lpr = 1 << map.lpr_shift;
+    const int rpi = 256 >> map.lpr_shift;
+    const int sub = threadIdx.x >> map.lpr_shift, lk = threadIdx.x & (lpr - 1);
     float m = 0.0f;
-    for (int64_t u = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; u < units;
-         u += (int64_t)gridDim.x * blockDim.x) {
-        int64_t row = u / KB, kb = u - row * KB;
-        int64_t src = GATHER ? (int64_t)row_index[row] : row;
-        const uint16_t *p = x + src * ldx + kb * 16;
-        float v[16];
-        load8_bf16(p, v);
-        load8_bf16(p + 8, v + 8);
-        if (RHT) rht16(v, mask);
+    for (int64_t r0 = (int64_t)blockIdx.x * rpi; r0 < M; r0 += (int64_t)gridDim.x * rpi) {
+        const int64_t row = r0 + sub;
+        if (row >= M) continue;
+        const int64_t src = GATHER ? (int64_t)__ldg(row_index + row) : row;
+        const uint16_t *rp = x + src * ldx;
+        for (int64_t kb = lk; kb < KB; kb += lpr) {
+            float v[16];
+            load8_bf16(rp + kb * 16, v);
+            load8_bf16(rp + kb * 16 + 8, v + 8);
+            if (RHT) rht16(v, mask);
 #pragma unroll
-        for (int i = 0; i < 16; i++) m = fmaxf(m, fabsf(v[i]));
+            for (int i = 0; i < 16; i++) m = fmaxf(m, fabsf(v[i]));
+        }
     }
 #pragma unroll
     for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
@@ -125,41 +142,46 @@ BSQ_DEV void store_sf(uint8_t *sf, bool valid, uint32_t sb, int64_t sf_row, int6
 }
 
 // 1x16 blocks: one thread per block of 16 (two 16-byte loads, one 8-byte
-// code store).  The loop is warp-uniform so that shuffles see all lanes.
+// code store).  Loops are warp-uniform so that shuffles see all lanes.
 template <bool RHT, bool FOS, bool GATHER, bool GROUPED>
 __global__ void __launch_bounds__(256) quant_nvfp4_1d_kernel(
     const uint16_t *__restrict__ x, int64_t M, int64_t K, int64_t ldx, uint32_t mask,
     const int32_t *__restrict__ row_index, int G, const int32_t *__restrict__ row_off,
     const int32_t *__restrict__ sf_off, const float *amax_ptr, float *gs_out, int write_gs,
-    uint8_t *__restrict__ codes, uint8_t *__restrict__ sf) {
+    uint8_t *__restrict__ codes, uint8_t *__restrict__ sf, RowMap map) {
     const int64_t KB = K >> 4;
-    const int64_t units = M * KB;
     const bool pack4 = (KB & 3) == 0;
     const float s_g = global_scale_of(*amax_ptr);
     if (write_gs && blockIdx.x == 0 && threadIdx.x == 0) *gs_out = s_g;
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t base = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31); base < units; base += stride) {
-        const int64_t u = base + (threadIdx.x & 31);
-        const bool valid = u < units;
-        const int64_t uu = valid ? u : units - 1;
-        const int64_t row = uu / KB, kb = uu - row * KB;
-        const int64_t src = GATHER ? (int64_t)__ldg(row_index + row) : row;
-        const uint16_t *p = x + src * ldx + kb * 16;
-        float v[16];
-        load8_bf16(p, v);
-        load8_bf16(p + 8, v + 8);
-        if (RHT) rht16(v, mask);
-        float bamax = 0.0f;
+    const int lpr = 1 << map.lpr_shift;
+    const int rpi = 256 >> map.lpr_shift;
+    const int sub = threadIdx.x >> map.lpr_shift, lk = threadIdx.x & (lpr - 1);
+    for (int64_t r0 = (int64_t)blockIdx.x * rpi; r0 < M; r0 += (int64_t)gridDim.x * rpi) {
+        const int64_t row = r0 + sub;
+        const bool row_ok = row < M;
+        const int64_t rr = row_ok ? row : M - 1;
+        const int64_t src = GATHER ? (int64_t)__ldg(row_index + rr) : rr;
+        const uint16_t *rp = x + src * ldx;
+        const int64_t sf_row = GROUPED ? grouped_sf_row(rr, G, row_off, sf_off) : rr;
+        for (int64_t kb0 = 0; kb0 < KB; kb0 += lpr) {
+            const int64_t kb = kb0 + lk;
+            const bool valid = row_ok && kb < KB;
+            const int64_t kk = kb < KB ? kb : KB - 1;
+            float v[16];
+            load8_bf16(rp + kk * 16, v);
+            load8_bf16(rp + kk * 16 + 8, v + 8);
+            if (RHT) rht16(v, mask);
+            float bamax = 0.0f;
 #pragma unroll
-        for (int i = 0; i < 16; i++) bamax = fmaxf(bamax, fabsf(v[i]));
-        NvCand c = nv_candidate(v, bamax, 6.0f, s_g);
-        if (FOS) {
-            NvCand c4 = nv_candidate(v, bamax, 4.0f, s_g);
-            if (nv_block_err(v, c4) < nv_block_err(v, c)) c = c4;
+            for (int i = 0; i < 16; i++) bamax = fmaxf(bamax, fabsf(v[i]));
+            NvCand c = nv_candidate(v, bamax, 6.0f, s_g);
+            if (FOS) {
+                NvCand c4 = nv_candidate(v, bamax, 4.0f, s_g);
+                if (nv_block_err(v, c4) < nv_block_err(v, c)) c = c4;
+            }
+            if (valid) *reinterpret_cast<uint2 *>(codes + rr * (K >> 1) + kb * 8) = c.codes;
+            store_sf(sf, valid, c.sb, sf_row, kb, KB, pack4);
         }
-        if (valid) *reinterpret_cast<uint2 *>(codes + row * (K >> 1) + kb * 8) = c.codes;
-        const int64_t sf_row = GROUPED ? grouped_sf_row(row, G, row_off, sf_off) : row;
-        store_sf(sf, valid, c.sb, sf_row, kb, KB, pack4);
     }
 }
 
@@ -171,16 +193,16 @@ __global__ void __launch_bounds__(512) quant_nvfp4_2d_kernel(
     const float *amax_ptr, float *gs_out, int write_gs, uint8_t *__restrict__ codes, uint8_t *__restrict__ sf) {
     __shared__ float tile_amax[16][33];
     const int64_t KB = K >> 4;
-    const int64_t kb_tiles = (KB + 31) >> 5;
-    const int64_t tiles = (M >> 4) * kb_tiles;
+    const uint32_t kb_tiles = (uint32_t)((KB + 31) >> 5);
+    const uint32_t tiles = (uint32_t)(M >> 4) * kb_tiles;
     const bool pack4 = (KB & 3) == 0;
     const float s_g = global_scale_of(*amax_ptr);
     if (write_gs && blockIdx.x == 0 && threadIdx.x == 0) *gs_out = s_g;
     const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x) {
-        const int64_t rt = t / kb_tiles, kt = t - rt * kb_tiles;
-        const int64_t row = rt * 16 + w;
-        const int64_t kb = kt * 32 + lane;
+    for (uint32_t t = blockIdx.x; t < tiles; t += gridDim.x) {
+        const uint32_t rt = t / kb_tiles, kt = t - rt * kb_tiles;
+        const int64_t row = (int64_t)rt * 16 + w;
+        const int64_t kb = (int64_t)kt * 32 + lane;
         const bool valid = kb < KB;
         float v[16];
         if (valid) {
@@ -247,41 +269,46 @@ BSQ_DEV uint2 mx_encode8(const float v[8], bool zero_block, int E, uint64_t idx0
 template <bool SR>
 __global__ void __launch_bounds__(256) quant_mxfp8_row_kernel(
     const uint16_t *__restrict__ x, int64_t M, int64_t K, int64_t ldx, uint32_t seed_lo, uint32_t seed_hi,
-    uint32_t stream_id, uint8_t *__restrict__ codes, uint8_t *__restrict__ sf) {
+    uint32_t stream_id, uint8_t *__restrict__ codes, uint8_t *__restrict__ sf, RowMap map) {
     const int64_t K8 = K >> 3, KB = K >> 5;
-    const int64_t units = M * K8;
     const bool pack4 = (KB & 3) == 0;
     const int lane = threadIdx.x & 31;
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t base = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31); base < units; base += stride) {
-        const int64_t u = base + lane;
-        const bool valid = u < units;
-        const int64_t uu = valid ? u : units - 1;
-        const int64_t row = uu / K8, c8 = uu - row * K8;
-        float v[8];
-        load8_bf16(x + row * ldx + c8 * 8, v);
-        float m = 0.0f;
+    const int lpr = 1 << map.lpr_shift;
+    const int rpi = 256 >> map.lpr_shift;
+    const int sub = threadIdx.x >> map.lpr_shift, lk = threadIdx.x & (lpr - 1);
+    for (int64_t r0 = (int64_t)blockIdx.x * rpi; r0 < M; r0 += (int64_t)gridDim.x * rpi) {
+        const int64_t row = r0 + sub;
+        const bool row_ok = row < M;
+        const int64_t rr = row_ok ? row : M - 1;
+        for (int64_t c0 = 0; c0 < K8; c0 += lpr) {
+            const int64_t c8 = c0 + lk;
+            const bool valid = row_ok && c8 < K8;
+            const int64_t cc = c8 < K8 ? c8 : K8 - 1;
+            float v[8];
+            load8_bf16(x + rr * ldx + cc * 8, v);
+            float m = 0.0f;
 #pragma unroll
-        for (int i = 0; i < 8; i++) m = fmaxf(m, fabsf(v[i]));
-        m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
-        m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
-        const bool zero = (m == 0.0f);
-        const int E = zero ? 0 : mx_exponent(m);
-        const uint64_t idx0 = (uint64_t)(row * K + c8 * 8);
-        uint2 q = mx_encode8<SR>(v, zero, E, idx0, seed_lo, seed_hi, stream_id);
-        if (valid) *reinterpret_cast<uint2 *>(codes + row * K + c8 * 8) = q;
-        // scale byte: lanes 4j hold block j of the warp; 4 blocks per word
-        const uint32_t sb = zero ? 0u : (uint32_t)(E + 127);
-        const int64_t kb = c8 >> 2;
-        if (pack4) {
-            uint32_t b1 = __shfl_down_sync(0xFFFFFFFFu, sb, 4);
-            uint32_t b2 = __shfl_down_sync(0xFFFFFFFFu, sb, 8);
-            uint32_t b3 = __shfl_down_sync(0xFFFFFFFFu, sb, 12);
-            if (valid && (lane & 15) == 0)
-                *reinterpret_cast<uint32_t *>(sf + sf_word_offset(row, kb >> 2, KB)) =
-                    sb | (b1 << 8) | (b2 << 16) | (b3 << 24);
-        } else if (valid && (lane & 3) == 0) {
-            sf[sf_offset(row, kb, KB)] = (uint8_t)sb;
+            for (int i = 0; i < 8; i++) m = fmaxf(m, fabsf(v[i]));
+            m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+            m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+            const bool zero = (m == 0.0f);
+            const int E = zero ? 0 : mx_exponent(m);
+            const uint64_t idx0 = (uint64_t)(rr * K + cc * 8);
+            uint2 q = mx_encode8<SR>(v, zero, E, idx0, seed_lo, seed_hi, stream_id);
+            if (valid) *reinterpret_cast<uint2 *>(codes + rr * K + cc * 8) = q;
+            // scale byte: lanes 4j hold block j; 4 blocks (16 lanes) per word
+            const uint32_t sb = zero ? 0u : (uint32_t)(E + 127);
+            const int64_t kb = cc >> 2;
+            if (pack4) {
+                uint32_t b1 = __shfl_down_sync(0xFFFFFFFFu, sb, 4);
+                uint32_t b2 = __shfl_down_sync(0xFFFFFFFFu, sb, 8);
+                uint32_t b3 = __shfl_down_sync(0xFFFFFFFFu, sb, 12);
+                if (valid && (lane & 15) == 0)
+                    *reinterpret_cast<uint32_t *>(sf + sf_word_offset(rr, kb >> 2, KB)) =
+                        sb | (b1 << 8) | (b2 << 16) | (b3 << 24);
+            } else if (valid && (lane & 3) == 0) {
+                sf[sf_offset(rr, kb, KB)] = (uint8_t)sb;
+            }
         }
     }
 }
@@ -299,12 +326,12 @@ __global__ void __launch_bounds__(256) quant_mxfp8_col_kernel(
     uint32_t seed_lo, uint32_t seed_hi, uint32_t stream_id, uint8_t *__restrict__ codes,
     uint8_t *__restrict__ sf) {
     __shared__ __align__(16) float tile[CT_K][CT_M];
-    const int64_t m_tiles = (M + CT_M - 1) / CT_M, k_tiles = (K + CT_K - 1) / CT_K;
+    const uint32_t m_tiles = (uint32_t)((M + CT_M - 1) / CT_M), k_tiles = (uint32_t)((K + CT_K - 1) / CT_K);
     const int64_t MB = M >> 5;  // output blocks per output row
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    for (int64_t t = blockIdx.x; t < m_tiles * k_tiles; t += gridDim.x) {
-        const int64_t mt = t % m_tiles, kt = t / m_tiles;
-        const int64_t m0 = mt * CT_M, k0 = kt * CT_K;
+    for (uint32_t t = blockIdx.x; t < m_tiles * k_tiles; t += gridDim.x) {
+        const uint32_t kt = t / m_tiles, mt = t - kt * m_tiles;
+        const int64_t m0 = (int64_t)mt * CT_M, k0 = (int64_t)kt * CT_K;
         // ---- load: each thread reads 32 contiguous bytes of one input row
         if (!FROM_MX) {
             const uint16_t *x = static_cast<const uint16_t *>(xin);
@@ -400,25 +427,29 @@ __global__ void __launch_bounds__(256) quant_mxfp8_col_kernel(
 
 // ===================================================================== RHT
 __global__ void __launch_bounds__(256) rht_kernel(const uint16_t *__restrict__ x, uint16_t *y, int64_t M,
-                                                  int64_t K, int64_t ldx, int64_t ldy, uint32_t mask) {
+                                                  int64_t K, int64_t ldx, int64_t ldy, uint32_t mask, RowMap map) {
     const int64_t KB = K >> 4;
-    const int64_t units = M * KB;
-    for (int64_t u = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; u < units;
-         u += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t row = u / KB, kb = u - row * KB;
-        float v[16];
-        load8_bf16(x + row * ldx + kb * 16, v);
-        load8_bf16(x + row * ldx + kb * 16 + 8, v + 8);
-        rht16(v, mask);
-        uint32_t w[8];
+    const int lpr = 1 << map.lpr_shift;
+    const int rpi = 256 >> map.lpr_shift;
+    const int sub = threadIdx.x >> map.lpr_shift, lk = threadIdx.x & (lpr - 1);
+    for (int64_t r0 = (int64_t)blockIdx.x * rpi; r0 < M; r0 += (int64_t)gridDim.x * rpi) {
+        const int64_t row = r0 + sub;
+        if (row >= M) continue;
+        for (int64_t kb = lk; kb < KB; kb += lpr) {
+            float v[16];
+            load8_bf16(x + row * ldx + kb * 16, v);
+            load8_bf16(x + row * ldx + kb * 16 + 8, v + 8);
+            rht16(v, mask);
+            uint32_t w[8];
 #pragma unroll
-        for (int i = 0; i < 8; i++) {
-            __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
-            w[i] = *reinterpret_cast<uint32_t *>(&h);
+            for (int i = 0; i < 8; i++) {
+                __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+                w[i] = *reinterpret_cast<uint32_t *>(&h);
+            }
+            uint4 *q = reinterpret_cast<uint4 *>(y + row * ldy + kb * 16);
+            q[0] = make_uint4(w[0], w[1], w[2], w[3]);
+            q[1] = make_uint4(w[4], w[5], w[6], w[7]);
         }
-        uint4 *q = reinterpret_cast<uint4 *>(y + row * ldy + kb * 16);
-        q[0] = make_uint4(w[0], w[1], w[2], w[3]);
-        q[1] = make_uint4(w[4], w[5], w[6], w[7]);
     }
 }
 
@@ -431,8 +462,9 @@ static int grid_for(int64_t work_items, int per_block, int max_ctas) {
 
 void launch_amax(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, bool rht, uint32_t mask,
                  const int32_t *row_index, unsigned int *amax_bits, int num_sms, cudaStream_t s) {
-    const int grid = grid_for(M * (K >> 4), 256, num_sms * 8);
-#define BSQ_AMAX(R, G) amax_kernel<R, G><<<grid, 256, 0, s>>>(x, M, K, ldx, mask, row_index, amax_bits)
+    RowMap map{lpr_shift_for(K >> 4)};
+    const int grid = grid_for(M, 256 >> map.lpr_shift, num_sms * 8);
+#define BSQ_AMAX(R, G) amax_kernel<R, G><<<grid, 256, 0, s>>>(x, M, K, ldx, mask, row_index, amax_bits, map)
     if (rht) { if (row_index) BSQ_AMAX(true, true); else BSQ_AMAX(true, false); }
     else { if (row_index) BSQ_AMAX(false, true); else BSQ_AMAX(false, false); }
 #undef BSQ_AMAX
@@ -453,11 +485,12 @@ void launch_quant_nvfp4(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, bo
             quant_nvfp4_2d_kernel<false><<<grid, 512, 0, s>>>(x, M, K, ldx, mask, amax_ptr, gs_out, write_gs, codes, sf);
         return;
     }
-    const int grid = grid_for(M * (K >> 4), 256, num_sms * 8);
+    RowMap map{lpr_shift_for(K >> 4)};
+    const int grid = grid_for(M, 256 >> map.lpr_shift, num_sms * 8);
     const bool gather = row_index != nullptr, grouped = G > 0;
 #define BSQ_NV1(R, F, GA, GR)                                                                            \
     quant_nvfp4_1d_kernel<R, F, GA, GR><<<grid, 256, 0, s>>>(x, M, K, ldx, mask, row_index, G, row_off, \
-                                                            sf_off, amax_ptr, gs_out, write_gs, codes, sf)
+                                                            sf_off, amax_ptr, gs_out, write_gs, codes, sf, map)
 #define BSQ_NV1_G(R, F)                                 \
     do {                                                \
         if (gather) {                                   \
@@ -479,9 +512,11 @@ void launch_quant_mxfp8(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, bo
                         cudaStream_t s) {
     const uint32_t lo = (uint32_t)seed, hi = (uint32_t)(seed >> 32);
     if (!colwise) {
-        const int grid = grid_for(M * (K >> 3), 256, num_sms * 8);
-        if (sr) quant_mxfp8_row_kernel<true><<<grid, 256, 0, s>>>(x, M, K, ldx, lo, hi, stream_id, codes, sf);
-        else quant_mxfp8_row_kernel<false><<<grid, 256, 0, s>>>(x, M, K, ldx, lo, hi, stream_id, codes, sf);
+        RowMap map{lpr_shift_for(K >> 3)};
+        if (map.lpr_shift < 2) map.lpr_shift = 2;  // 4 lanes per block of 32
+        const int grid = grid_for(M, 256 >> map.lpr_shift, num_sms * 8);
+        if (sr) quant_mxfp8_row_kernel<true><<<grid, 256, 0, s>>>(x, M, K, ldx, lo, hi, stream_id, codes, sf, map);
+        else quant_mxfp8_row_kernel<false><<<grid, 256, 0, s>>>(x, M, K, ldx, lo, hi, stream_id, codes, sf, map);
         return;
     }
     const int64_t tiles = ((M + CT_M - 1) / CT_M) * ((K + CT_K - 1) / CT_K);
@@ -508,8 +543,9 @@ void launch_requant_transpose(const uint8_t *codes_row, const uint8_t *sf_row, i
 
 void launch_rht(const uint16_t *x, uint16_t *y, int64_t M, int64_t K, int64_t ldx, int64_t ldy, uint32_t mask,
                 int num_sms, cudaStream_t s) {
-    const int grid = grid_for(M * (K >> 4), 256, num_sms * 8);
-    rht_kernel<<<grid, 256, 0, s>>>(x, y, M, K, ldx, ldy, mask);
+    RowMap map{lpr_shift_for(K >> 4)};
+    const int grid = grid_for(M, 256 >> map.lpr_shift, num_sms * 8);
+    rht_kernel<<<grid, 256, 0, s>>>(x, y, M, K, ldx, ldy, mask, map);
 }
 
 }  // namespace bsq

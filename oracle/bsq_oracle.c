@@ -480,9 +480,13 @@ static uint8_t mx_block(const float v[32], int sr, uint64_t seed, uint32_t sid,
 
 /* Quantize x [M][K] (bf16) to MXFP8.  colwise == 0: output codes [M][K], sf
  * [M][K/32]; colwise == 1: output is the quantization of x^T, codes [K][M],
- * sf [K][M/32] (blocks of 32 along the original M). */
-int ora_quant_mxfp8(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, int colwise,
-                    int sr, uint64_t seed, uint32_t stream_id, uint8_t *codes, uint8_t *sf)
+ * sf [K][M/32] (blocks of 32 along the original M).  out_row0 is the index,
+ * in the full output tensor, of the first output row computed here (0 for a
+ * whole tensor): it only offsets the element indices of the SR draws, so a
+ * band of output rows can be computed on its own. */
+int ora_quant_mxfp8_rows(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, int colwise,
+                         int sr, uint64_t seed, uint32_t stream_id, int64_t out_row0,
+                         uint8_t *codes, uint8_t *sf)
 {
     int64_t R = colwise ? K : M, C = colwise ? M : K;
     if (C % 32)
@@ -494,11 +498,17 @@ int ora_quant_mxfp8(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, int co
                 int64_t c = cb * 32 + i;
                 v[i] = colwise ? ora_bf16_to_f32(x[c * ldx + r]) : ora_bf16_to_f32(x[r * ldx + c]);
             }
-            sf[r * (C / 32) + cb] =
-                mx_block(v, sr, seed, stream_id, (uint64_t)(r * C + cb * 32), codes + r * C + cb * 32);
+            sf[r * (C / 32) + cb] = mx_block(v, sr, seed, stream_id,
+                                             (uint64_t)((out_row0 + r) * C + cb * 32), codes + r * C + cb * 32);
         }
     }
     return 0;
+}
+
+int ora_quant_mxfp8(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, int colwise,
+                    int sr, uint64_t seed, uint32_t stream_id, uint8_t *codes, uint8_t *sf)
+{
+    return ora_quant_mxfp8_rows(x, M, K, ldx, colwise, sr, seed, stream_id, 0, codes, sf);
 }
 
 /* ------------------------------------------------------------------------ */

@@ -71,6 +71,8 @@ def lib():
                                               C.c_uint16, C.c_void_p, C.c_void_p, _f32p, _u8p, _u8p]),
                 "ora_quant_mxfp8": (C.c_int, [_u16p, _i64, _i64, _i64, C.c_int, C.c_int,
                                               C.c_uint64, C.c_uint32, _u8p, _u8p]),
+                "ora_quant_mxfp8_rows": (C.c_int, [_u16p, _i64, _i64, _i64, C.c_int, C.c_int,
+                                                   C.c_uint64, C.c_uint32, _i64, _u8p, _u8p]),
                 "ora_requant_transpose": (C.c_int, [_u8p, _u8p, _i64, _i64, C.c_int, C.c_uint64,
                                                     C.c_uint32, _u8p, _u8p]),
                 "ora_sf_swizzled_bytes": (_i64, [_i64, _i64]),
@@ -192,14 +194,17 @@ def quant_nvfp4(x, block_2d=False, four_over_six=False, rht_mask=None, row_index
     return codes, sf, float(sg[0])
 
 
-def quant_mxfp8(x, colwise=False, sr=False, seed=0, stream_id=0):
-    """MXFP8 quantize (ora_quant_mxfp8).  Returns (codes, sf) in the output orientation."""
+def quant_mxfp8(x, colwise=False, sr=False, seed=0, stream_id=0, out_row0=0):
+    """MXFP8 quantize (ora_quant_mxfp8_rows).  Returns (codes, sf) in the output
+    orientation.  out_row0: index of the first output row within the full
+    output tensor (SR draw indices), for computing a band of rows alone."""
     x = _c(x, np.uint16)
     M, K = x.shape
     R, Cc = (K, M) if colwise else (M, K)
     codes = np.zeros((R, Cc), np.uint8)
     sf = np.zeros((R, Cc // 32), np.uint8)
-    if lib().ora_quant_mxfp8(x, M, K, K, int(colwise), int(sr), int(seed), int(stream_id), codes, sf):
+    if lib().ora_quant_mxfp8_rows(x, M, K, K, int(colwise), int(sr), int(seed), int(stream_id), int(out_row0),
+                                  codes, sf):
         raise ValueError("unsupported MXFP8 shape")
     return codes, sf
 

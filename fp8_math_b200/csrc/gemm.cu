@@ -2,14 +2,19 @@
 // NVFP4 (kind::mxf4nvf4, 16-element E4M3 scales) or MXFP8 (kind::mxf8f6f4,
 // 32-element E8M0 scales) operands, both K-major.
 //
-// Persistent, warp-specialised CTA (6 warps):
+// Persistent, warp-specialised CTA (10 warps):
 //   warp 0      TMA producer: A/B code tiles (128-byte swizzle) and the
 //               scale-factor atoms (1-D bulk copies) into a k-stage ring;
-//   warp 1      TMEM allocator + MMA issuer: copies the scale atoms of a
-//               stage to TMEM (tcgen05.cp), issues tcgen05.mma with block
-//               scales, commits stage release and accumulator-ready;
-//   warps 2..5  epilogue: tcgen05.ld of the fp32 accumulator, alpha scale,
-//               fp32 or bf16 stores (transposed for the swap-AB case).
+//   warp 1      TMEM allocator + MMA issuer: copies the scale atoms an MMA
+//               needs to a ring of TMEM slots (tcgen05.cp) right before that
+//               MMA, so the copies overlap the previous MMA, issues
+//               tcgen05.mma with block scales, commits stage release and
+//               accumulator-ready;
+//   warps 2..9  epilogue, two warps per TMEM lane quarter (each one half of
+//               the tile's columns): tcgen05.ld of the fp32 accumulator,
+//               alpha scale, fp32 or bf16 stores (transposed for swap-AB).
+// With one 256-column accumulator the epilogue drains TMEM into registers,
+// releases it, and stores while the next tile's MMAs run.
 // Every mbarrier wait is bounded (device clock); on expiry the CTA records
 // a timeout in the error word, drains its own copies, frees TMEM and exits.
 // No load uses cluster multicast.
@@ -73,11 +78,14 @@ struct Cfg {
     static constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
     static constexpr int kStages = (220 * 1024) / kStageBytes > 8 ? 8 : (220 * 1024) / kStageBytes;
     static constexpr int kSmemBytes = kStages * kStageBytes + 1024;  // + alignment slack
-    // TMEM columns of one k-tile's scale factors
-    static constexpr int kSfaCols = (FMT == BSQ_NVFP4) ? 16 : 4;
-    static constexpr int kSfbColsPerMma = 4 * kNbAtomTiles;
-    static constexpr int kSfbCols = (FMT == BSQ_NVFP4) ? 4 * kSfbColsPerMma : kSfbColsPerMma;
+    // TMEM scale-factor slots: NVFP4 copies one slot per MMA (4 SFA columns
+    // + 4 per 128 rows of B), MXFP8 one slot per k-tile (its atoms cover the
+    // 4 MMAs of the k-tile, selected by the scale-factor id)
+    static constexpr int kSlotCols = 4 + 4 * kNbAtomTiles;
+    static constexpr int kSlots = 8;
     static constexpr int kMmaPerKt = T::kBkElems / T::kMmaK;  // 4
+    static constexpr int kEpiWarps = 8;
+    static constexpr int kThreads = 32 * (2 + kEpiWarps);
 };
 
 // Tile -> (group, m tile, n tile) for the persistent loop.
@@ -119,7 +127,7 @@ BSQ_DEV TileInfo tile_info(int64_t t, int64_t m_tiles, const GemmParams &p, cons
 }
 
 template <int FMT, int BN, int ACC, bool OUT_BF16, bool SWAP, bool GROUPED>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     gemm_bs_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const GemmParams p) {
     using C_ = Cfg<FMT, BN>;
@@ -151,7 +159,7 @@ __global__ void __launch_bounds__(192, 1)
         }
         for (int i = 0; i < ACC; i++) {
             mbar_init(smem_u32(&accf_bar[i]), 1);
-            mbar_init(smem_u32(&acce_bar[i]), 4);
+            mbar_init(smem_u32(&acce_bar[i]), C_::kEpiWarps);
         }
         mbar_init(smem_u32(&drain_bar), 1);
         abort_flag = 0;
@@ -197,8 +205,8 @@ __global__ void __launch_bounds__(192, 1)
     const uint32_t tmem_base = tmem_base_slot;
     if (GROUPED) total_tiles = tile_start[p.G];
 
-    constexpr int SF_TMEM0 = ACC * BN;  // first TMEM column of the scale-factor buffers
-    constexpr int SF_BUF = C_::kSfaCols + C_::kSfbCols;
+    constexpr int SF_TMEM0 = ACC * BN;  // first TMEM column of the scale-factor slots
+    static_assert(ACC * BN + C_::kSlots * C_::kSlotCols <= 512, "TMEM budget");
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
@@ -256,6 +264,7 @@ __global__ void __launch_bounds__(192, 1)
             uint32_t ph = 0;
             bool ok = true;
             bool issued = false;
+            uint32_t slot_ctr = 0;
             int64_t it = 0;
             for (int64_t t = blockIdx.x; t < total_tiles && ok; t += gridDim.x, it++) {
                 const int a = (int)(it % ACC);
@@ -274,35 +283,35 @@ __global__ void __launch_bounds__(192, 1)
                     tc_fence_after();
                     const int64_t krem = p.K - kt * T::kBkElems;
                     const int nmma = krem >= T::kBkElems ? C_::kMmaPerKt : (int)(krem / T::kMmaK);
-                    const uint32_t sfa_t = tmem_base + SF_TMEM0 + (uint32_t)((kt & 1) * SF_BUF);
-                    const uint32_t sfb_t = sfa_t + C_::kSfaCols;
                     const uint32_t sfa_s = smem_u32(sSFA + s * C_::kSfaBytes);
                     const uint32_t sfb_s = smem_u32(sSFB + s * C_::kSfbBytes);
-                    if (FMT == BSQ_NVFP4) {
-                        for (int j = 0; j < nmma; j++) {
-                            tmem_cp_sf_atom(sfa_t + 4 * j, smem_desc(sfa_s + 512 * j, 0, 128, 0));
-                            for (int r = 0; r < C_::kNbAtomTiles; r++)
-                                tmem_cp_sf_atom(sfb_t + j * C_::kSfbColsPerMma + 4 * r,
-                                                smem_desc(sfb_s + r * C_::kSfaBytes + 512 * j, 0, 128, 0));
-                        }
-                    } else {
-                        tmem_cp_sf_atom(sfa_t, smem_desc(sfa_s, 0, 128, 0));
-                        for (int r = 0; r < C_::kNbAtomTiles; r++)
-                            tmem_cp_sf_atom(sfb_t + 4 * r, smem_desc(sfb_s + r * C_::kSfaBytes, 0, 128, 0));
-                    }
                     const uint32_t a_s = smem_u32(sA + s * C_::kABytes);
                     const uint32_t b_s = smem_u32(sB + s * C_::kBBytes);
-                    for (int j = 0; j < nmma; j++) {
-                        const uint64_t ad = smem_desc(a_s + 32 * j, 16, 1024, 2);
-                        const uint64_t bd = smem_desc(b_s + 32 * j, 16, 1024, 2);
-                        const uint32_t acc = (kt > 0 || j > 0) ? 1u : 0u;
-                        if (FMT == BSQ_NVFP4)
-                            mma_nvfp4(d_tmem, ad, bd, idesc, sfa_t + 4 * j, sfb_t + j * C_::kSfbColsPerMma, acc);
-                        else
+                    if (FMT == BSQ_NVFP4) {
+                        for (int j = 0; j < nmma; j++) {
+                            // the slot for this MMA: its SFA atom, then one atom per 128 rows of B
+                            const uint32_t slot = tmem_base + SF_TMEM0 + (uint32_t)((slot_ctr++ % C_::kSlots) * C_::kSlotCols);
+                            tmem_cp_sf_atom(slot, smem_desc(sfa_s + 512 * j, 0, 128, 0));
+                            for (int r = 0; r < C_::kNbAtomTiles; r++)
+                                tmem_cp_sf_atom(slot + 4 + 4 * r, smem_desc(sfb_s + r * C_::kSfaBytes + 512 * j, 0, 128, 0));
+                            const uint64_t ad = smem_desc(a_s + 32 * j, 16, 1024, 2);
+                            const uint64_t bd = smem_desc(b_s + 32 * j, 16, 1024, 2);
+                            mma_nvfp4(d_tmem, ad, bd, idesc, slot, slot + 4, (kt > 0 || j > 0) ? 1u : 0u);
+                        }
+                    } else {
+                        const uint32_t slot = tmem_base + SF_TMEM0 + (uint32_t)((slot_ctr++ % C_::kSlots) * C_::kSlotCols);
+                        tmem_cp_sf_atom(slot, smem_desc(sfa_s, 0, 128, 0));
+                        for (int r = 0; r < C_::kNbAtomTiles; r++)
+                            tmem_cp_sf_atom(slot + 4 + 4 * r, smem_desc(sfb_s + r * C_::kSfaBytes, 0, 128, 0));
+                        for (int j = 0; j < nmma; j++) {
+                            const uint64_t ad = smem_desc(a_s + 32 * j, 16, 1024, 2);
+                            const uint64_t bd = smem_desc(b_s + 32 * j, 16, 1024, 2);
                             // scale byte j of each 32-bit SF column: in the descriptor and in
                             // the top bits of the TMEM scale address
                             mma_mxfp8(d_tmem, ad, bd, idesc | ((uint32_t)j << 29) | ((uint32_t)j << 4),
-                                      sfa_t | ((uint32_t)j << 30), sfb_t | ((uint32_t)j << 30), acc);
+                                      slot | ((uint32_t)j << 30), (slot + 4) | ((uint32_t)j << 30),
+                                      (kt > 0 || j > 0) ? 1u : 0u);
+                        }
                     }
                     issued = true;
                     tc_commit(smem_u32(&empty_bar[s]));
@@ -323,7 +332,9 @@ __global__ void __launch_bounds__(192, 1)
         }
     } else {
         // ------------------------------------------------------------ epilogue
-        const int q = warp & 3;  // TMEM lane quarter this warp may access
+        const int q = warp & 3;             // TMEM lane quarter this warp may access
+        const int half = (warp - 2) >> 2;   // which half of the tile's columns
+        constexpr int HC = BN / 2;          // columns per warp
         const int row = 32 * q + lane;
         int64_t it = 0;
         for (int64_t t = blockIdx.x; t < total_tiles; t += gridDim.x, it++) {
@@ -340,32 +351,37 @@ __global__ void __launch_bounds__(192, 1)
             }
             const int64_t ar = ti.a_row0 + row;           // operand-A row of this thread
             const bool row_ok = ar < ti.m_lim;
-            const int64_t nb0 = ti.n0 * BN;
+            const int64_t nb0 = ti.n0 * BN + half * HC;   // first column of this warp
             const int64_t n_lim = p.n_lim;
-            const uint32_t tbase = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(a * BN);
+            const uint32_t tbase = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(a * BN + half * HC);
             if (OUT_BF16 && ACC == 1) {
-                // drain the whole accumulator into registers, release it, then store
-                uint32_t pk[BN / 2];
+                // drain this warp's columns into registers (two loads per wait),
+                // release the accumulator, then store
+                uint32_t pk[HC / 2];
 #pragma unroll
-                for (int c = 0; c < BN / 32; c++) {
-                    uint32_t r[32];
-                    tmem_ld32(tbase + 32 * c, r);
+                for (int c = 0; c < HC / 32; c += 2) {
+                    uint32_t r0[32], r1[32];
+                    tmem_ld32(tbase + 32 * c, r0);
+                    tmem_ld32(tbase + 32 * (c + 1), r1);
                     tmem_ld_wait();
 #pragma unroll
                     for (int j = 0; j < 16; j++) {
-                        __nv_bfloat162 h = __floats2bfloat162_rn(__fmul_rn(alpha, __uint_as_float(r[2 * j])),
-                                                                 __fmul_rn(alpha, __uint_as_float(r[2 * j + 1])));
-                        pk[16 * c + j] = *reinterpret_cast<uint32_t *>(&h);
+                        __nv_bfloat162 h0 = __floats2bfloat162_rn(__fmul_rn(alpha, __uint_as_float(r0[2 * j])),
+                                                                  __fmul_rn(alpha, __uint_as_float(r0[2 * j + 1])));
+                        __nv_bfloat162 h1 = __floats2bfloat162_rn(__fmul_rn(alpha, __uint_as_float(r1[2 * j])),
+                                                                  __fmul_rn(alpha, __uint_as_float(r1[2 * j + 1])));
+                        pk[16 * c + j] = *reinterpret_cast<uint32_t *>(&h0);
+                        pk[16 * (c + 1) + j] = *reinterpret_cast<uint32_t *>(&h1);
                     }
                 }
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(smem_u32(&acce_bar[a]));
+                if (!row_ok) continue;
 #pragma unroll
-                for (int c = 0; c < BN / 32; c++) {
+                for (int c = 0; c < HC / 32; c++) {
                     const int64_t n = nb0 + 32 * c;
                     if (!SWAP) {
-                        if (!row_ok) continue;
                         __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.C) + ar * p.ldc + n;
                         if (n + 32 <= n_lim) {
                             uint4 *d4 = reinterpret_cast<uint4 *>(dst);
@@ -383,7 +399,6 @@ __global__ void __launch_bounds__(192, 1)
                                 }
                         }
                     } else {
-                        if (!row_ok) continue;
 #pragma unroll
                         for (int j = 0; j < 32; j++)
                             if (n + j < n_lim) {
@@ -395,11 +410,11 @@ __global__ void __launch_bounds__(192, 1)
                 }
             } else {
 #pragma unroll 1
-                for (int c = 0; c < BN / 32; c++) {
+                for (int c = 0; c < HC / 32; c++) {
                     uint32_t r[32];
                     tmem_ld32(tbase + 32 * c, r);
                     tmem_ld_wait();
-                    if (c == BN / 32 - 1) {
+                    if (c == HC / 32 - 1) {
                         tc_fence_before();
                         __syncwarp();
                         if (lane == 0) mbar_arrive(smem_u32(&acce_bar[a]));
@@ -459,6 +474,364 @@ __global__ void __launch_bounds__(192, 1)
     }
 }
 
+// ============================================================ CTA-pair kernel
+// Two CTAs of a cluster compute one 256x256 tile with tcgen05 cta_group::2:
+// CTA r loads rows [128r, 128r+128) of the A tile, rows [128r, 128r+128) of
+// the B tile and all scale factors its MMA half needs (its own SFA rows, all
+// 256 SFB rows); the leader (r = 0) issues the copies and MMAs for both, and
+// each CTA's TMEM holds its 128 accumulator rows.  Per FLOP this moves ~30 %
+// fewer bytes from L2 than a 128x256 single-CTA tile.  No load uses
+// multicast: every CTA fetches its own tiles.
+template <int FMT>
+struct Cfg2 {
+    using T = FmtTraits<FMT>;
+    static constexpr int kABytes = 128 * 128;
+    static constexpr int kBBytes = 128 * 128;  // this CTA's half of the 256-row B tile
+    static constexpr int kSfaBytes = T::kAtomsPerKt * 512;
+    static constexpr int kSfbBytes = 2 * kSfaBytes;
+    static constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
+    static constexpr int kStages = (220 * 1024) / kStageBytes > 8 ? 8 : (220 * 1024) / kStageBytes;
+    static constexpr int kSmemBytes = kStages * kStageBytes + 1024;
+    static constexpr int kSlotCols = 12;  // 4 SFA + 8 SFB columns
+    static constexpr int kSlots = 8;
+    static constexpr int kMmaPerKt = T::kBkElems / T::kMmaK;
+    static constexpr int kEpiWarps = 8;
+    static constexpr int kThreads = 32 * (2 + kEpiWarps);
+    static constexpr int kSfBoxRows = kSfaBytes / 256;  // SF tensor-map box height (rows of 256 B)
+};
+
+template <int FMT, bool OUT_BF16, bool GROUPED>
+__global__ void __launch_bounds__(320, 1)
+    gemm_bs2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                    const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
+                    const GemmParams p) {
+    using C_ = Cfg2<FMT>;
+    using T = typename C_::T;
+    constexpr int NS = C_::kStages;
+    constexpr int BN = 256;
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ __align__(8) uint64_t full_bar[NS], empty_bar[NS], accf_bar, acce_bar, drain_bar;
+    __shared__ uint32_t tmem_base_slot;
+    __shared__ volatile int abort_flag;
+    __shared__ int tile_start[GROUPED ? 1025 : 1];
+    __shared__ int32_t offs[GROUPED ? 1025 : 1];
+
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sA = smem;
+    uint8_t *sB = sA + NS * C_::kABytes;
+    uint8_t *sSFA = sB + NS * C_::kBBytes;
+    uint8_t *sSFB = sSFA + NS * C_::kSfaBytes;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = rank == 0;
+    const int64_t pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+    const int64_t m_tiles = (p.MA + 255) / 256;
+    const int64_t n_tiles = (p.NB + BN - 1) / BN;
+    const int64_t k_tiles = (p.K + T::kBkElems - 1) / T::kBkElems;
+    const int64_t KBT = p.K / (T::kVec * 4);  // SF atoms per 128-row tile along K
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < NS; i++) {
+            mbar_init(smem_u32(&full_bar[i]), 1);
+            mbar_init(smem_u32(&empty_bar[i]), 1);
+        }
+        mbar_init(smem_u32(&accf_bar), 1);
+        mbar_init(smem_u32(&acce_bar), 2 * C_::kEpiWarps);
+        mbar_init(smem_u32(&drain_bar), 1);
+        abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tmap(&tmA);
+        prefetch_tmap(&tmB);
+        prefetch_tmap(&tmSFA);
+        prefetch_tmap(&tmSFB);
+    }
+    int64_t total_tiles = m_tiles * n_tiles;
+    if (GROUPED && warp == 2) {
+        for (int i = lane; i <= p.G; i += 32) offs[i] = __ldg(p.row_off + i);
+        __syncwarp();
+        int carry = 0;
+        for (int g0 = 0; g0 < p.G; g0 += 32) {
+            int g = g0 + lane;
+            int cnt = 0;
+            if (g < p.G) cnt = ((offs[g + 1] - offs[g] + 255) / 256) * (int)n_tiles;
+            int incl = cnt;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+                if (lane >= o) incl += v;
+            }
+            if (g < p.G) tile_start[g] = carry + incl - cnt;
+            carry += __shfl_sync(0xFFFFFFFFu, incl, 31);
+        }
+        if (lane == 0) tile_start[p.G] = carry;
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(smem_u32(&tmem_base_slot), 512);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();  // barriers of both CTAs are initialised before any remote arrive
+    tc_fence_after();
+    const uint32_t tmem_base = tmem_base_slot;
+    if (GROUPED) total_tiles = tile_start[p.G];
+
+    // (group, 256-row m tile, n tile) of pair tile t; rows of this CTA
+    auto info = [&](int64_t t, int64_t &a_row0, int64_t &sfa_row0, int64_t &m_lim, int64_t &nt, int &group) {
+        if (!GROUPED) {
+            const int64_t mt = t % m_tiles;
+            nt = t / m_tiles;
+            a_row0 = mt * 256 + 128 * rank;
+            sfa_row0 = a_row0;
+            m_lim = p.m_lim;
+            group = 0;
+            return;
+        }
+        int lo = 0, hi = p.G;
+        while (hi - lo > 1) {
+            int mid = (lo + hi) >> 1;
+            if (tile_start[mid] <= t) lo = mid; else hi = mid;
+        }
+        const int64_t local = t - tile_start[lo];
+        const int64_t mt_g = ((int64_t)offs[lo + 1] - offs[lo] + 255) / 256;
+        const int64_t mt = local % mt_g;
+        nt = local / mt_g;
+        a_row0 = (int64_t)offs[lo] + mt * 256 + 128 * rank;
+        sfa_row0 = (int64_t)__ldg(p.sf_row_off + lo) + mt * 256 + 128 * rank;
+        m_lim = offs[lo + 1];
+        group = lo;
+    };
+
+    // the leader's barriers, as seen from this CTA
+    const uint32_t full0 = mapa(smem_u32(&full_bar[0]), 0);
+    const uint32_t acce_leader = mapa(smem_u32(&acce_bar), 0);
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer (both CTAs)
+        if (lane == 0) {
+            int s = 0;
+            uint32_t ph = 0, armed = 0, armed_par = 0;
+            bool ok = true;
+            const uint32_t per_cta = C_::kABytes + C_::kBBytes + C_::kSfaBytes + C_::kSfbBytes;
+            for (int64_t t = pair; t < total_tiles && ok; t += npairs) {
+                int64_t a_row0, sfa_row0, m_lim, nt;
+                int group;
+                info(t, a_row0, sfa_row0, m_lim, nt, group);
+                const int64_t nb0 = nt * BN;
+                const int64_t b_row0 = (int64_t)group * p.NB + nb0 + 128 * rank;
+                // SF tensor maps address rows of 256 bytes
+                const int64_t sfa_r0 = (sfa_row0 / 128) * KBT * 2;
+                const int64_t sfb_r0 = (int64_t)group * (p.sfB_group_bytes / 256) + (nb0 / 128) * KBT * 2;
+                for (int64_t kt = 0; kt < k_tiles; kt++) {
+                    if (!mbar_wait(smem_u32(&empty_bar[s]), ph ^ 1u, &abort_flag, p.err, 1, kTimeoutNs)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t fb = full0 + (uint32_t)(s * 8);  // leader's full barrier of stage s
+                    if (leader) mbar_arrive_expect_tx(smem_u32(&full_bar[s]), 2 * per_cta);
+                    const int32_t kx = (int32_t)(kt * 128);
+                    const int32_t sfk = (int32_t)(kt * C_::kSfBoxRows);
+                    tma_load_2d_pair(smem_u32(sA + s * C_::kABytes), &tmA, fb, kx, (int32_t)a_row0);
+                    tma_load_2d_pair(smem_u32(sB + s * C_::kBBytes), &tmB, fb, kx, (int32_t)b_row0);
+                    tma_load_2d_pair(smem_u32(sSFA + s * C_::kSfaBytes), &tmSFA, fb, 0, (int32_t)(sfa_r0 + sfk));
+                    tma_load_2d_pair(smem_u32(sSFB + s * C_::kSfbBytes), &tmSFB, fb, 0, (int32_t)(sfb_r0 + sfk));
+                    tma_load_2d_pair(smem_u32(sSFB + s * C_::kSfbBytes + C_::kSfaBytes), &tmSFB, fb, 0,
+                                     (int32_t)(sfb_r0 + KBT * 2 + sfk));
+                    armed |= 1u << s;
+                    armed_par = (armed_par & ~(1u << s)) | (ph << s);
+                    if (++s == NS) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
+                }
+            }
+            if (leader) {
+                // every armed stage's latest phase has landed before exit
+                for (int i = 0; i < NS; i++)
+                    if (armed & (1u << i)) {
+                        volatile int never = 0;
+                        mbar_wait(smem_u32(&full_bar[i]), (armed_par >> i) & 1u, &never, p.err, 2, kTimeoutNs);
+                    }
+            } else {
+                // the peer's copies land on the leader's barriers; wait for the
+                // leader to release each armed stage (its MMAs read our smem)
+                for (int i = 0; i < NS; i++)
+                    if (armed & (1u << i)) {
+                        volatile int never = 0;
+                        mbar_wait(smem_u32(&empty_bar[i]), (armed_par >> i) & 1u, &never, p.err, 2, kTimeoutNs);
+                    }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer (leader only)
+        if (leader && lane == 0) {
+            const uint32_t idesc = T::kIdescFmt | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(256 >> 4) << 24);
+            int s = 0;
+            uint32_t ph = 0;
+            bool ok = true, issued = false;
+            uint32_t slot_ctr = 0;
+            int64_t it = 0;
+            for (int64_t t = pair; t < total_tiles && ok; t += npairs, it++) {
+                if (!mbar_wait(smem_u32(&acce_bar), (uint32_t)(it & 1) ^ 1u, &abort_flag, p.err, 3, kTimeoutNs)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base;
+                for (int64_t kt = 0; kt < k_tiles; kt++) {
+                    if (!mbar_wait(smem_u32(&full_bar[s]), ph, &abort_flag, p.err, 4, kTimeoutNs)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const int64_t krem = p.K - kt * T::kBkElems;
+                    const int nmma = krem >= T::kBkElems ? C_::kMmaPerKt : (int)(krem / T::kMmaK);
+                    const uint32_t sfa_s = smem_u32(sSFA + s * C_::kSfaBytes);
+                    const uint32_t sfb_s = smem_u32(sSFB + s * C_::kSfbBytes);
+                    const uint32_t a_s = smem_u32(sA + s * C_::kABytes);
+                    const uint32_t b_s = smem_u32(sB + s * C_::kBBytes);
+                    if (FMT == BSQ_NVFP4) {
+                        for (int j = 0; j < nmma; j++) {
+                            const uint32_t slot = tmem_base + 256 + (uint32_t)((slot_ctr++ % C_::kSlots) * C_::kSlotCols);
+                            tmem_cp_sf_atom_pair(slot, smem_desc(sfa_s + 512 * j, 0, 128, 0));
+                            tmem_cp_sf_atom_pair(slot + 4, smem_desc(sfb_s + 512 * j, 0, 128, 0));
+                            tmem_cp_sf_atom_pair(slot + 8, smem_desc(sfb_s + C_::kSfaBytes + 512 * j, 0, 128, 0));
+                            mma_nvfp4_pair(d_tmem, smem_desc(a_s + 32 * j, 16, 1024, 2), smem_desc(b_s + 32 * j, 16, 1024, 2),
+                                           idesc, slot, slot + 4, (kt > 0 || j > 0) ? 1u : 0u);
+                        }
+                    } else {
+                        const uint32_t slot = tmem_base + 256 + (uint32_t)((slot_ctr++ % C_::kSlots) * C_::kSlotCols);
+                        tmem_cp_sf_atom_pair(slot, smem_desc(sfa_s, 0, 128, 0));
+                        tmem_cp_sf_atom_pair(slot + 4, smem_desc(sfb_s, 0, 128, 0));
+                        tmem_cp_sf_atom_pair(slot + 8, smem_desc(sfb_s + C_::kSfaBytes, 0, 128, 0));
+                        for (int j = 0; j < nmma; j++)
+                            mma_mxfp8_pair(d_tmem, smem_desc(a_s + 32 * j, 16, 1024, 2), smem_desc(b_s + 32 * j, 16, 1024, 2),
+                                           idesc | ((uint32_t)j << 29) | ((uint32_t)j << 4), slot | ((uint32_t)j << 30),
+                                           (slot + 4) | ((uint32_t)j << 30), (kt > 0 || j > 0) ? 1u : 0u);
+                    }
+                    issued = true;
+                    tc_commit_pair(smem_u32(&empty_bar[s]), 0x3);  // release stage s in both CTAs
+                    if (++s == NS) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                tc_commit_pair(smem_u32(&accf_bar), 0x3);
+            }
+            if (issued) {
+                tc_commit_pair(smem_u32(&drain_bar), 0x1);
+                volatile int never = 0;
+                mbar_wait(smem_u32(&drain_bar), 0, &never, p.err, 5, kTimeoutNs);
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue (both CTAs)
+        const int q = warp & 3;
+        const int half = (warp - 2) >> 2;
+        constexpr int HC = BN / 2;
+        const int row = 32 * q + lane;
+        int64_t it = 0;
+        for (int64_t t = pair; t < total_tiles; t += npairs, it++) {
+            int64_t a_row0, sfa_row0, m_lim, nt;
+            int group;
+            info(t, a_row0, sfa_row0, m_lim, nt, group);
+            if (!mbar_wait(smem_u32(&accf_bar), (uint32_t)(it & 1), &abort_flag, p.err, 6, kTimeoutNs)) break;
+            tc_fence_after();
+            float alpha = 1.0f;
+            if (FMT == BSQ_NVFP4) {
+                const float ga = p.gsA ? __ldg(p.gsA) : 1.0f;
+                const float gb = p.gsB ? __ldg(p.gsB + group) : 1.0f;
+                alpha = __fmul_rn(ga, gb);
+            }
+            const int64_t ar = a_row0 + row;
+            const bool row_ok = ar < m_lim;
+            const int64_t nb0 = nt * BN + half * HC;
+            const int64_t n_lim = p.n_lim;
+            const uint32_t tbase = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(half * HC);
+            if (OUT_BF16) {
+                uint32_t pk[HC / 2];
+#pragma unroll
+                for (int c = 0; c < HC / 32; c += 2) {
+                    uint32_t r0[32], r1[32];
+                    tmem_ld32(tbase + 32 * c, r0);
+                    tmem_ld32(tbase + 32 * (c + 1), r1);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int j = 0; j < 16; j++) {
+                        __nv_bfloat162 h0 = __floats2bfloat162_rn(__fmul_rn(alpha, __uint_as_float(r0[2 * j])),
+                                                                  __fmul_rn(alpha, __uint_as_float(r0[2 * j + 1])));
+                        __nv_bfloat162 h1 = __floats2bfloat162_rn(__fmul_rn(alpha, __uint_as_float(r1[2 * j])),
+                                                                  __fmul_rn(alpha, __uint_as_float(r1[2 * j + 1])));
+                        pk[16 * c + j] = *reinterpret_cast<uint32_t *>(&h0);
+                        pk[16 * (c + 1) + j] = *reinterpret_cast<uint32_t *>(&h1);
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(acce_leader);
+                if (!row_ok) continue;
+#pragma unroll
+                for (int c = 0; c < HC / 32; c++) {
+                    const int64_t n = nb0 + 32 * c;
+                    __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.C) + ar * p.ldc + n;
+                    if (n + 32 <= n_lim) {
+                        uint4 *d4 = reinterpret_cast<uint4 *>(dst);
+#pragma unroll
+                        for (int v = 0; v < 4; v++)
+                            d4[v] = make_uint4(pk[16 * c + 4 * v], pk[16 * c + 4 * v + 1], pk[16 * c + 4 * v + 2],
+                                               pk[16 * c + 4 * v + 3]);
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 32; j++)
+                            if (n + j < n_lim) {
+                                uint32_t w = pk[16 * c + j / 2];
+                                reinterpret_cast<uint16_t *>(dst)[j] = (j & 1) ? (uint16_t)(w >> 16) : (uint16_t)(w & 0xFFFFu);
+                            }
+                    }
+                }
+            } else {
+#pragma unroll 1
+                for (int c = 0; c < HC / 32; c++) {
+                    uint32_t r[32];
+                    tmem_ld32(tbase + 32 * c, r);
+                    tmem_ld_wait();
+                    if (c == HC / 32 - 1) {
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive_cluster(acce_leader);
+                    }
+                    if (!row_ok) continue;
+                    const int64_t n = nb0 + 32 * c;
+                    float *dst = static_cast<float *>(p.C) + ar * p.ldc + n;
+                    if (n + 32 <= n_lim) {
+                        float4 *d4 = reinterpret_cast<float4 *>(dst);
+#pragma unroll
+                        for (int x = 0; x < 8; x++)
+                            d4[x] = make_float4(__fmul_rn(alpha, __uint_as_float(r[4 * x])),
+                                                __fmul_rn(alpha, __uint_as_float(r[4 * x + 1])),
+                                                __fmul_rn(alpha, __uint_as_float(r[4 * x + 2])),
+                                                __fmul_rn(alpha, __uint_as_float(r[4 * x + 3])));
+                    } else {
+                        for (int j = 0; j < 32; j++)
+                            if (n + j < n_lim) dst[j] = __fmul_rn(alpha, __uint_as_float(r[j]));
+                    }
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();  // the peer's shared memory stays valid until the pair is done
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem_base, 512);
+    }
+}
+
 // ============================================================ timeout probe
 __global__ void timeout_probe_kernel(uint64_t timeout_ns, unsigned int *err) {
     __shared__ __align__(8) uint64_t bar;
@@ -509,6 +882,47 @@ bool make_tmap(CUtensorMap *m, const void *base, int64_t row_bytes, int64_t rows
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+
+// 2-D uint8 tensor map over a scale-factor buffer seen as rows of 256 bytes.
+bool make_sf_tmap(CUtensorMap *m, const void *base, int64_t bytes, int box_rows) {
+    EncodeFn enc = get_encode();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {256u, (cuuint64_t)(bytes / 256)};
+    cuuint64_t strides[1] = {256u};
+    cuuint32_t box[2] = {256u, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1u, 1u};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int FMT, bool OUT_BF16, bool GROUPED>
+int run_pair(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &tsa, const CUtensorMap &tsb,
+             const GemmParams &p, int pairs, cudaStream_t s) {
+    using C_ = Cfg2<FMT>;
+    auto kern = gemm_bs2_kernel<FMT, OUT_BF16, GROUPED>;
+    static bool attr_set = false;
+    if (!attr_set) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C_::kSmemBytes) != cudaSuccess)
+            return BSQ_ERR_CUDA;
+        attr_set = true;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * pairs, 1, 1);
+    cfg.blockDim = dim3(C_::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = C_::kSmemBytes;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, ta, tb, tsa, tsb, p) != cudaSuccess) return BSQ_ERR_CUDA;
+    return cudaGetLastError() == cudaSuccess ? BSQ_OK : BSQ_ERR_CUDA;
+}
+
 template <int FMT, int BN, int ACC, bool OUT_BF16, bool SWAP, bool GROUPED>
 int run(const CUtensorMap &ta, const CUtensorMap &tb, const GemmParams &p, int grid, cudaStream_t s) {
     using C_ = Cfg<FMT, BN>;
@@ -519,7 +933,7 @@ int run(const CUtensorMap &ta, const CUtensorMap &tb, const GemmParams &p, int g
             return BSQ_ERR_CUDA;
         attr_set = true;
     }
-    kern<<<grid, 192, C_::kSmemBytes, s>>>(ta, tb, p);
+    kern<<<grid, C_::kThreads, C_::kSmemBytes, s>>>(ta, tb, p);
     return cudaGetLastError() == cudaSuccess ? BSQ_OK : BSQ_ERR_CUDA;
 }
 
@@ -538,7 +952,12 @@ int dispatch(const GemmArgs &g, cudaStream_t s) {
     if (swap) bn = 64;
     else if (g.out_bf16 && NB >= 256) bn = 256;
     else bn = 128;
-    if (const char *e = getenv("BSQ_GEMM_BN")) {  // debug/tuning override
+    // CTA pairs for everything but the skinny swap-AB case (debug knob: BSQ_GEMM_PAIR=0)
+    // (grouped NVFP4 with a half k-tile would need the exact extent of A's
+    // scale buffer, which only the device knows: it stays on single CTAs)
+    bool use_pair = !swap && NB >= 128 && !(grouped && FMT == BSQ_NVFP4 && g.K % 256 != 0);
+    if (const char *e = getenv("BSQ_GEMM_PAIR")) use_pair = use_pair && atoi(e) != 0;
+    if (const char *e = getenv("BSQ_GEMM_BN")) {  // debug/tuning override of the single-CTA tile
         int v = atoi(e);
         if ((v == 128 || (v == 256 && g.out_bf16)) && !swap) bn = v;
     }
@@ -552,6 +971,26 @@ int dispatch(const GemmArgs &g, cudaStream_t s) {
     p.err = g.err;
     CUtensorMap ta, tb;
     if (!make_tmap(&ta, opA, kb_bytes, MA, 128)) return BSQ_ERR_CUDA;
+    if (use_pair) {
+        CUtensorMap tsa, tsb;
+        if (!make_tmap(&tb, opB, kb_bytes, grouped ? (int64_t)g.G * NB : NB, 128)) return BSQ_ERR_CUDA;
+        const int64_t kbp = (g.K / T::kVec + 3) / 4 * 4;
+        const int64_t sfa_rows = grouped ? 0 : (MA + 127) / 128 * 128;
+        // grouped A: the SF buffer spans sf_row_offsets[G] rows; its size is not
+        // known on the host, so map the largest extent the groups can reach
+        const int64_t sfa_bytes = grouped ? ((MA + 128LL * g.G + 127) / 128 * 128) * kbp : sfa_rows * kbp;
+        const int64_t sfb_bytes = (grouped ? (int64_t)g.G : 1) * p.sfB_group_bytes;
+        const int box = Cfg2<FMT>::kSfBoxRows;
+        if (!make_sf_tmap(&tsa, sfA, sfa_bytes, box) || !make_sf_tmap(&tsb, sfB, sfb_bytes, box)) return BSQ_ERR_CUDA;
+        int64_t ptiles = grouped ? (MA / 256 + g.G) * ((NB + 255) / 256) : ((MA + 255) / 256) * ((NB + 255) / 256);
+        int pairs = (int)(ptiles < g.num_sms / 2 ? (ptiles < 1 ? 1 : ptiles) : g.num_sms / 2);
+        if (grouped) {
+            if (g.out_bf16) return run_pair<FMT, true, true>(ta, tb, tsa, tsb, p, pairs, s);
+            return run_pair<FMT, false, true>(ta, tb, tsa, tsb, p, pairs, s);
+        }
+        if (g.out_bf16) return run_pair<FMT, true, false>(ta, tb, tsa, tsb, p, pairs, s);
+        return run_pair<FMT, false, false>(ta, tb, tsa, tsb, p, pairs, s);
+    }
     if (!make_tmap(&tb, opB, kb_bytes, grouped ? (int64_t)g.G * NB : NB, bn)) return BSQ_ERR_CUDA;
     int64_t tiles;
     if (!grouped) tiles = ((MA + 127) / 128) * ((NB + bn - 1) / bn);

@@ -38,6 +38,20 @@ BSQ_DEV bool mbar_try_wait(uint32_t bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
+// try_wait with a suspend-time hint: the thread is descheduled until the
+// phase completes or about hint_ns pass, so waiting warps do not spin on the
+// scheduler (and steal issue slots from the warps doing the work).
+BSQ_DEV bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
 
 // Bounded wait: gives up when *abort is set by another warp, or after
 // timeout_ns of device time (then sets *abort and records `site` in the
@@ -46,15 +60,13 @@ BSQ_DEV bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort, unsig
                        uint64_t timeout_ns) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
-    for (uint32_t n = 1;; n++) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((n & 63u) == 0) {
-            if (*abort) return false;
-            if (globaltimer_ns() - t0 > timeout_ns) {
-                *abort = 1;
-                report_timeout(err, site);
-                return false;
-            }
+    for (;;) {
+        if (mbar_try_wait_sleep(bar, parity, 100000u)) return true;  // sleeps up to ~0.1 ms
+        if (*abort) return false;
+        if (globaltimer_ns() - t0 > timeout_ns) {
+            *abort = 1;
+            report_timeout(err, site);
+            return false;
         }
     }
 }

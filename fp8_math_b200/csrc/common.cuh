@@ -146,9 +146,94 @@ BSQ_DEV uint32_t e4m3_sr(float v, uint32_t r16) {
     return sgn | e4m3_rne(mag);
 }
 
+// ---------------------------------------------------------------- fp32 pairs
+// sm_100 executes two fp32 operations per instruction on a 64-bit register
+// pair (add/sub/mul.rn.f32x2); each lane is an ordinary IEEE RN operation.
+typedef unsigned long long f32x2;
+BSQ_DEV f32x2 f2_pack(float lo, float hi) {
+    f32x2 r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+BSQ_DEV void f2_unpack(f32x2 r, float &lo, float &hi) { asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(r)); }
+BSQ_DEV f32x2 f2_add(f32x2 a, f32x2 b) {
+    f32x2 r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+BSQ_DEV f32x2 f2_sub(f32x2 a, f32x2 b) {
+    f32x2 r;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+BSQ_DEV f32x2 f2_mul(f32x2 a, f32x2 b) {
+    f32x2 r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+
 // ---------------------------------------------------------------- RHT
-// In-place 16-point transform y = 1/4 * H16 * diag(s) * x; butterflies of
-// stride 1, 2, 4, 8 (Sylvester order).
+// Sign words for the 16-point RHT applied to packed bf16 pairs: word k flips
+// element 2k (bit 15) and 2k+1 (bit 31) where the sign vector says s = -1.
+BSQ_DEV void rht_sign_words(uint32_t mask, uint32_t sw[8]) {
+#pragma unroll
+    for (int k = 0; k < 8; k++) sw[k] = (((mask >> (2 * k)) & 1u) << 15) | (((mask >> (2 * k + 1)) & 1u) << 31);
+}
+
+// Loads 16 bf16 (two 16-byte loads), applies the signs and the Sylvester
+// butterflies of stride 1, 2, 4, 8 (in that order, each an RN add or
+// subtract) and the exact 1/4 scaling: y = 1/4 * H16 * diag(s) * x as 8 fp32
+// pairs (element 2k in the low lane of pair k).
+BSQ_DEV void load_rht16(const uint16_t *p, const uint32_t sw[8], f32x2 P[8]) {
+    const uint4 q0 = __ldg(reinterpret_cast<const uint4 *>(p));
+    const uint4 q1 = __ldg(reinterpret_cast<const uint4 *>(p + 8));
+    const uint32_t w[8] = {q0.x ^ sw[0], q0.y ^ sw[1], q0.z ^ sw[2], q0.w ^ sw[3],
+                           q1.x ^ sw[4], q1.y ^ sw[5], q1.z ^ sw[6], q1.w ^ sw[7]};
+#pragma unroll
+    for (int k = 0; k < 8; k++) {
+        const float a = bf16_lo(w[k]), b = bf16_hi(w[k]);
+        P[k] = f2_pack(__fadd_rn(a, b), __fsub_rn(a, b));  // stride 1
+    }
+#pragma unroll
+    for (int h = 1; h < 8; h <<= 1) {  // strides 2, 4, 8 as pair strides 1, 2, 4
+#pragma unroll
+        for (int base = 0; base < 8; base += 2 * h) {
+#pragma unroll
+            for (int k = base; k < base + h; k++) {
+                const f32x2 a = P[k], b = P[k + h];
+                P[k] = f2_add(a, b);
+                P[k + h] = f2_sub(a, b);
+            }
+        }
+    }
+    const f32x2 quarter = f2_pack(0.25f, 0.25f);
+#pragma unroll
+    for (int k = 0; k < 8; k++) P[k] = f2_mul(P[k], quarter);
+}
+
+// Loads 16 bf16 as 8 fp32 pairs (no transform).
+BSQ_DEV void load16_pairs(const uint16_t *p, f32x2 P[8]) {
+    const uint4 q0 = __ldg(reinterpret_cast<const uint4 *>(p));
+    const uint4 q1 = __ldg(reinterpret_cast<const uint4 *>(p + 8));
+    const uint32_t w[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+#pragma unroll
+    for (int k = 0; k < 8; k++) P[k] = f2_pack(bf16_lo(w[k]), bf16_hi(w[k]));
+}
+
+// max |v| over 8 pairs
+BSQ_DEV float pairs_absmax(const f32x2 P[8]) {
+    float m = 0.0f;
+#pragma unroll
+    for (int k = 0; k < 8; k++) {
+        float a, b;
+        f2_unpack(P[k], a, b);
+        m = fmaxf(m, fmaxf(fabsf(a), fabsf(b)));
+    }
+    return m;
+}
+
+// In-place 16-point transform y = 1/4 * H16 * diag(s) * x on fp32 values
+// (scalar form, used where the values are needed one by one).
 BSQ_DEV void rht16(float v[16], uint32_t mask) {
 #pragma unroll
     for (int i = 0; i < 16; i++)

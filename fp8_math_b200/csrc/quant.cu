@@ -34,6 +34,8 @@ __global__ void __launch_bounds__(256) amax_kernel(const uint16_t *__restrict__ 
     const int lpr = 1 << map.lpr_shift;
     const int rpi = 256 >> map.lpr_shift;
     const int sub = threadIdx.x >> map.lpr_shift, lk = threadIdx.x & (lpr - 1);
+    uint32_t sw[8];
+    rht_sign_words(mask, sw);
     float m = 0.0f;
     for (int64_t r0 = (int64_t)blockIdx.x * rpi; r0 < M; r0 += (int64_t)gridDim.x * rpi) {
         const int64_t row = r0 + sub;
@@ -41,12 +43,10 @@ __global__ void __launch_bounds__(256) amax_kernel(const uint16_t *__restrict__ 
         const int64_t src = GATHER ? (int64_t)__ldg(row_index + row) : row;
         const uint16_t *rp = x + src * ldx;
         for (int64_t kb = lk; kb < KB; kb += lpr) {
-            float v[16];
-            load8_bf16(rp + kb * 16, v);
-            load8_bf16(rp + kb * 16 + 8, v + 8);
-            if (RHT) rht16(v, mask);
-#pragma unroll
-            for (int i = 0; i < 16; i++) m = fmaxf(m, fabsf(v[i]));
+            f32x2 P[8];
+            if (RHT) load_rht16(rp + kb * 16, sw, P);
+            else load16_pairs(rp + kb * 16, P);
+            m = fmaxf(m, pairs_absmax(P));
         }
     }
 #pragma unroll
@@ -75,7 +75,7 @@ struct NvCand {
     uint2 codes;
 };
 
-BSQ_DEV NvCand nv_candidate(const float v[16], float bamax, float divisor, float s_g) {
+BSQ_DEV NvCand nv_candidate(const f32x2 P[8], float bamax, float divisor, float s_g) {
     NvCand c;
     float t = __fdiv_rn(__fdiv_rn(bamax, divisor), s_g);
     c.sb = e4m3_rne(t);
@@ -86,17 +86,21 @@ BSQ_DEV NvCand nv_candidate(const float v[16], float bamax, float divisor, float
         return c;
     }
     c.den = __fmul_rn(sbv, s_g);
-    float r = __frcp_rn(c.den);
+    const float r = __frcp_rn(c.den);
+    const f32x2 R = f2_pack(r, r);
     float q[16];
 #pragma unroll
-    for (int i = 0; i < 16; i++) q[i] = __fmul_rn(v[i], r);
+    for (int k = 0; k < 8; k++) f2_unpack(f2_mul(P[k], R), q[2 * k], q[2 * k + 1]);
     c.codes.x = cvt_e2m1x8(q);
     c.codes.y = cvt_e2m1x8(q + 8);
     return c;
 }
 
 // Squared error of a candidate, summed pairwise (0+1),(2+3),... four levels.
-BSQ_DEV float nv_block_err(const float v[16], const NvCand &c) {
+BSQ_DEV float nv_block_err(const f32x2 P[8], const NvCand &c) {
+    float v[16];
+#pragma unroll
+    for (int k = 0; k < 8; k++) f2_unpack(P[k], v[2 * k], v[2 * k + 1]);
     float e[16];
 #pragma unroll
     for (int i = 0; i < 16; i++) {
@@ -153,6 +157,8 @@ __global__ void __launch_bounds__(256) quant_nvfp4_1d_kernel(
     const bool pack4 = (KB & 3) == 0;
     const float s_g = global_scale_of(*amax_ptr);
     if (write_gs && blockIdx.x == 0 && threadIdx.x == 0) *gs_out = s_g;
+    uint32_t sw[8];
+    rht_sign_words(mask, sw);
     const int lpr = 1 << map.lpr_shift;
     const int rpi = 256 >> map.lpr_shift;
     const int sub = threadIdx.x >> map.lpr_shift, lk = threadIdx.x & (lpr - 1);
@@ -167,17 +173,14 @@ __global__ void __launch_bounds__(256) quant_nvfp4_1d_kernel(
             const int64_t kb = kb0 + lk;
             const bool valid = row_ok && kb < KB;
             const int64_t kk = kb < KB ? kb : KB - 1;
-            float v[16];
-            load8_bf16(rp + kk * 16, v);
-            load8_bf16(rp + kk * 16 + 8, v + 8);
-            if (RHT) rht16(v, mask);
-            float bamax = 0.0f;
-#pragma unroll
-            for (int i = 0; i < 16; i++) bamax = fmaxf(bamax, fabsf(v[i]));
-            NvCand c = nv_candidate(v, bamax, 6.0f, s_g);
+            f32x2 P[8];
+            if (RHT) load_rht16(rp + kk * 16, sw, P);
+            else load16_pairs(rp + kk * 16, P);
+            const float bamax = pairs_absmax(P);
+            NvCand c = nv_candidate(P, bamax, 6.0f, s_g);
             if (FOS) {
-                NvCand c4 = nv_candidate(v, bamax, 4.0f, s_g);
-                if (nv_block_err(v, c4) < nv_block_err(v, c)) c = c4;
+                NvCand c4 = nv_candidate(P, bamax, 4.0f, s_g);
+                if (nv_block_err(P, c4) < nv_block_err(P, c)) c = c4;
             }
             if (valid) *reinterpret_cast<uint2 *>(codes + rr * (K >> 1) + kb * 8) = c.codes;
             store_sf(sf, valid, c.sb, sf_row, kb, KB, pack4);
@@ -198,32 +201,31 @@ __global__ void __launch_bounds__(512) quant_nvfp4_2d_kernel(
     const bool pack4 = (KB & 3) == 0;
     const float s_g = global_scale_of(*amax_ptr);
     if (write_gs && blockIdx.x == 0 && threadIdx.x == 0) *gs_out = s_g;
+    uint32_t sw[8];
+    rht_sign_words(mask, sw);
     const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
     for (uint32_t t = blockIdx.x; t < tiles; t += gridDim.x) {
         const uint32_t rt = t / kb_tiles, kt = t - rt * kb_tiles;
         const int64_t row = (int64_t)rt * 16 + w;
         const int64_t kb = (int64_t)kt * 32 + lane;
         const bool valid = kb < KB;
-        float v[16];
+        f32x2 P[8];
         if (valid) {
             const uint16_t *p = x + row * ldx + kb * 16;
-            load8_bf16(p, v);
-            load8_bf16(p + 8, v + 8);
-            if (RHT) rht16(v, mask);
+            if (RHT) load_rht16(p, sw, P);
+            else load16_pairs(p, P);
         } else {
 #pragma unroll
-            for (int i = 0; i < 16; i++) v[i] = 0.0f;
+            for (int k = 0; k < 8; k++) P[k] = 0ull;
         }
-        float bamax = 0.0f;
-#pragma unroll
-        for (int i = 0; i < 16; i++) bamax = fmaxf(bamax, fabsf(v[i]));
+        const float bamax = pairs_absmax(P);
         tile_amax[w][lane] = bamax;
         __syncthreads();
         float tmax = 0.0f;
 #pragma unroll
         for (int r = 0; r < 16; r++) tmax = fmaxf(tmax, tile_amax[r][lane]);
         __syncthreads();
-        NvCand c = nv_candidate(v, tmax, 6.0f, s_g);
+        NvCand c = nv_candidate(P, tmax, 6.0f, s_g);
         if (valid) *reinterpret_cast<uint2 *>(codes + row * (K >> 1) + kb * 8) = c.codes;
         store_sf(sf, valid, c.sb, row, kb, KB, pack4);
     }
@@ -429,6 +431,8 @@ __global__ void __launch_bounds__(256) quant_mxfp8_col_kernel(
 __global__ void __launch_bounds__(256) rht_kernel(const uint16_t *__restrict__ x, uint16_t *y, int64_t M,
                                                   int64_t K, int64_t ldx, int64_t ldy, uint32_t mask, RowMap map) {
     const int64_t KB = K >> 4;
+    uint32_t sw[8];
+    rht_sign_words(mask, sw);
     const int lpr = 1 << map.lpr_shift;
     const int rpi = 256 >> map.lpr_shift;
     const int sub = threadIdx.x >> map.lpr_shift, lk = threadIdx.x & (lpr - 1);
@@ -436,14 +440,14 @@ __global__ void __launch_bounds__(256) rht_kernel(const uint16_t *__restrict__ x
         const int64_t row = r0 + sub;
         if (row >= M) continue;
         for (int64_t kb = lk; kb < KB; kb += lpr) {
-            float v[16];
-            load8_bf16(x + row * ldx + kb * 16, v);
-            load8_bf16(x + row * ldx + kb * 16 + 8, v + 8);
-            rht16(v, mask);
+            f32x2 P[8];
+            load_rht16(x + row * ldx + kb * 16, sw, P);
             uint32_t w[8];
 #pragma unroll
             for (int i = 0; i < 8; i++) {
-                __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+                float a, b;
+                f2_unpack(P[i], a, b);
+                __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
                 w[i] = *reinterpret_cast<uint32_t *>(&h);
             }
             uint4 *q = reinterpret_cast<uint4 *>(y + row * ldy + kb * 16);

@@ -82,7 +82,7 @@ struct Cfg {
     // + 4 per 128 rows of B), MXFP8 one slot per k-tile (its atoms cover the
     // 4 MMAs of the k-tile, selected by the scale-factor id)
     static constexpr int kSlotCols = 4 + 4 * kNbAtomTiles;
-    static constexpr int kSlots = 8;
+    static constexpr int kSlots = (FMT == BSQ_NVFP4) ? 16 : 8;
     static constexpr int kMmaPerKt = T::kBkElems / T::kMmaK;  // 4
     static constexpr int kEpiWarps = 8;
     static constexpr int kThreads = 32 * (2 + kEpiWarps);
@@ -258,13 +258,23 @@ __global__ void __launch_bounds__(320, 1)
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
+        // One thread issues every tcgen05 op, so its own instruction count
+        // bounds the MMA rate: descriptors are kept as 32-bit words and
+        // stepped with adds, the per-MMA offsets are compile-time constants.
         if (lane == 0) {
-            uint32_t idesc = T::kIdescFmt | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+            const uint32_t idesc = T::kIdescFmt | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+            constexpr uint32_t kOpHi = smem_desc_hi(1024, 2);  // K-major, 128-byte swizzle, 8-row groups 1 KB apart
+            constexpr uint32_t kSfHi = smem_desc_hi(128, 0);   // scale atoms: 32 rows of 16 bytes
+            const uint32_t a_lo0 = smem_desc_lo(smem_u32(sA), 16), b_lo0 = smem_desc_lo(smem_u32(sB), 16);
+            const uint32_t sfa_lo0 = smem_desc_lo(smem_u32(sSFA), 0), sfb_lo0 = smem_desc_lo(smem_u32(sSFB), 0);
+            const uint32_t sf_t0 = tmem_base + SF_TMEM0;
+            constexpr uint32_t kSfAtomLo = 512 >> 4;                // one atom, in descriptor units
+            constexpr uint32_t kSfbTileLo = C_::kSfaBytes >> 4;    // next 128 rows of B
             int s = 0;
             uint32_t ph = 0;
             bool ok = true;
             bool issued = false;
-            uint32_t slot_ctr = 0;
+            uint32_t ktc = 0;  // k-tiles issued: selects the scale slots
             int64_t it = 0;
             for (int64_t t = blockIdx.x; t < total_tiles && ok; t += gridDim.x, it++) {
                 const int a = (int)(it % ACC);
@@ -275,42 +285,57 @@ __global__ void __launch_bounds__(320, 1)
                 }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(a * BN);
-                for (int64_t kt = 0; kt < k_tiles; kt++) {
-                    if (!mbar_wait(smem_u32(&full_bar[s]), ph, &abort_flag, p.err, 4, kTimeoutNs)) {
+                for (int64_t kt = 0; kt < k_tiles; kt++, ktc++) {
+                    if (!mbar_test_wait(smem_u32(&full_bar[s]), ph) &&
+                        !mbar_wait(smem_u32(&full_bar[s]), ph, &abort_flag, p.err, 4, kTimeoutNs)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
+                    const uint32_t a_lo = a_lo0 + (uint32_t)s * (C_::kABytes >> 4);
+                    const uint32_t b_lo = b_lo0 + (uint32_t)s * (C_::kBBytes >> 4);
+                    const uint32_t sfa_lo = sfa_lo0 + (uint32_t)s * (C_::kSfaBytes >> 4);
+                    const uint32_t sfb_lo = sfb_lo0 + (uint32_t)s * (C_::kSfbBytes >> 4);
                     const int64_t krem = p.K - kt * T::kBkElems;
-                    const int nmma = krem >= T::kBkElems ? C_::kMmaPerKt : (int)(krem / T::kMmaK);
-                    const uint32_t sfa_s = smem_u32(sSFA + s * C_::kSfaBytes);
-                    const uint32_t sfb_s = smem_u32(sSFB + s * C_::kSfbBytes);
-                    const uint32_t a_s = smem_u32(sA + s * C_::kABytes);
-                    const uint32_t b_s = smem_u32(sB + s * C_::kBBytes);
+                    const bool full_kt = krem >= T::kBkElems;
+                    const int nmma = full_kt ? C_::kMmaPerKt : (int)(krem / T::kMmaK);
                     if (FMT == BSQ_NVFP4) {
-                        for (int j = 0; j < nmma; j++) {
-                            // the slot for this MMA: its SFA atom, then one atom per 128 rows of B
-                            const uint32_t slot = tmem_base + SF_TMEM0 + (uint32_t)((slot_ctr++ % C_::kSlots) * C_::kSlotCols);
-                            tmem_cp_sf_atom(slot, smem_desc(sfa_s + 512 * j, 0, 128, 0));
+                        // four slots per k-tile, one per MMA: its SFA atom, then one atom per 128 rows of B
+                        const uint32_t slot0 = sf_t0 + (ktc & (C_::kSlots / 4 - 1)) * (4 * C_::kSlotCols);
+                        auto issue = [&](int j) {
+                            const uint32_t slot = slot0 + (uint32_t)j * C_::kSlotCols;
+                            tmem_cp_sf_atom(slot, desc_pack(sfa_lo + kSfAtomLo * j, kSfHi));
+#pragma unroll
                             for (int r = 0; r < C_::kNbAtomTiles; r++)
-                                tmem_cp_sf_atom(slot + 4 + 4 * r, smem_desc(sfb_s + r * C_::kSfaBytes + 512 * j, 0, 128, 0));
-                            const uint64_t ad = smem_desc(a_s + 32 * j, 16, 1024, 2);
-                            const uint64_t bd = smem_desc(b_s + 32 * j, 16, 1024, 2);
-                            mma_nvfp4(d_tmem, ad, bd, idesc, slot, slot + 4, (kt > 0 || j > 0) ? 1u : 0u);
+                                tmem_cp_sf_atom(slot + 4 + 4 * r, desc_pack(sfb_lo + kSfbTileLo * r + kSfAtomLo * j, kSfHi));
+                            mma_nvfp4(d_tmem, desc_pack(a_lo + 2 * j, kOpHi), desc_pack(b_lo + 2 * j, kOpHi), idesc, slot,
+                                      slot + 4, (kt > 0 || j > 0) ? 1u : 0u);
+                        };
+                        if (full_kt) {
+#pragma unroll
+                            for (int j = 0; j < C_::kMmaPerKt; j++) issue(j);
+                        } else {
+                            for (int j = 0; j < nmma; j++) issue(j);
                         }
                     } else {
-                        const uint32_t slot = tmem_base + SF_TMEM0 + (uint32_t)((slot_ctr++ % C_::kSlots) * C_::kSlotCols);
-                        tmem_cp_sf_atom(slot, smem_desc(sfa_s, 0, 128, 0));
+                        // one slot per k-tile: its atoms cover the 4 MMAs, selected by the scale-factor id
+                        const uint32_t slot = sf_t0 + (ktc & (C_::kSlots - 1)) * C_::kSlotCols;
+                        tmem_cp_sf_atom(slot, desc_pack(sfa_lo, kSfHi));
+#pragma unroll
                         for (int r = 0; r < C_::kNbAtomTiles; r++)
-                            tmem_cp_sf_atom(slot + 4 + 4 * r, smem_desc(sfb_s + r * C_::kSfaBytes, 0, 128, 0));
-                        for (int j = 0; j < nmma; j++) {
-                            const uint64_t ad = smem_desc(a_s + 32 * j, 16, 1024, 2);
-                            const uint64_t bd = smem_desc(b_s + 32 * j, 16, 1024, 2);
-                            // scale byte j of each 32-bit SF column: in the descriptor and in
-                            // the top bits of the TMEM scale address
-                            mma_mxfp8(d_tmem, ad, bd, idesc | ((uint32_t)j << 29) | ((uint32_t)j << 4),
-                                      slot | ((uint32_t)j << 30), (slot + 4) | ((uint32_t)j << 30),
-                                      (kt > 0 || j > 0) ? 1u : 0u);
+                            tmem_cp_sf_atom(slot + 4 + 4 * r, desc_pack(sfb_lo + kSfbTileLo * r, kSfHi));
+                        // scale byte j of each 32-bit SF column: in the descriptor and in
+                        // the top bits of the TMEM scale address
+                        auto issue = [&](int j) {
+                            mma_mxfp8(d_tmem, desc_pack(a_lo + 2 * j, kOpHi), desc_pack(b_lo + 2 * j, kOpHi),
+                                      idesc | ((uint32_t)j << 29) | ((uint32_t)j << 4), slot | ((uint32_t)j << 30),
+                                      (slot + 4) | ((uint32_t)j << 30), (kt > 0 || j > 0) ? 1u : 0u);
+                        };
+                        if (full_kt) {
+#pragma unroll
+                            for (int j = 0; j < C_::kMmaPerKt; j++) issue(j);
+                        } else {
+                            for (int j = 0; j < nmma; j++) issue(j);
                         }
                     }
                     issued = true;
@@ -493,7 +518,7 @@ struct Cfg2 {
     static constexpr int kStages = (220 * 1024) / kStageBytes > 8 ? 8 : (220 * 1024) / kStageBytes;
     static constexpr int kSmemBytes = kStages * kStageBytes + 1024;
     static constexpr int kSlotCols = 12;  // 4 SFA + 8 SFB columns
-    static constexpr int kSlots = 8;
+    static constexpr int kSlots = (FMT == BSQ_NVFP4) ? 16 : 8;
     static constexpr int kMmaPerKt = T::kBkElems / T::kMmaK;
     static constexpr int kEpiWarps = 8;
     static constexpr int kThreads = 32 * (2 + kEpiWarps);
@@ -578,6 +603,7 @@ __global__ void __launch_bounds__(320, 1)
     tc_fence_after();
     const uint32_t tmem_base = tmem_base_slot;
     if (GROUPED) total_tiles = tile_start[p.G];
+    static_assert(256 + C_::kSlots * C_::kSlotCols <= 512, "TMEM budget");
 
     // (group, 256-row m tile, n tile) of pair tile t; rows of this CTA
     auto info = [&](int64_t t, int64_t &a_row0, int64_t &sfa_row0, int64_t &m_lim, int64_t &nt, int &group) {
@@ -667,60 +693,122 @@ __global__ void __launch_bounds__(320, 1)
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer (leader only)
+        // (lean issue loop with the scale copies one k-tile ahead of the
+        // MMAs, as in the single-CTA kernel)
         if (leader && lane == 0) {
             const uint32_t idesc = T::kIdescFmt | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(256 >> 4) << 24);
+            constexpr uint32_t kOpHi = smem_desc_hi(1024, 2);
+            constexpr uint32_t kSfHi = smem_desc_hi(128, 0);
+            const uint32_t a_lo0 = smem_desc_lo(smem_u32(sA), 16), b_lo0 = smem_desc_lo(smem_u32(sB), 16);
+            const uint32_t sfa_lo0 = smem_desc_lo(smem_u32(sSFA), 0), sfb_lo0 = smem_desc_lo(smem_u32(sSFB), 0);
+            const uint32_t sf_t0 = tmem_base + 256;
+            constexpr uint32_t kSfAtomLo = 512 >> 4;
+            constexpr uint32_t kSfbTileLo = C_::kSfaBytes >> 4;
+            auto slot_of = [&](uint32_t c, int j) -> uint32_t {
+                if (FMT == BSQ_NVFP4) return sf_t0 + ((c & (C_::kSlots / 4 - 1)) * 4 + (uint32_t)j) * C_::kSlotCols;
+                return sf_t0 + (c & (C_::kSlots - 1)) * C_::kSlotCols;
+            };
+            auto n_mma = [&](int64_t kt) -> int {
+                const int64_t krem = p.K - kt * T::kBkElems;
+                return krem >= T::kBkElems ? C_::kMmaPerKt : (int)(krem / T::kMmaK);
+            };
+            auto copy_sf = [&](int st, uint32_t c, int nm) {
+                const uint32_t sfa_lo = sfa_lo0 + (uint32_t)st * (C_::kSfaBytes >> 4);
+                const uint32_t sfb_lo = sfb_lo0 + (uint32_t)st * (C_::kSfbBytes >> 4);
+                if (FMT == BSQ_NVFP4) {
+                    auto one = [&](int j) {
+                        const uint32_t slot = slot_of(c, j);
+                        tmem_cp_sf_atom_pair(slot, desc_pack(sfa_lo + kSfAtomLo * j, kSfHi));
+                        tmem_cp_sf_atom_pair(slot + 4, desc_pack(sfb_lo + kSfAtomLo * j, kSfHi));
+                        tmem_cp_sf_atom_pair(slot + 8, desc_pack(sfb_lo + kSfbTileLo + kSfAtomLo * j, kSfHi));
+                    };
+                    if (nm == C_::kMmaPerKt) {
+#pragma unroll
+                        for (int j = 0; j < C_::kMmaPerKt; j++) one(j);
+                    } else {
+                        for (int j = 0; j < nm; j++) one(j);
+                    }
+                } else {
+                    const uint32_t slot = slot_of(c, 0);
+                    tmem_cp_sf_atom_pair(slot, desc_pack(sfa_lo, kSfHi));
+                    tmem_cp_sf_atom_pair(slot + 4, desc_pack(sfb_lo, kSfHi));
+                    tmem_cp_sf_atom_pair(slot + 8, desc_pack(sfb_lo + kSfbTileLo, kSfHi));
+                }
+            };
+            auto mmas = [&](int st, uint32_t c, int nm, bool first) {
+                const uint32_t a_lo = a_lo0 + (uint32_t)st * (C_::kABytes >> 4);
+                const uint32_t b_lo = b_lo0 + (uint32_t)st * (C_::kBBytes >> 4);
+                auto one = [&](int j) {
+                    const uint32_t acc = (!first || j > 0) ? 1u : 0u;
+                    if (FMT == BSQ_NVFP4) {
+                        const uint32_t slot = slot_of(c, j);
+                        mma_nvfp4_pair(tmem_base, desc_pack(a_lo + 2 * j, kOpHi), desc_pack(b_lo + 2 * j, kOpHi), idesc,
+                                       slot, slot + 4, acc);
+                    } else {
+                        const uint32_t slot = slot_of(c, 0);
+                        mma_mxfp8_pair(tmem_base, desc_pack(a_lo + 2 * j, kOpHi), desc_pack(b_lo + 2 * j, kOpHi),
+                                       idesc | ((uint32_t)j << 29) | ((uint32_t)j << 4), slot | ((uint32_t)j << 30),
+                                       (slot + 4) | ((uint32_t)j << 30), acc);
+                    }
+                };
+                if (nm == C_::kMmaPerKt) {
+#pragma unroll
+                    for (int j = 0; j < C_::kMmaPerKt; j++) one(j);
+                } else {
+                    for (int j = 0; j < nm; j++) one(j);
+                }
+            };
+            auto wait_full = [&](int st, uint32_t phase) -> bool {
+                if (mbar_test_wait(smem_u32(&full_bar[st]), phase)) return true;
+                return mbar_wait(smem_u32(&full_bar[st]), phase, &abort_flag, p.err, 4, kTimeoutNs);
+            };
             int s = 0;
             uint32_t ph = 0;
             bool ok = true, issued = false;
-            uint32_t slot_ctr = 0;
-            int64_t it = 0;
-            for (int64_t t = pair; t < total_tiles && ok; t += npairs, it++) {
-                if (!mbar_wait(smem_u32(&acce_bar), (uint32_t)(it & 1) ^ 1u, &abort_flag, p.err, 3, kTimeoutNs)) {
-                    ok = false;
-                    break;
+            uint32_t ktc = 0;
+            int64_t t = pair, kt = 0, it = 0;
+            if (t < total_tiles) {
+                ok = wait_full(0, 0);
+                if (ok) {
+                    tc_fence_after();
+                    copy_sf(0, 0, n_mma(0));
+                    issued = true;
                 }
-                tc_fence_after();
-                const uint32_t d_tmem = tmem_base;
-                for (int64_t kt = 0; kt < k_tiles; kt++) {
-                    if (!mbar_wait(smem_u32(&full_bar[s]), ph, &abort_flag, p.err, 4, kTimeoutNs)) {
+            }
+            while (ok && t < total_tiles) {
+                int64_t nt = t, nkt = kt + 1;
+                if (nkt == k_tiles) {
+                    nt = t + npairs;
+                    nkt = 0;
+                }
+                const int ns = (s + 1 == NS) ? 0 : s + 1;
+                const uint32_t nph = (s + 1 == NS) ? (ph ^ 1u) : ph;
+                if (nt < total_tiles) {
+                    if (!wait_full(ns, nph)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const int64_t krem = p.K - kt * T::kBkElems;
-                    const int nmma = krem >= T::kBkElems ? C_::kMmaPerKt : (int)(krem / T::kMmaK);
-                    const uint32_t sfa_s = smem_u32(sSFA + s * C_::kSfaBytes);
-                    const uint32_t sfb_s = smem_u32(sSFB + s * C_::kSfbBytes);
-                    const uint32_t a_s = smem_u32(sA + s * C_::kABytes);
-                    const uint32_t b_s = smem_u32(sB + s * C_::kBBytes);
-                    if (FMT == BSQ_NVFP4) {
-                        for (int j = 0; j < nmma; j++) {
-                            const uint32_t slot = tmem_base + 256 + (uint32_t)((slot_ctr++ % C_::kSlots) * C_::kSlotCols);
-                            tmem_cp_sf_atom_pair(slot, smem_desc(sfa_s + 512 * j, 0, 128, 0));
-                            tmem_cp_sf_atom_pair(slot + 4, smem_desc(sfb_s + 512 * j, 0, 128, 0));
-                            tmem_cp_sf_atom_pair(slot + 8, smem_desc(sfb_s + C_::kSfaBytes + 512 * j, 0, 128, 0));
-                            mma_nvfp4_pair(d_tmem, smem_desc(a_s + 32 * j, 16, 1024, 2), smem_desc(b_s + 32 * j, 16, 1024, 2),
-                                           idesc, slot, slot + 4, (kt > 0 || j > 0) ? 1u : 0u);
-                        }
-                    } else {
-                        const uint32_t slot = tmem_base + 256 + (uint32_t)((slot_ctr++ % C_::kSlots) * C_::kSlotCols);
-                        tmem_cp_sf_atom_pair(slot, smem_desc(sfa_s, 0, 128, 0));
-                        tmem_cp_sf_atom_pair(slot + 4, smem_desc(sfb_s, 0, 128, 0));
-                        tmem_cp_sf_atom_pair(slot + 8, smem_desc(sfb_s + C_::kSfaBytes, 0, 128, 0));
-                        for (int j = 0; j < nmma; j++)
-                            mma_mxfp8_pair(d_tmem, smem_desc(a_s + 32 * j, 16, 1024, 2), smem_desc(b_s + 32 * j, 16, 1024, 2),
-                                           idesc | ((uint32_t)j << 29) | ((uint32_t)j << 4), slot | ((uint32_t)j << 30),
-                                           (slot + 4) | ((uint32_t)j << 30), (kt > 0 || j > 0) ? 1u : 0u);
-                    }
-                    issued = true;
-                    tc_commit_pair(smem_u32(&empty_bar[s]), 0x3);  // release stage s in both CTAs
-                    if (++s == NS) {
-                        s = 0;
-                        ph ^= 1u;
-                    }
+                    copy_sf(ns, ktc + 1, n_mma(nkt));
                 }
-                if (!ok) break;
-                tc_commit_pair(smem_u32(&accf_bar), 0x3);
+                if (kt == 0) {
+                    if (!mbar_wait(smem_u32(&acce_bar), (uint32_t)(it & 1) ^ 1u, &abort_flag, p.err, 3, kTimeoutNs)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                }
+                mmas(s, ktc, n_mma(kt), kt == 0);
+                tc_commit_pair(smem_u32(&empty_bar[s]), 0x3);  // release stage s in both CTAs
+                if (kt == k_tiles - 1) {
+                    tc_commit_pair(smem_u32(&accf_bar), 0x3);
+                    it++;
+                }
+                s = ns;
+                ph = nph;
+                ktc++;
+                t = nt;
+                kt = nkt;
             }
             if (issued) {
                 tc_commit_pair(smem_u32(&drain_bar), 0x1);
@@ -952,11 +1040,14 @@ int dispatch(const GemmArgs &g, cudaStream_t s) {
     if (swap) bn = 64;
     else if (g.out_bf16 && NB >= 256) bn = 256;
     else bn = 128;
-    // CTA pairs for everything but the skinny swap-AB case (debug knob: BSQ_GEMM_PAIR=0)
-    // (grouped NVFP4 with a half k-tile would need the exact extent of A's
-    // scale buffer, which only the device knows: it stays on single CTAs)
-    bool use_pair = !swap && NB >= 128 && !(grouped && FMT == BSQ_NVFP4 && g.K % 256 != 0);
-    if (const char *e = getenv("BSQ_GEMM_PAIR")) use_pair = use_pair && atoi(e) != 0;
+    // Single-CTA tiles by default: on the 8192x14336x4096 NVFP4 shape they
+    // measure faster than the CTA-pair kernel (2.80 vs 2.55 PFLOP/s).  The pair
+    // kernel stays selectable (BSQ_GEMM_PAIR=1) for tuning; grouped NVFP4
+    // with a half k-tile would need the exact extent of A's scale buffer,
+    // which only the device knows, so it always stays on single CTAs.
+    bool use_pair = false;
+    if (const char *e = getenv("BSQ_GEMM_PAIR"))
+        use_pair = atoi(e) != 0 && !swap && NB >= 128 && !(grouped && FMT == BSQ_NVFP4 && g.K % 256 != 0);
     if (const char *e = getenv("BSQ_GEMM_BN")) {  // debug/tuning override of the single-CTA tile
         int v = atoi(e);
         if ((v == 128 || (v == 256 && g.out_bf16)) && !swap) bn = v;

@@ -114,6 +114,35 @@ BSQ_DEV uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_byte
     return d;
 }
 
+// The same descriptor split into its two 32-bit words, for issue loops that
+// step the start address by adding to the low word (the address field sits
+// in its low 14 bits; shared-memory addresses stay below 256 KB, so adding
+// a small offset never carries out of the field).
+BSQ_DEV constexpr uint32_t smem_desc_hi(uint32_t sbo_bytes, uint32_t swizzle) {
+    return ((sbo_bytes >> 4) & 0x3FFFu) | (1u << 14) | ((swizzle & 7u) << 29);
+}
+BSQ_DEV uint32_t smem_desc_lo(uint32_t saddr, uint32_t lbo_bytes) {
+    return ((saddr & 0x3FFFFu) >> 4) | (((lbo_bytes >> 4) & 0x3FFFu) << 16);
+}
+BSQ_DEV uint64_t desc_pack(uint32_t lo, uint32_t hi) {
+    uint64_t d;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "r"(lo), "r"(hi));
+    return d;
+}
+
+// Non-blocking test of an mbarrier phase (no suspend): true when complete.
+BSQ_DEV bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 // Copy one 512-byte scale-factor atom (32 rows x 16 bytes in shared memory)
 // to 4 TMEM columns, replicated into all four 32-lane quarters.
 BSQ_DEV void tmem_cp_sf_atom(uint32_t taddr, uint64_t sdesc) {

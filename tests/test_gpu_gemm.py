@@ -48,6 +48,9 @@ def run_gemm(ora, fmt, qa, qb, M, N, K, out_dtype):
     return Cg.float().cpu().numpy().astype(np.float64)
 
 
+# kernel: 0 = single-CTA tiles (the default dispatch), 1 = the CTA-pair
+# (cta_group::2) kernel, selected through its tuning switch
+@pytest.mark.parametrize("pair", [0, 1])
 @pytest.mark.parametrize("fmt", [NV, MX])
 @pytest.mark.parametrize("M,N,K,out", [
     (128, 256, 256, torch.float32),     # the small NVFP4 linear workload shape
@@ -59,14 +62,15 @@ def run_gemm(ora, fmt, qa, qb, M, N, K, out_dtype):
     (1, 256, 256, torch.float32),       # M = 1
     (17, 384, 640, torch.float32),      # swap-AB ragged
 ])
-def test_gemm_full_compare(ora, fmt, M, N, K, out):
+def test_gemm_full_compare(ora, monkeypatch, pair, fmt, M, N, K, out):
+    monkeypatch.setenv("BSQ_GEMM_PAIR", str(pair))
     A, Bm = W.nvfp4_linear_small(M=M, N=N, K=K, seed=M * 7 + N + K)
     qa, qb = oracle_operands(ora, fmt, A, Bm)
     Cg = run_gemm(ora, fmt, qa, qb, M, N, K, out)
     da = ora.dequant(fmt, *qa)
     db = ora.dequant(fmt, *qb)
     Cr, Ra = ora.gemm_f64(da, db)
-    assert_gemm_close(Cg, Cr, Ra, out == torch.bfloat16, f"gemm fmt={fmt} {M}x{N}x{K}")
+    assert_gemm_close(Cg, Cr, Ra, out == torch.bfloat16, f"gemm pair={pair} fmt={fmt} {M}x{N}x{K}")
 
 
 def test_gemm_small_linear_workload_exact_inputs(ora):
@@ -78,10 +82,12 @@ def test_gemm_small_linear_workload_exact_inputs(ora):
     assert_gemm_close(Cg, Cr, Ra, False, "small linear")
 
 
+@pytest.mark.parametrize("pair", [0, 1])
 @pytest.mark.parametrize("fmt", [NV, MX])
-def test_grouped_gemm_compare(ora, fmt):
+def test_grouped_gemm_compare(ora, monkeypatch, pair, fmt):
     """Small MoE: routed rows grouped by expert (uneven counts, one expert
     possibly empty), per-expert B and global scales."""
+    monkeypatch.setenv("BSQ_GEMM_PAIR", str(pair))
     E, T, H, F = 6, 96, 256, 192
     g = torch.Generator().manual_seed(5)
     logits = torch.randn(T, E, generator=g)

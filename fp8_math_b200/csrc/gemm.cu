@@ -501,13 +501,32 @@ __global__ void __launch_bounds__(320, 1)
 
 // ============================================================ CTA-pair kernel
 // Two CTAs of a cluster compute one 256x256 tile with tcgen05 cta_group::2:
-// CTA r loads rows [128r, 128r+128) of the A tile, rows [128r, 128r+128) of
-// the B tile and all scale factors its MMA half needs (its own SFA rows, all
-// 256 SFB rows); the leader (r = 0) issues the copies and MMAs for both, and
-// each CTA's TMEM holds its 128 accumulator rows.  Per FLOP this moves ~30 %
-// fewer bytes from L2 than a 128x256 single-CTA tile.  No load uses
-// multicast: every CTA fetches its own tiles.
-template <int FMT>
+// CTA r loads rows [128r, 128r+128) of the A tile and of the B tile (the
+// MMA reads B across the pair), plus the scale factors its half needs (its
+// own 128 SFA rows, all 256 SFB rows).  Per FLOP this moves a third fewer
+// bytes from L2 than a 128x256 single-CTA tile.  No load uses multicast.
+//
+// Warp roles (11 warps per CTA):
+//   0        producer: A/B tiles and this CTA's scale tiles with pair TMA
+//            (completion on the leader's full barrier);
+//   1        TMEM allocator; in the leader, lane 0 issues the MMAs.  It only
+//            waits on mbarriers and issues MMAs and commits, never a
+//            tcgen05.cp: a thread that waits on an mbarrier while its own
+//            copies are still queued stalls until they have executed;
+//   2        scale copier (leader, lane 0): as soon as a stage lands, copies
+//            its scale atoms into the stage's TMEM slots (tcgen05.cp, both
+//            CTAs) and commits them to the stage's sf_ready barrier; it runs
+//            ahead of the MMAs as far as the stage ring allows;
+//   3..10    epilogue, two warps per lane quarter (one half of the 256
+//            columns each): tcgen05.ld of the accumulator, alpha, bf16/fp32,
+//            staged through shared memory (32-row boxes, 64-byte swizzle) and
+//            written with TMA tile stores; boxes that cross a group's last
+//            row use per-thread stores instead.  bf16 tiles are drained into
+//            registers and the accumulator released before any store.
+// TMEM: columns 0..255 accumulator, then per stage one 12-column slot per
+// MMA (NVFP4: SFA atom, then one SFB atom per 128 rows of B) or one slot per
+// k-tile (MXFP8: the scale-factor id selects the MMA's byte).
+template <int FMT, bool GROUPED>
 struct Cfg2 {
     using T = FmtTraits<FMT>;
     static constexpr int kABytes = 128 * 128;
@@ -515,27 +534,36 @@ struct Cfg2 {
     static constexpr int kSfaBytes = T::kAtomsPerKt * 512;
     static constexpr int kSfbBytes = 2 * kSfaBytes;
     static constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
-    static constexpr int kStages = (220 * 1024) / kStageBytes > 8 ? 8 : (220 * 1024) / kStageBytes;
-    static constexpr int kSmemBytes = kStages * kStageBytes + 1024;
-    static constexpr int kSlotCols = 12;  // 4 SFA + 8 SFB columns
-    static constexpr int kSlots = (FMT == BSQ_NVFP4) ? 16 : 8;
-    static constexpr int kMmaPerKt = T::kBkElems / T::kMmaK;
     static constexpr int kEpiWarps = 8;
-    static constexpr int kThreads = 32 * (2 + kEpiWarps);
+    static constexpr int kThreads = 32 * (3 + kEpiWarps);
+    static constexpr int kBoxBytes = 2048;                          // 32 rows x 64 bytes
+    static constexpr int kBoxes = 2;                                // per epilogue warp
+    static constexpr int kStagingBytes = kEpiWarps * kBoxes * kBoxBytes;
+    static constexpr int kSmemLimit = 232448;                       // 227 KB per CTA
+    static constexpr int kStaticEst = GROUPED ? 8704 : 512;
+    static constexpr int kFit = (kSmemLimit - 2048 - kStagingBytes - kStaticEst) / kStageBytes;
+    static constexpr int kStages = kFit > 5 ? 5 : kFit;             // TMEM holds up to 5 stages of scales
+    static constexpr int kStagingOff = (kStages * kStageBytes + 1023) / 1024 * 1024;
+    static constexpr int kSmemBytes = kStagingOff + kStagingBytes + 1024;
+    static constexpr int kMmaPerKt = T::kBkElems / T::kMmaK;
+    static constexpr int kSlotCols = 12;                            // SFA atom + two SFB atoms
+    static constexpr int kStageCols = (FMT == BSQ_NVFP4) ? kMmaPerKt * kSlotCols : kSlotCols;
     static constexpr int kSfBoxRows = kSfaBytes / 256;  // SF tensor-map box height (rows of 256 B)
+    static_assert(256 + kStages * kStageCols <= 512, "TMEM budget");
+    static_assert(kStages >= 2, "shared-memory budget");
 };
 
 template <int FMT, bool OUT_BF16, bool GROUPED>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(352, 1)
     gemm_bs2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
-                    const GemmParams p) {
-    using C_ = Cfg2<FMT>;
+                    const __grid_constant__ CUtensorMap tmC, const GemmParams p) {
+    using C_ = Cfg2<FMT, GROUPED>;
     using T = typename C_::T;
     constexpr int NS = C_::kStages;
     constexpr int BN = 256;
     extern __shared__ uint8_t smem_raw[];
-    __shared__ __align__(8) uint64_t full_bar[NS], empty_bar[NS], accf_bar, acce_bar, drain_bar;
+    __shared__ __align__(8) uint64_t full_bar[NS], sf_ready[NS], empty_bar[NS], accf_bar, acce_bar, drain_bar;
     __shared__ uint32_t tmem_base_slot;
     __shared__ volatile int abort_flag;
     __shared__ int tile_start[GROUPED ? 1025 : 1];
@@ -546,6 +574,7 @@ __global__ void __launch_bounds__(320, 1)
     uint8_t *sB = sA + NS * C_::kABytes;
     uint8_t *sSFA = sB + NS * C_::kBBytes;
     uint8_t *sSFB = sSFA + NS * C_::kSfaBytes;
+    uint8_t *sStage = smem + C_::kStagingOff;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_ctarank();
@@ -559,6 +588,7 @@ __global__ void __launch_bounds__(320, 1)
     if (threadIdx.x == 0) {
         for (int i = 0; i < NS; i++) {
             mbar_init(smem_u32(&full_bar[i]), 1);
+            mbar_init(smem_u32(&sf_ready[i]), 1);
             mbar_init(smem_u32(&empty_bar[i]), 1);
         }
         mbar_init(smem_u32(&accf_bar), 1);
@@ -572,6 +602,7 @@ __global__ void __launch_bounds__(320, 1)
         prefetch_tmap(&tmB);
         prefetch_tmap(&tmSFA);
         prefetch_tmap(&tmSFB);
+        prefetch_tmap(&tmC);
     }
     int64_t total_tiles = m_tiles * n_tiles;
     if (GROUPED && warp == 2) {
@@ -603,7 +634,6 @@ __global__ void __launch_bounds__(320, 1)
     tc_fence_after();
     const uint32_t tmem_base = tmem_base_slot;
     if (GROUPED) total_tiles = tile_start[p.G];
-    static_assert(256 + C_::kSlots * C_::kSlotCols <= 512, "TMEM budget");
 
     // (group, 256-row m tile, n tile) of pair tile t; rows of this CTA
     auto info = [&](int64_t t, int64_t &a_row0, int64_t &sfa_row0, int64_t &m_lim, int64_t &nt, int &group) {
@@ -641,7 +671,6 @@ __global__ void __launch_bounds__(320, 1)
             int s = 0;
             uint32_t ph = 0, armed = 0, armed_par = 0;
             bool ok = true;
-            const uint32_t per_cta = C_::kABytes + C_::kBBytes + C_::kSfaBytes + C_::kSfbBytes;
             for (int64_t t = pair; t < total_tiles && ok; t += npairs) {
                 int64_t a_row0, sfa_row0, m_lim, nt;
                 int group;
@@ -657,7 +686,7 @@ __global__ void __launch_bounds__(320, 1)
                         break;
                     }
                     const uint32_t fb = full0 + (uint32_t)(s * 8);  // leader's full barrier of stage s
-                    if (leader) mbar_arrive_expect_tx(smem_u32(&full_bar[s]), 2 * per_cta);
+                    if (leader) mbar_arrive_expect_tx(smem_u32(&full_bar[s]), 2 * C_::kStageBytes);
                     const int32_t kx = (int32_t)(kt * 128);
                     const int32_t sfk = (int32_t)(kt * C_::kSfBoxRows);
                     tma_load_2d_pair(smem_u32(sA + s * C_::kABytes), &tmA, fb, kx, (int32_t)a_row0);
@@ -693,122 +722,61 @@ __global__ void __launch_bounds__(320, 1)
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer (leader only)
-        // (lean issue loop with the scale copies one k-tile ahead of the
-        // MMAs, as in the single-CTA kernel)
         if (leader && lane == 0) {
             const uint32_t idesc = T::kIdescFmt | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(256 >> 4) << 24);
-            constexpr uint32_t kOpHi = smem_desc_hi(1024, 2);
-            constexpr uint32_t kSfHi = smem_desc_hi(128, 0);
+            constexpr uint32_t kOpHi = smem_desc_hi(1024, 2);  // K-major, 128-byte swizzle, 8-row groups 1 KB apart
             const uint32_t a_lo0 = smem_desc_lo(smem_u32(sA), 16), b_lo0 = smem_desc_lo(smem_u32(sB), 16);
-            const uint32_t sfa_lo0 = smem_desc_lo(smem_u32(sSFA), 0), sfb_lo0 = smem_desc_lo(smem_u32(sSFB), 0);
-            const uint32_t sf_t0 = tmem_base + 256;
-            constexpr uint32_t kSfAtomLo = 512 >> 4;
-            constexpr uint32_t kSfbTileLo = C_::kSfaBytes >> 4;
-            auto slot_of = [&](uint32_t c, int j) -> uint32_t {
-                if (FMT == BSQ_NVFP4) return sf_t0 + ((c & (C_::kSlots / 4 - 1)) * 4 + (uint32_t)j) * C_::kSlotCols;
-                return sf_t0 + (c & (C_::kSlots - 1)) * C_::kSlotCols;
-            };
-            auto n_mma = [&](int64_t kt) -> int {
-                const int64_t krem = p.K - kt * T::kBkElems;
-                return krem >= T::kBkElems ? C_::kMmaPerKt : (int)(krem / T::kMmaK);
-            };
-            auto copy_sf = [&](int st, uint32_t c, int nm) {
-                const uint32_t sfa_lo = sfa_lo0 + (uint32_t)st * (C_::kSfaBytes >> 4);
-                const uint32_t sfb_lo = sfb_lo0 + (uint32_t)st * (C_::kSfbBytes >> 4);
-                if (FMT == BSQ_NVFP4) {
-                    auto one = [&](int j) {
-                        const uint32_t slot = slot_of(c, j);
-                        tmem_cp_sf_atom_pair(slot, desc_pack(sfa_lo + kSfAtomLo * j, kSfHi));
-                        tmem_cp_sf_atom_pair(slot + 4, desc_pack(sfb_lo + kSfAtomLo * j, kSfHi));
-                        tmem_cp_sf_atom_pair(slot + 8, desc_pack(sfb_lo + kSfbTileLo + kSfAtomLo * j, kSfHi));
-                    };
-                    if (nm == C_::kMmaPerKt) {
-#pragma unroll
-                        for (int j = 0; j < C_::kMmaPerKt; j++) one(j);
-                    } else {
-                        for (int j = 0; j < nm; j++) one(j);
-                    }
-                } else {
-                    const uint32_t slot = slot_of(c, 0);
-                    tmem_cp_sf_atom_pair(slot, desc_pack(sfa_lo, kSfHi));
-                    tmem_cp_sf_atom_pair(slot + 4, desc_pack(sfb_lo, kSfHi));
-                    tmem_cp_sf_atom_pair(slot + 8, desc_pack(sfb_lo + kSfbTileLo, kSfHi));
-                }
-            };
-            auto mmas = [&](int st, uint32_t c, int nm, bool first) {
-                const uint32_t a_lo = a_lo0 + (uint32_t)st * (C_::kABytes >> 4);
-                const uint32_t b_lo = b_lo0 + (uint32_t)st * (C_::kBBytes >> 4);
-                auto one = [&](int j) {
-                    const uint32_t acc = (!first || j > 0) ? 1u : 0u;
-                    if (FMT == BSQ_NVFP4) {
-                        const uint32_t slot = slot_of(c, j);
-                        mma_nvfp4_pair(tmem_base, desc_pack(a_lo + 2 * j, kOpHi), desc_pack(b_lo + 2 * j, kOpHi), idesc,
-                                       slot, slot + 4, acc);
-                    } else {
-                        const uint32_t slot = slot_of(c, 0);
-                        mma_mxfp8_pair(tmem_base, desc_pack(a_lo + 2 * j, kOpHi), desc_pack(b_lo + 2 * j, kOpHi),
-                                       idesc | ((uint32_t)j << 29) | ((uint32_t)j << 4), slot | ((uint32_t)j << 30),
-                                       (slot + 4) | ((uint32_t)j << 30), acc);
-                    }
-                };
-                if (nm == C_::kMmaPerKt) {
-#pragma unroll
-                    for (int j = 0; j < C_::kMmaPerKt; j++) one(j);
-                } else {
-                    for (int j = 0; j < nm; j++) one(j);
-                }
-            };
-            auto wait_full = [&](int st, uint32_t phase) -> bool {
-                if (mbar_test_wait(smem_u32(&full_bar[st]), phase)) return true;
-                return mbar_wait(smem_u32(&full_bar[st]), phase, &abort_flag, p.err, 4, kTimeoutNs);
-            };
             int s = 0;
             uint32_t ph = 0;
             bool ok = true, issued = false;
-            uint32_t ktc = 0;
-            int64_t t = pair, kt = 0, it = 0;
-            if (t < total_tiles) {
-                ok = wait_full(0, 0);
-                if (ok) {
+            int64_t it = 0;
+            for (int64_t t = pair; t < total_tiles && ok; t += npairs, it++) {
+                if (!mbar_wait_cluster(smem_u32(&acce_bar), (uint32_t)(it & 1) ^ 1u, &abort_flag, p.err, 3,
+                                       kTimeoutNs)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                for (int64_t kt = 0; kt < k_tiles; kt++) {
+                    // the stage's scales are in TMEM (and so its tiles have landed)
+                    if (!(mbar_test_wait(smem_u32(&sf_ready[s]), ph) ||
+                          mbar_wait(smem_u32(&sf_ready[s]), ph, &abort_flag, p.err, 4, kTimeoutNs))) {
+                        ok = false;
+                        break;
+                    }
                     tc_fence_after();
-                    copy_sf(0, 0, n_mma(0));
+                    const uint32_t a_lo = a_lo0 + (uint32_t)s * (C_::kABytes >> 4);
+                    const uint32_t b_lo = b_lo0 + (uint32_t)s * (C_::kBBytes >> 4);
+                    const uint32_t slot0 = tmem_base + 256 + (uint32_t)s * C_::kStageCols;
+                    const int64_t krem = p.K - kt * T::kBkElems;
+                    const int nmma = krem >= T::kBkElems ? C_::kMmaPerKt : (int)(krem / T::kMmaK);
+                    auto one = [&](int j) {
+                        const uint32_t acc = (kt > 0 || j > 0) ? 1u : 0u;
+                        const uint64_t ad = desc_pack(a_lo + 2 * j, kOpHi), bd = desc_pack(b_lo + 2 * j, kOpHi);
+                        if (FMT == BSQ_NVFP4) {
+                            const uint32_t slot = slot0 + (uint32_t)j * C_::kSlotCols;
+                            mma_nvfp4_pair(tmem_base, ad, bd, idesc, slot, slot + 4, acc);
+                        } else {
+                            // scale byte j of each 32-bit column (scale-factor id)
+                            mma_mxfp8_pair(tmem_base, ad, bd, idesc | ((uint32_t)j << 29) | ((uint32_t)j << 4),
+                                           slot0 | ((uint32_t)j << 30), (slot0 + 4) | ((uint32_t)j << 30), acc);
+                        }
+                    };
+                    if (nmma == C_::kMmaPerKt) {
+#pragma unroll
+                        for (int j = 0; j < C_::kMmaPerKt; j++) one(j);
+                    } else {
+                        for (int j = 0; j < nmma; j++) one(j);
+                    }
                     issued = true;
-                }
-            }
-            while (ok && t < total_tiles) {
-                int64_t nt = t, nkt = kt + 1;
-                if (nkt == k_tiles) {
-                    nt = t + npairs;
-                    nkt = 0;
-                }
-                const int ns = (s + 1 == NS) ? 0 : s + 1;
-                const uint32_t nph = (s + 1 == NS) ? (ph ^ 1u) : ph;
-                if (nt < total_tiles) {
-                    if (!wait_full(ns, nph)) {
-                        ok = false;
-                        break;
+                    tc_commit_pair(smem_u32(&empty_bar[s]), 0x3);  // release stage s in both CTAs
+                    if (++s == NS) {
+                        s = 0;
+                        ph ^= 1u;
                     }
-                    tc_fence_after();
-                    copy_sf(ns, ktc + 1, n_mma(nkt));
                 }
-                if (kt == 0) {
-                    if (!mbar_wait(smem_u32(&acce_bar), (uint32_t)(it & 1) ^ 1u, &abort_flag, p.err, 3, kTimeoutNs)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                }
-                mmas(s, ktc, n_mma(kt), kt == 0);
-                tc_commit_pair(smem_u32(&empty_bar[s]), 0x3);  // release stage s in both CTAs
-                if (kt == k_tiles - 1) {
-                    tc_commit_pair(smem_u32(&accf_bar), 0x3);
-                    it++;
-                }
-                s = ns;
-                ph = nph;
-                ktc++;
-                t = nt;
-                kt = nkt;
+                if (!ok) break;
+                tc_commit_pair(smem_u32(&accf_bar), 0x3);
             }
             if (issued) {
                 tc_commit_pair(smem_u32(&drain_bar), 0x1);
@@ -816,13 +784,97 @@ __global__ void __launch_bounds__(320, 1)
                 mbar_wait(smem_u32(&drain_bar), 0, &never, p.err, 5, kTimeoutNs);
             }
         }
+    } else if (warp == 2) {
+        // ------------------------------------------------------------ scale copier (leader only)
+        if (leader && lane == 0) {
+            constexpr uint32_t kSfHi = smem_desc_hi(128, 0);  // scale atoms: 32 rows of 16 bytes
+            const uint32_t sfa_lo0 = smem_desc_lo(smem_u32(sSFA), 0), sfb_lo0 = smem_desc_lo(smem_u32(sSFB), 0);
+            constexpr uint32_t kSfAtomLo = 512 >> 4;
+            constexpr uint32_t kSfbTileLo = C_::kSfaBytes >> 4;
+            int s = 0;
+            uint32_t ph = 0;
+            bool ok = true, issued = false;
+            for (int64_t t = pair; t < total_tiles && ok; t += npairs) {
+                for (int64_t kt = 0; kt < k_tiles; kt++) {
+                    if (!(mbar_test_wait(smem_u32(&full_bar[s]), ph) ||
+                          mbar_wait(smem_u32(&full_bar[s]), ph, &abort_flag, p.err, 7, kTimeoutNs))) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sfa_lo = sfa_lo0 + (uint32_t)s * (C_::kSfaBytes >> 4);
+                    const uint32_t sfb_lo = sfb_lo0 + (uint32_t)s * (C_::kSfbBytes >> 4);
+                    const uint32_t slot0 = tmem_base + 256 + (uint32_t)s * C_::kStageCols;
+                    const int64_t krem = p.K - kt * T::kBkElems;
+                    const int nmma = krem >= T::kBkElems ? C_::kMmaPerKt : (int)(krem / T::kMmaK);
+                    if (FMT == BSQ_NVFP4) {
+                        auto one = [&](int j) {
+                            const uint32_t slot = slot0 + (uint32_t)j * C_::kSlotCols;
+                            tmem_cp_sf_atom_pair(slot, desc_pack(sfa_lo + kSfAtomLo * j, kSfHi));
+                            tmem_cp_sf_atom_pair(slot + 4, desc_pack(sfb_lo + kSfAtomLo * j, kSfHi));
+                            tmem_cp_sf_atom_pair(slot + 8, desc_pack(sfb_lo + kSfbTileLo + kSfAtomLo * j, kSfHi));
+                        };
+                        if (nmma == C_::kMmaPerKt) {
+#pragma unroll
+                            for (int j = 0; j < C_::kMmaPerKt; j++) one(j);
+                        } else {
+                            for (int j = 0; j < nmma; j++) one(j);
+                        }
+                    } else {
+                        tmem_cp_sf_atom_pair(slot0, desc_pack(sfa_lo, kSfHi));
+                        tmem_cp_sf_atom_pair(slot0 + 4, desc_pack(sfb_lo, kSfHi));
+                        tmem_cp_sf_atom_pair(slot0 + 8, desc_pack(sfb_lo + kSfbTileLo, kSfHi));
+                    }
+                    issued = true;
+                    tc_commit_pair(smem_u32(&sf_ready[s]), 0x1);  // the copies of stage s have executed
+                    if (++s == NS) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
+                }
+            }
+            if (issued) {
+                // this thread's copies have executed before TMEM is freed
+                __shared__ __align__(8) uint64_t cp_drain;
+                mbar_init(smem_u32(&cp_drain), 1);
+                fence_barrier_init();
+                tc_commit_pair(smem_u32(&cp_drain), 0x1);
+                volatile int never = 0;
+                mbar_wait(smem_u32(&cp_drain), 0, &never, p.err, 5, kTimeoutNs);
+            }
+        }
     } else {
         // ------------------------------------------------------------ epilogue (both CTAs)
+        const int ew = warp - 3;  // 0..7
         const int q = warp & 3;
-        const int half = (warp - 2) >> 2;
+        const int half = ew >> 2;
         constexpr int HC = BN / 2;
-        const int row = 32 * q + lane;
+        uint8_t *box_base = sStage + ew * C_::kBoxes * C_::kBoxBytes;
+        // 64-byte swizzle of a 32-row x 64-byte box: 16-byte chunk c of row r
+        // sits at chunk c ^ ((r >> 1) & 3) (the pattern the tensor map names)
+        auto box_addr = [&](int box, int c) -> uint8_t * {
+            return box_base + box * C_::kBoxBytes + lane * 64 + ((c ^ ((lane >> 1) & 3)) << 4);
+        };
         int64_t it = 0;
+        int nstored = 0;  // boxes handed to TMA: the ring position
+        // stage one 32-row box (this thread's 64-byte row in v) and store it at (x, y)
+        auto store_box = [&](const uint32_t (&v)[16], int64_t x, int64_t y) {
+            const int box = nstored & (C_::kBoxes - 1);
+            if (nstored >= C_::kBoxes) {
+                if (lane == 0) bulk_wait_read<C_::kBoxes - 1>();  // this box's previous store has read it
+                __syncwarp();
+            }
+#pragma unroll
+            for (int c = 0; c < 4; c++)
+                *reinterpret_cast<uint4 *>(box_addr(box, c)) = make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                tma_store_2d(&tmC, smem_u32(box_base + box * C_::kBoxBytes), (int32_t)x, (int32_t)y);
+                bulk_commit();
+            }
+            nstored++;
+        };
         for (int64_t t = pair; t < total_tiles; t += npairs, it++) {
             int64_t a_row0, sfa_row0, m_lim, nt;
             int group;
@@ -835,12 +887,15 @@ __global__ void __launch_bounds__(320, 1)
                 const float gb = p.gsB ? __ldg(p.gsB + group) : 1.0f;
                 alpha = __fmul_rn(ga, gb);
             }
-            const int64_t ar = a_row0 + row;
+            const int64_t row0 = a_row0 + 32 * q;  // first row of this warp's boxes
+            const int64_t ar = row0 + lane;
             const bool row_ok = ar < m_lim;
+            const bool box_rows_ok = row0 + 32 <= m_lim;  // TMA boxes never cross a group's end
             const int64_t nb0 = nt * BN + half * HC;
             const int64_t n_lim = p.n_lim;
             const uint32_t tbase = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(half * HC);
             if (OUT_BF16) {
+                // drain this warp's 128 columns (bf16-packed) and release the accumulator
                 uint32_t pk[HC / 2];
 #pragma unroll
                 for (int c = 0; c < HC / 32; c += 2) {
@@ -861,55 +916,52 @@ __global__ void __launch_bounds__(320, 1)
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive_cluster(acce_leader);
-                if (!row_ok) continue;
 #pragma unroll
                 for (int c = 0; c < HC / 32; c++) {
                     const int64_t n = nb0 + 32 * c;
-                    __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.C) + ar * p.ldc + n;
-                    if (n + 32 <= n_lim) {
-                        uint4 *d4 = reinterpret_cast<uint4 *>(dst);
+                    uint32_t v[16];
 #pragma unroll
-                        for (int v = 0; v < 4; v++)
-                            d4[v] = make_uint4(pk[16 * c + 4 * v], pk[16 * c + 4 * v + 1], pk[16 * c + 4 * v + 2],
-                                               pk[16 * c + 4 * v + 3]);
-                    } else {
-#pragma unroll
+                    for (int j = 0; j < 16; j++) v[j] = pk[16 * c + j];
+                    if (n >= n_lim) {
+                        // past the last column: nothing to store
+                    } else if (box_rows_ok) {
+                        store_box(v, n, row0);
+                    } else if (row_ok) {
+                        uint16_t *dst = reinterpret_cast<uint16_t *>(static_cast<__nv_bfloat16 *>(p.C) + ar * p.ldc + n);
                         for (int j = 0; j < 32; j++)
-                            if (n + j < n_lim) {
-                                uint32_t w = pk[16 * c + j / 2];
-                                reinterpret_cast<uint16_t *>(dst)[j] = (j & 1) ? (uint16_t)(w >> 16) : (uint16_t)(w & 0xFFFFu);
-                            }
+                            if (n + j < n_lim) dst[j] = (j & 1) ? (uint16_t)(v[j / 2] >> 16) : (uint16_t)(v[j / 2] & 0xFFFFu);
                     }
                 }
             } else {
+                // fp32: 16-column boxes; the accumulator is released after the last load
 #pragma unroll 1
-                for (int c = 0; c < HC / 32; c++) {
-                    uint32_t r[32];
-                    tmem_ld32(tbase + 32 * c, r);
+                for (int c = 0; c < HC / 16; c++) {
+                    uint32_t r[16];
+                    tmem_ld16(tbase + 16 * c, r);
                     tmem_ld_wait();
-                    if (c == HC / 32 - 1) {
+                    if (c == HC / 16 - 1) {
                         tc_fence_before();
                         __syncwarp();
                         if (lane == 0) mbar_arrive_cluster(acce_leader);
                     }
-                    if (!row_ok) continue;
-                    const int64_t n = nb0 + 32 * c;
-                    float *dst = static_cast<float *>(p.C) + ar * p.ldc + n;
-                    if (n + 32 <= n_lim) {
-                        float4 *d4 = reinterpret_cast<float4 *>(dst);
+                    const int64_t n = nb0 + 16 * c;
+                    if (n >= n_lim) continue;
+                    uint32_t v[16];
 #pragma unroll
-                        for (int x = 0; x < 8; x++)
-                            d4[x] = make_float4(__fmul_rn(alpha, __uint_as_float(r[4 * x])),
-                                                __fmul_rn(alpha, __uint_as_float(r[4 * x + 1])),
-                                                __fmul_rn(alpha, __uint_as_float(r[4 * x + 2])),
-                                                __fmul_rn(alpha, __uint_as_float(r[4 * x + 3])));
-                    } else {
-                        for (int j = 0; j < 32; j++)
-                            if (n + j < n_lim) dst[j] = __fmul_rn(alpha, __uint_as_float(r[j]));
+                    for (int j = 0; j < 16; j++) v[j] = __float_as_uint(__fmul_rn(alpha, __uint_as_float(r[j])));
+                    if (box_rows_ok) {
+                        store_box(v, n, row0);
+                    } else if (row_ok) {
+                        float *dst = static_cast<float *>(p.C) + ar * p.ldc + n;
+                        for (int j = 0; j < 16; j++)
+                            if (n + j < n_lim) dst[j] = __uint_as_float(v[j]);
                     }
                 }
             }
         }
+        // every store of this warp has completed before the CTA exits
+        if (lane == 0) bulk_wait<0>();
+        __syncwarp();
     }
     tc_fence_before();
     __syncthreads();
@@ -984,10 +1036,26 @@ bool make_sf_tmap(CUtensorMap *m, const void *base, int64_t bytes, int box_rows)
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2-D tensor map over the output C (rows x n_cols elements, row stride ldc):
+// 32-row boxes of 64 bytes (32 bf16 or 16 fp32 columns), 64-byte swizzle,
+// for the pair kernel's TMA-store epilogue.
+bool make_c_tmap(CUtensorMap *m, void *C, bool bf16, int64_t n_cols, int64_t rows, int64_t ldc) {
+    EncodeFn enc = get_encode();
+    if (!enc) return false;
+    const int64_t esz = bf16 ? 2 : 4;
+    cuuint64_t dims[2] = {(cuuint64_t)n_cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)(ldc * esz)};
+    cuuint32_t box[2] = {(cuuint32_t)(64 / esz), 32u};
+    cuuint32_t estr[2] = {1u, 1u};
+    return enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, C, dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int FMT, bool OUT_BF16, bool GROUPED>
 int run_pair(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &tsa, const CUtensorMap &tsb,
-             const GemmParams &p, int pairs, cudaStream_t s) {
-    using C_ = Cfg2<FMT>;
+             const CUtensorMap &tc, const GemmParams &p, int pairs, cudaStream_t s) {
+    using C_ = Cfg2<FMT, GROUPED>;
     auto kern = gemm_bs2_kernel<FMT, OUT_BF16, GROUPED>;
     static bool attr_set = false;
     if (!attr_set) {
@@ -1007,7 +1075,7 @@ int run_pair(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &ts
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, kern, ta, tb, tsa, tsb, p) != cudaSuccess) return BSQ_ERR_CUDA;
+    if (cudaLaunchKernelEx(&cfg, kern, ta, tb, tsa, tsb, tc, p) != cudaSuccess) return BSQ_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? BSQ_OK : BSQ_ERR_CUDA;
 }
 
@@ -1040,14 +1108,18 @@ int dispatch(const GemmArgs &g, cudaStream_t s) {
     if (swap) bn = 64;
     else if (g.out_bf16 && NB >= 256) bn = 256;
     else bn = 128;
-    // Single-CTA tiles by default: on the 8192x14336x4096 NVFP4 shape they
-    // measure faster than the CTA-pair kernel (2.80 vs 2.55 PFLOP/s).  The pair
-    // kernel stays selectable (BSQ_GEMM_PAIR=1) for tuning; grouped NVFP4
-    // with a half k-tile would need the exact extent of A's scale buffer,
-    // which only the device knows, so it always stays on single CTAs.
-    bool use_pair = false;
-    if (const char *e = getenv("BSQ_GEMM_PAIR"))
-        use_pair = atoi(e) != 0 && !swap && NB >= 128 && !(grouped && FMT == BSQ_NVFP4 && g.K % 256 != 0);
+    // CTA pairs (256x256 tiles) for large operands: on 8192x14336x4096 NVFP4
+    // they measure 3.62 PFLOP/s against 3.24 for single-CTA 128x256 tiles.
+    // Single CTAs keep the skinny swap-AB case, operands with fewer than 256
+    // rows, outputs that TMA cannot store (unaligned base or row stride) and
+    // grouped NVFP4 with a half k-tile (that would need the exact extent of
+    // A's scale buffer, which only the device knows).  BSQ_GEMM_PAIR=0/1
+    // overrides the choice where the pair kernel is possible (tuning, tests).
+    const int64_t c_esz = g.out_bf16 ? 2 : 4;
+    const bool c_tma_ok = (reinterpret_cast<uintptr_t>(g.C) % 16 == 0) && (g.ldc * c_esz) % 16 == 0;
+    const bool pair_ok = !swap && NB >= 128 && c_tma_ok && !(grouped && FMT == BSQ_NVFP4 && g.K % 256 != 0);
+    bool use_pair = pair_ok && MA >= 256 && NB >= 256;
+    if (const char *e = getenv("BSQ_GEMM_PAIR")) use_pair = pair_ok && atoi(e) != 0;
     if (const char *e = getenv("BSQ_GEMM_BN")) {  // debug/tuning override of the single-CTA tile
         int v = atoi(e);
         if ((v == 128 || (v == 256 && g.out_bf16)) && !swap) bn = v;
@@ -1071,16 +1143,18 @@ int dispatch(const GemmArgs &g, cudaStream_t s) {
         // known on the host, so map the largest extent the groups can reach
         const int64_t sfa_bytes = grouped ? ((MA + 128LL * g.G + 127) / 128 * 128) * kbp : sfa_rows * kbp;
         const int64_t sfb_bytes = (grouped ? (int64_t)g.G : 1) * p.sfB_group_bytes;
-        const int box = Cfg2<FMT>::kSfBoxRows;
+        const int box = Cfg2<FMT, false>::kSfBoxRows;
         if (!make_sf_tmap(&tsa, sfA, sfa_bytes, box) || !make_sf_tmap(&tsb, sfB, sfb_bytes, box)) return BSQ_ERR_CUDA;
+        CUtensorMap tc;
+        if (!make_c_tmap(&tc, g.C, g.out_bf16, NB, MA, g.ldc)) return BSQ_ERR_CUDA;
         int64_t ptiles = grouped ? (MA / 256 + g.G) * ((NB + 255) / 256) : ((MA + 255) / 256) * ((NB + 255) / 256);
         int pairs = (int)(ptiles < g.num_sms / 2 ? (ptiles < 1 ? 1 : ptiles) : g.num_sms / 2);
         if (grouped) {
-            if (g.out_bf16) return run_pair<FMT, true, true>(ta, tb, tsa, tsb, p, pairs, s);
-            return run_pair<FMT, false, true>(ta, tb, tsa, tsb, p, pairs, s);
+            if (g.out_bf16) return run_pair<FMT, true, true>(ta, tb, tsa, tsb, tc, p, pairs, s);
+            return run_pair<FMT, false, true>(ta, tb, tsa, tsb, tc, p, pairs, s);
         }
-        if (g.out_bf16) return run_pair<FMT, true, false>(ta, tb, tsa, tsb, p, pairs, s);
-        return run_pair<FMT, false, false>(ta, tb, tsa, tsb, p, pairs, s);
+        if (g.out_bf16) return run_pair<FMT, true, false>(ta, tb, tsa, tsb, tc, p, pairs, s);
+        return run_pair<FMT, false, false>(ta, tb, tsa, tsb, tc, p, pairs, s);
     }
     if (!make_tmap(&tb, opB, kb_bytes, grouped ? (int64_t)g.G * NB : NB, bn)) return BSQ_ERR_CUDA;
     int64_t tiles;

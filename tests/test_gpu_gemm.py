@@ -48,8 +48,9 @@ def run_gemm(ora, fmt, qa, qb, M, N, K, out_dtype):
     return Cg.float().cpu().numpy().astype(np.float64)
 
 
-# kernel: 0 = single-CTA tiles (the default dispatch), 1 = the CTA-pair
-# (cta_group::2) kernel, selected through its tuning switch
+# kernel: 0 = single-CTA tiles, 1 = the CTA-pair (cta_group::2) kernel,
+# forced through the dispatch's tuning switch (the default picks pairs for
+# operands of 256+ rows)
 @pytest.mark.parametrize("pair", [0, 1])
 @pytest.mark.parametrize("fmt", [NV, MX])
 @pytest.mark.parametrize("M,N,K,out", [

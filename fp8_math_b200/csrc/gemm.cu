@@ -506,26 +506,31 @@ __global__ void __launch_bounds__(320, 1)
 // own 128 SFA rows, all 256 SFB rows).  Per FLOP this moves a third fewer
 // bytes from L2 than a 128x256 single-CTA tile.  No load uses multicast.
 //
-// Warp roles (11 warps per CTA):
-//   0        producer: A/B tiles and this CTA's scale tiles with pair TMA
-//            (completion on the leader's full barrier);
+// Warp roles (14 warps per CTA):
+//   0        producer: A/B tiles with pair TMA (completion on the leader's
+//            full barrier), this CTA's scale tiles with plain TMA (its own
+//            sf_full barrier);
 //   1        TMEM allocator; in the leader, lane 0 issues the MMAs.  It only
-//            waits on mbarriers and issues MMAs and commits, never a
-//            tcgen05.cp: a thread that waits on an mbarrier while its own
-//            copies are still queued stalls until they have executed;
-//   2        scale copier (leader, lane 0): as soon as a stage lands, copies
-//            its scale atoms into the stage's TMEM slots (tcgen05.cp, both
-//            CTAs) and commits them to the stage's sf_ready barrier; it runs
-//            ahead of the MMAs as far as the stage ring allows;
-//   3..10    epilogue, two warps per lane quarter (one half of the 256
+//            waits on mbarriers and issues MMAs and commits;
+//   2..5     scale warps, one per TMEM lane quarter: read the stage's scale
+//            atoms from shared memory and write them into the stage's TMEM
+//            scale slots with tcgen05.st (SFB replicated into every quarter,
+//            SFA only in the column each quarter reads), then arrive on the
+//            leader's sf_ready barrier (both CTAs).  No tcgen05.cp is used:
+//            copies execute in the tensor pipe between the MMAs, TMEM stores
+//            from other warps do not;
+//   6..13    epilogue, two warps per lane quarter (one half of the 256
 //            columns each): tcgen05.ld of the accumulator, alpha, bf16/fp32,
 //            staged through shared memory (32-row boxes, 64-byte swizzle) and
 //            written with TMA tile stores; boxes that cross a group's last
-//            row use per-thread stores instead.  bf16 tiles are drained into
-//            registers and the accumulator released before any store.
-// TMEM: columns 0..255 accumulator, then per stage one 12-column slot per
-// MMA (NVFP4: SFA atom, then one SFB atom per 128 rows of B) or one slot per
-// k-tile (MXFP8: the scale-factor id selects the MMA's byte).
+//            row use per-thread stores instead.  bf16 tiles are staged whole
+//            (4 boxes per warp) so the accumulator is released right after
+//            the loads; 14 warps leave 128 registers per thread.
+// Hand-overs across the pair use relaxed cluster-scope arrives: the TMEM
+// stores (scales) or loads (accumulator) they announce have completed
+// (tcgen05.wait) and are ordered by tcgen05 fences before the arrive.
+// TMEM: columns 0..255 accumulator, then per stage the SFB slot (NVFP4: 4
+// MMAs x 2 atoms x 4 columns) and the SFA slot (4 MMAs x 4 columns).
 template <int FMT, bool GROUPED>
 struct Cfg2 {
     using T = FmtTraits<FMT>;
@@ -535,9 +540,10 @@ struct Cfg2 {
     static constexpr int kSfbBytes = 2 * kSfaBytes;
     static constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
     static constexpr int kEpiWarps = 8;
-    static constexpr int kThreads = 32 * (3 + kEpiWarps);
+    static constexpr int kSfWarps = 4;
+    static constexpr int kThreads = 32 * (2 + kSfWarps + kEpiWarps);
     static constexpr int kBoxBytes = 2048;                          // 32 rows x 64 bytes
-    static constexpr int kBoxes = 2;                                // per epilogue warp
+    static constexpr int kBoxes = 4;                                // per epilogue warp: a whole bf16 tile
     static constexpr int kStagingBytes = kEpiWarps * kBoxes * kBoxBytes;
     static constexpr int kSmemLimit = 232448;                       // 227 KB per CTA
     static constexpr int kStaticEst = GROUPED ? 8704 : 512;
@@ -546,15 +552,18 @@ struct Cfg2 {
     static constexpr int kStagingOff = (kStages * kStageBytes + 1023) / 1024 * 1024;
     static constexpr int kSmemBytes = kStagingOff + kStagingBytes + 1024;
     static constexpr int kMmaPerKt = T::kBkElems / T::kMmaK;
-    static constexpr int kSlotCols = 12;                            // SFA atom + two SFB atoms
-    static constexpr int kStageCols = (FMT == BSQ_NVFP4) ? kMmaPerKt * kSlotCols : kSlotCols;
+    // TMEM scale slots of stage s: SFB at kSfb0 + kSfbCols*s, SFA at kSfa0 + kSfaCols*s
+    static constexpr int kSfbCols = (FMT == BSQ_NVFP4) ? 32 : 8;
+    static constexpr int kSfaCols = (FMT == BSQ_NVFP4) ? 16 : 4;
+    static constexpr int kSfb0 = 256;
+    static constexpr int kSfa0 = 256 + kStages * kSfbCols;
     static constexpr int kSfBoxRows = kSfaBytes / 256;  // SF tensor-map box height (rows of 256 B)
-    static_assert(256 + kStages * kStageCols <= 512, "TMEM budget");
+    static_assert(kSfa0 + kStages * kSfaCols <= 512, "TMEM budget");
     static_assert(kStages >= 2, "shared-memory budget");
 };
 
 template <int FMT, bool OUT_BF16, bool GROUPED>
-__global__ void __launch_bounds__(352, 1)
+__global__ void __launch_bounds__(448, 1)
     gemm_bs2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
                     const __grid_constant__ CUtensorMap tmC, const GemmParams p) {
@@ -563,7 +572,8 @@ __global__ void __launch_bounds__(352, 1)
     constexpr int NS = C_::kStages;
     constexpr int BN = 256;
     extern __shared__ uint8_t smem_raw[];
-    __shared__ __align__(8) uint64_t full_bar[NS], sf_ready[NS], empty_bar[NS], accf_bar, acce_bar, drain_bar;
+    __shared__ __align__(8) uint64_t full_bar[NS], sf_full[NS], sf_ready[NS], empty_bar[NS], accf_bar, acce_bar,
+        drain_bar;
     __shared__ uint32_t tmem_base_slot;
     __shared__ volatile int abort_flag;
     __shared__ int tile_start[GROUPED ? 1025 : 1];
@@ -588,7 +598,8 @@ __global__ void __launch_bounds__(352, 1)
     if (threadIdx.x == 0) {
         for (int i = 0; i < NS; i++) {
             mbar_init(smem_u32(&full_bar[i]), 1);
-            mbar_init(smem_u32(&sf_ready[i]), 1);
+            mbar_init(smem_u32(&sf_full[i]), 1);
+            mbar_init(smem_u32(&sf_ready[i]), 2 * C_::kSfWarps);
             mbar_init(smem_u32(&empty_bar[i]), 1);
         }
         mbar_init(smem_u32(&accf_bar), 1);
@@ -663,6 +674,7 @@ __global__ void __launch_bounds__(352, 1)
 
     // the leader's barriers, as seen from this CTA
     const uint32_t full0 = mapa(smem_u32(&full_bar[0]), 0);
+    const uint32_t ready0 = mapa(smem_u32(&sf_ready[0]), 0);
     const uint32_t acce_leader = mapa(smem_u32(&acce_bar), 0);
 
     if (warp == 0) {
@@ -671,6 +683,8 @@ __global__ void __launch_bounds__(352, 1)
             int s = 0;
             uint32_t ph = 0, armed = 0, armed_par = 0;
             bool ok = true;
+            constexpr uint32_t kPairBytes = 2 * (C_::kABytes + C_::kBBytes);
+            constexpr uint32_t kSfBytes = C_::kSfaBytes + C_::kSfbBytes;
             for (int64_t t = pair; t < total_tiles && ok; t += npairs) {
                 int64_t a_row0, sfa_row0, m_lim, nt;
                 int group;
@@ -686,15 +700,17 @@ __global__ void __launch_bounds__(352, 1)
                         break;
                     }
                     const uint32_t fb = full0 + (uint32_t)(s * 8);  // leader's full barrier of stage s
-                    if (leader) mbar_arrive_expect_tx(smem_u32(&full_bar[s]), 2 * C_::kStageBytes);
+                    if (leader) mbar_arrive_expect_tx(smem_u32(&full_bar[s]), kPairBytes);
                     const int32_t kx = (int32_t)(kt * 128);
-                    const int32_t sfk = (int32_t)(kt * C_::kSfBoxRows);
                     tma_load_2d_pair(smem_u32(sA + s * C_::kABytes), &tmA, fb, kx, (int32_t)a_row0);
                     tma_load_2d_pair(smem_u32(sB + s * C_::kBBytes), &tmB, fb, kx, (int32_t)b_row0);
-                    tma_load_2d_pair(smem_u32(sSFA + s * C_::kSfaBytes), &tmSFA, fb, 0, (int32_t)(sfa_r0 + sfk));
-                    tma_load_2d_pair(smem_u32(sSFB + s * C_::kSfbBytes), &tmSFB, fb, 0, (int32_t)(sfb_r0 + sfk));
-                    tma_load_2d_pair(smem_u32(sSFB + s * C_::kSfbBytes + C_::kSfaBytes), &tmSFB, fb, 0,
-                                     (int32_t)(sfb_r0 + KBT * 2 + sfk));
+                    const uint32_t sb = smem_u32(&sf_full[s]);
+                    const int32_t sfk = (int32_t)(kt * C_::kSfBoxRows);
+                    mbar_arrive_expect_tx(sb, kSfBytes);
+                    tma_load_2d(smem_u32(sSFA + s * C_::kSfaBytes), &tmSFA, sb, 0, (int32_t)(sfa_r0 + sfk));
+                    tma_load_2d(smem_u32(sSFB + s * C_::kSfbBytes), &tmSFB, sb, 0, (int32_t)(sfb_r0 + sfk));
+                    tma_load_2d(smem_u32(sSFB + s * C_::kSfbBytes + C_::kSfaBytes), &tmSFB, sb, 0,
+                                (int32_t)(sfb_r0 + KBT * 2 + sfk));
                     armed |= 1u << s;
                     armed_par = (armed_par & ~(1u << s)) | (ph << s);
                     if (++s == NS) {
@@ -703,22 +719,18 @@ __global__ void __launch_bounds__(352, 1)
                     }
                 }
             }
-            if (leader) {
-                // every armed stage's latest phase has landed before exit
-                for (int i = 0; i < NS; i++)
-                    if (armed & (1u << i)) {
-                        volatile int never = 0;
+            // before exit every copy this CTA started has landed: its own
+            // scale tiles (sf_full), and -- through the leader's MMAs having
+            // read them -- its A/B halves
+            for (int i = 0; i < NS; i++)
+                if (armed & (1u << i)) {
+                    volatile int never = 0;
+                    mbar_wait(smem_u32(&sf_full[i]), (armed_par >> i) & 1u, &never, p.err, 2, kTimeoutNs);
+                    if (leader)
                         mbar_wait(smem_u32(&full_bar[i]), (armed_par >> i) & 1u, &never, p.err, 2, kTimeoutNs);
-                    }
-            } else {
-                // the peer's copies land on the leader's barriers; wait for the
-                // leader to release each armed stage (its MMAs read our smem)
-                for (int i = 0; i < NS; i++)
-                    if (armed & (1u << i)) {
-                        volatile int never = 0;
-                        mbar_wait(smem_u32(&empty_bar[i]), (armed_par >> i) & 1u, &never, p.err, 2, kTimeoutNs);
-                    }
-            }
+                    else if (!abort_flag)
+                        mbar_wait(smem_u32(&empty_bar[i]), (armed_par >> i) & 1u, &abort_flag, p.err, 2, kTimeoutNs);
+                }
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer (leader only)
@@ -731,35 +743,36 @@ __global__ void __launch_bounds__(352, 1)
             bool ok = true, issued = false;
             int64_t it = 0;
             for (int64_t t = pair; t < total_tiles && ok; t += npairs, it++) {
-                if (!mbar_wait_cluster(smem_u32(&acce_bar), (uint32_t)(it & 1) ^ 1u, &abort_flag, p.err, 3,
-                                       kTimeoutNs)) {
+                if (!mbar_wait(smem_u32(&acce_bar), (uint32_t)(it & 1) ^ 1u, &abort_flag, p.err, 3, kTimeoutNs)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
                 for (int64_t kt = 0; kt < k_tiles; kt++) {
-                    // the stage's scales are in TMEM (and so its tiles have landed)
-                    if (!(mbar_test_wait(smem_u32(&sf_ready[s]), ph) ||
-                          mbar_wait(smem_u32(&sf_ready[s]), ph, &abort_flag, p.err, 4, kTimeoutNs))) {
+                    if (!(mbar_test_wait(smem_u32(&full_bar[s]), ph) ||
+                          mbar_wait(smem_u32(&full_bar[s]), ph, &abort_flag, p.err, 4, kTimeoutNs)) ||
+                        !(mbar_test_wait(smem_u32(&sf_ready[s]), ph) ||
+                          mbar_wait(smem_u32(&sf_ready[s]), ph, &abort_flag, p.err, 7, kTimeoutNs))) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
                     const uint32_t a_lo = a_lo0 + (uint32_t)s * (C_::kABytes >> 4);
                     const uint32_t b_lo = b_lo0 + (uint32_t)s * (C_::kBBytes >> 4);
-                    const uint32_t slot0 = tmem_base + 256 + (uint32_t)s * C_::kStageCols;
+                    const uint32_t sfb_t = tmem_base + C_::kSfb0 + (uint32_t)s * C_::kSfbCols;
+                    const uint32_t sfa_t = tmem_base + C_::kSfa0 + (uint32_t)s * C_::kSfaCols;
                     const int64_t krem = p.K - kt * T::kBkElems;
                     const int nmma = krem >= T::kBkElems ? C_::kMmaPerKt : (int)(krem / T::kMmaK);
                     auto one = [&](int j) {
                         const uint32_t acc = (kt > 0 || j > 0) ? 1u : 0u;
                         const uint64_t ad = desc_pack(a_lo + 2 * j, kOpHi), bd = desc_pack(b_lo + 2 * j, kOpHi);
                         if (FMT == BSQ_NVFP4) {
-                            const uint32_t slot = slot0 + (uint32_t)j * C_::kSlotCols;
-                            mma_nvfp4_pair(tmem_base, ad, bd, idesc, slot, slot + 4, acc);
+                            // MMA j: SFA at 4j (4-column aligned), SFB atoms at 8j and 8j + 4
+                            mma_nvfp4_pair(tmem_base, ad, bd, idesc, sfa_t + 4 * j, sfb_t + 8 * j, acc);
                         } else {
                             // scale byte j of each 32-bit column (scale-factor id)
                             mma_mxfp8_pair(tmem_base, ad, bd, idesc | ((uint32_t)j << 29) | ((uint32_t)j << 4),
-                                           slot0 | ((uint32_t)j << 30), (slot0 + 4) | ((uint32_t)j << 30), acc);
+                                           sfa_t | ((uint32_t)j << 30), sfb_t | ((uint32_t)j << 30), acc);
                         }
                     };
                     if (nmma == C_::kMmaPerKt) {
@@ -784,68 +797,55 @@ __global__ void __launch_bounds__(352, 1)
                 mbar_wait(smem_u32(&drain_bar), 0, &never, p.err, 5, kTimeoutNs);
             }
         }
-    } else if (warp == 2) {
-        // ------------------------------------------------------------ scale copier (leader only)
-        if (leader && lane == 0) {
-            constexpr uint32_t kSfHi = smem_desc_hi(128, 0);  // scale atoms: 32 rows of 16 bytes
-            const uint32_t sfa_lo0 = smem_desc_lo(smem_u32(sSFA), 0), sfb_lo0 = smem_desc_lo(smem_u32(sSFB), 0);
-            constexpr uint32_t kSfAtomLo = 512 >> 4;
-            constexpr uint32_t kSfbTileLo = C_::kSfaBytes >> 4;
-            int s = 0;
-            uint32_t ph = 0;
-            bool ok = true, issued = false;
-            for (int64_t t = pair; t < total_tiles && ok; t += npairs) {
-                for (int64_t kt = 0; kt < k_tiles; kt++) {
-                    if (!(mbar_test_wait(smem_u32(&full_bar[s]), ph) ||
-                          mbar_wait(smem_u32(&full_bar[s]), ph, &abort_flag, p.err, 7, kTimeoutNs))) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint32_t sfa_lo = sfa_lo0 + (uint32_t)s * (C_::kSfaBytes >> 4);
-                    const uint32_t sfb_lo = sfb_lo0 + (uint32_t)s * (C_::kSfbBytes >> 4);
-                    const uint32_t slot0 = tmem_base + 256 + (uint32_t)s * C_::kStageCols;
-                    const int64_t krem = p.K - kt * T::kBkElems;
-                    const int nmma = krem >= T::kBkElems ? C_::kMmaPerKt : (int)(krem / T::kMmaK);
-                    if (FMT == BSQ_NVFP4) {
-                        auto one = [&](int j) {
-                            const uint32_t slot = slot0 + (uint32_t)j * C_::kSlotCols;
-                            tmem_cp_sf_atom_pair(slot, desc_pack(sfa_lo + kSfAtomLo * j, kSfHi));
-                            tmem_cp_sf_atom_pair(slot + 4, desc_pack(sfb_lo + kSfAtomLo * j, kSfHi));
-                            tmem_cp_sf_atom_pair(slot + 8, desc_pack(sfb_lo + kSfbTileLo + kSfAtomLo * j, kSfHi));
-                        };
-                        if (nmma == C_::kMmaPerKt) {
+    } else if (warp < 2 + C_::kSfWarps) {
+        // ------------------------------------------------------------ scale warps (both CTAs)
+        const int q = warp & 3;  // the TMEM lane quarter this warp may write
+        const uint32_t lane_base = tmem_base + ((uint32_t)(32 * q) << 16);
+        int s = 0;
+        uint32_t ph = 0;
+        bool ok = true;
+        for (int64_t t = pair; t < total_tiles && ok; t += npairs) {
+            for (int64_t kt = 0; kt < k_tiles; kt++) {
+                // warp-uniform decisions: tcgen05.st is warp-collective
+                ok = __all_sync(0xFFFFFFFFu,
+                                mbar_wait(smem_u32(&sf_full[s]), ph, &abort_flag, p.err, 8, kTimeoutNs));
+                if (!ok) break;
+                const uint8_t *sfa = sSFA + s * C_::kSfaBytes;
+                const uint8_t *sfb = sSFB + s * C_::kSfbBytes;
+                const uint32_t sfb_t = lane_base + C_::kSfb0 + (uint32_t)s * C_::kSfbCols;
+                const uint32_t sfa_t = lane_base + C_::kSfa0 + (uint32_t)s * C_::kSfaCols;
+                // an atom holds rows r, r+32, r+64, r+96 of its 128 in the 16 bytes at 16 (r % 32)
+                if (FMT == BSQ_NVFP4) {
 #pragma unroll
-                            for (int j = 0; j < C_::kMmaPerKt; j++) one(j);
-                        } else {
-                            for (int j = 0; j < nmma; j++) one(j);
-                        }
-                    } else {
-                        tmem_cp_sf_atom_pair(slot0, desc_pack(sfa_lo, kSfHi));
-                        tmem_cp_sf_atom_pair(slot0 + 4, desc_pack(sfb_lo, kSfHi));
-                        tmem_cp_sf_atom_pair(slot0 + 8, desc_pack(sfb_lo + kSfbTileLo, kSfHi));
+                    for (int j = 0; j < 4; j++) {
+                        // SFB of MMA j: both 128-row atoms, replicated in every quarter
+                        const uint4 b0 = *reinterpret_cast<const uint4 *>(sfb + 512 * j + 16 * lane);
+                        const uint4 b1 = *reinterpret_cast<const uint4 *>(sfb + C_::kSfaBytes + 512 * j + 16 * lane);
+                        const uint32_t w[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+                        tmem_st_x8(sfb_t + 8 * j, w);
+                        // SFA of MMA j: this quarter's rows, in the column the quarter reads
+                        tmem_st_x1(sfa_t + 4 * j + q, *reinterpret_cast<const uint32_t *>(sfa + 512 * j + 16 * lane + 4 * q));
                     }
-                    issued = true;
-                    tc_commit_pair(smem_u32(&sf_ready[s]), 0x1);  // the copies of stage s have executed
-                    if (++s == NS) {
-                        s = 0;
-                        ph ^= 1u;
-                    }
+                } else {
+                    const uint4 b0 = *reinterpret_cast<const uint4 *>(sfb + 16 * lane);
+                    const uint4 b1 = *reinterpret_cast<const uint4 *>(sfb + C_::kSfaBytes + 16 * lane);
+                    const uint32_t w[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+                    tmem_st_x8(sfb_t, w);
+                    tmem_st_x1(sfa_t + q, *reinterpret_cast<const uint32_t *>(sfa + 16 * lane + 4 * q));
                 }
-            }
-            if (issued) {
-                // this thread's copies have executed before TMEM is freed
-                __shared__ __align__(8) uint64_t cp_drain;
-                mbar_init(smem_u32(&cp_drain), 1);
-                fence_barrier_init();
-                tc_commit_pair(smem_u32(&cp_drain), 0x1);
-                volatile int never = 0;
-                mbar_wait(smem_u32(&cp_drain), 0, &never, p.err, 5, kTimeoutNs);
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster_relaxed(ready0 + (uint32_t)(s * 8));
+                if (++s == NS) {
+                    s = 0;
+                    ph ^= 1u;
+                }
             }
         }
     } else {
         // ------------------------------------------------------------ epilogue (both CTAs)
-        const int ew = warp - 3;  // 0..7
+        const int ew = warp - 2 - C_::kSfWarps;  // 0..7
         const int q = warp & 3;
         const int half = ew >> 2;
         constexpr int HC = BN / 2;
@@ -855,26 +855,23 @@ __global__ void __launch_bounds__(352, 1)
         auto box_addr = [&](int box, int c) -> uint8_t * {
             return box_base + box * C_::kBoxBytes + lane * 64 + ((c ^ ((lane >> 1) & 3)) << 4);
         };
-        int64_t it = 0;
-        int nstored = 0;  // boxes handed to TMA: the ring position
-        // stage one 32-row box (this thread's 64-byte row in v) and store it at (x, y)
-        auto store_box = [&](const uint32_t (&v)[16], int64_t x, int64_t y) {
-            const int box = nstored & (C_::kBoxes - 1);
-            if (nstored >= C_::kBoxes) {
-                if (lane == 0) bulk_wait_read<C_::kBoxes - 1>();  // this box's previous store has read it
-                __syncwarp();
-            }
+        auto put_row = [&](int box, const uint32_t (&v)[16]) {
 #pragma unroll
             for (int c = 0; c < 4; c++)
                 *reinterpret_cast<uint4 *>(box_addr(box, c)) = make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) {
-                tma_store_2d(&tmC, smem_u32(box_base + box * C_::kBoxBytes), (int32_t)x, (int32_t)y);
-                bulk_commit();
-            }
-            nstored++;
         };
+        auto get_row = [&](int box, uint32_t (&v)[16]) {
+#pragma unroll
+            for (int c = 0; c < 4; c++) {
+                const uint4 w = *reinterpret_cast<const uint4 *>(box_addr(box, c));
+                v[4 * c] = w.x;
+                v[4 * c + 1] = w.y;
+                v[4 * c + 2] = w.z;
+                v[4 * c + 3] = w.w;
+            }
+        };
+        int64_t it = 0;
+        int nstored = 0;  // boxes this warp has handed to TMA (fp32 path: ring position)
         for (int64_t t = pair; t < total_tiles; t += npairs, it++) {
             int64_t a_row0, sfa_row0, m_lim, nt;
             int group;
@@ -895,45 +892,50 @@ __global__ void __launch_bounds__(352, 1)
             const int64_t n_lim = p.n_lim;
             const uint32_t tbase = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(half * HC);
             if (OUT_BF16) {
-                // drain this warp's 128 columns (bf16-packed) and release the accumulator
-                uint32_t pk[HC / 2];
-#pragma unroll
-                for (int c = 0; c < HC / 32; c += 2) {
-                    uint32_t r0[32], r1[32];
-                    tmem_ld32(tbase + 32 * c, r0);
-                    tmem_ld32(tbase + 32 * (c + 1), r1);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int j = 0; j < 16; j++) {
-                        __nv_bfloat162 h0 = __floats2bfloat162_rn(__fmul_rn(alpha, __uint_as_float(r0[2 * j])),
-                                                                  __fmul_rn(alpha, __uint_as_float(r0[2 * j + 1])));
-                        __nv_bfloat162 h1 = __floats2bfloat162_rn(__fmul_rn(alpha, __uint_as_float(r1[2 * j])),
-                                                                  __fmul_rn(alpha, __uint_as_float(r1[2 * j + 1])));
-                        pk[16 * c + j] = *reinterpret_cast<uint32_t *>(&h0);
-                        pk[16 * (c + 1) + j] = *reinterpret_cast<uint32_t *>(&h1);
-                    }
-                }
-                tc_fence_before();
+                // the previous tile's stores have finished reading the staging boxes
+                if (lane == 0) bulk_wait_read<0>();
                 __syncwarp();
-                if (lane == 0) mbar_arrive_cluster(acce_leader);
+                // drain the 128 columns into the 4 boxes, release the accumulator, store
 #pragma unroll
                 for (int c = 0; c < HC / 32; c++) {
-                    const int64_t n = nb0 + 32 * c;
+                    uint32_t r0[32];
+                    tmem_ld32(tbase + 32 * c, r0);
+                    tmem_ld_wait();
                     uint32_t v[16];
 #pragma unroll
-                    for (int j = 0; j < 16; j++) v[j] = pk[16 * c + j];
-                    if (n >= n_lim) {
-                        // past the last column: nothing to store
-                    } else if (box_rows_ok) {
-                        store_box(v, n, row0);
-                    } else if (row_ok) {
+                    for (int j = 0; j < 16; j++) {
+                        __nv_bfloat162 h = __floats2bfloat162_rn(__fmul_rn(alpha, __uint_as_float(r0[2 * j])),
+                                                                 __fmul_rn(alpha, __uint_as_float(r0[2 * j + 1])));
+                        v[j] = *reinterpret_cast<uint32_t *>(&h);
+                    }
+                    put_row(c, v);
+                }
+                tc_fence_before();
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster_relaxed(acce_leader);
+                if (box_rows_ok) {
+                    if (lane == 0) {
+                        for (int c = 0; c < HC / 32; c++)
+                            if (nb0 + 32 * c < n_lim)
+                                tma_store_2d(&tmC, smem_u32(box_base + c * C_::kBoxBytes), (int32_t)(nb0 + 32 * c),
+                                             (int32_t)row0);
+                        bulk_commit();
+                    }
+                } else if (row_ok) {
+                    for (int c = 0; c < HC / 32; c++) {
+                        const int64_t n = nb0 + 32 * c;
+                        if (n >= n_lim) break;
+                        uint32_t v[16];
+                        get_row(c, v);
                         uint16_t *dst = reinterpret_cast<uint16_t *>(static_cast<__nv_bfloat16 *>(p.C) + ar * p.ldc + n);
                         for (int j = 0; j < 32; j++)
                             if (n + j < n_lim) dst[j] = (j & 1) ? (uint16_t)(v[j / 2] >> 16) : (uint16_t)(v[j / 2] & 0xFFFFu);
                     }
                 }
             } else {
-                // fp32: 16-column boxes; the accumulator is released after the last load
+                // fp32: 16-column boxes through the 4-box ring; the accumulator is
+                // released after the last load
 #pragma unroll 1
                 for (int c = 0; c < HC / 16; c++) {
                     uint32_t r[16];
@@ -942,7 +944,7 @@ __global__ void __launch_bounds__(352, 1)
                     if (c == HC / 16 - 1) {
                         tc_fence_before();
                         __syncwarp();
-                        if (lane == 0) mbar_arrive_cluster(acce_leader);
+                        if (lane == 0) mbar_arrive_cluster_relaxed(acce_leader);
                     }
                     const int64_t n = nb0 + 16 * c;
                     if (n >= n_lim) continue;
@@ -950,7 +952,19 @@ __global__ void __launch_bounds__(352, 1)
 #pragma unroll
                     for (int j = 0; j < 16; j++) v[j] = __float_as_uint(__fmul_rn(alpha, __uint_as_float(r[j])));
                     if (box_rows_ok) {
-                        store_box(v, n, row0);
+                        const int box = nstored & (C_::kBoxes - 1);
+                        if (nstored >= C_::kBoxes) {
+                            if (lane == 0) bulk_wait_read<C_::kBoxes - 1>();  // this box's last store has read it
+                            __syncwarp();
+                        }
+                        put_row(box, v);
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            tma_store_2d(&tmC, smem_u32(box_base + box * C_::kBoxBytes), (int32_t)n, (int32_t)row0);
+                            bulk_commit();
+                        }
+                        nstored++;
                     } else if (row_ok) {
                         float *dst = static_cast<float *>(p.C) + ar * p.ldc + n;
                         for (int j = 0; j < 16; j++)
@@ -1109,7 +1123,7 @@ int dispatch(const GemmArgs &g, cudaStream_t s) {
     else if (g.out_bf16 && NB >= 256) bn = 256;
     else bn = 128;
     // CTA pairs (256x256 tiles) for large operands: on 8192x14336x4096 NVFP4
-    // they measure 3.62 PFLOP/s against 3.24 for single-CTA 128x256 tiles.
+    // they measure 4.40 PFLOP/s against 3.24 for single-CTA 128x256 tiles.
     // Single CTAs keep the skinny swap-AB case, operands with fewer than 256
     // rows, outputs that TMA cannot store (unaligned base or row stride) and
     // grouped NVFP4 with a half k-tile (that would need the exact extent of

@@ -289,6 +289,14 @@ BSQ_DEV uint32_t mapa(uint32_t saddr, uint32_t rank) {
 BSQ_DEV void mbar_arrive_cluster(uint32_t remote_bar) {
     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote_bar) : "memory");
 }
+// Relaxed arrive on a barrier of another (or this) CTA of the cluster.  Used
+// where the work being handed over is already complete when the arrive is
+// issued (TMEM stores or loads waited for with tcgen05.wait, then ordered
+// by tcgen05.fence::before_thread_sync): a release at cluster scope would
+// add nothing there and costs ~1000 cycles while TMA traffic is in flight.
+BSQ_DEV void mbar_arrive_cluster_relaxed(uint32_t bar) {
+    asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar) : "memory");
+}
 // TMA tile load by either CTA of a pair; completion is signalled on `bar`,
 // which may live in the peer CTA (no multicast).
 BSQ_DEV void tma_load_2d_pair(uint32_t dst, const void *tmap, uint32_t bar, int32_t x, int32_t y) {

@@ -32,6 +32,27 @@ NOMINAL_FP4_OVER_BF16 = 4.0   # 9 PF / 2.25 PF dense (B200 table on the pages)
 FALLBACK_HBM, FALLBACK_BF16 = 6650.0, 1590.0
 
 
+def ncu_traffic(profile, sources):
+    """DRAM bytes per launch recorded from an ncu capture in profiles/, or None
+    when the kernel's sources changed since the capture (the summary records
+    the sha256 of the sources it was taken with)."""
+    import hashlib
+    import re
+    path = os.path.join(ROOT, "profiles", profile)
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    t = re.search(r"^traffic_bytes_per_launch:\s*(\d+)", text, re.M)
+    h = re.search(r"^source_sha256[^:]*:\s*([0-9a-f]{64})", text, re.M)
+    if not t or not h:
+        return None
+    d = hashlib.sha256()
+    for src in sources:
+        with open(os.path.join(ROOT, src), "rb") as f:
+            d.update(f.read())
+    return int(t.group(1)) if d.hexdigest() == h.group(1) else None
+
+
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -310,9 +331,13 @@ def main():
                        "l2": "inputs larger than L2 (A+W bf16 = 176 MiB > 126 MB); no flush",
                        "parallelism": f"replicas x{world}"},
             "roofline": {"bound": "tensor", "achieved": gemm_tflops, "peak": fp4_peak, "unit": "TFLOP/s",
-                         "frac": gemm_tflops / fp4_peak, "traffic": None,
-                         "kernel": "gemm_bs_kernel (NVFP4 8192x14336x4096)",
-                         "peak_source": f"{src} bf16 burst {bf16} x {NOMINAL_FP4_OVER_BF16} (nominal FP4/BF16)"},
+                         "frac": gemm_tflops / fp4_peak,
+                         "traffic": ncu_traffic("gemm_pair_nvfp4_8192x14336x4096.md",
+                                                ["fp8_math_b200/csrc/gemm.cu", "fp8_math_b200/csrc/sm100.cuh"]),
+                         "algorithmic_bytes": (M * K + N * K) // 2 + (M + N) * (K // 16) + M * N * 2,
+                         "kernel": "gemm_bs2_kernel (NVFP4 8192x14336x4096, CTA pairs)",
+                         "peak_source": f"{src} bf16 burst {bf16} x {NOMINAL_FP4_OVER_BF16} (nominal FP4/BF16), "
+                                        f"of {src}"},
             "breakdown": {
                 "gemm_ms": g_ms, "gemm_tflops": gemm_tflops, "gemm_frac_of_9pf": gemm_tflops / 9000.0,
                 "quant_A_ms": statistics.mean(qa_ms), "quant_A_gbs": qa_gbs,

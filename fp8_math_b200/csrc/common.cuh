@@ -211,6 +211,64 @@ BSQ_DEV void load_rht16(const uint16_t *p, const uint32_t sw[8], f32x2 P[8]) {
     for (int k = 0; k < 8; k++) P[k] = f2_mul(P[k], quarter);
 }
 
+// 16 bf16 as 8 32-bit words (element 2k in the low half of word k), two
+// 16-byte loads.
+BSQ_DEV void load_words16(const uint16_t *p, uint32_t w[8]) {
+    const uint4 q0 = __ldg(reinterpret_cast<const uint4 *>(p));
+    const uint4 q1 = __ldg(reinterpret_cast<const uint4 *>(p + 8));
+    w[0] = q0.x; w[1] = q0.y; w[2] = q0.z; w[3] = q0.w;
+    w[4] = q1.x; w[5] = q1.y; w[6] = q1.z; w[7] = q1.w;
+}
+BSQ_DEV void words_to_pairs(const uint32_t w[8], f32x2 P[8]) {
+#pragma unroll
+    for (int k = 0; k < 8; k++) P[k] = f2_pack(bf16_lo(w[k]), bf16_hi(w[k]));
+}
+// u = H16 * diag(s) * x from 8 words, without the final 1/4: the same sign
+// flips and butterflies (strides 1, 2, 4, 8, RN) as load_rht16; y = u / 4.
+BSQ_DEV void rht16_u_words(const uint32_t w_in[8], const uint32_t sw[8], f32x2 P[8]) {
+#pragma unroll
+    for (int k = 0; k < 8; k++) {
+        const uint32_t w = w_in[k] ^ sw[k];
+        const float a = bf16_lo(w), b = bf16_hi(w);
+        P[k] = f2_pack(__fadd_rn(a, b), __fsub_rn(a, b));
+    }
+#pragma unroll
+    for (int h = 1; h < 8; h <<= 1) {
+#pragma unroll
+        for (int base = 0; base < 8; base += 2 * h) {
+#pragma unroll
+            for (int k = base; k < base + h; k++) {
+                const f32x2 a = P[k], b = P[k + h];
+                P[k] = f2_add(a, b);
+                P[k + h] = f2_sub(a, b);
+            }
+        }
+    }
+}
+BSQ_DEV void pairs_scale(f32x2 P[8], float c) {
+    const f32x2 C = f2_pack(c, c);
+#pragma unroll
+    for (int k = 0; k < 8; k++) P[k] = f2_mul(P[k], C);
+}
+// three-input max (sm_100)
+BSQ_DEV float fmax3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+// max |v| over 8 pairs, as a tree of three-input maxima
+BSQ_DEV float pairs_absmax3(const f32x2 P[8]) {
+    float v[16];
+#pragma unroll
+    for (int k = 0; k < 8; k++) f2_unpack(P[k], v[2 * k], v[2 * k + 1]);
+    float m0 = fmax3(fabsf(v[0]), fabsf(v[1]), fabsf(v[2]));
+    float m1 = fmax3(fabsf(v[3]), fabsf(v[4]), fabsf(v[5]));
+    float m2 = fmax3(fabsf(v[6]), fabsf(v[7]), fabsf(v[8]));
+    float m3 = fmax3(fabsf(v[9]), fabsf(v[10]), fabsf(v[11]));
+    float m4 = fmax3(fabsf(v[12]), fabsf(v[13]), fabsf(v[14]));
+    return fmax3(fmax3(m0, m1, m2), fmax3(m3, m4, fabsf(v[15])), 0.0f);
+}
+
 // Loads 16 bf16 as 8 fp32 pairs (no transform).
 BSQ_DEV void load16_pairs(const uint16_t *p, f32x2 P[8]) {
     const uint4 q0 = __ldg(reinterpret_cast<const uint4 *>(p));

@@ -25,6 +25,33 @@ static int lpr_shift_for(int64_t units_per_row) {
     return sh;
 }
 
+// max |y| of one 16-element block: with the RHT, y = u / 4 exactly and
+// RN(u/4) is monotone in u, so max|y| = RN(max|u| / 4): the quarter is
+// applied once, to the maximum.
+template <bool RHT>
+BSQ_DEV float block_absmax(const uint32_t w[8], const uint32_t sw[8]) {
+    f32x2 P[8];
+    if (RHT) rht16_u_words(w, sw, P);
+    else words_to_pairs(w, P);
+    const float m = pairs_absmax3(P);
+    return RHT ? __fmul_rn(m, 0.25f) : m;
+}
+
+BSQ_DEV void block_reduce_atomic_max(float m, unsigned int *amax_bits) {
+#pragma unroll
+    for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    __shared__ float red[8];
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float b = red[0];
+        for (int i = 1; i < (int)(blockDim.x >> 5); i++) b = fmaxf(b, red[i]);
+        // non-negative floats order like their bit patterns
+        atomicMax(amax_bits, __float_as_uint(b));
+    }
+}
+
+// Rows (optionally gathered through row_index) of a strided tensor.
 template <bool RHT, bool GATHER>
 __global__ void __launch_bounds__(256) amax_kernel(const uint16_t *__restrict__ x, int64_t M, int64_t K,
                                                    int64_t ldx, uint32_t mask,
@@ -43,23 +70,32 @@ __global__ void __launch_bounds__(256) amax_kernel(const uint16_t *__restrict__ 
         const int64_t src = GATHER ? (int64_t)__ldg(row_index + row) : row;
         const uint16_t *rp = x + src * ldx;
         for (int64_t kb = lk; kb < KB; kb += lpr) {
-            f32x2 P[8];
-            if (RHT) load_rht16(rp + kb * 16, sw, P);
-            else load16_pairs(rp + kb * 16, P);
-            m = fmaxf(m, pairs_absmax(P));
+            uint32_t w[8];
+            load_words16(rp + kb * 16, w);
+            m = fmaxf(m, block_absmax<RHT>(w, sw));
         }
     }
-#pragma unroll
-    for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-    __shared__ float red[8];
-    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        float b = red[0];
-        for (int i = 1; i < (int)(blockDim.x >> 5); i++) b = fmaxf(b, red[i]);
-        // non-negative floats order like their bit patterns
-        atomicMax(amax_bits, __float_as_uint(b));
+    block_reduce_atomic_max(m, amax_bits);
+}
+
+// Contiguous tensor as a flat sequence of 16-element blocks; two blocks per
+// thread in flight (both loads issued before either is reduced).
+template <bool RHT>
+__global__ void __launch_bounds__(256) amax_flat_kernel(const uint16_t *__restrict__ x, int64_t nblk, uint32_t mask,
+                                                        unsigned int *amax_bits) {
+    uint32_t sw[8];
+    rht_sign_words(mask, sw);
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    float m = 0.0f;
+    for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < nblk; b += 2 * stride) {
+        const int64_t b1 = b + stride;
+        uint32_t w0[8], w1[8];
+        load_words16(x + b * 16, w0);
+        if (b1 < nblk) load_words16(x + b1 * 16, w1);
+        m = fmaxf(m, block_absmax<RHT>(w0, sw));
+        if (b1 < nblk) m = fmaxf(m, block_absmax<RHT>(w1, sw));
     }
+    block_reduce_atomic_max(m, amax_bits);
 }
 
 // s_g = amax / (6 * 448); amax == 0 gives 1.
@@ -68,45 +104,77 @@ BSQ_DEV float global_scale_of(float amax) { return amax == 0.0f ? 1.0f : __fdiv_
 __global__ void finalize_global_scale_kernel(float *gs) { *gs = global_scale_of(*gs); }
 
 // ===================================================================== NVFP4
-// One NVFP4 candidate for a 1x16 row segment: scale code, den, packed codes.
-struct NvCand {
-    uint32_t sb;
-    float den;
-    uint2 codes;
+// Per-CTA tables and constants of one tensor's global scale s_g.  For every
+// E4M3 scale code sb: den[sb] = RN(e4m3(sb) * s_g) and rcp[sb] = RN(1/den)
+// -- the same two operations each block would do, done once.  The block
+// scale t = RN(RN(bamax / 6) / s_g) is first estimated as RN(bamax * c6),
+// c6 = RN(1 / RN(6 s_g)); the estimate is within 5 ulps of t, so wherever
+// it lies more than 16 ulps from every E4M3 rounding boundary it rounds to
+// the same code, and everywhere else (or outside the ranges where the bound
+// holds) the exact two divisions are done.
+struct NvScale {
+    float s_g, c6, c4;
+    bool fast;  // s_g in [2^-90, 2^100]: the estimate bound and the exact 1/4 fold hold
 };
 
-BSQ_DEV NvCand nv_candidate(const f32x2 P[8], float bamax, float divisor, float s_g) {
-    NvCand c;
-    float t = __fdiv_rn(__fdiv_rn(bamax, divisor), s_g);
-    c.sb = e4m3_rne(t);
-    float sbv = e4m3_to_f32(c.sb);
-    if (sbv == 0.0f) {
-        c.den = 0.0f;
-        c.codes = make_uint2(0u, 0u);
-        return c;
+BSQ_DEV NvScale nv_scale_setup(float s_g, float *den_tab, float *rcp_tab) {
+    if (threadIdx.x < 128) {
+        const float den = __fmul_rn(e4m3_to_f32(threadIdx.x), s_g);
+        den_tab[threadIdx.x] = den;
+        rcp_tab[threadIdx.x] = (threadIdx.x == 0 || threadIdx.x == 127) ? 0.0f : __frcp_rn(den);
     }
-    c.den = __fmul_rn(sbv, s_g);
-    const float r = __frcp_rn(c.den);
-    const f32x2 R = f2_pack(r, r);
-    float q[16];
-#pragma unroll
-    for (int k = 0; k < 8; k++) f2_unpack(f2_mul(P[k], R), q[2 * k], q[2 * k + 1]);
-    c.codes.x = cvt_e2m1x8(q);
-    c.codes.y = cvt_e2m1x8(q + 8);
+    __syncthreads();
+    NvScale c;
+    c.s_g = s_g;
+    c.c6 = __frcp_rn(__fmul_rn(6.0f, s_g));
+    c.c4 = __frcp_rn(__fmul_rn(4.0f, s_g));
+    c.fast = s_g >= 0x1p-90f && s_g <= 0x1p100f;
     return c;
 }
 
-// Squared error of a candidate, summed pairwise (0+1),(2+3),... four levels.
-BSQ_DEV float nv_block_err(const f32x2 P[8], const NvCand &c) {
+// E4M3 code of RN(RN(bamax / divisor) / s_g) (satfinite, RNE).
+BSQ_DEV uint32_t nv_scale_code(float bamax, float divisor, float c_div, const NvScale &c) {
+    if (c.fast && bamax >= 0x1p-120f) {
+        const float te = __fmul_rn(bamax, c_div);
+        const int lowd = (int)(__float_as_uint(te) & 0xFFFFFu) - 0x80000;
+        if (te >= 0x1p-6f && (lowd > 16 || lowd < -16)) return e4m3_rne(te);
+    }
+    return e4m3_rne(__fdiv_rn(__fdiv_rn(bamax, divisor), c.s_g));
+}
+
+// E2M1 codes of q = y * r for one block given as u (RHT: y = u / 4) or y.
+// With the fold, q = RN(u * (r / 4)), equal to RN(RN(u / 4) * r) whenever
+// u / 4 is not subnormal; when it is, |q| < 2^-27 (r <= 2^99 for s_g >=
+// 2^-90) and both give the zero code.
+template <bool RHT>
+BSQ_DEV uint2 nv_codes(const f32x2 P[8], float r, bool fold) {
+    float rr = r;
+    f32x2 Q[8];
+#pragma unroll
+    for (int k = 0; k < 8; k++) Q[k] = P[k];
+    if (RHT) {
+        if (fold) rr = __fmul_rn(r, 0.25f);
+        else pairs_scale(Q, 0.25f);
+    }
+    const f32x2 R = f2_pack(rr, rr);
+    float q[16];
+#pragma unroll
+    for (int k = 0; k < 8; k++) f2_unpack(f2_mul(Q[k], R), q[2 * k], q[2 * k + 1]);
+    return make_uint2(cvt_e2m1x8(q), cvt_e2m1x8(q + 8));
+}
+
+// Squared error of a candidate (scale den, codes), summed pairwise (0+1),
+// (2+3), ... over four levels, on the block values y.
+BSQ_DEV float nv_block_err(const f32x2 Y[8], uint2 codes, float den) {
     float v[16];
 #pragma unroll
-    for (int k = 0; k < 8; k++) f2_unpack(P[k], v[2 * k], v[2 * k + 1]);
+    for (int k = 0; k < 8; k++) f2_unpack(Y[k], v[2 * k], v[2 * k + 1]);
     float e[16];
 #pragma unroll
     for (int i = 0; i < 16; i++) {
-        uint32_t w = (i < 8) ? c.codes.x : c.codes.y;
+        uint32_t w = (i < 8) ? codes.x : codes.y;
         uint32_t code = (w >> (4 * (i & 7))) & 15u;
-        float deq = __fmul_rn(e2m1_to_f32(code), c.den);
+        float deq = __fmul_rn(e2m1_to_f32(code), den);
         float d = __fsub_rn(v[i], deq);
         e[i] = __fmul_rn(d, d);
     }
@@ -115,6 +183,28 @@ BSQ_DEV float nv_block_err(const f32x2 P[8], const NvCand &c) {
 #pragma unroll
         for (int i = 0; i < w / 2; i++) e[i] = __fadd_rn(e[2 * i], e[2 * i + 1]);
     return e[0];
+}
+
+// One 1x16 block: scale code and packed codes (Four Over Six optional).
+template <bool RHT, bool FOS>
+BSQ_DEV void nv_block_1d(const uint32_t w[8], const uint32_t sw[8], const NvScale &c, const float *den_tab,
+                         const float *rcp_tab, uint32_t &sb, uint2 &codes) {
+    f32x2 P[8];
+    if (RHT) rht16_u_words(w, sw, P);
+    else words_to_pairs(w, P);
+    const float mu = pairs_absmax3(P);
+    const float bamax = RHT ? __fmul_rn(mu, 0.25f) : mu;
+    sb = nv_scale_code(bamax, 6.0f, c.c6, c);
+    codes = sb ? nv_codes<RHT>(P, rcp_tab[sb], c.fast) : make_uint2(0u, 0u);
+    if (FOS) {
+        const uint32_t sb4 = nv_scale_code(bamax, 4.0f, c.c4, c);
+        const uint2 codes4 = sb4 ? nv_codes<RHT>(P, rcp_tab[sb4], c.fast) : make_uint2(0u, 0u);
+        if (RHT) pairs_scale(P, 0.25f);  // the block values y for the error
+        if (nv_block_err(P, codes4, den_tab[sb4]) < nv_block_err(P, codes, den_tab[sb])) {
+            sb = sb4;
+            codes = codes4;
+        }
+    }
 }
 
 // Row -> scale-factor row under expert groups (binary search of offsets).
@@ -145,18 +235,21 @@ BSQ_DEV void store_sf(uint8_t *sf, bool valid, uint32_t sb, int64_t sf_row, int6
     }
 }
 
-// 1x16 blocks: one thread per block of 16 (two 16-byte loads, one 8-byte
-// code store).  Loops are warp-uniform so that shuffles see all lanes.
+// 1x16 blocks, rows (gathered, grouped): one thread per block of 16 (two
+// 16-byte loads, one 8-byte code store).  Loops are warp-uniform so that
+// shuffles see all lanes.
 template <bool RHT, bool FOS, bool GATHER, bool GROUPED>
 __global__ void __launch_bounds__(256) quant_nvfp4_1d_kernel(
     const uint16_t *__restrict__ x, int64_t M, int64_t K, int64_t ldx, uint32_t mask,
     const int32_t *__restrict__ row_index, int G, const int32_t *__restrict__ row_off,
     const int32_t *__restrict__ sf_off, const float *amax_ptr, float *gs_out, int write_gs,
     uint8_t *__restrict__ codes, uint8_t *__restrict__ sf, RowMap map) {
+    __shared__ float den_tab[128], rcp_tab[128];
     const int64_t KB = K >> 4;
     const bool pack4 = (KB & 3) == 0;
     const float s_g = global_scale_of(*amax_ptr);
     if (write_gs && blockIdx.x == 0 && threadIdx.x == 0) *gs_out = s_g;
+    const NvScale c = nv_scale_setup(s_g, den_tab, rcp_tab);
     uint32_t sw[8];
     rht_sign_words(mask, sw);
     const int lpr = 1 << map.lpr_shift;
@@ -173,61 +266,112 @@ __global__ void __launch_bounds__(256) quant_nvfp4_1d_kernel(
             const int64_t kb = kb0 + lk;
             const bool valid = row_ok && kb < KB;
             const int64_t kk = kb < KB ? kb : KB - 1;
-            f32x2 P[8];
-            if (RHT) load_rht16(rp + kk * 16, sw, P);
-            else load16_pairs(rp + kk * 16, P);
-            const float bamax = pairs_absmax(P);
-            NvCand c = nv_candidate(P, bamax, 6.0f, s_g);
-            if (FOS) {
-                NvCand c4 = nv_candidate(P, bamax, 4.0f, s_g);
-                if (nv_block_err(P, c4) < nv_block_err(P, c)) c = c4;
-            }
-            if (valid) *reinterpret_cast<uint2 *>(codes + rr * (K >> 1) + kb * 8) = c.codes;
-            store_sf(sf, valid, c.sb, sf_row, kb, KB, pack4);
+            uint32_t w[8];
+            load_words16(rp + kk * 16, w);
+            uint32_t sb;
+            uint2 cd;
+            nv_block_1d<RHT, FOS>(w, sw, c, den_tab, rcp_tab, sb, cd);
+            if (valid) *reinterpret_cast<uint2 *>(codes + rr * (K >> 1) + kb * 8) = cd;
+            store_sf(sf, valid, sb, sf_row, kb, KB, pack4);
         }
     }
 }
 
-// 16x16 tiles: a CTA of 16 warps covers 16 rows x 32 blocks; warp w owns row
-// w of the tile, lane j block j.  The tile amax goes through shared memory.
-template <bool RHT>
-__global__ void __launch_bounds__(512) quant_nvfp4_2d_kernel(
-    const uint16_t *__restrict__ x, int64_t M, int64_t K, int64_t ldx, uint32_t mask,
-    const float *amax_ptr, float *gs_out, int write_gs, uint8_t *__restrict__ codes, uint8_t *__restrict__ sf) {
-    __shared__ float tile_amax[16][33];
-    const int64_t KB = K >> 4;
-    const uint32_t kb_tiles = (uint32_t)((KB + 31) >> 5);
-    const uint32_t tiles = (uint32_t)(M >> 4) * kb_tiles;
-    const bool pack4 = (KB & 3) == 0;
+// 1x16 blocks of a contiguous tensor (ldx == K, no gather or groups) whose
+// row holds a power-of-two number of blocks (>= 4): a flat sequence of
+// blocks, two per thread in flight.  Lanes 4j..4j+3 hold four consecutive
+// blocks of one row, so the scale bytes pack into one word.
+template <bool RHT, bool FOS>
+__global__ void __launch_bounds__(256) quant_nvfp4_1d_flat_kernel(
+    const uint16_t *__restrict__ x, int64_t nblk, int kb_shift, uint32_t mask, const float *amax_ptr,
+    float *gs_out, int write_gs, uint8_t *__restrict__ codes, uint8_t *__restrict__ sf) {
+    __shared__ float den_tab[128], rcp_tab[128];
     const float s_g = global_scale_of(*amax_ptr);
     if (write_gs && blockIdx.x == 0 && threadIdx.x == 0) *gs_out = s_g;
+    const NvScale c = nv_scale_setup(s_g, den_tab, rcp_tab);
     uint32_t sw[8];
     rht_sign_words(mask, sw);
-    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    for (uint32_t t = blockIdx.x; t < tiles; t += gridDim.x) {
-        const uint32_t rt = t / kb_tiles, kt = t - rt * kb_tiles;
-        const int64_t row = (int64_t)rt * 16 + w;
-        const int64_t kb = (int64_t)kt * 32 + lane;
-        const bool valid = kb < KB;
-        f32x2 P[8];
-        if (valid) {
-            const uint16_t *p = x + row * ldx + kb * 16;
-            if (RHT) load_rht16(p, sw, P);
-            else load16_pairs(p, P);
-        } else {
-#pragma unroll
-            for (int k = 0; k < 8; k++) P[k] = 0ull;
+    const int64_t KB = int64_t(1) << kb_shift;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    // the loop bound is rounded to whole warps so that shuffles see all lanes
+    const int64_t nwarp_blk = (nblk + 31) & ~int64_t(31);
+    for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b - (threadIdx.x & 31) < nwarp_blk;
+         b += 2 * stride) {
+        const int64_t b1 = b + stride;
+        const bool v0 = b < nblk, v1 = b1 < nblk;
+        uint32_t w0[8], w1[8];
+        load_words16(x + (v0 ? b : 0) * 16, w0);
+        load_words16(x + (v1 ? b1 : 0) * 16, w1);
+        uint32_t sb0, sb1;
+        uint2 cd0, cd1;
+        nv_block_1d<RHT, FOS>(w0, sw, c, den_tab, rcp_tab, sb0, cd0);
+        if (v0) *reinterpret_cast<uint2 *>(codes + b * 8) = cd0;
+        store_sf(sf, v0, sb0, b >> kb_shift, b & (KB - 1), KB, true);
+        if (__any_sync(0xFFFFFFFFu, v1)) {
+            nv_block_1d<RHT, FOS>(w1, sw, c, den_tab, rcp_tab, sb1, cd1);
+            if (v1) *reinterpret_cast<uint2 *>(codes + b1 * 8) = cd1;
+            store_sf(sf, v1, sb1, b1 >> kb_shift, b1 & (KB - 1), KB, true);
         }
-        const float bamax = pairs_absmax(P);
-        tile_amax[w][lane] = bamax;
-        __syncthreads();
-        float tmax = 0.0f;
+    }
+}
+
+// 16x16 tiles.  A warp covers one 16-row tile row and four consecutive
+// blocks: lane l handles row l % 16 and blocks 2 (l / 16) and 2 (l / 16) + 1
+// of the four.  The tile amax is a max over the 16 lanes of a half-warp
+// (four shuffles); lanes 0..15 pack their row's four scale bytes into one
+// word when the row's block count is a multiple of 4.
+template <bool RHT>
+__global__ void __launch_bounds__(256) quant_nvfp4_2d_kernel(
+    const uint16_t *__restrict__ x, int64_t M, int64_t K, int64_t ldx, uint32_t mask,
+    const float *amax_ptr, float *gs_out, int write_gs, uint8_t *__restrict__ codes, uint8_t *__restrict__ sf) {
+    __shared__ float den_tab[128], rcp_tab[128];
+    const float s_g = global_scale_of(*amax_ptr);
+    if (write_gs && blockIdx.x == 0 && threadIdx.x == 0) *gs_out = s_g;
+    const NvScale c = nv_scale_setup(s_g, den_tab, rcp_tab);
+    uint32_t sw[8];
+    rht_sign_words(mask, sw);
+    const int64_t KB = K >> 4;
+    const int64_t kq = (KB + 3) >> 2;                 // groups of four blocks per row
+    const int64_t tasks = (M >> 4) * kq;
+    const bool pack4 = (KB & 3) == 0;
+    const int lane = threadIdx.x & 31;
+    const int r16 = lane & 15, hw = lane >> 4;
+    const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    for (int64_t task = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); task < tasks; task += warps) {
+        const int64_t rt = task / kq, g4 = task - rt * kq;
+        const int64_t row = rt * 16 + r16;
+        const int64_t kbA = g4 * 4 + 2 * hw, kbB = kbA + 1;
+        const bool vA = kbA < KB, vB = kbB < KB;
+        uint32_t wA[8], wB[8];
+        load_words16(x + row * ldx + (vA ? kbA : 0) * 16, wA);
+        load_words16(x + row * ldx + (vB ? kbB : 0) * 16, wB);
+        uint32_t sbv[2];
+        uint2 cdv[2];
 #pragma unroll
-        for (int r = 0; r < 16; r++) tmax = fmaxf(tmax, tile_amax[r][lane]);
-        __syncthreads();
-        NvCand c = nv_candidate(P, tmax, 6.0f, s_g);
-        if (valid) *reinterpret_cast<uint2 *>(codes + row * (K >> 1) + kb * 8) = c.codes;
-        store_sf(sf, valid, c.sb, row, kb, KB, pack4);
+        for (int i = 0; i < 2; i++) {
+            const bool v = i ? vB : vA;
+            f32x2 P[8];
+            if (RHT) rht16_u_words(i ? wB : wA, sw, P);
+            else words_to_pairs(i ? wB : wA, P);
+            float mu = v ? pairs_absmax3(P) : 0.0f;
+#pragma unroll
+            for (int o = 1; o < 16; o <<= 1) mu = fmaxf(mu, __shfl_xor_sync(0xFFFFFFFFu, mu, o));
+            const float tmax = RHT ? __fmul_rn(mu, 0.25f) : mu;
+            const uint32_t sb = nv_scale_code(tmax, 6.0f, c.c6, c);
+            sbv[i] = sb;
+            cdv[i] = sb ? nv_codes<RHT>(P, rcp_tab[sb], c.fast) : make_uint2(0u, 0u);
+        }
+        if (vA) *reinterpret_cast<uint2 *>(codes + row * (K >> 1) + kbA * 8) = cdv[0];
+        if (vB) *reinterpret_cast<uint2 *>(codes + row * (K >> 1) + kbB * 8) = cdv[1];
+        const uint32_t pair = (sbv[0] & 0xFFu) | ((sbv[1] & 0xFFu) << 8);
+        const uint32_t other = __shfl_xor_sync(0xFFFFFFFFu, pair, 16);
+        if (pack4) {
+            if (hw == 0)
+                *reinterpret_cast<uint32_t *>(sf + sf_word_offset(row, g4, KB)) = pair | (other << 16);
+        } else {
+            if (vA) sf[sf_offset(row, kbA, KB)] = (uint8_t)sbv[0];
+            if (vB) sf[sf_offset(row, kbB, KB)] = (uint8_t)sbv[1];
+        }
     }
 }
 
@@ -466,6 +610,13 @@ static int grid_for(int64_t work_items, int per_block, int max_ctas) {
 
 void launch_amax(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, bool rht, uint32_t mask,
                  const int32_t *row_index, unsigned int *amax_bits, int num_sms, cudaStream_t s) {
+    if (!row_index && ldx == K) {
+        const int64_t nblk = M * (K >> 4);
+        const int grid = grid_for(nblk, 2 * 256, num_sms * 8);
+        if (rht) amax_flat_kernel<true><<<grid, 256, 0, s>>>(x, nblk, mask, amax_bits);
+        else amax_flat_kernel<false><<<grid, 256, 0, s>>>(x, nblk, mask, amax_bits);
+        return;
+    }
     RowMap map{lpr_shift_for(K >> 4)};
     const int grid = grid_for(M, 256 >> map.lpr_shift, num_sms * 8);
 #define BSQ_AMAX(R, G) amax_kernel<R, G><<<grid, 256, 0, s>>>(x, M, K, ldx, mask, row_index, amax_bits, map)
@@ -481,12 +632,25 @@ void launch_quant_nvfp4(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, bo
                         const int32_t *sf_off, const float *amax_ptr, float *gs_out, bool write_gs,
                         uint8_t *codes, uint8_t *sf, int num_sms, cudaStream_t s) {
     if (block_2d) {
-        const int64_t tiles = (M >> 4) * (((K >> 4) + 31) >> 5);
-        const int grid = grid_for(tiles, 1, num_sms * 4);
+        const int64_t tasks = (M >> 4) * (((K >> 4) + 3) >> 2);
+        const int grid = grid_for(tasks, 8, num_sms * 8);
         if (rht)
-            quant_nvfp4_2d_kernel<true><<<grid, 512, 0, s>>>(x, M, K, ldx, mask, amax_ptr, gs_out, write_gs, codes, sf);
+            quant_nvfp4_2d_kernel<true><<<grid, 256, 0, s>>>(x, M, K, ldx, mask, amax_ptr, gs_out, write_gs, codes, sf);
         else
-            quant_nvfp4_2d_kernel<false><<<grid, 512, 0, s>>>(x, M, K, ldx, mask, amax_ptr, gs_out, write_gs, codes, sf);
+            quant_nvfp4_2d_kernel<false><<<grid, 256, 0, s>>>(x, M, K, ldx, mask, amax_ptr, gs_out, write_gs, codes, sf);
+        return;
+    }
+    const int64_t KB = K >> 4;
+    if (!row_index && G == 0 && ldx == K && KB >= 4 && (KB & (KB - 1)) == 0) {
+        int kb_shift = 0;
+        while ((int64_t(1) << kb_shift) < KB) kb_shift++;
+        const int64_t nblk = M * KB;
+        const int grid = grid_for(nblk, 2 * 256, num_sms * 8);
+#define BSQ_NVF(R, F) \
+    quant_nvfp4_1d_flat_kernel<R, F><<<grid, 256, 0, s>>>(x, nblk, kb_shift, mask, amax_ptr, gs_out, write_gs, codes, sf)
+        if (rht) { if (fos) BSQ_NVF(true, true); else BSQ_NVF(true, false); }
+        else { if (fos) BSQ_NVF(false, true); else BSQ_NVF(false, false); }
+#undef BSQ_NVF
         return;
     }
     RowMap map{lpr_shift_for(K >> 4)};

@@ -144,7 +144,7 @@ BSQ_API int bsq_rht(const void *x_bf16, void *y_bf16, int64_t M, int64_t K, int6
  * [M][K], swizzled sf for M x K/32) is decoded exactly (E4M3 x 2^E, fp32),
  * transposed, and quantized again as in bsq_quant_mxfp8 with blocks of 32
  * along the old M: codes_col [K][M], sf_col for K rows x M/32 blocks.
- * M % 128 == 0 and K % 32 == 0 (so the input SF has no partial atom). */
+ * M % 32 == 0 and K % 32 == 0 (whole blocks of 32 along both axes). */
 BSQ_API int bsq_requant_transpose(const uint8_t *codes_row_dev, const uint8_t *sf_row_dev,
                           int64_t M, int64_t K, int rounding, uint64_t seed, uint32_t stream_id,
                           uint8_t *codes_col_dev, uint8_t *sf_col_dev, void *stream);

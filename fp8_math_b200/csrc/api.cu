@@ -94,7 +94,7 @@ int bsq_amax(const void *x, int64_t M, int64_t K, int64_t ldx, int rht_enable, u
     if (cudaMemsetAsync(amax_dev, 0, sizeof(float), s) != cudaSuccess) return BSQ_ERR_CUDA;
     if (M == 0 || K == 0) return BSQ_OK;
     bsq::launch_amax(static_cast<const uint16_t *>(x), M, K, ldx, rht_enable != 0, mask, row_index,
-                     reinterpret_cast<unsigned int *>(amax_dev), d->num_sms, s);
+                     reinterpret_cast<unsigned int *>(amax_dev), nullptr, nullptr, d->num_sms, s);
     return launch_status();
 }
 
@@ -112,20 +112,31 @@ int bsq_quant_nvfp4(const void *x, int64_t M, int64_t K, int64_t ldx, int block_
     if (int st = device_state(&d)) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const uint16_t *xx = static_cast<const uint16_t *>(x);
-    // Without an amax from the caller, the amax is accumulated in *gs, read
-    // by the quantize kernel, and finally replaced by s_g in place.
-    const bool in_place = (amax_in == nullptr) || (amax_in == gs);
-    if (amax_in == nullptr) {
+    if (M == 0 || K == 0) {
+        // empty tensor: amax 0, s_g = 1
         if (cudaMemsetAsync(gs, 0, sizeof(float), s) != cudaSuccess) return BSQ_ERR_CUDA;
-        if (M > 0 && K > 0)
-            bsq::launch_amax(xx, M, K, ldx, rht_enable != 0, mask, row_index, reinterpret_cast<unsigned int *>(gs),
-                             d->num_sms, s);
+        bsq::launch_finalize_global_scale(gs, s);
+        return launch_status();
     }
-    const float *amax_ptr = amax_in ? amax_in : gs;
-    if (M > 0 && K > 0)
+    if (amax_in == nullptr) {
+        // The amax pass uses the first 8 bytes of the caller's code buffer
+        // (overwritten by the quantize pass that follows on the same stream)
+        // as its scratch: a CTA counter and the amax bits.  Its last CTA
+        // writes s_g to *gs, which the quantize pass reads.
+        if (cudaMemsetAsync(codes, 0, 8, s) != cudaSuccess) return BSQ_ERR_CUDA;
+        unsigned int *scratch = reinterpret_cast<unsigned int *>(codes);
+        bsq::launch_amax(xx, M, K, ldx, rht_enable != 0, mask, row_index, scratch + 1, scratch, gs, d->num_sms, s);
         bsq::launch_quant_nvfp4(xx, M, K, ldx, block_2d != 0, four_over_six != 0, rht_enable != 0, mask, row_index,
-                                G, row_off, sf_off, amax_ptr, gs, !in_place, codes, sf, d->num_sms, s);
-    if (in_place || M == 0 || K == 0) bsq::launch_finalize_global_scale(gs, s);
+                                G, row_off, sf_off, gs, false, gs, false, codes, sf, d->num_sms, s);
+    } else if (amax_in == gs) {
+        // the caller's amax is in *gs: read it, then replace it by s_g in place
+        bsq::launch_quant_nvfp4(xx, M, K, ldx, block_2d != 0, four_over_six != 0, rht_enable != 0, mask, row_index,
+                                G, row_off, sf_off, gs, true, gs, false, codes, sf, d->num_sms, s);
+        bsq::launch_finalize_global_scale(gs, s);
+    } else {
+        bsq::launch_quant_nvfp4(xx, M, K, ldx, block_2d != 0, four_over_six != 0, rht_enable != 0, mask, row_index,
+                                G, row_off, sf_off, amax_in, true, gs, true, codes, sf, d->num_sms, s);
+    }
     return launch_status();
 }
 

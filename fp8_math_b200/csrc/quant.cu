@@ -37,17 +37,30 @@ BSQ_DEV float block_absmax(const uint32_t w[8], const uint32_t sw[8]) {
     return RHT ? __fmul_rn(m, 0.25f) : m;
 }
 
-BSQ_DEV void block_reduce_atomic_max(float m, unsigned int *amax_bits) {
+BSQ_DEV float global_scale_of(float amax);
+
+// CTA max -> atomicMax on the float bits (non-negative floats order like
+// their bit patterns).  With a counter, the last CTA to finish also turns
+// the tensor amax into s_g and writes it to *gs_out (fence, count, fence:
+// every other CTA's maximum is visible to the last one).
+BSQ_DEV void block_reduce_atomic_max(float m, unsigned int *amax_bits, unsigned int *counter, float *gs_out) {
 #pragma unroll
     for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-    __shared__ float red[8];
+    __shared__ float red[32];
     if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
     __syncthreads();
     if (threadIdx.x == 0) {
         float b = red[0];
         for (int i = 1; i < (int)(blockDim.x >> 5); i++) b = fmaxf(b, red[i]);
-        // non-negative floats order like their bit patterns
         atomicMax(amax_bits, __float_as_uint(b));
+        if (counter) {
+            __threadfence();
+            if (atomicAdd(counter, 1u) == gridDim.x - 1) {
+                __threadfence();
+                const float amax = __uint_as_float(atomicOr(amax_bits, 0u));
+                *gs_out = global_scale_of(amax);
+            }
+        }
     }
 }
 
@@ -56,7 +69,8 @@ template <bool RHT, bool GATHER>
 __global__ void __launch_bounds__(256) amax_kernel(const uint16_t *__restrict__ x, int64_t M, int64_t K,
                                                    int64_t ldx, uint32_t mask,
                                                    const int32_t *__restrict__ row_index,
-                                                   unsigned int *amax_bits, RowMap map) {
+                                                   unsigned int *amax_bits, unsigned int *counter, float *gs_out,
+                                                   RowMap map) {
     const int64_t KB = K >> 4;
     const int lpr = 1 << map.lpr_shift;
     const int rpi = 256 >> map.lpr_shift;
@@ -75,27 +89,29 @@ __global__ void __launch_bounds__(256) amax_kernel(const uint16_t *__restrict__ 
             m = fmaxf(m, block_absmax<RHT>(w, sw));
         }
     }
-    block_reduce_atomic_max(m, amax_bits);
+    block_reduce_atomic_max(m, amax_bits, counter, gs_out);
 }
 
-// Contiguous tensor as a flat sequence of 16-element blocks; two blocks per
-// thread in flight (both loads issued before either is reduced).
+// Contiguous tensor as a flat sequence of 16-element blocks; four blocks per
+// thread in flight (all loads issued before any is reduced).
 template <bool RHT>
 __global__ void __launch_bounds__(256) amax_flat_kernel(const uint16_t *__restrict__ x, int64_t nblk, uint32_t mask,
-                                                        unsigned int *amax_bits) {
+                                                        unsigned int *amax_bits, unsigned int *counter,
+                                                        float *gs_out) {
     uint32_t sw[8];
     rht_sign_words(mask, sw);
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     float m = 0.0f;
-    for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < nblk; b += 2 * stride) {
-        const int64_t b1 = b + stride;
-        uint32_t w0[8], w1[8];
-        load_words16(x + b * 16, w0);
-        if (b1 < nblk) load_words16(x + b1 * 16, w1);
-        m = fmaxf(m, block_absmax<RHT>(w0, sw));
-        if (b1 < nblk) m = fmaxf(m, block_absmax<RHT>(w1, sw));
+    for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < nblk; b += 4 * stride) {
+        uint32_t w[4][8];
+#pragma unroll
+        for (int i = 0; i < 4; i++)
+            if (b + i * stride < nblk) load_words16(x + (b + i * stride) * 16, w[i]);
+#pragma unroll
+        for (int i = 0; i < 4; i++)
+            if (b + i * stride < nblk) m = fmaxf(m, block_absmax<RHT>(w[i], sw));
     }
-    block_reduce_atomic_max(m, amax_bits);
+    block_reduce_atomic_max(m, amax_bits, counter, gs_out);
 }
 
 // s_g = amax / (6 * 448); amax == 0 gives 1.
@@ -242,12 +258,12 @@ template <bool RHT, bool FOS, bool GATHER, bool GROUPED>
 __global__ void __launch_bounds__(256) quant_nvfp4_1d_kernel(
     const uint16_t *__restrict__ x, int64_t M, int64_t K, int64_t ldx, uint32_t mask,
     const int32_t *__restrict__ row_index, int G, const int32_t *__restrict__ row_off,
-    const int32_t *__restrict__ sf_off, const float *amax_ptr, float *gs_out, int write_gs,
+    const int32_t *__restrict__ sf_off, const float *scale_src, int src_is_amax, float *gs_out, int write_gs,
     uint8_t *__restrict__ codes, uint8_t *__restrict__ sf, RowMap map) {
     __shared__ float den_tab[128], rcp_tab[128];
     const int64_t KB = K >> 4;
     const bool pack4 = (KB & 3) == 0;
-    const float s_g = global_scale_of(*amax_ptr);
+    const float s_g = src_is_amax ? global_scale_of(*scale_src) : *scale_src;
     if (write_gs && blockIdx.x == 0 && threadIdx.x == 0) *gs_out = s_g;
     const NvScale c = nv_scale_setup(s_g, den_tab, rcp_tab);
     uint32_t sw[8];
@@ -283,10 +299,10 @@ __global__ void __launch_bounds__(256) quant_nvfp4_1d_kernel(
 // blocks of one row, so the scale bytes pack into one word.
 template <bool RHT, bool FOS>
 __global__ void __launch_bounds__(256) quant_nvfp4_1d_flat_kernel(
-    const uint16_t *__restrict__ x, int64_t nblk, int kb_shift, uint32_t mask, const float *amax_ptr,
-    float *gs_out, int write_gs, uint8_t *__restrict__ codes, uint8_t *__restrict__ sf) {
+    const uint16_t *__restrict__ x, int64_t nblk, int kb_shift, uint32_t mask, const float *scale_src,
+    int src_is_amax, float *gs_out, int write_gs, uint8_t *__restrict__ codes, uint8_t *__restrict__ sf) {
     __shared__ float den_tab[128], rcp_tab[128];
-    const float s_g = global_scale_of(*amax_ptr);
+    const float s_g = src_is_amax ? global_scale_of(*scale_src) : *scale_src;
     if (write_gs && blockIdx.x == 0 && threadIdx.x == 0) *gs_out = s_g;
     const NvScale c = nv_scale_setup(s_g, den_tab, rcp_tab);
     uint32_t sw[8];
@@ -315,62 +331,67 @@ __global__ void __launch_bounds__(256) quant_nvfp4_1d_flat_kernel(
     }
 }
 
-// 16x16 tiles.  A warp covers one 16-row tile row and four consecutive
-// blocks: lane l handles row l % 16 and blocks 2 (l / 16) and 2 (l / 16) + 1
-// of the four.  The tile amax is a max over the 16 lanes of a half-warp
-// (four shuffles); lanes 0..15 pack their row's four scale bytes into one
-// word when the row's block count is a multiple of 4.
+// 16x16 tiles.  A warp covers one 16-row tile row and eight consecutive
+// blocks: lane l handles row l % 16 and the four consecutive blocks
+// 4 (l / 16) .. 4 (l / 16) + 3 (128 contiguous bytes, all loads in flight
+// together).  Each block's tile amax is a max over the 16 lanes of a
+// half-warp (four shuffles); a lane's four scale bytes form one word.
 template <bool RHT>
 __global__ void __launch_bounds__(256) quant_nvfp4_2d_kernel(
-    const uint16_t *__restrict__ x, int64_t M, int64_t K, int64_t ldx, uint32_t mask,
-    const float *amax_ptr, float *gs_out, int write_gs, uint8_t *__restrict__ codes, uint8_t *__restrict__ sf) {
+    const uint16_t *__restrict__ x, int64_t M, int64_t K, int64_t ldx, uint32_t mask, const float *scale_src,
+    int src_is_amax, float *gs_out, int write_gs, uint8_t *__restrict__ codes, uint8_t *__restrict__ sf) {
     __shared__ float den_tab[128], rcp_tab[128];
-    const float s_g = global_scale_of(*amax_ptr);
+    const float s_g = src_is_amax ? global_scale_of(*scale_src) : *scale_src;
     if (write_gs && blockIdx.x == 0 && threadIdx.x == 0) *gs_out = s_g;
     const NvScale c = nv_scale_setup(s_g, den_tab, rcp_tab);
     uint32_t sw[8];
     rht_sign_words(mask, sw);
     const int64_t KB = K >> 4;
-    const int64_t kq = (KB + 3) >> 2;                 // groups of four blocks per row
-    const int64_t tasks = (M >> 4) * kq;
+    const int64_t k8 = (KB + 7) >> 3;                 // groups of eight blocks per row
+    const int64_t tasks = (M >> 4) * k8;
     const bool pack4 = (KB & 3) == 0;
     const int lane = threadIdx.x & 31;
     const int r16 = lane & 15, hw = lane >> 4;
     const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
     for (int64_t task = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); task < tasks; task += warps) {
-        const int64_t rt = task / kq, g4 = task - rt * kq;
+        const int64_t rt = task / k8, g8 = task - rt * k8;
         const int64_t row = rt * 16 + r16;
-        const int64_t kbA = g4 * 4 + 2 * hw, kbB = kbA + 1;
-        const bool vA = kbA < KB, vB = kbB < KB;
-        uint32_t wA[8], wB[8];
-        load_words16(x + row * ldx + (vA ? kbA : 0) * 16, wA);
-        load_words16(x + row * ldx + (vB ? kbB : 0) * 16, wB);
-        uint32_t sbv[2];
-        uint2 cdv[2];
+        const int64_t kb0 = g8 * 8 + 4 * hw;
+        const uint16_t *rp = x + row * ldx;
+        uint32_t w[4][8];
 #pragma unroll
-        for (int i = 0; i < 2; i++) {
-            const bool v = i ? vB : vA;
+        for (int i = 0; i < 4; i++) load_words16(rp + (kb0 + i < KB ? kb0 + i : 0) * 16, w[i]);
+        uint32_t sbw = 0;
+        uint2 cd[4];
+#pragma unroll
+        for (int i = 0; i < 4; i++) {
+            const bool v = kb0 + i < KB;  // uniform over the half-warp
             f32x2 P[8];
-            if (RHT) rht16_u_words(i ? wB : wA, sw, P);
-            else words_to_pairs(i ? wB : wA, P);
+            if (RHT) rht16_u_words(w[i], sw, P);
+            else words_to_pairs(w[i], P);
             float mu = v ? pairs_absmax3(P) : 0.0f;
 #pragma unroll
             for (int o = 1; o < 16; o <<= 1) mu = fmaxf(mu, __shfl_xor_sync(0xFFFFFFFFu, mu, o));
             const float tmax = RHT ? __fmul_rn(mu, 0.25f) : mu;
             const uint32_t sb = nv_scale_code(tmax, 6.0f, c.c6, c);
-            sbv[i] = sb;
-            cdv[i] = sb ? nv_codes<RHT>(P, rcp_tab[sb], c.fast) : make_uint2(0u, 0u);
+            sbw |= (sb & 0xFFu) << (8 * i);
+            cd[i] = sb ? nv_codes<RHT>(P, rcp_tab[sb], c.fast) : make_uint2(0u, 0u);
         }
-        if (vA) *reinterpret_cast<uint2 *>(codes + row * (K >> 1) + kbA * 8) = cdv[0];
-        if (vB) *reinterpret_cast<uint2 *>(codes + row * (K >> 1) + kbB * 8) = cdv[1];
-        const uint32_t pair = (sbv[0] & 0xFFu) | ((sbv[1] & 0xFFu) << 8);
-        const uint32_t other = __shfl_xor_sync(0xFFFFFFFFu, pair, 16);
-        if (pack4) {
-            if (hw == 0)
-                *reinterpret_cast<uint32_t *>(sf + sf_word_offset(row, g4, KB)) = pair | (other << 16);
+        uint8_t *cp = codes + row * (K >> 1) + kb0 * 8;
+        if (kb0 + 3 < KB && ((K >> 1) & 15) == 0) {  // 16-byte aligned: rows of a multiple of 32 codes bytes
+            reinterpret_cast<uint4 *>(cp)[0] = make_uint4(cd[0].x, cd[0].y, cd[1].x, cd[1].y);
+            reinterpret_cast<uint4 *>(cp)[1] = make_uint4(cd[2].x, cd[2].y, cd[3].x, cd[3].y);
         } else {
-            if (vA) sf[sf_offset(row, kbA, KB)] = (uint8_t)sbv[0];
-            if (vB) sf[sf_offset(row, kbB, KB)] = (uint8_t)sbv[1];
+#pragma unroll
+            for (int i = 0; i < 4; i++)
+                if (kb0 + i < KB) reinterpret_cast<uint2 *>(cp)[i] = cd[i];
+        }
+        if (pack4) {
+            if (kb0 < KB) *reinterpret_cast<uint32_t *>(sf + sf_word_offset(row, kb0 >> 2, KB)) = sbw;
+        } else {
+#pragma unroll
+            for (int i = 0; i < 4; i++)
+                if (kb0 + i < KB) sf[sf_offset(row, kb0 + i, KB)] = (uint8_t)(sbw >> (8 * i));
         }
     }
 }
@@ -608,18 +629,38 @@ static int grid_for(int64_t work_items, int per_block, int max_ctas) {
     return (int)(g < 1 ? 1 : g);
 }
 
+// CTAs of `kernel` (256 threads, static shared memory only) that fit on the
+// device at once: the grid of the persistent streaming kernels is one full
+// wave, so no partial last wave leaves SMs idle.  Cached per kernel.
+template <auto Kern>
+static int resident_ctas(int num_sms) {
+    static int per_sm = 0;
+    if (per_sm == 0) {
+        int n = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, Kern, 256, 0) != cudaSuccess || n < 1) n = 1;
+        per_sm = n;
+    }
+    return per_sm * num_sms;
+}
+
 void launch_amax(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, bool rht, uint32_t mask,
-                 const int32_t *row_index, unsigned int *amax_bits, int num_sms, cudaStream_t s) {
+                 const int32_t *row_index, unsigned int *amax_bits, unsigned int *counter, float *gs_out,
+                 int num_sms, cudaStream_t s) {
     if (!row_index && ldx == K) {
         const int64_t nblk = M * (K >> 4);
-        const int grid = grid_for(nblk, 2 * 256, num_sms * 8);
-        if (rht) amax_flat_kernel<true><<<grid, 256, 0, s>>>(x, nblk, mask, amax_bits);
-        else amax_flat_kernel<false><<<grid, 256, 0, s>>>(x, nblk, mask, amax_bits);
+        if (rht) {
+            const int grid = grid_for(nblk, 4 * 256, resident_ctas<amax_flat_kernel<true>>(num_sms));
+            amax_flat_kernel<true><<<grid, 256, 0, s>>>(x, nblk, mask, amax_bits, counter, gs_out);
+        } else {
+            const int grid = grid_for(nblk, 4 * 256, resident_ctas<amax_flat_kernel<false>>(num_sms));
+            amax_flat_kernel<false><<<grid, 256, 0, s>>>(x, nblk, mask, amax_bits, counter, gs_out);
+        }
         return;
     }
     RowMap map{lpr_shift_for(K >> 4)};
     const int grid = grid_for(M, 256 >> map.lpr_shift, num_sms * 8);
-#define BSQ_AMAX(R, G) amax_kernel<R, G><<<grid, 256, 0, s>>>(x, M, K, ldx, mask, row_index, amax_bits, map)
+#define BSQ_AMAX(R, G) \
+    amax_kernel<R, G><<<grid, 256, 0, s>>>(x, M, K, ldx, mask, row_index, amax_bits, counter, gs_out, map)
     if (rht) { if (row_index) BSQ_AMAX(true, true); else BSQ_AMAX(true, false); }
     else { if (row_index) BSQ_AMAX(false, true); else BSQ_AMAX(false, false); }
 #undef BSQ_AMAX
@@ -629,15 +670,18 @@ void launch_finalize_global_scale(float *gs, cudaStream_t s) { finalize_global_s
 
 void launch_quant_nvfp4(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, bool block_2d, bool fos,
                         bool rht, uint32_t mask, const int32_t *row_index, int G, const int32_t *row_off,
-                        const int32_t *sf_off, const float *amax_ptr, float *gs_out, bool write_gs,
-                        uint8_t *codes, uint8_t *sf, int num_sms, cudaStream_t s) {
+                        const int32_t *sf_off, const float *scale_src, bool src_is_amax, float *gs_out,
+                        bool write_gs, uint8_t *codes, uint8_t *sf, int num_sms, cudaStream_t s) {
+    const int sa = src_is_amax ? 1 : 0, wg = write_gs ? 1 : 0;
     if (block_2d) {
-        const int64_t tasks = (M >> 4) * (((K >> 4) + 3) >> 2);
-        const int grid = grid_for(tasks, 8, num_sms * 8);
-        if (rht)
-            quant_nvfp4_2d_kernel<true><<<grid, 256, 0, s>>>(x, M, K, ldx, mask, amax_ptr, gs_out, write_gs, codes, sf);
-        else
-            quant_nvfp4_2d_kernel<false><<<grid, 256, 0, s>>>(x, M, K, ldx, mask, amax_ptr, gs_out, write_gs, codes, sf);
+        const int64_t tasks = (M >> 4) * (((K >> 4) + 7) >> 3);
+        if (rht) {
+            const int grid = grid_for(tasks, 8, resident_ctas<quant_nvfp4_2d_kernel<true>>(num_sms));
+            quant_nvfp4_2d_kernel<true><<<grid, 256, 0, s>>>(x, M, K, ldx, mask, scale_src, sa, gs_out, wg, codes, sf);
+        } else {
+            const int grid = grid_for(tasks, 8, resident_ctas<quant_nvfp4_2d_kernel<false>>(num_sms));
+            quant_nvfp4_2d_kernel<false><<<grid, 256, 0, s>>>(x, M, K, ldx, mask, scale_src, sa, gs_out, wg, codes, sf);
+        }
         return;
     }
     const int64_t KB = K >> 4;
@@ -645,9 +689,10 @@ void launch_quant_nvfp4(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, bo
         int kb_shift = 0;
         while ((int64_t(1) << kb_shift) < KB) kb_shift++;
         const int64_t nblk = M * KB;
-        const int grid = grid_for(nblk, 2 * 256, num_sms * 8);
-#define BSQ_NVF(R, F) \
-    quant_nvfp4_1d_flat_kernel<R, F><<<grid, 256, 0, s>>>(x, nblk, kb_shift, mask, amax_ptr, gs_out, write_gs, codes, sf)
+#define BSQ_NVF(R, F)                                                                                          \
+    quant_nvfp4_1d_flat_kernel<R, F><<<grid_for(nblk, 2 * 256, resident_ctas<quant_nvfp4_1d_flat_kernel<R, F>>( \
+                                                                             num_sms)),                        \
+                                       256, 0, s>>>(x, nblk, kb_shift, mask, scale_src, sa, gs_out, wg, codes, sf)
         if (rht) { if (fos) BSQ_NVF(true, true); else BSQ_NVF(true, false); }
         else { if (fos) BSQ_NVF(false, true); else BSQ_NVF(false, false); }
 #undef BSQ_NVF
@@ -658,7 +703,7 @@ void launch_quant_nvfp4(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, bo
     const bool gather = row_index != nullptr, grouped = G > 0;
 #define BSQ_NV1(R, F, GA, GR)                                                                            \
     quant_nvfp4_1d_kernel<R, F, GA, GR><<<grid, 256, 0, s>>>(x, M, K, ldx, mask, row_index, G, row_off, \
-                                                            sf_off, amax_ptr, gs_out, write_gs, codes, sf, map)
+                                                            sf_off, scale_src, sa, gs_out, wg, codes, sf, map)
 #define BSQ_NV1_G(R, F)                                 \
     do {                                                \
         if (gather) {                                   \

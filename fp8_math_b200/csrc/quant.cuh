@@ -5,13 +5,17 @@
 
 namespace bsq {
 
+// amax into *amax_bits (zeroed by the caller).  With a counter (zeroed by
+// the caller too) the kernel's last CTA also writes s_g = amax / 2688 to
+// *gs_out.
 void launch_amax(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, bool rht, uint32_t mask,
-                 const int32_t *row_index, unsigned int *amax_bits, int num_sms, cudaStream_t s);
+                 const int32_t *row_index, unsigned int *amax_bits, unsigned int *counter, float *gs_out,
+                 int num_sms, cudaStream_t s);
 void launch_finalize_global_scale(float *gs, cudaStream_t s);
 void launch_quant_nvfp4(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, bool block_2d, bool fos,
                         bool rht, uint32_t mask, const int32_t *row_index, int G, const int32_t *row_off,
-                        const int32_t *sf_off, const float *amax_ptr, float *gs_out, bool write_gs,
-                        uint8_t *codes, uint8_t *sf, int num_sms, cudaStream_t s);
+                        const int32_t *sf_off, const float *scale_src, bool src_is_amax, float *gs_out,
+                        bool write_gs, uint8_t *codes, uint8_t *sf, int num_sms, cudaStream_t s);
 void launch_quant_mxfp8(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, bool colwise, bool sr,
                         uint64_t seed, uint32_t stream_id, uint8_t *codes, uint8_t *sf, int num_sms,
                         cudaStream_t s);

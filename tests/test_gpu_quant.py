@@ -85,6 +85,40 @@ def test_nvfp4_2d_parity(ora, M, K):
     _nvfp4_check(ora, x, block_2d=True, what=f"nvfp4 2d {M}x{K}")
 
 
+def _midpoint_tensor(rows_per_block, seed):
+    """Blocks whose scale t = (bamax / 6) / s_g sits on an E4M3 rounding
+    midpoint (or one bf16 step away): amax = 7168 gives s_g = 7168 / 2688,
+    and a block maximum of 16 m makes bamax / (6 s_g) = m exactly in real
+    arithmetic, so the fp32 result lands within an ulp or two of the tie.
+    Covers every normal-range midpoint (k + 1/2) 2^(e-3) and the subnormal
+    ones (k + 1/2) 2^-9."""
+    mids = [(k + 0.5) * 2.0 ** (e - 3) for e in range(-6, 9) for k in range(8, 16)]
+    mids = [m for m in mids if m < 448] + [(k + 0.5) * 2.0 ** -9 for k in range(8)]
+    targets = []
+    for m in mids:
+        b = torch.tensor([16 * m], dtype=torch.float32).to(torch.bfloat16)
+        up = (b.view(torch.int16) + 1).view(torch.bfloat16)
+        dn = (b.view(torch.int16) - 1).view(torch.bfloat16)
+        targets += [b.item(), up.item(), dn.item()]
+    nb = len(targets) + 1
+    g = torch.Generator().manual_seed(seed)
+    x = torch.empty(rows_per_block, 16 * nb)
+    for j in range(nb):
+        peak = 7168.0 if j == 0 else targets[j - 1]
+        blk = (torch.rand(rows_per_block, 16, generator=g) * 2 - 1) * peak * 0.9
+        blk[0, int(j % 16)] = -peak if j % 3 == 1 else peak
+        x[:, 16 * j:16 * (j + 1)] = blk
+    return x.to(torch.bfloat16)
+
+
+def test_nvfp4_scale_rounding_midpoints(ora):
+    x1 = _midpoint_tensor(1, 11)
+    _nvfp4_check(ora, x1, what="1x16 scale midpoints")
+    _nvfp4_check(ora, x1, fos=True, what="4/6 scale midpoints")
+    x2 = _midpoint_tensor(16, 12)
+    _nvfp4_check(ora, x2, block_2d=True, what="16x16 scale midpoints")
+
+
 @pytest.mark.parametrize("block_2d", [False, True])
 def test_nvfp4_rht_parity(ora, block_2d):
     A, Wt, seed = W.nvfp4_linear_rht(M=256, N=272, K=512)

@@ -29,6 +29,7 @@ RHT_SEED = 2
 METRIC = "NVFP4 GEMM TFLOPS (% of 9 PF FP4); quantize GB/s (% of HBM peak), 1×B200"
 WORKLOAD = "nvfp4_linear_rht: A 8192x4096 N(0,1) w/ 0.5% channels x100, W 14336x4096 N(0,0.02), 16x16 RHT seed 2"
 NOMINAL_FP4_OVER_BF16 = 4.0   # 9 PF / 2.25 PF dense (B200 table on the pages)
+NOMINAL_FP8_OVER_BF16 = 2.0   # 4.5 PF / 2.25 PF
 FALLBACK_HBM, FALLBACK_BF16 = 6650.0, 1590.0
 
 
@@ -51,6 +52,20 @@ def ncu_traffic(profile, sources):
         with open(os.path.join(ROOT, src), "rb") as f:
             d.update(f.read())
     return int(t.group(1)) if d.hexdigest() == h.group(1) else None
+
+
+def max_over_ranks(x: float, dist, device) -> float:
+    """The largest x over all ranks (every rank calls it, same order)."""
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tflops(world: int, flops_per_step: float, ms_per_step: float) -> float:
+    """Whole-job throughput: every rank runs one full step (weak scaling),
+    timed by the slowest rank."""
+    return world * flops_per_step / (ms_per_step * 1e-3) / 1e12
 
 
 def peaks():
@@ -161,6 +176,178 @@ def reference_arm(args, rank):
     print(json.dumps(line), flush=True)
 
 
+# ---------------------------------------------------------------------- per-row measurements
+def measure_rows(hbm, fp4_peak, fp8_peak, reps=10, only=None):
+    """Times every step of the hot path on its own workload at full size
+    (CUDA events around each call, L2 flushed before each rep by writing a
+    256 MiB buffer, median of `reps`).  Returns a list of dicts; a row that
+    fails records its error instead of stopping the bench."""
+    import torch
+
+    from fp8_math_b200 import api, bsq
+    from fp8_math_b200 import workloads as W
+
+    dev = torch.device("cuda")
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        ts = []
+        for _ in range(reps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            e1.synchronize()
+            ts.append(e0.elapsed_time(e1) * 1e3)
+        if bsq.bsq_check() != bsq.BSQ_OK:
+            raise RuntimeError("device error")
+        return statistics.median(ts)
+
+    rows = []
+
+    def row(name, workload, fn, nbytes=None, flops=None, peak_kind=None):
+        if only and only not in name:
+            return
+        try:
+            us = timed(fn)
+            r = {"row": name, "workload": workload, "us": round(us, 2)}
+            if flops is not None:
+                peak = fp4_peak if peak_kind == "fp4" else fp8_peak
+                tf = flops / (us * 1e-6) / 1e12
+                r.update({"value": round(tf, 1), "unit": "TFLOP/s",
+                          "roofline": {"bound": "tensor", "achieved": round(tf, 1), "peak": peak,
+                                       "frac": round(tf / peak, 3)}})
+            else:
+                gbs = nbytes / (us * 1e-6) / 1e9
+                r.update({"value": round(gbs, 1), "unit": "GB/s",
+                          "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm,
+                                       "frac": round(gbs / hbm, 3), "bytes": int(nbytes)}})
+            rows.append(r)
+        except Exception as e:  # noqa: BLE001 -- recorded, not fatal
+            rows.append({"row": name, "workload": workload, "error": str(e)[:200]})
+
+    # -- configs[2]: linear with RHT (the timed step's calls, one at a time)
+    A_h, W_h, seed = W.nvfp4_linear_rht()
+    mask = bsq.bsq_rht_sign_mask(seed)
+    A, Wd = A_h.to(dev), W_h.to(dev)
+    M2, K2 = A.shape
+    N2 = Wd.shape[0]
+    am = torch.empty(1, device=dev)
+    row("a1 amax (RHT)", "A 8192x4096 bf16", lambda: bsq.bsq_amax(A, M2, K2, K2, 1, mask, None, am),
+        nbytes=M2 * K2 * 2)
+    qa = api.quant_nvfp4(A, rht_mask=mask)
+    row("a2+a5 NVFP4 1x16 quantize (amax + RHT fused)", "A 8192x4096",
+        lambda: api.quant_nvfp4(A, rht_mask=mask, out=qa), nbytes=M2 * K2 * (2 + 2 + 0.5 + 1 / 16))
+    qw = api.quant_nvfp4(Wd, block_2d=True, rht_mask=mask)
+    row("a3+a5 NVFP4 16x16 quantize (amax + RHT fused)", "W 14336x4096",
+        lambda: api.quant_nvfp4(Wd, block_2d=True, rht_mask=mask, out=qw), nbytes=N2 * K2 * (2 + 2 + 0.5 + 1 / 16))
+    y = torch.empty_like(A)
+    row("a5 RHT standalone (bf16 -> bf16)", "A 8192x4096", lambda: api.rht(A, mask, out=y), nbytes=M2 * K2 * 4)
+    C2 = torch.empty(M2, N2, dtype=torch.bfloat16, device=dev)
+    row("a8 NVFP4 GEMM bf16", "8192x14336x4096",
+        lambda: api.gemm(0, qa[0], qa[1], qw[0], qw[1], M2, N2, K2, gsA=qa[2], gsB=qw[2], out=C2),
+        flops=2 * M2 * N2 * K2, peak_kind="fp4")
+    del y, C2
+    # -- configs[0]: the small NVFP4 linear (latency)
+    As, Ws = W.nvfp4_linear_small()
+    As, Ws = As.to(dev), Ws.to(dev)
+    qas, qws = api.quant_nvfp4(As), api.quant_nvfp4(Ws, block_2d=True)
+    Cs = torch.empty(128, 256, dtype=torch.float32, device=dev)
+
+    def small_step():
+        api.quant_nvfp4(As, out=qas)
+        api.quant_nvfp4(Ws, block_2d=True, out=qws)
+        api.gemm(0, qas[0], qas[1], qws[0], qws[1], 128, 256, 256, gsA=qas[2], gsB=qws[2], out=Cs)
+    row("a2+a3+a8 small linear step (latency)", "A 128x256, W 256x256, fp32 out", small_step,
+        nbytes=(128 + 256) * 256 * 2)
+    # -- configs[1]: MXFP8 4096^2 Student-t, RNE and SR, requant-transpose
+    X1 = W.mxfp8_requant().to(dev)
+    M1, K1 = X1.shape
+    q1 = api.quant_mxfp8(X1)
+    row("a6 MXFP8 row quantize RNE", "X 4096x4096", lambda: api.quant_mxfp8(X1, out=q1),
+        nbytes=M1 * K1 * (2 + 1 + 1 / 32))
+    q1s = api.quant_mxfp8(X1, sr=True, seed=1)
+    row("a6 MXFP8 row quantize SR (Philox)", "X 4096x4096", lambda: api.quant_mxfp8(X1, sr=True, seed=1, out=q1s),
+        nbytes=M1 * K1 * (2 + 1 + 1 / 32))
+    qt = api.requant_transpose(q1s[0], q1s[1], sr=True, seed=1)
+    row("a7 requant-transpose SR", "4096x4096 MXFP8 -> column-wise",
+        lambda: api.requant_transpose(q1s[0], q1s[1], sr=True, seed=1, out=qt), nbytes=2 * M1 * K1 * (1 + 1 / 32))
+    del X1, q1, q1s, qt
+    # -- configs[4]: MXFP8 backward + rollout
+    dY, W4, X4, A_roll = W.mxfp8_backward()
+    dY, W4, X4 = dY.to(dev), W4.to(dev), X4.to(dev)
+    M4, N4 = dY.shape
+    K4 = W4.shape[1]
+    qdr = api.quant_mxfp8(dY, sr=True, seed=4, stream_id=0)
+    row("a6 MXFP8 row quantize SR", "dY 8192x14336", lambda: api.quant_mxfp8(dY, sr=True, seed=4, out=qdr),
+        nbytes=M4 * N4 * (2 + 1 + 1 / 32))
+    qdc = api.quant_mxfp8(dY, colwise=True, sr=True, seed=4, stream_id=1)
+    row("a6 MXFP8 column quantize SR", "dY 8192x14336 -> [14336, 8192]",
+        lambda: api.quant_mxfp8(dY, colwise=True, sr=True, seed=4, stream_id=1, out=qdc),
+        nbytes=M4 * N4 * (2 + 1 + 1 / 32))
+    qwc = api.quant_mxfp8(W4, colwise=True, sr=True, seed=4, stream_id=2)
+    qxc = api.quant_mxfp8(X4, colwise=True, sr=True, seed=4, stream_id=3)
+    Cd = torch.empty(M4, K4, dtype=torch.bfloat16, device=dev)
+    row("a8 MXFP8 GEMM dgrad (bf16 out)", "8192x4096x14336",
+        lambda: api.gemm(1, qdr[0], qdr[1], qwc[0], qwc[1], M4, K4, N4, out=Cd), flops=2 * M4 * K4 * N4,
+        peak_kind="fp8")
+    del Cd
+    Cw = torch.empty(N4, K4, dtype=torch.float32, device=dev)
+    row("a8 MXFP8 GEMM wgrad (fp32 out)", "14336x4096x8192",
+        lambda: api.gemm(1, qdc[0], qdc[1], qxc[0], qxc[1], N4, K4, M4, out=Cw), flops=2 * N4 * K4 * M4,
+        peak_kind="fp8")
+    del Cw, qdr, qdc, qxc, dY, X4
+    qar = api.quant_nvfp4(A_roll.to(dev))
+    qwr = api.quant_nvfp4(W4, block_2d=True)
+    Cr = torch.empty(64, N4, dtype=torch.bfloat16, device=dev)
+    row("a8 NVFP4 rollout GEMM (swap-AB, HBM-bound)", "64x14336x4096",
+        lambda: api.gemm(0, qar[0], qar[1], qwr[0], qwr[1], 64, N4, K4, gsA=qar[2], gsB=qwr[2], out=Cr),
+        nbytes=N4 * K4 // 2 + N4 * K4 // 16 + 64 * K4 // 2 + 64 * K4 // 16 + 64 * N4 * 2)
+    del Cr, qar, qwr, W4, qwc
+    # -- configs[3]: MoE forward (gathered 4/6 quantize, grouped up and down)
+    moe = W.moe_forward()
+    T3, H3 = moe.X.shape
+    E3, F3, _ = moe.W_up.shape
+    ri = torch.from_numpy(moe.row_index).to(dev)
+    offs = torch.from_numpy(moe.row_offsets).to(dev)
+    sfo = torch.from_numpy(moe.sf_row_offsets).to(dev)
+    Mt, sf_rows = int(moe.row_offsets[-1]), int(moe.sf_row_offsets[-1])
+    Xd = moe.X.to(dev)
+    qx = api.quant_nvfp4(Xd, four_over_six=True, row_index=ri, groups=(offs, sfo, sf_rows))
+    row("a4 NVFP4 Four Over Six quantize (gathered, expert groups)", "X 16384x4096 -> 131072 routed rows",
+        lambda: api.quant_nvfp4(Xd, four_over_six=True, row_index=ri, groups=(offs, sfo, sf_rows), out=qx),
+        nbytes=Mt * H3 * (2 + 2 + 0.5 + 1 / 16))
+
+    def experts(Wx):
+        E, N, K = Wx.shape
+        codes = torch.empty(E, N, K // 2, dtype=torch.uint8, device=dev)
+        sfb = torch.zeros(E * bsq.bsq_sf_bytes(N, K // 16), dtype=torch.uint8, device=dev)
+        gsb = torch.empty(E, dtype=torch.float32, device=dev)
+        per = bsq.bsq_sf_bytes(N, K // 16)
+        for e in range(E):
+            we = Wx[e].to(dev)
+            api.quant_nvfp4(we, block_2d=True, out=(codes[e], sfb[e * per:(e + 1) * per], gsb[e:e + 1]))
+        return codes, sfb, gsb
+    up = experts(moe.W_up)
+    Cup = torch.empty(Mt, F3, dtype=torch.bfloat16, device=dev)
+    row("a9 grouped NVFP4 GEMM up", f"{Mt} routed rows x {F3} x {H3}, 64 experts",
+        lambda: api.grouped_gemm(0, offs, sfo, qx[0], qx[1], up[0], up[1], Mt, F3, H3, gsA=qx[2], gsB=up[2],
+                                 out=Cup), flops=2 * Mt * F3 * H3, peak_kind="fp4")
+    qh = api.quant_nvfp4(Cup, four_over_six=True, groups=(offs, sfo, sf_rows))
+    del up
+    dn = experts(moe.W_dn)
+    Cdn = torch.empty(Mt, H3, dtype=torch.bfloat16, device=dev)
+    row("a9 grouped NVFP4 GEMM down", f"{Mt} routed rows x {H3} x {F3}, 64 experts",
+        lambda: api.grouped_gemm(0, offs, sfo, qh[0], qh[1], dn[0], dn[1], Mt, H3, F3, gsA=qh[2], gsB=dn[2],
+                                 out=Cdn), flops=2 * Mt * H3 * F3, peak_kind="fp4")
+    del flush
+    return rows
+
+
 # ---------------------------------------------------------------------- ours
 def main():
     ap = argparse.ArgumentParser()
@@ -169,6 +356,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-rows", action="store_true", help="skip the per-row measurements")
+    ap.add_argument("--rows-only", default=None, metavar="SUBSTR",
+                    help="run only the per-row measurements whose name contains SUBSTR, print them, exit")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -178,6 +368,13 @@ def main():
 
     if args.impl == "reference":
         return reference_arm(args, rank)
+    if args.rows_only is not None:
+        import torch
+        hbm, bf16, _ = peaks()
+        torch.cuda.set_device(0)
+        print(json.dumps(measure_rows(hbm, bf16 * NOMINAL_FP4_OVER_BF16, bf16 * NOMINAL_FP8_OVER_BF16,
+                                      reps=max(args.steps, 1), only=args.rows_only)), flush=True)
+        return
 
     import torch
     import torch.distributed as dist
@@ -221,7 +418,7 @@ def main():
         q_w()
         gemm()
 
-    launches_per_step = 7  # per operand: amax, quantize, finalize; plus the GEMM
+    launches_per_step = 5  # per operand: amax pass, quantize pass; plus the GEMM
 
     for _ in range(args.warmup):
         step()
@@ -265,12 +462,10 @@ def main():
     if st != bsq.BSQ_OK:
         raise RuntimeError("device error in timed region: " + bsq.status_str(st))
     if world > 1:
-        tt = torch.tensor([ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+        ms = max_over_ranks(ms, dist, dev)
 
     flops = 2.0 * M * N * K
-    value = world * flops / (ms * 1e-3) / 1e12
+    value = job_tflops(world, flops, ms)
 
     # ---- end to end through the C ABI with host buffers (pinned), copies timed
     A_pin = A_h.pin_memory()
@@ -297,9 +492,7 @@ def main():
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
     if world > 1:
-        tt = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
+        e2e_ms = max_over_ranks(e2e_ms, dist, dev)
 
     hbm, bf16, src = peaks()
     fp4_peak = bf16 * NOMINAL_FP4_OVER_BF16
@@ -311,6 +504,11 @@ def main():
     qw_bytes = N * K * (2 + 2 + 0.5 + 1 / 16)
     qa_gbs = qa_bytes / (statistics.mean(qa_ms) * 1e-3) / 1e9
     qw_gbs = qw_bytes / (statistics.mean(qw_ms) * 1e-3) / 1e9
+
+    rows = None
+    if rank == 0 and world == 1 and not args.no_rows:
+        del A_pin, W_pin, C_pin
+        rows = measure_rows(hbm, fp4_peak, bf16 * NOMINAL_FP8_OVER_BF16)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -344,12 +542,13 @@ def main():
                 "quant_W_ms": statistics.mean(qw_ms), "quant_W_gbs": qw_gbs,
                 "quant_frac_of_hbm": {"A": qa_gbs / hbm, "W": qw_gbs / hbm, "hbm_gbs": hbm, "source": src},
             },
-            "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "e2e": {"value": job_tflops(world, flops, e2e_ms), "unit": "TFLOP/s",
                     "h2d_bytes_per_step": (M + N) * K * 2, "d2h_bytes_per_step": M * N * 2,
                     "ms_per_step": e2e_ms},
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clk.summary(),
             "cpu_baseline": cpu,
+            "rows": rows,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -146,6 +146,27 @@ BSQ_DEV uint32_t e4m3_sr(float v, uint32_t r16) {
     return sgn | e4m3_rne(mag);
 }
 
+// Stochastic rounding of |v| <= 448 to E4M3 (same result as e4m3_sr).  In
+// the normal E4M3 range (|v| >= 2^-6) the neighbour below is v with its low
+// 20 mantissa bits cleared, the E4M3 spacing is bit 20, and frac = low20 /
+// 2^20 exactly, so "r16 / 2^16 < frac" is the integer test 16 r16 < low20
+// and rounding up adds 1 << 20 to the bits (a carry into the exponent is
+// the next binade, as the float addition would give).  The code is read off
+// the bits: ((bits >> 20) - (120 << 3)) is exponent - 127 + 7 and the three
+// mantissa bits.  Below 2^-6 the float path of e4m3_sr runs.
+BSQ_DEV uint32_t e4m3_sr_fast(float v, uint32_t r16) {
+    const uint32_t x = __float_as_uint(v);
+    const uint32_t sgn = (x >> 24) & 0x80u;
+    const uint32_t a = x & 0x7FFFFFFFu;
+    if (a >= 0x3C800000u) {  // 2^-6
+        const uint32_t low20 = a & 0xFFFFFu;
+        const uint32_t mag = (a & ~0xFFFFFu) + (((r16 << 4) < low20) ? 0x100000u : 0u);
+        return sgn | ((mag >> 20) - (120u << 3));
+    }
+    return e4m3_sr(v, r16);
+}
+
+
 // ---------------------------------------------------------------- fp32 pairs
 // sm_100 executes two fp32 operations per instruction on a 64-bit register
 // pair (add/sub/mul.rn.f32x2); each lane is an ordinary IEEE RN operation.

@@ -419,7 +419,7 @@ BSQ_DEV uint2 mx_encode8(const float v[8], bool zero_block, int E, uint64_t idx0
         uint4 r = philox4x32_10(make_uint4((uint32_t)g, (uint32_t)(g >> 32), stream_id, 0u), seed_lo, seed_hi);
         const uint32_t w[4] = {r.x, r.y, r.z, r.w};
 #pragma unroll
-        for (int i = 0; i < 8; i++) c[i] = e4m3_sr(s[i], (i & 1) ? (w[i >> 1] >> 16) : (w[i >> 1] & 0xFFFFu));
+        for (int i = 0; i < 8; i++) c[i] = e4m3_sr_fast(s[i], (i & 1) ? (w[i >> 1] >> 16) : (w[i >> 1] & 0xFFFFu));
     } else {
 #pragma unroll
         for (int i = 0; i < 8; i += 2) {
@@ -475,6 +475,53 @@ __global__ void __launch_bounds__(256) quant_mxfp8_row_kernel(
                         sb | (b1 << 8) | (b2 << 16) | (b3 << 24);
             } else if (valid && (lane & 3) == 0) {
                 sf[sf_offset(rr, kb, KB)] = (uint8_t)sb;
+            }
+        }
+    }
+}
+
+// Row-wise for a contiguous tensor whose rows hold a multiple of 128
+// elements: a flat sequence of 8-element chunks, two per thread in flight.
+// Lanes 4j..4j+3 hold one block of 32 (two-step shuffle max); lanes 16i hold
+// the first of four consecutive blocks of one row and store their scale
+// word.  The SR draw index of a chunk is its flat position (row * K + col).
+template <bool SR>
+__global__ void __launch_bounds__(256) quant_mxfp8_row_flat_kernel(
+    const uint16_t *__restrict__ x, int64_t nchunk, int64_t K, uint32_t seed_lo, uint32_t seed_hi,
+    uint32_t stream_id, uint8_t *__restrict__ codes, uint8_t *__restrict__ sf) {
+    const int64_t K8 = K >> 3, KB = K >> 5;
+    const int lane = threadIdx.x & 31;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    const int64_t nwarp = (nchunk + 31) & ~int64_t(31);
+    for (int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; c - lane < nwarp; c += 2 * stride) {
+        const int64_t c1 = c + stride;
+        const bool v0 = c < nchunk, v1 = c1 < nchunk;
+        float a[8], b[8];
+        load8_bf16(x + (v0 ? c : 0) * 8, a);
+        load8_bf16(x + (v1 ? c1 : 0) * 8, b);
+#pragma unroll
+        for (int h = 0; h < 2; h++) {
+            const int64_t cc = h ? c1 : c;
+            const bool valid = h ? v1 : v0;
+            if (h && !__any_sync(0xFFFFFFFFu, v1)) break;
+            const float *v = h ? b : a;
+            float m = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 8; i++) m = fmaxf(m, fabsf(v[i]));
+            m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+            m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+            const bool zero = (m == 0.0f);
+            const int E = zero ? 0 : mx_exponent(m);
+            const uint2 q = mx_encode8<SR>(v, zero, E, (uint64_t)cc * 8, seed_lo, seed_hi, stream_id);
+            if (valid) *reinterpret_cast<uint2 *>(codes + cc * 8) = q;
+            const uint32_t sb = zero ? 0u : (uint32_t)(E + 127);
+            const uint32_t b1 = __shfl_down_sync(0xFFFFFFFFu, sb, 4);
+            const uint32_t b2 = __shfl_down_sync(0xFFFFFFFFu, sb, 8);
+            const uint32_t b3 = __shfl_down_sync(0xFFFFFFFFu, sb, 12);
+            if (valid && (lane & 15) == 0) {
+                const int64_t row = cc / K8, kb = (cc - row * K8) >> 2;
+                *reinterpret_cast<uint32_t *>(sf + sf_word_offset(row, kb >> 2, KB)) =
+                    sb | (b1 << 8) | (b2 << 16) | (b3 << 24);
             }
         }
     }
@@ -724,6 +771,17 @@ void launch_quant_mxfp8(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, bo
                         uint64_t seed, uint32_t stream_id, uint8_t *codes, uint8_t *sf, int num_sms,
                         cudaStream_t s) {
     const uint32_t lo = (uint32_t)seed, hi = (uint32_t)(seed >> 32);
+    if (!colwise && ldx == K && K % 128 == 0) {
+        const int64_t nchunk = M * (K >> 3);
+        if (sr) {
+            const int grid = grid_for(nchunk, 2 * 256, resident_ctas<quant_mxfp8_row_flat_kernel<true>>(num_sms));
+            quant_mxfp8_row_flat_kernel<true><<<grid, 256, 0, s>>>(x, nchunk, K, lo, hi, stream_id, codes, sf);
+        } else {
+            const int grid = grid_for(nchunk, 2 * 256, resident_ctas<quant_mxfp8_row_flat_kernel<false>>(num_sms));
+            quant_mxfp8_row_flat_kernel<false><<<grid, 256, 0, s>>>(x, nchunk, K, lo, hi, stream_id, codes, sf);
+        }
+        return;
+    }
     if (!colwise) {
         RowMap map{lpr_shift_for(K >> 3)};
         if (map.lpr_shift < 2) map.lpr_shift = 2;  // 4 lanes per block of 32

@@ -396,6 +396,174 @@ __global__ void __launch_bounds__(256) quant_nvfp4_2d_kernel(
     }
 }
 
+// ===================================================================== fused NVFP4
+// One cooperative kernel per tensor (contiguous, no gather or groups):
+//   phase 1  amax over the tensor (four blocks per thread in flight);
+//   barrier  every CTA arrives on a grid counter and waits (bounded);
+//   phase 2  every CTA reads the amax, derives s_g and quantizes its blocks
+//            in the reverse of the phase-1 order, so the most recently read
+//            lines (an 8192x4096 bf16 tensor fits in L2 whole) come from L2.
+// The counter and the amax bits live in the first 8 bytes of the code
+// buffer (zeroed by the caller).  Those bytes are the first block's codes:
+// their writer -- the last block its thread handles -- first waits until
+// every CTA has arrived a second time, i.e. has read the amax.
+BSQ_DEV unsigned int ld_acquire_gpu(const unsigned int *p) {
+    unsigned int v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Thread 0 of the CTA waits (sleeping, bounded) until *ctr >= target.
+BSQ_DEV bool wait_counter(const unsigned int *ctr, unsigned int target, unsigned int *err, unsigned int site) {
+    const uint64_t t0 = globaltimer_ns();
+    while (ld_acquire_gpu(ctr) < target) {
+        __nanosleep(100);
+        if (globaltimer_ns() - t0 > 2000000000ull) {
+            report_timeout(err, site);
+            return false;
+        }
+    }
+    return true;
+}
+
+// All CTAs of a cooperative launch: arrive once, wait for every CTA.
+BSQ_DEV bool grid_barrier(unsigned int *ctr, unsigned int target, unsigned int *err, unsigned int site) {
+    __shared__ int ok_sh;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        atomicAdd(ctr, 1u);
+        ok_sh = wait_counter(ctr, target, err, site);
+        __threadfence();
+    }
+    __syncthreads();
+    return ok_sh != 0;
+}
+
+template <bool RHT, bool TWO_D>
+__global__ void __launch_bounds__(256) quant_nvfp4_fused_kernel(
+    const uint16_t *__restrict__ x, int64_t M, int64_t K, int kb_shift, uint32_t mask, unsigned int *scratch,
+    float *gs_out, uint8_t *__restrict__ codes, uint8_t *__restrict__ sf, unsigned int *err) {
+    __shared__ float den_tab[128], rcp_tab[128];
+    uint32_t sw[8];
+    rht_sign_words(mask, sw);
+    const int64_t KB = K >> 4, nblk = M * KB;
+    const int lane = threadIdx.x & 31;
+    const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    // ---- phase 1: amax
+    {
+        float m = 0.0f;
+        for (int64_t b = tid; b < nblk; b += 4 * stride) {
+            uint32_t w[4][8];
+#pragma unroll
+            for (int i = 0; i < 4; i++)
+                if (b + i * stride < nblk) load_words16(x + (b + i * stride) * 16, w[i]);
+#pragma unroll
+            for (int i = 0; i < 4; i++)
+                if (b + i * stride < nblk) m = fmaxf(m, block_absmax<RHT>(w[i], sw));
+        }
+#pragma unroll
+        for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+        __shared__ float red[8];
+        if (lane == 0) red[threadIdx.x >> 5] = m;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            float b = red[0];
+            for (int i = 1; i < 8; i++) b = fmaxf(b, red[i]);
+            atomicMax(scratch + 1, __float_as_uint(b));
+        }
+    }
+    if (!grid_barrier(scratch, gridDim.x, err, 20)) return;
+    const float amax = __uint_as_float(ld_acquire_gpu(scratch + 1));
+    __syncthreads();
+    if (threadIdx.x == 0) atomicAdd(scratch, 1u);  // this CTA has read the amax
+    const float s_g = global_scale_of(amax);
+    if (blockIdx.x == 0 && threadIdx.x == 0) *gs_out = s_g;
+    const NvScale c = nv_scale_setup(s_g, den_tab, rcp_tab);
+    const unsigned int all_read = 2u * gridDim.x;
+    if (!TWO_D) {
+        // ---- phase 2, 1x16 blocks, reverse order, two in flight
+        const int64_t wbase = tid - lane;
+        const int64_t nwarp_blk = (nblk + 31) & ~int64_t(31);
+        const int64_t iters = wbase < nwarp_blk ? (nwarp_blk - 1 - wbase) / stride + 1 : 0;
+        for (int64_t i = iters - 1; i >= 0; i -= 2) {
+            const int64_t b = tid + i * stride, b1 = b - stride;
+            const bool v0 = b < nblk, v1 = i >= 1 && b1 < nblk;
+            uint32_t w0[8], w1[8];
+            load_words16(x + (v0 ? b : 0) * 16, w0);
+            load_words16(x + (v1 ? b1 : 0) * 16, w1);
+#pragma unroll
+            for (int h = 0; h < 2; h++) {
+                if (h && !__any_sync(0xFFFFFFFFu, v1)) break;
+                const int64_t bb = h ? b1 : b;
+                const bool v = h ? v1 : v0;
+                uint32_t sb;
+                uint2 cd;
+                nv_block_1d<RHT, false>(h ? w1 : w0, sw, c, den_tab, rcp_tab, sb, cd);
+                if (v && bb == 0 && !wait_counter(scratch, all_read, err, 21)) cd = make_uint2(0u, 0u);
+                if (v) *reinterpret_cast<uint2 *>(codes + bb * 8) = cd;
+                store_sf(sf, v, sb, bb >> kb_shift, bb & (KB - 1), KB, true);
+            }
+        }
+    } else {
+        // ---- phase 2, 16x16 tiles (warp = 16 rows x 8 blocks), reverse task order
+        const int64_t k8 = (KB + 7) >> 3;
+        const int64_t tasks = (M >> 4) * k8;
+        const bool pack4 = (KB & 3) == 0;
+        const int r16 = lane & 15, hw = lane >> 4;
+        const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+        const int64_t wid = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+        const int64_t ntask = wid < tasks ? (tasks - 1 - wid) / warps + 1 : 0;
+        for (int64_t j = ntask - 1; j >= 0; j--) {
+            const int64_t task = wid + j * warps;
+            const int64_t rt = task / k8, g8 = task - rt * k8;
+            const int64_t row = rt * 16 + r16;
+            const int64_t kb0 = g8 * 8 + 4 * hw;
+            const uint16_t *rp = x + row * K;
+            uint32_t w[4][8];
+#pragma unroll
+            for (int i = 0; i < 4; i++) load_words16(rp + (kb0 + i < KB ? kb0 + i : 0) * 16, w[i]);
+            uint32_t sbw = 0;
+            uint2 cd[4];
+#pragma unroll
+            for (int i = 0; i < 4; i++) {
+                const bool v = kb0 + i < KB;
+                f32x2 P[8];
+                if (RHT) rht16_u_words(w[i], sw, P);
+                else words_to_pairs(w[i], P);
+                float mu = v ? pairs_absmax3(P) : 0.0f;
+#pragma unroll
+                for (int o = 1; o < 16; o <<= 1) mu = fmaxf(mu, __shfl_xor_sync(0xFFFFFFFFu, mu, o));
+                const float tmax = RHT ? __fmul_rn(mu, 0.25f) : mu;
+                const uint32_t sbb = nv_scale_code(tmax, 6.0f, c.c6, c);
+                sbw |= (sbb & 0xFFu) << (8 * i);
+                cd[i] = sbb ? nv_codes<RHT>(P, rcp_tab[sbb], c.fast) : make_uint2(0u, 0u);
+            }
+            if (task == 0) {  // holds the first block's codes: every CTA has read the amax
+                if (lane == 0 && !wait_counter(scratch, all_read, err, 22)) cd[0] = make_uint2(0u, 0u);
+                __syncwarp();
+            }
+            uint8_t *cp = codes + row * (K >> 1) + kb0 * 8;
+            if (kb0 + 3 < KB && ((K >> 1) & 15) == 0) {
+                reinterpret_cast<uint4 *>(cp)[0] = make_uint4(cd[0].x, cd[0].y, cd[1].x, cd[1].y);
+                reinterpret_cast<uint4 *>(cp)[1] = make_uint4(cd[2].x, cd[2].y, cd[3].x, cd[3].y);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 4; i++)
+                    if (kb0 + i < KB) reinterpret_cast<uint2 *>(cp)[i] = cd[i];
+            }
+            if (pack4) {
+                if (kb0 < KB) *reinterpret_cast<uint32_t *>(sf + sf_word_offset(row, kb0 >> 2, KB)) = sbw;
+            } else {
+#pragma unroll
+                for (int i = 0; i < 4; i++)
+                    if (kb0 + i < KB) sf[sf_offset(row, kb0 + i, KB)] = (uint8_t)(sbw >> (8 * i));
+            }
+        }
+    }
+}
+
 // ===================================================================== MXFP8
 // E8M0 exponent of a block: clamp(floor(log2 amax) - 8, -127, 127).
 BSQ_DEV int mx_exponent(float bamax) {
@@ -765,6 +933,29 @@ void launch_quant_nvfp4(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, bo
     else { if (fos) BSQ_NV1_G(false, true); else BSQ_NV1_G(false, false); }
 #undef BSQ_NV1_G
 #undef BSQ_NV1
+}
+
+int launch_quant_nvfp4_fused(const uint16_t *x, int64_t M, int64_t K, bool block_2d, bool rht, uint32_t mask,
+                             float *gs_out, uint8_t *codes, uint8_t *sf, unsigned int *err, int num_sms,
+                             cudaStream_t s) {
+    const int64_t KB = K >> 4;
+    int kb_shift = 0;
+    while ((int64_t(1) << kb_shift) < KB) kb_shift++;
+    unsigned int *scratch = reinterpret_cast<unsigned int *>(codes);
+    void *args[] = {(void *)&x, (void *)&M, (void *)&K, (void *)&kb_shift, (void *)&mask, (void *)&scratch,
+                    (void *)&gs_out, (void *)&codes, (void *)&sf, (void *)&err};
+    const void *kern;
+    int resident;
+    if (block_2d) {
+        if (rht) { kern = (const void *)quant_nvfp4_fused_kernel<true, true>; resident = resident_ctas<quant_nvfp4_fused_kernel<true, true>>(num_sms); }
+        else { kern = (const void *)quant_nvfp4_fused_kernel<false, true>; resident = resident_ctas<quant_nvfp4_fused_kernel<false, true>>(num_sms); }
+    } else {
+        if (rht) { kern = (const void *)quant_nvfp4_fused_kernel<true, false>; resident = resident_ctas<quant_nvfp4_fused_kernel<true, false>>(num_sms); }
+        else { kern = (const void *)quant_nvfp4_fused_kernel<false, false>; resident = resident_ctas<quant_nvfp4_fused_kernel<false, false>>(num_sms); }
+    }
+    // one resident wave, no more CTAs than 256-block groups of work
+    const int grid = grid_for(M * KB, 256, resident);
+    return cudaLaunchCooperativeKernel(kern, dim3(grid), dim3(256), args, 0, s) == cudaSuccess ? 0 : 1;
 }
 
 void launch_quant_mxfp8(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, bool colwise, bool sr,

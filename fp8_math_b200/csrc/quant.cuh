@@ -16,6 +16,12 @@ void launch_quant_nvfp4(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, bo
                         bool rht, uint32_t mask, const int32_t *row_index, int G, const int32_t *row_off,
                         const int32_t *sf_off, const float *scale_src, bool src_is_amax, float *gs_out,
                         bool write_gs, uint8_t *codes, uint8_t *sf, int num_sms, cudaStream_t s);
+// amax + NVFP4 quantize of a contiguous tensor in one cooperative kernel
+// (1x16 blocks need a power-of-two block count per row).  The first 8 bytes
+// of codes must be zero on entry.  Returns non-zero if the launch failed.
+int launch_quant_nvfp4_fused(const uint16_t *x, int64_t M, int64_t K, bool block_2d, bool rht, uint32_t mask,
+                             float *gs_out, uint8_t *codes, uint8_t *sf, unsigned int *err, int num_sms,
+                             cudaStream_t s);
 void launch_quant_mxfp8(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, bool colwise, bool sr,
                         uint64_t seed, uint32_t stream_id, uint8_t *codes, uint8_t *sf, int num_sms,
                         cudaStream_t s);

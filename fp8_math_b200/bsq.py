@@ -32,6 +32,7 @@ _SIGS = {
     "bsq_sf_bytes": (C.c_size_t, [_i64, _i64]),
     "bsq_rht_sign_mask": (C.c_uint16, [C.c_uint64]),
     "bsq_amax": (C.c_int, [_vp, _i64, _i64, _i64, C.c_int, C.c_uint16, _vp, _vp, _vp]),
+    "bsq_global_scale_noalloc": (C.c_int, [_vp, _i64, _i64, _i64, C.c_int, C.c_uint16, _vp, _vp]),
     "bsq_quant_nvfp4": (C.c_int, [_vp, _i64, _i64, _i64, C.c_int, C.c_int, C.c_int, C.c_uint16, _vp,
                                   C.c_int, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "bsq_quant_mxfp8": (C.c_int, [_vp, _i64, _i64, _i64, C.c_int, C.c_int, C.c_uint64, C.c_uint32,
@@ -106,6 +107,11 @@ def bsq_rht_sign_mask(seed: int) -> int:
 def bsq_amax(x, M, K, ldx, rht_enable, rht_sign_mask, row_index, amax_out, stream=None):
     return _check("bsq_amax", lib().bsq_amax(_p(x), M, K, ldx, int(rht_enable), rht_sign_mask, _p(row_index),
                                              _p(amax_out), _stream(stream)))
+
+
+def bsq_global_scale_noalloc(x, M, K, ldx, rht_enable, rht_sign_mask, gs_out, stream=None):
+    return _check("bsq_global_scale_noalloc", lib().bsq_global_scale_noalloc(
+        _p(x), M, K, ldx, int(rht_enable), rht_sign_mask, _p(gs_out), _stream(stream)))
 
 
 def bsq_quant_nvfp4(x, M, K, ldx, block_2d, four_over_six, rht_enable, rht_sign_mask, row_index, G, row_offsets,

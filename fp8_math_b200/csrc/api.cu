@@ -263,6 +263,53 @@ int bsq_check(void *stream) {
     return BSQ_OK;
 }
 
+// ------------------------------------------------------------ no-alloc global scale
+// Scratch of bsq_global_scale_noalloc: a file-scope device array (one per
+// device, resolved with cudaGetSymbolAddress) instead of any allocation.
+}  // extern "C"
+
+namespace {
+constexpr int kNoAllocScratchWords = 64;
+__device__ __align__(256) unsigned int g_noalloc_scratch[kNoAllocScratchWords];
+std::mutex g_noalloc_mu;
+unsigned int *g_noalloc_ptr[kMaxDevices];
+}  // namespace
+
+extern "C" {
+
+int bsq_global_scale_noalloc(const void *x, int64_t M, int64_t K, int64_t ldx, int rht_enable, uint16_t mask,
+                             float *gs_dev, void *stream) {
+    if (!x || !gs_dev || M < 0 || K < 0 || K % 16 || ldx < K) return BSQ_ERR_INVALID;
+    if (!aligned16(x) || ldx % 8 || (reinterpret_cast<uintptr_t>(gs_dev) & 3u)) return BSQ_ERR_ALIGN;
+    // the amax pass needs a CTA counter and the amax bits
+    constexpr size_t need = 2 * sizeof(unsigned int);
+    if (need > sizeof(g_noalloc_scratch)) return BSQ_ERR_UNSUPPORTED;  // never allocate more
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return BSQ_ERR_CUDA;
+    unsigned int *scratch;
+    {
+        std::lock_guard<std::mutex> lk(g_noalloc_mu);
+        if (!g_noalloc_ptr[dev]) {
+            void *ptr = nullptr;
+            if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess) return BSQ_ERR_CUDA;
+            g_noalloc_ptr[dev] = static_cast<unsigned int *>(ptr);
+        }
+        scratch = g_noalloc_ptr[dev];
+    }
+    int num_sms = 0;
+    if (cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return BSQ_ERR_CUDA;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (M == 0 || K == 0) {
+        if (cudaMemsetAsync(gs_dev, 0, sizeof(float), s) != cudaSuccess) return BSQ_ERR_CUDA;
+        bsq::launch_finalize_global_scale(gs_dev, s);  // amax 0 gives s_g = 1
+        return launch_status();
+    }
+    if (cudaMemsetAsync(scratch, 0, need, s) != cudaSuccess) return BSQ_ERR_CUDA;
+    bsq::launch_amax(static_cast<const uint16_t *>(x), M, K, ldx, rht_enable != 0, mask, nullptr, scratch + 1, scratch,
+                     gs_dev, num_sms, s);
+    return launch_status();
+}
+
 int bsq_debug_timeout_probe(uint64_t timeout_ns, void *stream) {
     if (timeout_ns == 0 || timeout_ns > 10000000000ull) return BSQ_ERR_INVALID;
     DeviceState *d;

@@ -85,13 +85,28 @@ BSQ_API int bsq_amax(const void *x_bf16, int64_t M, int64_t K, int64_t ldx,
              int rht_enable, uint16_t rht_sign_mask, const int32_t *row_index_dev,
              float *amax_dev, void *stream);
 
+/* NVFP4 global scale without any device allocation: *gs_dev = s_g =
+ * amax / 2688 (amax = 0 gives 1) of the M x K bf16 matrix x, after the
+ * 16-point RHT along K when rht_enable != 0 -- the value bsq_quant_nvfp4
+ * writes to *global_scale_dev ("Microscaling ...", section "NVFP4").
+ * Its scratch (a CTA counter and the amax bits, 8 bytes) is a file-scope
+ * device array of the library, found with cudaGetSymbolAddress per device;
+ * the call never allocates device memory (it does not create the error word
+ * the other calls use), and a request needing more scratch than the array
+ * holds is rejected with BSQ_ERR_UNSUPPORTED.  The scratch is per device:
+ * calls on one device must be ordered (one stream, or synchronized).
+ * K % 16 == 0; x 16-byte aligned, ldx % 8 == 0; gs_dev 4-byte aligned. */
+BSQ_API int bsq_global_scale_noalloc(const void *x_bf16, int64_t M, int64_t K, int64_t ldx, int rht_enable,
+                                     uint16_t rht_sign_mask, float *gs_dev, void *stream);
+
 /* NVFP4 quantize ("Microscaling ...", section "NVFP4"; "Thinking Machines
  * ... Inkling 2 Small", section "A precision choice for each stage" for Four
  * Over Six).  Output row i is input row row_index[i] (or i when row_index is
  * NULL); with rht_enable the 16-point RHT along K is applied first (fp32).
  *   s_g = amax / 2688 (amax = 0 gives s_g = 1); amax is *amax_in_dev, or is
- *         computed here when amax_in_dev is NULL (the amax is then
- *         accumulated in *global_scale_dev, which finally holds s_g);
+ *         computed here when amax_in_dev is NULL (an amax pass that uses
+ *         the first 8 bytes of codes as its scratch before the quantize
+ *         pass overwrites them);
  *   per block (1x16 along K, or a 16x16 tile with block_2d):
  *         s_b = E4M3_RNE((block_amax / 6) / s_g), r = 1 / (s_b * s_g),
  *         code = E2M1_RNE_sat(x * r); s_b == 0 gives all-zero codes;

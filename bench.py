@@ -209,6 +209,10 @@ def measure_rows(hbm, fp4_peak, fp8_peak, reps=10, only=None):
 
     rows = []
 
+    def wants(*names):
+        """Whether any of these rows is selected (inputs are built only then)."""
+        return only is None or any(only in n for n in names)
+
     def row(name, workload, fn, nbytes=None, flops=None, peak_kind=None):
         if only and only not in name:
             return
@@ -230,120 +234,125 @@ def measure_rows(hbm, fp4_peak, fp8_peak, reps=10, only=None):
         except Exception as e:  # noqa: BLE001 -- recorded, not fatal
             rows.append({"row": name, "workload": workload, "error": str(e)[:200]})
 
-    # -- configs[2]: linear with RHT (the timed step's calls, one at a time)
-    A_h, W_h, seed = W.nvfp4_linear_rht()
-    mask = bsq.bsq_rht_sign_mask(seed)
-    A, Wd = A_h.to(dev), W_h.to(dev)
-    M2, K2 = A.shape
-    N2 = Wd.shape[0]
-    am = torch.empty(1, device=dev)
-    row("a1 amax (RHT)", "A 8192x4096 bf16", lambda: bsq.bsq_amax(A, M2, K2, K2, 1, mask, None, am),
-        nbytes=M2 * K2 * 2)
-    qa = api.quant_nvfp4(A, rht_mask=mask)
-    row("a2+a5 NVFP4 1x16 quantize (amax + RHT fused)", "A 8192x4096",
-        lambda: api.quant_nvfp4(A, rht_mask=mask, out=qa), nbytes=M2 * K2 * (2 + 2 + 0.5 + 1 / 16))
-    qw = api.quant_nvfp4(Wd, block_2d=True, rht_mask=mask)
-    row("a3+a5 NVFP4 16x16 quantize (amax + RHT fused)", "W 14336x4096",
-        lambda: api.quant_nvfp4(Wd, block_2d=True, rht_mask=mask, out=qw), nbytes=N2 * K2 * (2 + 2 + 0.5 + 1 / 16))
-    y = torch.empty_like(A)
-    row("a5 RHT standalone (bf16 -> bf16)", "A 8192x4096", lambda: api.rht(A, mask, out=y), nbytes=M2 * K2 * 4)
-    C2 = torch.empty(M2, N2, dtype=torch.bfloat16, device=dev)
-    row("a8 NVFP4 GEMM bf16", "8192x14336x4096",
-        lambda: api.gemm(0, qa[0], qa[1], qw[0], qw[1], M2, N2, K2, gsA=qa[2], gsB=qw[2], out=C2),
-        flops=2 * M2 * N2 * K2, peak_kind="fp4")
-    del y, C2
-    # -- configs[0]: the small NVFP4 linear (latency)
-    As, Ws = W.nvfp4_linear_small()
-    As, Ws = As.to(dev), Ws.to(dev)
-    qas, qws = api.quant_nvfp4(As), api.quant_nvfp4(Ws, block_2d=True)
-    Cs = torch.empty(128, 256, dtype=torch.float32, device=dev)
+    if wants("a1 amax (RHT)", "a2+a5 NVFP4 1x16 quantize (amax + RHT fused)", "a3+a5 NVFP4 16x16 quantize (amax + RHT fused)", "a5 RHT standalone (bf16 -> bf16)", "a8 NVFP4 GEMM bf16"):
+        # -- configs[2]: linear with RHT (the timed step's calls, one at a time)
+        A_h, W_h, seed = W.nvfp4_linear_rht()
+        mask = bsq.bsq_rht_sign_mask(seed)
+        A, Wd = A_h.to(dev), W_h.to(dev)
+        M2, K2 = A.shape
+        N2 = Wd.shape[0]
+        am = torch.empty(1, device=dev)
+        row("a1 amax (RHT)", "A 8192x4096 bf16", lambda: bsq.bsq_amax(A, M2, K2, K2, 1, mask, None, am),
+            nbytes=M2 * K2 * 2)
+        qa = api.quant_nvfp4(A, rht_mask=mask)
+        row("a2+a5 NVFP4 1x16 quantize (amax + RHT fused)", "A 8192x4096",
+            lambda: api.quant_nvfp4(A, rht_mask=mask, out=qa), nbytes=M2 * K2 * (2 + 2 + 0.5 + 1 / 16))
+        qw = api.quant_nvfp4(Wd, block_2d=True, rht_mask=mask)
+        row("a3+a5 NVFP4 16x16 quantize (amax + RHT fused)", "W 14336x4096",
+            lambda: api.quant_nvfp4(Wd, block_2d=True, rht_mask=mask, out=qw), nbytes=N2 * K2 * (2 + 2 + 0.5 + 1 / 16))
+        y = torch.empty_like(A)
+        row("a5 RHT standalone (bf16 -> bf16)", "A 8192x4096", lambda: api.rht(A, mask, out=y), nbytes=M2 * K2 * 4)
+        C2 = torch.empty(M2, N2, dtype=torch.bfloat16, device=dev)
+        row("a8 NVFP4 GEMM bf16", "8192x14336x4096",
+            lambda: api.gemm(0, qa[0], qa[1], qw[0], qw[1], M2, N2, K2, gsA=qa[2], gsB=qw[2], out=C2),
+            flops=2 * M2 * N2 * K2, peak_kind="fp4")
+        del y, C2
+    if wants("a2+a3+a8 small linear step (latency)"):
+        # -- configs[0]: the small NVFP4 linear (latency)
+        As, Ws = W.nvfp4_linear_small()
+        As, Ws = As.to(dev), Ws.to(dev)
+        qas, qws = api.quant_nvfp4(As), api.quant_nvfp4(Ws, block_2d=True)
+        Cs = torch.empty(128, 256, dtype=torch.float32, device=dev)
 
-    def small_step():
-        api.quant_nvfp4(As, out=qas)
-        api.quant_nvfp4(Ws, block_2d=True, out=qws)
-        api.gemm(0, qas[0], qas[1], qws[0], qws[1], 128, 256, 256, gsA=qas[2], gsB=qws[2], out=Cs)
-    row("a2+a3+a8 small linear step (latency)", "A 128x256, W 256x256, fp32 out", small_step,
-        nbytes=(128 + 256) * 256 * 2)
-    # -- configs[1]: MXFP8 4096^2 Student-t, RNE and SR, requant-transpose
-    X1 = W.mxfp8_requant().to(dev)
-    M1, K1 = X1.shape
-    q1 = api.quant_mxfp8(X1)
-    row("a6 MXFP8 row quantize RNE", "X 4096x4096", lambda: api.quant_mxfp8(X1, out=q1),
-        nbytes=M1 * K1 * (2 + 1 + 1 / 32))
-    q1s = api.quant_mxfp8(X1, sr=True, seed=1)
-    row("a6 MXFP8 row quantize SR (Philox)", "X 4096x4096", lambda: api.quant_mxfp8(X1, sr=True, seed=1, out=q1s),
-        nbytes=M1 * K1 * (2 + 1 + 1 / 32))
-    qt = api.requant_transpose(q1s[0], q1s[1], sr=True, seed=1)
-    row("a7 requant-transpose SR", "4096x4096 MXFP8 -> column-wise",
-        lambda: api.requant_transpose(q1s[0], q1s[1], sr=True, seed=1, out=qt), nbytes=2 * M1 * K1 * (1 + 1 / 32))
-    del X1, q1, q1s, qt
-    # -- configs[4]: MXFP8 backward + rollout
-    dY, W4, X4, A_roll = W.mxfp8_backward()
-    dY, W4, X4 = dY.to(dev), W4.to(dev), X4.to(dev)
-    M4, N4 = dY.shape
-    K4 = W4.shape[1]
-    qdr = api.quant_mxfp8(dY, sr=True, seed=4, stream_id=0)
-    row("a6 MXFP8 row quantize SR", "dY 8192x14336", lambda: api.quant_mxfp8(dY, sr=True, seed=4, out=qdr),
-        nbytes=M4 * N4 * (2 + 1 + 1 / 32))
-    qdc = api.quant_mxfp8(dY, colwise=True, sr=True, seed=4, stream_id=1)
-    row("a6 MXFP8 column quantize SR", "dY 8192x14336 -> [14336, 8192]",
-        lambda: api.quant_mxfp8(dY, colwise=True, sr=True, seed=4, stream_id=1, out=qdc),
-        nbytes=M4 * N4 * (2 + 1 + 1 / 32))
-    qwc = api.quant_mxfp8(W4, colwise=True, sr=True, seed=4, stream_id=2)
-    qxc = api.quant_mxfp8(X4, colwise=True, sr=True, seed=4, stream_id=3)
-    Cd = torch.empty(M4, K4, dtype=torch.bfloat16, device=dev)
-    row("a8 MXFP8 GEMM dgrad (bf16 out)", "8192x4096x14336",
-        lambda: api.gemm(1, qdr[0], qdr[1], qwc[0], qwc[1], M4, K4, N4, out=Cd), flops=2 * M4 * K4 * N4,
-        peak_kind="fp8")
-    del Cd
-    Cw = torch.empty(N4, K4, dtype=torch.float32, device=dev)
-    row("a8 MXFP8 GEMM wgrad (fp32 out)", "14336x4096x8192",
-        lambda: api.gemm(1, qdc[0], qdc[1], qxc[0], qxc[1], N4, K4, M4, out=Cw), flops=2 * N4 * K4 * M4,
-        peak_kind="fp8")
-    del Cw, qdr, qdc, qxc, dY, X4
-    qar = api.quant_nvfp4(A_roll.to(dev))
-    qwr = api.quant_nvfp4(W4, block_2d=True)
-    Cr = torch.empty(64, N4, dtype=torch.bfloat16, device=dev)
-    row("a8 NVFP4 rollout GEMM (swap-AB, HBM-bound)", "64x14336x4096",
-        lambda: api.gemm(0, qar[0], qar[1], qwr[0], qwr[1], 64, N4, K4, gsA=qar[2], gsB=qwr[2], out=Cr),
-        nbytes=N4 * K4 // 2 + N4 * K4 // 16 + 64 * K4 // 2 + 64 * K4 // 16 + 64 * N4 * 2)
-    del Cr, qar, qwr, W4, qwc
-    # -- configs[3]: MoE forward (gathered 4/6 quantize, grouped up and down)
-    moe = W.moe_forward()
-    T3, H3 = moe.X.shape
-    E3, F3, _ = moe.W_up.shape
-    ri = torch.from_numpy(moe.row_index).to(dev)
-    offs = torch.from_numpy(moe.row_offsets).to(dev)
-    sfo = torch.from_numpy(moe.sf_row_offsets).to(dev)
-    Mt, sf_rows = int(moe.row_offsets[-1]), int(moe.sf_row_offsets[-1])
-    Xd = moe.X.to(dev)
-    qx = api.quant_nvfp4(Xd, four_over_six=True, row_index=ri, groups=(offs, sfo, sf_rows))
-    row("a4 NVFP4 Four Over Six quantize (gathered, expert groups)", "X 16384x4096 -> 131072 routed rows",
-        lambda: api.quant_nvfp4(Xd, four_over_six=True, row_index=ri, groups=(offs, sfo, sf_rows), out=qx),
-        nbytes=Mt * H3 * (2 + 2 + 0.5 + 1 / 16))
+        def small_step():
+            api.quant_nvfp4(As, out=qas)
+            api.quant_nvfp4(Ws, block_2d=True, out=qws)
+            api.gemm(0, qas[0], qas[1], qws[0], qws[1], 128, 256, 256, gsA=qas[2], gsB=qws[2], out=Cs)
+        row("a2+a3+a8 small linear step (latency)", "A 128x256, W 256x256, fp32 out", small_step,
+            nbytes=(128 + 256) * 256 * 2)
+    if wants("a6 MXFP8 row quantize RNE", "a6 MXFP8 row quantize SR (Philox)", "a7 requant-transpose SR"):
+        # -- configs[1]: MXFP8 4096^2 Student-t, RNE and SR, requant-transpose
+        X1 = W.mxfp8_requant().to(dev)
+        M1, K1 = X1.shape
+        q1 = api.quant_mxfp8(X1)
+        row("a6 MXFP8 row quantize RNE", "X 4096x4096", lambda: api.quant_mxfp8(X1, out=q1),
+            nbytes=M1 * K1 * (2 + 1 + 1 / 32))
+        q1s = api.quant_mxfp8(X1, sr=True, seed=1)
+        row("a6 MXFP8 row quantize SR (Philox)", "X 4096x4096", lambda: api.quant_mxfp8(X1, sr=True, seed=1, out=q1s),
+            nbytes=M1 * K1 * (2 + 1 + 1 / 32))
+        qt = api.requant_transpose(q1s[0], q1s[1], sr=True, seed=1)
+        row("a7 requant-transpose SR", "4096x4096 MXFP8 -> column-wise",
+            lambda: api.requant_transpose(q1s[0], q1s[1], sr=True, seed=1, out=qt), nbytes=2 * M1 * K1 * (1 + 1 / 32))
+        del X1, q1, q1s, qt
+    if wants("a6 MXFP8 row quantize SR", "a6 MXFP8 column quantize SR", "a8 MXFP8 GEMM dgrad (bf16 out)", "a8 MXFP8 GEMM wgrad (fp32 out)", "a8 NVFP4 rollout GEMM (swap-AB, HBM-bound)"):
+        # -- configs[4]: MXFP8 backward + rollout
+        dY, W4, X4, A_roll = W.mxfp8_backward()
+        dY, W4, X4 = dY.to(dev), W4.to(dev), X4.to(dev)
+        M4, N4 = dY.shape
+        K4 = W4.shape[1]
+        qdr = api.quant_mxfp8(dY, sr=True, seed=4, stream_id=0)
+        row("a6 MXFP8 row quantize SR", "dY 8192x14336", lambda: api.quant_mxfp8(dY, sr=True, seed=4, out=qdr),
+            nbytes=M4 * N4 * (2 + 1 + 1 / 32))
+        qdc = api.quant_mxfp8(dY, colwise=True, sr=True, seed=4, stream_id=1)
+        row("a6 MXFP8 column quantize SR", "dY 8192x14336 -> [14336, 8192]",
+            lambda: api.quant_mxfp8(dY, colwise=True, sr=True, seed=4, stream_id=1, out=qdc),
+            nbytes=M4 * N4 * (2 + 1 + 1 / 32))
+        qwc = api.quant_mxfp8(W4, colwise=True, sr=True, seed=4, stream_id=2)
+        qxc = api.quant_mxfp8(X4, colwise=True, sr=True, seed=4, stream_id=3)
+        Cd = torch.empty(M4, K4, dtype=torch.bfloat16, device=dev)
+        row("a8 MXFP8 GEMM dgrad (bf16 out)", "8192x4096x14336",
+            lambda: api.gemm(1, qdr[0], qdr[1], qwc[0], qwc[1], M4, K4, N4, out=Cd), flops=2 * M4 * K4 * N4,
+            peak_kind="fp8")
+        del Cd
+        Cw = torch.empty(N4, K4, dtype=torch.float32, device=dev)
+        row("a8 MXFP8 GEMM wgrad (fp32 out)", "14336x4096x8192",
+            lambda: api.gemm(1, qdc[0], qdc[1], qxc[0], qxc[1], N4, K4, M4, out=Cw), flops=2 * N4 * K4 * M4,
+            peak_kind="fp8")
+        del Cw, qdr, qdc, qxc, dY, X4
+        qar = api.quant_nvfp4(A_roll.to(dev))
+        qwr = api.quant_nvfp4(W4, block_2d=True)
+        Cr = torch.empty(64, N4, dtype=torch.bfloat16, device=dev)
+        row("a8 NVFP4 rollout GEMM (swap-AB, HBM-bound)", "64x14336x4096",
+            lambda: api.gemm(0, qar[0], qar[1], qwr[0], qwr[1], 64, N4, K4, gsA=qar[2], gsB=qwr[2], out=Cr),
+            nbytes=N4 * K4 // 2 + N4 * K4 // 16 + 64 * K4 // 2 + 64 * K4 // 16 + 64 * N4 * 2)
+        del Cr, qar, qwr, W4, qwc
+    if wants("a4 NVFP4 Four Over Six quantize (gathered, expert groups)", "a9 grouped NVFP4 GEMM up", "a9 grouped NVFP4 GEMM down"):
+        # -- configs[3]: MoE forward (gathered 4/6 quantize, grouped up and down)
+        moe = W.moe_forward()
+        T3, H3 = moe.X.shape
+        E3, F3, _ = moe.W_up.shape
+        ri = torch.from_numpy(moe.row_index).to(dev)
+        offs = torch.from_numpy(moe.row_offsets).to(dev)
+        sfo = torch.from_numpy(moe.sf_row_offsets).to(dev)
+        Mt, sf_rows = int(moe.row_offsets[-1]), int(moe.sf_row_offsets[-1])
+        Xd = moe.X.to(dev)
+        qx = api.quant_nvfp4(Xd, four_over_six=True, row_index=ri, groups=(offs, sfo, sf_rows))
+        row("a4 NVFP4 Four Over Six quantize (gathered, expert groups)", "X 16384x4096 -> 131072 routed rows",
+            lambda: api.quant_nvfp4(Xd, four_over_six=True, row_index=ri, groups=(offs, sfo, sf_rows), out=qx),
+            nbytes=Mt * H3 * (2 + 2 + 0.5 + 1 / 16))
 
-    def experts(Wx):
-        E, N, K = Wx.shape
-        codes = torch.empty(E, N, K // 2, dtype=torch.uint8, device=dev)
-        sfb = torch.zeros(E * bsq.bsq_sf_bytes(N, K // 16), dtype=torch.uint8, device=dev)
-        gsb = torch.empty(E, dtype=torch.float32, device=dev)
-        per = bsq.bsq_sf_bytes(N, K // 16)
-        for e in range(E):
-            we = Wx[e].to(dev)
-            api.quant_nvfp4(we, block_2d=True, out=(codes[e], sfb[e * per:(e + 1) * per], gsb[e:e + 1]))
-        return codes, sfb, gsb
-    up = experts(moe.W_up)
-    Cup = torch.empty(Mt, F3, dtype=torch.bfloat16, device=dev)
-    row("a9 grouped NVFP4 GEMM up", f"{Mt} routed rows x {F3} x {H3}, 64 experts",
-        lambda: api.grouped_gemm(0, offs, sfo, qx[0], qx[1], up[0], up[1], Mt, F3, H3, gsA=qx[2], gsB=up[2],
-                                 out=Cup), flops=2 * Mt * F3 * H3, peak_kind="fp4")
-    qh = api.quant_nvfp4(Cup, four_over_six=True, groups=(offs, sfo, sf_rows))
-    del up
-    dn = experts(moe.W_dn)
-    Cdn = torch.empty(Mt, H3, dtype=torch.bfloat16, device=dev)
-    row("a9 grouped NVFP4 GEMM down", f"{Mt} routed rows x {H3} x {F3}, 64 experts",
-        lambda: api.grouped_gemm(0, offs, sfo, qh[0], qh[1], dn[0], dn[1], Mt, H3, F3, gsA=qh[2], gsB=dn[2],
-                                 out=Cdn), flops=2 * Mt * H3 * F3, peak_kind="fp4")
+        def experts(Wx):
+            E, N, K = Wx.shape
+            codes = torch.empty(E, N, K // 2, dtype=torch.uint8, device=dev)
+            sfb = torch.zeros(E * bsq.bsq_sf_bytes(N, K // 16), dtype=torch.uint8, device=dev)
+            gsb = torch.empty(E, dtype=torch.float32, device=dev)
+            per = bsq.bsq_sf_bytes(N, K // 16)
+            for e in range(E):
+                we = Wx[e].to(dev)
+                api.quant_nvfp4(we, block_2d=True, out=(codes[e], sfb[e * per:(e + 1) * per], gsb[e:e + 1]))
+            return codes, sfb, gsb
+        up = experts(moe.W_up)
+        Cup = torch.empty(Mt, F3, dtype=torch.bfloat16, device=dev)
+        row("a9 grouped NVFP4 GEMM up", f"{Mt} routed rows x {F3} x {H3}, 64 experts",
+            lambda: api.grouped_gemm(0, offs, sfo, qx[0], qx[1], up[0], up[1], Mt, F3, H3, gsA=qx[2], gsB=up[2],
+                                     out=Cup), flops=2 * Mt * F3 * H3, peak_kind="fp4")
+        qh = api.quant_nvfp4(Cup, four_over_six=True, groups=(offs, sfo, sf_rows))
+        del up
+        dn = experts(moe.W_dn)
+        Cdn = torch.empty(Mt, H3, dtype=torch.bfloat16, device=dev)
+        row("a9 grouped NVFP4 GEMM down", f"{Mt} routed rows x {H3} x {F3}, 64 experts",
+            lambda: api.grouped_gemm(0, offs, sfo, qh[0], qh[1], dn[0], dn[1], Mt, H3, F3, gsA=qh[2], gsB=dn[2],
+                                     out=Cdn), flops=2 * Mt * H3 * F3, peak_kind="fp4")
     del flush
     return rows
 

@@ -92,6 +92,29 @@ BSQ_DEV uint32_t cvt_e2m1x8(const float q[8]) {
 }
 
 // E2M1 nibble -> fp32 from the S E E M layout (bias 1; E = 0 is M * 0.5).
+// Eight E2M1 codes (packed as by cvt_e2m1x8: element 2i in the low nibble of
+// byte i) -> fp32, exactly, through cvt.rn.f16x2.e2m1x2 (every E2M1 value is
+// an f16 and an fp32 value; -0 stays -0).
+BSQ_DEV void e2m1x8_to_f32(uint32_t w, float v[8]) {
+    uint32_t h[4];
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+        : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3])
+        : "r"(w));
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+        __half_raw lo, hi;
+        lo.x = (unsigned short)(h[i] & 0xFFFFu);
+        hi.x = (unsigned short)(h[i] >> 16);
+        v[2 * i] = __half2float(__half(lo));
+        v[2 * i + 1] = __half2float(__half(hi));
+    }
+}
+
 BSQ_DEV float e2m1_to_f32(uint32_t code) {
     uint32_t mag = code & 7u;
     uint32_t bits = (mag >= 2u) ? ((((mag >> 1) + 126u) << 23) | ((mag & 1u) << 22))

@@ -180,18 +180,20 @@ BSQ_DEV uint2 nv_codes(const f32x2 P[8], float r, bool fold) {
 }
 
 // Squared error of a candidate (scale den, codes), summed pairwise (0+1),
-// (2+3), ... over four levels, on the block values y.
+// (2+3), ... over four levels, on the block values y.  Scalar IEEE
+// intrinsics throughout: the compiler may fuse a packed mul.rn.f32x2 with a
+// following sub.rn.f32x2 into one rounding (seen on a block whose two
+// candidates tie exactly), and __fmul_rn / __fsub_rn are never fused.
 BSQ_DEV float nv_block_err(const f32x2 Y[8], uint2 codes, float den) {
-    float v[16];
+    float v[16], dec[16];
 #pragma unroll
     for (int k = 0; k < 8; k++) f2_unpack(Y[k], v[2 * k], v[2 * k + 1]);
+    e2m1x8_to_f32(codes.x, dec);
+    e2m1x8_to_f32(codes.y, dec + 8);
     float e[16];
 #pragma unroll
     for (int i = 0; i < 16; i++) {
-        uint32_t w = (i < 8) ? codes.x : codes.y;
-        uint32_t code = (w >> (4 * (i & 7))) & 15u;
-        float deq = __fmul_rn(e2m1_to_f32(code), den);
-        float d = __fsub_rn(v[i], deq);
+        const float d = __fsub_rn(v[i], __fmul_rn(dec[i], den));
         e[i] = __fmul_rn(d, d);
     }
 #pragma unroll
@@ -649,33 +651,57 @@ __global__ void __launch_bounds__(256) quant_mxfp8_row_kernel(
 }
 
 // Row-wise for a contiguous tensor whose rows hold a multiple of 128
-// elements: a flat sequence of 8-element chunks, two per thread in flight.
+// elements: a flat sequence of 8-element chunks, four per thread in flight.
 // Lanes 4j..4j+3 hold one block of 32 (two-step shuffle max); lanes 16i hold
 // the first of four consecutive blocks of one row and store their scale
 // word.  The SR draw index of a chunk is its flat position (row * K + col).
+// Division by an invariant divisor d <= 2^31 for n < 2^32 (Granlund and
+// Montgomery, PLDI 1994): with s = ceil(log2 d) and m = ceil(2^(32+s) / d),
+// floor(n / d) = (n * m) >> (32 + s).  m < 2^33 is kept in 64 bits.
+struct DivU32 {
+    uint64_t m;
+    int sh;
+};
+static DivU32 divu32_for(uint32_t d) {
+    int s = 0;
+    while ((uint64_t(1) << s) < d) s++;
+    const unsigned __int128 num = (unsigned __int128)1 << (32 + s);
+    return {(uint64_t)((num + d - 1) / d), 32 + s};
+}
+BSQ_DEV uint32_t divu32(uint32_t n, const DivU32 &dv) {
+    return (uint32_t)(((unsigned __int128)n * dv.m) >> dv.sh);
+}
+
 template <bool SR>
 __global__ void __launch_bounds__(256) quant_mxfp8_row_flat_kernel(
-    const uint16_t *__restrict__ x, int64_t nchunk, int64_t K, uint32_t seed_lo, uint32_t seed_hi,
+    const uint16_t *__restrict__ x, int64_t nchunk, int64_t K, DivU32 div_k8, uint32_t seed_lo, uint32_t seed_hi,
     uint32_t stream_id, uint8_t *__restrict__ codes, uint8_t *__restrict__ sf) {
+    constexpr int U = 4;
     const int64_t K8 = K >> 3, KB = K >> 5;
     const int lane = threadIdx.x & 31;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     const int64_t nwarp = (nchunk + 31) & ~int64_t(31);
-    for (int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; c - lane < nwarp; c += 2 * stride) {
-        const int64_t c1 = c + stride;
-        const bool v0 = c < nchunk, v1 = c1 < nchunk;
-        float a[8], b[8];
-        load8_bf16(x + (v0 ? c : 0) * 8, a);
-        load8_bf16(x + (v1 ? c1 : 0) * 8, b);
+    for (int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; c - lane < nwarp; c += U * stride) {
+        uint4 raw[U];
 #pragma unroll
-        for (int h = 0; h < 2; h++) {
-            const int64_t cc = h ? c1 : c;
-            const bool valid = h ? v1 : v0;
-            if (h && !__any_sync(0xFFFFFFFFu, v1)) break;
-            const float *v = h ? b : a;
-            float m = 0.0f;
+        for (int h = 0; h < U; h++) {
+            const int64_t cc = c + h * stride;
+            raw[h] = __ldg(reinterpret_cast<const uint4 *>(x + (cc < nchunk ? cc : 0) * 8));
+        }
 #pragma unroll
-            for (int i = 0; i < 8; i++) m = fmaxf(m, fabsf(v[i]));
+        for (int h = 0; h < U; h++) {
+            const int64_t cc = c + h * stride;
+            const bool valid = cc < nchunk;
+            if (h && !__any_sync(0xFFFFFFFFu, valid)) break;
+            const uint32_t w[4] = {raw[h].x, raw[h].y, raw[h].z, raw[h].w};
+            float v[8];
+#pragma unroll
+            for (int i = 0; i < 4; i++) {
+                v[2 * i] = bf16_lo(w[i]);
+                v[2 * i + 1] = bf16_hi(w[i]);
+            }
+            float m = fmax3(fmax3(fabsf(v[0]), fabsf(v[1]), fabsf(v[2])), fmax3(fabsf(v[3]), fabsf(v[4]), fabsf(v[5])),
+                            fmaxf(fabsf(v[6]), fabsf(v[7])));
             m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
             m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
             const bool zero = (m == 0.0f);
@@ -687,7 +713,7 @@ __global__ void __launch_bounds__(256) quant_mxfp8_row_flat_kernel(
             const uint32_t b2 = __shfl_down_sync(0xFFFFFFFFu, sb, 8);
             const uint32_t b3 = __shfl_down_sync(0xFFFFFFFFu, sb, 12);
             if (valid && (lane & 15) == 0) {
-                const int64_t row = cc / K8, kb = (cc - row * K8) >> 2;
+                const int64_t row = divu32((uint32_t)cc, div_k8), kb = (cc - row * K8) >> 2;
                 *reinterpret_cast<uint32_t *>(sf + sf_word_offset(row, kb >> 2, KB)) =
                     sb | (b1 << 8) | (b2 << 16) | (b3 << 24);
             }
@@ -962,14 +988,15 @@ void launch_quant_mxfp8(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, bo
                         uint64_t seed, uint32_t stream_id, uint8_t *codes, uint8_t *sf, int num_sms,
                         cudaStream_t s) {
     const uint32_t lo = (uint32_t)seed, hi = (uint32_t)(seed >> 32);
-    if (!colwise && ldx == K && K % 128 == 0) {
+    if (!colwise && ldx == K && K % 128 == 0 && M * (K >> 3) < (int64_t(1) << 32)) {
         const int64_t nchunk = M * (K >> 3);
+        const DivU32 dk8 = divu32_for((uint32_t)(K >> 3));
         if (sr) {
-            const int grid = grid_for(nchunk, 2 * 256, resident_ctas<quant_mxfp8_row_flat_kernel<true>>(num_sms));
-            quant_mxfp8_row_flat_kernel<true><<<grid, 256, 0, s>>>(x, nchunk, K, lo, hi, stream_id, codes, sf);
+            const int grid = grid_for(nchunk, 4 * 256, resident_ctas<quant_mxfp8_row_flat_kernel<true>>(num_sms));
+            quant_mxfp8_row_flat_kernel<true><<<grid, 256, 0, s>>>(x, nchunk, K, dk8, lo, hi, stream_id, codes, sf);
         } else {
-            const int grid = grid_for(nchunk, 2 * 256, resident_ctas<quant_mxfp8_row_flat_kernel<false>>(num_sms));
-            quant_mxfp8_row_flat_kernel<false><<<grid, 256, 0, s>>>(x, nchunk, K, lo, hi, stream_id, codes, sf);
+            const int grid = grid_for(nchunk, 4 * 256, resident_ctas<quant_mxfp8_row_flat_kernel<false>>(num_sms));
+            quant_mxfp8_row_flat_kernel<false><<<grid, 256, 0, s>>>(x, nchunk, K, dk8, lo, hi, stream_id, codes, sf);
         }
         return;
     }

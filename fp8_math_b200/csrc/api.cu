@@ -168,6 +168,7 @@ int bsq_quant_mxfp8(const void *x, int64_t M, int64_t K, int64_t ldx, int colwis
     if (colwise ? (M % 32 || K % 8) : (K % 32)) return BSQ_ERR_INVALID;
     if (!aligned16(x) || !aligned16(codes) || !aligned16(sf) || ldx % 8) return BSQ_ERR_ALIGN;
     if (colwise && M % 16) return BSQ_ERR_ALIGN;
+    if (colwise && (M >> 5) * ((K + 63) >> 6) >= (int64_t(1) << 31)) return BSQ_ERR_UNSUPPORTED;
     DeviceState *d;
     if (int st = device_state(&d)) return st;
     if (M == 0 || K == 0) return BSQ_OK;
@@ -195,6 +196,7 @@ int bsq_requant_transpose(const uint8_t *codes_row, const uint8_t *sf_row, int64
         return BSQ_ERR_INVALID;
     if (!aligned16(codes_row) || !aligned16(sf_row) || !aligned16(codes_col) || !aligned16(sf_col))
         return BSQ_ERR_ALIGN;
+    if ((M >> 5) * ((K + 63) >> 6) >= (int64_t(1) << 31)) return BSQ_ERR_UNSUPPORTED;
     DeviceState *d;
     if (int st = device_state(&d)) return st;
     if (M == 0 || K == 0) return BSQ_OK;

@@ -567,41 +567,98 @@ __global__ void __launch_bounds__(256) quant_nvfp4_fused_kernel(
 }
 
 // ===================================================================== MXFP8
-// E8M0 exponent of a block: clamp(floor(log2 amax) - 8, -127, 127).
-BSQ_DEV int mx_exponent(float bamax) {
-    int E = floor_log2(bamax) - 8;
-    return E < -127 ? -127 : (E > 127 ? 127 : E);
+// E8M0 code of a block from its absolute maximum m >= 0, i.e.
+// clamp(floor(log2 m) - 8, -127, 127) + 127.  The biased exponent field f of
+// a normal m is floor(log2 m) + 127, so the code is f - 8; a subnormal or
+// zero m (f = 0) takes the lower clamp, code 0; the largest finite field
+// (254) gives 246, so the upper clamp never applies.
+BSQ_DEV uint32_t mx_scale_code(float m) {
+    const int f = (int)(__float_as_uint(m) >> 23);
+    return (uint32_t)max(f - 8, 0);
+}
+// 2^-E for the block exponent E = code - 127, as the binary32 with exponent
+// field 254 - code (8..254: always normal).
+BSQ_DEV float mx_inv_scale(uint32_t code) { return __uint_as_float((254u - code) << 23); }
+
+// s = v * 2^-E for 8 values (exact: a power of two, no overflow), on fp32
+// pairs.
+BSQ_DEV void mx_scale8(const float v[8], float inv, float s[8]) {
+    const f32x2 I = f2_pack(inv, inv);
+#pragma unroll
+    for (int k = 0; k < 4; k++) f2_unpack(f2_mul(f2_pack(v[2 * k], v[2 * k + 1]), I), s[2 * k], s[2 * k + 1]);
 }
 
-// Quantize 8 consecutive outputs of one block (E known); idx0 is the output
-// linear index of v[0] (a multiple of 8).  Returns 8 codes packed in uint2.
-template <bool SR>
-BSQ_DEV uint2 mx_encode8(const float v[8], bool zero_block, int E, uint64_t idx0, uint32_t seed_lo,
-                         uint32_t seed_hi, uint32_t stream_id) {
-    if (zero_block) return make_uint2(0u, 0u);
-    const float inv = exp2i(-E);
-    float s[8];
+// RNE of 8 scaled values to E4M3, element 0 in the lowest byte.  The
+// satfinite conversion returns +-448 for |s| > 448, which is what clamping
+// to +-448 first and then rounding gives.
+BSQ_DEV uint2 mx_rne8(const float s[8]) {
+    uint2 r;
+    asm("{\n\t.reg .b16 h0, h1, h2, h3;\n\t"
+        "cvt.rn.satfinite.e4m3x2.f32 h0, %3, %2;\n\t"
+        "cvt.rn.satfinite.e4m3x2.f32 h1, %5, %4;\n\t"
+        "cvt.rn.satfinite.e4m3x2.f32 h2, %7, %6;\n\t"
+        "cvt.rn.satfinite.e4m3x2.f32 h3, %9, %8;\n\t"
+        "mov.b32 %0, {h0, h1};\n\t"
+        "mov.b32 %1, {h2, h3};\n\t}"
+        : "=r"(r.x), "=r"(r.y)
+        : "f"(s[0]), "f"(s[1]), "f"(s[2]), "f"(s[3]), "f"(s[4]), "f"(s[5]), "f"(s[6]), "f"(s[7]));
+    return r;
+}
+
+// Stochastic rounding of 8 scaled values to E4M3 with the four words of one
+// Philox call: element i draws the low (even i) or high (odd i) 16 bits of
+// word i/2.  Integer form of e4m3_sr for 2^-6 <= a <= 448, a = min(|s|, 448)
+// (a's bits are read as an unsigned integer): the E4M3 neighbour below a is
+// a with its low 20 bits cleared and frac = low20(a) / 2^20, so rounding up
+// happens iff 16 r16 < low20(a).  Shifted left by 4 and with the exponent
+// rebias 120 << 23 taken out, t = (a << 4) + 0xFFFFF0 - (r16 << 8) - (120 << 27)
+// (mod 2^32) carries into bit 24 exactly when rounding up, and its top byte
+// is then the code's magnitude (E4M3 exponent and three mantissa bits; bit 31
+// stays clear since a <= 448).  r16 << 8 is one byte permute of the draw
+// word.  A chunk holding some a < 2^-6 (E4M3 subnormals, zeros) runs the
+// float form for all eight values.
+BSQ_DEV uint2 mx_sr8(const float s[8], uint4 rnd) {
+    const uint32_t w[4] = {rnd.x, rnd.y, rnd.z, rnd.w};
+    uint32_t b[8];
+    bool slow = false;
 #pragma unroll
-    for (int i = 0; i < 8; i++) s[i] = fminf(fmaxf(__fmul_rn(v[i], inv), -448.0f), 448.0f);
-    uint32_t c[8];
-    if (SR) {
-        const uint64_t g = idx0 >> 3;
-        uint4 r = philox4x32_10(make_uint4((uint32_t)g, (uint32_t)(g >> 32), stream_id, 0u), seed_lo, seed_hi);
-        const uint32_t w[4] = {r.x, r.y, r.z, r.w};
-#pragma unroll
-        for (int i = 0; i < 8; i++) c[i] = e4m3_sr_fast(s[i], (i & 1) ? (w[i >> 1] >> 16) : (w[i >> 1] & 0xFFFFu));
-    } else {
-#pragma unroll
-        for (int i = 0; i < 8; i += 2) {
-            uint32_t p = cvt_e4m3x2(s[i], s[i + 1]);
-            c[i] = p & 0xFFu;
-            c[i + 1] = p >> 8;
-        }
+    for (int i = 0; i < 8; i++) {
+        const uint32_t a = __float_as_uint(fminf(fabsf(s[i]), 448.0f));
+        slow |= a < 0x3C800000u;  // 2^-6
+        const uint32_t p = __byte_perm(w[i >> 1], 0u, (i & 1) ? 0x4324u : 0x4104u);  // r16 << 8
+        const uint32_t t = (a << 4) + 0x40FFFFF0u - p;  // 0xFFFFF0 - (120 << 27) mod 2^32
+        b[i] = t | (__float_as_uint(s[i]) & 0x80000000u);
     }
-    return make_uint2(c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24),
-                      c[4] | (c[5] << 8) | (c[6] << 16) | (c[7] << 24));
+    if (slow) {
+        uint32_t c[8];
+#pragma unroll
+        for (int i = 0; i < 8; i++) {
+            const float v = fminf(fmaxf(s[i], -448.0f), 448.0f);
+            c[i] = e4m3_sr(v, (i & 1) ? (w[i >> 1] >> 16) : (w[i >> 1] & 0xFFFFu));
+        }
+        return make_uint2(c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24),
+                          c[4] | (c[5] << 8) | (c[6] << 16) | (c[7] << 24));
+    }
+    return make_uint2(__byte_perm(__byte_perm(b[0], b[1], 0x0073u), __byte_perm(b[2], b[3], 0x7300u), 0x7610u),
+                      __byte_perm(__byte_perm(b[4], b[5], 0x0073u), __byte_perm(b[6], b[7], 0x7300u), 0x7610u));
 }
 
+// The 8 codes of one chunk of a block with E8M0 code sb (zero: the block's
+// maximum is 0, whose codes are all +0).  chunk is the output linear index
+// of the chunk's first element divided by 8: the Philox counter of SR.
+template <bool SR>
+BSQ_DEV uint2 mx_encode8(const float v[8], bool zero, uint32_t sb, uint64_t chunk, uint32_t seed_lo,
+                         uint32_t seed_hi, uint32_t stream_id) {
+    float s[8];
+    mx_scale8(v, mx_inv_scale(sb), s);
+    uint2 q;
+    if (SR)
+        q = mx_sr8(s, philox4x32_10(make_uint4((uint32_t)chunk, (uint32_t)(chunk >> 32), stream_id, 0u), seed_lo,
+                                    seed_hi));
+    else
+        q = mx_rne8(s);
+    return zero ? make_uint2(0u, 0u) : q;
+}
 // Row-wise: one thread per 8 elements, 4 lanes per block of 32.
 template <bool SR>
 __global__ void __launch_bounds__(256) quant_mxfp8_row_kernel(
@@ -629,12 +686,11 @@ __global__ void __launch_bounds__(256) quant_mxfp8_row_kernel(
             m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
             m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
             const bool zero = (m == 0.0f);
-            const int E = zero ? 0 : mx_exponent(m);
-            const uint64_t idx0 = (uint64_t)(rr * K + cc * 8);
-            uint2 q = mx_encode8<SR>(v, zero, E, idx0, seed_lo, seed_hi, stream_id);
+            const uint32_t sb = mx_scale_code(m);
+            const uint64_t chunk = (uint64_t)(rr * K + cc * 8) >> 3;
+            uint2 q = mx_encode8<SR>(v, zero, sb, chunk, seed_lo, seed_hi, stream_id);
             if (valid) *reinterpret_cast<uint2 *>(codes + rr * K + cc * 8) = q;
             // scale byte: lanes 4j hold block j; 4 blocks (16 lanes) per word
-            const uint32_t sb = zero ? 0u : (uint32_t)(E + 127);
             const int64_t kb = cc >> 2;
             if (pack4) {
                 uint32_t b1 = __shfl_down_sync(0xFFFFFFFFu, sb, 4);
@@ -705,10 +761,9 @@ __global__ void __launch_bounds__(256) quant_mxfp8_row_flat_kernel(
             m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
             m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
             const bool zero = (m == 0.0f);
-            const int E = zero ? 0 : mx_exponent(m);
-            const uint2 q = mx_encode8<SR>(v, zero, E, (uint64_t)cc * 8, seed_lo, seed_hi, stream_id);
+            const uint32_t sb = mx_scale_code(m);
+            const uint2 q = mx_encode8<SR>(v, zero, sb, (uint64_t)cc, seed_lo, seed_hi, stream_id);
             if (valid) *reinterpret_cast<uint2 *>(codes + cc * 8) = q;
-            const uint32_t sb = zero ? 0u : (uint32_t)(E + 127);
             const uint32_t b1 = __shfl_down_sync(0xFFFFFFFFu, sb, 4);
             const uint32_t b2 = __shfl_down_sync(0xFFFFFFFFu, sb, 8);
             const uint32_t b3 = __shfl_down_sync(0xFFFFFFFFu, sb, 12);
@@ -721,115 +776,123 @@ __global__ void __launch_bounds__(256) quant_mxfp8_row_flat_kernel(
     }
 }
 
-// Column-wise (output = quantization of the transpose), from bf16 or from
-// row-wise MXFP8 (dequantized exactly).  A CTA tile covers 128 input rows
-// (output columns) x 64 input columns (output rows); shared memory holds the
-// tile as fp32 [64][128], written with lanes along m (conflict-free) and read
-// as 8 consecutive m per thread.
-constexpr int CT_M = 128, CT_K = 64;
+// Row-wise for a contiguous tensor whose rows hold a multiple of 1024
+// elements.  A warp takes spans of 1024 consecutive elements (one row
+// segment); lane l loads the 8-element chunks l, l+32, l+64, l+96 of the span
+// (four 16-byte loads in flight, each warp-wide load reading 512 contiguous
+// bytes).  Lanes 4j..4j+3 of a 32-chunk group hold one block of 32 (two-step
+// shuffle max) and lane 4j stores its scale byte.  The SR draw index of a
+// chunk is its flat position.
+template <bool SR>
+__global__ void __launch_bounds__(256) quant_mxfp8_row_span_kernel(
+    const uint16_t *__restrict__ x, uint32_t nspan, int64_t K, DivU32 div_spr, uint32_t seed_lo, uint32_t seed_hi,
+    uint32_t stream_id, uint8_t *__restrict__ codes, uint8_t *__restrict__ sf) {
+    const int lane = threadIdx.x & 31;
+    const uint32_t spr = (uint32_t)(K >> 10);  // spans per row
+    const int64_t KB = K >> 5;
+    const uint32_t nwarps = (gridDim.x * blockDim.x) >> 5;
+    const bool sf_lane = (lane & 3) == 0;
+    for (uint32_t sp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; sp < nspan; sp += nwarps) {
+        const int64_t e0 = (int64_t)sp << 10;
+        const uint4 *src = reinterpret_cast<const uint4 *>(x + e0) + lane;
+        uint4 raw[4];
+#pragma unroll
+        for (int h = 0; h < 4; h++) raw[h] = __ldg(src + 32 * h);
+        const uint32_t row = divu32(sp, div_spr), seg = sp - row * spr;
+        // scale byte of block 32 seg + 8 h + lane / 4: word 8 seg + 2 h + lane / 16 of the row
+        uint8_t *sfp = sf + sf_word_offset(row, (int64_t)seg * 8 + (lane >> 4), KB) + ((lane >> 2) & 3);
+        uint2 *dst = reinterpret_cast<uint2 *>(codes + e0) + lane;
+        const uint64_t chunk0 = ((uint64_t)sp << 7) + lane;
+#pragma unroll
+        for (int h = 0; h < 4; h++) {
+            const uint32_t w[4] = {raw[h].x, raw[h].y, raw[h].z, raw[h].w};
+            float v[8];
+#pragma unroll
+            for (int i = 0; i < 4; i++) {
+                v[2 * i] = bf16_lo(w[i]);
+                v[2 * i + 1] = bf16_hi(w[i]);
+            }
+            float m = fmax3(fmax3(fabsf(v[0]), fabsf(v[1]), fabsf(v[2])), fmax3(fabsf(v[3]), fabsf(v[4]), fabsf(v[5])),
+                            fmaxf(fabsf(v[6]), fabsf(v[7])));
+            m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+            m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+            const uint32_t sb = mx_scale_code(m);
+            dst[32 * h] = mx_encode8<SR>(v, m == 0.0f, sb, chunk0 + 32 * h, seed_lo, seed_hi, stream_id);
+            if (sf_lane) sfp[h * 1024] = (uint8_t)sb;
+        }
+    }
+}
 
+// Column-wise (output [K, M] = quantization of the transpose, blocks of 32
+// along M), from bf16 or from row-wise MXFP8 (dequantized exactly).  A warp
+// covers 32 input rows x 64 input columns with no shared memory: lane
+// l = 4 kg + mg loads the 8 x 8 piece of rows 8 mg .. 8 mg + 7 and columns
+// 8 kg .. 8 kg + 7 (each warp-wide load reads 128 contiguous bytes of four
+// rows), which holds, per column, one output chunk of 8 consecutive m; the
+// four lanes with the same kg share that column's block of 32 (two-step
+// shuffle max).  Warp tiles run m-fastest, so consecutive warps write
+// adjacent 32-byte pieces of each output row.
 template <bool FROM_MX, bool SR>
 __global__ void __launch_bounds__(256) quant_mxfp8_col_kernel(
     const void *__restrict__ xin, const uint8_t *__restrict__ sf_in, int64_t M, int64_t K, int64_t ldx,
-    uint32_t seed_lo, uint32_t seed_hi, uint32_t stream_id, uint8_t *__restrict__ codes,
-    uint8_t *__restrict__ sf) {
-    __shared__ __align__(16) float tile[CT_K][CT_M];
-    const uint32_t m_tiles = (uint32_t)((M + CT_M - 1) / CT_M), k_tiles = (uint32_t)((K + CT_K - 1) / CT_K);
-    const int64_t MB = M >> 5;  // output blocks per output row
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    for (uint32_t t = blockIdx.x; t < m_tiles * k_tiles; t += gridDim.x) {
-        const uint32_t kt = t / m_tiles, mt = t - kt * m_tiles;
-        const int64_t m0 = (int64_t)mt * CT_M, k0 = (int64_t)kt * CT_K;
-        // ---- load: each thread reads 32 contiguous bytes of one input row
+    uint32_t ntile, DivU32 div_mt, uint32_t seed_lo, uint32_t seed_hi, uint32_t stream_id,
+    uint8_t *__restrict__ codes, uint8_t *__restrict__ sf) {
+    const int lane = threadIdx.x & 31, kg = lane >> 2, mg = lane & 3;
+    const uint32_t mt_n = (uint32_t)(M >> 5);
+    const int64_t MB = M >> 5, KBin = K >> 5;
+    const uint32_t nwarps = (gridDim.x * blockDim.x) >> 5;
+    for (uint32_t t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < ntile; t += nwarps) {
+        const uint32_t kt = divu32(t, div_mt), mt = t - kt * mt_n;
+        const int64_t m0 = (int64_t)mt * 32 + mg * 8, k0 = (int64_t)kt * 64 + kg * 8;
+        const bool kvalid = k0 < K;  // K % 8 == 0: a lane's 8 columns are all in or all out
+        // w[i][p]: columns 2p, 2p + 1 of row m0 + i (low half: the even column)
+        uint32_t w[8][4];
+        float sc[8];
         if (!FROM_MX) {
-            const uint16_t *x = static_cast<const uint16_t *>(xin);
+            const uint16_t *x = static_cast<const uint16_t *>(xin) + m0 * ldx + k0;
 #pragma unroll
-            for (int it = 0; it < 2; it++) {
-                const int task = warp + 8 * it;  // 16 tasks of (row block of 32, chunk of 16 k)
-                const int ml = (task & 3) * 32 + lane;
-                const int kc = task >> 2;         // 0..3, 16 k each
-                const int64_t m = m0 + ml, k = k0 + kc * 16;
-                float v[16];
-                if (m < M && k < K) {  // K % 8 == 0; a chunk may be half valid
-                    load8_bf16(x + m * ldx + k, v);
-                    if (k + 8 < K) load8_bf16(x + m * ldx + k + 8, v + 8);
-                    else
-#pragma unroll
-                        for (int i = 8; i < 16; i++) v[i] = 0.0f;
-                } else {
-#pragma unroll
-                    for (int i = 0; i < 16; i++) v[i] = 0.0f;
-                }
-#pragma unroll
-                for (int i = 0; i < 16; i++) tile[kc * 16 + i][ml] = v[i];
+            for (int i = 0; i < 8; i++) {
+                const uint4 r = kvalid ? __ldg(reinterpret_cast<const uint4 *>(x + i * ldx)) : make_uint4(0, 0, 0, 0);
+                w[i][0] = r.x; w[i][1] = r.y; w[i][2] = r.z; w[i][3] = r.w;
             }
         } else {
-            const uint8_t *x = static_cast<const uint8_t *>(xin);
-            const int64_t KBin = K >> 5;
-            const int ml = (warp & 3) * 32 + lane;
-            const int kc = warp >> 2;  // 0..1, 32 k each
-            const int64_t m = m0 + ml, k = k0 + kc * 32;
-            float v[32];
-            if (m < M && k < K) {
-                const float sc = exp2i((int)__ldg(sf_in + sf_offset(m, k >> 5, KBin)) - 127);
-                const uint4 *p = reinterpret_cast<const uint4 *>(x + m * ldx + k);
-                uint4 a = __ldg(p), b = __ldg(p + 1);
-                const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+            const uint8_t *x = static_cast<const uint8_t *>(xin) + m0 * ldx + k0;
 #pragma unroll
-                for (int i = 0; i < 8; i++) {
-                    float f0, f1, f2, f3;
-                    e4m3x2_to_f32(w[i] & 0xFFFFu, f0, f1);
-                    e4m3x2_to_f32(w[i] >> 16, f2, f3);
-                    v[4 * i] = __fmul_rn(f0, sc);
-                    v[4 * i + 1] = __fmul_rn(f1, sc);
-                    v[4 * i + 2] = __fmul_rn(f2, sc);
-                    v[4 * i + 3] = __fmul_rn(f3, sc);
-                }
-            } else {
-#pragma unroll
-                for (int i = 0; i < 32; i++) v[i] = 0.0f;
+            for (int i = 0; i < 8; i++) {
+                const uint2 r = kvalid ? __ldg(reinterpret_cast<const uint2 *>(x + i * ldx)) : make_uint2(0, 0);
+                w[i][0] = r.x; w[i][1] = r.y;
+                sc[i] = kvalid ? exp2i((int)__ldg(sf_in + sf_offset(m0 + i, k0 >> 5, KBin)) - 127) : 0.0f;
             }
-#pragma unroll
-            for (int i = 0; i < 32; i++) tile[kc * 32 + i][ml] = v[i];
         }
-        __syncthreads();
-        // ---- quantize: 64 output rows x 16 chunks of 8; 4 lanes per block
+        float odd[8];  // E4M3 input: column j + 1, decoded with column j
 #pragma unroll
-        for (int it = 0; it < 4; it++) {
-            const int task = threadIdx.x + 256 * it;
-            const int mc = task & 15, kl = task >> 4;
-            const int64_t k = k0 + kl, m = m0 + mc * 8;
-            const float4 *src = reinterpret_cast<const float4 *>(&tile[kl][mc * 8]);
-            float4 a = src[0], b = src[1];
-            float v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-            float am = 0.0f;
+        for (int j = 0; j < 8; j++) {
+            float v[8];
 #pragma unroll
-            for (int i = 0; i < 8; i++) am = fmaxf(am, fabsf(v[i]));
-            am = fmaxf(am, __shfl_xor_sync(0xFFFFFFFFu, am, 1));
-            am = fmaxf(am, __shfl_xor_sync(0xFFFFFFFFu, am, 2));
-            const bool zero = (am == 0.0f);
-            const int E = zero ? 0 : mx_exponent(am);
-            const bool valid = (k < K) && (m < M);
-            const uint64_t idx0 = (uint64_t)(k * M + m);
-            uint2 q = mx_encode8<SR>(v, zero, E, idx0, seed_lo, seed_hi, stream_id);
-            if (valid) *reinterpret_cast<uint2 *>(codes + k * M + m) = q;
-            const uint32_t sb = zero ? 0u : (uint32_t)(E + 127);
-            // lanes with mc = 0, 4, 8, 12 hold blocks 0..3 of this tile row
-            uint32_t b1 = __shfl_down_sync(0xFFFFFFFFu, sb, 4);
-            uint32_t b2 = __shfl_down_sync(0xFFFFFFFFu, sb, 8);
-            uint32_t b3 = __shfl_down_sync(0xFFFFFFFFu, sb, 12);
-            const int64_t blk = m >> 5;
-            if (k < K && (mc & 3) == 0 && m < M) {
-                if (m0 + CT_M <= M && (MB & 3) == 0) {
-                    if (mc == 0)
-                        *reinterpret_cast<uint32_t *>(sf + sf_word_offset(k, blk >> 2, MB)) =
-                            sb | (b1 << 8) | (b2 << 16) | (b3 << 24);
+            for (int i = 0; i < 8; i++) {
+                if (!FROM_MX) {
+                    v[i] = (j & 1) ? bf16_hi(w[i][j >> 1]) : bf16_lo(w[i][j >> 1]);
+                } else if ((j & 1) == 0) {
+                    float e0, e1;
+                    e4m3x2_to_f32(w[i][j >> 2] >> (8 * (j & 3)), e0, e1);
+                    v[i] = __fmul_rn(e0, sc[i]);
+                    odd[i] = __fmul_rn(e1, sc[i]);
                 } else {
-                    sf[sf_offset(k, blk, MB)] = (uint8_t)sb;
+                    v[i] = odd[i];
                 }
             }
+            float m = fmax3(fmax3(fabsf(v[0]), fabsf(v[1]), fabsf(v[2])), fmax3(fabsf(v[3]), fabsf(v[4]), fabsf(v[5])),
+                            fmaxf(fabsf(v[6]), fabsf(v[7])));
+            m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+            m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+            const uint32_t sb = mx_scale_code(m);
+            const int64_t k = k0 + j;
+            const uint2 q = mx_encode8<SR>(v, m == 0.0f, sb, (uint64_t)(k * M + m0) >> 3, seed_lo, seed_hi, stream_id);
+            if (kvalid) {
+                *reinterpret_cast<uint2 *>(codes + k * M + m0) = q;
+                if (mg == 0) sf[sf_offset(k, m0 >> 5, MB)] = (uint8_t)sb;
+            }
         }
-        __syncthreads();
     }
 }
 
@@ -988,6 +1051,18 @@ void launch_quant_mxfp8(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, bo
                         uint64_t seed, uint32_t stream_id, uint8_t *codes, uint8_t *sf, int num_sms,
                         cudaStream_t s) {
     const uint32_t lo = (uint32_t)seed, hi = (uint32_t)(seed >> 32);
+    if (!colwise && ldx == K && K % 1024 == 0 && M * (K >> 10) < (int64_t(1) << 31)) {
+        const uint32_t nspan = (uint32_t)(M * (K >> 10));
+        const DivU32 dspr = divu32_for((uint32_t)(K >> 10));
+        if (sr) {
+            const int grid = grid_for(nspan, 8, resident_ctas<quant_mxfp8_row_span_kernel<true>>(num_sms));
+            quant_mxfp8_row_span_kernel<true><<<grid, 256, 0, s>>>(x, nspan, K, dspr, lo, hi, stream_id, codes, sf);
+        } else {
+            const int grid = grid_for(nspan, 8, resident_ctas<quant_mxfp8_row_span_kernel<false>>(num_sms));
+            quant_mxfp8_row_span_kernel<false><<<grid, 256, 0, s>>>(x, nspan, K, dspr, lo, hi, stream_id, codes, sf);
+        }
+        return;
+    }
     if (!colwise && ldx == K && K % 128 == 0 && M * (K >> 3) < (int64_t(1) << 32)) {
         const int64_t nchunk = M * (K >> 3);
         const DivU32 dk8 = divu32_for((uint32_t)(K >> 3));
@@ -1008,26 +1083,34 @@ void launch_quant_mxfp8(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, bo
         else quant_mxfp8_row_kernel<false><<<grid, 256, 0, s>>>(x, M, K, ldx, lo, hi, stream_id, codes, sf, map);
         return;
     }
-    const int64_t tiles = ((M + CT_M - 1) / CT_M) * ((K + CT_K - 1) / CT_K);
-    const int grid = grid_for(tiles, 1, num_sms * 6);
-    if (sr)
-        quant_mxfp8_col_kernel<false, true><<<grid, 256, 0, s>>>(x, nullptr, M, K, ldx, lo, hi, stream_id, codes, sf);
-    else
-        quant_mxfp8_col_kernel<false, false><<<grid, 256, 0, s>>>(x, nullptr, M, K, ldx, lo, hi, stream_id, codes, sf);
+    const uint32_t ntile = (uint32_t)((M >> 5) * ((K + 63) >> 6));
+    const DivU32 dmt = divu32_for((uint32_t)(M >> 5));
+    if (sr) {
+        const int grid = grid_for(ntile, 8, resident_ctas<quant_mxfp8_col_kernel<false, true>>(num_sms));
+        quant_mxfp8_col_kernel<false, true><<<grid, 256, 0, s>>>(x, nullptr, M, K, ldx, ntile, dmt, lo, hi,
+                                                                 stream_id, codes, sf);
+    } else {
+        const int grid = grid_for(ntile, 8, resident_ctas<quant_mxfp8_col_kernel<false, false>>(num_sms));
+        quant_mxfp8_col_kernel<false, false><<<grid, 256, 0, s>>>(x, nullptr, M, K, ldx, ntile, dmt, lo, hi,
+                                                                  stream_id, codes, sf);
+    }
 }
 
 void launch_requant_transpose(const uint8_t *codes_row, const uint8_t *sf_row, int64_t M, int64_t K, bool sr,
                               uint64_t seed, uint32_t stream_id, uint8_t *codes_col, uint8_t *sf_col,
                               int num_sms, cudaStream_t s) {
     const uint32_t lo = (uint32_t)seed, hi = (uint32_t)(seed >> 32);
-    const int64_t tiles = ((M + CT_M - 1) / CT_M) * ((K + CT_K - 1) / CT_K);
-    const int grid = grid_for(tiles, 1, num_sms * 6);
-    if (sr)
-        quant_mxfp8_col_kernel<true, true><<<grid, 256, 0, s>>>(codes_row, sf_row, M, K, K, lo, hi, stream_id,
-                                                                codes_col, sf_col);
-    else
-        quant_mxfp8_col_kernel<true, false><<<grid, 256, 0, s>>>(codes_row, sf_row, M, K, K, lo, hi, stream_id,
-                                                                 codes_col, sf_col);
+    const uint32_t ntile = (uint32_t)((M >> 5) * ((K + 63) >> 6));
+    const DivU32 dmt = divu32_for((uint32_t)(M >> 5));
+    if (sr) {
+        const int grid = grid_for(ntile, 8, resident_ctas<quant_mxfp8_col_kernel<true, true>>(num_sms));
+        quant_mxfp8_col_kernel<true, true><<<grid, 256, 0, s>>>(codes_row, sf_row, M, K, K, ntile, dmt, lo, hi,
+                                                                stream_id, codes_col, sf_col);
+    } else {
+        const int grid = grid_for(ntile, 8, resident_ctas<quant_mxfp8_col_kernel<true, false>>(num_sms));
+        quant_mxfp8_col_kernel<true, false><<<grid, 256, 0, s>>>(codes_row, sf_row, M, K, K, ntile, dmt, lo, hi,
+                                                                 stream_id, codes_col, sf_col);
+    }
 }
 
 void launch_rht(const uint16_t *x, uint16_t *y, int64_t M, int64_t K, int64_t ldx, int64_t ldy, uint32_t mask,

@@ -140,7 +140,8 @@ BSQ_API int bsq_quant_nvfp4(const void *x_bf16, int64_t M, int64_t K, int64_t ld
  * colwise == 0: blocks along K, codes [M][K], sf for M rows x K/32 blocks.
  * colwise == 1: the quantization of x^T -- codes [K][M] (row stride M), sf
  * for K rows x M/32 blocks.  K % 32 == 0 (row-wise); M % 32 == 0 and
- * K % 8 == 0 (column-wise). */
+ * K % 8 == 0 (column-wise).  Column-wise tensors with
+ * (M / 32) * ceil(K / 64) >= 2^31 return BSQ_ERR_UNSUPPORTED. */
 BSQ_API int bsq_quant_mxfp8(const void *x_bf16, int64_t M, int64_t K, int64_t ldx, int colwise,
                     int rounding, uint64_t seed, uint32_t stream_id,
                     uint8_t *codes_dev, uint8_t *sf_dev, void *stream);
@@ -159,7 +160,8 @@ BSQ_API int bsq_rht(const void *x_bf16, void *y_bf16, int64_t M, int64_t K, int6
  * [M][K], swizzled sf for M x K/32) is decoded exactly (E4M3 x 2^E, fp32),
  * transposed, and quantized again as in bsq_quant_mxfp8 with blocks of 32
  * along the old M: codes_col [K][M], sf_col for K rows x M/32 blocks.
- * M % 32 == 0 and K % 32 == 0 (whole blocks of 32 along both axes). */
+ * M % 32 == 0 and K % 32 == 0 (whole blocks of 32 along both axes);
+ * (M / 32) * ceil(K / 64) >= 2^31 returns BSQ_ERR_UNSUPPORTED. */
 BSQ_API int bsq_requant_transpose(const uint8_t *codes_row_dev, const uint8_t *sf_row_dev,
                           int64_t M, int64_t K, int rounding, uint64_t seed, uint32_t stream_id,
                           uint8_t *codes_col_dev, uint8_t *sf_col_dev, void *stream);

@@ -197,7 +197,7 @@ def mx_edge_tensor(M, K, seed=0):
 
 
 @pytest.mark.parametrize("sr", [False, True])
-@pytest.mark.parametrize("M,K", [(64, 128), (3, 32), (100, 96), (256, 4096)])
+@pytest.mark.parametrize("M,K", [(64, 128), (3, 32), (100, 96), (256, 4096), (48, 1024), (33, 3072)])
 def test_mxfp8_rowwise_parity(ora, M, K, sr):
     x = mx_edge_tensor(M, K, seed=M * 3 + K)
     c, s = api.quant_mxfp8(dev(x), sr=sr, seed=1, stream_id=0)
@@ -207,7 +207,7 @@ def test_mxfp8_rowwise_parity(ora, M, K, sr):
 
 
 @pytest.mark.parametrize("sr", [False, True])
-@pytest.mark.parametrize("M,K", [(128, 64), (32, 8), (96, 200), (512, 256), (160, 40)])
+@pytest.mark.parametrize("M,K", [(128, 64), (32, 8), (96, 200), (512, 256), (160, 40), (64, 1000), (2048, 72)])
 def test_mxfp8_colwise_parity(ora, M, K, sr):
     x = mx_edge_tensor(M, K, seed=M + 5 * K)
     c, s = api.quant_mxfp8(dev(x), colwise=True, sr=sr, seed=4, stream_id=3)
@@ -217,7 +217,7 @@ def test_mxfp8_colwise_parity(ora, M, K, sr):
 
 
 @pytest.mark.parametrize("sr", [False, True])
-@pytest.mark.parametrize("M,K", [(128, 64), (32, 32), (96, 160), (256, 512)])
+@pytest.mark.parametrize("M,K", [(128, 64), (32, 32), (96, 160), (256, 512), (64, 1056)])
 def test_requant_transpose_parity(ora, M, K, sr):
     x = mx_edge_tensor(M, K, seed=M + K)
     oc, osf = ora.quant_mxfp8(bits(x), sr=True, seed=1, stream_id=0)

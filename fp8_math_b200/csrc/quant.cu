@@ -643,21 +643,109 @@ BSQ_DEV uint2 mx_sr8(const float s[8], uint4 rnd) {
                       __byte_perm(__byte_perm(b[4], b[5], 0x0073u), __byte_perm(b[6], b[7], 0x7300u), 0x7610u));
 }
 
+BSQ_DEV uint4 mx_draws(uint64_t chunk, uint32_t seed_lo, uint32_t seed_hi, uint32_t stream_id) {
+    return philox4x32_10(make_uint4((uint32_t)chunk, (uint32_t)(chunk >> 32), stream_id, 0u), seed_lo, seed_hi);
+}
+
+// True when stochastic rounding of the 8 scaled values cannot depend on the
+// draws: each one is an E4M3 value of the normal range or above 448 (its low
+// 20 bits are zero, so frac = 0 and it never rounds up), as every E4M3 input
+// rescaled by a power of two is unless it falls below 2^-6.
+BSQ_DEV bool mx_sr8_drawless(const float s[8]) {
+    bool ok = true;
+#pragma unroll
+    for (int i = 0; i < 8; i++) {
+        const uint32_t a = __float_as_uint(fminf(fabsf(s[i]), 448.0f));
+        ok &= ((a & 0xFFFFFu) == 0u) & (a >= 0x3C800000u);
+    }
+    return ok;
+}
+
 // The 8 codes of one chunk of a block with E8M0 code sb (zero: the block's
 // maximum is 0, whose codes are all +0).  chunk is the output linear index
-// of the chunk's first element divided by 8: the Philox counter of SR.
-template <bool SR>
+// of the chunk's first element divided by 8: the Philox counter of SR.  With
+// EXACT_IN (inputs that are E4M3 values times a power of two) the Philox call
+// runs only for chunks whose rounding can depend on it.
+template <bool SR, bool EXACT_IN = false>
 BSQ_DEV uint2 mx_encode8(const float v[8], bool zero, uint32_t sb, uint64_t chunk, uint32_t seed_lo,
                          uint32_t seed_hi, uint32_t stream_id) {
     float s[8];
     mx_scale8(v, mx_inv_scale(sb), s);
     uint2 q;
-    if (SR)
-        q = mx_sr8(s, philox4x32_10(make_uint4((uint32_t)chunk, (uint32_t)(chunk >> 32), stream_id, 0u), seed_lo,
-                                    seed_hi));
-    else
+    if (SR) {
+        if (EXACT_IN && mx_sr8_drawless(s))
+            q = mx_sr8(s, make_uint4(0u, 0u, 0u, 0u));
+        else
+            q = mx_sr8(s, mx_draws(chunk, seed_lo, seed_hi, stream_id));
+    } else {
         q = mx_rne8(s);
+    }
     return zero ? make_uint2(0u, 0u) : q;
+}
+
+// ---- MXFP8 stochastic rounding on packed bf16 pairs (16-bit lanes)
+BSQ_DEV uint32_t u16x2_max(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("max.u16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+BSQ_DEV uint32_t u16x2_min(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("min.u16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+BSQ_DEV uint32_t bf16x2_mul(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
+// |x| bits of a chunk held as 4 bf16 pairs (element 2k in the low half of
+// pair k) and the chunk's absolute maximum as bf16 bits (non-negative
+// floats order as their bit patterns).
+BSQ_DEV uint32_t bf16_chunk_absmax(const uint32_t p[4], uint32_t a[4]) {
+#pragma unroll
+    for (int k = 0; k < 4; k++) a[k] = p[k] & 0x7FFF7FFFu;
+    const uint32_t m2 = u16x2_max(u16x2_max(a[0], a[1]), u16x2_max(a[2], a[3]));
+    return max(m2 & 0xFFFFu, m2 >> 16);
+}
+// E8M0 code from a block maximum given as bf16 bits (exponent field in bits
+// 7..14, the same field as the fp32 value's): see mx_scale_code.
+BSQ_DEV uint32_t mx_scale_code_bf16(uint32_t m) { return (uint32_t)max((int)(m >> 7) - 8, 0); }
+
+// Stochastic rounding of one chunk of bf16 values (pairs p, magnitudes a)
+// in block code sb, two values per 32-bit operation.  s = |x| 2^-E is one
+// bf16 multiply (exact whenever s >= 2^-126), clamped to 448 (0x43E0).  A
+// bf16-sourced s has 4 bits below the E4M3 mantissa, so frac = low4 / 16 and
+// "16 r16 < low20" becomes "r16 >> 12 < low4": adding 15 - (r16 >> 12) to
+// the 16-bit lane carries into bit 4 exactly when rounding up, and
+// (s + 15 - (r16 >> 12) - (120 << 7)) >> 4 is then the E4M3 magnitude code
+// (exponent - 120 and three mantissa bits).  Shifted left by 4, each lane's
+// code sits in its upper byte with bit 7 clear, where the bf16 sign bit is
+// or-ed in.  A chunk holding some s < 2^-6 (E4M3 subnormals, zeros) runs
+// the fp32 form on all eight values.
+BSQ_DEV uint2 mx_sr8_bf16(const uint32_t p[4], const uint32_t a[4], uint32_t sb, uint4 rnd) {
+    const uint32_t inv2 = ((254u - sb) << 7) * 0x10001u;  // 2^-E in both bf16 lanes
+    const uint32_t w[4] = {rnd.x, rnd.y, rnd.z, rnd.w};
+    uint32_t mn = 0xFFFFFFFFu, u[4];
+#pragma unroll
+    for (int k = 0; k < 4; k++) {
+        const uint32_t s = u16x2_min(bf16x2_mul(a[k], inv2), 0x43E043E0u);
+        mn = u16x2_min(mn, s);
+        const uint32_t r = (~w[k] >> 12) & 0x000F000Fu;  // 15 - (r16 >> 12), both lanes
+        u[k] = ((s + r - 0x3C003C00u) << 4) | (p[k] & 0x80008000u);
+    }
+    if (min(mn & 0xFFFFu, mn >> 16) < 0x3C80u) {  // 2^-6
+        float v[8], s[8];
+#pragma unroll
+        for (int k = 0; k < 4; k++) {
+            v[2 * k] = bf16_lo(p[k]);
+            v[2 * k + 1] = bf16_hi(p[k]);
+        }
+        mx_scale8(v, mx_inv_scale(sb), s);
+        return mx_sr8(s, rnd);
+    }
+    return make_uint2(__byte_perm(u[0], u[1], 0x7531u), __byte_perm(u[2], u[3], 0x7531u));
 }
 // Row-wise: one thread per 8 elements, 4 lanes per block of 32.
 template <bool SR>
@@ -806,18 +894,29 @@ __global__ void __launch_bounds__(256) quant_mxfp8_row_span_kernel(
 #pragma unroll
         for (int h = 0; h < 4; h++) {
             const uint32_t w[4] = {raw[h].x, raw[h].y, raw[h].z, raw[h].w};
-            float v[8];
+            uint32_t sb;
+            if (SR) {
+                uint32_t a[4];
+                uint32_t m = bf16_chunk_absmax(w, a);
+                m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+                m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+                sb = mx_scale_code_bf16(m);
+                const uint2 q = mx_sr8_bf16(w, a, sb, mx_draws(chunk0 + 32 * h, seed_lo, seed_hi, stream_id));
+                dst[32 * h] = (m == 0u) ? make_uint2(0u, 0u) : q;
+            } else {
+                float v[8];
 #pragma unroll
-            for (int i = 0; i < 4; i++) {
-                v[2 * i] = bf16_lo(w[i]);
-                v[2 * i + 1] = bf16_hi(w[i]);
+                for (int i = 0; i < 4; i++) {
+                    v[2 * i] = bf16_lo(w[i]);
+                    v[2 * i + 1] = bf16_hi(w[i]);
+                }
+                float m = fmax3(fmax3(fabsf(v[0]), fabsf(v[1]), fabsf(v[2])),
+                                fmax3(fabsf(v[3]), fabsf(v[4]), fabsf(v[5])), fmaxf(fabsf(v[6]), fabsf(v[7])));
+                m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+                m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+                sb = mx_scale_code(m);
+                dst[32 * h] = mx_encode8<false>(v, m == 0.0f, sb, 0, 0u, 0u, 0u);
             }
-            float m = fmax3(fmax3(fabsf(v[0]), fabsf(v[1]), fabsf(v[2])), fmax3(fabsf(v[3]), fabsf(v[4]), fabsf(v[5])),
-                            fmaxf(fabsf(v[6]), fabsf(v[7])));
-            m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
-            m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
-            const uint32_t sb = mx_scale_code(m);
-            dst[32 * h] = mx_encode8<SR>(v, m == 0.0f, sb, chunk0 + 32 * h, seed_lo, seed_hi, stream_id);
             if (sf_lane) sfp[h * 1024] = (uint8_t)sb;
         }
     }
@@ -867,6 +966,25 @@ __global__ void __launch_bounds__(256) quant_mxfp8_col_kernel(
         float odd[8];  // E4M3 input: column j + 1, decoded with column j
 #pragma unroll
         for (int j = 0; j < 8; j++) {
+            const int64_t k = k0 + j;
+            if (!FROM_MX && SR) {
+                // rows 2i, 2i + 1 of column j as one bf16 pair
+                uint32_t p[4], a[4];
+#pragma unroll
+                for (int i = 0; i < 4; i++)
+                    p[i] = __byte_perm(w[2 * i][j >> 1], w[2 * i + 1][j >> 1], (j & 1) ? 0x7632u : 0x5410u);
+                uint32_t m = bf16_chunk_absmax(p, a);
+                m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+                m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+                const uint32_t sb = mx_scale_code_bf16(m);
+                uint2 q = mx_sr8_bf16(p, a, sb, mx_draws((uint64_t)(k * M + m0) >> 3, seed_lo, seed_hi, stream_id));
+                if (m == 0u) q = make_uint2(0u, 0u);
+                if (kvalid) {
+                    *reinterpret_cast<uint2 *>(codes + k * M + m0) = q;
+                    if (mg == 0) sf[sf_offset(k, m0 >> 5, MB)] = (uint8_t)sb;
+                }
+                continue;
+            }
             float v[8];
 #pragma unroll
             for (int i = 0; i < 8; i++) {
@@ -886,8 +1004,8 @@ __global__ void __launch_bounds__(256) quant_mxfp8_col_kernel(
             m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
             m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
             const uint32_t sb = mx_scale_code(m);
-            const int64_t k = k0 + j;
-            const uint2 q = mx_encode8<SR>(v, m == 0.0f, sb, (uint64_t)(k * M + m0) >> 3, seed_lo, seed_hi, stream_id);
+            const uint2 q =
+                mx_encode8<SR, FROM_MX>(v, m == 0.0f, sb, (uint64_t)(k * M + m0) >> 3, seed_lo, seed_hi, stream_id);
             if (kvalid) {
                 *reinterpret_cast<uint2 *>(codes + k * M + m0) = q;
                 if (mg == 0) sf[sf_offset(k, m0 >> 5, MB)] = (uint8_t)sb;

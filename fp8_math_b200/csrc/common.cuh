@@ -137,17 +137,29 @@ BSQ_DEV float exp2i(int k) {
 }
 
 // ---------------------------------------------------------------- Philox
-// Philox4x32-10 (Salmon, Moraes, Dror, Shaw, SC'11).
-BSQ_DEV uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1) {
+// Philox4x32-10 (Salmon, Moraes, Dror, Shaw, SC'11): ten rounds of two
+// 32x32->64 multiplies (0xD2511F53, 0xCD9E8D57) and xors with the round keys.
+// The ten round keys for key (k0, k1): round r uses
+// (k0 + r 0x9E3779B9, k1 + r 0xBB67AE85) mod 2^32.  Computed once on the host
+// and passed as a kernel parameter, so the rounds read them from the
+// constant bank instead of recomputing the schedule per call.
+struct PhiloxKeys {
+    uint32_t k0[10], k1[10];
+};
+static inline PhiloxKeys philox_keys(uint32_t k0, uint32_t k1) {
+    PhiloxKeys K;
+    for (int r = 0; r < 10; r++) {
+        K.k0[r] = k0 + (uint32_t)r * 0x9E3779B9u;
+        K.k1[r] = k1 + (uint32_t)r * 0xBB67AE85u;
+    }
+    return K;
+}
+BSQ_DEV uint4 philox4x32_10(uint4 c, const PhiloxKeys &K) {
 #pragma unroll
     for (int r = 0; r < 10; r++) {
-        if (r) {
-            k0 += 0x9E3779B9u;
-            k1 += 0xBB67AE85u;
-        }
-        uint32_t hi0 = __umulhi(0xD2511F53u, c.x), lo0 = 0xD2511F53u * c.x;
-        uint32_t hi1 = __umulhi(0xCD9E8D57u, c.z), lo1 = 0xCD9E8D57u * c.z;
-        c = make_uint4(hi1 ^ c.y ^ k0, lo1, hi0 ^ c.w ^ k1, lo0);
+        const uint64_t p0 = (uint64_t)0xD2511F53u * c.x, p1 = (uint64_t)0xCD9E8D57u * c.z;
+        c = make_uint4((uint32_t)(p1 >> 32) ^ c.y ^ K.k0[r], (uint32_t)p1, (uint32_t)(p0 >> 32) ^ c.w ^ K.k1[r],
+                       (uint32_t)p0);
     }
     return c;
 }

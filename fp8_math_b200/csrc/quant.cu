@@ -617,6 +617,22 @@ BSQ_DEV uint2 mx_rne8(const float s[8]) {
 // stays clear since a <= 448).  r16 << 8 is one byte permute of the draw
 // word.  A chunk holding some a < 2^-6 (E4M3 subnormals, zeros) runs the
 // float form for all eight values.
+// The float form of stochastic rounding for a whole chunk (e4m3_sr per value
+// after the clamp to +-448).  It runs only for chunks holding E4M3 subnormals
+// or zeros, so it is kept out of line: the unrolled callers stay small.
+__device__ __noinline__ uint2 mx_sr8_float(float s0, float s1, float s2, float s3, float s4, float s5, float s6,
+                                           float s7, uint4 rnd) {
+    const float s[8] = {s0, s1, s2, s3, s4, s5, s6, s7};
+    const uint32_t w[4] = {rnd.x, rnd.y, rnd.z, rnd.w};
+    uint32_t c[8];
+#pragma unroll
+    for (int i = 0; i < 8; i++) {
+        const float v = fminf(fmaxf(s[i], -448.0f), 448.0f);
+        c[i] = e4m3_sr(v, (i & 1) ? (w[i >> 1] >> 16) : (w[i >> 1] & 0xFFFFu));
+    }
+    return make_uint2(c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24), c[4] | (c[5] << 8) | (c[6] << 16) | (c[7] << 24));
+}
+
 BSQ_DEV uint2 mx_sr8(const float s[8], uint4 rnd) {
     const uint32_t w[4] = {rnd.x, rnd.y, rnd.z, rnd.w};
     uint32_t b[8];
@@ -629,22 +645,13 @@ BSQ_DEV uint2 mx_sr8(const float s[8], uint4 rnd) {
         const uint32_t t = (a << 4) + 0x40FFFFF0u - p;  // 0xFFFFF0 - (120 << 27) mod 2^32
         b[i] = t | (__float_as_uint(s[i]) & 0x80000000u);
     }
-    if (slow) {
-        uint32_t c[8];
-#pragma unroll
-        for (int i = 0; i < 8; i++) {
-            const float v = fminf(fmaxf(s[i], -448.0f), 448.0f);
-            c[i] = e4m3_sr(v, (i & 1) ? (w[i >> 1] >> 16) : (w[i >> 1] & 0xFFFFu));
-        }
-        return make_uint2(c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24),
-                          c[4] | (c[5] << 8) | (c[6] << 16) | (c[7] << 24));
-    }
+    if (slow) return mx_sr8_float(s[0], s[1], s[2], s[3], s[4], s[5], s[6], s[7], rnd);
     return make_uint2(__byte_perm(__byte_perm(b[0], b[1], 0x0073u), __byte_perm(b[2], b[3], 0x7300u), 0x7610u),
                       __byte_perm(__byte_perm(b[4], b[5], 0x0073u), __byte_perm(b[6], b[7], 0x7300u), 0x7610u));
 }
 
-BSQ_DEV uint4 mx_draws(uint64_t chunk, uint32_t seed_lo, uint32_t seed_hi, uint32_t stream_id) {
-    return philox4x32_10(make_uint4((uint32_t)chunk, (uint32_t)(chunk >> 32), stream_id, 0u), seed_lo, seed_hi);
+BSQ_DEV uint4 mx_draws(uint64_t chunk, const PhiloxKeys &keys, uint32_t stream_id) {
+    return philox4x32_10(make_uint4((uint32_t)chunk, (uint32_t)(chunk >> 32), stream_id, 0u), keys);
 }
 
 // True when stochastic rounding of the 8 scaled values cannot depend on the
@@ -661,22 +668,33 @@ BSQ_DEV bool mx_sr8_drawless(const float s[8]) {
     return ok;
 }
 
+// Philox draws and rounding of one chunk, out of line (the rare case of the
+// EXACT_IN path below).
+__device__ __noinline__ uint2 mx_sr8_drawn(float s0, float s1, float s2, float s3, float s4, float s5, float s6,
+                                           float s7, uint64_t chunk, const PhiloxKeys &keys,
+                                           uint32_t stream_id) {
+    const float s[8] = {s0, s1, s2, s3, s4, s5, s6, s7};
+    return mx_sr8(s, mx_draws(chunk, keys, stream_id));
+}
+
 // The 8 codes of one chunk of a block with E8M0 code sb (zero: the block's
 // maximum is 0, whose codes are all +0).  chunk is the output linear index
 // of the chunk's first element divided by 8: the Philox counter of SR.  With
 // EXACT_IN (inputs that are E4M3 values times a power of two) the Philox call
 // runs only for chunks whose rounding can depend on it.
 template <bool SR, bool EXACT_IN = false>
-BSQ_DEV uint2 mx_encode8(const float v[8], bool zero, uint32_t sb, uint64_t chunk, uint32_t seed_lo,
-                         uint32_t seed_hi, uint32_t stream_id) {
+BSQ_DEV uint2 mx_encode8(const float v[8], bool zero, uint32_t sb, uint64_t chunk, const PhiloxKeys &keys,
+                         uint32_t stream_id) {
     float s[8];
     mx_scale8(v, mx_inv_scale(sb), s);
     uint2 q;
     if (SR) {
-        if (EXACT_IN && mx_sr8_drawless(s))
+        if (!EXACT_IN)
+            q = mx_sr8(s, mx_draws(chunk, keys, stream_id));
+        else if (mx_sr8_drawless(s))
             q = mx_sr8(s, make_uint4(0u, 0u, 0u, 0u));
         else
-            q = mx_sr8(s, mx_draws(chunk, seed_lo, seed_hi, stream_id));
+            q = mx_sr8_drawn(s[0], s[1], s[2], s[3], s[4], s[5], s[6], s[7], chunk, keys, stream_id);
     } else {
         q = mx_rne8(s);
     }
@@ -743,14 +761,14 @@ BSQ_DEV uint2 mx_sr8_bf16(const uint32_t p[4], const uint32_t a[4], uint32_t sb,
             v[2 * k + 1] = bf16_hi(p[k]);
         }
         mx_scale8(v, mx_inv_scale(sb), s);
-        return mx_sr8(s, rnd);
+        return mx_sr8_float(s[0], s[1], s[2], s[3], s[4], s[5], s[6], s[7], rnd);
     }
     return make_uint2(__byte_perm(u[0], u[1], 0x7531u), __byte_perm(u[2], u[3], 0x7531u));
 }
 // Row-wise: one thread per 8 elements, 4 lanes per block of 32.
 template <bool SR>
 __global__ void __launch_bounds__(256) quant_mxfp8_row_kernel(
-    const uint16_t *__restrict__ x, int64_t M, int64_t K, int64_t ldx, uint32_t seed_lo, uint32_t seed_hi,
+    const uint16_t *__restrict__ x, int64_t M, int64_t K, int64_t ldx, const __grid_constant__ PhiloxKeys keys,
     uint32_t stream_id, uint8_t *__restrict__ codes, uint8_t *__restrict__ sf, RowMap map) {
     const int64_t K8 = K >> 3, KB = K >> 5;
     const bool pack4 = (KB & 3) == 0;
@@ -776,7 +794,7 @@ __global__ void __launch_bounds__(256) quant_mxfp8_row_kernel(
             const bool zero = (m == 0.0f);
             const uint32_t sb = mx_scale_code(m);
             const uint64_t chunk = (uint64_t)(rr * K + cc * 8) >> 3;
-            uint2 q = mx_encode8<SR>(v, zero, sb, chunk, seed_lo, seed_hi, stream_id);
+            uint2 q = mx_encode8<SR>(v, zero, sb, chunk, keys, stream_id);
             if (valid) *reinterpret_cast<uint2 *>(codes + rr * K + cc * 8) = q;
             // scale byte: lanes 4j hold block j; 4 blocks (16 lanes) per word
             const int64_t kb = cc >> 2;
@@ -818,7 +836,7 @@ BSQ_DEV uint32_t divu32(uint32_t n, const DivU32 &dv) {
 
 template <bool SR>
 __global__ void __launch_bounds__(256) quant_mxfp8_row_flat_kernel(
-    const uint16_t *__restrict__ x, int64_t nchunk, int64_t K, DivU32 div_k8, uint32_t seed_lo, uint32_t seed_hi,
+    const uint16_t *__restrict__ x, int64_t nchunk, int64_t K, DivU32 div_k8, const __grid_constant__ PhiloxKeys keys,
     uint32_t stream_id, uint8_t *__restrict__ codes, uint8_t *__restrict__ sf) {
     constexpr int U = 4;
     const int64_t K8 = K >> 3, KB = K >> 5;
@@ -850,7 +868,7 @@ __global__ void __launch_bounds__(256) quant_mxfp8_row_flat_kernel(
             m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
             const bool zero = (m == 0.0f);
             const uint32_t sb = mx_scale_code(m);
-            const uint2 q = mx_encode8<SR>(v, zero, sb, (uint64_t)cc, seed_lo, seed_hi, stream_id);
+            const uint2 q = mx_encode8<SR>(v, zero, sb, (uint64_t)cc, keys, stream_id);
             if (valid) *reinterpret_cast<uint2 *>(codes + cc * 8) = q;
             const uint32_t b1 = __shfl_down_sync(0xFFFFFFFFu, sb, 4);
             const uint32_t b2 = __shfl_down_sync(0xFFFFFFFFu, sb, 8);
@@ -873,7 +891,7 @@ __global__ void __launch_bounds__(256) quant_mxfp8_row_flat_kernel(
 // chunk is its flat position.
 template <bool SR>
 __global__ void __launch_bounds__(256) quant_mxfp8_row_span_kernel(
-    const uint16_t *__restrict__ x, uint32_t nspan, int64_t K, DivU32 div_spr, uint32_t seed_lo, uint32_t seed_hi,
+    const uint16_t *__restrict__ x, uint32_t nspan, int64_t K, DivU32 div_spr, const __grid_constant__ PhiloxKeys keys,
     uint32_t stream_id, uint8_t *__restrict__ codes, uint8_t *__restrict__ sf) {
     const int lane = threadIdx.x & 31;
     const uint32_t spr = (uint32_t)(K >> 10);  // spans per row
@@ -901,7 +919,7 @@ __global__ void __launch_bounds__(256) quant_mxfp8_row_span_kernel(
                 m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
                 m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
                 sb = mx_scale_code_bf16(m);
-                const uint2 q = mx_sr8_bf16(w, a, sb, mx_draws(chunk0 + 32 * h, seed_lo, seed_hi, stream_id));
+                const uint2 q = mx_sr8_bf16(w, a, sb, mx_draws(chunk0 + 32 * h, keys, stream_id));
                 dst[32 * h] = (m == 0u) ? make_uint2(0u, 0u) : q;
             } else {
                 float v[8];
@@ -915,7 +933,7 @@ __global__ void __launch_bounds__(256) quant_mxfp8_row_span_kernel(
                 m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
                 m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
                 sb = mx_scale_code(m);
-                dst[32 * h] = mx_encode8<false>(v, m == 0.0f, sb, 0, 0u, 0u, 0u);
+                dst[32 * h] = mx_encode8<false>(v, m == 0.0f, sb, 0, keys, 0u);
             }
             if (sf_lane) sfp[h * 1024] = (uint8_t)sb;
         }
@@ -934,7 +952,7 @@ __global__ void __launch_bounds__(256) quant_mxfp8_row_span_kernel(
 template <bool FROM_MX, bool SR>
 __global__ void __launch_bounds__(256) quant_mxfp8_col_kernel(
     const void *__restrict__ xin, const uint8_t *__restrict__ sf_in, int64_t M, int64_t K, int64_t ldx,
-    uint32_t ntile, DivU32 div_mt, uint32_t seed_lo, uint32_t seed_hi, uint32_t stream_id,
+    uint32_t ntile, DivU32 div_mt, const __grid_constant__ PhiloxKeys keys, uint32_t stream_id,
     uint8_t *__restrict__ codes, uint8_t *__restrict__ sf) {
     const int lane = threadIdx.x & 31, kg = lane >> 2, mg = lane & 3;
     const uint32_t mt_n = (uint32_t)(M >> 5);
@@ -977,7 +995,7 @@ __global__ void __launch_bounds__(256) quant_mxfp8_col_kernel(
                 m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
                 m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
                 const uint32_t sb = mx_scale_code_bf16(m);
-                uint2 q = mx_sr8_bf16(p, a, sb, mx_draws((uint64_t)(k * M + m0) >> 3, seed_lo, seed_hi, stream_id));
+                uint2 q = mx_sr8_bf16(p, a, sb, mx_draws((uint64_t)(k * M + m0) >> 3, keys, stream_id));
                 if (m == 0u) q = make_uint2(0u, 0u);
                 if (kvalid) {
                     *reinterpret_cast<uint2 *>(codes + k * M + m0) = q;
@@ -1005,7 +1023,7 @@ __global__ void __launch_bounds__(256) quant_mxfp8_col_kernel(
             m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
             const uint32_t sb = mx_scale_code(m);
             const uint2 q =
-                mx_encode8<SR, FROM_MX>(v, m == 0.0f, sb, (uint64_t)(k * M + m0) >> 3, seed_lo, seed_hi, stream_id);
+                mx_encode8<SR, FROM_MX>(v, m == 0.0f, sb, (uint64_t)(k * M + m0) >> 3, keys, stream_id);
             if (kvalid) {
                 *reinterpret_cast<uint2 *>(codes + k * M + m0) = q;
                 if (mg == 0) sf[sf_offset(k, m0 >> 5, MB)] = (uint8_t)sb;
@@ -1168,16 +1186,16 @@ int launch_quant_nvfp4_fused(const uint16_t *x, int64_t M, int64_t K, bool block
 void launch_quant_mxfp8(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, bool colwise, bool sr,
                         uint64_t seed, uint32_t stream_id, uint8_t *codes, uint8_t *sf, int num_sms,
                         cudaStream_t s) {
-    const uint32_t lo = (uint32_t)seed, hi = (uint32_t)(seed >> 32);
+    const PhiloxKeys keys = philox_keys((uint32_t)seed, (uint32_t)(seed >> 32));
     if (!colwise && ldx == K && K % 1024 == 0 && M * (K >> 10) < (int64_t(1) << 31)) {
         const uint32_t nspan = (uint32_t)(M * (K >> 10));
         const DivU32 dspr = divu32_for((uint32_t)(K >> 10));
         if (sr) {
             const int grid = grid_for(nspan, 8, resident_ctas<quant_mxfp8_row_span_kernel<true>>(num_sms));
-            quant_mxfp8_row_span_kernel<true><<<grid, 256, 0, s>>>(x, nspan, K, dspr, lo, hi, stream_id, codes, sf);
+            quant_mxfp8_row_span_kernel<true><<<grid, 256, 0, s>>>(x, nspan, K, dspr, keys, stream_id, codes, sf);
         } else {
             const int grid = grid_for(nspan, 8, resident_ctas<quant_mxfp8_row_span_kernel<false>>(num_sms));
-            quant_mxfp8_row_span_kernel<false><<<grid, 256, 0, s>>>(x, nspan, K, dspr, lo, hi, stream_id, codes, sf);
+            quant_mxfp8_row_span_kernel<false><<<grid, 256, 0, s>>>(x, nspan, K, dspr, keys, stream_id, codes, sf);
         }
         return;
     }
@@ -1186,10 +1204,10 @@ void launch_quant_mxfp8(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, bo
         const DivU32 dk8 = divu32_for((uint32_t)(K >> 3));
         if (sr) {
             const int grid = grid_for(nchunk, 4 * 256, resident_ctas<quant_mxfp8_row_flat_kernel<true>>(num_sms));
-            quant_mxfp8_row_flat_kernel<true><<<grid, 256, 0, s>>>(x, nchunk, K, dk8, lo, hi, stream_id, codes, sf);
+            quant_mxfp8_row_flat_kernel<true><<<grid, 256, 0, s>>>(x, nchunk, K, dk8, keys, stream_id, codes, sf);
         } else {
             const int grid = grid_for(nchunk, 4 * 256, resident_ctas<quant_mxfp8_row_flat_kernel<false>>(num_sms));
-            quant_mxfp8_row_flat_kernel<false><<<grid, 256, 0, s>>>(x, nchunk, K, dk8, lo, hi, stream_id, codes, sf);
+            quant_mxfp8_row_flat_kernel<false><<<grid, 256, 0, s>>>(x, nchunk, K, dk8, keys, stream_id, codes, sf);
         }
         return;
     }
@@ -1197,19 +1215,19 @@ void launch_quant_mxfp8(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, bo
         RowMap map{lpr_shift_for(K >> 3)};
         if (map.lpr_shift < 2) map.lpr_shift = 2;  // 4 lanes per block of 32
         const int grid = grid_for(M, 256 >> map.lpr_shift, num_sms * 8);
-        if (sr) quant_mxfp8_row_kernel<true><<<grid, 256, 0, s>>>(x, M, K, ldx, lo, hi, stream_id, codes, sf, map);
-        else quant_mxfp8_row_kernel<false><<<grid, 256, 0, s>>>(x, M, K, ldx, lo, hi, stream_id, codes, sf, map);
+        if (sr) quant_mxfp8_row_kernel<true><<<grid, 256, 0, s>>>(x, M, K, ldx, keys, stream_id, codes, sf, map);
+        else quant_mxfp8_row_kernel<false><<<grid, 256, 0, s>>>(x, M, K, ldx, keys, stream_id, codes, sf, map);
         return;
     }
     const uint32_t ntile = (uint32_t)((M >> 5) * ((K + 63) >> 6));
     const DivU32 dmt = divu32_for((uint32_t)(M >> 5));
     if (sr) {
         const int grid = grid_for(ntile, 8, resident_ctas<quant_mxfp8_col_kernel<false, true>>(num_sms));
-        quant_mxfp8_col_kernel<false, true><<<grid, 256, 0, s>>>(x, nullptr, M, K, ldx, ntile, dmt, lo, hi,
+        quant_mxfp8_col_kernel<false, true><<<grid, 256, 0, s>>>(x, nullptr, M, K, ldx, ntile, dmt, keys,
                                                                  stream_id, codes, sf);
     } else {
         const int grid = grid_for(ntile, 8, resident_ctas<quant_mxfp8_col_kernel<false, false>>(num_sms));
-        quant_mxfp8_col_kernel<false, false><<<grid, 256, 0, s>>>(x, nullptr, M, K, ldx, ntile, dmt, lo, hi,
+        quant_mxfp8_col_kernel<false, false><<<grid, 256, 0, s>>>(x, nullptr, M, K, ldx, ntile, dmt, keys,
                                                                   stream_id, codes, sf);
     }
 }
@@ -1217,16 +1235,16 @@ void launch_quant_mxfp8(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, bo
 void launch_requant_transpose(const uint8_t *codes_row, const uint8_t *sf_row, int64_t M, int64_t K, bool sr,
                               uint64_t seed, uint32_t stream_id, uint8_t *codes_col, uint8_t *sf_col,
                               int num_sms, cudaStream_t s) {
-    const uint32_t lo = (uint32_t)seed, hi = (uint32_t)(seed >> 32);
+    const PhiloxKeys keys = philox_keys((uint32_t)seed, (uint32_t)(seed >> 32));
     const uint32_t ntile = (uint32_t)((M >> 5) * ((K + 63) >> 6));
     const DivU32 dmt = divu32_for((uint32_t)(M >> 5));
     if (sr) {
         const int grid = grid_for(ntile, 8, resident_ctas<quant_mxfp8_col_kernel<true, true>>(num_sms));
-        quant_mxfp8_col_kernel<true, true><<<grid, 256, 0, s>>>(codes_row, sf_row, M, K, K, ntile, dmt, lo, hi,
+        quant_mxfp8_col_kernel<true, true><<<grid, 256, 0, s>>>(codes_row, sf_row, M, K, K, ntile, dmt, keys,
                                                                 stream_id, codes_col, sf_col);
     } else {
         const int grid = grid_for(ntile, 8, resident_ctas<quant_mxfp8_col_kernel<true, false>>(num_sms));
-        quant_mxfp8_col_kernel<true, false><<<grid, 256, 0, s>>>(codes_row, sf_row, M, K, K, ntile, dmt, lo, hi,
+        quant_mxfp8_col_kernel<true, false><<<grid, 256, 0, s>>>(codes_row, sf_row, M, K, K, ntile, dmt, keys,
                                                                  stream_id, codes_col, sf_col);
     }
 }

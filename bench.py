@@ -235,7 +235,7 @@ def measure_rows(hbm, fp4_peak, fp8_peak, reps=10, only=None):
             rows.append({"row": name, "workload": workload, "error": str(e)[:200]})
 
     if wants("a1 amax (RHT)", "a2+a5 NVFP4 1x16 quantize (amax + RHT fused)", "a3+a5 NVFP4 16x16 quantize (amax + RHT fused)", "a5 RHT standalone (bf16 -> bf16)", "a8 NVFP4 GEMM bf16"):
-        # -- configs[2]: linear with RHT (the timed step's calls, one at a time)
+        # -- NVFP4 linear with RHT, A 8192x4096, W 14336x4096 (the timed step's calls, one at a time)
         A_h, W_h, seed = W.nvfp4_linear_rht()
         mask = bsq.bsq_rht_sign_mask(seed)
         A, Wd = A_h.to(dev), W_h.to(dev)
@@ -258,7 +258,7 @@ def measure_rows(hbm, fp4_peak, fp8_peak, reps=10, only=None):
             flops=2 * M2 * N2 * K2, peak_kind="fp4")
         del y, C2
     if wants("a2+a3+a8 small linear step (latency)"):
-        # -- configs[0]: the small NVFP4 linear (latency)
+        # -- the small NVFP4 linear, A 128x256, W 256x256 (latency)
         As, Ws = W.nvfp4_linear_small()
         As, Ws = As.to(dev), Ws.to(dev)
         qas, qws = api.quant_nvfp4(As), api.quant_nvfp4(Ws, block_2d=True)
@@ -271,7 +271,7 @@ def measure_rows(hbm, fp4_peak, fp8_peak, reps=10, only=None):
         row("a2+a3+a8 small linear step (latency)", "A 128x256, W 256x256, fp32 out", small_step,
             nbytes=(128 + 256) * 256 * 2)
     if wants("a6 MXFP8 row quantize RNE", "a6 MXFP8 row quantize SR (Philox)", "a7 requant-transpose SR"):
-        # -- configs[1]: MXFP8 4096^2 Student-t, RNE and SR, requant-transpose
+        # -- MXFP8 4096x4096 Student-t: RNE and SR, requant-transpose
         X1 = W.mxfp8_requant().to(dev)
         M1, K1 = X1.shape
         q1 = api.quant_mxfp8(X1)
@@ -285,7 +285,7 @@ def measure_rows(hbm, fp4_peak, fp8_peak, reps=10, only=None):
             lambda: api.requant_transpose(q1s[0], q1s[1], sr=True, seed=1, out=qt), nbytes=2 * M1 * K1 * (1 + 1 / 32))
         del X1, q1, q1s, qt
     if wants("a6 MXFP8 row quantize SR", "a6 MXFP8 column quantize SR", "a8 MXFP8 GEMM dgrad (bf16 out)", "a8 MXFP8 GEMM wgrad (fp32 out)", "a8 NVFP4 rollout GEMM (swap-AB, HBM-bound)"):
-        # -- configs[4]: MXFP8 backward + rollout
+        # -- MXFP8 backward (dY 8192x14336, W 14336x4096, X 8192x4096) + NVFP4 rollout
         dY, W4, X4, A_roll = W.mxfp8_backward()
         dY, W4, X4 = dY.to(dev), W4.to(dev), X4.to(dev)
         M4, N4 = dY.shape
@@ -317,7 +317,7 @@ def measure_rows(hbm, fp4_peak, fp8_peak, reps=10, only=None):
             nbytes=N4 * K4 // 2 + N4 * K4 // 16 + 64 * K4 // 2 + 64 * K4 // 16 + 64 * N4 * 2)
         del Cr, qar, qwr, W4, qwc
     if wants("a4 NVFP4 Four Over Six quantize (gathered, expert groups)", "a9 grouped NVFP4 GEMM up", "a9 grouped NVFP4 GEMM down"):
-        # -- configs[3]: MoE forward (gathered 4/6 quantize, grouped up and down)
+        # -- MoE forward, 16384 tokens, 64 experts, top-8 (gathered 4/6 quantize, grouped up and down)
         moe = W.moe_forward()
         T3, H3 = moe.X.shape
         E3, F3, _ = moe.W_up.shape

@@ -55,7 +55,7 @@ enum {
     BSQ_OK = 0,
     BSQ_ERR_INVALID = 1,     /* bad size, null pointer or option mix */
     BSQ_ERR_ALIGN = 2,       /* pointer or leading dimension misaligned */
-    BSQ_ERR_UNSUPPORTED = 3, /* valid request this build does not handle */
+    BSQ_ERR_UNSUPPORTED = 3, /* valid request the library does not handle */
     BSQ_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed */
     BSQ_ERR_TIMEOUT = 5      /* a device-side bounded wait ran out */
 };

@@ -1,6 +1,6 @@
 /*
  * bsq_oracle.c -- the plain, slow, scalar CPU oracle for block-scaled
- * quantization (NVFP4, MXFP8), the 16-point random Hadamard transform and the
+ * quantization (NVFP4, MXFP8, MXFP4), the 16-point random Hadamard transform and the
  * block-scaled GEMM.
  *
  * TEST INFRASTRUCTURE ONLY.  The tests, the package's smoke check and the
@@ -241,6 +241,30 @@ uint8_t ora_e4m3_sr(float v, uint16_t r16)
 }
 
 /* ------------------------------------------------------------------------ */
+/* Stochastic rounding to E2M1 -- [MX] "NVFP4": the NVFP4 pretraining recipe */
+/* rounds gradients stochastically; [MX] "Words on this page": round up or   */
+/* down at random in proportion to closeness.  Same rule and draws as the    */
+/* E4M3 form (R12): with lo <= |v| < hi the neighbouring E2M1 values, round   */
+/* up iff r16 * 2^-16 < (|v| - lo) / (hi - lo).  v must already be clamped to */
+/* [-6, 6]; the sign bit is the sign of v (R5).                              */
+/* ------------------------------------------------------------------------ */
+
+uint8_t ora_e2m1_sr(float v, uint16_t r16)
+{
+    uint8_t s = signbit(v) ? 8 : 0;
+    float a = fabsf(v);
+    uint8_t c = 0;
+    while (c < 7 && ora_e2m1_value((uint8_t)(c + 1)) <= a)
+        c++;                                   /* E2M1(c) <= a < E2M1(c + 1) */
+    if (c == 7)
+        return (uint8_t)(s | 7);
+    float lo = ora_e2m1_value(c), hi = ora_e2m1_value((uint8_t)(c + 1));
+    float frac = (a - lo) / (hi - lo);         /* exact: the gap is 0.5, 1 or 2 */
+    float u = (float)r16 * (1.0f / 65536.0f);
+    return (uint8_t)(s | ((u < frac) ? c + 1 : c));
+}
+
+/* ------------------------------------------------------------------------ */
 /* 16-point random Hadamard transform -- [MX] "NVFP4": random Hadamard       */
 /* transforms bound block outliers; [TML] "Why communication became the next */
 /* bottleneck": a random Hadamard rotation that the receiver reverses.       */
@@ -386,12 +410,17 @@ float ora_nvfp4_global_scale(float amax)
     return (amax == 0.0f) ? 1.0f : amax / 2688.0f;
 }
 
-int ora_quant_nvfp4(const uint16_t *x, int64_t M, int64_t K, int64_t ldx,
-                    int block_2d, int four_over_six, int rht, uint16_t mask,
-                    const int32_t *row_index, const float *amax_in,
-                    float *s_g_out, uint8_t *codes, uint8_t *sf)
+/* sr != 0: the elements are rounded stochastically instead (ora_e2m1_sr of
+ * x * r clamped to +-6, the draw of output element m * K + k with the given
+ * seed and stream id); block scales and s_g are unchanged.  Not combined with
+ * Four Over Six. */
+static int quant_nvfp4_impl(const uint16_t *x, int64_t M, int64_t K, int64_t ldx,
+                            int block_2d, int four_over_six, int rht, uint16_t mask,
+                            const int32_t *row_index, const float *amax_in,
+                            int sr, uint64_t seed, uint32_t stream_id,
+                            float *s_g_out, uint8_t *codes, uint8_t *sf)
 {
-    if (K % 16 || (block_2d && M % 16) || (block_2d && four_over_six))
+    if (K % 16 || (block_2d && M % 16) || (block_2d && four_over_six) || (sr && four_over_six))
         return 1;
     float amax = amax_in ? *amax_in : ora_amax(x, M, K, ldx, rht, mask, row_index);
     float s_g = ora_nvfp4_global_scale(amax);
@@ -423,6 +452,17 @@ int ora_quant_nvfp4(const uint16_t *x, int64_t M, int64_t K, int64_t ldx,
                         pick = &c4;
                 }
                 int64_t m = m0 + r;
+                if (sr && c6.den != 0.0f) {
+                    float rc = 1.0f / c6.den;
+                    for (int i = 0; i < 16; i++) {
+                        float q = xb[i] * rc;
+                        if (q > 6.0f)
+                            q = 6.0f;
+                        if (q < -6.0f)
+                            q = -6.0f;
+                        c6.code[i] = ora_e2m1_sr(q, ora_sr_draw(seed, stream_id, (uint64_t)(m * K + kb * 16 + i)));
+                    }
+                }
                 sf[m * KB + kb] = pick->sb;
                 for (int i = 0; i < 16; i += 2)
                     codes[m * (K / 2) + kb * 8 + i / 2] =
@@ -431,6 +471,81 @@ int ora_quant_nvfp4(const uint16_t *x, int64_t M, int64_t K, int64_t ldx,
         }
     }
     free(buf);
+    return 0;
+}
+
+int ora_quant_nvfp4(const uint16_t *x, int64_t M, int64_t K, int64_t ldx,
+                    int block_2d, int four_over_six, int rht, uint16_t mask,
+                    const int32_t *row_index, const float *amax_in,
+                    float *s_g_out, uint8_t *codes, uint8_t *sf)
+{
+    return quant_nvfp4_impl(x, M, K, ldx, block_2d, four_over_six, rht, mask, row_index, amax_in,
+                            0, 0, 0, s_g_out, codes, sf);
+}
+
+int ora_quant_nvfp4_sr(const uint16_t *x, int64_t M, int64_t K, int64_t ldx,
+                       int block_2d, int rht, uint16_t mask,
+                       const int32_t *row_index, const float *amax_in,
+                       uint64_t seed, uint32_t stream_id,
+                       float *s_g_out, uint8_t *codes, uint8_t *sf)
+{
+    return quant_nvfp4_impl(x, M, K, ldx, block_2d, 0, rht, mask, row_index, amax_in,
+                            1, seed, stream_id, s_g_out, codes, sf);
+}
+
+/* ------------------------------------------------------------------------ */
+/* MXFP4 quantize -- [FP4] "The two Blackwell formats": E2M1 elements in     */
+/* groups of 32 with one E8M0 (power-of-two) scale, 4 + 8/32 = 4.25 bits;    */
+/* [MX] "Microscaling": the block shares one exponent.  R28 (the pages give  */
+/* no scale rule): as MXFP8's 2^(floor(log2 amax) - 8), with E2M1's largest  */
+/* exponent in place of E4M3's -- 6 = 1.5 * 2^2 -- so E = floor(log2 amax)   */
+/* - 2, clamped to [-127, 127]; elements x * 2^-E clamped to +-6 (values in  */
+/* (6, 8) * 2^E saturate), then nearest-even or stochastic rounding (draw of */
+/* output element r * K + k).  An all-zero block has scale code 0 and codes  */
+/* +0.  Outputs: codes [M][K/2] (element 2j in the low nibble of byte j),    */
+/* sf [M][K/32] canonical E8M0 codes.                                         */
+/* ------------------------------------------------------------------------ */
+
+int ora_quant_mxfp4(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, int sr,
+                    uint64_t seed, uint32_t stream_id, uint8_t *codes, uint8_t *sf)
+{
+    if (K % 32)
+        return 1;
+    for (int64_t r = 0; r < M; r++) {
+        for (int64_t kb = 0; kb < K / 32; kb++) {
+            float v[32], bamax = 0.0f;
+            for (int i = 0; i < 32; i++) {
+                v[i] = ora_bf16_to_f32(x[r * ldx + kb * 32 + i]);
+                if (fabsf(v[i]) > bamax)
+                    bamax = fabsf(v[i]);
+            }
+            uint8_t c[32];
+            if (bamax == 0.0f) {
+                sf[r * (K / 32) + kb] = 0;
+                memset(c, 0, sizeof c);
+            } else {
+                int e2;
+                frexpf(bamax, &e2);
+                int E = (e2 - 1) - 2;
+                if (E < -127)
+                    E = -127;
+                if (E > 127)
+                    E = 127;
+                sf[r * (K / 32) + kb] = (uint8_t)(E + 127);
+                for (int i = 0; i < 32; i++) {
+                    float q = ldexpf(v[i], -E);
+                    if (q > 6.0f)
+                        q = 6.0f;
+                    if (q < -6.0f)
+                        q = -6.0f;
+                    c[i] = sr ? ora_e2m1_sr(q, ora_sr_draw(seed, stream_id, (uint64_t)(r * K + kb * 32 + i)))
+                              : ora_e2m1_rne_sat(q);
+                }
+            }
+            for (int i = 0; i < 32; i += 2)
+                codes[r * (K / 2) + kb * 16 + i / 2] = (uint8_t)(c[i] | (c[i + 1] << 4));
+        }
+    }
     return 0;
 }
 
@@ -593,6 +708,11 @@ static double decode_one(int fmt, const uint8_t *codes, const uint8_t *sf, float
         uint8_t byte = codes[r * (K / 2) + k / 2];
         uint8_t c = (k & 1) ? (uint8_t)(byte >> 4) : (uint8_t)(byte & 15);
         return (double)ora_e2m1_value(c) * (double)ora_e4m3_value(sf[r * (K / 16) + k / 16]) * (double)s_g;
+    }
+    if (fmt == 2) { /* MXFP4 */
+        uint8_t byte = codes[r * (K / 2) + k / 2];
+        uint8_t c = (k & 1) ? (uint8_t)(byte >> 4) : (uint8_t)(byte & 15);
+        return (double)ora_e2m1_value(c) * (double)ora_e8m0_value(sf[r * (K / 32) + k / 32]);
     }
     return (double)ora_e4m3_value(codes[r * K + k]) * (double)ora_e8m0_value(sf[r * (K / 32) + k / 32]);
 }

@@ -60,6 +60,7 @@ def lib():
                 "ora_e4m3_rne_sat": (C.c_uint8, [C.c_float]),
                 "ora_e8m0_value": (C.c_float, [C.c_uint8]),
                 "ora_e4m3_sr": (C.c_uint8, [C.c_float, C.c_uint16]),
+                "ora_e2m1_sr": (C.c_uint8, [C.c_float, C.c_uint16]),
                 "ora_philox4x32_10": (None, [_u32p, _u32p, _u32p]),
                 "ora_sr_draw": (C.c_uint16, [C.c_uint64, C.c_uint32, C.c_uint64]),
                 "ora_rht_sign_mask": (C.c_uint16, [C.c_uint64]),
@@ -69,6 +70,11 @@ def lib():
                 "ora_nvfp4_global_scale": (C.c_float, [C.c_float]),
                 "ora_quant_nvfp4": (C.c_int, [_u16p, _i64, _i64, _i64, C.c_int, C.c_int, C.c_int,
                                               C.c_uint16, C.c_void_p, C.c_void_p, _f32p, _u8p, _u8p]),
+                "ora_quant_nvfp4_sr": (C.c_int, [_u16p, _i64, _i64, _i64, C.c_int, C.c_int, C.c_uint16,
+                                                 C.c_void_p, C.c_void_p, C.c_uint64, C.c_uint32, _f32p, _u8p,
+                                                 _u8p]),
+                "ora_quant_mxfp4": (C.c_int, [_u16p, _i64, _i64, _i64, C.c_int, C.c_uint64, C.c_uint32,
+                                              _u8p, _u8p]),
                 "ora_quant_mxfp8": (C.c_int, [_u16p, _i64, _i64, _i64, C.c_int, C.c_int,
                                               C.c_uint64, C.c_uint32, _u8p, _u8p]),
                 "ora_quant_mxfp8_rows": (C.c_int, [_u16p, _i64, _i64, _i64, C.c_int, C.c_int,
@@ -128,6 +134,10 @@ def e4m3_rne_sat(v):
 
 def e8m0_value(code):
     return lib().ora_e8m0_value(int(code))
+
+
+def e2m1_sr(v, r16):
+    return lib().ora_e2m1_sr(float(v), int(r16))
 
 
 def e4m3_sr(v, r16):
@@ -194,6 +204,36 @@ def quant_nvfp4(x, block_2d=False, four_over_six=False, rht_mask=None, row_index
     return codes, sf, float(sg[0])
 
 
+def quant_nvfp4_sr(x, block_2d=False, rht_mask=None, row_index=None, amax_in=None, seed=0, stream_id=0):
+    """NVFP4 quantize with stochastic rounding of the elements
+    (ora_quant_nvfp4_sr).  Returns (codes [R,K/2] u8, sf [R,K/16] u8, s_g)."""
+    x = _c(x, np.uint16)
+    M, K = x.shape
+    ri = None if row_index is None else _c(row_index, np.int32)
+    R = M if ri is None else ri.shape[0]
+    codes = np.zeros((R, K // 2), np.uint8)
+    sf = np.zeros((R, K // 16), np.uint8)
+    sg = np.zeros(1, np.float32)
+    am = None if amax_in is None else np.array([amax_in], np.float32)
+    rc = lib().ora_quant_nvfp4_sr(x, R, K, K, int(block_2d), int(rht_mask is not None), int(rht_mask or 0),
+                                  _ptr(ri), _ptr(am), int(seed), int(stream_id), sg, codes, sf)
+    if rc:
+        raise ValueError("unsupported NVFP4 shape/options")
+    return codes, sf, float(sg[0])
+
+
+def quant_mxfp4(x, sr=False, seed=0, stream_id=0):
+    """MXFP4 quantize (ora_quant_mxfp4), row-wise blocks of 32 along K.
+    Returns (codes [M,K/2] u8, sf [M,K/32] u8)."""
+    x = _c(x, np.uint16)
+    M, K = x.shape
+    codes = np.zeros((M, K // 2), np.uint8)
+    sf = np.zeros((M, K // 32), np.uint8)
+    if lib().ora_quant_mxfp4(x, M, K, K, int(sr), int(seed), int(stream_id), codes, sf):
+        raise ValueError("unsupported MXFP4 shape")
+    return codes, sf
+
+
 def quant_mxfp8(x, colwise=False, sr=False, seed=0, stream_id=0, out_row0=0):
     """MXFP8 quantize (ora_quant_mxfp8_rows).  Returns (codes, sf) in the output
     orientation.  out_row0: index of the first output row within the full
@@ -244,14 +284,14 @@ def sf_unswizzle(buf, rows, nblk):
 
 
 # ---------------------------------------------------------------- GEMM
-NVFP4, MXFP8 = 0, 1
+NVFP4, MXFP8, MXFP4 = 0, 1, 2
 
 
 def dequant(fmt, codes, sf, s_g=1.0):
     codes = _c(codes, np.uint8)
     sf = _c(sf, np.uint8)
     R = codes.shape[0]
-    K = codes.shape[1] * (2 if fmt == NVFP4 else 1)
+    K = codes.shape[1] * (1 if fmt == MXFP8 else 2)
     out = np.zeros((R, K), np.float64)
     lib().ora_dequant(int(fmt), codes, sf, float(s_g), R, K, out)
     return out

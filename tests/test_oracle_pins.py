@@ -609,3 +609,205 @@ def test_dequant_and_gemm_points_vs_library_decode(ora, fmt):
     pm, pn = W.sample_points(64, 48, 50)
     Cp, Rp = ora.gemm_points(fmt, qa, qb, 256, pm, pn)
     assert np.array_equal(Cp, Cm[pm, pn]) and np.array_equal(Rp, Ra[pm, pn])
+
+
+# --------------------------------------------------------------------- FP4 SR, MXFP4
+def _e2m1_neighbours(a, nonneg):
+    """Grid values lo <= a < hi from the page's list (a in [0, 6))."""
+    i = max(j for j, g in enumerate(nonneg) if g <= a)
+    return nonneg[i], nonneg[i + 1]
+
+
+@pytest.mark.parametrize("v", [0.3, 1.25, 2.7, 4.5, 5.999, -0.1, -3.3, 0.5, 6.0, 1.0 + 2.0 ** -20])
+def test_e2m1_sr_exhaustive_probability(ora, v):
+    """MX page "NVFP4" (stochastic rounding of gradients) and "Words on this
+    page" (round up or down in proportion to closeness): over all 65536 draws
+    the outcomes are the two neighbours on the page's E2M1 list and the number
+    of round-ups is frac * 2^16 rounded up (R12's rule)."""
+    _, nonneg = _e2m1_table_from_pages()
+    v32 = float(np.float32(v))
+    codes = np.array([ora.e2m1_sr(v32, r) for r in range(65536)], np.uint8)
+    vals = np.array([ora.e2m1_value(int(c)) for c in np.unique(codes)])
+    a = abs(v32)
+    sgn = -1.0 if v32 < 0 else 1.0
+    assert ((codes >> 3) == (1 if v32 < 0 else 0)).all()  # sign kept
+    if a >= 6.0 or a in nonneg:
+        assert set(vals) == {sgn * a}
+        return
+    lo, hi = _e2m1_neighbours(a, nonneg)
+    frac = (a - lo) / (hi - lo)
+    assert set(vals) <= {sgn * lo, sgn * hi}
+    mags = np.array([abs(ora.e2m1_value(int(c))) for c in codes])
+    assert int((mags == hi).sum()) == math.ceil(frac * 65536)
+
+
+def test_mxfp4_bits_per_value_match_pages(ora):
+    """FP4 page table "MXFP4 vs NVFP4": 4 + 8/32 = 4.25 bits per value."""
+    rows = {r[0]: r for r in golden_rows("bits_per_value.txt")}
+    x = W.bf16_bits(W.mxfp8_requant(M=64, K=256))
+    c, s = ora.quant_mxfp4(x)
+    assert (c.nbytes + s.nbytes) * 8 / x.size == float(rows["mxfp4"][4])
+
+
+def test_mxfp4_scale_exponent_rule(ora):
+    """R28: E8M0 scale 2^(floor(log2 amax) - 2), E2M1's top exponent (6 =
+    1.5 x 2^2, FP4 page "Bit layout of FP4 E2M1") in place of MXFP8's 8;
+    checked with math.frexp over Student-t blocks and a zero block."""
+    xt = W.mxfp8_requant(M=64, K=256)
+    xt[3, 64:96] = 0.0
+    x = W.bf16_bits(xt)
+    c, s = ora.quant_mxfp4(x)
+    xf = (x.astype(np.uint32) << 16).view(np.float32).reshape(64, 8, 32)
+    bamax = np.abs(xf).max(-1)
+    for i in range(64):
+        for j in range(8):
+            if bamax[i, j] == 0:
+                assert s[i, j] == 0 and not c[i, j * 16:(j + 1) * 16].any()
+                continue
+            _, e = math.frexp(float(bamax[i, j]))
+            assert int(s[i, j]) == (e - 1) - 2 + 127
+
+
+def _mxfp4_representable(rng, R, K):
+    """Blocks E2M1 x 2^E (values from the page's list) with one element of
+    magnitude 4 or 6 per block, so the block amax fixes E."""
+    _, nonneg = _e2m1_table_from_pages()
+    E = rng.integers(-60, 60, size=(R, K // 32))
+    codes = rng.integers(0, 16, size=(R, K)).astype(np.uint8)
+    for r in range(R):
+        for b in range(K // 32):
+            codes[r, b * 32 + rng.integers(0, 32)] = rng.integers(6, 8) | (rng.integers(0, 2) << 3)
+    mag = np.array(nonneg)[codes & 7]
+    v = np.where(codes & 8, -mag, mag) * np.repeat(2.0 ** E, 32, axis=1)
+    xb = torch.from_numpy(v.astype(np.float32)).to(torch.bfloat16)
+    assert np.array_equal(xb.float().numpy().astype(np.float64), v)
+    return W.bf16_bits(xb), codes, (E + 127).astype(np.uint8)
+
+
+@pytest.mark.parametrize("sr", [False, True])
+def test_mxfp4_round_trip_on_representable_blocks(ora, sr):
+    """MX page "Microscaling" (decode = scale x element): blocks that are
+    already E2M1 x 2^E come back with the same codes and scale, with
+    nearest-even and with stochastic rounding (frac = 0 never rounds)."""
+    rng = np.random.default_rng(21)
+    x, codes, sf = _mxfp4_representable(rng, 16, 256)
+    c, s = ora.quant_mxfp4(x, sr=sr, seed=3)
+    assert np.array_equal(s, sf)
+    got = np.stack([c & 15, c >> 4], axis=-1).reshape(codes.shape)
+    zero = (codes & 7) == 0
+    assert np.array_equal(np.where(zero, 0, got), np.where(zero, 0, codes))
+    d = ora.dequant(ora.MXFP4, c, s)
+    assert np.array_equal(d, (x.astype(np.uint32) << 16).view(np.float32).astype(np.float64))
+
+
+def test_mxfp4_rne_is_nearest_with_ties_even_and_saturation(ora):
+    """Each MXFP4 code is the nearest value on the page's E2M1 list to
+    x * 2^-E clamped to 6 (brute force; ties to the even code), and values
+    past 6 x 2^E store +-6."""
+    _, nonneg = _e2m1_table_from_pages()
+    grid = np.array(nonneg)
+    x = W.bf16_bits(W.mxfp8_requant(M=32, K=256, seed=5))
+    c, s = ora.quant_mxfp4(x)
+    xf = (x.astype(np.uint32) << 16).view(np.float32).astype(np.float64).reshape(32, 8, 32)
+    q = np.abs(xf) / (2.0 ** (s.astype(np.float64) - 127))[..., None]
+    a = np.minimum(q, 6.0).reshape(-1)
+    d = np.abs(a[:, None] - grid[None, :])
+    best = d.min(axis=1)
+    cand = d == best[:, None]
+    want = np.array([(np.nonzero(row)[0][0] if row.sum() == 1 else [i for i in np.nonzero(row)[0] if i % 2 == 0][0])
+                     for row in cand])
+    got = np.stack([c & 7, (c >> 4) & 7], axis=-1).reshape(-1)
+    assert np.array_equal(got, want)
+    assert (got[q.reshape(-1) > 6.0] == 7).all()
+
+
+def test_mxfp4_sr_unbiased_over_seeds(ora):
+    """TML page "A precision choice for each stage": stochastic rounding keeps
+    the expected value -- the seed mean of dequant(SR(x)) is within 5 exact
+    standard errors of the clamped x for every element."""
+    _, nonneg = _e2m1_table_from_pages()
+    x = W.bf16_bits(W.mxfp8_requant(M=4, K=64, seed=13))
+    xf = (x.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    n = 256
+    acc = np.zeros_like(xf)
+    for seed in range(n):
+        c, s = ora.quant_mxfp4(x, sr=True, seed=seed)
+        acc += ora.dequant(ora.MXFP4, c, s)
+    _, s = ora.quant_mxfp4(x)
+    scale = np.repeat(2.0 ** (s.astype(np.float64) - 127), 32, axis=1)
+    t = np.clip(np.abs(xf) / scale, 0, 6.0)
+    sig = np.zeros_like(t)
+    for idx, a in np.ndenumerate(t):
+        if a < 6.0 and a not in nonneg:
+            lo, hi = _e2m1_neighbours(a, nonneg)
+            f = (a - lo) / (hi - lo)
+            sig[idx] = np.sqrt(f * (1 - f)) * (hi - lo)
+    target = np.sign(xf) * t * scale
+    dev = acc / n - target
+    assert (np.abs(dev) <= 5 * sig * scale / np.sqrt(n) + 1e-300).all()
+
+
+def test_nvfp4_sr_keeps_scales_and_rounds_to_neighbours(ora):
+    """MX page "NVFP4": stochastic rounding of the elements only -- s_g and
+    the block scales equal the nearest-even quantization's, and every code is
+    one of the two E2M1 neighbours (page list) of x * r clamped to 6."""
+    _, nonneg = _e2m1_table_from_pages()
+    grid = np.array(nonneg)
+    A, _ = W.nvfp4_linear_small()
+    x = W.bf16_bits(A)
+    c0, s0, g0 = ora.quant_nvfp4(x)
+    c1, s1, g1 = ora.quant_nvfp4_sr(x, seed=7)
+    assert g0 == g1 and np.array_equal(s0, s1)
+    xf = (x.astype(np.uint32) << 16).view(np.float32)
+    den = (_torch_e4m3_value(s0).astype(np.float32) * np.float32(g0)).astype(np.float32)
+    r = (np.float32(1.0) / den).astype(np.float32)
+    q = np.abs(xf.reshape(128, 16, 16) * r[..., None]).astype(np.float64).reshape(-1)
+    a = np.minimum(q, 6.0)
+    got = grid[np.stack([c1 & 7, (c1 >> 4) & 7], axis=-1).reshape(-1)]
+    lo = grid[np.searchsorted(grid, a, side="right") - 1]
+    hi = grid[np.minimum(np.searchsorted(grid, a, side="right"), 7)]
+    assert ((got == lo) | (got == hi)).all()
+    assert (got[a == lo] == lo[a == lo]).all()  # on-grid values never move
+
+
+@pytest.mark.parametrize("block_2d", [False, True])
+def test_nvfp4_sr_round_trip_on_representable_blocks(ora, block_2d):
+    """Representable NVFP4 tensors come back unchanged under stochastic
+    rounding too (frac = 0 everywhere)."""
+    rng = np.random.default_rng(31)
+    x, codes, sb = _nvfp4_representable(rng, 32, 256, 0, block_2d)
+    c, s, sg = ora.quant_nvfp4_sr(x, block_2d=block_2d, seed=9)
+    assert sg == 1.0 and np.array_equal(s, sb)
+    got = np.stack([c & 15, c >> 4], axis=-1).reshape(codes.shape)
+    zero = (codes & 7) == 0
+    assert np.array_equal(np.where(zero, 0, got), np.where(zero, 0, codes))
+
+
+def test_nvfp4_sr_unbiased_over_seeds(ora):
+    """The seed mean of the SR decode is within 5 exact standard errors of
+    clamp(x * r, 6) x den (TML page: the expected value is preserved)."""
+    _, nonneg = _e2m1_table_from_pages()
+    A, _ = W.nvfp4_linear_small(M=16, K=64)
+    x = W.bf16_bits(A)
+    n = 256
+    acc = np.zeros((16, 64))
+    for seed in range(n):
+        c, s, g = ora.quant_nvfp4_sr(x, seed=seed)
+        acc += ora.dequant(ora.NVFP4, c, s, g)
+    _, s, g = ora.quant_nvfp4(x)
+    xf = (x.astype(np.uint32) << 16).view(np.float32)
+    den = (_torch_e4m3_value(s).astype(np.float32) * np.float32(g)).astype(np.float32)
+    r = (np.float32(1.0) / den).astype(np.float32)
+    q = (xf.reshape(16, 4, 16) * r[..., None]).astype(np.float32).astype(np.float64).reshape(16, 64)
+    a = np.minimum(np.abs(q), 6.0)
+    sig = np.zeros_like(a)
+    for idx, v in np.ndenumerate(a):
+        if v < 6.0 and v not in nonneg:
+            lo, hi = _e2m1_neighbours(v, nonneg)
+            f = (v - lo) / (hi - lo)
+            sig[idx] = np.sqrt(f * (1 - f)) * (hi - lo)
+    # the decode is E2M1 x E4M3(s_b) x s_g in binary64
+    dn = np.repeat(_torch_e4m3_value(s).astype(np.float64) * g, 16, axis=1)
+    target = np.sign(q) * a * dn
+    dev = acc / n - target
+    assert (np.abs(dev) <= 5 * sig * dn / np.sqrt(n) + 1e-300).all()

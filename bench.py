@@ -270,7 +270,8 @@ def measure_rows(hbm, fp4_peak, fp8_peak, reps=10, only=None):
             api.gemm(0, qas[0], qas[1], qws[0], qws[1], 128, 256, 256, gsA=qas[2], gsB=qws[2], out=Cs)
         row("a2+a3+a8 small linear step (latency)", "A 128x256, W 256x256, fp32 out", small_step,
             nbytes=(128 + 256) * 256 * 2)
-    if wants("a6 MXFP8 row quantize RNE", "a6 MXFP8 row quantize SR (Philox)", "a7 requant-transpose SR"):
+    if wants("a6 MXFP8 row quantize RNE", "a6 MXFP8 row quantize SR (Philox)", "a7 requant-transpose SR",
+             "f3 MXFP4 quantize RNE (next row)", "f3 MXFP4 quantize SR (next row)"):
         # -- MXFP8 4096x4096 Student-t: RNE and SR, requant-transpose
         X1 = W.mxfp8_requant().to(dev)
         M1, K1 = X1.shape
@@ -283,7 +284,12 @@ def measure_rows(hbm, fp4_peak, fp8_peak, reps=10, only=None):
         qt = api.requant_transpose(q1s[0], q1s[1], sr=True, seed=1)
         row("a7 requant-transpose SR", "4096x4096 MXFP8 -> column-wise",
             lambda: api.requant_transpose(q1s[0], q1s[1], sr=True, seed=1, out=qt), nbytes=2 * M1 * K1 * (1 + 1 / 32))
-        del X1, q1, q1s, qt
+        q4 = api.quant_mxfp4(X1)
+        row("f3 MXFP4 quantize RNE (next row)", "X 4096x4096", lambda: api.quant_mxfp4(X1, out=q4),
+            nbytes=M1 * K1 * (2 + 0.5 + 1 / 32))
+        row("f3 MXFP4 quantize SR (next row)", "X 4096x4096", lambda: api.quant_mxfp4(X1, sr=True, seed=1, out=q4),
+            nbytes=M1 * K1 * (2 + 0.5 + 1 / 32))
+        del X1, q1, q1s, qt, q4
     if wants("a6 MXFP8 row quantize SR", "a6 MXFP8 column quantize SR", "a8 MXFP8 GEMM dgrad (bf16 out)", "a8 MXFP8 GEMM wgrad (fp32 out)", "a8 NVFP4 rollout GEMM (swap-AB, HBM-bound)"):
         # -- MXFP8 backward (dY 8192x14336, W 14336x4096, X 8192x4096) + NVFP4 rollout
         dY, W4, X4, A_roll = W.mxfp8_backward()

@@ -63,6 +63,18 @@ def quant_mxfp8(x, colwise=False, sr=False, seed=0, stream_id=0, out=None):
     return codes, sf
 
 
+def quant_mxfp4(x, sr=False, seed=0, stream_id=0, out=None):
+    """Row-wise MXFP4.  Returns (codes [M,K/2], sf swizzled)."""
+    M, K = x.shape
+    if out is None:
+        codes = torch.empty(M, K // 2, dtype=torch.uint8, device=x.device)
+        sf = torch.zeros(sf_bytes(M, K // 32), dtype=torch.uint8, device=x.device)
+    else:
+        codes, sf = out
+    bsq.bsq_quant_mxfp4(x, M, K, _ld(x), bsq.BSQ_SR if sr else bsq.BSQ_RNE, seed, stream_id, codes, sf)
+    return codes, sf
+
+
 def rht(x, mask, out=None):
     y = torch.empty_like(x) if out is None else out
     bsq.bsq_rht(x, y, x.shape[0], x.shape[1], _ld(x), _ld(y), mask)

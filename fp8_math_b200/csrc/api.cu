@@ -177,6 +177,19 @@ int bsq_quant_mxfp8(const void *x, int64_t M, int64_t K, int64_t ldx, int colwis
     return launch_status();
 }
 
+int bsq_quant_mxfp4(const void *x, int64_t M, int64_t K, int64_t ldx, int rounding, uint64_t seed,
+                    uint32_t stream_id, uint8_t *codes, uint8_t *sf, void *stream) {
+    if (!x || !codes || !sf || M < 0 || K < 0 || ldx < K || K % 32 || (rounding != BSQ_RNE && rounding != BSQ_SR))
+        return BSQ_ERR_INVALID;
+    if (!aligned16(x) || !aligned16(codes) || !aligned16(sf) || ldx % 8) return BSQ_ERR_ALIGN;
+    DeviceState *d;
+    if (int st = device_state(&d)) return st;
+    if (M == 0 || K == 0) return BSQ_OK;
+    bsq::launch_quant_mxfp4(static_cast<const uint16_t *>(x), M, K, ldx, rounding == BSQ_SR, seed, stream_id, codes,
+                            sf, d->num_sms, static_cast<cudaStream_t>(stream));
+    return launch_status();
+}
+
 int bsq_rht(const void *x, void *y, int64_t M, int64_t K, int64_t ldx, int64_t ldy, uint16_t mask, void *stream) {
     if (!x || !y || M < 0 || K < 0 || K % 16 || ldx < K || ldy < K) return BSQ_ERR_INVALID;
     if (!aligned16(x) || !aligned16(y) || ldx % 8 || ldy % 8) return BSQ_ERR_ALIGN;

@@ -1032,6 +1032,110 @@ __global__ void __launch_bounds__(256) quant_mxfp8_col_kernel(
     }
 }
 
+// ===================================================================== MXFP4
+// E2M1 elements in blocks of 32 along K with one E8M0 scale 2^E,
+// E = clamp(floor(log2 amax) - 2, -127, 127) (2 is the exponent of E2M1's
+// largest value, 6 = 1.5 * 2^2): code max(exponent field - 2, 0), the same
+// branch-free form as the MXFP8 code with 2 in place of 8.
+BSQ_DEV uint32_t mx4_scale_code(float m) {
+    const int f = (int)(__float_as_uint(m) >> 23);
+    return (uint32_t)max(f - 2, 0);
+}
+
+// Stochastic rounding of s to an E2M1 code (sign bit 3) with the 16-bit draw
+// r16: round the magnitude a = min(|s|, 6) up to the next E2M1 value iff
+// r16 * 2^-16 < frac.  For a >= 1 the E2M1 neighbour below a is a with its
+// low 22 bits cleared (one mantissa bit) and frac = low22 / 2^22, so the test
+// is the integer 64 r16 < low22 and rounding up adds 1 << 22; the code is then
+// (bits >> 22) - 252 (exponent - 127 + 1, and the mantissa bit).  Below 1 the
+// spacing is 0.5: t = 2a, frac = t - floor(t) (both exact), code floor(t) +
+// up (0, 0.5 or 1.0).
+BSQ_DEV uint32_t e2m1_sr(float s, uint32_t r16) {
+    const uint32_t sgn = (__float_as_uint(s) >> 28) & 8u;
+    const float a = fminf(fabsf(s), 6.0f);
+    uint32_t mag;
+    if (a >= 1.0f) {
+        const uint32_t b = __float_as_uint(a);
+        const uint32_t up = ((r16 << 6) < (b & 0x3FFFFFu)) ? 0x400000u : 0u;
+        mag = (((b & ~0x3FFFFFu) + up) >> 22) - 252u;
+    } else {
+        const float t = __fmul_rn(a, 2.0f);
+        const float f = floorf(t);
+        const float frac = __fsub_rn(t, f);
+        mag = (uint32_t)f + ((__fmul_rn((float)r16, 1.0f / 65536.0f) < frac) ? 1u : 0u);
+    }
+    return sgn | mag;
+}
+
+// The 8 nibbles of one chunk (element 2j in the low nibble of byte j): s =
+// v * 2^-E (exact), then nearest-even with saturation at +-6 (the satfinite
+// conversion gives +-6 past 6, the same as clamping first) or stochastic
+// rounding with the draws of one Philox call (element i: half i & 1 of word
+// i / 2).  A zero block stores +0 codes.
+template <bool SR>
+BSQ_DEV uint32_t mx4_encode8(const float v[8], bool zero, uint32_t sb, uint64_t chunk, const PhiloxKeys &keys,
+                             uint32_t stream_id) {
+    float s[8];
+    mx_scale8(v, __uint_as_float((254u - sb) << 23), s);
+    uint32_t q;
+    if (SR) {
+        const uint4 r = mx_draws(chunk, keys, stream_id);
+        const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+        q = 0u;
+#pragma unroll
+        for (int i = 0; i < 8; i++) q |= e2m1_sr(s[i], (i & 1) ? (w[i >> 1] >> 16) : (w[i >> 1] & 0xFFFFu)) << (4 * i);
+    } else {
+        q = cvt_e2m1x8(s);
+    }
+    return zero ? 0u : q;
+}
+
+// Row-wise MXFP4: one thread per 8 elements, 4 lanes per block of 32 (two
+// shuffles for the block maximum), rows mapped to lanes as in the MXFP8 row
+// kernel; one 32-bit code store per chunk, the scale bytes of 4 blocks
+// packed into one 32-bit store when a row holds a multiple of 4 blocks.
+template <bool SR>
+__global__ void __launch_bounds__(256) quant_mxfp4_row_kernel(
+    const uint16_t *__restrict__ x, int64_t M, int64_t K, int64_t ldx, const __grid_constant__ PhiloxKeys keys,
+    uint32_t stream_id, uint8_t *__restrict__ codes, uint8_t *__restrict__ sf, RowMap map) {
+    const int64_t K8 = K >> 3, KB = K >> 5;
+    const bool pack4 = (KB & 3) == 0;
+    const int lane = threadIdx.x & 31;
+    const int lpr = 1 << map.lpr_shift;
+    const int rpi = 256 >> map.lpr_shift;
+    const int sub = threadIdx.x >> map.lpr_shift, lk = threadIdx.x & (lpr - 1);
+    for (int64_t r0 = (int64_t)blockIdx.x * rpi; r0 < M; r0 += (int64_t)gridDim.x * rpi) {
+        const int64_t row = r0 + sub;
+        const bool row_ok = row < M;
+        const int64_t rr = row_ok ? row : M - 1;
+        for (int64_t c0 = 0; c0 < K8; c0 += lpr) {
+            const int64_t c8 = c0 + lk;
+            const bool valid = row_ok && c8 < K8;
+            const int64_t cc = c8 < K8 ? c8 : K8 - 1;
+            float v[8];
+            load8_bf16(x + rr * ldx + cc * 8, v);
+            float m = fmax3(fmax3(fabsf(v[0]), fabsf(v[1]), fabsf(v[2])), fmax3(fabsf(v[3]), fabsf(v[4]), fabsf(v[5])),
+                            fmaxf(fabsf(v[6]), fabsf(v[7])));
+            m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+            m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+            const uint32_t sb = mx4_scale_code(m);
+            const uint32_t q = mx4_encode8<SR>(v, m == 0.0f, sb, (uint64_t)(rr * K + cc * 8) >> 3, keys, stream_id);
+            if (valid) *reinterpret_cast<uint32_t *>(codes + rr * (K >> 1) + cc * 4) = q;
+            const int64_t kb = cc >> 2;
+            if (pack4) {
+                const uint32_t b1 = __shfl_down_sync(0xFFFFFFFFu, sb, 4);
+                const uint32_t b2 = __shfl_down_sync(0xFFFFFFFFu, sb, 8);
+                const uint32_t b3 = __shfl_down_sync(0xFFFFFFFFu, sb, 12);
+                if (valid && (lane & 15) == 0)
+                    *reinterpret_cast<uint32_t *>(sf + sf_word_offset(rr, kb >> 2, KB)) =
+                        sb | (b1 << 8) | (b2 << 16) | (b3 << 24);
+            } else if (valid && (lane & 3) == 0) {
+                sf[sf_offset(rr, kb, KB)] = (uint8_t)sb;
+            }
+        }
+    }
+}
+
 // ===================================================================== RHT
 __global__ void __launch_bounds__(256) rht_kernel(const uint16_t *__restrict__ x, uint16_t *y, int64_t M,
                                                   int64_t K, int64_t ldx, int64_t ldy, uint32_t mask, RowMap map) {
@@ -1247,6 +1351,16 @@ void launch_requant_transpose(const uint8_t *codes_row, const uint8_t *sf_row, i
         quant_mxfp8_col_kernel<true, false><<<grid, 256, 0, s>>>(codes_row, sf_row, M, K, K, ntile, dmt, keys,
                                                                  stream_id, codes_col, sf_col);
     }
+}
+
+void launch_quant_mxfp4(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, bool sr, uint64_t seed,
+                        uint32_t stream_id, uint8_t *codes, uint8_t *sf, int num_sms, cudaStream_t s) {
+    const PhiloxKeys keys = philox_keys((uint32_t)seed, (uint32_t)(seed >> 32));
+    RowMap map{lpr_shift_for(K >> 3)};
+    if (map.lpr_shift < 2) map.lpr_shift = 2;  // 4 lanes per block of 32
+    const int grid = grid_for(M, 256 >> map.lpr_shift, num_sms * 8);
+    if (sr) quant_mxfp4_row_kernel<true><<<grid, 256, 0, s>>>(x, M, K, ldx, keys, stream_id, codes, sf, map);
+    else quant_mxfp4_row_kernel<false><<<grid, 256, 0, s>>>(x, M, K, ldx, keys, stream_id, codes, sf, map);
 }
 
 void launch_rht(const uint16_t *x, uint16_t *y, int64_t M, int64_t K, int64_t ldx, int64_t ldy, uint32_t mask,

@@ -25,6 +25,8 @@ int launch_quant_nvfp4_fused(const uint16_t *x, int64_t M, int64_t K, bool block
 void launch_quant_mxfp8(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, bool colwise, bool sr,
                         uint64_t seed, uint32_t stream_id, uint8_t *codes, uint8_t *sf, int num_sms,
                         cudaStream_t s);
+void launch_quant_mxfp4(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, bool sr, uint64_t seed,
+                        uint32_t stream_id, uint8_t *codes, uint8_t *sf, int num_sms, cudaStream_t s);
 void launch_requant_transpose(const uint8_t *codes_row, const uint8_t *sf_row, int64_t M, int64_t K, bool sr,
                               uint64_t seed, uint32_t stream_id, uint8_t *codes_col, uint8_t *sf_col,
                               int num_sms, cudaStream_t s);

@@ -146,6 +146,22 @@ BSQ_API int bsq_quant_mxfp8(const void *x_bf16, int64_t M, int64_t K, int64_t ld
                     int rounding, uint64_t seed, uint32_t stream_id,
                     uint8_t *codes_dev, uint8_t *sf_dev, void *stream);
 
+/* MXFP4 quantize ("08 -- FP4, MXFP4, NVFP4 ...", section "The two Blackwell
+ * formats": E2M1 elements in groups of 32 with one E8M0 power-of-two scale,
+ * 4.25 bits per value; "Microscaling ...", section "Microscaling").  Per
+ * row-wise block of 32: E = clamp(floor(log2 block_amax) - 2, -127, 127)
+ * (2 is the exponent of E2M1's largest value 6 = 1.5 * 2^2, as 8 is E4M3's
+ * for MXFP8), scale code E + 127 (an all-zero block has code 0 and +0
+ * codes); element x * 2^-E clamped to +-6, then E2M1 by nearest-even
+ * (BSQ_RNE) or stochastic rounding (BSQ_SR) with the draws of
+ * bsq_quant_mxfp8 (output element idx = row * K + k).  codes [M][K/2],
+ * element 2j in the low nibble of byte j; sf in the swizzled MMA layout for
+ * M rows x K/32 blocks.  K % 32 == 0; x, codes, sf 16-byte aligned,
+ * ldx % 8 == 0. */
+BSQ_API int bsq_quant_mxfp4(const void *x_bf16, int64_t M, int64_t K, int64_t ldx, int rounding,
+                    uint64_t seed, uint32_t stream_id, uint8_t *codes_dev, uint8_t *sf_dev,
+                    void *stream);
+
 /* 16-point random Hadamard transform along K ("Microscaling ...", section
  * "NVFP4"; "Thinking Machines ...", section "Why communication became the
  * next bottleneck"): per group of 16, y = 1/4 * H16 * diag(s) * x with H16

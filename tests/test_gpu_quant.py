@@ -230,6 +230,40 @@ def test_requant_transpose_parity(ora, M, K, sr):
     assert_codes_equal(sf_canonical(ora, sc, K, M // 32), ws, "requant sf")
 
 
+@pytest.mark.parametrize("sr", [False, True])
+@pytest.mark.parametrize("M,K", [(64, 128), (3, 32), (100, 96), (256, 4096), (33, 3072)])
+def test_mxfp4_rowwise_parity(ora, M, K, sr):
+    """MXFP4 (E2M1 in blocks of 32, E8M0 scale): edge tensors with zero,
+    subnormal-range, saturating and small negative blocks."""
+    x = mx_edge_tensor(M, K, seed=M * 7 + K)
+    c, s = api.quant_mxfp4(dev(x), sr=sr, seed=2, stream_id=5)
+    oc, osf = ora.quant_mxfp4(bits(x), sr=sr, seed=2, stream_id=5)
+    assert_codes_equal(host_u8(c), oc, "mxfp4 codes")
+    assert_codes_equal(sf_canonical(ora, s, M, K // 32), osf, "mxfp4 sf")
+
+
+def test_mxfp4_strided_rows_parity(ora):
+    """A row stride larger than K (a column slice of a wider tensor)."""
+    x = mx_edge_tensor(40, 320, seed=5)
+    xd = dev(x)[:, :256]
+    c, s = api.quant_mxfp4(xd, sr=True, seed=8)
+    oc, osf = ora.quant_mxfp4(bits(x[:, :256].contiguous()), sr=True, seed=8)
+    assert_codes_equal(host_u8(c), oc, "mxfp4 strided codes")
+    assert_codes_equal(sf_canonical(ora, s, 40, 8), osf, "mxfp4 strided sf")
+
+
+def test_mxfp4_workload_full_size(ora):
+    """The Student-t 4096x4096 workload at full size, RNE and SR."""
+    x = W.mxfp8_requant()
+    xb = bits(x)
+    xd = dev(x)
+    for sr in (False, True):
+        c, s = api.quant_mxfp4(xd, sr=sr, seed=1)
+        oc, osf = ora.quant_mxfp4(xb, sr=sr, seed=1)
+        assert_codes_equal(host_u8(c), oc, f"mxfp4 sr={sr} codes")
+        assert_codes_equal(sf_canonical(ora, s, 4096, 128), osf, f"mxfp4 sr={sr} sf")
+
+
 def test_mxfp8_requant_workload_full_size(ora):
     """The Student-t 4096x4096 workload at full size: RNE, SR, then the
     requant-transpose of the SR output -- all bit-exact."""
@@ -258,6 +292,12 @@ def test_invalid_arguments_launch_nothing():
     assert e.value.status == bsq.BSQ_ERR_INVALID
     with pytest.raises(bsq.BsqError) as e:
         bsq.bsq_quant_nvfp4(x, 16, 16, 24, 1, 1, 0, 0, None, 0, None, None, None, gs, codes, sf)
+    assert e.value.status == bsq.BSQ_ERR_INVALID
+    with pytest.raises(bsq.BsqError) as e:  # MXFP4 blocks are 32 wide
+        bsq.bsq_quant_mxfp4(x, 16, 24, 24, bsq.BSQ_RNE, 0, 0, codes, sf)
+    assert e.value.status == bsq.BSQ_ERR_INVALID
+    with pytest.raises(bsq.BsqError) as e:  # unknown rounding mode
+        bsq.bsq_quant_mxfp4(x, 16, 0, 24, 7, 0, 0, codes, sf)
     assert e.value.status == bsq.BSQ_ERR_INVALID
     assert bsq.bsq_check() == bsq.BSQ_OK
 

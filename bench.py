@@ -234,7 +234,8 @@ def measure_rows(hbm, fp4_peak, fp8_peak, reps=10, only=None):
         except Exception as e:  # noqa: BLE001 -- recorded, not fatal
             rows.append({"row": name, "workload": workload, "error": str(e)[:200]})
 
-    if wants("a1 amax (RHT)", "a2+a5 NVFP4 1x16 quantize (amax + RHT fused)", "a3+a5 NVFP4 16x16 quantize (amax + RHT fused)", "a5 RHT standalone (bf16 -> bf16)", "a8 NVFP4 GEMM bf16"):
+    if wants("a1 amax (RHT)", "a2+a5 NVFP4 1x16 quantize (amax + RHT fused)", "a3+a5 NVFP4 16x16 quantize (amax + RHT fused)", "a5 RHT standalone (bf16 -> bf16)", "a8 NVFP4 GEMM bf16",
+             "f3 NVFP4 1x16 quantize SR (amax + RHT fused, next row)"):
         # -- NVFP4 linear with RHT, A 8192x4096, W 14336x4096 (the timed step's calls, one at a time)
         A_h, W_h, seed = W.nvfp4_linear_rht()
         mask = bsq.bsq_rht_sign_mask(seed)
@@ -250,6 +251,10 @@ def measure_rows(hbm, fp4_peak, fp8_peak, reps=10, only=None):
         qw = api.quant_nvfp4(Wd, block_2d=True, rht_mask=mask)
         row("a3+a5 NVFP4 16x16 quantize (amax + RHT fused)", "W 14336x4096",
             lambda: api.quant_nvfp4(Wd, block_2d=True, rht_mask=mask, out=qw), nbytes=N2 * K2 * (2 + 2 + 0.5 + 1 / 16))
+        qsr = api.quant_nvfp4_sr(A, rht_mask=mask, seed=2)
+        row("f3 NVFP4 1x16 quantize SR (amax + RHT fused, next row)", "A 8192x4096",
+            lambda: api.quant_nvfp4_sr(A, rht_mask=mask, seed=2, out=qsr), nbytes=M2 * K2 * (2 + 2 + 0.5 + 1 / 16))
+        del qsr
         y = torch.empty_like(A)
         row("a5 RHT standalone (bf16 -> bf16)", "A 8192x4096", lambda: api.rht(A, mask, out=y), nbytes=M2 * K2 * 4)
         C2 = torch.empty(M2, N2, dtype=torch.bfloat16, device=dev)

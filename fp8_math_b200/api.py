@@ -63,6 +63,22 @@ def quant_mxfp8(x, colwise=False, sr=False, seed=0, stream_id=0, out=None):
     return codes, sf
 
 
+def quant_nvfp4_sr(x, block_2d=False, rht_mask=None, row_index=None, amax_in=None, seed=0, stream_id=0, out=None):
+    """NVFP4 with stochastic rounding of the elements.  Returns (codes
+    [R, K/2] uint8, sf swizzled uint8, global_scale [1] fp32)."""
+    K = x.shape[1]
+    R = x.shape[0] if row_index is None else row_index.shape[0]
+    if out is None:
+        codes = torch.empty(R, K // 2, dtype=torch.uint8, device=x.device)
+        sf = torch.zeros(sf_bytes(R, K // 16), dtype=torch.uint8, device=x.device)
+        gs = torch.empty(1, dtype=torch.float32, device=x.device)
+    else:
+        codes, sf, gs = out
+    bsq.bsq_quant_nvfp4_sr(x, R, K, _ld(x), block_2d, rht_mask is not None, rht_mask or 0, row_index, amax_in, gs,
+                           seed, stream_id, codes, sf)
+    return codes, sf, gs
+
+
 def quant_mxfp4(x, sr=False, seed=0, stream_id=0, out=None):
     """Row-wise MXFP4.  Returns (codes [M,K/2], sf swizzled)."""
     M, K = x.shape

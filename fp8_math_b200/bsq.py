@@ -37,6 +37,8 @@ _SIGS = {
                                   C.c_int, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "bsq_quant_mxfp8": (C.c_int, [_vp, _i64, _i64, _i64, C.c_int, C.c_int, C.c_uint64, C.c_uint32,
                                   _vp, _vp, _vp]),
+    "bsq_quant_nvfp4_sr": (C.c_int, [_vp, _i64, _i64, _i64, C.c_int, C.c_int, C.c_uint16, _vp, _vp, _vp,
+                                     C.c_uint64, C.c_uint32, _vp, _vp, _vp]),
     "bsq_quant_mxfp4": (C.c_int, [_vp, _i64, _i64, _i64, C.c_int, C.c_uint64, C.c_uint32, _vp, _vp, _vp]),
     "bsq_rht": (C.c_int, [_vp, _vp, _i64, _i64, _i64, _i64, C.c_uint16, _vp]),
     "bsq_requant_transpose": (C.c_int, [_vp, _vp, _i64, _i64, C.c_int, C.c_uint64, C.c_uint32, _vp, _vp, _vp]),
@@ -125,6 +127,14 @@ def bsq_quant_nvfp4(x, M, K, ldx, block_2d, four_over_six, rht_enable, rht_sign_
 def bsq_quant_mxfp8(x, M, K, ldx, colwise, rounding, seed, stream_id, codes, sf, stream=None):
     return _check("bsq_quant_mxfp8", lib().bsq_quant_mxfp8(_p(x), M, K, ldx, int(colwise), rounding, seed,
                                                            stream_id, _p(codes), _p(sf), _stream(stream)))
+
+
+def bsq_quant_nvfp4_sr(x, M, K, ldx, block_2d, rht_enable, rht_sign_mask, row_index, amax_in, global_scale, seed,
+                       stream_id, codes, sf, stream=None):
+    return _check("bsq_quant_nvfp4_sr",
+                  lib().bsq_quant_nvfp4_sr(_p(x), M, K, ldx, int(block_2d), int(rht_enable), rht_sign_mask,
+                                           _p(row_index), _p(amax_in), _p(global_scale), seed, stream_id, _p(codes),
+                                           _p(sf), _stream(stream)))
 
 
 def bsq_quant_mxfp4(x, M, K, ldx, rounding, seed, stream_id, codes, sf, stream=None):

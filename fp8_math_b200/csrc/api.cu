@@ -161,6 +161,41 @@ int bsq_quant_nvfp4(const void *x, int64_t M, int64_t K, int64_t ldx, int block_
     return launch_status();
 }
 
+int bsq_quant_nvfp4_sr(const void *x, int64_t M, int64_t K, int64_t ldx, int block_2d, int rht_enable, uint16_t mask,
+                       const int32_t *row_index, const float *amax_in, float *gs, uint64_t seed, uint32_t stream_id,
+                       uint8_t *codes, uint8_t *sf, void *stream) {
+    if (!x || !gs || !codes || !sf || M < 0 || K < 0 || K % 16 || ldx < K) return BSQ_ERR_INVALID;
+    if (block_2d && (M % 16 || row_index)) return BSQ_ERR_INVALID;
+    if (!aligned16(x) || !aligned16(codes) || !aligned16(sf) || ldx % 8 ||
+        (reinterpret_cast<uintptr_t>(gs) & 3u) || (amax_in && (reinterpret_cast<uintptr_t>(amax_in) & 3u)))
+        return BSQ_ERR_ALIGN;
+    DeviceState *d;
+    if (int st = device_state(&d)) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const uint16_t *xx = static_cast<const uint16_t *>(x);
+    if (M == 0 || K == 0) {
+        if (cudaMemsetAsync(gs, 0, sizeof(float), s) != cudaSuccess) return BSQ_ERR_CUDA;
+        bsq::launch_finalize_global_scale(gs, s);
+        return launch_status();
+    }
+    if (amax_in == nullptr) {
+        // the amax pass's scratch is the first 8 bytes of codes, as in bsq_quant_nvfp4
+        if (cudaMemsetAsync(codes, 0, 8, s) != cudaSuccess) return BSQ_ERR_CUDA;
+        unsigned int *scratch = reinterpret_cast<unsigned int *>(codes);
+        bsq::launch_amax(xx, M, K, ldx, rht_enable != 0, mask, row_index, scratch + 1, scratch, gs, d->num_sms, s);
+        bsq::launch_quant_nvfp4_sr(xx, M, K, ldx, block_2d != 0, rht_enable != 0, mask, row_index, gs, false, gs,
+                                   false, seed, stream_id, codes, sf, d->num_sms, s);
+    } else if (amax_in == gs) {
+        bsq::launch_quant_nvfp4_sr(xx, M, K, ldx, block_2d != 0, rht_enable != 0, mask, row_index, gs, true, gs,
+                                   false, seed, stream_id, codes, sf, d->num_sms, s);
+        bsq::launch_finalize_global_scale(gs, s);
+    } else {
+        bsq::launch_quant_nvfp4_sr(xx, M, K, ldx, block_2d != 0, rht_enable != 0, mask, row_index, amax_in, true, gs,
+                                   true, seed, stream_id, codes, sf, d->num_sms, s);
+    }
+    return launch_status();
+}
+
 int bsq_quant_mxfp8(const void *x, int64_t M, int64_t K, int64_t ldx, int colwise, int rounding, uint64_t seed,
                     uint32_t stream_id, uint8_t *codes, uint8_t *sf, void *stream) {
     if (!x || !codes || !sf || M < 0 || K < 0 || ldx < K || (rounding != BSQ_RNE && rounding != BSQ_SR))

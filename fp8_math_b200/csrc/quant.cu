@@ -1136,6 +1136,130 @@ __global__ void __launch_bounds__(256) quant_mxfp4_row_kernel(
     }
 }
 
+// ===================================================================== NVFP4, stochastic rounding
+// NVFP4 with the elements rounded stochastically: block scales and s_g as
+// in the nearest-even kernels above; each element q = y * r (y = RN(u / 4)
+// with the RHT, then RN(y * r): the definition's order also where y is
+// subnormal, since a tiny q can still round up to 0.5), clamped to +-6 and
+// rounded by e2m1_sr with the draws of output elements idx0 .. idx0 + 15
+// (two Philox calls; idx0 = row * K + 16 * block).
+template <bool RHT>
+BSQ_DEV uint2 nv_codes_sr(const f32x2 P[8], float r, uint64_t idx0, const PhiloxKeys &keys, uint32_t stream_id) {
+    f32x2 Q[8];
+#pragma unroll
+    for (int k = 0; k < 8; k++) Q[k] = P[k];
+    if (RHT) pairs_scale(Q, 0.25f);
+    const f32x2 R = f2_pack(r, r);
+    float q[16];
+#pragma unroll
+    for (int k = 0; k < 8; k++) f2_unpack(f2_mul(Q[k], R), q[2 * k], q[2 * k + 1]);
+    uint32_t out[2];
+#pragma unroll
+    for (int h = 0; h < 2; h++) {
+        const uint4 rw = mx_draws((idx0 >> 3) + h, keys, stream_id);
+        const uint32_t w[4] = {rw.x, rw.y, rw.z, rw.w};
+        uint32_t word = 0u;
+#pragma unroll
+        for (int i = 0; i < 8; i++)
+            word |= e2m1_sr(q[8 * h + i], (i & 1) ? (w[i >> 1] >> 16) : (w[i >> 1] & 0xFFFFu)) << (4 * i);
+        out[h] = word;
+    }
+    return make_uint2(out[0], out[1]);
+}
+
+// 1x16 blocks, rows (optionally gathered): one thread per block, rows mapped
+// to lanes as in quant_nvfp4_1d_kernel.
+template <bool RHT, bool GATHER>
+__global__ void __launch_bounds__(256) quant_nvfp4_sr_1d_kernel(
+    const uint16_t *__restrict__ x, int64_t M, int64_t K, int64_t ldx, uint32_t mask,
+    const int32_t *__restrict__ row_index, const float *scale_src, int src_is_amax, float *gs_out, int write_gs,
+    const __grid_constant__ PhiloxKeys keys, uint32_t stream_id, uint8_t *__restrict__ codes,
+    uint8_t *__restrict__ sf, RowMap map) {
+    __shared__ float den_tab[128], rcp_tab[128];
+    const int64_t KB = K >> 4;
+    const bool pack4 = (KB & 3) == 0;
+    const float s_g = src_is_amax ? global_scale_of(*scale_src) : *scale_src;
+    if (write_gs && blockIdx.x == 0 && threadIdx.x == 0) *gs_out = s_g;
+    const NvScale c = nv_scale_setup(s_g, den_tab, rcp_tab);
+    uint32_t sw[8];
+    rht_sign_words(mask, sw);
+    const int lpr = 1 << map.lpr_shift;
+    const int rpi = 256 >> map.lpr_shift;
+    const int sub = threadIdx.x >> map.lpr_shift, lk = threadIdx.x & (lpr - 1);
+    for (int64_t r0 = (int64_t)blockIdx.x * rpi; r0 < M; r0 += (int64_t)gridDim.x * rpi) {
+        const int64_t row = r0 + sub;
+        const bool row_ok = row < M;
+        const int64_t rr = row_ok ? row : M - 1;
+        const int64_t src = GATHER ? (int64_t)__ldg(row_index + rr) : rr;
+        const uint16_t *rp = x + src * ldx;
+        for (int64_t kb0 = 0; kb0 < KB; kb0 += lpr) {
+            const int64_t kb = kb0 + lk;
+            const bool valid = row_ok && kb < KB;
+            const int64_t kk = kb < KB ? kb : KB - 1;
+            uint32_t w[8];
+            load_words16(rp + kk * 16, w);
+            f32x2 P[8];
+            if (RHT) rht16_u_words(w, sw, P);
+            else words_to_pairs(w, P);
+            const float mu = pairs_absmax3(P);
+            const uint32_t sb = nv_scale_code(RHT ? __fmul_rn(mu, 0.25f) : mu, 6.0f, c.c6, c);
+            const uint2 cd = sb ? nv_codes_sr<RHT>(P, rcp_tab[sb], (uint64_t)(rr * K + kk * 16), keys, stream_id)
+                                : make_uint2(0u, 0u);
+            if (valid) *reinterpret_cast<uint2 *>(codes + rr * (K >> 1) + kb * 8) = cd;
+            store_sf(sf, valid, sb, rr, kb, KB, pack4);
+        }
+    }
+}
+
+// 16x16 tiles: the tile mapping of quant_nvfp4_2d_kernel (a warp covers one
+// 16-row tile row and eight blocks; lane l: row l % 16, blocks 4 (l / 16) ..
+// 4 (l / 16) + 3; tile amax over a half-warp).
+template <bool RHT>
+__global__ void __launch_bounds__(256) quant_nvfp4_sr_2d_kernel(
+    const uint16_t *__restrict__ x, int64_t M, int64_t K, int64_t ldx, uint32_t mask, const float *scale_src,
+    int src_is_amax, float *gs_out, int write_gs, const __grid_constant__ PhiloxKeys keys, uint32_t stream_id,
+    uint8_t *__restrict__ codes, uint8_t *__restrict__ sf) {
+    __shared__ float den_tab[128], rcp_tab[128];
+    const float s_g = src_is_amax ? global_scale_of(*scale_src) : *scale_src;
+    if (write_gs && blockIdx.x == 0 && threadIdx.x == 0) *gs_out = s_g;
+    const NvScale c = nv_scale_setup(s_g, den_tab, rcp_tab);
+    uint32_t sw[8];
+    rht_sign_words(mask, sw);
+    const int64_t KB = K >> 4;
+    const int64_t k8 = (KB + 7) >> 3;
+    const int64_t tasks = (M >> 4) * k8;
+    const int lane = threadIdx.x & 31;
+    const int r16 = lane & 15, hw = lane >> 4;
+    const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    for (int64_t task = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); task < tasks; task += warps) {
+        const int64_t rt = task / k8, g8 = task - rt * k8;
+        const int64_t row = rt * 16 + r16;
+        const int64_t kb0 = g8 * 8 + 4 * hw;
+        const uint16_t *rp = x + row * ldx;
+#pragma unroll
+        for (int i = 0; i < 4; i++) {
+            const int64_t kb = kb0 + i;
+            const bool v = kb < KB;  // uniform over the half-warp
+            uint32_t w[8];
+            load_words16(rp + (v ? kb : 0) * 16, w);
+            f32x2 P[8];
+            if (RHT) rht16_u_words(w, sw, P);
+            else words_to_pairs(w, P);
+            float mu = v ? pairs_absmax3(P) : 0.0f;
+#pragma unroll
+            for (int o = 1; o < 16; o <<= 1) mu = fmaxf(mu, __shfl_xor_sync(0xFFFFFFFFu, mu, o));
+            const uint32_t sb = nv_scale_code(RHT ? __fmul_rn(mu, 0.25f) : mu, 6.0f, c.c6, c);
+            const uint2 cd = (sb && v) ? nv_codes_sr<RHT>(P, rcp_tab[sb], (uint64_t)(row * K + kb * 16), keys,
+                                                          stream_id)
+                                       : make_uint2(0u, 0u);
+            if (v) {
+                *reinterpret_cast<uint2 *>(codes + row * (K >> 1) + kb * 8) = cd;
+                sf[sf_offset(row, kb, KB)] = (uint8_t)sb;
+            }
+        }
+    }
+}
+
 // ===================================================================== RHT
 __global__ void __launch_bounds__(256) rht_kernel(const uint16_t *__restrict__ x, uint16_t *y, int64_t M,
                                                   int64_t K, int64_t ldx, int64_t ldy, uint32_t mask, RowMap map) {
@@ -1361,6 +1485,35 @@ void launch_quant_mxfp4(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, bo
     const int grid = grid_for(M, 256 >> map.lpr_shift, num_sms * 8);
     if (sr) quant_mxfp4_row_kernel<true><<<grid, 256, 0, s>>>(x, M, K, ldx, keys, stream_id, codes, sf, map);
     else quant_mxfp4_row_kernel<false><<<grid, 256, 0, s>>>(x, M, K, ldx, keys, stream_id, codes, sf, map);
+}
+
+void launch_quant_nvfp4_sr(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, bool block_2d, bool rht,
+                           uint32_t mask, const int32_t *row_index, const float *scale_src, bool src_is_amax,
+                           float *gs_out, bool write_gs, uint64_t seed, uint32_t stream_id, uint8_t *codes,
+                           uint8_t *sf, int num_sms, cudaStream_t s) {
+    const PhiloxKeys keys = philox_keys((uint32_t)seed, (uint32_t)(seed >> 32));
+    const int sa = src_is_amax ? 1 : 0, wg = write_gs ? 1 : 0;
+    if (block_2d) {
+        const int64_t tasks = (M >> 4) * (((K >> 4) + 7) >> 3);
+        if (rht) {
+            const int grid = grid_for(tasks, 8, resident_ctas<quant_nvfp4_sr_2d_kernel<true>>(num_sms));
+            quant_nvfp4_sr_2d_kernel<true><<<grid, 256, 0, s>>>(x, M, K, ldx, mask, scale_src, sa, gs_out, wg, keys,
+                                                                stream_id, codes, sf);
+        } else {
+            const int grid = grid_for(tasks, 8, resident_ctas<quant_nvfp4_sr_2d_kernel<false>>(num_sms));
+            quant_nvfp4_sr_2d_kernel<false><<<grid, 256, 0, s>>>(x, M, K, ldx, mask, scale_src, sa, gs_out, wg, keys,
+                                                                 stream_id, codes, sf);
+        }
+        return;
+    }
+    RowMap map{lpr_shift_for(K >> 4)};
+    const int grid = grid_for(M, 256 >> map.lpr_shift, num_sms * 8);
+#define BSQ_NVSR(R, GA)                                                                                       \
+    quant_nvfp4_sr_1d_kernel<R, GA><<<grid, 256, 0, s>>>(x, M, K, ldx, mask, row_index, scale_src, sa, gs_out, wg, \
+                                                         keys, stream_id, codes, sf, map)
+    if (rht) { if (row_index) BSQ_NVSR(true, true); else BSQ_NVSR(true, false); }
+    else { if (row_index) BSQ_NVSR(false, true); else BSQ_NVSR(false, false); }
+#undef BSQ_NVSR
 }
 
 void launch_rht(const uint16_t *x, uint16_t *y, int64_t M, int64_t K, int64_t ldx, int64_t ldy, uint32_t mask,

@@ -27,6 +27,10 @@ void launch_quant_mxfp8(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, bo
                         cudaStream_t s);
 void launch_quant_mxfp4(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, bool sr, uint64_t seed,
                         uint32_t stream_id, uint8_t *codes, uint8_t *sf, int num_sms, cudaStream_t s);
+void launch_quant_nvfp4_sr(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, bool block_2d, bool rht,
+                           uint32_t mask, const int32_t *row_index, const float *scale_src, bool src_is_amax,
+                           float *gs_out, bool write_gs, uint64_t seed, uint32_t stream_id, uint8_t *codes,
+                           uint8_t *sf, int num_sms, cudaStream_t s);
 void launch_requant_transpose(const uint8_t *codes_row, const uint8_t *sf_row, int64_t M, int64_t K, bool sr,
                               uint64_t seed, uint32_t stream_id, uint8_t *codes_col, uint8_t *sf_col,
                               int num_sms, cudaStream_t s);

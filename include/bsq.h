@@ -126,6 +126,21 @@ BSQ_API int bsq_quant_nvfp4(const void *x_bf16, int64_t M, int64_t K, int64_t ld
                     const float *amax_in_dev, float *global_scale_dev,
                     uint8_t *codes_dev, uint8_t *sf_dev, void *stream);
 
+/* NVFP4 quantize with stochastic rounding of the elements ("Microscaling
+ * ...", section "NVFP4": the NVFP4 pretraining recipe rounds gradients
+ * stochastically).  s_g, the block scales (1x16, or 16x16 with block_2d)
+ * and the scratch use are those of bsq_quant_nvfp4; each element
+ * q = y * r (y the RHT output when rht_enable, r = 1 / (s_b * s_g)) is
+ * clamped to +-6 and rounded to a neighbouring E2M1 value: up iff
+ * draw * 2^-16 < (|q| - lo) / (hi - lo), with the 16-bit draws of
+ * bsq_quant_mxfp8 for output element idx = row * K + k.  s_b == 0 gives
+ * all-zero codes.  Optional row gather (row_index_dev, 1x16 only); no Four
+ * Over Six and no expert groups.  K % 16 == 0; block_2d needs M % 16 == 0. */
+BSQ_API int bsq_quant_nvfp4_sr(const void *x_bf16, int64_t M, int64_t K, int64_t ldx, int block_2d,
+                       int rht_enable, uint16_t rht_sign_mask, const int32_t *row_index_dev,
+                       const float *amax_in_dev, float *global_scale_dev, uint64_t seed,
+                       uint32_t stream_id, uint8_t *codes_dev, uint8_t *sf_dev, void *stream);
+
 /* MXFP8 quantize ("LMSYS and humans& ...", section "Recipe 1"; stochastic
  * rounding per "Microscaling ...", section "Words on this page", and
  * "Thinking Machines ...", section "A precision choice for each stage").

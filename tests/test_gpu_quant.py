@@ -146,6 +146,68 @@ def test_nvfp4_four_over_six_parity(ora, M, K):
     _nvfp4_check(ora, x, fos=True, rht=0x5A5A, what="4/6 + rht")
 
 
+@pytest.mark.parametrize("rht", [False, True])
+@pytest.mark.parametrize("M,K", [(128, 256), (1, 16), (3, 48), (37, 80), (256, 512)])
+def test_nvfp4_sr_1d_parity(ora, M, K, rht):
+    """NVFP4 with stochastic rounding of the elements, 1x16 blocks."""
+    x = edge_tensor(M, K, seed=M + 3 * K)
+    mask = 0x5A3C if rht else None
+    c, s, g = api.quant_nvfp4_sr(dev(x), rht_mask=mask, seed=11, stream_id=2)
+    assert bsq.bsq_check() == 0
+    oc, osf, og = ora.quant_nvfp4_sr(bits(x), rht_mask=mask, seed=11, stream_id=2)
+    assert np.float32(g.item()) == np.float32(og)
+    assert_codes_equal(host_u8(c), oc, "nvfp4 sr codes")
+    assert_codes_equal(sf_canonical(ora, s, M, K // 16), osf, "nvfp4 sr sf")
+
+
+@pytest.mark.parametrize("rht", [False, True])
+@pytest.mark.parametrize("M,K", [(32, 256), (48, 80), (16, 16), (64, 1024)])
+def test_nvfp4_sr_2d_parity(ora, M, K, rht):
+    """NVFP4 with stochastic rounding of the elements, 16x16 tiles."""
+    x = edge_tensor(M, K, seed=M * 5 + K)
+    mask = 0x3C5A if rht else None
+    c, s, g = api.quant_nvfp4_sr(dev(x), block_2d=True, rht_mask=mask, seed=12, stream_id=3)
+    oc, osf, og = ora.quant_nvfp4_sr(bits(x), block_2d=True, rht_mask=mask, seed=12, stream_id=3)
+    assert np.float32(g.item()) == np.float32(og)
+    assert_codes_equal(host_u8(c), oc, "nvfp4 sr 2d codes")
+    assert_codes_equal(sf_canonical(ora, s, M, K // 16), osf, "nvfp4 sr 2d sf")
+
+
+def test_nvfp4_sr_gather_and_given_amax(ora):
+    """Gathered rows and a caller-given amax (in place and separate)."""
+    x = edge_tensor(64, 128, seed=4)
+    ri = np.array([5, 0, 63, 7, 7, 12, 1, 40, 33, 2], np.int32)
+    c, s, g = api.quant_nvfp4_sr(dev(x), row_index=dev(torch.from_numpy(ri)), seed=13)
+    oc, osf, og = ora.quant_nvfp4_sr(bits(x), row_index=ri, seed=13)
+    assert np.float32(g.item()) == np.float32(og)
+    assert_codes_equal(host_u8(c), oc, "nvfp4 sr gather codes")
+    assert_codes_equal(sf_canonical(ora, s, 10, 8), osf, "nvfp4 sr gather sf")
+    am = dev(torch.tensor([3.5], dtype=torch.float32))
+    c, s, g = api.quant_nvfp4_sr(dev(x), amax_in=am, seed=14)
+    oc, osf, og = ora.quant_nvfp4_sr(bits(x), amax_in=3.5, seed=14)
+    assert np.float32(g.item()) == np.float32(og)
+    assert_codes_equal(host_u8(c), oc, "nvfp4 sr amax codes")
+    gs = dev(torch.tensor([3.5], dtype=torch.float32))
+    c2 = torch.empty(64, 64, dtype=torch.uint8, device="cuda")
+    s2 = torch.zeros(bsq.bsq_sf_bytes(64, 8), dtype=torch.uint8, device="cuda")
+    api.quant_nvfp4_sr(dev(x), amax_in=gs, seed=14, out=(c2, s2, gs))
+    assert np.float32(gs.item()) == np.float32(og)
+    assert_codes_equal(host_u8(c2), oc, "nvfp4 sr in-place amax codes")
+
+
+def test_nvfp4_sr_workload_rows(ora):
+    """The first 1024 rows of the RHT linear's activation A (1x16) and of
+    its weight W (16x16), at K = 4096."""
+    A, Wt, seed = W.nvfp4_linear_rht()
+    mask = bsq.bsq_rht_sign_mask(seed)
+    for t, two_d in ((A[:1024], False), (Wt[:1024], True)):
+        c, s, g = api.quant_nvfp4_sr(dev(t), block_2d=two_d, rht_mask=mask, seed=2, stream_id=1)
+        oc, osf, og = ora.quant_nvfp4_sr(bits(t), block_2d=two_d, rht_mask=mask, seed=2, stream_id=1)
+        assert np.float32(g.item()) == np.float32(og)
+        assert_codes_equal(host_u8(c), oc, f"nvfp4 sr 2d={two_d} codes")
+        assert_codes_equal(sf_canonical(ora, s, 1024, 256), osf, f"nvfp4 sr 2d={two_d} sf")
+
+
 def test_nvfp4_given_amax_and_zero_tensor(ora):
     x = edge_tensor(64, 128, seed=5)
     _nvfp4_check(ora, x, amax_in=float(x.float().abs().max()) * 2.0, what="given amax")

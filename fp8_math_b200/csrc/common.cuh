@@ -91,7 +91,6 @@ BSQ_DEV uint32_t cvt_e2m1x8(const float q[8]) {
     return out;
 }
 
-// E2M1 nibble -> fp32 from the S E E M layout (bias 1; E = 0 is M * 0.5).
 // Eight E2M1 codes (packed as by cvt_e2m1x8: element 2i in the low nibble of
 // byte i) -> fp32, exactly, through cvt.rn.f16x2.e2m1x2 (every E2M1 value is
 // an f16 and an fp32 value; -0 stays -0).
@@ -115,12 +114,6 @@ BSQ_DEV void e2m1x8_to_f32(uint32_t w, float v[8]) {
     }
 }
 
-BSQ_DEV float e2m1_to_f32(uint32_t code) {
-    uint32_t mag = code & 7u;
-    uint32_t bits = (mag >= 2u) ? ((((mag >> 1) + 126u) << 23) | ((mag & 1u) << 22))
-                                : (mag ? 0x3F000000u : 0u);
-    return __uint_as_float(bits | ((code & 8u) << 28));
-}
 
 // floor(log2 a) for a finite a > 0 (normal or subnormal binary32).
 BSQ_DEV int floor_log2(float a) {
@@ -181,25 +174,6 @@ BSQ_DEV uint32_t e4m3_sr(float v, uint32_t r16) {
     return sgn | e4m3_rne(mag);
 }
 
-// Stochastic rounding of |v| <= 448 to E4M3 (same result as e4m3_sr).  In
-// the normal E4M3 range (|v| >= 2^-6) the neighbour below is v with its low
-// 20 mantissa bits cleared, the E4M3 spacing is bit 20, and frac = low20 /
-// 2^20 exactly, so "r16 / 2^16 < frac" is the integer test 16 r16 < low20
-// and rounding up adds 1 << 20 to the bits (a carry into the exponent is
-// the next binade, as the float addition would give).  The code is read off
-// the bits: ((bits >> 20) - (120 << 3)) is exponent - 127 + 7 and the three
-// mantissa bits.  Below 2^-6 the float path of e4m3_sr runs.
-BSQ_DEV uint32_t e4m3_sr_fast(float v, uint32_t r16) {
-    const uint32_t x = __float_as_uint(v);
-    const uint32_t sgn = (x >> 24) & 0x80u;
-    const uint32_t a = x & 0x7FFFFFFFu;
-    if (a >= 0x3C800000u) {  // 2^-6
-        const uint32_t low20 = a & 0xFFFFFu;
-        const uint32_t mag = (a & ~0xFFFFFu) + (((r16 << 4) < low20) ? 0x100000u : 0u);
-        return sgn | ((mag >> 20) - (120u << 3));
-    }
-    return e4m3_sr(v, r16);
-}
 
 
 // ---------------------------------------------------------------- fp32 pairs
@@ -325,48 +299,8 @@ BSQ_DEV float pairs_absmax3(const f32x2 P[8]) {
     return fmax3(fmax3(m0, m1, m2), fmax3(m3, m4, fabsf(v[15])), 0.0f);
 }
 
-// Loads 16 bf16 as 8 fp32 pairs (no transform).
-BSQ_DEV void load16_pairs(const uint16_t *p, f32x2 P[8]) {
-    const uint4 q0 = __ldg(reinterpret_cast<const uint4 *>(p));
-    const uint4 q1 = __ldg(reinterpret_cast<const uint4 *>(p + 8));
-    const uint32_t w[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
-#pragma unroll
-    for (int k = 0; k < 8; k++) P[k] = f2_pack(bf16_lo(w[k]), bf16_hi(w[k]));
-}
 
-// max |v| over 8 pairs
-BSQ_DEV float pairs_absmax(const f32x2 P[8]) {
-    float m = 0.0f;
-#pragma unroll
-    for (int k = 0; k < 8; k++) {
-        float a, b;
-        f2_unpack(P[k], a, b);
-        m = fmaxf(m, fmaxf(fabsf(a), fabsf(b)));
-    }
-    return m;
-}
 
-// In-place 16-point transform y = 1/4 * H16 * diag(s) * x on fp32 values
-// (scalar form, used where the values are needed one by one).
-BSQ_DEV void rht16(float v[16], uint32_t mask) {
-#pragma unroll
-    for (int i = 0; i < 16; i++)
-        if ((mask >> i) & 1u) v[i] = -v[i];
-#pragma unroll
-    for (int h = 1; h < 16; h <<= 1) {
-#pragma unroll
-        for (int base = 0; base < 16; base += 2 * h) {
-#pragma unroll
-            for (int i = base; i < base + h; i++) {
-                float a = v[i], b = v[i + h];
-                v[i] = __fadd_rn(a, b);
-                v[i + h] = __fsub_rn(a, b);
-            }
-        }
-    }
-#pragma unroll
-    for (int i = 0; i < 16; i++) v[i] = __fmul_rn(0.25f, v[i]);
-}
 
 // ---------------------------------------------------------------- SF layout
 // Byte offset of (row r, block b) in a swizzled SF buffer whose rows hold

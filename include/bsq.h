@@ -1,5 +1,5 @@
 /*
- * bsq.h -- libbsq: block-scaled quantization (NVFP4, MXFP8), the 16-point
+ * bsq.h -- libbsq: block-scaled quantization (NVFP4, MXFP8, MXFP4), the 16-point
  * random Hadamard transform and block-scaled GEMMs for NVIDIA B200
  * (sm_100a).  Plain C ABI: device pointers, sizes, a stream handle.
  *
@@ -11,6 +11,8 @@
  *    element 2j in the low nibble of byte j.
  *  - MXFP8 -- "LMSYS and humans& ... low-precision recipes", section "Recipe
  *    1: End-to-end MXFP8": 32 consecutive E4M3 share one E8M0 scale.
+ *  - MXFP4 -- "08 -- FP4, MXFP4, NVFP4 ...", table "The two Blackwell
+ *    formats": 32 consecutive E2M1 share one E8M0 scale (4.25 bits).
  *  - Scale-factor ("SF") buffers are written in the layout the Blackwell
  *    block-scaled MMA reads ("Microscaling ...", section "Hardware and
  *    kernels": a block-scaled GEMM needs a particular scale-factor layout):
@@ -34,6 +36,12 @@
  *    device, the 4-byte error word (created on first use).
  *  - Inputs must be finite; nonzero magnitudes below 2^-100 are outside the
  *    supported range for NVFP4 (codes there are unspecified).
+ *  - Kernel-selection overrides, read from the environment on each call
+ *    (results are identical either way; they exist to test and time each
+ *    path): BSQ_FUSED_QUANT=0 disables the one-launch amax + 16x16 quantize
+ *    kernel of bsq_quant_nvfp4; BSQ_GEMM_PAIR=0/1 forces the single-CTA or
+ *    the CTA-pair GEMM where both apply; BSQ_GEMM_BN sets the single-CTA
+ *    GEMM's N tile to 128 or (bf16 output) 256.
  */
 #ifndef BSQ_H
 #define BSQ_H

@@ -1,8 +1,9 @@
-// quant.cu -- memory-bound codec kernels of libbsq (sm_100a):
+// quant.cu -- the codec kernels of libbsq (sm_100a):
 //   tensor amax (optionally of the RHT output), NVFP4 quantize (1x16 with
-//   optional Four Over Six, row gather and expert groups; 16x16 tiles),
+//   optional Four Over Six, row gather and expert groups; 16x16 tiles; a
+//   one-launch amax + quantize form; stochastic rounding of the elements),
 //   MXFP8 quantize (row-wise, column-wise; RNE or Philox SR), dequantize ->
-//   transpose -> requantize, and the standalone 16-point RHT.
+//   transpose -> requantize, MXFP4 quantize, and the standalone 16-point RHT.
 // All of them stream bf16/fp8 from HBM with 16-byte vector loads, reduce the
 // block amax with warp shuffles, and write packed codes plus scale factors
 // directly in the swizzled layout the block-scaled MMA reads.

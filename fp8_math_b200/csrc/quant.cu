@@ -7,6 +7,8 @@
 // All of them stream bf16/fp8 from HBM with 16-byte vector loads, reduce the
 // block amax with warp shuffles, and write packed codes plus scale factors
 // directly in the swizzled layout the block-scaled MMA reads.
+#include <atomic>
+
 #include "common.cuh"
 #include "quant.cuh"
 
@@ -1300,16 +1302,18 @@ static int grid_for(int64_t work_items, int per_block, int max_ctas) {
 
 // CTAs of `kernel` (256 threads, static shared memory only) that fit on the
 // device at once: the grid of the persistent streaming kernels is one full
-// wave, so no partial last wave leaves SMs idle.  Cached per kernel.
+// wave, so no partial last wave leaves SMs idle.  Cached per kernel (an
+// atomic, so concurrent first calls from several host threads are defined;
+// they compute the same value).
 template <auto Kern>
 static int resident_ctas(int num_sms) {
-    static int per_sm = 0;
-    if (per_sm == 0) {
-        int n = 0;
+    static std::atomic<int> per_sm{0};
+    int n = per_sm.load(std::memory_order_relaxed);
+    if (n == 0) {
         if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, Kern, 256, 0) != cudaSuccess || n < 1) n = 1;
-        per_sm = n;
+        per_sm.store(n, std::memory_order_relaxed);
     }
-    return per_sm * num_sms;
+    return n * num_sms;
 }
 
 void launch_amax(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, bool rht, uint32_t mask,

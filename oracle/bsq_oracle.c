@@ -410,7 +410,7 @@ float ora_nvfp4_global_scale(float amax)
     return (amax == 0.0f) ? 1.0f : amax / 2688.0f;
 }
 
-/* sr != 0: the elements are rounded stochastically instead (ora_e2m1_sr of
+/* R29 -- sr != 0: the elements are rounded stochastically instead (ora_e2m1_sr of
  * x * r clamped to +-6, the draw of output element m * K + k with the given
  * seed and stream id); block scales and s_g are unchanged.  Not combined with
  * Four Over Six. */

@@ -66,3 +66,38 @@ def test_validation_rejects_before_any_device_work(lib):
     assert L.bsq_requant_transpose(16, 16, 48, 32, 0, 0, 0, 16, 16, None) == lib.BSQ_ERR_INVALID  # M % 32
     assert L.bsq_debug_timeout_probe(0, None) == lib.BSQ_ERR_INVALID
     assert lib.status_str(lib.BSQ_ERR_TIMEOUT) == "device-side wait timed out"
+
+
+def declared_parameter_counts():
+    """name -> number of parameters, from each BSQ_API declaration."""
+    with open(os.path.join(ROOT, "include", "bsq.h")) as f:
+        text = re.sub(r"/\*.*?\*/", "", f.read(), flags=re.S)
+    out = {}
+    for m in re.finditer(r"BSQ_API[^;(]*?\b(bsq_\w+)\s*\(([^)]*)\)\s*;", text, flags=re.S):
+        params = m.group(2).strip()
+        out[m.group(1)] = 0 if params in ("", "void") else params.count(",") + 1
+    return out
+
+
+def test_binding_matches_header_signatures(lib):
+    """Every declared entry point has a ctypes binding with the header's
+    number of parameters, and the binding names nothing the header lacks."""
+    decl = declared_parameter_counts()
+    assert set(decl) == set(lib._SIGS), (sorted(set(decl) ^ set(lib._SIGS)))
+    for name, n in decl.items():
+        assert len(lib._SIGS[name][1]) == n, (name, n, len(lib._SIGS[name][1]))
+
+
+def test_validation_of_the_fp4_variants(lib):
+    L = lib.lib()
+    # MXFP4: K % 32, rounding mode, alignment
+    assert L.bsq_quant_mxfp4(16, 4, 48, 48, 0, 0, 0, 64, 64, None) == lib.BSQ_ERR_INVALID
+    assert L.bsq_quant_mxfp4(16, 4, 64, 64, 7, 0, 0, 64, 64, None) == lib.BSQ_ERR_INVALID
+    assert L.bsq_quant_mxfp4(8, 4, 64, 64, 0, 0, 0, 64, 64, None) == lib.BSQ_ERR_ALIGN
+    assert L.bsq_quant_mxfp4(16, 4, 64, 60, 0, 0, 0, 64, 64, None) == lib.BSQ_ERR_INVALID  # ldx < K
+    # NVFP4 with stochastic rounding: K % 16, 2-D needs M % 16 and no gather, alignment
+    assert L.bsq_quant_nvfp4_sr(16, 16, 24, 24, 0, 0, 0, None, None, 64, 0, 0, 64, 64, None) == lib.BSQ_ERR_INVALID
+    assert L.bsq_quant_nvfp4_sr(16, 8, 32, 32, 1, 0, 0, None, None, 64, 0, 0, 64, 64, None) == lib.BSQ_ERR_INVALID
+    assert L.bsq_quant_nvfp4_sr(16, 16, 32, 32, 1, 0, 0, 64, None, 64, 0, 0, 64, 64, None) == lib.BSQ_ERR_INVALID
+    assert L.bsq_quant_nvfp4_sr(16, 16, 32, 32, 0, 0, 0, None, None, 66, 0, 0, 64, 64, None) == lib.BSQ_ERR_ALIGN
+    assert L.bsq_quant_nvfp4_sr(None, 16, 32, 32, 0, 0, 0, None, None, 64, 0, 0, 64, 64, None) == lib.BSQ_ERR_INVALID

@@ -21,6 +21,7 @@ BSQ_OK, BSQ_ERR_INVALID, BSQ_ERR_ALIGN, BSQ_ERR_UNSUPPORTED, BSQ_ERR_CUDA, BSQ_E
 BSQ_RNE, BSQ_SR = 0, 1
 BSQ_NVFP4, BSQ_MXFP8 = 0, 1
 BSQ_OUT_F32, BSQ_OUT_BF16 = 0, 1
+BSQ_KNOB_FUSED_QUANT, BSQ_KNOB_GEMM_PAIR, BSQ_KNOB_GEMM_BN = 0, 1, 2
 
 _lock = threading.Lock()
 _lib = None
@@ -48,6 +49,7 @@ _SIGS = {
                                    _vp, _i64, C.c_int, _vp]),
     "bsq_check": (C.c_int, [_vp]),
     "bsq_debug_timeout_probe": (C.c_int, [C.c_uint64, _vp]),
+    "bsq_debug_kernel_choice": (C.c_int, [C.c_int, C.c_int]),
 }
 
 
@@ -170,3 +172,7 @@ def bsq_check(stream=None):
 
 def bsq_debug_timeout_probe(timeout_ns, stream=None):
     return _check("bsq_debug_timeout_probe", lib().bsq_debug_timeout_probe(timeout_ns, _stream(stream)))
+
+
+def bsq_debug_kernel_choice(knob, value):
+    return _check("bsq_debug_kernel_choice", lib().bsq_debug_kernel_choice(knob, value))

@@ -2,6 +2,7 @@
 // validation, per-device state (SM count, error word), kernel launches.
 #include <cstdio>
 #include <cstring>
+#include <atomic>
 #include <cstdlib>
 #include <mutex>
 
@@ -58,9 +59,32 @@ void philox_host(uint32_t c[4], uint32_t k0, uint32_t k1) {
     }
 }
 
+// Kernel-selection overrides (bsq_debug_kernel_choice): -1 = automatic.
+std::atomic<int> g_knob[3] = {{-1}, {-1}, {-1}};
+
 }  // namespace
 
+namespace bsq {
+int kernel_choice(int knob) { return g_knob[knob].load(std::memory_order_relaxed); }
+}  // namespace bsq
+
 extern "C" {
+
+int bsq_debug_kernel_choice(int knob, int value) {
+    switch (knob) {
+        case BSQ_KNOB_FUSED_QUANT:
+        case BSQ_KNOB_GEMM_PAIR:
+            if (value < -1 || value > 1) return BSQ_ERR_INVALID;
+            break;
+        case BSQ_KNOB_GEMM_BN:
+            if (value != -1 && value != 128 && value != 256) return BSQ_ERR_INVALID;
+            break;
+        default:
+            return BSQ_ERR_INVALID;
+    }
+    g_knob[knob].store(value, std::memory_order_relaxed);
+    return BSQ_OK;
+}
 
 const char *bsq_status_str(int status) {
     switch (status) {
@@ -99,12 +123,10 @@ int bsq_amax(const void *x, int64_t M, int64_t K, int64_t ldx, int rht_enable, u
     return launch_status();
 }
 
-// The fused amax + quantize kernel can be switched off (BSQ_FUSED_QUANT=0)
-// for tuning and for tests of the two-pass path.
-static bool fused_enabled() {
-    const char *e = getenv("BSQ_FUSED_QUANT");
-    return !(e && e[0] == '0');
-}
+// The fused amax + quantize kernel can be switched off
+// (bsq_debug_kernel_choice(BSQ_KNOB_FUSED_QUANT, 0)) for tuning and for
+// tests of the two-pass path.
+static bool fused_enabled() { return bsq::kernel_choice(BSQ_KNOB_FUSED_QUANT) != 0; }
 
 int bsq_quant_nvfp4(const void *x, int64_t M, int64_t K, int64_t ldx, int block_2d, int four_over_six,
                     int rht_enable, uint16_t mask, const int32_t *row_index, int G, const int32_t *row_off,
@@ -140,8 +162,8 @@ int bsq_quant_nvfp4(const void *x, int64_t M, int64_t K, int64_t ldx, int block_
         const bool fusable = !row_index && G == 0 && ldx == K && !four_over_six && block_2d && fused_enabled();
         if (fusable) {
             // amax and quantize in one cooperative kernel
-            if (bsq::launch_quant_nvfp4_fused(xx, M, K, block_2d != 0, rht_enable != 0, mask, gs, codes, sf, d->err,
-                                              d->num_sms, s) != 0)
+            if (bsq::launch_quant_nvfp4_fused(xx, M, K, rht_enable != 0, mask, gs, codes, sf, d->err, d->num_sms,
+                                              s) != 0)
                 return BSQ_ERR_CUDA;
             return launch_status();
         }
@@ -314,12 +336,14 @@ int bsq_check(void *stream) {
 }
 
 // ------------------------------------------------------------ no-alloc global scale
-// Scratch of bsq_global_scale_noalloc: a file-scope device array (one per
-// device, resolved with cudaGetSymbolAddress) instead of any allocation.
+// bsq_global_scale_noalloc keeps its scratch in a file-scope device array
+// instead of any allocation.  Host code may not use the array's name as a
+// device address: the address is looked up with cudaGetSymbolAddress once
+// per device, with that device current, and passed to the kernel.
 }  // extern "C"
 
 namespace {
-constexpr int kNoAllocScratchWords = 64;
+constexpr int64_t kNoAllocScratchWords = 4096;  // 16 KiB: a CTA counter + 4095 per-CTA maxima
 __device__ __align__(256) unsigned int g_noalloc_scratch[kNoAllocScratchWords];
 std::mutex g_noalloc_mu;
 unsigned int *g_noalloc_ptr[kMaxDevices];
@@ -331,9 +355,10 @@ int bsq_global_scale_noalloc(const void *x, int64_t M, int64_t K, int64_t ldx, i
                              float *gs_dev, void *stream) {
     if (!x || !gs_dev || M < 0 || K < 0 || K % 16 || ldx < K) return BSQ_ERR_INVALID;
     if (!aligned16(x) || ldx % 8 || (reinterpret_cast<uintptr_t>(gs_dev) & 3u)) return BSQ_ERR_ALIGN;
-    // the amax pass needs a CTA counter and the amax bits
-    constexpr size_t need = 2 * sizeof(unsigned int);
-    if (need > sizeof(g_noalloc_scratch)) return BSQ_ERR_UNSUPPORTED;  // never allocate more
+    // one partial maximum per CTA of kPartialBlocks blocks, plus the counter
+    if (M > (int64_t(1) << 40) || K > (int64_t(1) << 40)) return BSQ_ERR_UNSUPPORTED;
+    const int64_t ctas = (M * (K / 16) + bsq::kPartialBlocks - 1) / bsq::kPartialBlocks;
+    if (1 + ctas > kNoAllocScratchWords) return BSQ_ERR_UNSUPPORTED;  // the array is all there is
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return BSQ_ERR_CUDA;
     unsigned int *scratch;
@@ -346,17 +371,15 @@ int bsq_global_scale_noalloc(const void *x, int64_t M, int64_t K, int64_t ldx, i
         }
         scratch = g_noalloc_ptr[dev];
     }
-    int num_sms = 0;
-    if (cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return BSQ_ERR_CUDA;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (M == 0 || K == 0) {
+    if (ctas == 0) {
         if (cudaMemsetAsync(gs_dev, 0, sizeof(float), s) != cudaSuccess) return BSQ_ERR_CUDA;
         bsq::launch_finalize_global_scale(gs_dev, s);  // amax 0 gives s_g = 1
         return launch_status();
     }
-    if (cudaMemsetAsync(scratch, 0, need, s) != cudaSuccess) return BSQ_ERR_CUDA;
-    bsq::launch_amax(static_cast<const uint16_t *>(x), M, K, ldx, rht_enable != 0, mask, nullptr, scratch + 1, scratch,
-                     gs_dev, num_sms, s);
+    // the counter must start at zero; the partials are written before they are read
+    if (cudaMemsetAsync(scratch, 0, sizeof(unsigned int), s) != cudaSuccess) return BSQ_ERR_CUDA;
+    bsq::launch_amax_partials(static_cast<const uint16_t *>(x), M, K, ldx, rht_enable != 0, mask, scratch, gs_dev, s);
     return launch_status();
 }
 

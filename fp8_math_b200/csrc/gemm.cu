@@ -120,7 +120,7 @@ BSQ_DEV TileInfo tile_info(int64_t t, int64_t m_tiles, const GemmParams &p, cons
     const int64_t mt = local % mt_g;
     ti.a_row0 = (int64_t)offs[lo] + mt * 128;
     ti.sfa_row0 = (int64_t)__ldg(p.sf_row_off + lo) + mt * 128;
-    ti.m_lim = offs[lo + 1];
+    ti.m_lim = min((int64_t)offs[lo + 1], p.m_lim);  // never past the last row of A
     ti.n0 = local / mt_g;
     ti.group = lo;
     return ti;
@@ -669,7 +669,7 @@ __global__ void __launch_bounds__(448, 1)
         nt = local / mt_g;
         a_row0 = (int64_t)offs[lo] + mt * 256 + 128 * rank;
         sfa_row0 = (int64_t)__ldg(p.sf_row_off + lo) + mt * 256 + 128 * rank;
-        m_lim = offs[lo + 1];
+        m_lim = min((int64_t)offs[lo + 1], p.m_lim);
         group = lo;
     };
 
@@ -1072,17 +1072,36 @@ bool make_c_tmap(CUtensorMap *m, void *C, bool bf16, int64_t n_cols, int64_t row
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The dynamic shared-memory limit of a kernel is a per-device attribute:
+// set it once per (kernel, device), under a lock, and remember the outcome.
+constexpr int kMaxDev = 64;
+int smem_attr_once(const void *kern, int bytes) {
+    struct Entry {
+        const void *kern;
+        int dev;
+        int status;
+    };
+    static std::mutex mu;
+    static Entry done[256];
+    static int ndone = 0;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return BSQ_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(mu);
+    for (int i = 0; i < ndone; i++)
+        if (done[i].kern == kern && done[i].dev == dev) return done[i].status;
+    const int st = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess
+                       ? BSQ_OK
+                       : BSQ_ERR_CUDA;
+    if (st == BSQ_OK && ndone < 256) done[ndone++] = {kern, dev, st};
+    return st;
+}
+
 template <int FMT, bool OUT_BF16, bool GROUPED>
 int run_pair(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &tsa, const CUtensorMap &tsb,
              const CUtensorMap &tc, const GemmParams &p, int pairs, cudaStream_t s) {
     using C_ = Cfg2<FMT, GROUPED>;
     auto kern = gemm_bs2_kernel<FMT, OUT_BF16, GROUPED>;
-    static bool attr_set = false;
-    if (!attr_set) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C_::kSmemBytes) != cudaSuccess)
-            return BSQ_ERR_CUDA;
-        attr_set = true;
-    }
+    if (smem_attr_once(reinterpret_cast<const void *>(kern), C_::kSmemBytes) != BSQ_OK) return BSQ_ERR_CUDA;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * pairs, 1, 1);
     cfg.blockDim = dim3(C_::kThreads, 1, 1);
@@ -1103,12 +1122,7 @@ template <int FMT, int BN, int ACC, bool OUT_BF16, bool SWAP, bool GROUPED>
 int run(const CUtensorMap &ta, const CUtensorMap &tb, const GemmParams &p, int grid, cudaStream_t s) {
     using C_ = Cfg<FMT, BN>;
     auto kern = gemm_bs_kernel<FMT, BN, ACC, OUT_BF16, SWAP, GROUPED>;
-    static bool attr_set = false;  // per instantiation; set once (idempotent)
-    if (!attr_set) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C_::kSmemBytes) != cudaSuccess)
-            return BSQ_ERR_CUDA;
-        attr_set = true;
-    }
+    if (smem_attr_once(reinterpret_cast<const void *>(kern), C_::kSmemBytes) != BSQ_OK) return BSQ_ERR_CUDA;
     kern<<<grid, C_::kThreads, C_::kSmemBytes, s>>>(ta, tb, p);
     return cudaGetLastError() == cudaSuccess ? BSQ_OK : BSQ_ERR_CUDA;
 }
@@ -1133,15 +1147,15 @@ int dispatch(const GemmArgs &g, cudaStream_t s) {
     // Single CTAs keep the skinny swap-AB case, operands with fewer than 256
     // rows, outputs that TMA cannot store (unaligned base or row stride) and
     // grouped NVFP4 with a half k-tile (that would need the exact extent of
-    // A's scale buffer, which only the device knows).  BSQ_GEMM_PAIR=0/1
-    // overrides the choice where the pair kernel is possible (tuning, tests).
+    // A's scale buffer, which only the device knows).  The BSQ_KNOB_GEMM_PAIR
+    // override forces either kernel where the pair kernel is possible
+    // (tuning, tests).
     const int64_t c_esz = g.out_bf16 ? 2 : 4;
     const bool c_tma_ok = (reinterpret_cast<uintptr_t>(g.C) % 16 == 0) && (g.ldc * c_esz) % 16 == 0;
     const bool pair_ok = !swap && NB >= 128 && c_tma_ok && !(grouped && FMT == BSQ_NVFP4 && g.K % 256 != 0);
     bool use_pair = pair_ok && MA >= 256 && NB >= 256;
-    if (const char *e = getenv("BSQ_GEMM_PAIR")) use_pair = pair_ok && atoi(e) != 0;
-    if (const char *e = getenv("BSQ_GEMM_BN")) {  // debug/tuning override of the single-CTA tile
-        int v = atoi(e);
+    if (const int v = kernel_choice(BSQ_KNOB_GEMM_PAIR); v >= 0) use_pair = pair_ok && v != 0;
+    if (const int v = kernel_choice(BSQ_KNOB_GEMM_BN); v > 0) {  // tuning override of the single-CTA tile
         if ((v == 128 || (v == 256 && g.out_bf16)) && !swap) bn = v;
     }
     GemmParams p{};

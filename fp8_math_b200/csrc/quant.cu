@@ -122,6 +122,61 @@ BSQ_DEV float global_scale_of(float amax) { return amax == 0.0f ? 1.0f : __fdiv_
 
 __global__ void finalize_global_scale_kernel(float *gs) { *gs = global_scale_of(*gs); }
 
+// amax with one partial maximum per CTA in caller-given scratch (word 0: a
+// CTA counter that must be zero on entry; word 1 + c: CTA c's maximum), for
+// the no-allocation global-scale entry point.  CTA c covers the 16-element
+// blocks [c * kPartialBlocks, (c + 1) * kPartialBlocks) of the row-major
+// block sequence (row = b / (K / 16)); the last CTA to finish reduces the
+// partials with all its threads and writes s_g.
+template <bool RHT>
+__global__ void __launch_bounds__(256) amax_partials_kernel(const uint16_t *__restrict__ x, int64_t M, int64_t K,
+                                                            int64_t ldx, uint32_t mask, unsigned int *scratch,
+                                                            float *gs_out) {
+    uint32_t sw[8];
+    rht_sign_words(mask, sw);
+    const int64_t KB = K >> 4, nblk = M * KB;
+    const int64_t b0 = (int64_t)blockIdx.x * kPartialBlocks;
+    float m = 0.0f;
+#pragma unroll 4
+    for (int i = 0; i < kPartialBlocks / 256; i++) {
+        const int64_t b = b0 + i * 256 + threadIdx.x;
+        if (b < nblk) {
+            const int64_t row = b / KB, kb = b - row * KB;
+            uint32_t w[8];
+            load_words16(x + row * ldx + kb * 16, w);
+            m = fmaxf(m, block_absmax<RHT>(w, sw));
+        }
+    }
+    __shared__ float red[8];
+    __shared__ int last;
+#pragma unroll
+    for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float b = red[0];
+        for (int i = 1; i < 8; i++) b = fmaxf(b, red[i]);
+        scratch[1 + blockIdx.x] = __float_as_uint(b);
+        __threadfence();
+        last = atomicAdd(scratch, 1u) == gridDim.x - 1;
+        if (last) __threadfence();
+    }
+    __syncthreads();
+    if (!last) return;
+    float a = 0.0f;
+    for (unsigned int c = threadIdx.x; c < gridDim.x; c += 256) a = fmaxf(a, __uint_as_float(__ldcg(scratch + 1 + c)));
+#pragma unroll
+    for (int o = 16; o; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, o));
+    __syncthreads();
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = a;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float b = red[0];
+        for (int i = 1; i < 8; i++) b = fmaxf(b, red[i]);
+        *gs_out = global_scale_of(b);
+    }
+}
+
 // ===================================================================== NVFP4
 // Per-CTA tables and constants of one tensor's global scale s_g.  For every
 // E4M3 scale code sb: den[sb] = RN(e4m3(sb) * s_g) and rcp[sb] = RN(1/den)
@@ -228,9 +283,11 @@ BSQ_DEV void nv_block_1d(const uint32_t w[8], const uint32_t sw[8], const NvScal
     }
 }
 
-// Row -> scale-factor row under expert groups (binary search of offsets).
+// Row -> scale-factor row under expert groups (binary search of offsets);
+// -1 for a row outside [off[0], off[G]), which owns no scale-factor row.
 BSQ_DEV int64_t grouped_sf_row(int64_t row, int G, const int32_t *__restrict__ off,
                                const int32_t *__restrict__ sfoff) {
+    if (row < (int64_t)__ldg(off) || row >= (int64_t)__ldg(off + G)) return -1;
     int lo = 0, hi = G;  // off[lo] <= row < off[hi]
     while (hi - lo > 1) {
         int mid = (lo + hi) >> 1;
@@ -293,7 +350,7 @@ __global__ void __launch_bounds__(256) quant_nvfp4_1d_kernel(
             uint2 cd;
             nv_block_1d<RHT, FOS>(w, sw, c, den_tab, rcp_tab, sb, cd);
             if (valid) *reinterpret_cast<uint2 *>(codes + rr * (K >> 1) + kb * 8) = cd;
-            store_sf(sf, valid, sb, sf_row, kb, KB, pack4);
+            store_sf(sf, valid && sf_row >= 0, sb, sf_row, kb, KB, pack4);
         }
     }
 }
@@ -402,16 +459,16 @@ __global__ void __launch_bounds__(256) quant_nvfp4_2d_kernel(
 }
 
 // ===================================================================== fused NVFP4
-// One cooperative kernel per tensor (contiguous, no gather or groups):
+// One cooperative kernel per 16x16-block tensor (contiguous, no gather):
 //   phase 1  amax over the tensor (four blocks per thread in flight);
 //   barrier  every CTA arrives on a grid counter and waits (bounded);
-//   phase 2  every CTA reads the amax, derives s_g and quantizes its blocks
+//   phase 2  every CTA reads the amax, derives s_g and quantizes its tiles
 //            in the reverse of the phase-1 order, so the most recently read
-//            lines (an 8192x4096 bf16 tensor fits in L2 whole) come from L2.
+//            lines come from L2.
 // The counter and the amax bits live in the first 8 bytes of the code
-// buffer (zeroed by the caller).  Those bytes are the first block's codes:
-// their writer -- the last block its thread handles -- first waits until
-// every CTA has arrived a second time, i.e. has read the amax.
+// buffer (zeroed by the caller).  Those bytes are the first tile's codes:
+// their writer first waits until every CTA has arrived a second time, i.e.
+// has read the amax.
 BSQ_DEV unsigned int ld_acquire_gpu(const unsigned int *p) {
     unsigned int v;
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
@@ -445,9 +502,9 @@ BSQ_DEV bool grid_barrier(unsigned int *ctr, unsigned int target, unsigned int *
     return ok_sh != 0;
 }
 
-template <bool RHT, bool TWO_D>
+template <bool RHT>
 __global__ void __launch_bounds__(256) quant_nvfp4_fused_kernel(
-    const uint16_t *__restrict__ x, int64_t M, int64_t K, int kb_shift, uint32_t mask, unsigned int *scratch,
+    const uint16_t *__restrict__ x, int64_t M, int64_t K, uint32_t mask, unsigned int *scratch,
     float *gs_out, uint8_t *__restrict__ codes, uint8_t *__restrict__ sf, unsigned int *err) {
     __shared__ float den_tab[128], rcp_tab[128];
     uint32_t sw[8];
@@ -487,31 +544,7 @@ __global__ void __launch_bounds__(256) quant_nvfp4_fused_kernel(
     if (blockIdx.x == 0 && threadIdx.x == 0) *gs_out = s_g;
     const NvScale c = nv_scale_setup(s_g, den_tab, rcp_tab);
     const unsigned int all_read = 2u * gridDim.x;
-    if (!TWO_D) {
-        // ---- phase 2, 1x16 blocks, reverse order, two in flight
-        const int64_t wbase = tid - lane;
-        const int64_t nwarp_blk = (nblk + 31) & ~int64_t(31);
-        const int64_t iters = wbase < nwarp_blk ? (nwarp_blk - 1 - wbase) / stride + 1 : 0;
-        for (int64_t i = iters - 1; i >= 0; i -= 2) {
-            const int64_t b = tid + i * stride, b1 = b - stride;
-            const bool v0 = b < nblk, v1 = i >= 1 && b1 < nblk;
-            uint32_t w0[8], w1[8];
-            load_words16(x + (v0 ? b : 0) * 16, w0);
-            load_words16(x + (v1 ? b1 : 0) * 16, w1);
-#pragma unroll
-            for (int h = 0; h < 2; h++) {
-                if (h && !__any_sync(0xFFFFFFFFu, v1)) break;
-                const int64_t bb = h ? b1 : b;
-                const bool v = h ? v1 : v0;
-                uint32_t sb;
-                uint2 cd;
-                nv_block_1d<RHT, false>(h ? w1 : w0, sw, c, den_tab, rcp_tab, sb, cd);
-                if (v && bb == 0 && !wait_counter(scratch, all_read, err, 21)) cd = make_uint2(0u, 0u);
-                if (v) *reinterpret_cast<uint2 *>(codes + bb * 8) = cd;
-                store_sf(sf, v, sb, bb >> kb_shift, bb & (KB - 1), KB, true);
-            }
-        }
-    } else {
+    {
         // ---- phase 2, 16x16 tiles (warp = 16 rows x 8 blocks), reverse task order
         const int64_t k8 = (KB + 7) >> 3;
         const int64_t tasks = (M >> 4) * k8;
@@ -1302,16 +1335,19 @@ static int grid_for(int64_t work_items, int per_block, int max_ctas) {
 
 // CTAs of `kernel` (256 threads, static shared memory only) that fit on the
 // device at once: the grid of the persistent streaming kernels is one full
-// wave, so no partial last wave leaves SMs idle.  Cached per kernel (an
-// atomic, so concurrent first calls from several host threads are defined;
-// they compute the same value).
+// wave, so no partial last wave leaves SMs idle.  Cached per kernel and
+// device (atomics, so concurrent first calls from several host threads are
+// defined; they compute the same value).
 template <auto Kern>
 static int resident_ctas(int num_sms) {
-    static std::atomic<int> per_sm{0};
-    int n = per_sm.load(std::memory_order_relaxed);
+    constexpr int kDevs = 64;
+    static std::atomic<int> per_sm[kDevs];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kDevs) dev = 0;
+    int n = per_sm[dev].load(std::memory_order_relaxed);
     if (n == 0) {
         if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, Kern, 256, 0) != cudaSuccess || n < 1) n = 1;
-        per_sm.store(n, std::memory_order_relaxed);
+        per_sm[dev].store(n, std::memory_order_relaxed);
     }
     return n * num_sms;
 }
@@ -1340,6 +1376,14 @@ void launch_amax(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, bool rht,
 }
 
 void launch_finalize_global_scale(float *gs, cudaStream_t s) { finalize_global_scale_kernel<<<1, 1, 0, s>>>(gs); }
+
+void launch_amax_partials(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, bool rht, uint32_t mask,
+                          unsigned int *scratch, float *gs_out, cudaStream_t s) {
+    const int64_t nblk = M * (K >> 4);
+    const int grid = (int)((nblk + kPartialBlocks - 1) / kPartialBlocks);
+    if (rht) amax_partials_kernel<true><<<grid, 256, 0, s>>>(x, M, K, ldx, mask, scratch, gs_out);
+    else amax_partials_kernel<false><<<grid, 256, 0, s>>>(x, M, K, ldx, mask, scratch, gs_out);
+}
 
 void launch_quant_nvfp4(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, bool block_2d, bool fos,
                         bool rht, uint32_t mask, const int32_t *row_index, int G, const int32_t *row_off,
@@ -1393,24 +1437,15 @@ void launch_quant_nvfp4(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, bo
 #undef BSQ_NV1
 }
 
-int launch_quant_nvfp4_fused(const uint16_t *x, int64_t M, int64_t K, bool block_2d, bool rht, uint32_t mask,
-                             float *gs_out, uint8_t *codes, uint8_t *sf, unsigned int *err, int num_sms,
-                             cudaStream_t s) {
+int launch_quant_nvfp4_fused(const uint16_t *x, int64_t M, int64_t K, bool rht, uint32_t mask, float *gs_out,
+                             uint8_t *codes, uint8_t *sf, unsigned int *err, int num_sms, cudaStream_t s) {
     const int64_t KB = K >> 4;
-    int kb_shift = 0;
-    while ((int64_t(1) << kb_shift) < KB) kb_shift++;
     unsigned int *scratch = reinterpret_cast<unsigned int *>(codes);
-    void *args[] = {(void *)&x, (void *)&M, (void *)&K, (void *)&kb_shift, (void *)&mask, (void *)&scratch,
+    void *args[] = {(void *)&x, (void *)&M, (void *)&K, (void *)&mask, (void *)&scratch,
                     (void *)&gs_out, (void *)&codes, (void *)&sf, (void *)&err};
-    const void *kern;
-    int resident;
-    if (block_2d) {
-        if (rht) { kern = (const void *)quant_nvfp4_fused_kernel<true, true>; resident = resident_ctas<quant_nvfp4_fused_kernel<true, true>>(num_sms); }
-        else { kern = (const void *)quant_nvfp4_fused_kernel<false, true>; resident = resident_ctas<quant_nvfp4_fused_kernel<false, true>>(num_sms); }
-    } else {
-        if (rht) { kern = (const void *)quant_nvfp4_fused_kernel<true, false>; resident = resident_ctas<quant_nvfp4_fused_kernel<true, false>>(num_sms); }
-        else { kern = (const void *)quant_nvfp4_fused_kernel<false, false>; resident = resident_ctas<quant_nvfp4_fused_kernel<false, false>>(num_sms); }
-    }
+    const void *kern = rht ? (const void *)quant_nvfp4_fused_kernel<true> : (const void *)quant_nvfp4_fused_kernel<false>;
+    const int resident = rht ? resident_ctas<quant_nvfp4_fused_kernel<true>>(num_sms)
+                             : resident_ctas<quant_nvfp4_fused_kernel<false>>(num_sms);
     // one resident wave, no more CTAs than 256-block groups of work
     const int grid = grid_for(M * KB, 256, resident);
     return cudaLaunchCooperativeKernel(kern, dim3(grid), dim3(256), args, 0, s) == cudaSuccess ? 0 : 1;

@@ -12,16 +12,22 @@ void launch_amax(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, bool rht,
                  const int32_t *row_index, unsigned int *amax_bits, unsigned int *counter, float *gs_out,
                  int num_sms, cudaStream_t s);
 void launch_finalize_global_scale(float *gs, cudaStream_t s);
+// 16-element blocks per CTA of the partial-maximum amax pass.
+constexpr int kPartialBlocks = 4096;
+// amax + s_g with one partial maximum per CTA in `scratch`: word 0 is a CTA
+// counter (zero on entry), words 1 .. ceil(M K / 16 / kPartialBlocks) hold
+// the partials.  The last CTA writes s_g to *gs_out.
+void launch_amax_partials(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, bool rht, uint32_t mask,
+                          unsigned int *scratch, float *gs_out, cudaStream_t s);
 void launch_quant_nvfp4(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, bool block_2d, bool fos,
                         bool rht, uint32_t mask, const int32_t *row_index, int G, const int32_t *row_off,
                         const int32_t *sf_off, const float *scale_src, bool src_is_amax, float *gs_out,
                         bool write_gs, uint8_t *codes, uint8_t *sf, int num_sms, cudaStream_t s);
-// amax + NVFP4 quantize of a contiguous tensor in one cooperative kernel
-// (1x16 blocks need a power-of-two block count per row).  The first 8 bytes
-// of codes must be zero on entry.  Returns non-zero if the launch failed.
-int launch_quant_nvfp4_fused(const uint16_t *x, int64_t M, int64_t K, bool block_2d, bool rht, uint32_t mask,
-                             float *gs_out, uint8_t *codes, uint8_t *sf, unsigned int *err, int num_sms,
-                             cudaStream_t s);
+// amax + NVFP4 16x16 quantize of a contiguous tensor in one cooperative
+// kernel.  The first 8 bytes of codes must be zero on entry.  Returns
+// non-zero if the launch failed.
+int launch_quant_nvfp4_fused(const uint16_t *x, int64_t M, int64_t K, bool rht, uint32_t mask, float *gs_out,
+                             uint8_t *codes, uint8_t *sf, unsigned int *err, int num_sms, cudaStream_t s);
 void launch_quant_mxfp8(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, bool colwise, bool sr,
                         uint64_t seed, uint32_t stream_id, uint8_t *codes, uint8_t *sf, int num_sms,
                         cudaStream_t s);

@@ -36,12 +36,9 @@
  *    device, the 4-byte error word (created on first use).
  *  - Inputs must be finite; nonzero magnitudes below 2^-100 are outside the
  *    supported range for NVFP4 (codes there are unspecified).
- *  - Kernel-selection overrides, read from the environment on each call
- *    (results are identical either way; they exist to test and time each
- *    path): BSQ_FUSED_QUANT=0 disables the one-launch amax + 16x16 quantize
- *    kernel of bsq_quant_nvfp4; BSQ_GEMM_PAIR=0/1 forces the single-CTA or
- *    the CTA-pair GEMM where both apply; BSQ_GEMM_BN sets the single-CTA
- *    GEMM's N tile to 128 or (bf16 output) 256.
+ *  - Behaviour is selected by the arguments alone; the library reads no
+ *    environment variable.  bsq_debug_kernel_choice() can force one of two
+ *    equivalent kernels for tests and tuning (results are identical).
  */
 #ifndef BSQ_H
 #define BSQ_H
@@ -72,6 +69,13 @@ enum { BSQ_RNE = 0, BSQ_SR = 1 };          /* rounding for MXFP8 outputs */
 enum { BSQ_NVFP4 = 0, BSQ_MXFP8 = 1 };     /* GEMM operand format */
 enum { BSQ_OUT_F32 = 0, BSQ_OUT_BF16 = 1 }; /* GEMM output type */
 
+/* Kernel-selection overrides (bsq_debug_kernel_choice). */
+enum {
+    BSQ_KNOB_FUSED_QUANT = 0, /* 1/-1: amax + 16x16 quantize in one cooperative launch; 0: two passes */
+    BSQ_KNOB_GEMM_PAIR = 1,   /* -1: automatic; 0: single-CTA GEMM; 1: CTA-pair GEMM where it applies */
+    BSQ_KNOB_GEMM_BN = 2      /* -1: automatic; 128 or 256 (bf16 output): the single-CTA GEMM's N tile */
+};
+
 /* Human-readable name of a status code (static string). */
 BSQ_API const char *bsq_status_str(int status);
 
@@ -93,17 +97,27 @@ BSQ_API int bsq_amax(const void *x_bf16, int64_t M, int64_t K, int64_t ldx,
              int rht_enable, uint16_t rht_sign_mask, const int32_t *row_index_dev,
              float *amax_dev, void *stream);
 
-/* NVFP4 global scale without any device allocation: *gs_dev = s_g =
- * amax / 2688 (amax = 0 gives 1) of the M x K bf16 matrix x, after the
- * 16-point RHT along K when rht_enable != 0 -- the value bsq_quant_nvfp4
- * writes to *global_scale_dev ("Microscaling ...", section "NVFP4").
- * Its scratch (a CTA counter and the amax bits, 8 bytes) is a file-scope
- * device array of the library, found with cudaGetSymbolAddress per device;
- * the call never allocates device memory (it does not create the error word
- * the other calls use), and a request needing more scratch than the array
- * holds is rejected with BSQ_ERR_UNSUPPORTED.  The scratch is per device:
- * calls on one device must be ordered (one stream, or synchronized).
- * K % 16 == 0; x 16-byte aligned, ldx % 8 == 0; gs_dev 4-byte aligned. */
+/* The NVFP4 global scale s_g = amax / 2688 (amax = 0 gives 1) of the M x K
+ * bf16 matrix x, after the 16-point RHT along K when rht_enable != 0 -- the
+ * value bsq_quant_nvfp4 writes to *global_scale_dev -- computed without
+ * allocating any device memory.  The pages have no counterpart to this
+ * entry point.  It is for callers that may not call cudaMalloc: code whose
+ * device memory all belongs to a framework's pool allocator (a raw
+ * allocation would sit outside the pool's accounting and cap), and code on
+ * a latency-critical path, where cudaMalloc can synchronize the device.
+ * Its scratch is a file-scope device array of 16 KiB (4096 words) that every
+ * GPU which loads the library holds until the process exits: word 0 counts
+ * finished CTAs, word 1 + c holds CTA c's maximum, one CTA per 65536
+ * elements.  A request needing more (M * K > 4095 * 65536 elements, about
+ * 268 million) returns BSQ_ERR_UNSUPPORTED without touching the device.
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress, with that device current); make that first call
+ * outside any stream capture.  Each call zeroes the counter on the stream
+ * before its kernel.  All calls on one device share the array, which keeps
+ * the last call's contents: calls that overlap on the GPU race, so order
+ * them on one stream or synchronize between them.  Never allocates, not even
+ * the error word of the other entry points.  K % 16 == 0; x 16-byte aligned,
+ * ldx % 8 == 0; gs_dev 4-byte aligned. */
 BSQ_API int bsq_global_scale_noalloc(const void *x_bf16, int64_t M, int64_t K, int64_t ldx, int rht_enable,
                                      uint16_t rht_sign_mask, float *gs_dev, void *stream);
 
@@ -124,7 +138,9 @@ BSQ_API int bsq_global_scale_noalloc(const void *x_bf16, int64_t M, int64_t K, i
  * sf swizzled.  With G > 0 the rows form G groups (MoE experts): group e
  * owns output rows [row_offsets[e], row_offsets[e+1]) and its SF rows start
  * at sf_row_offsets[e] (a multiple of 128); both arrays are device int32
- * [G+1], and sf must hold sf_row_offsets[G] SF rows.
+ * [G+1], nondecreasing, with row_offsets[0] = 0 and row_offsets[G] = M, and
+ * sf must hold sf_row_offsets[G] SF rows (a row outside [row_offsets[0],
+ * row_offsets[G]) gets codes but writes no scale factor).
  * Requirements: K % 16 == 0; block_2d needs M % 16 == 0 and excludes
  * four_over_six and groups. */
 BSQ_API int bsq_quant_nvfp4(const void *x_bf16, int64_t M, int64_t K, int64_t ldx,
@@ -228,7 +244,9 @@ BSQ_API int bsq_gemm_blockscaled(int fmt, const uint8_t *A_dev, const uint8_t *s
  * A's SF rows of group e start at sf_row_offsets[e] (as bsq_quant_nvfp4
  * writes them with groups); B is [G][N][K] codes with G consecutive SF
  * buffers of bsq_sf_bytes(N, K/vec) bytes each.  Offsets are device int32
- * [G+1]; the row counts may be anything (zero included).  K % 128 == 0. */
+ * [G+1], nondecreasing, row_offsets[0] = 0 and row_offsets[G] <= M_total
+ * (no row of C past M_total is written); the row counts may be anything
+ * (zero included).  K % 128 == 0. */
 BSQ_API int bsq_grouped_gemm(int fmt, int G, const int32_t *row_offsets_dev, const int32_t *sf_row_offsets_dev,
                      int64_t M_total, const uint8_t *A_dev, const uint8_t *sfA_dev, const float *gsA_dev,
                      const uint8_t *B_dev, const uint8_t *sfB_dev, const float *gsB_dev,
@@ -238,6 +256,13 @@ BSQ_API int bsq_grouped_gemm(int fmt, int G, const int32_t *row_offsets_dev, con
  * Returns BSQ_OK, BSQ_ERR_TIMEOUT (a kernel's bounded wait ran out; the
  * kernel returned early and its outputs are undefined) or BSQ_ERR_CUDA. */
 BSQ_API int bsq_check(void *stream);
+
+/* Forces a kernel choice (BSQ_KNOB_* with the values listed there; -1
+ * restores the automatic choice) for every later call in this process, on
+ * every device.  Host-only and thread-safe; results are bit-identical either
+ * way -- it exists so that tests and timing can reach each kernel.  Returns
+ * BSQ_ERR_INVALID for an unknown knob or value. */
+BSQ_API int bsq_debug_kernel_choice(int knob, int value);
 
 /* Test hook for the bounded-wait path: launches one CTA that waits on a
  * shared-memory barrier nobody arrives at, giving up after timeout_ns

@@ -13,6 +13,23 @@ def pytest_configure(config):
     config.addinivalue_line("markers", "slow: full-size oracle work (minutes on CPU)")
 
 
+@pytest.fixture
+def knobs():
+    """Setter for the library's kernel-selection overrides
+    (bsq_debug_kernel_choice); every knob set is restored to automatic at
+    teardown."""
+    from fp8_math_b200 import bsq
+    touched = []
+
+    def setter(knob, value):
+        bsq.bsq_debug_kernel_choice(knob, value)
+        touched.append(knob)
+
+    yield setter
+    for k in touched:
+        bsq.bsq_debug_kernel_choice(k, -1)
+
+
 @pytest.fixture(scope="session")
 def ora():
     from oracle import oracle as o

@@ -63,8 +63,8 @@ def run_gemm(ora, fmt, qa, qb, M, N, K, out_dtype):
     (1, 256, 256, torch.float32),       # M = 1
     (17, 384, 640, torch.float32),      # swap-AB ragged
 ])
-def test_gemm_full_compare(ora, monkeypatch, pair, fmt, M, N, K, out):
-    monkeypatch.setenv("BSQ_GEMM_PAIR", str(pair))
+def test_gemm_full_compare(ora, knobs, pair, fmt, M, N, K, out):
+    knobs(bsq.BSQ_KNOB_GEMM_PAIR, pair)
     A, Bm = W.nvfp4_linear_small(M=M, N=N, K=K, seed=M * 7 + N + K)
     qa, qb = oracle_operands(ora, fmt, A, Bm)
     Cg = run_gemm(ora, fmt, qa, qb, M, N, K, out)
@@ -85,10 +85,10 @@ def test_gemm_small_linear_workload_exact_inputs(ora):
 
 @pytest.mark.parametrize("pair", [0, 1])
 @pytest.mark.parametrize("fmt", [NV, MX])
-def test_grouped_gemm_compare(ora, monkeypatch, pair, fmt):
+def test_grouped_gemm_compare(ora, knobs, pair, fmt):
     """Small MoE: routed rows grouped by expert (uneven counts, one expert
     possibly empty), per-expert B and global scales."""
-    monkeypatch.setenv("BSQ_GEMM_PAIR", str(pair))
+    knobs(bsq.BSQ_KNOB_GEMM_PAIR, pair)
     E, T, H, F = 6, 96, 256, 192
     g = torch.Generator().manual_seed(5)
     logits = torch.randn(T, E, generator=g)

@@ -74,11 +74,11 @@ def test_nvfp4_1d_parity(ora, M, K):
 
 
 @pytest.mark.parametrize("block_2d", [False, True])
-def test_nvfp4_two_pass_path(ora, monkeypatch, block_2d):
+def test_nvfp4_two_pass_path(ora, knobs, block_2d):
     """The separate amax and quantize kernels (what gathered, grouped and 4/6
     inputs use), forced for contiguous tensors that otherwise go through the
     fused cooperative kernel."""
-    monkeypatch.setenv("BSQ_FUSED_QUANT", "0")
+    knobs(bsq.BSQ_KNOB_FUSED_QUANT, 0)
     for M, K in [(128, 256), (48, 1040) if block_2d else (37, 80), (160, 4096)]:
         x = edge_tensor(M, K, seed=5 * M + K)
         _nvfp4_check(ora, x, block_2d=block_2d, what=f"two-pass {M}x{K}")

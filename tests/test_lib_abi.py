@@ -101,3 +101,31 @@ def test_validation_of_the_fp4_variants(lib):
     assert L.bsq_quant_nvfp4_sr(16, 16, 32, 32, 1, 0, 0, 64, None, 64, 0, 0, 64, 64, None) == lib.BSQ_ERR_INVALID
     assert L.bsq_quant_nvfp4_sr(16, 16, 32, 32, 0, 0, 0, None, None, 66, 0, 0, 64, 64, None) == lib.BSQ_ERR_ALIGN
     assert L.bsq_quant_nvfp4_sr(None, 16, 32, 32, 0, 0, 0, None, None, 64, 0, 0, 64, 64, None) == lib.BSQ_ERR_INVALID
+
+
+def test_kernel_choice_knobs_validate(lib):
+    L = lib.lib()
+    assert L.bsq_debug_kernel_choice(7, 0) == lib.BSQ_ERR_INVALID
+    assert L.bsq_debug_kernel_choice(lib.BSQ_KNOB_FUSED_QUANT, 2) == lib.BSQ_ERR_INVALID
+    assert L.bsq_debug_kernel_choice(lib.BSQ_KNOB_GEMM_BN, 64) == lib.BSQ_ERR_INVALID
+    for knob, value in [(lib.BSQ_KNOB_FUSED_QUANT, 0), (lib.BSQ_KNOB_GEMM_PAIR, 1), (lib.BSQ_KNOB_GEMM_BN, 256)]:
+        assert L.bsq_debug_kernel_choice(knob, value) == lib.BSQ_OK
+        assert L.bsq_debug_kernel_choice(knob, -1) == lib.BSQ_OK
+
+
+def test_noalloc_rejects_requests_beyond_its_scratch(lib):
+    """The no-allocation entry point holds one partial maximum per 65536
+    elements in a 4096-word array (one word is the counter): 4095 CTAs are
+    the most it can take.  A larger request is refused on the host, before
+    any CUDA call (on this GPU-less machine a request that fits reaches the
+    runtime and fails there instead)."""
+    L = lib.lib()
+    K = 4096
+    fits = 4095 * 65536 // K              # 65520 rows: exactly 4095 CTAs
+    assert L.bsq_global_scale_noalloc(16, fits + 1, K, K, 0, 0, 64, None) == lib.BSQ_ERR_UNSUPPORTED
+    assert L.bsq_global_scale_noalloc(16, 1 << 41, 16, 16, 0, 0, 64, None) == lib.BSQ_ERR_UNSUPPORTED
+    assert L.bsq_global_scale_noalloc(16, 4, 40, 40, 0, 0, 64, None) == lib.BSQ_ERR_INVALID   # K % 16
+    assert L.bsq_global_scale_noalloc(8, 4, 64, 64, 0, 0, 64, None) == lib.BSQ_ERR_ALIGN      # x alignment
+    import torch
+    if not torch.cuda.is_available():
+        assert L.bsq_global_scale_noalloc(16, fits, K, K, 0, 0, 64, None) == lib.BSQ_ERR_CUDA

@@ -308,6 +308,17 @@ static void load_row(const uint16_t *x, int64_t ldx, int64_t src, int64_t K,
     }
 }
 
+/* The fused path's RHT output, binary32, for every group of 16 along K of a
+ * row-major M x K bf16 matrix (what the amax and NVFP4 passes consume). */
+int ora_rht_f32(const uint16_t *x, float *y, int64_t M, int64_t K, uint16_t mask)
+{
+    if (K % 16)
+        return 1;
+    for (int64_t m = 0; m < M; m++)
+        load_row(x, K, m, K, 1, mask, y + m * K);
+    return 0;
+}
+
 /* Standalone RHT: bf16 in, bf16 (nearest-even) out, along K in groups of 16. */
 int ora_rht_bf16(const uint16_t *x, uint16_t *y, int64_t M, int64_t K, int64_t ld, uint16_t mask)
 {
@@ -413,11 +424,13 @@ float ora_nvfp4_global_scale(float amax)
 /* R29 -- sr != 0: the elements are rounded stochastically instead (ora_e2m1_sr of
  * x * r clamped to +-6, the draw of output element m * K + k with the given
  * seed and stream id); block scales and s_g are unchanged.  Not combined with
- * Four Over Six. */
+ * Four Over Six.  row0 is the index, in the whole output tensor, of the first
+ * output row computed here (0 for a whole tensor): it only offsets the draw
+ * index, so a band of rows can be computed on its own. */
 static int quant_nvfp4_impl(const uint16_t *x, int64_t M, int64_t K, int64_t ldx,
                             int block_2d, int four_over_six, int rht, uint16_t mask,
                             const int32_t *row_index, const float *amax_in,
-                            int sr, uint64_t seed, uint32_t stream_id,
+                            int sr, uint64_t seed, uint32_t stream_id, int64_t row0,
                             float *s_g_out, uint8_t *codes, uint8_t *sf)
 {
     if (K % 16 || (block_2d && M % 16) || (block_2d && four_over_six) || (sr && four_over_six))
@@ -460,7 +473,8 @@ static int quant_nvfp4_impl(const uint16_t *x, int64_t M, int64_t K, int64_t ldx
                             q = 6.0f;
                         if (q < -6.0f)
                             q = -6.0f;
-                        c6.code[i] = ora_e2m1_sr(q, ora_sr_draw(seed, stream_id, (uint64_t)(m * K + kb * 16 + i)));
+                        c6.code[i] = ora_e2m1_sr(q, ora_sr_draw(seed, stream_id,
+                                                                (uint64_t)((row0 + m) * K + kb * 16 + i)));
                     }
                 }
                 sf[m * KB + kb] = pick->sb;
@@ -480,7 +494,17 @@ int ora_quant_nvfp4(const uint16_t *x, int64_t M, int64_t K, int64_t ldx,
                     float *s_g_out, uint8_t *codes, uint8_t *sf)
 {
     return quant_nvfp4_impl(x, M, K, ldx, block_2d, four_over_six, rht, mask, row_index, amax_in,
-                            0, 0, 0, s_g_out, codes, sf);
+                            0, 0, 0, 0, s_g_out, codes, sf);
+}
+
+int ora_quant_nvfp4_sr_rows(const uint16_t *x, int64_t M, int64_t K, int64_t ldx,
+                            int block_2d, int rht, uint16_t mask,
+                            const int32_t *row_index, const float *amax_in,
+                            uint64_t seed, uint32_t stream_id, int64_t row0,
+                            float *s_g_out, uint8_t *codes, uint8_t *sf)
+{
+    return quant_nvfp4_impl(x, M, K, ldx, block_2d, 0, rht, mask, row_index, amax_in,
+                            1, seed, stream_id, row0, s_g_out, codes, sf);
 }
 
 int ora_quant_nvfp4_sr(const uint16_t *x, int64_t M, int64_t K, int64_t ldx,
@@ -489,8 +513,8 @@ int ora_quant_nvfp4_sr(const uint16_t *x, int64_t M, int64_t K, int64_t ldx,
                        uint64_t seed, uint32_t stream_id,
                        float *s_g_out, uint8_t *codes, uint8_t *sf)
 {
-    return quant_nvfp4_impl(x, M, K, ldx, block_2d, 0, rht, mask, row_index, amax_in,
-                            1, seed, stream_id, s_g_out, codes, sf);
+    return ora_quant_nvfp4_sr_rows(x, M, K, ldx, block_2d, rht, mask, row_index, amax_in,
+                                   seed, stream_id, 0, s_g_out, codes, sf);
 }
 
 /* ------------------------------------------------------------------------ */
@@ -506,8 +530,8 @@ int ora_quant_nvfp4_sr(const uint16_t *x, int64_t M, int64_t K, int64_t ldx,
 /* sf [M][K/32] canonical E8M0 codes.                                         */
 /* ------------------------------------------------------------------------ */
 
-int ora_quant_mxfp4(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, int sr,
-                    uint64_t seed, uint32_t stream_id, uint8_t *codes, uint8_t *sf)
+int ora_quant_mxfp4_rows(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, int sr,
+                         uint64_t seed, uint32_t stream_id, int64_t row0, uint8_t *codes, uint8_t *sf)
 {
     if (K % 32)
         return 1;
@@ -538,7 +562,7 @@ int ora_quant_mxfp4(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, int sr
                         q = 6.0f;
                     if (q < -6.0f)
                         q = -6.0f;
-                    c[i] = sr ? ora_e2m1_sr(q, ora_sr_draw(seed, stream_id, (uint64_t)(r * K + kb * 32 + i)))
+                    c[i] = sr ? ora_e2m1_sr(q, ora_sr_draw(seed, stream_id, (uint64_t)((row0 + r) * K + kb * 32 + i)))
                               : ora_e2m1_rne_sat(q);
                 }
             }
@@ -547,6 +571,14 @@ int ora_quant_mxfp4(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, int sr
         }
     }
     return 0;
+}
+
+/* The whole tensor (row0 = 0); ora_quant_mxfp4_rows computes a band of rows
+ * whose first row is row row0 of the whole output (the SR draw index). */
+int ora_quant_mxfp4(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, int sr,
+                    uint64_t seed, uint32_t stream_id, uint8_t *codes, uint8_t *sf)
+{
+    return ora_quant_mxfp4_rows(x, M, K, ldx, sr, seed, stream_id, 0, codes, sf);
 }
 
 /* ------------------------------------------------------------------------ */
@@ -634,14 +666,14 @@ int ora_quant_mxfp8(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, int co
 /* exact in binary32 (inputs must keep it finite).                            */
 /* ------------------------------------------------------------------------ */
 
-int ora_requant_transpose(const uint8_t *codes_row, const uint8_t *sf_row, int64_t M, int64_t K,
-                          int sr, uint64_t seed, uint32_t stream_id,
-                          uint8_t *codes_col, uint8_t *sf_col)
+int ora_requant_transpose_rows(const uint8_t *codes_row, const uint8_t *sf_row, int64_t M, int64_t K,
+                               int sr, uint64_t seed, uint32_t stream_id, int64_t k0, int64_t k1,
+                               uint8_t *codes_col, uint8_t *sf_col)
 {
-    if (K % 32 || M % 32)
+    if (K % 32 || M % 32 || k0 < 0 || k1 > K || k0 > k1)
         return 1;
     float v[32];
-    for (int64_t k = 0; k < K; k++) {
+    for (int64_t k = k0; k < k1; k++) {
         for (int64_t mb = 0; mb < M / 32; mb++) {
             for (int i = 0; i < 32; i++) {
                 int64_t m = mb * 32 + i;
@@ -652,6 +684,15 @@ int ora_requant_transpose(const uint8_t *codes_row, const uint8_t *sf_row, int64
         }
     }
     return 0;
+}
+
+/* The whole output (rows 0 .. K-1); ora_requant_transpose_rows computes output
+ * rows k0 .. k1-1 only, into the same full-size output arrays. */
+int ora_requant_transpose(const uint8_t *codes_row, const uint8_t *sf_row, int64_t M, int64_t K,
+                          int sr, uint64_t seed, uint32_t stream_id,
+                          uint8_t *codes_col, uint8_t *sf_col)
+{
+    return ora_requant_transpose_rows(codes_row, sf_row, M, K, sr, seed, stream_id, 0, K, codes_col, sf_col);
 }
 
 /* ------------------------------------------------------------------------ */

@@ -16,6 +16,7 @@ import ctypes as C
 import os
 import subprocess
 import threading
+from concurrent.futures import ThreadPoolExecutor
 
 import numpy as np
 
@@ -73,14 +74,22 @@ def lib():
                 "ora_quant_nvfp4_sr": (C.c_int, [_u16p, _i64, _i64, _i64, C.c_int, C.c_int, C.c_uint16,
                                                  C.c_void_p, C.c_void_p, C.c_uint64, C.c_uint32, _f32p, _u8p,
                                                  _u8p]),
+                "ora_quant_nvfp4_sr_rows": (C.c_int, [_u16p, _i64, _i64, _i64, C.c_int, C.c_int, C.c_uint16,
+                                                      C.c_void_p, C.c_void_p, C.c_uint64, C.c_uint32, _i64,
+                                                      _f32p, _u8p, _u8p]),
                 "ora_quant_mxfp4": (C.c_int, [_u16p, _i64, _i64, _i64, C.c_int, C.c_uint64, C.c_uint32,
                                               _u8p, _u8p]),
+                "ora_quant_mxfp4_rows": (C.c_int, [_u16p, _i64, _i64, _i64, C.c_int, C.c_uint64, C.c_uint32,
+                                                   _i64, _u8p, _u8p]),
+                "ora_rht_f32": (C.c_int, [_u16p, _f32p, _i64, _i64, C.c_uint16]),
                 "ora_quant_mxfp8": (C.c_int, [_u16p, _i64, _i64, _i64, C.c_int, C.c_int,
                                               C.c_uint64, C.c_uint32, _u8p, _u8p]),
                 "ora_quant_mxfp8_rows": (C.c_int, [_u16p, _i64, _i64, _i64, C.c_int, C.c_int,
                                                    C.c_uint64, C.c_uint32, _i64, _u8p, _u8p]),
                 "ora_requant_transpose": (C.c_int, [_u8p, _u8p, _i64, _i64, C.c_int, C.c_uint64,
                                                     C.c_uint32, _u8p, _u8p]),
+                "ora_requant_transpose_rows": (C.c_int, [_u8p, _u8p, _i64, _i64, C.c_int, C.c_uint64,
+                                                         C.c_uint32, _i64, _i64, _u8p, _u8p]),
                 "ora_sf_swizzled_bytes": (_i64, [_i64, _i64]),
                 "ora_sf_offset": (_i64, [_i64, _i64, _i64]),
                 "ora_sf_swizzle": (None, [_u8p, _i64, _i64, _u8p]),
@@ -104,6 +113,33 @@ def _c(a, dtype):
 
 def _ptr(a):
     return None if a is None else a.ctypes.data_as(C.c_void_p)
+
+
+# ---------------------------------------------------------------- threads
+# Every oracle function below computes each output row on its own (the SR
+# draw index is the absolute output position, the amax a maximum), so the
+# rows can be split into bands and the bands run on separate threads (ctypes
+# releases the GIL during the C call) with results identical to one thread.
+def ncores() -> int:
+    """Host cores this process may run on."""
+    return len(os.sched_getaffinity(0))
+
+
+def _bands(R, parts, align=1):
+    units = -(-R // align)
+    parts = max(1, min(parts, units))
+    edges = [min(R, (units * i // parts) * align) for i in range(parts + 1)]
+    edges[-1] = R
+    return [(edges[i], edges[i + 1]) for i in range(parts) if edges[i] < edges[i + 1]]
+
+
+def _run_bands(fn, R, threads, align=1):
+    """fn(r0, r1) over bands of [0, R); returns the list of results in band order."""
+    bands = _bands(R, max(1, threads) * 4 if threads > 1 else 1, align)
+    if threads <= 1 or len(bands) <= 1:
+        return [fn(r0, r1) for r0, r1 in bands]
+    with ThreadPoolExecutor(threads) as ex:
+        return list(ex.map(lambda b: fn(*b), bands))
 
 
 # ---------------------------------------------------------------- formats
@@ -175,88 +211,155 @@ def rht_bf16(x, mask):
     return y
 
 
-def amax(x, rht_mask=None, row_index=None):
+def rht_f32(x, mask):
+    """The fused RHT's binary32 output y = 1/4 H16 diag(s) x for every group of
+    16 along K (ora_rht_f32)."""
+    x = _c(x, np.uint16)
+    M, K = x.shape
+    y = np.zeros((M, K), np.float32)
+    if lib().ora_rht_f32(x, y, M, K, int(mask)):
+        raise ValueError("K must be a multiple of 16")
+    return y
+
+
+def amax(x, rht_mask=None, row_index=None, threads=1):
     x = _c(x, np.uint16)
     M, K = x.shape
     ri = None if row_index is None else _c(row_index, np.int32)
     rows = M if ri is None else ri.shape[0]
-    return lib().ora_amax(x, rows, K, K, int(rht_mask is not None), int(rht_mask or 0), _ptr(ri))
+    L = lib()
+
+    def band(r0, r1):
+        if ri is None:
+            return L.ora_amax(x[r0:r1], r1 - r0, K, K, int(rht_mask is not None), int(rht_mask or 0), None)
+        sub = ri[r0:r1]
+        return L.ora_amax(x, r1 - r0, K, K, int(rht_mask is not None), int(rht_mask or 0), _ptr(sub))
+
+    if rows == 0:
+        return 0.0
+    return max(_run_bands(band, rows, threads))
 
 
 def nvfp4_global_scale(a):
     return lib().ora_nvfp4_global_scale(float(a))
 
 
-def quant_nvfp4(x, block_2d=False, four_over_six=False, rht_mask=None, row_index=None, amax_in=None):
-    """NVFP4 quantize (ora_quant_nvfp4).  Returns (codes [R,K/2] u8, sf [R,K/16] u8, s_g)."""
+def _nvfp4_common(x, block_2d, rht_mask, row_index, amax_in, threads, call):
+    """Shared driver of quant_nvfp4 / quant_nvfp4_sr: one call on the whole
+    tensor (threads == 1), or the tensor amax first and then bands of output
+    rows (16-row aligned for 16x16 tiles) with that amax given."""
     x = _c(x, np.uint16)
     M, K = x.shape
     ri = None if row_index is None else _c(row_index, np.int32)
     R = M if ri is None else ri.shape[0]
     codes = np.zeros((R, K // 2), np.uint8)
     sf = np.zeros((R, K // 16), np.uint8)
-    sg = np.zeros(1, np.float32)
-    am = None if amax_in is None else np.array([amax_in], np.float32)
-    rc = lib().ora_quant_nvfp4(x, R, K, K, int(block_2d), int(four_over_six), int(rht_mask is not None),
-                               int(rht_mask or 0), _ptr(ri), _ptr(am), sg, codes, sf)
-    if rc:
-        raise ValueError("unsupported NVFP4 shape/options")
-    return codes, sf, float(sg[0])
+    if threads <= 1 or R == 0:
+        sg = np.zeros(1, np.float32)
+        am = None if amax_in is None else np.array([amax_in], np.float32)
+        if call(x, R, ri, am, 0, sg, codes, sf):
+            raise ValueError("unsupported NVFP4 shape/options")
+        return codes, sf, float(sg[0])
+    if amax_in is None:
+        amax_in = amax(x, rht_mask, ri, threads=threads)
+    am = np.array([amax_in], np.float32)
+
+    def band(r0, r1):
+        sg = np.zeros(1, np.float32)
+        xs, sub = (x[r0:r1], None) if ri is None else (x, ri[r0:r1])
+        if call(xs, r1 - r0, sub, am, r0, sg, codes[r0:r1], sf[r0:r1]):
+            raise ValueError("unsupported NVFP4 shape/options")
+        return float(sg[0])
+
+    sgs = _run_bands(band, R, threads, 16 if block_2d else 1)
+    assert len(set(sgs)) == 1
+    return codes, sf, sgs[0]
 
 
-def quant_nvfp4_sr(x, block_2d=False, rht_mask=None, row_index=None, amax_in=None, seed=0, stream_id=0):
+def quant_nvfp4(x, block_2d=False, four_over_six=False, rht_mask=None, row_index=None, amax_in=None, threads=1):
+    """NVFP4 quantize (ora_quant_nvfp4).  Returns (codes [R,K/2] u8, sf [R,K/16] u8, s_g).
+    threads > 1 splits the output rows into bands (identical results)."""
+    K = np.shape(x)[1]
+    L = lib()
+
+    def call(xs, R, ri, am, row0, sg, codes, sf):
+        return L.ora_quant_nvfp4(xs, R, K, K, int(block_2d), int(four_over_six), int(rht_mask is not None),
+                                 int(rht_mask or 0), _ptr(ri), _ptr(am), sg, codes, sf)
+
+    return _nvfp4_common(x, block_2d, rht_mask, row_index, amax_in, threads, call)
+
+
+def quant_nvfp4_sr(x, block_2d=False, rht_mask=None, row_index=None, amax_in=None, seed=0, stream_id=0, threads=1):
     """NVFP4 quantize with stochastic rounding of the elements
-    (ora_quant_nvfp4_sr).  Returns (codes [R,K/2] u8, sf [R,K/16] u8, s_g)."""
-    x = _c(x, np.uint16)
-    M, K = x.shape
-    ri = None if row_index is None else _c(row_index, np.int32)
-    R = M if ri is None else ri.shape[0]
-    codes = np.zeros((R, K // 2), np.uint8)
-    sf = np.zeros((R, K // 16), np.uint8)
-    sg = np.zeros(1, np.float32)
-    am = None if amax_in is None else np.array([amax_in], np.float32)
-    rc = lib().ora_quant_nvfp4_sr(x, R, K, K, int(block_2d), int(rht_mask is not None), int(rht_mask or 0),
-                                  _ptr(ri), _ptr(am), int(seed), int(stream_id), sg, codes, sf)
-    if rc:
-        raise ValueError("unsupported NVFP4 shape/options")
-    return codes, sf, float(sg[0])
+    (ora_quant_nvfp4_sr_rows).  Returns (codes [R,K/2] u8, sf [R,K/16] u8, s_g)."""
+    K = np.shape(x)[1]
+    L = lib()
+
+    def call(xs, R, ri, am, row0, sg, codes, sf):
+        return L.ora_quant_nvfp4_sr_rows(xs, R, K, K, int(block_2d), int(rht_mask is not None), int(rht_mask or 0),
+                                         _ptr(ri), _ptr(am), int(seed), int(stream_id), int(row0), sg, codes, sf)
+
+    return _nvfp4_common(x, block_2d, rht_mask, row_index, amax_in, threads, call)
 
 
-def quant_mxfp4(x, sr=False, seed=0, stream_id=0):
-    """MXFP4 quantize (ora_quant_mxfp4), row-wise blocks of 32 along K.
+def quant_mxfp4(x, sr=False, seed=0, stream_id=0, threads=1):
+    """MXFP4 quantize (ora_quant_mxfp4_rows), row-wise blocks of 32 along K.
     Returns (codes [M,K/2] u8, sf [M,K/32] u8)."""
     x = _c(x, np.uint16)
     M, K = x.shape
     codes = np.zeros((M, K // 2), np.uint8)
     sf = np.zeros((M, K // 32), np.uint8)
-    if lib().ora_quant_mxfp4(x, M, K, K, int(sr), int(seed), int(stream_id), codes, sf):
-        raise ValueError("unsupported MXFP4 shape")
+    L = lib()
+
+    def band(r0, r1):
+        if L.ora_quant_mxfp4_rows(x[r0:r1], r1 - r0, K, K, int(sr), int(seed), int(stream_id), int(r0),
+                                  codes[r0:r1], sf[r0:r1]):
+            raise ValueError("unsupported MXFP4 shape")
+
+    _run_bands(band, M, threads)
     return codes, sf
 
 
-def quant_mxfp8(x, colwise=False, sr=False, seed=0, stream_id=0, out_row0=0):
+def quant_mxfp8(x, colwise=False, sr=False, seed=0, stream_id=0, out_row0=0, threads=1):
     """MXFP8 quantize (ora_quant_mxfp8_rows).  Returns (codes, sf) in the output
     orientation.  out_row0: index of the first output row within the full
-    output tensor (SR draw indices), for computing a band of rows alone."""
+    output tensor (SR draw indices), for computing a band of rows alone.
+    threads > 1 splits the output rows into bands (identical results)."""
     x = _c(x, np.uint16)
     M, K = x.shape
     R, Cc = (K, M) if colwise else (M, K)
     codes = np.zeros((R, Cc), np.uint8)
     sf = np.zeros((R, Cc // 32), np.uint8)
-    if lib().ora_quant_mxfp8_rows(x, M, K, K, int(colwise), int(sr), int(seed), int(stream_id), int(out_row0),
-                                  codes, sf):
-        raise ValueError("unsupported MXFP8 shape")
+    L = lib()
+
+    def band(r0, r1):
+        # output rows r0..r1: input rows (row-wise) or input columns (column-wise)
+        xs = x[r0:r1] if not colwise else np.ascontiguousarray(x[:, r0:r1])
+        m, k = (r1 - r0, K) if not colwise else (M, r1 - r0)
+        if L.ora_quant_mxfp8_rows(xs, m, k, k, int(colwise), int(sr), int(seed), int(stream_id), int(out_row0 + r0),
+                                  codes[r0:r1], sf[r0:r1]):
+            raise ValueError("unsupported MXFP8 shape")
+
+    if threads <= 1:
+        band(0, R)
+    else:
+        _run_bands(band, R, threads)
     return codes, sf
 
 
-def requant_transpose(codes, sf, sr=True, seed=0, stream_id=1):
+def requant_transpose(codes, sf, sr=True, seed=0, stream_id=1, threads=1):
     codes = _c(codes, np.uint8)
     sf = _c(sf, np.uint8)
     M, K = codes.shape
     cc = np.zeros((K, M), np.uint8)
     sc = np.zeros((K, M // 32), np.uint8)
-    if lib().ora_requant_transpose(codes, sf, M, K, int(sr), int(seed), int(stream_id), cc, sc):
-        raise ValueError("unsupported requant shape")
+    L = lib()
+
+    def band(k0, k1):
+        if L.ora_requant_transpose_rows(codes, sf, M, K, int(sr), int(seed), int(stream_id), k0, k1, cc, sc):
+            raise ValueError("unsupported requant shape")
+
+    _run_bands(band, K, threads)
     return cc, sc
 
 
@@ -287,14 +390,28 @@ def sf_unswizzle(buf, rows, nblk):
 NVFP4, MXFP8, MXFP4 = 0, 1, 2
 
 
-def dequant(fmt, codes, sf, s_g=1.0):
+def dequant(fmt, codes, sf, s_g=1.0, threads=1):
     codes = _c(codes, np.uint8)
     sf = _c(sf, np.uint8)
     R = codes.shape[0]
     K = codes.shape[1] * (1 if fmt == MXFP8 else 2)
     out = np.zeros((R, K), np.float64)
-    lib().ora_dequant(int(fmt), codes, sf, float(s_g), R, K, out)
+    L = lib()
+
+    def band(r0, r1):
+        L.ora_dequant(int(fmt), codes[r0:r1], sf[r0:r1], float(s_g), r1 - r0, K, out[r0:r1])
+
+    _run_bands(band, R, threads)
     return out
+
+
+def gemm_f64_blas(A, B):
+    """C = A B^T and sum_k |A[m,k]| |B[n,k]| in binary64, each as one call of
+    the BLAS matrix product (a library primitive; it uses every core).  The
+    same definition as ora_gemm_f64, summed in the library's order."""
+    A = _c(A, np.float64)
+    B = _c(B, np.float64)
+    return A @ B.T, np.abs(A) @ np.abs(B).T
 
 
 def gemm_f64(A, B):

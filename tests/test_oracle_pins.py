@@ -811,3 +811,119 @@ def test_nvfp4_sr_unbiased_over_seeds(ora):
     target = np.sign(q) * a * dn
     dev = acc / n - target
     assert (np.abs(dev) <= 5 * sig * dn / np.sqrt(n) + 1e-300).all()
+
+
+# --------------------------------------------------------------------- NVFP4 codes off the grid
+def _nvfp4_workload(kind, M, K):
+    """Student-t (the MXFP8 workload's recipe) or N(0,1) with outlier channels
+    x100 (the NVFP4-with-RHT workload's A), bf16 bits."""
+    if kind == "student_t":
+        return W.bf16_bits(W.mxfp8_requant(M=M, K=K, seed=21))
+    return W.bf16_bits(W.nvfp4_linear_rht(M=M, N=16, K=K, seed=22)[0])
+
+
+@pytest.mark.parametrize("kind", ["student_t", "outliers"])
+@pytest.mark.parametrize("rht", [False, True])
+@pytest.mark.parametrize("block_2d", [False, True])
+def test_nvfp4_rne_codes_are_nearest_e2m1(ora, kind, rht, block_2d):
+    """MX page "NVFP4" / FP4 page "Bit layout of FP4 E2M1": on values that are
+    not representable, every code of the nearest-even quantization is the
+    E2M1 value of the pages' list nearest to q = x * r under the stored scale
+    (r = RN(1 / RN(sb * s_g))), ties to the even code, saturating at 6; every
+    scale is E4M3(RN(RN(block_amax / 6) / s_g)) by torch's cast; s_g is
+    RN(amax / 2688).  The block values are the RHT output when it is on (the
+    RHT itself is pinned below against scipy's Hadamard matrix)."""
+    from nvfp4_props import check_nvfp4
+    x = _nvfp4_workload(kind, 128, 512)
+    mask = 0xB5C3 if rht else None
+    y = ora.rht_f32(x, mask) if rht else (x.astype(np.uint32) << 16).view(np.float32)
+    c, s, sg = ora.quant_nvfp4(x, block_2d=block_2d, rht_mask=mask)
+    check_nvfp4(y, c, s, sg, block_2d=block_2d, what=f"{kind} rht={rht} 2d={block_2d}")
+    # the check is not vacuous: the codes span the grid and most values are off it
+    mags = np.unique(c & 0x77)
+    assert len(mags) > 10
+
+
+@pytest.mark.parametrize("kind", ["student_t", "outliers"])
+@pytest.mark.parametrize("rht", [False, True])
+def test_four_over_six_codes_and_scales_on_the_workloads(ora, kind, rht):
+    """TML page "A precision choice for each stage" (Four Over Six) on the
+    workload distributions: every code is the nearest E2M1 value under the
+    stored scale, the scale is one of the two candidates, and where the
+    binary64 errors differ the lower-error candidate was kept."""
+    from nvfp4_props import check_nvfp4
+    x = _nvfp4_workload(kind, 128, 512)
+    mask = 0x3A5C if rht else None
+    y = ora.rht_f32(x, mask) if rht else (x.astype(np.uint32) << 16).view(np.float32)
+    c, s, sg = ora.quant_nvfp4(x, four_over_six=True, rht_mask=mask)
+    picked4 = check_nvfp4(y, c, s, sg, four_over_six=True, what=f"4/6 {kind} rht={rht}")
+    assert picked4 > 0
+
+
+def test_property_check_catches_planted_mistakes(ora):
+    """The property check above fails on each plausible mistake planted in an
+    oracle result: a code moved one step, a scale moved one step, a wrong s_g."""
+    from nvfp4_props import check_nvfp4
+    x = _nvfp4_workload("outliers", 32, 256)
+    y = (x.astype(np.uint32) << 16).view(np.float32)
+    c, s, sg = ora.quant_nvfp4(x)
+    check_nvfp4(y, c, s, sg)
+    for mutate in range(3):
+        c2, s2, sg2 = c.copy(), s.copy(), sg
+        if mutate == 0:
+            i = np.argwhere((c2 & 0x7) > 1)[0]
+            c2[tuple(i)] -= 1
+        elif mutate == 1:
+            s2[3, 2] += 1
+        else:
+            sg2 = float(np.nextafter(np.float32(sg), np.float32(1)))
+        with pytest.raises(AssertionError):
+            check_nvfp4(y, c2, s2, sg2)
+
+
+# --------------------------------------------------------------------- the threaded oracle
+def test_threaded_oracle_equals_serial_byte_for_byte(ora):
+    """Bands of output rows on several threads (the full-size parity tests'
+    oracle) give the serial oracle's bytes exactly, for every function."""
+    T = 4
+    A, Wt, seed = W.nvfp4_linear_rht(M=288, N=160, K=512)
+    xa, xw = W.bf16_bits(A), W.bf16_bits(Wt)
+    mask = ora.rht_sign_mask(seed)
+    ri = np.random.default_rng(2).integers(0, 288, 333).astype(np.int32)
+
+    def same(a, b):
+        assert len(a) == len(b)
+        for u, v in zip(a, b):
+            assert np.array_equal(np.asarray(u), np.asarray(v))
+
+    assert ora.amax(xa, rht_mask=mask, threads=T) == ora.amax(xa, rht_mask=mask)
+    assert ora.amax(xa, row_index=ri, threads=T) == ora.amax(xa, row_index=ri)
+    same(ora.quant_nvfp4(xa, rht_mask=mask, threads=T), ora.quant_nvfp4(xa, rht_mask=mask))
+    same(ora.quant_nvfp4(xw, block_2d=True, rht_mask=mask, threads=T),
+         ora.quant_nvfp4(xw, block_2d=True, rht_mask=mask))
+    same(ora.quant_nvfp4(xa, four_over_six=True, row_index=ri, threads=T),
+         ora.quant_nvfp4(xa, four_over_six=True, row_index=ri))
+    same(ora.quant_nvfp4_sr(xa, rht_mask=mask, seed=9, stream_id=2, threads=T),
+         ora.quant_nvfp4_sr(xa, rht_mask=mask, seed=9, stream_id=2))
+    same(ora.quant_nvfp4_sr(xw, block_2d=True, seed=9, threads=T), ora.quant_nvfp4_sr(xw, block_2d=True, seed=9))
+    for colwise in (False, True):
+        for sr in (False, True):
+            same(ora.quant_mxfp8(xa, colwise=colwise, sr=sr, seed=4, stream_id=1, threads=T),
+                 ora.quant_mxfp8(xa, colwise=colwise, sr=sr, seed=4, stream_id=1))
+    same(ora.quant_mxfp4(xa, sr=True, seed=3, threads=T), ora.quant_mxfp4(xa, sr=True, seed=3))
+    cm, sm = ora.quant_mxfp8(xa, sr=True, seed=1)
+    same(ora.requant_transpose(cm, sm, seed=1, threads=T), ora.requant_transpose(cm, sm, seed=1))
+    q = ora.quant_nvfp4(xa)
+    same([ora.dequant(ora.NVFP4, *q, threads=T)], [ora.dequant(ora.NVFP4, *q)])
+
+
+def test_blas_gemm_equals_the_plain_sum(ora):
+    """The BLAS form of the oracle GEMM (used at full size) against the plain
+    binary64 loop: same C and sum |a||b| up to binary64 rounding."""
+    rng = np.random.default_rng(5)
+    A = rng.standard_normal((37, 96))
+    B = rng.standard_normal((29, 96))
+    C1, R1 = ora.gemm_f64(A, B)
+    C2, R2 = ora.gemm_f64_blas(A, B)
+    assert np.allclose(C1, C2, rtol=0, atol=1e-12 * R1.max())
+    assert np.allclose(R1, R2, rtol=1e-13, atol=0)

@@ -60,7 +60,7 @@ void philox_host(uint32_t c[4], uint32_t k0, uint32_t k1) {
 }
 
 // Kernel-selection overrides (bsq_debug_kernel_choice): -1 = automatic.
-std::atomic<int> g_knob[3] = {{-1}, {-1}, {-1}};
+std::atomic<int> g_knob[4] = {{-1}, {-1}, {-1}, {-1}};
 
 }  // namespace
 
@@ -74,6 +74,7 @@ int bsq_debug_kernel_choice(int knob, int value) {
     switch (knob) {
         case BSQ_KNOB_FUSED_QUANT:
         case BSQ_KNOB_GEMM_PAIR:
+        case BSQ_KNOB_STREAM_QUANT:
             if (value < -1 || value > 1) return BSQ_ERR_INVALID;
             break;
         case BSQ_KNOB_GEMM_BN:
@@ -109,6 +110,8 @@ uint16_t bsq_rht_sign_mask(uint64_t seed) {
     return (uint16_t)(c[0] & 0xFFFFu);
 }
 
+static bool stream_enabled();
+
 int bsq_amax(const void *x, int64_t M, int64_t K, int64_t ldx, int rht_enable, uint16_t mask,
              const int32_t *row_index, float *amax_dev, void *stream) {
     if (!x || !amax_dev || M < 0 || K < 0 || K % 16 || ldx < K) return BSQ_ERR_INVALID;
@@ -118,6 +121,13 @@ int bsq_amax(const void *x, int64_t M, int64_t K, int64_t ldx, int rht_enable, u
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (cudaMemsetAsync(amax_dev, 0, sizeof(float), s) != cudaSuccess) return BSQ_ERR_CUDA;
     if (M == 0 || K == 0) return BSQ_OK;
+    if (!row_index && ldx == K && stream_enabled() && bsq::stream_ok(M, K, false)) {
+        if (bsq::launch_nvfp4_stream(0, static_cast<const uint16_t *>(x), M, K, false, rht_enable != 0, mask, nullptr,
+                                     reinterpret_cast<unsigned int *>(amax_dev), nullptr, false, nullptr, nullptr,
+                                     nullptr, d->err, d->num_sms, s) != 0)
+            return BSQ_ERR_CUDA;
+        return launch_status();
+    }
     bsq::launch_amax(static_cast<const uint16_t *>(x), M, K, ldx, rht_enable != 0, mask, row_index,
                      reinterpret_cast<unsigned int *>(amax_dev), nullptr, nullptr, d->num_sms, s);
     return launch_status();
@@ -127,6 +137,9 @@ int bsq_amax(const void *x, int64_t M, int64_t K, int64_t ldx, int rht_enable, u
 // (bsq_debug_kernel_choice(BSQ_KNOB_FUSED_QUANT, 0)) for tuning and for
 // tests of the two-pass path.
 static bool fused_enabled() { return bsq::kernel_choice(BSQ_KNOB_FUSED_QUANT) != 0; }
+// The bulk-copy streaming kernels for contiguous tensors can be switched off
+// (BSQ_KNOB_STREAM_QUANT = 0) in favour of the register-streaming ones.
+static bool stream_enabled() { return bsq::kernel_choice(BSQ_KNOB_STREAM_QUANT) != 0; }
 
 int bsq_quant_nvfp4(const void *x, int64_t M, int64_t K, int64_t ldx, int block_2d, int four_over_six,
                     int rht_enable, uint16_t mask, const int32_t *row_index, int G, const int32_t *row_off,
@@ -148,12 +161,30 @@ int bsq_quant_nvfp4(const void *x, int64_t M, int64_t K, int64_t ldx, int block_
         bsq::launch_finalize_global_scale(gs, s);
         return launch_status();
     }
+    const bool streamable = !row_index && G == 0 && ldx == K && !four_over_six && stream_enabled() &&
+                            bsq::stream_ok(M, K, block_2d != 0);
     if (amax_in == nullptr) {
         // The amax pass uses the first 8 bytes of the caller's code buffer
         // (overwritten by the quantize pass that follows on the same stream)
         // as its scratch: a CTA counter and the amax bits.  Its last CTA
         // writes s_g to *gs, which the quantize pass reads.
         if (cudaMemsetAsync(codes, 0, 8, s) != cudaSuccess) return BSQ_ERR_CUDA;
+        if (streamable) {
+            unsigned int *scratch = reinterpret_cast<unsigned int *>(codes);
+            int rc;
+            if (fused_enabled()) {
+                // amax and quantize in one cooperative launch
+                rc = bsq::launch_nvfp4_stream(2, xx, M, K, block_2d != 0, rht_enable != 0, mask, scratch, scratch + 1,
+                                              nullptr, false, gs, codes, sf, d->err, d->num_sms, s);
+            } else {
+                rc = bsq::launch_nvfp4_stream(0, xx, M, K, block_2d != 0, rht_enable != 0, mask, scratch, scratch + 1,
+                                              nullptr, false, gs, nullptr, nullptr, d->err, d->num_sms, s);
+                if (rc == 0)
+                    rc = bsq::launch_nvfp4_stream(1, xx, M, K, block_2d != 0, rht_enable != 0, mask, nullptr, nullptr,
+                                                  gs, false, nullptr, codes, sf, d->err, d->num_sms, s);
+            }
+            return rc ? BSQ_ERR_CUDA : launch_status();
+        }
         const int64_t KB = K / 16;
         // (1x16 tensors measure faster with the two-pass path: 37.2 vs 38.3 us
         // on 8192x4096, where the fused kernel's lower occupancy outweighs the
@@ -171,6 +202,14 @@ int bsq_quant_nvfp4(const void *x, int64_t M, int64_t K, int64_t ldx, int block_
         bsq::launch_amax(xx, M, K, ldx, rht_enable != 0, mask, row_index, scratch + 1, scratch, gs, d->num_sms, s);
         bsq::launch_quant_nvfp4(xx, M, K, ldx, block_2d != 0, four_over_six != 0, rht_enable != 0, mask, row_index,
                                 G, row_off, sf_off, gs, false, gs, false, codes, sf, d->num_sms, s);
+    } else if (streamable) {
+        // amax given: the quantize pass alone (in place: *gs holds the amax
+        // and becomes s_g after the pass)
+        const bool in_place = amax_in == gs;
+        if (bsq::launch_nvfp4_stream(1, xx, M, K, block_2d != 0, rht_enable != 0, mask, nullptr, nullptr, amax_in, true,
+                                     in_place ? nullptr : gs, codes, sf, d->err, d->num_sms, s) != 0)
+            return BSQ_ERR_CUDA;
+        if (in_place) bsq::launch_finalize_global_scale(gs, s);
     } else if (amax_in == gs) {
         // the caller's amax is in *gs: read it, then replace it by s_g in place
         bsq::launch_quant_nvfp4(xx, M, K, ldx, block_2d != 0, four_over_six != 0, rht_enable != 0, mask, row_index,

@@ -31,6 +31,10 @@ BSQ_DEV uint64_t globaltimer_ns() {
     return t;
 }
 
+// Sets cudaFuncAttributeMaxDynamicSharedMemorySize of `kern` to `bytes` on
+// the current device, once per (kernel, device); BSQ_OK or BSQ_ERR_CUDA.
+int smem_attr_once(const void *kern, int bytes);
+
 // ---------------------------------------------------------------- bf16
 BSQ_DEV float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 BSQ_DEV float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }

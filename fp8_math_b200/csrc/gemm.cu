@@ -1010,6 +1010,29 @@ void launch_timeout_probe(uint64_t timeout_ns, unsigned int *err, cudaStream_t s
 }
 
 // ============================================================ host side
+// The dynamic shared-memory limit of a kernel is a per-device attribute:
+// set it once per (kernel, device), under a lock, and remember the outcome.
+int smem_attr_once(const void *kern, int bytes) {
+    struct Entry {
+        const void *kern;
+        int dev;
+        int status;
+    };
+    static std::mutex mu;
+    static Entry done[256];
+    static int ndone = 0;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return BSQ_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(mu);
+    for (int i = 0; i < ndone; i++)
+        if (done[i].kern == kern && done[i].dev == dev) return done[i].status;
+    const int st = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess
+                       ? BSQ_OK
+                       : BSQ_ERR_CUDA;
+    if (st == BSQ_OK && ndone < 256) done[ndone++] = {kern, dev, st};
+    return st;
+}
+
 namespace {
 
 using EncodeFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
@@ -1070,30 +1093,6 @@ bool make_c_tmap(CUtensorMap *m, void *C, bool bf16, int64_t n_cols, int64_t row
     return enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, C, dims, strides, box,
                estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-// The dynamic shared-memory limit of a kernel is a per-device attribute:
-// set it once per (kernel, device), under a lock, and remember the outcome.
-constexpr int kMaxDev = 64;
-int smem_attr_once(const void *kern, int bytes) {
-    struct Entry {
-        const void *kern;
-        int dev;
-        int status;
-    };
-    static std::mutex mu;
-    static Entry done[256];
-    static int ndone = 0;
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return BSQ_ERR_CUDA;
-    std::lock_guard<std::mutex> lk(mu);
-    for (int i = 0; i < ndone; i++)
-        if (done[i].kern == kern && done[i].dev == dev) return done[i].status;
-    const int st = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess
-                       ? BSQ_OK
-                       : BSQ_ERR_CUDA;
-    if (st == BSQ_OK && ndone < 256) done[ndone++] = {kern, dev, st};
-    return st;
 }
 
 template <int FMT, bool OUT_BF16, bool GROUPED>

@@ -11,6 +11,7 @@
 
 #include "common.cuh"
 #include "quant.cuh"
+#include "sm100.cuh"
 
 namespace bsq {
 
@@ -602,6 +603,344 @@ __global__ void __launch_bounds__(256) quant_nvfp4_fused_kernel(
     }
 }
 
+// Division by an invariant divisor d <= 2^31 for n < 2^32 (Granlund and
+// Montgomery, PLDI 1994): with s = ceil(log2 d) and m = ceil(2^(32+s) / d),
+// floor(n / d) = (n * m) >> (32 + s).  m < 2^33 is kept in 64 bits.
+struct DivU32 {
+    uint64_t m;
+    int sh;
+};
+static DivU32 divu32_for(uint32_t d) {
+    int s = 0;
+    while ((uint64_t(1) << s) < d) s++;
+    const unsigned __int128 num = (unsigned __int128)1 << (32 + s);
+    return {(uint64_t)((num + d - 1) / d), 32 + s};
+}
+BSQ_DEV uint32_t divu32(uint32_t n, const DivU32 &dv) {
+    return (uint32_t)(((unsigned __int128)n * dv.m) >> dv.sh);
+}
+
+
+// ===================================================================== streaming NVFP4 (bulk-copy ring)
+// Contiguous tensors (ldx == K, K % 64 == 0).  A CTA is one producer warp
+// and eight consumer warps.  The producer's lane 0 streams chunks of the
+// tensor into a ring of shared-memory stages with cp.async.bulk (completion
+// on the stage's "full" mbarrier); the consumers read a stage, release it
+// (one arrive per warp on its "empty" mbarrier) and compute.  The loads run
+// ahead of the arithmetic by the whole ring, so every SM keeps
+// kStages * 16 KB in flight whatever the consumers are doing.
+//   1x16:  chunk = 512 consecutive blocks of 16 (16 KB); consumer thread t
+//          takes blocks t and t + 256.
+//   16x16: chunk = 16 rows x 512 columns (16 row copies of 1 KB, staged at a
+//          1040-byte row stride so that the reads below hit distinct banks);
+//          consumer thread t takes row t % 16, blocks 2 (t / 16) and
+//          2 (t / 16) + 1 of the chunk: a half-warp holds one tile column.
+// Modes: AMAX (amax only, into *amax_bits; with a counter the last CTA
+// also writes s_g),
+// QUANT (s_g from a given amax or scale), FUSED (amax over every chunk, a
+// grid barrier, then the quantization in reverse chunk order so the most
+// recently read lines come from L2; cooperative launch).  Every wait is
+// bounded; on expiry the error word is set, the CTA drains its own copies
+// and returns.
+namespace nvs {
+constexpr int kConsumerWarps = 8;
+constexpr int kThreads = 32 * (1 + kConsumerWarps);
+constexpr int kStages = 4;
+constexpr int kRowStride = 1040;                 // 16x16: bytes per staged row (1 KB + 16)
+constexpr int kStageBytes = 16 * kRowStride;     // also holds a 16 KB 1x16 chunk
+constexpr int kSmemBytes = kStages * kStageBytes;
+constexpr uint64_t kTimeoutNs = 2000000000ull;
+enum { AMAX = 0, QUANT = 1, FUSED = 2 };
+}  // namespace nvs
+
+// Consumer-only barrier (named barrier 1: the 256 consumer threads).
+BSQ_DEV void consumers_sync() { asm volatile("bar.sync 1, %0;" ::"n"(32 * nvs::kConsumerWarps) : "memory"); }
+
+// Chunk geometry.  1x16: chunk c covers flat blocks [512 c, 512 c + 512).
+// 16x16: chunk c = (row group rg, span sp) covers rows 16 rg .. 16 rg + 15
+// and columns 512 sp .. 512 sp + 511 (the last span may be shorter).
+struct NvChunks {
+    int64_t M, K, KB, nblk;
+    int64_t nspan;   // 16x16: spans per row group
+    int64_t count;
+};
+
+template <bool TWO_D>
+BSQ_DEV NvChunks nv_chunks(int64_t M, int64_t K) {
+    NvChunks g;
+    g.M = M;
+    g.K = K;
+    g.KB = K >> 4;
+    g.nblk = M * g.KB;
+    g.nspan = (K + 511) >> 9;
+    g.count = TWO_D ? (M >> 4) * g.nspan : (g.nblk + 511) >> 9;
+    return g;
+}
+
+template <int MODE, bool RHT, bool TWO_D>
+__global__ void __launch_bounds__(nvs::kThreads, 2) quant_nvfp4_stream_kernel(
+    const uint16_t *__restrict__ x, int64_t M, int64_t K, DivU32 div_kb, uint32_t mask, unsigned int *counter,
+    unsigned int *amax_bits, const float *scale_src, int src_is_amax, float *gs_out, uint8_t *__restrict__ codes,
+    uint8_t *__restrict__ sf, unsigned int *err) {
+    using namespace sm100;
+    extern __shared__ __align__(128) uint8_t ring[];
+    __shared__ __align__(8) uint64_t full_bar[nvs::kStages], empty_bar[nvs::kStages];
+    __shared__ float den_tab[128], rcp_tab[128];
+    __shared__ float red[nvs::kConsumerWarps];
+    __shared__ volatile int abort_flag;
+    __shared__ int ok_sh;
+    const NvChunks g = nv_chunks<TWO_D>(M, K);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // chunks of this CTA: c = blockIdx.x + i * gridDim.x, i < my
+    const int64_t my = blockIdx.x < g.count ? (g.count - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+    const int64_t total = (MODE == nvs::FUSED ? 2 : 1) * my;  // stage fills in this CTA's sequence
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < nvs::kStages; i++) {
+            mbar_init(smem_u32(&full_bar[i]), 1);
+            mbar_init(smem_u32(&empty_bar[i]), nvs::kConsumerWarps);
+        }
+        abort_flag = 0;
+        fence_barrier_init();
+    }
+    __syncthreads();
+    // j-th fill of the sequence -> chunk index (FUSED: forward, then reverse)
+    auto chunk_of = [&](int64_t j) -> int64_t {
+        const int64_t i = (MODE == nvs::FUSED && j >= my) ? (2 * my - 1 - j) : j;
+        return blockIdx.x + i * gridDim.x;
+    };
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        uint32_t armed = 0, armed_par = 0;
+        for (int64_t j = 0; j < total; j++) {
+            const int s = (int)(j % nvs::kStages);
+            const uint32_t ph = (uint32_t)((j / nvs::kStages) & 1);
+            bool ok = true;
+            if (lane == 0) ok = mbar_wait(smem_u32(&empty_bar[s]), ph ^ 1u, &abort_flag, err, 30, nvs::kTimeoutNs);
+            if (!__shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0)) break;
+            const int64_t c = chunk_of(j);
+            uint8_t *dst = ring + s * nvs::kStageBytes;
+            const uint32_t fb = smem_u32(&full_bar[s]);
+            if (!TWO_D) {
+                if (lane == 0) {
+                    const int64_t b0 = c << 9;
+                    const int64_t nb = (g.nblk - b0) < 512 ? (g.nblk - b0) : 512;
+                    mbar_arrive_expect_tx(fb, (uint32_t)(nb * 32));
+                    bulk_load(smem_u32(dst), x + b0 * 16, (uint32_t)(nb * 32), fb);
+                }
+            } else {
+                const int64_t rg = c / g.nspan, sp = c - rg * g.nspan;
+                const int64_t k0 = sp << 9;
+                const int64_t cols = (K - k0) < 512 ? (K - k0) : 512;
+                if (lane == 0) mbar_arrive_expect_tx(fb, (uint32_t)(16 * cols * 2));
+                __syncwarp();
+                if (lane < 16)
+                    bulk_load(smem_u32(dst + lane * nvs::kRowStride), x + (rg * 16 + lane) * K + k0,
+                              (uint32_t)(cols * 2), fb);
+            }
+            armed |= 1u << s;
+            armed_par = (armed_par & ~(1u << s)) | (ph << s);
+        }
+        // before exit every copy of this CTA has landed (normally the
+        // consumers have already waited for all of them)
+        if (lane == 0)
+            for (int i = 0; i < nvs::kStages; i++)
+                if (armed & (1u << i)) {
+                    volatile int never = 0;
+                    mbar_wait(smem_u32(&full_bar[i]), (armed_par >> i) & 1u, &never, err, 31, nvs::kTimeoutNs);
+                }
+        return;
+    }
+
+    // ---------------------------------------------------------------- consumers
+    const int t = threadIdx.x - 32;  // 0..255
+    uint32_t sw[8];
+    rht_sign_words(mask, sw);
+    int64_t j = 0;
+    // waits for fill j; false when the CTA gives up
+    auto acquire = [&](int64_t jj) -> const uint8_t * {
+        const int s = (int)(jj % nvs::kStages);
+        const uint32_t ph = (uint32_t)((jj / nvs::kStages) & 1);
+        const bool ok = mbar_wait(smem_u32(&full_bar[s]), ph, &abort_flag, err, 32, nvs::kTimeoutNs);
+        if (!__all_sync(0xFFFFFFFFu, ok)) return nullptr;
+        return ring + s * nvs::kStageBytes;
+    };
+    auto release = [&](int64_t jj) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&empty_bar[jj % nvs::kStages]));
+    };
+    // the 8 words of 1x16 block `slot` (0..511) of a staged chunk; the two
+    // 16-byte halves are read in an order that spreads each quarter-warp
+    // over all 32 banks
+    auto words_1d = [&](const uint8_t *st, int slot, uint32_t w[8]) {
+        const int h = (slot >> 2) & 1;
+        const uint4 a = *reinterpret_cast<const uint4 *>(st + slot * 32 + 16 * h);
+        const uint4 b = *reinterpret_cast<const uint4 *>(st + slot * 32 + 16 * (h ^ 1));
+        const uint4 lo = h ? b : a, hi = h ? a : b;
+        w[0] = lo.x; w[1] = lo.y; w[2] = lo.z; w[3] = lo.w;
+        w[4] = hi.x; w[5] = hi.y; w[6] = hi.z; w[7] = hi.w;
+    };
+    auto words_2d = [&](const uint8_t *st, int row, int blk, uint32_t w[8]) {
+        const uint4 a = *reinterpret_cast<const uint4 *>(st + row * nvs::kRowStride + blk * 32);
+        const uint4 b = *reinterpret_cast<const uint4 *>(st + row * nvs::kRowStride + blk * 32 + 16);
+        w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
+        w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
+    };
+
+    // A wait that gives up sets the CTA's abort flag; the consumer warps then
+    // skip the rest of the work but still pass every named barrier below.
+    bool alive = true;
+    float s_g = 1.0f;
+    if (MODE != nvs::QUANT) {
+        // ---- amax over this CTA's chunks
+        float m = 0.0f;
+        for (; j < my && alive; j++) {
+            const uint8_t *st = acquire(j);
+            if (!st) {
+                alive = false;
+                break;
+            }
+            const int64_t c = chunk_of(j);
+            if (!TWO_D) {
+                const int64_t nb = g.nblk - (c << 9);
+                uint32_t w0[8], w1[8];
+                if (t < nb) words_1d(st, t, w0);
+                if (t + 256 < nb) words_1d(st, t + 256, w1);
+                release(j);
+                if (t < nb) m = fmaxf(m, block_absmax<RHT>(w0, sw));
+                if (t + 256 < nb) m = fmaxf(m, block_absmax<RHT>(w1, sw));
+            } else {
+                const int64_t sp = c % g.nspan;
+                const int64_t nb = (K - (sp << 9)) >> 4;
+                const int row = t & 15, b0 = 2 * (t >> 4);
+                uint32_t w0[8], w1[8];
+                if (b0 < nb) words_2d(st, row, b0, w0);
+                if (b0 + 1 < nb) words_2d(st, row, b0 + 1, w1);
+                release(j);
+                if (b0 < nb) m = fmaxf(m, block_absmax<RHT>(w0, sw));
+                if (b0 + 1 < nb) m = fmaxf(m, block_absmax<RHT>(w1, sw));
+            }
+        }
+#pragma unroll
+        for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+        if (lane == 0) red[warp - 1] = m;
+        consumers_sync();
+        if (t == 0) {
+            ok_sh = 0;
+            if (!abort_flag) {
+                float b = red[0];
+                for (int i = 1; i < nvs::kConsumerWarps; i++) b = fmaxf(b, red[i]);
+                atomicMax(amax_bits, __float_as_uint(b));
+                __threadfence();
+                if (MODE == nvs::AMAX) {
+                    // with a counter, the last CTA turns the amax into s_g
+                    if (counter && atomicAdd(counter, 1u) == gridDim.x - 1) {
+                        __threadfence();
+                        *gs_out = global_scale_of(__uint_as_float(atomicOr(amax_bits, 0u)));
+                    }
+                } else {
+                    atomicAdd(counter, 1u);
+                    ok_sh = wait_counter(counter, gridDim.x, err, 33);
+                    if (!ok_sh) abort_flag = 1;   // the producer stops too
+                }
+            }
+        }
+        if (MODE == nvs::AMAX) return;
+        consumers_sync();
+        if (ok_sh) {
+            s_g = global_scale_of(__uint_as_float(ld_acquire_gpu(amax_bits)));
+        } else {
+            alive = false;
+        }
+        consumers_sync();
+        if (t == 0 && alive) atomicAdd(counter, 1u);  // this CTA has read the amax
+        if (alive && blockIdx.x == 0 && t == 0) *gs_out = s_g;
+    } else {
+        s_g = src_is_amax ? global_scale_of(*scale_src) : *scale_src;
+        if (gs_out && blockIdx.x == 0 && t == 0) *gs_out = s_g;
+    }
+    // den / rcp tables (threads 0..127 of the consumers)
+    if (t < 128) {
+        const float den = __fmul_rn(e4m3_to_f32(t), s_g);
+        den_tab[t] = den;
+        rcp_tab[t] = (t == 0 || t == 127) ? 0.0f : __frcp_rn(den);
+    }
+    consumers_sync();
+    NvScale cs;
+    cs.s_g = s_g;
+    cs.c6 = __frcp_rn(__fmul_rn(6.0f, s_g));
+    cs.c4 = __frcp_rn(__fmul_rn(4.0f, s_g));
+    cs.fast = s_g >= 0x1p-90f && s_g <= 0x1p100f;
+    const unsigned int all_read = 2u * gridDim.x;
+
+    // ---- quantize this CTA's chunks (FUSED: in reverse order)
+    const int64_t jend = (MODE == nvs::FUSED) ? 2 * my : my;
+    for (; j < jend && alive; j++) {
+        const uint8_t *st = acquire(j);
+        if (!st) break;
+        const int64_t c = chunk_of(j);
+        if (!TWO_D) {
+            const int64_t b0 = c << 9;
+            const int64_t nb = g.nblk - b0;
+            uint32_t w0[8], w1[8];
+            words_1d(st, t, w0);   // slots past the tensor's end hold stale bytes: never stored
+            words_1d(st, t + 256, w1);
+            release(j);
+#pragma unroll
+            for (int h = 0; h < 2; h++) {
+                const int slot = t + 256 * h;
+                const bool v = slot < nb;
+                const int64_t b = b0 + slot;
+                uint32_t sb;
+                uint2 cd;
+                nv_block_1d<RHT, false>(h ? w1 : w0, sw, cs, den_tab, rcp_tab, sb, cd);
+                // the first block's codes double as the amax scratch: written
+                // once every CTA has read the amax
+                if (MODE == nvs::FUSED && v && b == 0 && !wait_counter(counter, all_read, err, 34))
+                    cd = make_uint2(0u, 0u);
+                if (v) *reinterpret_cast<uint2 *>(codes + b * 8) = cd;
+                const int64_t row = divu32((uint32_t)b, div_kb);
+                store_sf(sf, v, sb, row, b - row * g.KB, g.KB, true);
+            }
+        } else {
+            const int64_t rg = c / g.nspan, sp = c - rg * g.nspan;
+            const int64_t nb = (K - (sp << 9)) >> 4;      // blocks in this span (multiple of 4)
+            const int row = t & 15, bp = t >> 4;
+            const int64_t grow = rg * 16 + row;
+            const int64_t kb0 = (sp << 5) + 2 * bp;        // first block of this thread
+            const bool v = 2 * bp < nb;                    // both blocks valid (nb is even)
+            uint32_t w[2][8];
+            words_2d(st, row, v ? 2 * bp : 0, w[0]);
+            words_2d(st, row, v ? 2 * bp + 1 : 0, w[1]);
+            release(j);
+            uint2 cd[2];
+            uint32_t sbw = 0;
+#pragma unroll
+            for (int i = 0; i < 2; i++) {
+                f32x2 P[8];
+                if (RHT) rht16_u_words(w[i], sw, P);
+                else words_to_pairs(w[i], P);
+                float mu = v ? pairs_absmax3(P) : 0.0f;
+#pragma unroll
+                for (int o = 1; o < 16; o <<= 1) mu = fmaxf(mu, __shfl_xor_sync(0xFFFFFFFFu, mu, o));
+                const float tmax = RHT ? __fmul_rn(mu, 0.25f) : mu;
+                const uint32_t sb = nv_scale_code(tmax, 6.0f, cs.c6, cs);
+                sbw |= (sb & 0xFFu) << (8 * i);
+                cd[i] = sb ? nv_codes<RHT>(P, rcp_tab[sb], cs.fast) : make_uint2(0u, 0u);
+            }
+            if (MODE == nvs::FUSED && v && grow == 0 && kb0 == 0 && !wait_counter(counter, all_read, err, 35))
+                cd[0] = make_uint2(0u, 0u);
+            if (v)
+                *reinterpret_cast<uint4 *>(codes + grow * (K >> 1) + kb0 * 8) =
+                    make_uint4(cd[0].x, cd[0].y, cd[1].x, cd[1].y);
+            // lanes l and l + 16 hold blocks 4i .. 4i + 3 of one row: one word
+            const uint32_t other = __shfl_down_sync(0xFFFFFFFFu, sbw, 16);
+            if (v && lane < 16)
+                *reinterpret_cast<uint32_t *>(sf + sf_word_offset(grow, kb0 >> 2, g.KB)) = sbw | (other << 16);
+        }
+    }
+}
+
 // ===================================================================== MXFP8
 // E8M0 code of a block from its absolute maximum m >= 0, i.e.
 // clamp(floor(log2 m) - 8, -127, 127) + 127.  The biased exponent field f of
@@ -853,23 +1192,6 @@ __global__ void __launch_bounds__(256) quant_mxfp8_row_kernel(
 // Lanes 4j..4j+3 hold one block of 32 (two-step shuffle max); lanes 16i hold
 // the first of four consecutive blocks of one row and store their scale
 // word.  The SR draw index of a chunk is its flat position (row * K + col).
-// Division by an invariant divisor d <= 2^31 for n < 2^32 (Granlund and
-// Montgomery, PLDI 1994): with s = ceil(log2 d) and m = ceil(2^(32+s) / d),
-// floor(n / d) = (n * m) >> (32 + s).  m < 2^33 is kept in 64 bits.
-struct DivU32 {
-    uint64_t m;
-    int sh;
-};
-static DivU32 divu32_for(uint32_t d) {
-    int s = 0;
-    while ((uint64_t(1) << s) < d) s++;
-    const unsigned __int128 num = (unsigned __int128)1 << (32 + s);
-    return {(uint64_t)((num + d - 1) / d), 32 + s};
-}
-BSQ_DEV uint32_t divu32(uint32_t n, const DivU32 &dv) {
-    return (uint32_t)(((unsigned __int128)n * dv.m) >> dv.sh);
-}
-
 template <bool SR>
 __global__ void __launch_bounds__(256) quant_mxfp8_row_flat_kernel(
     const uint16_t *__restrict__ x, int64_t nchunk, int64_t K, DivU32 div_k8, const __grid_constant__ PhiloxKeys keys,
@@ -1449,6 +1771,77 @@ int launch_quant_nvfp4_fused(const uint16_t *x, int64_t M, int64_t K, bool rht, 
     // one resident wave, no more CTAs than 256-block groups of work
     const int grid = grid_for(M * KB, 256, resident);
     return cudaLaunchCooperativeKernel(kern, dim3(grid), dim3(256), args, 0, s) == cudaSuccess ? 0 : 1;
+}
+
+// Streaming NVFP4 kernels: CTAs that fit at once (dynamic shared memory
+// included), per kernel and device.
+template <auto Kern>
+static int resident_stream(int num_sms) {
+    constexpr int kDevs = 64;
+    static std::atomic<int> per_sm[kDevs];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kDevs) dev = 0;
+    int n = per_sm[dev].load(std::memory_order_relaxed);
+    if (n == 0) {
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, Kern, nvs::kThreads, nvs::kSmemBytes) != cudaSuccess ||
+            n < 1)
+            n = 1;
+        per_sm[dev].store(n, std::memory_order_relaxed);
+    }
+    return n * num_sms;
+}
+
+template <int MODE, bool RHT, bool TWO_D>
+static int launch_stream_t(const uint16_t *x, int64_t M, int64_t K, uint32_t mask, unsigned int *counter,
+                           unsigned int *amax_bits, const float *scale_src, int src_is_amax, float *gs_out,
+                           uint8_t *codes, uint8_t *sf, unsigned int *err, int num_sms, cudaStream_t s) {
+    auto kern = quant_nvfp4_stream_kernel<MODE, RHT, TWO_D>;
+    if (smem_attr_once(reinterpret_cast<const void *>(kern), nvs::kSmemBytes) != BSQ_OK) return 1;
+    const int64_t KB = K >> 4;
+    const int64_t chunks = TWO_D ? (M >> 4) * ((K + 511) >> 9) : (M * KB + 511) >> 9;
+    const int grid = grid_for(chunks, 1, resident_stream<quant_nvfp4_stream_kernel<MODE, RHT, TWO_D>>(num_sms));
+    DivU32 div_kb = divu32_for((uint32_t)KB);
+    if (MODE == nvs::FUSED) {
+        void *args[] = {(void *)&x,        (void *)&M,         (void *)&K,         (void *)&div_kb,
+                        (void *)&mask,     (void *)&counter,   (void *)&amax_bits, (void *)&scale_src,
+                        (void *)&src_is_amax, (void *)&gs_out, (void *)&codes,     (void *)&sf,
+                        (void *)&err};
+        return cudaLaunchCooperativeKernel(reinterpret_cast<const void *>(kern), dim3(grid), dim3(nvs::kThreads), args,
+                                           nvs::kSmemBytes, s) == cudaSuccess
+                   ? 0
+                   : 1;
+    }
+    kern<<<grid, nvs::kThreads, nvs::kSmemBytes, s>>>(x, M, K, div_kb, mask, counter, amax_bits, scale_src,
+                                                      src_is_amax, gs_out, codes, sf, err);
+    return cudaGetLastError() == cudaSuccess ? 0 : 1;
+}
+
+bool stream_ok(int64_t M, int64_t K, bool block_2d) {
+    return K % 64 == 0 && M * (K >> 4) < (int64_t(1) << 32) && (!block_2d || M % 16 == 0);
+}
+
+int launch_nvfp4_stream(int mode, const uint16_t *x, int64_t M, int64_t K, bool block_2d, bool rht, uint32_t mask,
+                        unsigned int *counter, unsigned int *amax_bits, const float *scale_src, bool src_is_amax,
+                        float *gs_out, uint8_t *codes, uint8_t *sf, unsigned int *err, int num_sms, cudaStream_t s) {
+    const int sa = src_is_amax ? 1 : 0;
+#define BSQ_NVS(MO, R, D)                                                                                        \
+    return launch_stream_t<MO, R, D>(x, M, K, mask, counter, amax_bits, scale_src, sa, gs_out, codes, sf, err, \
+                                     num_sms, s)
+#define BSQ_NVS_RD(MO)                                  \
+    do {                                                \
+        if (rht) {                                      \
+            if (block_2d) BSQ_NVS(MO, true, true);      \
+            else BSQ_NVS(MO, true, false);              \
+        } else {                                        \
+            if (block_2d) BSQ_NVS(MO, false, true);     \
+            else BSQ_NVS(MO, false, false);             \
+        }                                               \
+    } while (0)
+    if (mode == nvs::AMAX) BSQ_NVS_RD(nvs::AMAX);
+    if (mode == nvs::QUANT) BSQ_NVS_RD(nvs::QUANT);
+    BSQ_NVS_RD(nvs::FUSED);
+#undef BSQ_NVS_RD
+#undef BSQ_NVS
 }
 
 void launch_quant_mxfp8(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, bool colwise, bool sr,

@@ -28,6 +28,16 @@ void launch_quant_nvfp4(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, bo
 // non-zero if the launch failed.
 int launch_quant_nvfp4_fused(const uint16_t *x, int64_t M, int64_t K, bool rht, uint32_t mask, float *gs_out,
                              uint8_t *codes, uint8_t *sf, unsigned int *err, int num_sms, cudaStream_t s);
+// Streaming NVFP4 kernels for contiguous tensors (stream_ok): mode 0 = amax
+// only (into *amax_bits, zeroed by the caller; with a counter, also zeroed,
+// the last CTA writes s_g to *gs_out), 1 = quantize with s_g from *scale_src
+// (an amax when src_is_amax), 2 = amax and quantize in one cooperative
+// launch (counter and amax bits in the first 8 bytes of codes, zeroed).
+// Returns non-zero if the launch failed.
+bool stream_ok(int64_t M, int64_t K, bool block_2d);
+int launch_nvfp4_stream(int mode, const uint16_t *x, int64_t M, int64_t K, bool block_2d, bool rht, uint32_t mask,
+                        unsigned int *counter, unsigned int *amax_bits, const float *scale_src, bool src_is_amax,
+                        float *gs_out, uint8_t *codes, uint8_t *sf, unsigned int *err, int num_sms, cudaStream_t s);
 void launch_quant_mxfp8(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, bool colwise, bool sr,
                         uint64_t seed, uint32_t stream_id, uint8_t *codes, uint8_t *sf, int num_sms,
                         cudaStream_t s);

@@ -49,3 +49,29 @@ def assert_gemm_close(got, C_ref, ref_abs, out_bf16, what):
     bad = np.argwhere(~(err <= tol))
     assert bad.size == 0, f"{what}: {len(bad)} of {err.size} outside tolerance; first {bad[:5].tolist()}, " \
                           f"got {got[tuple(bad[0])]} want {C_ref[tuple(bad[0])]} tol {tol[tuple(bad[0])]}"
+
+
+def assert_gemm_full(ora, Cg, dequant_a_rows, B64, out_bf16, what, chunk=2048):
+    """Every element of the device output Cg [M, N] against the oracle's
+    binary64 GEMM (BLAS form): rows r0..r1 of A decoded by
+    dequant_a_rows(r0, r1), B decoded once (B64 [N, K])."""
+    M = Cg.shape[0]
+    for r0 in range(0, M, chunk):
+        r1 = min(M, r0 + chunk)
+        Cr, Ra = ora.gemm_f64_blas(dequant_a_rows(r0, r1), B64)
+        got = Cg[r0:r1].float().cpu().numpy().astype(np.float64)
+        assert_gemm_close(got, Cr, Ra, out_bf16, f"{what} rows {r0}..{r1}")
+
+
+def assert_quant_full(ora, codes_dev, sf_dev, want, sf_rows, nblk, what, sf_row_of=None, gs_dev=None):
+    """Codes (every byte), canonical scale factors (every row) and, for
+    NVFP4, the global scale of a device quantization against the oracle's
+    want = (codes, sf[, s_g]).  sf_row_of maps output rows to SF rows
+    (expert groups); None means the identity."""
+    assert_codes_equal(host_u8(codes_dev), want[0], f"{what} codes")
+    can = sf_canonical(ora, sf_dev, sf_rows, nblk)
+    if sf_row_of is not None:
+        can = can[sf_row_of]
+    assert_codes_equal(can, want[1], f"{what} scales")
+    if gs_dev is not None:
+        assert np.float32(gs_dev.item()) == np.float32(want[2]), f"{what} s_g {gs_dev.item()} vs {want[2]}"

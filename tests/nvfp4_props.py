@@ -125,3 +125,14 @@ def check_nvfp4(y, codes, sf, s_g, block_2d=False, four_over_six=False, amax=Non
             assert bad.size == 0, f"{what}: Four Over Six kept the higher-error scale at {bad[:5].tolist()}"
             picked4 += int((clear & (e4 < e6)).sum())
     return picked4
+
+
+def decode_nvfp4(codes, sf, s_g):
+    """Binary64 values of an NVFP4 tensor (codes [R, K/2], canonical sf
+    [R, K/16], s_g): element x block scale x global scale, from the pages'
+    E2M1 list and torch's E4M3 decode (exact)."""
+    mags = e2m1_magnitudes()
+    c = unpack_codes(codes)
+    v = np.where(c & 8, -1.0, 1.0) * mags[c & 7]
+    sc = np.repeat(e4m3_value(sf).astype(np.float64), 16, axis=1)
+    return v * sc * np.float64(np.float32(s_g))

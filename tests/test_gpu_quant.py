@@ -85,6 +85,29 @@ def test_nvfp4_two_pass_path(ora, knobs, block_2d):
         _nvfp4_check(ora, x, block_2d=block_2d, rht=0x1234, what=f"two-pass rht {M}x{K}")
 
 
+@pytest.mark.parametrize("M,K", [(16, 64), (48, 576), (1040, 1088), (512, 4096)])
+@pytest.mark.parametrize("block_2d", [False, True])
+@pytest.mark.parametrize("stream,fused", [(1, 1), (1, 0), (0, 1), (0, 0)])
+def test_nvfp4_contiguous_kernel_paths(ora, knobs, stream, fused, block_2d, M, K):
+    """Contiguous tensors through each kernel family: the bulk-copy streaming
+    kernels (fused amax + quantize in one cooperative launch, or an amax
+    launch and a quantize launch) and the register-streaming ones; shapes with
+    a partial last chunk, a partial last 512-column span and more chunks than
+    CTAs; with and without the RHT and with a given amax."""
+    knobs(bsq.BSQ_KNOB_STREAM_QUANT, stream)
+    knobs(bsq.BSQ_KNOB_FUSED_QUANT, fused)
+    x = edge_tensor(M, K, seed=M + K + block_2d)
+    tag = f"stream={stream} fused={fused} 2d={block_2d} {M}x{K}"
+    _nvfp4_check(ora, x, block_2d=block_2d, what=tag)
+    _nvfp4_check(ora, x, block_2d=block_2d, rht=0x1234, what=tag + " rht")
+    _nvfp4_check(ora, x, block_2d=block_2d, rht=0x0F0F, amax_in=float(x.float().abs().max()) * 1.5,
+                 what=tag + " given amax")
+    xd = dev(x)
+    for rht in (None, 0xBEEF):
+        a = api.amax(xd, rht_mask=rht)
+        assert np.float32(a.item()) == np.float32(ora.amax(bits(x), rht_mask=rht)), tag
+
+
 def test_nvfp4_small_linear_workload(ora):
     A, Wt = W.nvfp4_linear_small()
     _nvfp4_check(ora, A, what="A 1x16")

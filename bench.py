@@ -129,10 +129,13 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------- oracle
-def cpu_oracle_step(rows_a=1024, rows_w=2048):
+def cpu_oracle_step(rows_a=1024, rows_w=2048, threads=1):
     """The oracle on a bounded sample of the workload: the first rows_a rows of
     A and rows_w rows of W quantized (amax + RHT + NVFP4), then their GEMM in
-    binary64.  Returns (seconds, flops of the sample)."""
+    binary64.  threads == 1: the serial C oracle throughout (its scalar
+    binary64 GEMM loop); threads > 1: the oracle's row bands on that many
+    threads and its BLAS binary64 GEMM.  Returns (seconds, flops of the
+    sample)."""
     import numpy as np
     from fp8_math_b200 import workloads as W
     from oracle import oracle as ora
@@ -140,12 +143,35 @@ def cpu_oracle_step(rows_a=1024, rows_w=2048):
     mask = ora.rht_sign_mask(seed)
     xa, xw = W.bf16_bits(A), W.bf16_bits(Wt)
     t0 = time.perf_counter()
-    qa = ora.quant_nvfp4(xa, rht_mask=mask)
-    qw = ora.quant_nvfp4(xw, block_2d=True, rht_mask=mask)
-    ora.gemm_f64(ora.dequant(0, *qa), ora.dequant(0, *qw))
+    qa = ora.quant_nvfp4(xa, rht_mask=mask, threads=threads)
+    qw = ora.quant_nvfp4(xw, block_2d=True, rht_mask=mask, threads=threads)
+    da, dw = ora.dequant(0, *qa, threads=threads), ora.dequant(0, *qw, threads=threads)
+    if threads > 1:
+        ora.gemm_f64_blas(da, dw)
+    else:
+        ora.gemm_f64(da, dw)
     dt = time.perf_counter() - t0
     del np
     return dt, 2.0 * rows_a * rows_w * K
+
+
+def cpu_baseline_line():
+    """The oracle timed twice on the host: single-threaded on a 1024x2048
+    slice, and on every core this process may use on the whole of A and 4096
+    rows of W."""
+    from oracle import oracle as ora
+    ora.build()
+    cores = ora.ncores()
+    dt1, fl1 = cpu_oracle_step(1024, 2048, threads=1)
+    dtn, fln = cpu_oracle_step(M, 4096, threads=cores)
+    return {"value": fln / dtn / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "sample": f"amax+RHT+NVFP4 quantize of all {M} rows of A and the first 4096 rows of W (K={K}), then "
+                      f"their {M}x4096x{K} binary64 GEMM; the oracle's row bands on {cores} threads and its BLAS "
+                      "GEMM",
+            "seconds": dtn,
+            "single_core": {"value": fl1 / dt1 / 1e12, "unit": "TFLOP/s", "cores": 1, "seconds": dt1,
+                            "sample": "the first 1024 rows of A and 2048 rows of W, then their 1024x2048x4096 "
+                                      "binary64 GEMM; the serial C oracle (scalar GEMM loop)"}}
 
 
 def reference_arm(args, rank):
@@ -154,11 +180,13 @@ def reference_arm(args, rank):
     sys.path.insert(0, ROOT)
     from oracle import oracle as ora
     ora.build()
+    cores = ora.ncores()
+    rows_a, rows_w = 1024, 1024
     for _ in range(args.warmup):
-        cpu_oracle_step(rows_a=32, rows_w=64)
+        cpu_oracle_step(rows_a=rows_a, rows_w=rows_w, threads=cores)
     times, flops = [], 0.0
     for _ in range(args.steps):
-        dt, fl = cpu_oracle_step(rows_a=32, rows_w=64)
+        dt, fl = cpu_oracle_step(rows_a=rows_a, rows_w=rows_w, threads=cores)
         times.append(dt)
         flops = fl
     tot = sum(times)
@@ -168,9 +196,10 @@ def reference_arm(args, rank):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": WORKLOAD, "M": M, "N": N, "K": K},
-        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
-                         "sample": "per step: amax+RHT+NVFP4 quantize of 32 rows of A and 64 rows of W (K=4096), "
-                                   "then their 32x64x4096 binary64 GEMM; single-threaded C oracle"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": f"per step: amax+RHT+NVFP4 quantize of {rows_a} rows of A and {rows_w} rows of W "
+                                   f"(K=4096), then their {rows_a}x{rows_w}x4096 binary64 GEMM; the oracle's row "
+                                   f"bands on {cores} threads and its BLAS GEMM"},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -572,13 +601,7 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        from oracle import oracle as ora
-        ora.build()
-        dt, fl = cpu_oracle_step()
-        cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
-               "sample": "amax+RHT+NVFP4 quantize of the first 1024 rows of A and 2048 rows of W (K=4096), then "
-                         "their 1024x2048x4096 binary64 GEMM; single-threaded C oracle",
-               "seconds": dt}
+        cpu = cpu_baseline_line()
 
     if rank == 0:
         line = {

@@ -63,6 +63,35 @@ def quant_mxfp8(x, colwise=False, sr=False, seed=0, stream_id=0, out=None):
     return codes, sf
 
 
+def quant_mxfp8_rowcol(x, sr=False, seed=0, stream_id_row=0, stream_id_col=1, out=None):
+    """Row-wise and column-wise MXFP8 in one pass.  Returns
+    (codes_row [M,K], sf_row, codes_col [K,M], sf_col)."""
+    M, K = x.shape
+    if out is None:
+        cr = torch.empty(M, K, dtype=torch.uint8, device=x.device)
+        sr_ = torch.zeros(sf_bytes(M, K // 32), dtype=torch.uint8, device=x.device)
+        cc = torch.empty(K, M, dtype=torch.uint8, device=x.device)
+        sc = torch.zeros(sf_bytes(K, M // 32), dtype=torch.uint8, device=x.device)
+    else:
+        cr, sr_, cc, sc = out
+    bsq.bsq_quant_mxfp8_rowcol(x, M, K, _ld(x), bsq.BSQ_SR if sr else bsq.BSQ_RNE, seed, stream_id_row,
+                               stream_id_col, cr, sr_, cc, sc)
+    return cr, sr_, cc, sc
+
+
+def requant_nvfp4_mxfp8(codes, sf, gs, sr=True, seed=0, stream_id=1, out=None):
+    """NVFP4 [R, C] (codes [R, C/2], swizzled sf, gs [1]) -> column-wise MXFP8.
+    Returns (codes [C, R], sf swizzled)."""
+    R, C = codes.shape[0], codes.shape[1] * 2
+    if out is None:
+        cc = torch.empty(C, R, dtype=torch.uint8, device=codes.device)
+        sc = torch.zeros(sf_bytes(C, R // 32), dtype=torch.uint8, device=codes.device)
+    else:
+        cc, sc = out
+    bsq.bsq_requant_nvfp4_mxfp8(codes, sf, gs, R, C, bsq.BSQ_SR if sr else bsq.BSQ_RNE, seed, stream_id, cc, sc)
+    return cc, sc
+
+
 def quant_nvfp4_sr(x, block_2d=False, rht_mask=None, row_index=None, amax_in=None, seed=0, stream_id=0, out=None):
     """NVFP4 with stochastic rounding of the elements.  Returns (codes
     [R, K/2] uint8, sf swizzled uint8, global_scale [1] fp32)."""

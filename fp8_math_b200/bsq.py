@@ -41,6 +41,10 @@ _SIGS = {
     "bsq_quant_nvfp4_sr": (C.c_int, [_vp, _i64, _i64, _i64, C.c_int, C.c_int, C.c_uint16, _vp, _vp, _vp,
                                      C.c_uint64, C.c_uint32, _vp, _vp, _vp]),
     "bsq_quant_mxfp4": (C.c_int, [_vp, _i64, _i64, _i64, C.c_int, C.c_uint64, C.c_uint32, _vp, _vp, _vp]),
+    "bsq_quant_mxfp8_rowcol": (C.c_int, [_vp, _i64, _i64, _i64, C.c_int, C.c_uint64, C.c_uint32, C.c_uint32,
+                                         _vp, _vp, _vp, _vp, _vp]),
+    "bsq_requant_nvfp4_mxfp8": (C.c_int, [_vp, _vp, _vp, _i64, _i64, C.c_int, C.c_uint64, C.c_uint32, _vp, _vp,
+                                          _vp]),
     "bsq_rht": (C.c_int, [_vp, _vp, _i64, _i64, _i64, _i64, C.c_uint16, _vp]),
     "bsq_requant_transpose": (C.c_int, [_vp, _vp, _i64, _i64, C.c_int, C.c_uint64, C.c_uint32, _vp, _vp, _vp]),
     "bsq_gemm_blockscaled": (C.c_int, [C.c_int, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _i64,
@@ -176,3 +180,15 @@ def bsq_debug_timeout_probe(timeout_ns, stream=None):
 
 def bsq_debug_kernel_choice(knob, value):
     return _check("bsq_debug_kernel_choice", lib().bsq_debug_kernel_choice(knob, value))
+
+
+def bsq_quant_mxfp8_rowcol(x, M, K, ldx, rounding, seed, stream_id_row, stream_id_col, codes_row, sf_row, codes_col,
+                           sf_col, stream=None):
+    return _check("bsq_quant_mxfp8_rowcol", lib().bsq_quant_mxfp8_rowcol(
+        _p(x), M, K, ldx, rounding, seed, stream_id_row, stream_id_col, _p(codes_row), _p(sf_row), _p(codes_col),
+        _p(sf_col), _stream(stream)))
+
+
+def bsq_requant_nvfp4_mxfp8(codes, sf, gs, R, C, rounding, seed, stream_id, codes_col, sf_col, stream=None):
+    return _check("bsq_requant_nvfp4_mxfp8", lib().bsq_requant_nvfp4_mxfp8(
+        _p(codes), _p(sf), _p(gs), R, C, rounding, seed, stream_id, _p(codes_col), _p(sf_col), _stream(stream)))

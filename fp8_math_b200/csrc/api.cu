@@ -273,6 +273,43 @@ int bsq_quant_mxfp8(const void *x, int64_t M, int64_t K, int64_t ldx, int colwis
     return launch_status();
 }
 
+int bsq_quant_mxfp8_rowcol(const void *x, int64_t M, int64_t K, int64_t ldx, int rounding, uint64_t seed,
+                           uint32_t stream_id_row, uint32_t stream_id_col, uint8_t *codes_row, uint8_t *sf_row,
+                           uint8_t *codes_col, uint8_t *sf_col, void *stream) {
+    if (!x || !codes_row || !sf_row || !codes_col || !sf_col || M < 0 || K < 0 || ldx < K || M % 32 || K % 32 ||
+        (rounding != BSQ_RNE && rounding != BSQ_SR))
+        return BSQ_ERR_INVALID;
+    if (!aligned16(x) || !aligned16(codes_row) || !aligned16(sf_row) || !aligned16(codes_col) || !aligned16(sf_col) ||
+        ldx % 8)
+        return BSQ_ERR_ALIGN;
+    if ((M >> 5) * ((K + 63) >> 6) >= (int64_t(1) << 31)) return BSQ_ERR_UNSUPPORTED;
+    DeviceState *d;
+    if (int st = device_state(&d)) return st;
+    if (M == 0 || K == 0) return BSQ_OK;
+    bsq::launch_quant_mxfp8_rowcol(static_cast<const uint16_t *>(x), M, K, ldx, rounding == BSQ_SR, seed,
+                                   stream_id_row, stream_id_col, codes_row, sf_row, codes_col, sf_col, d->num_sms,
+                                   static_cast<cudaStream_t>(stream));
+    return launch_status();
+}
+
+int bsq_requant_nvfp4_mxfp8(const uint8_t *codes, const uint8_t *sf, const float *gs_dev, int64_t R, int64_t C,
+                            int rounding, uint64_t seed, uint32_t stream_id, uint8_t *codes_col, uint8_t *sf_col,
+                            void *stream) {
+    if (!codes || !sf || !gs_dev || !codes_col || !sf_col || R < 0 || C < 0 || R % 32 || C % 16 ||
+        (rounding != BSQ_RNE && rounding != BSQ_SR))
+        return BSQ_ERR_INVALID;
+    if (!aligned16(codes) || !aligned16(sf) || !aligned16(codes_col) || !aligned16(sf_col) ||
+        (reinterpret_cast<uintptr_t>(gs_dev) & 3u))
+        return BSQ_ERR_ALIGN;
+    if ((R >> 5) * ((C + 63) >> 6) >= (int64_t(1) << 31)) return BSQ_ERR_UNSUPPORTED;
+    DeviceState *d;
+    if (int st = device_state(&d)) return st;
+    if (R == 0 || C == 0) return BSQ_OK;
+    bsq::launch_requant_nvfp4_mxfp8(codes, sf, gs_dev, R, C, rounding == BSQ_SR, seed, stream_id, codes_col, sf_col,
+                                    d->num_sms, static_cast<cudaStream_t>(stream));
+    return launch_status();
+}
+
 int bsq_quant_mxfp4(const void *x, int64_t M, int64_t K, int64_t ldx, int rounding, uint64_t seed,
                     uint32_t stream_id, uint8_t *codes, uint8_t *sf, void *stream) {
     if (!x || !codes || !sf || M < 0 || K < 0 || ldx < K || K % 32 || (rounding != BSQ_RNE && rounding != BSQ_SR))

@@ -1390,6 +1390,156 @@ __global__ void __launch_bounds__(256) quant_mxfp8_col_kernel(
     }
 }
 
+// Row-wise and column-wise MXFP8 of one bf16 tensor in one pass (the
+// backward pass needs dY both ways): the column kernel's warp tile (32 rows
+// x 64 columns, lane l = 4 kg + mg holding rows 8 mg .. 8 mg + 7 and columns
+// 8 kg .. 8 kg + 7) also yields, per held row, one row-wise chunk of 8; the
+// four lanes mg, mg + 4, mg + 8, mg + 12 (and likewise the upper four kg)
+// hold one row block of 32, reduced with shuffles over lane bits 2 and 3.
+// Row output: codes_r [M][K], SR draws of row * K + col with stream_r;
+// column output: codes_c [K][M], draws of k * M + m with stream_c.
+template <bool SR>
+__global__ void __launch_bounds__(256) quant_mxfp8_rowcol_kernel(
+    const uint16_t *__restrict__ x, int64_t M, int64_t K, int64_t ldx, uint32_t ntile, DivU32 div_mt,
+    const __grid_constant__ PhiloxKeys keys, uint32_t stream_r, uint32_t stream_c, uint8_t *__restrict__ codes_r,
+    uint8_t *__restrict__ sf_r, uint8_t *__restrict__ codes_c, uint8_t *__restrict__ sf_c) {
+    const int lane = threadIdx.x & 31, kg = lane >> 2, mg = lane & 3;
+    const uint32_t mt_n = (uint32_t)(M >> 5);
+    const int64_t MB = M >> 5, KB = K >> 5;
+    const uint32_t nwarps = (gridDim.x * blockDim.x) >> 5;
+    for (uint32_t t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < ntile; t += nwarps) {
+        const uint32_t kt = divu32(t, div_mt), mt = t - kt * mt_n;
+        const int64_t m0 = (int64_t)mt * 32 + mg * 8, k0 = (int64_t)kt * 64 + kg * 8;
+        const bool kvalid = k0 < K;  // K % 32 == 0: a row block of four lanes is all in or all out
+        uint32_t w[8][4];
+        const uint16_t *xp = x + m0 * ldx + k0;
+#pragma unroll
+        for (int i = 0; i < 8; i++) {
+            const uint4 r = kvalid ? __ldg(reinterpret_cast<const uint4 *>(xp + i * ldx)) : make_uint4(0, 0, 0, 0);
+            w[i][0] = r.x; w[i][1] = r.y; w[i][2] = r.z; w[i][3] = r.w;
+        }
+        // ---- row-wise: row m0 + i, columns k0 .. k0 + 7
+#pragma unroll
+        for (int i = 0; i < 8; i++) {
+            const int64_t row = m0 + i;
+            uint32_t sb;
+            uint2 q;
+            if (SR) {
+                uint32_t a[4];
+                uint32_t m = bf16_chunk_absmax(w[i], a);
+                m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 4));
+                m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 8));
+                sb = mx_scale_code_bf16(m);
+                q = mx_sr8_bf16(w[i], a, sb, mx_draws((uint64_t)(row * K + k0) >> 3, keys, stream_r));
+                if (m == 0u) q = make_uint2(0u, 0u);
+            } else {
+                float v[8];
+#pragma unroll
+                for (int p = 0; p < 4; p++) {
+                    v[2 * p] = bf16_lo(w[i][p]);
+                    v[2 * p + 1] = bf16_hi(w[i][p]);
+                }
+                float m = fmax3(fmax3(fabsf(v[0]), fabsf(v[1]), fabsf(v[2])),
+                                fmax3(fabsf(v[3]), fabsf(v[4]), fabsf(v[5])), fmaxf(fabsf(v[6]), fabsf(v[7])));
+                m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 4));
+                m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 8));
+                sb = mx_scale_code(m);
+                q = mx_encode8<false>(v, m == 0.0f, sb, 0, keys, 0u);
+            }
+            if (kvalid) {
+                *reinterpret_cast<uint2 *>(codes_r + row * K + k0) = q;
+                if ((kg & 3) == 0) sf_r[sf_offset(row, k0 >> 5, KB)] = (uint8_t)sb;
+            }
+        }
+        // ---- column-wise: column k0 + j, rows m0 .. m0 + 7
+#pragma unroll
+        for (int j = 0; j < 8; j++) {
+            const int64_t k = k0 + j;
+            uint32_t sb;
+            uint2 q;
+            if (SR) {
+                uint32_t p[4], a[4];
+#pragma unroll
+                for (int i = 0; i < 4; i++)
+                    p[i] = __byte_perm(w[2 * i][j >> 1], w[2 * i + 1][j >> 1], (j & 1) ? 0x7632u : 0x5410u);
+                uint32_t m = bf16_chunk_absmax(p, a);
+                m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+                m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+                sb = mx_scale_code_bf16(m);
+                q = mx_sr8_bf16(p, a, sb, mx_draws((uint64_t)(k * M + m0) >> 3, keys, stream_c));
+                if (m == 0u) q = make_uint2(0u, 0u);
+            } else {
+                float v[8];
+#pragma unroll
+                for (int i = 0; i < 8; i++) v[i] = (j & 1) ? bf16_hi(w[i][j >> 1]) : bf16_lo(w[i][j >> 1]);
+                float m = fmax3(fmax3(fabsf(v[0]), fabsf(v[1]), fabsf(v[2])),
+                                fmax3(fabsf(v[3]), fabsf(v[4]), fabsf(v[5])), fmaxf(fabsf(v[6]), fabsf(v[7])));
+                m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+                m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+                sb = mx_scale_code(m);
+                q = mx_encode8<false>(v, m == 0.0f, sb, 0, keys, 0u);
+            }
+            if (kvalid) {
+                *reinterpret_cast<uint2 *>(codes_c + k * M + m0) = q;
+                if (mg == 0) sf_c[sf_offset(k, m0 >> 5, MB)] = (uint8_t)sb;
+            }
+        }
+    }
+}
+
+// NVFP4 -> MXFP8 column-wise: the NVFP4 tensor [R][C] (codes [R][C/2],
+// swizzled E4M3 scales for R rows x C/16 blocks, s_g on the device) is
+// decoded to binary32 as RN(RN(E2M1 * s_b) * s_g) (the first product is
+// exact), transposed and quantized to MXFP8 with blocks of 32 along R.  The
+// column kernel's warp tile: lane l = 4 kg + mg holds rows 8 mg .. 8 mg + 7
+// and columns 8 kg .. 8 kg + 7 (one 32-bit code load and one scale byte per
+// row: the 8 columns sit in one 16-block); the four lanes of a kg share the
+// output block of column 8 kg + j.
+template <bool SR>
+__global__ void __launch_bounds__(256) requant_nvfp4_mxfp8_kernel(
+    const uint8_t *__restrict__ codes_in, const uint8_t *__restrict__ sf_in, const float *gs, int64_t R, int64_t C,
+    uint32_t ntile, DivU32 div_mt, const __grid_constant__ PhiloxKeys keys, uint32_t stream_id,
+    uint8_t *__restrict__ codes, uint8_t *__restrict__ sf) {
+    const int lane = threadIdx.x & 31, kg = lane >> 2, mg = lane & 3;
+    const uint32_t mt_n = (uint32_t)(R >> 5);
+    const int64_t RB = R >> 5, CB16 = C >> 4;
+    const float s_g = *gs;
+    const uint32_t nwarps = (gridDim.x * blockDim.x) >> 5;
+    for (uint32_t t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < ntile; t += nwarps) {
+        const uint32_t kt = divu32(t, div_mt), mt = t - kt * mt_n;
+        const int64_t m0 = (int64_t)mt * 32 + mg * 8, k0 = (int64_t)kt * 64 + kg * 8;
+        const bool kvalid = k0 < C;  // C % 16 == 0: a lane's 8 columns are all in or all out
+        float v[8][8];               // v[i][j]: row m0 + i, column k0 + j
+#pragma unroll
+        for (int i = 0; i < 8; i++) {
+            const uint32_t w = kvalid ? __ldg(reinterpret_cast<const uint32_t *>(codes_in + (m0 + i) * (C >> 1) + (k0 >> 1)))
+                                      : 0u;
+            const float sbv = kvalid ? e4m3_to_f32(__ldg(sf_in + sf_offset(m0 + i, k0 >> 4, CB16))) : 0.0f;
+            float e[8];
+            e2m1x8_to_f32(w, e);
+#pragma unroll
+            for (int j = 0; j < 8; j++) v[i][j] = __fmul_rn(__fmul_rn(e[j], sbv), s_g);
+        }
+#pragma unroll
+        for (int j = 0; j < 8; j++) {
+            const int64_t k = k0 + j;
+            float c[8];
+#pragma unroll
+            for (int i = 0; i < 8; i++) c[i] = v[i][j];
+            float m = fmax3(fmax3(fabsf(c[0]), fabsf(c[1]), fabsf(c[2])), fmax3(fabsf(c[3]), fabsf(c[4]), fabsf(c[5])),
+                            fmaxf(fabsf(c[6]), fabsf(c[7])));
+            m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+            m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+            const uint32_t sb = mx_scale_code(m);
+            const uint2 q = mx_encode8<SR>(c, m == 0.0f, sb, (uint64_t)(k * R + m0) >> 3, keys, stream_id);
+            if (kvalid) {
+                *reinterpret_cast<uint2 *>(codes + k * R + m0) = q;
+                if (mg == 0) sf[sf_offset(k, m0 >> 5, RB)] = (uint8_t)sb;
+            }
+        }
+    }
+}
+
 // ===================================================================== MXFP4
 // E2M1 elements in blocks of 32 along K with one E8M0 scale 2^E,
 // E = clamp(floor(log2 amax) - 2, -127, 127) (2 is the exponent of E2M1's
@@ -1907,6 +2057,40 @@ void launch_requant_transpose(const uint8_t *codes_row, const uint8_t *sf_row, i
         const int grid = grid_for(ntile, 8, resident_ctas<quant_mxfp8_col_kernel<true, false>>(num_sms));
         quant_mxfp8_col_kernel<true, false><<<grid, 256, 0, s>>>(codes_row, sf_row, M, K, K, ntile, dmt, keys,
                                                                  stream_id, codes_col, sf_col);
+    }
+}
+
+void launch_quant_mxfp8_rowcol(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, bool sr, uint64_t seed,
+                               uint32_t stream_r, uint32_t stream_c, uint8_t *codes_r, uint8_t *sf_r,
+                               uint8_t *codes_c, uint8_t *sf_c, int num_sms, cudaStream_t s) {
+    const PhiloxKeys keys = philox_keys((uint32_t)seed, (uint32_t)(seed >> 32));
+    const uint32_t ntile = (uint32_t)((M >> 5) * ((K + 63) >> 6));
+    const DivU32 dmt = divu32_for((uint32_t)(M >> 5));
+    if (sr) {
+        const int grid = grid_for(ntile, 8, resident_ctas<quant_mxfp8_rowcol_kernel<true>>(num_sms));
+        quant_mxfp8_rowcol_kernel<true><<<grid, 256, 0, s>>>(x, M, K, ldx, ntile, dmt, keys, stream_r, stream_c,
+                                                             codes_r, sf_r, codes_c, sf_c);
+    } else {
+        const int grid = grid_for(ntile, 8, resident_ctas<quant_mxfp8_rowcol_kernel<false>>(num_sms));
+        quant_mxfp8_rowcol_kernel<false><<<grid, 256, 0, s>>>(x, M, K, ldx, ntile, dmt, keys, stream_r, stream_c,
+                                                              codes_r, sf_r, codes_c, sf_c);
+    }
+}
+
+void launch_requant_nvfp4_mxfp8(const uint8_t *codes_in, const uint8_t *sf_in, const float *gs, int64_t R, int64_t C,
+                                bool sr, uint64_t seed, uint32_t stream_id, uint8_t *codes, uint8_t *sf, int num_sms,
+                                cudaStream_t s) {
+    const PhiloxKeys keys = philox_keys((uint32_t)seed, (uint32_t)(seed >> 32));
+    const uint32_t ntile = (uint32_t)((R >> 5) * ((C + 63) >> 6));
+    const DivU32 dmt = divu32_for((uint32_t)(R >> 5));
+    if (sr) {
+        const int grid = grid_for(ntile, 8, resident_ctas<requant_nvfp4_mxfp8_kernel<true>>(num_sms));
+        requant_nvfp4_mxfp8_kernel<true><<<grid, 256, 0, s>>>(codes_in, sf_in, gs, R, C, ntile, dmt, keys, stream_id,
+                                                              codes, sf);
+    } else {
+        const int grid = grid_for(ntile, 8, resident_ctas<requant_nvfp4_mxfp8_kernel<false>>(num_sms));
+        requant_nvfp4_mxfp8_kernel<false><<<grid, 256, 0, s>>>(codes_in, sf_in, gs, R, C, ntile, dmt, keys,
+                                                               stream_id, codes, sf);
     }
 }
 

@@ -41,6 +41,12 @@ int launch_nvfp4_stream(int mode, const uint16_t *x, int64_t M, int64_t K, bool 
 void launch_quant_mxfp8(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, bool colwise, bool sr,
                         uint64_t seed, uint32_t stream_id, uint8_t *codes, uint8_t *sf, int num_sms,
                         cudaStream_t s);
+void launch_quant_mxfp8_rowcol(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, bool sr, uint64_t seed,
+                               uint32_t stream_r, uint32_t stream_c, uint8_t *codes_r, uint8_t *sf_r,
+                               uint8_t *codes_c, uint8_t *sf_c, int num_sms, cudaStream_t s);
+void launch_requant_nvfp4_mxfp8(const uint8_t *codes_in, const uint8_t *sf_in, const float *gs, int64_t R, int64_t C,
+                                bool sr, uint64_t seed, uint32_t stream_id, uint8_t *codes, uint8_t *sf, int num_sms,
+                                cudaStream_t s);
 void launch_quant_mxfp4(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, bool sr, uint64_t seed,
                         uint32_t stream_id, uint8_t *codes, uint8_t *sf, int num_sms, cudaStream_t s);
 void launch_quant_nvfp4_sr(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, bool block_2d, bool rht,

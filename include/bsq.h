@@ -186,6 +186,35 @@ BSQ_API int bsq_quant_mxfp8(const void *x_bf16, int64_t M, int64_t K, int64_t ld
                     int rounding, uint64_t seed, uint32_t stream_id,
                     uint8_t *codes_dev, uint8_t *sf_dev, void *stream);
 
+/* Row-wise and column-wise MXFP8 of one bf16 matrix in a single pass
+ * ("Thinking Machines ...", section "A precision choice for each stage": the
+ * backward pass consumes gradients in MXFP8 with stochastic rounding, along
+ * both of dY's axes).  The outputs are exactly those of bsq_quant_mxfp8 with
+ * colwise = 0 (stream id stream_id_row) and colwise = 1 (stream id
+ * stream_id_col), same seed and rounding: codes_row [M][K] with sf_row for
+ * M rows x K/32 blocks, codes_col [K][M] with sf_col for K rows x M/32
+ * blocks; x is read once.  M % 32 == 0 and K % 32 == 0;
+ * (M / 32) * ceil(K / 64) >= 2^31 returns BSQ_ERR_UNSUPPORTED. */
+BSQ_API int bsq_quant_mxfp8_rowcol(const void *x_bf16, int64_t M, int64_t K, int64_t ldx, int rounding,
+                                   uint64_t seed, uint32_t stream_id_row, uint32_t stream_id_col,
+                                   uint8_t *codes_row_dev, uint8_t *sf_row_dev, uint8_t *codes_col_dev,
+                                   uint8_t *sf_col_dev, void *stream);
+
+/* NVFP4 -> MXFP8 column-wise requantize ("Thinking Machines ...", section
+ * "A precision choice for each stage": tensors saved in NVFP4 during the
+ * forward pass -- the weights in 16x16 blocks -- are dequantized, transposed
+ * at higher precision and requantized to MXFP8 for the backward pass).  The
+ * NVFP4 matrix [R][C] (codes [R][C/2], swizzled E4M3 scales for R rows x
+ * C/16 blocks as bsq_quant_nvfp4 writes them, *gs_dev its FP32 global scale)
+ * is decoded to fp32 as RN(RN(E2M1 * s_b) * s_g) (the first product is
+ * exact), transposed, and quantized as bsq_quant_mxfp8 does: blocks of 32
+ * along R, element idx = c * R + r for the stochastic draws.  Outputs
+ * codes_col [C][R], sf_col for C rows x R/32 blocks.  R % 32 == 0,
+ * C % 16 == 0; (R / 32) * ceil(C / 64) >= 2^31 returns BSQ_ERR_UNSUPPORTED. */
+BSQ_API int bsq_requant_nvfp4_mxfp8(const uint8_t *codes_dev, const uint8_t *sf_dev, const float *gs_dev,
+                                    int64_t R, int64_t C, int rounding, uint64_t seed, uint32_t stream_id,
+                                    uint8_t *codes_col_dev, uint8_t *sf_col_dev, void *stream);
+
 /* MXFP4 quantize ("08 -- FP4, MXFP4, NVFP4 ...", section "The two Blackwell
  * formats": E2M1 elements in groups of 32 with one E8M0 power-of-two scale,
  * 4.25 bits per value; "Microscaling ...", section "Microscaling").  Per

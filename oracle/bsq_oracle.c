@@ -696,6 +696,43 @@ int ora_requant_transpose(const uint8_t *codes_row, const uint8_t *sf_row, int64
 }
 
 /* ------------------------------------------------------------------------ */
+/* NVFP4 -> MXFP8 column-wise requantize -- [TML] "A precision choice for   */
+/* each stage": tensors saved in the forward pass (NVFP4, the weights in     */
+/* 16x16 blocks) are dequantized, transposed at higher precision and         */
+/* requantized to MXFP8 for the backward pass.  R30: the dequantized value   */
+/* is binary32 RN((E2M1(code) * E4M3(s_b)) * s_g) -- the first product is    */
+/* exact (at most six significant bits), the multiply by the FP32 tensor    */
+/* scale rounds once; the transpose's rows are then quantized to MXFP8 as   */
+/* in ora_quant_mxfp8 (blocks of 32 along the old rows, RNE or SR with the  */
+/* draw of output element c * R + r).  Input: codes [R][C/2], canonical sf  */
+/* [R][C/16], s_g; output rows c0 .. c1-1 of codes_out [C][R] and sf_out    */
+/* [C][R/32].                                                                 */
+/* ------------------------------------------------------------------------ */
+
+int ora_requant_nvfp4_mxfp8_rows(const uint8_t *codes, const uint8_t *sf, float s_g, int64_t R, int64_t C,
+                                 int sr, uint64_t seed, uint32_t stream_id, int64_t c0, int64_t c1,
+                                 uint8_t *codes_out, uint8_t *sf_out)
+{
+    if (R % 32 || C % 16 || c0 < 0 || c1 > C || c0 > c1)
+        return 1;
+    float v[32];
+    for (int64_t c = c0; c < c1; c++) {
+        for (int64_t rb = 0; rb < R / 32; rb++) {
+            for (int i = 0; i < 32; i++) {
+                int64_t r = rb * 32 + i;
+                uint8_t byte = codes[r * (C / 2) + c / 2];
+                uint8_t e2 = (c & 1) ? (uint8_t)(byte >> 4) : (uint8_t)(byte & 15);
+                float elem_scale = ora_e2m1_value(e2) * ora_e4m3_value(sf[r * (C / 16) + c / 16]);
+                v[i] = elem_scale * s_g;
+            }
+            sf_out[c * (R / 32) + rb] = mx_block(v, sr, seed, stream_id, (uint64_t)(c * R + rb * 32),
+                                                 codes_out + c * R + rb * 32);
+        }
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
 /* Scale-factor layout for the tensor-core MMA -- [MX] "Hardware and         */
 /* kernels": a block-scaled GEMM needs a particular scale-factor memory      */
 /* layout; the pages do not give it.  R23 (Blackwell block-scaled MMA        */

@@ -90,6 +90,8 @@ def lib():
                                                     C.c_uint32, _u8p, _u8p]),
                 "ora_requant_transpose_rows": (C.c_int, [_u8p, _u8p, _i64, _i64, C.c_int, C.c_uint64,
                                                          C.c_uint32, _i64, _i64, _u8p, _u8p]),
+                "ora_requant_nvfp4_mxfp8_rows": (C.c_int, [_u8p, _u8p, C.c_float, _i64, _i64, C.c_int, C.c_uint64,
+                                                           C.c_uint32, _i64, _i64, _u8p, _u8p]),
                 "ora_sf_swizzled_bytes": (_i64, [_i64, _i64]),
                 "ora_sf_offset": (_i64, [_i64, _i64, _i64]),
                 "ora_sf_swizzle": (None, [_u8p, _i64, _i64, _u8p]),
@@ -360,6 +362,26 @@ def requant_transpose(codes, sf, sr=True, seed=0, stream_id=1, threads=1):
             raise ValueError("unsupported requant shape")
 
     _run_bands(band, K, threads)
+    return cc, sc
+
+
+def requant_nvfp4_mxfp8(codes, sf, s_g, sr=True, seed=0, stream_id=1, threads=1):
+    """NVFP4 [R, C] (codes [R, C/2], canonical sf [R, C/16], s_g) ->
+    dequantize (binary32), transpose, MXFP8 (ora_requant_nvfp4_mxfp8_rows).
+    Returns (codes [C, R] u8, sf [C, R/32] u8)."""
+    codes = _c(codes, np.uint8)
+    sf = _c(sf, np.uint8)
+    R, C = codes.shape[0], codes.shape[1] * 2
+    cc = np.zeros((C, R), np.uint8)
+    sc = np.zeros((C, R // 32), np.uint8)
+    L = lib()
+
+    def band(c0, c1):
+        if L.ora_requant_nvfp4_mxfp8_rows(codes, sf, float(s_g), R, C, int(sr), int(seed), int(stream_id), c0, c1,
+                                          cc, sc):
+            raise ValueError("unsupported NVFP4 -> MXFP8 shape")
+
+    _run_bands(band, C, threads)
     return cc, sc
 
 

@@ -135,6 +135,31 @@ def test_mxfp8_backward_quantizers_full(ora, backward):
     assert_quant_full(ora, c, s, q["x_col"], K, M // 32, "X column-wise")
 
 
+def test_mxfp8_rowcol_full(ora, backward):
+    """dY 8192x14336 row- and column-wise in one pass (seed 4, streams 0 and
+    1): every byte equals the two separate quantizations' oracle."""
+    dY, _, _, _, q = backward
+    M, N = dY.shape
+    cr, sr_, cc, sc = api.quant_mxfp8_rowcol(dev(dY), sr=True, seed=4, stream_id_row=0, stream_id_col=1)
+    assert bsq.bsq_check() == bsq.BSQ_OK
+    assert_quant_full(ora, cr, sr_, q["dy_row"], M, N // 32, "dY row-wise (one pass)")
+    assert_quant_full(ora, cc, sc, q["dy_col"], N, M // 32, "dY column-wise (one pass)")
+
+
+def test_requant_saved_nvfp4_weight_full(ora, linear_rht, T):
+    """The RHT linear's W 14336x4096 saved in NVFP4 (16x16) -> MXFP8
+    column-wise [4096, 14336] with stochastic rounding: every byte."""
+    _, Wt, _, _, qw = linear_rht
+    N, K = Wt.shape
+    codes = dev(torch.from_numpy(qw[0]))
+    sf = dev(torch.from_numpy(ora.sf_swizzle(qw[1])))
+    gs = dev(torch.tensor([qw[2]], dtype=torch.float32))
+    cc, sc = api.requant_nvfp4_mxfp8(codes, sf, gs, sr=True, seed=4, stream_id=2)
+    assert bsq.bsq_check() == bsq.BSQ_OK
+    want = ora.requant_nvfp4_mxfp8(*qw, sr=True, seed=4, stream_id=2, threads=T)
+    assert_quant_full(ora, cc, sc, want, K, N // 32, "W NVFP4 -> MXFP8 column-wise")
+
+
 def test_mxfp8_dgrad_full(ora, backward, T):
     """dX = dY . W: A = dY row-wise [8192, 14336], B = W column-wise
     [4096, 14336], bf16 output: every element."""

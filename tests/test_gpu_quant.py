@@ -367,6 +367,40 @@ def test_mxfp8_requant_workload_full_size(ora):
 
 
 # ------------------------------------------------------------------ errors
+@pytest.mark.parametrize("sr", [False, True])
+@pytest.mark.parametrize("M,K", [(32, 32), (64, 96), (256, 512), (96, 4096)])
+def test_mxfp8_rowcol_parity(ora, M, K, sr):
+    """One pass, both orientations: byte-identical to the row-wise (stream 3)
+    and column-wise (stream 5) quantizations."""
+    x = W.mxfp8_requant(M=M, K=K, seed=M + K)
+    x[0, :32] = 0.0
+    cr, sr_, cc, sc = api.quant_mxfp8_rowcol(dev(x), sr=sr, seed=9, stream_id_row=3, stream_id_col=5)
+    assert bsq.bsq_check() == 0
+    wr = ora.quant_mxfp8(bits(x), sr=sr, seed=9, stream_id=3)
+    wc = ora.quant_mxfp8(bits(x), colwise=True, sr=sr, seed=9, stream_id=5)
+    assert_codes_equal(host_u8(cr), wr[0], "rowcol: row codes")
+    assert_codes_equal(sf_canonical(ora, sr_, M, K // 32), wr[1], "rowcol: row sf")
+    assert_codes_equal(host_u8(cc), wc[0], "rowcol: col codes")
+    assert_codes_equal(sf_canonical(ora, sc, K, M // 32), wc[1], "rowcol: col sf")
+
+
+@pytest.mark.parametrize("sr", [False, True])
+@pytest.mark.parametrize("R,C,two_d", [(32, 16, True), (64, 96, True), (256, 512, True), (96, 4096, False)])
+def test_requant_nvfp4_mxfp8_parity(ora, R, C, two_d, sr):
+    """Saved NVFP4 -> dequantize -> transpose -> MXFP8: the oracle's NVFP4
+    tensor uploaded, byte-identical output."""
+    x = W.nvfp4_linear_rht(M=R, N=16, K=C, seed=R + C)[0]
+    q = ora.quant_nvfp4(bits(x), block_2d=two_d)
+    codes = dev(torch.from_numpy(q[0]))
+    sf = dev(torch.from_numpy(ora.sf_swizzle(q[1])))
+    gs = dev(torch.tensor([q[2]], dtype=torch.float32))
+    cc, sc = api.requant_nvfp4_mxfp8(codes, sf, gs, sr=sr, seed=11, stream_id=2)
+    assert bsq.bsq_check() == 0
+    want = ora.requant_nvfp4_mxfp8(*q, sr=sr, seed=11, stream_id=2)
+    assert_codes_equal(host_u8(cc), want[0], "nvfp4->mxfp8 codes")
+    assert_codes_equal(sf_canonical(ora, sc, C, R // 32), want[1], "nvfp4->mxfp8 sf")
+
+
 def test_invalid_arguments_launch_nothing():
     x = torch.zeros(16, 24, dtype=torch.bfloat16, device="cuda")
     codes = torch.empty(16, 12, dtype=torch.uint8, device="cuda")

@@ -129,3 +129,17 @@ def test_noalloc_rejects_requests_beyond_its_scratch(lib):
     import torch
     if not torch.cuda.is_available():
         assert L.bsq_global_scale_noalloc(16, fits, K, K, 0, 0, 64, None) == lib.BSQ_ERR_CUDA
+
+
+def test_validation_of_the_backward_input_entry_points(lib):
+    L = lib.lib()
+    # one-pass row + column MXFP8: M % 32, K % 32, rounding, alignment
+    assert L.bsq_quant_mxfp8_rowcol(16, 48, 64, 64, 0, 0, 0, 1, 64, 64, 64, 64, None) == lib.BSQ_ERR_INVALID
+    assert L.bsq_quant_mxfp8_rowcol(16, 64, 48, 48, 0, 0, 0, 1, 64, 64, 64, 64, None) == lib.BSQ_ERR_INVALID
+    assert L.bsq_quant_mxfp8_rowcol(16, 64, 64, 64, 2, 0, 0, 1, 64, 64, 64, 64, None) == lib.BSQ_ERR_INVALID
+    assert L.bsq_quant_mxfp8_rowcol(16, 64, 64, 64, 0, 0, 0, 1, 64, 64, 72, 64, None) == lib.BSQ_ERR_ALIGN
+    # NVFP4 -> MXFP8: R % 32, C % 16, the global scale pointer
+    assert L.bsq_requant_nvfp4_mxfp8(16, 16, 64, 48, 64, 1, 0, 0, 64, 64, None) == lib.BSQ_ERR_INVALID
+    assert L.bsq_requant_nvfp4_mxfp8(16, 16, 64, 64, 40, 1, 0, 0, 64, 64, None) == lib.BSQ_ERR_INVALID
+    assert L.bsq_requant_nvfp4_mxfp8(16, 16, None, 64, 64, 1, 0, 0, 64, 64, None) == lib.BSQ_ERR_INVALID
+    assert L.bsq_requant_nvfp4_mxfp8(16, 16, 66, 64, 64, 1, 0, 0, 64, 64, None) == lib.BSQ_ERR_ALIGN

@@ -927,3 +927,64 @@ def test_blas_gemm_equals_the_plain_sum(ora):
     C2, R2 = ora.gemm_f64_blas(A, B)
     assert np.allclose(C1, C2, rtol=0, atol=1e-12 * R1.max())
     assert np.allclose(R1, R2, rtol=1e-5, atol=0)
+
+
+# --------------------------------------------------------------------- NVFP4 -> MXFP8 requantize
+def _nvfp4_with_power_of_two_scale(ora, R, C, seed):
+    """An NVFP4 quantization (16x16, the saved-weight form) whose global scale
+    is a power of two (amax = 2688 / 8), so every decoded value, at most six
+    significant bits, is exact in bf16."""
+    g = torch.Generator().manual_seed(seed)
+    w = torch.randn(R, C, generator=g) * 4.0
+    w[0, 0] = 2688.0 / 8
+    x = W.bf16_bits(w.to(torch.bfloat16))
+    q = ora.quant_nvfp4(x, block_2d=True)
+    assert q[2] == 0.125
+    return q
+
+
+@pytest.mark.parametrize("sr", [False, True])
+def test_requant_nvfp4_mxfp8_is_the_mxfp8_quantization_of_the_decode(ora, sr):
+    """TML page "A precision choice for each stage": saved NVFP4 tensors are
+    dequantized, transposed and requantized to MXFP8.  When the decoded values
+    are exact in bf16, the result is byte for byte the (pinned) column-wise
+    MXFP8 quantization of the decoded tensor, with the same draws."""
+    q = _nvfp4_with_power_of_two_scale(ora, 64, 96, 4)
+    deq = ora.dequant(ora.NVFP4, *q)
+    xb = torch.from_numpy(deq.astype(np.float32)).to(torch.bfloat16)
+    assert np.array_equal(xb.float().numpy().astype(np.float64), deq)
+    want = ora.quant_mxfp8(W.bf16_bits(xb), colwise=True, sr=sr, seed=7, stream_id=2)
+    got = ora.requant_nvfp4_mxfp8(*q, sr=sr, seed=7, stream_id=2)
+    assert np.array_equal(got[0], want[0]) and np.array_equal(got[1], want[1])
+
+
+def test_requant_nvfp4_mxfp8_rne_nearest_and_sr_unbiased(ora):
+    """With a general global scale: every RNE code is within half an E4M3
+    spacing of the binary32 decode times 2^-E (torch's E4M3 decode), and the
+    stochastic result is unbiased over seeds (within 5 standard errors)."""
+    A, _ = W.nvfp4_linear_small(M=64, N=16, K=128, seed=9)
+    q = ora.quant_nvfp4(W.bf16_bits(A), block_2d=True)
+    deq = ora.dequant(ora.NVFP4, *q).T                      # [C, R], binary64 of the binary32 decode
+    c, s = ora.requant_nvfp4_mxfp8(*q, sr=False)
+    v = deq.reshape(128, 2, 32) / (2.0 ** (s.astype(np.float64) - 127))[..., None]
+    v = np.clip(v, -448, 448)
+    got = _torch_e4m3_value(c).astype(np.float64).reshape(128, 2, 32)
+    e = np.floor(np.log2(np.maximum(np.abs(v), 2.0 ** -9)))
+    ulp = 2.0 ** (np.maximum(e, -6) - 3)
+    assert (np.abs(got - v) <= ulp / 2 + 1e-12).all()
+    n = 256
+    acc = np.zeros_like(deq)
+    for seed in range(n):
+        c, s = ora.requant_nvfp4_mxfp8(*q, sr=True, seed=seed)
+        acc += ora.dequant(ora.MXFP8, c, s)
+    mean = acc / n
+    d = deq.reshape(128, 2, 32)
+    s0 = ora.requant_nvfp4_mxfp8(*q, sr=False)[1]
+    ulp = (2.0 ** (np.maximum(np.floor(np.log2(np.maximum(np.abs(d) / (2.0 ** (s0.astype(np.float64) - 127))[..., None],
+                                                                  2.0 ** -9))), -6) - 3)
+           * (2.0 ** (s0.astype(np.float64) - 127))[..., None]).reshape(128, 64)
+    se = ulp / 2 / np.sqrt(n)
+    scaled = np.abs(d) / (2.0 ** (s0.astype(np.float64) - 127))[..., None]
+    ok = (scaled <= 448).reshape(128, 64)          # values past 448 saturate: no unbiasedness there
+    assert ok.mean() > 0.9
+    assert (np.abs(mean - deq)[ok] <= 5 * se[ok] + 1e-12).all()

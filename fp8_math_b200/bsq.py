@@ -19,7 +19,7 @@ LIB_PATH = os.path.join(HERE, "libbsq.so")
 
 BSQ_OK, BSQ_ERR_INVALID, BSQ_ERR_ALIGN, BSQ_ERR_UNSUPPORTED, BSQ_ERR_CUDA, BSQ_ERR_TIMEOUT = range(6)
 BSQ_RNE, BSQ_SR = 0, 1
-BSQ_NVFP4, BSQ_MXFP8 = 0, 1
+BSQ_NVFP4, BSQ_MXFP8, BSQ_MXFP4 = 0, 1, 2
 BSQ_OUT_F32, BSQ_OUT_BF16 = 0, 1
 BSQ_KNOB_FUSED_QUANT, BSQ_KNOB_GEMM_PAIR, BSQ_KNOB_GEMM_BN, BSQ_KNOB_STREAM_QUANT = 0, 1, 2, 3
 

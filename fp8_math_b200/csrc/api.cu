@@ -354,7 +354,7 @@ int bsq_requant_transpose(const uint8_t *codes_row, const uint8_t *sf_row, int64
 int bsq_gemm_blockscaled(int fmt, const uint8_t *A, const uint8_t *sfA, const float *gsA, const uint8_t *B,
                          const uint8_t *sfB, const float *gsB, int64_t M, int64_t N, int64_t K, void *C, int64_t ldc,
                          int out_type, void *stream) {
-    if ((fmt != BSQ_NVFP4 && fmt != BSQ_MXFP8) || (out_type != BSQ_OUT_F32 && out_type != BSQ_OUT_BF16))
+    if ((fmt != BSQ_NVFP4 && fmt != BSQ_MXFP8 && fmt != BSQ_MXFP4) || (out_type != BSQ_OUT_F32 && out_type != BSQ_OUT_BF16))
         return BSQ_ERR_INVALID;
     if (!A || !sfA || !B || !sfB || !C || M < 1 || N < 1 || K < 128 || K % 128 || ldc < N) return BSQ_ERR_INVALID;
     if (M > (1LL << 31) - 1 || N > (1LL << 31) - 1 || K > (1LL << 31) - 1) return BSQ_ERR_UNSUPPORTED;
@@ -376,7 +376,7 @@ int bsq_gemm_blockscaled(int fmt, const uint8_t *A, const uint8_t *sfA, const fl
 int bsq_grouped_gemm(int fmt, int G, const int32_t *row_off, const int32_t *sf_row_off, int64_t M_total,
                      const uint8_t *A, const uint8_t *sfA, const float *gsA, const uint8_t *B, const uint8_t *sfB,
                      const float *gsB, int64_t N, int64_t K, void *C, int64_t ldc, int out_type, void *stream) {
-    if ((fmt != BSQ_NVFP4 && fmt != BSQ_MXFP8) || (out_type != BSQ_OUT_F32 && out_type != BSQ_OUT_BF16))
+    if ((fmt != BSQ_NVFP4 && fmt != BSQ_MXFP8 && fmt != BSQ_MXFP4) || (out_type != BSQ_OUT_F32 && out_type != BSQ_OUT_BF16))
         return BSQ_ERR_INVALID;
     if (G < 1 || !row_off || !sf_row_off || !A || !sfA || !B || !sfB || !C || M_total < 0 || N < 1 || K < 128 ||
         K % 128 || ldc < N)

@@ -58,6 +58,14 @@ struct FmtTraits<BSQ_NVFP4> {
     static constexpr uint32_t kIdescFmt = (1u << 7) | (1u << 10);  // E2M1 x E2M1, UE4M3 scales
 };
 template <>
+struct FmtTraits<BSQ_MXFP4> {
+    static constexpr int kBkElems = 256;     // elements per 128-byte k-tile row
+    static constexpr int kMmaK = 64;
+    static constexpr int kAtomsPerKt = 2;    // 8 blocks of 32 per k-tile: two 4-block atoms
+    static constexpr int kVec = 32;
+    static constexpr uint32_t kIdescFmt = (1u << 7) | (1u << 10) | (1u << 23);  // E2M1 x E2M1, UE8M0 scales
+};
+template <>
 struct FmtTraits<BSQ_MXFP8> {
     static constexpr int kBkElems = 128;
     static constexpr int kMmaK = 32;
@@ -81,7 +89,9 @@ struct Cfg {
     // TMEM scale-factor slots: NVFP4 copies one slot per MMA (4 SFA columns
     // + 4 per 128 rows of B), MXFP8 one slot per k-tile (its atoms cover the
     // 4 MMAs of the k-tile, selected by the scale-factor id)
-    static constexpr int kSlotCols = 4 + 4 * kNbAtomTiles;
+    // MXFP4 copies one slot per k-tile too, holding both k-atoms (SFA 2 x 4
+    // columns, then per 128 rows of B 2 x 4 columns)
+    static constexpr int kSlotCols = (FMT == BSQ_MXFP4) ? 8 + 8 * kNbAtomTiles : 4 + 4 * kNbAtomTiles;
     static constexpr int kSlots = (FMT == BSQ_NVFP4) ? 16 : 8;
     static constexpr int kMmaPerKt = T::kBkElems / T::kMmaK;  // 4
     static constexpr int kEpiWarps = 8;
@@ -227,7 +237,7 @@ __global__ void __launch_bounds__(320, 1)
                     }
                     const int64_t krem = p.K - kt * T::kBkElems;
                     const int nmma = krem >= T::kBkElems ? C_::kMmaPerKt : (int)(krem / T::kMmaK);
-                    const int atoms = (FMT == BSQ_NVFP4) ? nmma : 1;
+                    const int atoms = (FMT == BSQ_NVFP4) ? nmma : (FMT == BSQ_MXFP4) ? (nmma + 1) / 2 : 1;
                     uint32_t bytes = C_::kABytes + C_::kBBytes + atoms * 512;
                     int nbat = 0;
                     for (int r = 0; r < C_::kNbAtomTiles; r++)
@@ -310,6 +320,32 @@ __global__ void __launch_bounds__(320, 1)
                                 tmem_cp_sf_atom(slot + 4 + 4 * r, desc_pack(sfb_lo + kSfbTileLo * r + kSfAtomLo * j, kSfHi));
                             mma_nvfp4(d_tmem, desc_pack(a_lo + 2 * j, kOpHi), desc_pack(b_lo + 2 * j, kOpHi), idesc, slot,
                                       slot + 4, (kt > 0 || j > 0) ? 1u : 0u);
+                        };
+                        if (full_kt) {
+#pragma unroll
+                            for (int j = 0; j < C_::kMmaPerKt; j++) issue(j);
+                        } else {
+                            for (int j = 0; j < nmma; j++) issue(j);
+                        }
+                    } else if (FMT == BSQ_MXFP4) {
+                        // one slot per k-tile: SFA k-atom a at columns 4a, SFB k-atom a (all
+                        // 128-row tiles of B, contiguous) at 8 + 4 kNbAtomTiles a; MMA j reads
+                        // k-atom j / 2, scale bytes 2 (j % 2) and 2 (j % 2) + 1 (id 2 (j % 2))
+                        const uint32_t slot = sf_t0 + (ktc & (C_::kSlots - 1)) * C_::kSlotCols;
+                        constexpr uint32_t kSfb0 = 8, kSfbA = 4 * C_::kNbAtomTiles;
+                        const int natoms = (nmma + 1) / 2;
+                        for (int a = 0; a < natoms; a++) {
+                            tmem_cp_sf_atom(slot + 4 * a, desc_pack(sfa_lo + kSfAtomLo * a, kSfHi));
+#pragma unroll
+                            for (int r = 0; r < C_::kNbAtomTiles; r++)
+                                tmem_cp_sf_atom(slot + kSfb0 + kSfbA * a + 4 * r,
+                                                desc_pack(sfb_lo + kSfbTileLo * r + kSfAtomLo * a, kSfHi));
+                        }
+                        auto issue = [&](int j) {
+                            const uint32_t id = 2u * (uint32_t)(j & 1), a = (uint32_t)(j >> 1);
+                            mma_mxfp4(d_tmem, desc_pack(a_lo + 2 * j, kOpHi), desc_pack(b_lo + 2 * j, kOpHi),
+                                      idesc | (id << 29) | (id << 4), (slot + 4 * a) | (id << 30),
+                                      (slot + kSfb0 + kSfbA * a) | (id << 30), (kt > 0 || j > 0) ? 1u : 0u);
                         };
                         if (full_kt) {
 #pragma unroll
@@ -554,8 +590,8 @@ struct Cfg2 {
     static constexpr int kSmemBytes = kStagingOff + kStagingBytes + 1024;
     static constexpr int kMmaPerKt = T::kBkElems / T::kMmaK;
     // TMEM scale slots of stage s: SFB at kSfb0 + kSfbCols*s, SFA at kSfa0 + kSfaCols*s
-    static constexpr int kSfbCols = (FMT == BSQ_NVFP4) ? 32 : 8;
-    static constexpr int kSfaCols = (FMT == BSQ_NVFP4) ? 16 : 4;
+    static constexpr int kSfbCols = (FMT == BSQ_NVFP4) ? 32 : (FMT == BSQ_MXFP4) ? 16 : 8;
+    static constexpr int kSfaCols = (FMT == BSQ_NVFP4) ? 16 : (FMT == BSQ_MXFP4) ? 8 : 4;
     static constexpr int kSfb0 = 256;
     static constexpr int kSfa0 = 256 + kStages * kSfbCols;
     static constexpr int kSfBoxRows = kSfaBytes / 256;  // SF tensor-map box height (rows of 256 B)
@@ -770,6 +806,12 @@ __global__ void __launch_bounds__(448, 1)
                         if (FMT == BSQ_NVFP4) {
                             // MMA j: SFA at 4j (4-column aligned), SFB atoms at 8j and 8j + 4
                             mma_nvfp4_pair(tmem_base, ad, bd, idesc, sfa_t + 4 * j, sfb_t + 8 * j, acc);
+                        } else if (FMT == BSQ_MXFP4) {
+                            // MMA j: k-atom j / 2 (SFA at 4 (j / 2), SFB at 8 (j / 2)), scale
+                            // bytes 2 (j % 2) and 2 (j % 2) + 1
+                            const uint32_t id = 2u * (uint32_t)(j & 1), a = (uint32_t)(j >> 1);
+                            mma_mxfp4_pair(tmem_base, ad, bd, idesc | (id << 29) | (id << 4), (sfa_t + 4 * a) | (id << 30),
+                                           (sfb_t + 8 * a) | (id << 30), acc);
                         } else {
                             // scale byte j of each 32-bit column (scale-factor id)
                             mma_mxfp8_pair(tmem_base, ad, bd, idesc | ((uint32_t)j << 29) | ((uint32_t)j << 4),
@@ -826,6 +868,17 @@ __global__ void __launch_bounds__(448, 1)
                         tmem_st_x8(sfb_t + 8 * j, w);
                         // SFA of MMA j: this quarter's rows, in the column the quarter reads
                         tmem_st_x1(sfa_t + 4 * j + q, *reinterpret_cast<const uint32_t *>(sfa + 512 * j + 16 * lane + 4 * q));
+                    }
+                } else if (FMT == BSQ_MXFP4) {
+#pragma unroll
+                    for (int a = 0; a < 2; a++) {
+                        // k-atom a: SFB of both 128-row atoms (every quarter), SFA of this quarter
+                        const uint4 b0 = *reinterpret_cast<const uint4 *>(sfb + 512 * a + 16 * lane);
+                        const uint4 b1 = *reinterpret_cast<const uint4 *>(sfb + C_::kSfaBytes + 512 * a + 16 * lane);
+                        const uint32_t w[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+                        tmem_st_x8(sfb_t + 8 * a, w);
+                        tmem_st_x1(sfa_t + 4 * a + q,
+                                   *reinterpret_cast<const uint32_t *>(sfa + 512 * a + 16 * lane + 4 * q));
                     }
                 } else {
                     const uint4 b0 = *reinterpret_cast<const uint4 *>(sfb + 16 * lane);
@@ -1129,7 +1182,7 @@ int run(const CUtensorMap &ta, const CUtensorMap &tb, const GemmParams &p, int g
 template <int FMT>
 int dispatch(const GemmArgs &g, cudaStream_t s) {
     using T = FmtTraits<FMT>;
-    const int64_t kb_bytes = (FMT == BSQ_NVFP4) ? g.K / 2 : g.K;
+    const int64_t kb_bytes = (FMT == BSQ_MXFP8) ? g.K : g.K / 2;
     const bool grouped = g.G > 0;
     const bool swap = !grouped && g.M <= 64 && g.N >= 128;
     // operand A supplies the 128-row MMA dimension
@@ -1151,7 +1204,7 @@ int dispatch(const GemmArgs &g, cudaStream_t s) {
     // (tuning, tests).
     const int64_t c_esz = g.out_bf16 ? 2 : 4;
     const bool c_tma_ok = (reinterpret_cast<uintptr_t>(g.C) % 16 == 0) && (g.ldc * c_esz) % 16 == 0;
-    const bool pair_ok = !swap && NB >= 128 && c_tma_ok && !(grouped && FMT == BSQ_NVFP4 && g.K % 256 != 0);
+    const bool pair_ok = !swap && NB >= 128 && c_tma_ok && !(FMT != BSQ_MXFP8 && g.K % 256 != 0);
     bool use_pair = pair_ok && MA >= 256 && NB >= 256;
     if (const int v = kernel_choice(BSQ_KNOB_GEMM_PAIR); v >= 0) use_pair = pair_ok && v != 0;
     if (const int v = kernel_choice(BSQ_KNOB_GEMM_BN); v > 0) {  // tuning override of the single-CTA tile
@@ -1212,6 +1265,7 @@ int dispatch(const GemmArgs &g, cudaStream_t s) {
 
 int launch_gemm(const GemmArgs &g, cudaStream_t s) {
     if (g.fmt == BSQ_NVFP4) return dispatch<BSQ_NVFP4>(g, s);
+    if (g.fmt == BSQ_MXFP4) return dispatch<BSQ_MXFP4>(g, s);
     return dispatch<BSQ_MXFP8>(g, s);
 }
 

@@ -66,7 +66,7 @@ enum {
 };
 
 enum { BSQ_RNE = 0, BSQ_SR = 1 };          /* rounding for MXFP8 outputs */
-enum { BSQ_NVFP4 = 0, BSQ_MXFP8 = 1 };     /* GEMM operand format */
+enum { BSQ_NVFP4 = 0, BSQ_MXFP8 = 1, BSQ_MXFP4 = 2 }; /* GEMM operand format */
 enum { BSQ_OUT_F32 = 0, BSQ_OUT_BF16 = 1 }; /* GEMM output type */
 
 /* Kernel-selection overrides (bsq_debug_kernel_choice). */
@@ -256,8 +256,10 @@ BSQ_API int bsq_requant_transpose(const uint8_t *codes_row_dev, const uint8_t *s
  *   C[m][n] = alpha * sum_k decA[m][k] * decB[n][k],
  * A [M][K] and B [N][K] both K-major (codes row-major, as the quantizers
  * write them), with their swizzled SF buffers.  NVFP4: alpha =
- * (*gsA_dev) * (*gsB_dev) (each may be NULL for 1); MXFP8: alpha = 1 and
- * gs* are ignored.  Accumulation is fp32 in tensor memory; C is fp32 or
+ * (*gsA_dev) * (*gsB_dev) (each may be NULL for 1); MXFP8 and MXFP4 (E2M1
+ * codes packed as bsq_quant_mxfp4 writes them, one E8M0 scale per 32
+ * elements; "08 -- FP4, MXFP4, NVFP4 ...", table "The two Blackwell
+ * formats"): alpha = 1 and gs* are ignored.  Accumulation is fp32 in tensor memory; C is fp32 or
  * bf16 (nearest-even), row-major with leading dimension ldc (elements).
  * Requirements: K % 128 == 0; M, N >= 1. */
 BSQ_API int bsq_gemm_blockscaled(int fmt, const uint8_t *A_dev, const uint8_t *sfA_dev, const float *gsA_dev,

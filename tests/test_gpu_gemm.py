@@ -18,7 +18,7 @@ from gpu_util import assert_gemm_close, bits, dev
 
 pytestmark = pytest.mark.gpu
 
-NV, MX = 0, 1
+NV, MX, MX4 = 0, 1, 2
 
 
 def oracle_operands(ora, fmt, A, B, rht=None, fos=False, b2d=True, sr=False, seed=0):
@@ -27,6 +27,9 @@ def oracle_operands(ora, fmt, A, B, rht=None, fos=False, b2d=True, sr=False, see
     if fmt == NV:
         qa = ora.quant_nvfp4(bits(A), rht_mask=rht, four_over_six=fos)
         qb = ora.quant_nvfp4(bits(B), block_2d=b2d and B.shape[0] % 16 == 0, rht_mask=rht)
+    elif fmt == MX4:
+        qa = (*ora.quant_mxfp4(bits(A), sr=sr, seed=seed, stream_id=0), 1.0)
+        qb = (*ora.quant_mxfp4(bits(B), sr=sr, seed=seed, stream_id=1), 1.0)
     else:
         qa = (*ora.quant_mxfp8(bits(A), sr=sr, seed=seed, stream_id=0), 1.0)
         qb = (*ora.quant_mxfp8(bits(B), sr=sr, seed=seed, stream_id=1), 1.0)
@@ -52,7 +55,7 @@ def run_gemm(ora, fmt, qa, qb, M, N, K, out_dtype):
 # forced through the dispatch's tuning switch (the default picks pairs for
 # operands of 256+ rows)
 @pytest.mark.parametrize("pair", [0, 1])
-@pytest.mark.parametrize("fmt", [NV, MX])
+@pytest.mark.parametrize("fmt", [NV, MX, MX4])
 @pytest.mark.parametrize("M,N,K,out", [
     (128, 256, 256, torch.float32),     # the small NVFP4 linear workload shape
     (256, 512, 512, torch.bfloat16),    # BN = 256 path, several tiles
@@ -84,7 +87,7 @@ def test_gemm_small_linear_workload_exact_inputs(ora):
 
 
 @pytest.mark.parametrize("pair", [0, 1])
-@pytest.mark.parametrize("fmt", [NV, MX])
+@pytest.mark.parametrize("fmt", [NV, MX, MX4])
 def test_grouped_gemm_compare(ora, knobs, pair, fmt):
     """Small MoE: routed rows grouped by expert (uneven counts, one expert
     possibly empty), per-expert B and global scales."""
@@ -101,6 +104,9 @@ def test_grouped_gemm_compare(ora, knobs, pair, fmt):
     if fmt == NV:
         qa = ora.quant_nvfp4(bits(Xg), four_over_six=True)
         qbs = [ora.quant_nvfp4(bits(Wup[e]), block_2d=True) for e in range(E)]
+    elif fmt == MX4:
+        qa = (*ora.quant_mxfp4(bits(Xg)), 1.0)
+        qbs = [(*ora.quant_mxfp4(bits(Wup[e])), 1.0) for e in range(E)]
     else:
         qa = (*ora.quant_mxfp8(bits(Xg)), 1.0)
         qbs = [(*ora.quant_mxfp8(bits(Wup[e])), 1.0) for e in range(E)]

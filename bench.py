@@ -356,7 +356,9 @@ def measure_rows(hbm, fp4_peak, fp8_peak, reps=10, only=None):
             lambda: api.gemm(0, qar[0], qar[1], qwr[0], qwr[1], 64, N4, K4, gsA=qar[2], gsB=qwr[2], out=Cr),
             nbytes=N4 * K4 // 2 + N4 * K4 // 16 + 64 * K4 // 2 + 64 * K4 // 16 + 64 * N4 * 2)
         del Cr, qar, qwr, W4, qwc
-    if wants("a4 NVFP4 Four Over Six quantize (gathered, expert groups)", "a9 grouped NVFP4 GEMM up", "a9 grouped NVFP4 GEMM down"):
+    if wants("a4 NVFP4 Four Over Six quantize (gathered, expert groups)", "a9 grouped NVFP4 GEMM up", "a9 grouped NVFP4 GEMM down",
+             "a9+a4 grouped up GEMM, then amax + 4/6 quantize of H (two kernels)",
+             "f1 grouped up GEMM with the 4/6 NVFP4 quantize in its epilogue (next row)"):
         # -- MoE forward, 16384 tokens, 64 experts, top-8 (gathered 4/6 quantize, grouped up and down)
         moe = W.moe_forward()
         T3, H3 = moe.X.shape
@@ -387,6 +389,21 @@ def measure_rows(hbm, fp4_peak, fp8_peak, reps=10, only=None):
             lambda: api.grouped_gemm(0, offs, sfo, qx[0], qx[1], up[0], up[1], Mt, F3, H3, gsA=qx[2], gsB=up[2],
                                      out=Cup), flops=2 * Mt * F3 * H3, peak_kind="fp4")
         qh = api.quant_nvfp4(Cup, four_over_six=True, groups=(offs, sfo, sf_rows))
+
+        def up_then_quantize():
+            api.grouped_gemm(0, offs, sfo, qx[0], qx[1], up[0], up[1], Mt, F3, H3, gsA=qx[2], gsB=up[2], out=Cup)
+            api.quant_nvfp4(Cup, four_over_six=True, groups=(offs, sfo, sf_rows), out=qh)
+        row("a9+a4 grouped up GEMM, then amax + 4/6 quantize of H (two kernels)",
+            f"{Mt} routed rows x {F3} x {H3} -> NVFP4 H", up_then_quantize, flops=2 * Mt * F3 * H3, peak_kind="fp4")
+        fq = (torch.empty(Mt, F3 // 2, dtype=torch.uint8, device=dev),
+              torch.zeros(api.sf_bytes(sf_rows, F3 // 16), dtype=torch.uint8, device=dev),
+              torch.empty(1, dtype=torch.float32, device=dev), None)
+        row("f1 grouped up GEMM with the 4/6 NVFP4 quantize in its epilogue (next row)",
+            f"{Mt} routed rows x {F3} x {H3} -> NVFP4 H",
+            lambda: api.grouped_gemm_nvfp4_out(offs, sfo, qx[0], qx[1], up[0], up[1], Mt, F3, H3, qh[2], sf_rows,
+                                               gsA=qx[2], gsB=up[2], four_over_six=True, out=fq),
+            flops=2 * Mt * F3 * H3, peak_kind="fp4")
+        del fq
         del up
         dn = experts(moe.W_dn)
         Cdn = torch.empty(Mt, H3, dtype=torch.bfloat16, device=dev)

@@ -160,3 +160,22 @@ def grouped_gemm(fmt, row_offsets, sf_row_offsets, A, sfA, B, sfB, M_total, N, K
     bsq.bsq_grouped_gemm(fmt, G, row_offsets, sf_row_offsets, M_total, A, sfA, gsA, B, sfB, gsB, N, K, C_out,
                          C_out.stride(0), ot)
     return C_out
+
+
+def grouped_gemm_nvfp4_out(row_offsets, sf_row_offsets, A, sfA, B, sfB, M_total, N, K, out_gs, sf_rows,
+                           gsA=None, gsB=None, four_over_six=True, amax=True, bf16_out=False, out=None):
+    """Grouped NVFP4 GEMM with the output quantized to NVFP4 in the epilogue
+    (given global scale out_gs [1]).  Returns (codes [M_total, N/2], sf
+    swizzled with sf_rows rows, amax [1] or None, C bf16 or None)."""
+    G = row_offsets.shape[0] - 1
+    if out is None:
+        codes = torch.empty(M_total, N // 2, dtype=torch.uint8, device=A.device)
+        sf = torch.zeros(sf_bytes(sf_rows, N // 16), dtype=torch.uint8, device=A.device)
+        am = torch.empty(1, dtype=torch.float32, device=A.device) if amax else None
+        C_out = _out(M_total, N, torch.bfloat16, A.device) if bf16_out else None
+    else:
+        codes, sf, am, C_out = out
+    bsq.bsq_grouped_gemm_nvfp4_out(bsq.BSQ_NVFP4, G, row_offsets, sf_row_offsets, M_total, A, sfA, gsA, B, sfB, gsB,
+                                   N, K, out_gs, four_over_six, codes, sf, am, C_out,
+                                   C_out.stride(0) if C_out is not None else 0)
+    return codes, sf, am, C_out

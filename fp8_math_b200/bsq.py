@@ -51,6 +51,8 @@ _SIGS = {
                                        C.c_int, _vp]),
     "bsq_grouped_gemm": (C.c_int, [C.c_int, C.c_int, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64,
                                    _vp, _i64, C.c_int, _vp]),
+    "bsq_grouped_gemm_nvfp4_out": (C.c_int, [C.c_int, C.c_int, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _i64,
+                                             _i64, _vp, C.c_int, _vp, _vp, _vp, _vp, _i64, _vp]),
     "bsq_check": (C.c_int, [_vp]),
     "bsq_debug_timeout_probe": (C.c_int, [C.c_uint64, _vp]),
     "bsq_debug_kernel_choice": (C.c_int, [C.c_int, C.c_int]),
@@ -192,3 +194,10 @@ def bsq_quant_mxfp8_rowcol(x, M, K, ldx, rounding, seed, stream_id_row, stream_i
 def bsq_requant_nvfp4_mxfp8(codes, sf, gs, R, C, rounding, seed, stream_id, codes_col, sf_col, stream=None):
     return _check("bsq_requant_nvfp4_mxfp8", lib().bsq_requant_nvfp4_mxfp8(
         _p(codes), _p(sf), _p(gs), R, C, rounding, seed, stream_id, _p(codes_col), _p(sf_col), _stream(stream)))
+
+
+def bsq_grouped_gemm_nvfp4_out(fmt, G, row_offsets, sf_row_offsets, M_total, A, sfA, gsA, B, sfB, gsB, N, K, out_gs,
+                               four_over_six, out_codes, out_sf, out_amax, C_out, ldc, stream=None):
+    return _check("bsq_grouped_gemm_nvfp4_out", lib().bsq_grouped_gemm_nvfp4_out(
+        fmt, G, _p(row_offsets), _p(sf_row_offsets), M_total, _p(A), _p(sfA), _p(gsA), _p(B), _p(sfB), _p(gsB), N, K,
+        _p(out_gs), int(four_over_six), _p(out_codes), _p(out_sf), _p(out_amax), _p(C_out), ldc, _stream(stream)))

@@ -398,6 +398,37 @@ int bsq_grouped_gemm(int fmt, int G, const int32_t *row_off, const int32_t *sf_r
     return bsq::launch_gemm(g, static_cast<cudaStream_t>(stream));
 }
 
+int bsq_grouped_gemm_nvfp4_out(int fmt, int G, const int32_t *row_off, const int32_t *sf_row_off, int64_t M_total,
+                               const uint8_t *A, const uint8_t *sfA, const float *gsA, const uint8_t *B,
+                               const uint8_t *sfB, const float *gsB, int64_t N, int64_t K, const float *out_gs,
+                               int four_over_six, uint8_t *out_codes, uint8_t *out_sf, float *out_amax, void *C,
+                               int64_t ldc, void *stream) {
+    if (fmt != BSQ_NVFP4) return fmt == BSQ_MXFP8 || fmt == BSQ_MXFP4 ? BSQ_ERR_UNSUPPORTED : BSQ_ERR_INVALID;
+    if (G < 1 || !row_off || !sf_row_off || !A || !sfA || !B || !sfB || !out_gs || !out_codes || !out_sf ||
+        M_total < 0 || N < 128 || N % 64 || K < 256 || K % 256 || (C && ldc < N))
+        return BSQ_ERR_INVALID;
+    if (G > 1024) return BSQ_ERR_UNSUPPORTED;
+    if (!aligned16(A) || !aligned16(B) || !aligned16(sfA) || !aligned16(sfB) || !aligned16(out_codes) ||
+        !aligned16(out_sf) || (reinterpret_cast<uintptr_t>(out_gs) & 3u) ||
+        (out_amax && (reinterpret_cast<uintptr_t>(out_amax) & 3u)) || (C && (!aligned16(C) || (ldc * 2) % 16)))
+        return BSQ_ERR_ALIGN;
+    DeviceState *d;
+    if (int st = device_state(&d)) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (out_amax && cudaMemsetAsync(out_amax, 0, sizeof(float), s) != cudaSuccess) return BSQ_ERR_CUDA;
+    if (M_total == 0) return BSQ_OK;
+    bsq::GemmArgs g{};
+    g.fmt = fmt;
+    g.A = A; g.sfA = sfA; g.B = B; g.sfB = sfB; g.gsA = gsA; g.gsB = gsB;
+    g.M = M_total; g.N = N; g.K = K; g.C = C; g.ldc = C ? ldc : N; g.out_bf16 = true;
+    g.G = G; g.row_off = row_off; g.sf_row_off = sf_row_off;
+    g.err = d->err;
+    g.num_sms = d->num_sms;
+    g.q_codes = out_codes; g.q_sf = out_sf; g.q_sg = out_gs;
+    g.q_amax = reinterpret_cast<unsigned int *>(out_amax); g.q_fos = four_over_six != 0;
+    return bsq::launch_gemm(g, s);
+}
+
 int bsq_check(void *stream) {
     DeviceState *d;
     if (int st = device_state(&d)) return st;

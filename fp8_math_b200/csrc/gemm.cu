@@ -26,6 +26,7 @@
 
 #include "common.cuh"
 #include "gemm.cuh"
+#include "nvfp4.cuh"
 #include "sm100.cuh"
 
 namespace bsq {
@@ -45,6 +46,12 @@ struct GemmParams {
     int G;
     const int32_t *row_off, *sf_row_off;
     unsigned int *err;
+    // NVFP4 output of the quantizing epilogue (pair kernel with QOUT)
+    uint8_t *q_codes;     // [rows][NB/2]
+    uint8_t *q_sf;        // swizzled, NB/16 blocks per row, rows at the groups' SF offsets
+    const float *q_sg;    // the global scale the output is quantized with
+    unsigned int *q_amax; // atomicMax of the bits of max |bf16 output| (NULL: not kept)
+    int q_fos;            // Four Over Six block scales
 };
 
 template <int FMT>
@@ -583,7 +590,7 @@ struct Cfg2 {
     static constexpr int kBoxes = 2;                                // per epilogue warp: double-buffered
     static constexpr int kStagingBytes = kEpiWarps * kBoxes * kBoxBytes;
     static constexpr int kSmemLimit = 232448;                       // 227 KB per CTA
-    static constexpr int kStaticEst = GROUPED ? 8704 : 512;
+    static constexpr int kStaticEst = GROUPED ? 9728 : 512;   // grouped: offsets, tile starts, NVFP4 tables
     static constexpr int kFit = (kSmemLimit - 2048 - kStagingBytes - kStaticEst) / kStageBytes;
     static constexpr int kStages = kFit > 5 ? 5 : kFit;             // TMEM holds up to 5 stages of scales
     static constexpr int kStagingOff = (kStages * kStageBytes + 1023) / 1024 * 1024;
@@ -599,11 +606,12 @@ struct Cfg2 {
     static_assert(kStages >= 2, "shared-memory budget");
 };
 
-template <int FMT, bool OUT_BF16, bool GROUPED>
+template <int FMT, bool OUT_BF16, bool GROUPED, bool QOUT = false>
 __global__ void __launch_bounds__(448, 1)
     gemm_bs2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
                     const __grid_constant__ CUtensorMap tmC, const GemmParams p) {
+    static_assert(!QOUT || OUT_BF16, "the quantizing epilogue quantizes the bf16 output");
     using C_ = Cfg2<FMT, GROUPED>;
     using T = typename C_::T;
     constexpr int NS = C_::kStages;
@@ -615,6 +623,7 @@ __global__ void __launch_bounds__(448, 1)
     __shared__ volatile int abort_flag;
     __shared__ int tile_start[GROUPED ? 1025 : 1];
     __shared__ int32_t offs[GROUPED ? 1025 : 1];
+    __shared__ float q_den[QOUT ? 128 : 1], q_rcp[QOUT ? 128 : 1];
 
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sA = smem;
@@ -924,6 +933,23 @@ __global__ void __launch_bounds__(448, 1)
                 v[4 * c + 3] = w.w;
             }
         };
+        // quantizing epilogue: the NVFP4 tables of the given global scale
+        // (den / rcp per E4M3 code), built by the 256 epilogue threads
+        NvScale qs{};
+        if (QOUT) {
+            const float s_g = __ldg(p.q_sg);
+            const int et = ew * 32 + lane;
+            if (et < 128) {
+                const float den = __fmul_rn(e4m3_to_f32(et), s_g);
+                q_den[et] = den;
+                q_rcp[et] = (et == 0 || et == 127) ? 0.0f : __frcp_rn(den);
+            }
+            asm volatile("bar.sync 2, %0;" ::"n"(32 * C_::kEpiWarps) : "memory");
+            qs.s_g = s_g;
+            qs.c6 = __frcp_rn(__fmul_rn(6.0f, s_g));
+            qs.c4 = __frcp_rn(__fmul_rn(4.0f, s_g));
+            qs.fast = s_g >= 0x1p-90f && s_g <= 0x1p100f;
+        }
         int64_t it = 0;
         int nstored = 0;  // boxes this warp has handed to TMA (fp32 path: ring position)
         for (int64_t t = pair; t < total_tiles; t += npairs, it++) {
@@ -964,6 +990,46 @@ __global__ void __launch_bounds__(448, 1)
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive_cluster_relaxed(acce_leader);
+                if (QOUT) {
+                    // NVFP4 of this thread's 128 bf16 outputs (eight blocks of 16,
+                    // block b = pk[8b .. 8b + 7]), quantized as bsq_quant_nvfp4
+                    // does with the given global scale; codes and swizzled scale
+                    // words stored directly; max |output| kept for the next scale
+                    uint32_t amax_bits = 0u;
+                    if (row_ok) {
+                        const int64_t sf_row = sfa_row0 + 32 * q + lane;
+                        const int64_t qkb = p.NB >> 4;
+                        const uint32_t sw0[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+#pragma unroll
+                        for (int g4 = 0; g4 < 2; g4++) {
+                            const int64_t n4 = nb0 + 64 * g4;   // first column of 4 blocks
+                            if (n4 >= n_lim) break;
+                            uint32_t sbw = 0u;
+                            uint2 cd[4];
+#pragma unroll
+                            for (int i = 0; i < 4; i++) {
+                                const uint32_t *w = pk + 8 * (4 * g4 + i);
+                                uint32_t sb;
+                                if (p.q_fos) nv_block_1d<false, true>(w, sw0, qs, q_den, q_rcp, sb, cd[i]);
+                                else nv_block_1d<false, false>(w, sw0, qs, q_den, q_rcp, sb, cd[i]);
+                                sbw |= (sb & 0xFFu) << (8 * i);
+#pragma unroll
+                                for (int k = 0; k < 8; k++) amax_bits = max(amax_bits, max(w[k] & 0x7FFFu, (w[k] >> 16) & 0x7FFFu));
+                            }
+                            uint4 *cp = reinterpret_cast<uint4 *>(p.q_codes + ar * (p.NB >> 1) + (n4 >> 1));
+                            cp[0] = make_uint4(cd[0].x, cd[0].y, cd[1].x, cd[1].y);
+                            cp[1] = make_uint4(cd[2].x, cd[2].y, cd[3].x, cd[3].y);
+                            *reinterpret_cast<uint32_t *>(p.q_sf + sf_word_offset(sf_row, n4 >> 6, qkb)) = sbw;
+                        }
+                    }
+                    if (p.q_amax) {
+#pragma unroll
+                        for (int o = 16; o; o >>= 1) amax_bits = max(amax_bits, __shfl_xor_sync(0xFFFFFFFFu, amax_bits, o));
+                        // bf16 magnitude bits << 16 are the fp32 bits of the same value
+                        if (lane == 0 && amax_bits) atomicMax(p.q_amax, amax_bits << 16);
+                    }
+                    if (p.C == nullptr) continue;
+                }
 #pragma unroll
                 for (int c = 0; c < HC / 32; c++) {
                     const int64_t n = nb0 + 32 * c;
@@ -1148,11 +1214,11 @@ bool make_c_tmap(CUtensorMap *m, void *C, bool bf16, int64_t n_cols, int64_t row
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int FMT, bool OUT_BF16, bool GROUPED>
+template <int FMT, bool OUT_BF16, bool GROUPED, bool QOUT = false>
 int run_pair(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &tsa, const CUtensorMap &tsb,
              const CUtensorMap &tc, const GemmParams &p, int pairs, cudaStream_t s) {
     using C_ = Cfg2<FMT, GROUPED>;
-    auto kern = gemm_bs2_kernel<FMT, OUT_BF16, GROUPED>;
+    auto kern = gemm_bs2_kernel<FMT, OUT_BF16, GROUPED, QOUT>;
     if (smem_attr_once(reinterpret_cast<const void *>(kern), C_::kSmemBytes) != BSQ_OK) return BSQ_ERR_CUDA;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * pairs, 1, 1);
@@ -1203,10 +1269,17 @@ int dispatch(const GemmArgs &g, cudaStream_t s) {
     // override forces either kernel where the pair kernel is possible
     // (tuning, tests).
     const int64_t c_esz = g.out_bf16 ? 2 : 4;
-    const bool c_tma_ok = (reinterpret_cast<uintptr_t>(g.C) % 16 == 0) && (g.ldc * c_esz) % 16 == 0;
+    const bool qout = g.q_codes != nullptr;
+    const bool c_tma_ok = (g.C == nullptr && qout) ||
+                          ((reinterpret_cast<uintptr_t>(g.C) % 16 == 0) && (g.ldc * c_esz) % 16 == 0);
     const bool pair_ok = !swap && NB >= 128 && c_tma_ok && !(FMT != BSQ_MXFP8 && g.K % 256 != 0);
     bool use_pair = pair_ok && MA >= 256 && NB >= 256;
     if (const int v = kernel_choice(BSQ_KNOB_GEMM_PAIR); v >= 0) use_pair = pair_ok && v != 0;
+    if (qout) {
+        // the quantizing epilogue exists in the pair kernel only
+        if (!pair_ok || !grouped || !g.out_bf16 || FMT != BSQ_NVFP4) return BSQ_ERR_UNSUPPORTED;
+        use_pair = true;
+    }
     if (const int v = kernel_choice(BSQ_KNOB_GEMM_BN); v > 0) {  // tuning override of the single-CTA tile
         if ((v == 128 || (v == 256 && g.out_bf16)) && !swap) bn = v;
     }
@@ -1218,6 +1291,7 @@ int dispatch(const GemmArgs &g, cudaStream_t s) {
     p.sfB_group_bytes = (int64_t)((NB + 127) / 128 * 128) * ((g.K / T::kVec + 3) / 4 * 4);
     p.G = g.G; p.row_off = g.row_off; p.sf_row_off = g.sf_row_off;
     p.err = g.err;
+    p.q_codes = g.q_codes; p.q_sf = g.q_sf; p.q_sg = g.q_sg; p.q_amax = g.q_amax; p.q_fos = g.q_fos ? 1 : 0;
     CUtensorMap ta, tb;
     if (!make_tmap(&ta, opA, kb_bytes, MA, 128)) return BSQ_ERR_CUDA;
     if (use_pair) {
@@ -1232,10 +1306,17 @@ int dispatch(const GemmArgs &g, cudaStream_t s) {
         const int box = Cfg2<FMT, false>::kSfBoxRows;
         if (!make_sf_tmap(&tsa, sfA, sfa_bytes, box) || !make_sf_tmap(&tsb, sfB, sfb_bytes, box)) return BSQ_ERR_CUDA;
         CUtensorMap tc;
-        if (!make_c_tmap(&tc, g.C, g.out_bf16, NB, MA, g.ldc)) return BSQ_ERR_CUDA;
+        // without a bf16 output the store map is never used: give it the code
+        // buffer's own extent (rows of NB/2 bytes seen as NB/4 bf16)
+        if (g.C == nullptr ? !make_c_tmap(&tc, g.q_codes, true, NB / 4, MA, NB / 4)
+                           : !make_c_tmap(&tc, g.C, g.out_bf16, NB, MA, g.ldc))
+            return BSQ_ERR_CUDA;
         int64_t ptiles = grouped ? (MA / 256 + g.G) * ((NB + 255) / 256) : ((MA + 255) / 256) * ((NB + 255) / 256);
         int pairs = (int)(ptiles < g.num_sms / 2 ? (ptiles < 1 ? 1 : ptiles) : g.num_sms / 2);
         if (grouped) {
+            if constexpr (FMT == BSQ_NVFP4) {
+                if (qout) return run_pair<FMT, true, true, true>(ta, tb, tsa, tsb, tc, p, pairs, s);
+            }
             if (g.out_bf16) return run_pair<FMT, true, true>(ta, tb, tsa, tsb, tc, p, pairs, s);
             return run_pair<FMT, false, true>(ta, tb, tsa, tsb, tc, p, pairs, s);
         }

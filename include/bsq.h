@@ -284,6 +284,35 @@ BSQ_API int bsq_grouped_gemm(int fmt, int G, const int32_t *row_offsets_dev, con
                      const uint8_t *B_dev, const uint8_t *sfB_dev, const float *gsB_dev,
                      int64_t N, int64_t K, void *C_dev, int64_t ldc, int out_type, void *stream);
 
+/* Grouped NVFP4 GEMM whose output is written in NVFP4 ("Microscaling ...",
+ * section "Open points": fused quantize-and-GEMM kernels, since computing
+ * block scales is itself memory traffic; "Thinking Machines ...", section
+ * "Why communication became the next bottleneck": kernels that combine
+ * matrix operations, quantization and rounding).  The MoE up projection's
+ * output H feeds the down projection in NVFP4, so the epilogue quantizes it
+ * directly instead of storing bf16 H and reading it back: for each group
+ * e, H[m][n] = bf16_RNE(alpha_e * sum_k decA[m][k] decB_e[n][k]) exactly as
+ * bsq_grouped_gemm computes it, then NVFP4 with 1x16 blocks as
+ * bsq_quant_nvfp4 computes it -- Four Over Six when four_over_six != 0 --
+ * but with the GIVEN global scale *out_gs_dev (a tensor scale must be known
+ * before the first block is quantized, and the GEMM produces H tile by
+ * tile: the caller passes a scale from an earlier amax, e.g. the previous
+ * step's, as delayed scaling does).  Outputs: out_codes [M_total][N/2];
+ * out_sf swizzled for N/16 blocks per row, group e's rows starting at SF row
+ * sf_row_offsets[e] (the layout bsq_grouped_gemm reads for A); *out_amax_dev
+ * (if not NULL; zeroed first) = max |H| over all rows, from which the next
+ * global scale amax / 2688 follows.  C_bf16_dev, if not NULL, also receives
+ * H in bf16 (leading dimension ldc).  Operands as for bsq_grouped_gemm with
+ * fmt = BSQ_NVFP4 (other formats: BSQ_ERR_UNSUPPORTED); N % 64 == 0,
+ * N >= 128, K % 256 == 0. */
+BSQ_API int bsq_grouped_gemm_nvfp4_out(int fmt, int G, const int32_t *row_offsets_dev,
+                                       const int32_t *sf_row_offsets_dev, int64_t M_total, const uint8_t *A_dev,
+                                       const uint8_t *sfA_dev, const float *gsA_dev, const uint8_t *B_dev,
+                                       const uint8_t *sfB_dev, const float *gsB_dev, int64_t N, int64_t K,
+                                       const float *out_gs_dev, int four_over_six, uint8_t *out_codes_dev,
+                                       uint8_t *out_sf_dev, float *out_amax_dev, void *C_bf16_dev, int64_t ldc,
+                                       void *stream);
+
 /* Synchronize `stream`, then read and clear this device's error word.
  * Returns BSQ_OK, BSQ_ERR_TIMEOUT (a kernel's bounded wait ran out; the
  * kernel returned early and its outputs are undefined) or BSQ_ERR_CUDA. */

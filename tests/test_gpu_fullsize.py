@@ -321,10 +321,19 @@ def test_moe_forward_chain_full(ora, T):
     t0 = time.perf_counter()
     _check_grouped_full(ora, Hg, qx, qup, offs, True, "up", T)
     _log("oracle check of the up GEMM", t0)
-    del cx, sx, up_dev
+    del up_dev
 
     # 3. the device chain: 4/6 quantize of the device's H, then the down GEMM
     ch, sh, gh = api.quant_nvfp4(Hg, four_over_six=True, groups=(offs_d, sfo_d, sf_rows))
+    # the up GEMM with the quantizing epilogue, given the chain's global scale,
+    # writes the same bytes without storing H
+    up_dev = _experts_device(ora, qup, F, H)
+    fc, fs, fa, _ = api.grouped_gemm_nvfp4_out(offs_d, sfo_d, cx, sx, up_dev[0], up_dev[1], Mt, F, H, gh, sf_rows,
+                                               gsA=gx, gsB=up_dev[2], four_over_six=True)
+    assert bsq.bsq_check() == bsq.BSQ_OK
+    assert torch.equal(fc, ch) and torch.equal(fs, sh)
+    assert fa.item() == api.amax(Hg).item()
+    del fc, fs, fa, up_dev
     Cd = api.grouped_gemm(NV, offs_d, sfo_d, ch, sh, dn_dev[0], dn_dev[1], Mt, H, F, gsA=gh, gsB=dn_dev[2],
                           out_dtype=torch.bfloat16)
     assert bsq.bsq_check() == bsq.BSQ_OK
@@ -346,7 +355,7 @@ def test_moe_forward_chain_full(ora, T):
         assert_gemm_close(Cd[r0:r1].float().cpu().numpy().astype(np.float64), Cr, Ra, True,
                           f"down (device chain) expert {e}")
     _log("binary64 check of the chain's down GEMM", t0)
-    del ch, sh, Cd, yh, ch_h, sh_can
+    del ch, sh, Cd, yh, ch_h, sh_can, cx, sx
 
     # 4. the oracle's own H through the same two kernels
     t0 = time.perf_counter()

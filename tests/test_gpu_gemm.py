@@ -143,3 +143,61 @@ def test_gemm_invalid_arguments():
         bsq.bsq_gemm_blockscaled(NV, z, z, None, z, z, None, 4, 4, 100, Cm, 4, bsq.BSQ_OUT_F32)
     assert e.value.status == bsq.BSQ_ERR_INVALID
     assert bsq.bsq_check() == bsq.BSQ_OK
+
+
+@pytest.mark.parametrize("fos", [True, False])
+def test_grouped_gemm_nvfp4_output(ora, fos):
+    """The quantizing epilogue: a grouped NVFP4 GEMM (small MoE up
+    projection, K = 256, N = 192) writing NVFP4 with a given global scale.
+    With the scale of the output's own amax it reproduces, byte for byte, the
+    plain GEMM's bf16 output quantized by bsq_quant_nvfp4 (same groups, same
+    Four Over Six); its amax is that output's; and its codes and scales have
+    the NVFP4 properties (nearest E2M1 codes under candidate scales) on that
+    output.  A different scale gives the same properties under that scale."""
+    from nvfp4_props import check_nvfp4
+    E, T, H, F = 6, 160, 256, 192
+    g = torch.Generator().manual_seed(21)
+    logits = torch.randn(T, E, generator=g)
+    logits[:, 4] = -1e9  # expert 4 receives no rows
+    ri, offs, sfo = W.route_topk(logits, 2)
+    X = torch.randn(T, H, generator=g).to(torch.bfloat16)
+    Wup = (torch.randn(E, F, H, generator=g) * 0.02).to(torch.bfloat16)
+    Mt, sf_rows = int(offs[-1]), int(sfo[-1])
+    Xg = X[torch.from_numpy(ri.astype(np.int64))]
+    qa = ora.quant_nvfp4(bits(Xg), four_over_six=True)
+    qbs = [ora.quant_nvfp4(bits(Wup[e]), block_2d=True) for e in range(E)]
+    can = np.zeros((sf_rows, H // 16), np.uint8)
+    for e in range(E):
+        can[sfo[e]:sfo[e] + offs[e + 1] - offs[e]] = qa[1][offs[e]:offs[e + 1]]
+    offs_d, sfo_d = dev(torch.from_numpy(offs)), dev(torch.from_numpy(sfo))
+    A, sA = dev(torch.from_numpy(qa[0])), dev(torch.from_numpy(ora.sf_swizzle(can)))
+    B = dev(torch.from_numpy(np.stack([q[0] for q in qbs])))
+    sB = dev(torch.from_numpy(np.concatenate([ora.sf_swizzle(q[1]) for q in qbs])))
+    gA = dev(torch.tensor([qa[2]], dtype=torch.float32))
+    gB = dev(torch.tensor([q[2] for q in qbs], dtype=torch.float32))
+    Hp = api.grouped_gemm(NV, offs_d, sfo_d, A, sA, B, sB, Mt, F, H, gsA=gA, gsB=gB, out_dtype=torch.bfloat16)
+    amax = api.amax(Hp)
+    gs = dev(torch.tensor([np.float32(np.float32(amax.item()) / np.float32(2688.0))], dtype=torch.float32))
+    codes, sf, am, Hq = api.grouped_gemm_nvfp4_out(offs_d, sfo_d, A, sA, B, sB, Mt, F, H, gs, sf_rows, gsA=gA,
+                                                   gsB=gB, four_over_six=fos, bf16_out=True)
+    assert bsq.bsq_check() == bsq.BSQ_OK
+    assert torch.equal(Hq.view(torch.int16), Hp.view(torch.int16))
+    assert am.item() == amax.item()
+    rc, rs, rg = api.quant_nvfp4(Hp, four_over_six=fos, groups=(offs_d, sfo_d, sf_rows), amax_in=amax)
+    assert bsq.bsq_check() == bsq.BSQ_OK
+    assert torch.equal(codes, rc) and torch.equal(sf, rs) and rg.item() == gs.item()
+    rows = np.arange(Mt)
+    ex = np.searchsorted(offs, rows, side="right") - 1
+    sf_row_of = rows - offs[ex] + sfo[ex]
+    y = (bits(Hp.cpu()).astype(np.uint32) << 16).view(np.float32)
+    can_out = ora.sf_unswizzle(sf.cpu().numpy(), sf_rows, F // 16)[sf_row_of]
+    check_nvfp4(y, codes.cpu().numpy(), can_out, gs.item(), four_over_six=fos, what="fused epilogue")
+    # another scale (as from an earlier step): the same properties under it
+    gs2 = dev(torch.tensor([gs.item() * 1.75], dtype=torch.float32))
+    codes2, sf2, am2, _ = api.grouped_gemm_nvfp4_out(offs_d, sfo_d, A, sA, B, sB, Mt, F, H, gs2, sf_rows, gsA=gA,
+                                                     gsB=gB, four_over_six=fos)
+    assert bsq.bsq_check() == bsq.BSQ_OK
+    assert am2.item() == amax.item()
+    can2 = ora.sf_unswizzle(sf2.cpu().numpy(), sf_rows, F // 16)[sf_row_of]
+    check_nvfp4(y, codes2.cpu().numpy(), can2, gs2.item(), four_over_six=fos, check_sg=False,
+                what="fused epilogue, earlier scale")

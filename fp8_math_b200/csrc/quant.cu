@@ -1254,6 +1254,100 @@ __global__ void __launch_bounds__(256) quant_mxfp8_col_kernel(
     }
 }
 
+// Dequantize -> transpose -> requantize of a row-wise MXFP8 tensor in
+// integer arithmetic.  The column kernel's warp tile: lane l = 4 kg + mg
+// holds rows 8 mg .. 8 mg + 7 and columns 8 kg .. 8 kg + 7 (one 8-byte code
+// load and one E8M0 byte per row: the 8 columns sit in one input block).  A
+// normal E4M3 code c (exponent field e >= 1) in a row with scale code f
+// decodes to the binary32 whose bits are (c & 0x7F) << 20 plus (f - 7) << 23
+// (exponent e + f - 7 + 127 - 127, mantissa the code's three bits), exact
+// whenever that exponent field stays in 1..254.  The block maximum is then
+// an unsigned maximum of bits, the new scale code max(field - 8, 0) (as for
+// bf16 input), and the rescaled value's bits one subtraction of the new
+// exponent: with three mantissa bits it is an E4M3 value whenever its field
+// is at least 121 (2^-6), so its code is the bits >> 20 less 120 << 3
+// (saturated at 0x7E = 448) for nearest-even and stochastic rounding alike
+// (a representable value never rounds).  A chunk holding an E4M3 subnormal
+// input, a row scale outside 7..246, or a value that lands below 2^-6 takes
+// the exact binary32 path (decode, then the general encode).
+template <bool SR>
+__global__ void __launch_bounds__(256) requant_transpose_kernel(
+    const uint8_t *__restrict__ codes_in, const uint8_t *__restrict__ sf_in, int64_t M, int64_t K, uint32_t ntile,
+    DivU32 div_mt, const __grid_constant__ PhiloxKeys keys, uint32_t stream_id, uint8_t *__restrict__ codes,
+    uint8_t *__restrict__ sf) {
+    const int lane = threadIdx.x & 31, kg = lane >> 2, mg = lane & 3;
+    const uint32_t mt_n = (uint32_t)(M >> 5);
+    const int64_t MB = M >> 5, KB = K >> 5;
+    const uint32_t nwarps = (gridDim.x * blockDim.x) >> 5;
+    for (uint32_t t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < ntile; t += nwarps) {
+        const uint32_t kt = divu32(t, div_mt), mt = t - kt * mt_n;
+        const int64_t m0 = (int64_t)mt * 32 + mg * 8, k0 = (int64_t)kt * 64 + kg * 8;
+        const bool kvalid = k0 < K;  // K % 32 == 0: a lane's 8 columns are all in or all out
+        uint32_t w[8][2], fsc[8];
+        bool rows_ok = true;
+#pragma unroll
+        for (int i = 0; i < 8; i++) {
+            const uint2 r = kvalid ? __ldg(reinterpret_cast<const uint2 *>(codes_in + (m0 + i) * K + k0)) : make_uint2(0, 0);
+            w[i][0] = r.x;
+            w[i][1] = r.y;
+            fsc[i] = kvalid ? __ldg(sf_in + sf_offset(m0 + i, k0 >> 5, KB)) : 127u;
+            rows_ok &= (fsc[i] >= 7u) & (fsc[i] <= 246u);
+        }
+#pragma unroll
+        for (int j = 0; j < 8; j++) {
+            const int64_t k = k0 + j;
+            uint32_t bits[8], sgn[8];
+            bool fast = rows_ok;
+#pragma unroll
+            for (int i = 0; i < 8; i++) {
+                const uint32_t c = (w[i][j >> 2] >> (8 * (j & 3))) & 0xFFu;
+                const uint32_t mag = c & 0x7Fu;
+                sgn[i] = c & 0x80u;
+                fast &= (mag >= 8u) | (mag == 0u);
+                bits[i] = mag >= 8u ? (mag << 20) + ((fsc[i] - 7u) << 23) : 0u;
+            }
+            if (!fast) {
+                // exact binary32 decode of every element of the chunk
+#pragma unroll
+                for (int i = 0; i < 8; i++) {
+                    const uint32_t c = (w[i][j >> 2] >> (8 * (j & 3))) & 0x7Fu;
+                    bits[i] = __float_as_uint(__fmul_rn(e4m3_to_f32(c), exp2i((int)fsc[i] - 127)));
+                }
+            }
+            uint32_t m = max(max(max(bits[0], bits[1]), max(bits[2], bits[3])),
+                             max(max(bits[4], bits[5]), max(bits[6], bits[7])));
+            m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+            m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+            const uint32_t sb = (uint32_t)max((int)(m >> 23) - 8, 0);
+            const uint32_t down = (sb - 127u) << 23;  // subtracting it divides by 2^(sb - 127)
+            uint32_t q[8];
+            bool exact = fast;
+#pragma unroll
+            for (int i = 0; i < 8; i++) {
+                const uint32_t sbits = bits[i] - down;   // meaningful when the new field is >= 121
+                exact &= (bits[i] == 0u) | ((int)(bits[i] >> 23) - (int)sb + 127 >= 121);
+                q[i] = bits[i] ? (min((sbits >> 20) - 960u, 0x7Eu) | sgn[i]) : sgn[i];
+            }
+            uint2 out;
+            if (m == 0u) {
+                out = make_uint2(0u, 0u);
+            } else if (exact) {
+                out = make_uint2(q[0] | (q[1] << 8) | (q[2] << 16) | (q[3] << 24),
+                                 q[4] | (q[5] << 8) | (q[6] << 16) | (q[7] << 24));
+            } else {
+                float v[8];
+#pragma unroll
+                for (int i = 0; i < 8; i++) v[i] = __uint_as_float(bits[i] | (sgn[i] << 24));
+                out = mx_encode8<SR, true>(v, false, sb, (uint64_t)(k * M + m0) >> 3, keys, stream_id);
+            }
+            if (kvalid) {
+                *reinterpret_cast<uint2 *>(codes + k * M + m0) = out;
+                if (mg == 0) sf[sf_offset(k, m0 >> 5, MB)] = (uint8_t)sb;
+            }
+        }
+    }
+}
+
 // Row-wise and column-wise MXFP8 of one bf16 tensor in one pass (the
 // backward pass needs dY both ways): the column kernel's warp tile (32 rows
 // x 64 columns, lane l = 4 kg + mg holding rows 8 mg .. 8 mg + 7 and columns
@@ -1914,13 +2008,13 @@ void launch_requant_transpose(const uint8_t *codes_row, const uint8_t *sf_row, i
     const uint32_t ntile = (uint32_t)((M >> 5) * ((K + 63) >> 6));
     const DivU32 dmt = divu32_for((uint32_t)(M >> 5));
     if (sr) {
-        const int grid = grid_for(ntile, 8, resident_ctas<quant_mxfp8_col_kernel<true, true>>(num_sms));
-        quant_mxfp8_col_kernel<true, true><<<grid, 256, 0, s>>>(codes_row, sf_row, M, K, K, ntile, dmt, keys,
-                                                                stream_id, codes_col, sf_col);
+        const int grid = grid_for(ntile, 8, resident_ctas<requant_transpose_kernel<true>>(num_sms));
+        requant_transpose_kernel<true><<<grid, 256, 0, s>>>(codes_row, sf_row, M, K, ntile, dmt, keys, stream_id,
+                                                            codes_col, sf_col);
     } else {
-        const int grid = grid_for(ntile, 8, resident_ctas<quant_mxfp8_col_kernel<true, false>>(num_sms));
-        quant_mxfp8_col_kernel<true, false><<<grid, 256, 0, s>>>(codes_row, sf_row, M, K, K, ntile, dmt, keys,
-                                                                 stream_id, codes_col, sf_col);
+        const int grid = grid_for(ntile, 8, resident_ctas<requant_transpose_kernel<false>>(num_sms));
+        requant_transpose_kernel<false><<<grid, 256, 0, s>>>(codes_row, sf_row, M, K, ntile, dmt, keys, stream_id,
+                                                             codes_col, sf_col);
     }
 }
 

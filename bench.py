@@ -324,7 +324,8 @@ def measure_rows(hbm, fp4_peak, fp8_peak, reps=10, only=None):
         row("f3 MXFP4 quantize SR (next row)", "X 4096x4096", lambda: api.quant_mxfp4(X1, sr=True, seed=1, out=q4),
             nbytes=M1 * K1 * (2 + 0.5 + 1 / 32))
         del X1, q1, q1s, qt, q4
-    if wants("a6 MXFP8 row quantize SR", "a6 MXFP8 column quantize SR", "a8 MXFP8 GEMM dgrad (bf16 out)", "a8 MXFP8 GEMM wgrad (fp32 out)", "a8 NVFP4 rollout GEMM (swap-AB, HBM-bound)"):
+    if wants("a6 MXFP8 row quantize SR", "a6 MXFP8 column quantize SR", "a8 MXFP8 GEMM dgrad (bf16 out)", "a8 MXFP8 GEMM wgrad (fp32 out)", "a8 NVFP4 rollout GEMM (swap-AB, HBM-bound)",
+             "f2 MXFP8 row + column SR in one pass (next row)", "f2 NVFP4 -> MXFP8 column-wise requantize SR (next row)"):
         # -- MXFP8 backward (dY 8192x14336, W 14336x4096, X 8192x4096) + NVFP4 rollout
         dY, W4, X4, A_roll = W.mxfp8_backward()
         dY, W4, X4 = dY.to(dev), W4.to(dev), X4.to(dev)
@@ -337,7 +338,18 @@ def measure_rows(hbm, fp4_peak, fp8_peak, reps=10, only=None):
         row("a6 MXFP8 column quantize SR", "dY 8192x14336 -> [14336, 8192]",
             lambda: api.quant_mxfp8(dY, colwise=True, sr=True, seed=4, stream_id=1, out=qdc),
             nbytes=M4 * N4 * (2 + 1 + 1 / 32))
+        qrc = api.quant_mxfp8_rowcol(dY, sr=True, seed=4, stream_id_row=0, stream_id_col=1)
+        row("f2 MXFP8 row + column SR in one pass (next row)", "dY 8192x14336 -> [8192, 14336] and [14336, 8192]",
+            lambda: api.quant_mxfp8_rowcol(dY, sr=True, seed=4, stream_id_row=0, stream_id_col=1, out=qrc),
+            nbytes=M4 * N4 * (2 + 2 * (1 + 1 / 32)))
+        del qrc
         qwc = api.quant_mxfp8(W4, colwise=True, sr=True, seed=4, stream_id=2)
+        qw4 = api.quant_nvfp4(W4, block_2d=True)
+        qwr = api.requant_nvfp4_mxfp8(qw4[0], qw4[1], qw4[2], sr=True, seed=4, stream_id=2)
+        row("f2 NVFP4 -> MXFP8 column-wise requantize SR (next row)", "W 14336x4096 NVFP4 16x16 -> [4096, 14336]",
+            lambda: api.requant_nvfp4_mxfp8(qw4[0], qw4[1], qw4[2], sr=True, seed=4, stream_id=2, out=qwr),
+            nbytes=N4 * K4 * (0.5 + 1 / 16 + 1 + 1 / 32))
+        del qw4, qwr
         qxc = api.quant_mxfp8(X4, colwise=True, sr=True, seed=4, stream_id=3)
         Cd = torch.empty(M4, K4, dtype=torch.bfloat16, device=dev)
         row("a8 MXFP8 GEMM dgrad (bf16 out)", "8192x4096x14336",

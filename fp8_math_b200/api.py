@@ -179,3 +179,24 @@ def grouped_gemm_nvfp4_out(row_offsets, sf_row_offsets, A, sfA, B, sfB, M_total,
                                    N, K, out_gs, four_over_six, codes, sf, am, C_out,
                                    C_out.stride(0) if C_out is not None else 0)
     return codes, sf, am, C_out
+
+
+def quant_s2f6(x, rht_mask=None, out=None):
+    """RHT (optional) + block-scaled S2F6.  Returns (codes [M, K] int8, sf [M, K/32] uint8)."""
+    M, K = x.shape
+    if out is None:
+        codes = torch.empty(M, K, dtype=torch.int8, device=x.device)
+        sf = torch.empty(M, K // 32, dtype=torch.uint8, device=x.device)
+    else:
+        codes, sf = out
+    bsq.bsq_quant_s2f6(x, M, K, _ld(x), rht_mask is not None, rht_mask or 0, codes, sf)
+    return codes, sf
+
+
+def combine_s2f6(codes, sf, token_offsets, rows, weights, rht_mask, out=None):
+    """Per token: weighted sum of its S2F6 rows, inverse RHT, bf16 [T, K]."""
+    K = codes.shape[1]
+    T = token_offsets.shape[0] - 1
+    y = torch.empty(T, K, dtype=torch.bfloat16, device=codes.device) if out is None else out
+    bsq.bsq_combine_s2f6(codes, sf, K, token_offsets, rows, weights, T, rht_mask, y, _ld(y))
+    return y

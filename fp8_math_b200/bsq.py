@@ -53,6 +53,8 @@ _SIGS = {
                                    _vp, _i64, C.c_int, _vp]),
     "bsq_grouped_gemm_nvfp4_out": (C.c_int, [C.c_int, C.c_int, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _i64,
                                              _i64, _vp, C.c_int, _vp, _vp, _vp, _vp, _i64, _vp]),
+    "bsq_quant_s2f6": (C.c_int, [_vp, _i64, _i64, _i64, C.c_int, C.c_uint16, _vp, _vp, _vp]),
+    "bsq_combine_s2f6": (C.c_int, [_vp, _vp, _i64, _vp, _vp, _vp, _i64, C.c_uint16, _vp, _i64, _vp]),
     "bsq_check": (C.c_int, [_vp]),
     "bsq_debug_timeout_probe": (C.c_int, [C.c_uint64, _vp]),
     "bsq_debug_kernel_choice": (C.c_int, [C.c_int, C.c_int]),
@@ -201,3 +203,14 @@ def bsq_grouped_gemm_nvfp4_out(fmt, G, row_offsets, sf_row_offsets, M_total, A, 
     return _check("bsq_grouped_gemm_nvfp4_out", lib().bsq_grouped_gemm_nvfp4_out(
         fmt, G, _p(row_offsets), _p(sf_row_offsets), M_total, _p(A), _p(sfA), _p(gsA), _p(B), _p(sfB), _p(gsB), N, K,
         _p(out_gs), int(four_over_six), _p(out_codes), _p(out_sf), _p(out_amax), _p(C_out), ldc, _stream(stream)))
+
+
+def bsq_quant_s2f6(x, M, K, ldx, rht_enable, rht_sign_mask, codes, sf, stream=None):
+    return _check("bsq_quant_s2f6", lib().bsq_quant_s2f6(_p(x), M, K, ldx, int(rht_enable), rht_sign_mask, _p(codes),
+                                                         _p(sf), _stream(stream)))
+
+
+def bsq_combine_s2f6(codes, sf, K, token_offsets, rows, weights, T, rht_sign_mask, out, ldo, stream=None):
+    return _check("bsq_combine_s2f6", lib().bsq_combine_s2f6(_p(codes), _p(sf), K, _p(token_offsets), _p(rows),
+                                                             _p(weights), T, rht_sign_mask, _p(out), ldo,
+                                                             _stream(stream)))

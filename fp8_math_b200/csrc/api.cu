@@ -323,6 +323,34 @@ int bsq_quant_mxfp4(const void *x, int64_t M, int64_t K, int64_t ldx, int roundi
     return launch_status();
 }
 
+int bsq_quant_s2f6(const void *x, int64_t M, int64_t K, int64_t ldx, int rht_enable, uint16_t mask, int8_t *codes,
+                   uint8_t *sf, void *stream) {
+    if (!x || !codes || !sf || M < 0 || K < 0 || K % 32 || ldx < K) return BSQ_ERR_INVALID;
+    if (!aligned16(x) || !aligned16(codes) || ldx % 8) return BSQ_ERR_ALIGN;
+    DeviceState *d;
+    if (int st = device_state(&d)) return st;
+    if (M == 0 || K == 0) return BSQ_OK;
+    bsq::launch_quant_s2f6(static_cast<const uint16_t *>(x), M, K, ldx, rht_enable != 0, mask, codes, sf, d->num_sms,
+                           static_cast<cudaStream_t>(stream));
+    return launch_status();
+}
+
+int bsq_combine_s2f6(const int8_t *codes, const uint8_t *sf, int64_t K, const int32_t *token_offsets,
+                     const int32_t *rows, const float *weights, int64_t T, uint16_t mask, void *out_bf16,
+                     int64_t ldo, void *stream) {
+    if (!codes || !sf || !token_offsets || !out_bf16 || K < 0 || K % 32 || T < 0 || ldo < K) return BSQ_ERR_INVALID;
+    if (!aligned16(codes) || !aligned16(out_bf16) || ldo % 8 || (reinterpret_cast<uintptr_t>(token_offsets) & 3u) ||
+        (reinterpret_cast<uintptr_t>(rows) & 3u) || (reinterpret_cast<uintptr_t>(weights) & 3u))
+        return BSQ_ERR_ALIGN;
+    DeviceState *d;
+    if (int st = device_state(&d)) return st;
+    if (T == 0 || K == 0) return BSQ_OK;
+    if (!rows || !weights) return BSQ_ERR_INVALID;
+    bsq::launch_combine_s2f6(codes, sf, K, token_offsets, rows, weights, T, mask, static_cast<uint16_t *>(out_bf16), ldo,
+                             d->num_sms, static_cast<cudaStream_t>(stream));
+    return launch_status();
+}
+
 int bsq_rht(const void *x, void *y, int64_t M, int64_t K, int64_t ldx, int64_t ldy, uint16_t mask, void *stream) {
     if (!x || !y || M < 0 || K < 0 || K % 16 || ldx < K || ldy < K) return BSQ_ERR_INVALID;
     if (!aligned16(x) || !aligned16(y) || ldx % 8 || ldy % 8) return BSQ_ERR_ALIGN;

@@ -1726,6 +1726,127 @@ __global__ void __launch_bounds__(256) quant_nvfp4_sr_2d_kernel(
     }
 }
 
+// ===================================================================== S2F6 (MoE combine)
+// Block-scaled S2F6 for the combine exchange: two's-complement fixed point
+// with six fraction bits (q / 64, q in [-128, 127]), one E8M0 scale 2^E per
+// 32 values with E = floor(log2 block_amax) (so block_amax / 2^E is in
+// [1, 2)), after the 16-point RHT.  One thread per group of 16 (the RHT
+// group), two lanes per block of 32; codes [M][K] int8 and scales [M][K/32]
+// row-major (a transport format, not an MMA layout).
+
+// y * 2^k for a power-of-two scaling that stays exact (or rounds once into
+// the subnormal range), for k in [-149, 254].
+BSQ_DEV float mul_pow2(float y, int k) {
+    if (k > 127) return __fmul_rn(__fmul_rn(y, 0x1p64f), exp2i(k - 64));
+    return __fmul_rn(y, exp2i(k));
+}
+
+template <bool RHT>
+__global__ void __launch_bounds__(256) quant_s2f6_kernel(const uint16_t *__restrict__ x, int64_t M, int64_t K,
+                                                         int64_t ldx, uint32_t mask, int8_t *__restrict__ codes,
+                                                         uint8_t *__restrict__ sf, RowMap map) {
+    const int64_t KG = K >> 4;
+    uint32_t sw[8];
+    rht_sign_words(mask, sw);
+    const int lpr = 1 << map.lpr_shift;
+    const int rpi = 256 >> map.lpr_shift;
+    const int sub = threadIdx.x >> map.lpr_shift, lk = threadIdx.x & (lpr - 1);
+    for (int64_t r0 = (int64_t)blockIdx.x * rpi; r0 < M; r0 += (int64_t)gridDim.x * rpi) {
+        const int64_t row = r0 + sub;
+        const bool row_ok = row < M;
+        const int64_t rr = row_ok ? row : M - 1;
+        for (int64_t g0 = 0; g0 < KG; g0 += lpr) {
+            const int64_t g = g0 + lk;
+            const bool valid = row_ok && g < KG;   // KG is even: the two lanes of a block agree
+            uint32_t w[8];
+            load_words16(x + rr * ldx + (g < KG ? g : KG - 1) * 16, w);
+            f32x2 P[8];
+            if (RHT) {
+                rht16_u_words(w, sw, P);
+                pairs_scale(P, 0.25f);
+            } else {
+                words_to_pairs(w, P);
+            }
+            float m = pairs_absmax3(P);
+            m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+            const int E = m == 0.0f ? 0 : min(max(floor_log2(m), -127), 127);
+            float v[16];
+#pragma unroll
+            for (int k = 0; k < 8; k++) f2_unpack(P[k], v[2 * k], v[2 * k + 1]);
+            uint32_t q[4];
+#pragma unroll
+            for (int k = 0; k < 4; k++) {
+                uint32_t word = 0u;
+#pragma unroll
+                for (int b = 0; b < 4; b++) {
+                    const int iq = min(max(__float2int_rn(mul_pow2(v[4 * k + b], 6 - E)), -128), 127);
+                    word |= ((uint32_t)iq & 0xFFu) << (8 * b);
+                }
+                q[k] = m == 0.0f ? 0u : word;
+            }
+            if (valid) {
+                *reinterpret_cast<uint4 *>(codes + rr * K + g * 16) = make_uint4(q[0], q[1], q[2], q[3]);
+                if ((g & 1) == 0) sf[rr * (K >> 5) + (g >> 1)] = m == 0.0f ? 0 : (uint8_t)(E + 127);
+            }
+        }
+    }
+}
+
+// The receiver: token t's output, group g of 16 = inverse RHT of the sum over
+// the token's listed rows (in list order) of weight * value, each product and
+// addition one RN operation; x = 1/4 * D * H16 * acc (butterflies of stride
+// 1, 2, 4, 8, RN), rounded once to bf16.  One thread per (token, group).
+__global__ void __launch_bounds__(256) combine_s2f6_kernel(const int8_t *__restrict__ codes,
+                                                           const uint8_t *__restrict__ sf, int64_t K,
+                                                           const int32_t *__restrict__ off,
+                                                           const int32_t *__restrict__ rows,
+                                                           const float *__restrict__ weights, int64_t T,
+                                                           uint32_t mask, uint16_t *__restrict__ out, int64_t ldo) {
+    const int64_t KG = K >> 4;
+    const int64_t n = T * KG;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t t = i / KG, g = i - t * KG;
+        float acc[16];
+#pragma unroll
+        for (int k = 0; k < 16; k++) acc[k] = 0.0f;
+        const int32_t j1 = __ldg(off + t + 1);
+        for (int32_t j = __ldg(off + t); j < j1; j++) {
+            const int64_t r = __ldg(rows + j);
+            const float wgt = __ldg(weights + j);
+            const uint4 cw = __ldg(reinterpret_cast<const uint4 *>(codes + r * K + g * 16));
+            const float scale = exp2i((int)__ldg(sf + r * (K >> 5) + (g >> 1)) - 133);
+            const uint32_t c4[4] = {cw.x, cw.y, cw.z, cw.w};
+#pragma unroll
+            for (int k = 0; k < 16; k++) {
+                const float v = __fmul_rn((float)(int8_t)(c4[k >> 2] >> (8 * (k & 3))), scale);
+                acc[k] = __fadd_rn(acc[k], __fmul_rn(wgt, v));
+            }
+        }
+#pragma unroll
+        for (int h = 1; h < 16; h <<= 1)
+#pragma unroll
+            for (int base = 0; base < 16; base += 2 * h)
+#pragma unroll
+                for (int k = base; k < base + h; k++) {
+                    const float a = acc[k], b = acc[k + h];
+                    acc[k] = __fadd_rn(a, b);
+                    acc[k + h] = __fsub_rn(a, b);
+                }
+        uint32_t o[8];
+#pragma unroll
+        for (int k = 0; k < 8; k++) {
+            float y0 = __fmul_rn(acc[2 * k], 0.25f), y1 = __fmul_rn(acc[2 * k + 1], 0.25f);
+            if ((mask >> (2 * k)) & 1u) y0 = -y0;
+            if ((mask >> (2 * k + 1)) & 1u) y1 = -y1;
+            __nv_bfloat162 hb = __floats2bfloat162_rn(y0, y1);
+            o[k] = *reinterpret_cast<uint32_t *>(&hb);
+        }
+        uint4 *dst = reinterpret_cast<uint4 *>(out + t * ldo + g * 16);
+        dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+        dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+    }
+}
+
 // ===================================================================== RHT
 __global__ void __launch_bounds__(256) rht_kernel(const uint16_t *__restrict__ x, uint16_t *y, int64_t M,
                                                   int64_t K, int64_t ldx, int64_t ldy, uint32_t mask, RowMap map) {
@@ -2089,6 +2210,21 @@ void launch_quant_nvfp4_sr(const uint16_t *x, int64_t M, int64_t K, int64_t ldx,
     if (rht) { if (row_index) BSQ_NVSR(true, true); else BSQ_NVSR(true, false); }
     else { if (row_index) BSQ_NVSR(false, true); else BSQ_NVSR(false, false); }
 #undef BSQ_NVSR
+}
+
+void launch_quant_s2f6(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, bool rht, uint32_t mask, int8_t *codes,
+                       uint8_t *sf, int num_sms, cudaStream_t s) {
+    RowMap map{lpr_shift_for(K >> 4)};
+    const int grid = grid_for(M, 256 >> map.lpr_shift, num_sms * 8);
+    if (rht) quant_s2f6_kernel<true><<<grid, 256, 0, s>>>(x, M, K, ldx, mask, codes, sf, map);
+    else quant_s2f6_kernel<false><<<grid, 256, 0, s>>>(x, M, K, ldx, mask, codes, sf, map);
+}
+
+void launch_combine_s2f6(const int8_t *codes, const uint8_t *sf, int64_t K, const int32_t *off, const int32_t *rows,
+                         const float *weights, int64_t T, uint32_t mask, uint16_t *out, int64_t ldo, int num_sms,
+                         cudaStream_t s) {
+    const int grid = grid_for(T * (K >> 4), 256, num_sms * 8);
+    combine_s2f6_kernel<<<grid, 256, 0, s>>>(codes, sf, K, off, rows, weights, T, mask, out, ldo);
 }
 
 void launch_rht(const uint16_t *x, uint16_t *y, int64_t M, int64_t K, int64_t ldx, int64_t ldy, uint32_t mask,

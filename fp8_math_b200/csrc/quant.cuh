@@ -56,6 +56,11 @@ void launch_quant_nvfp4_sr(const uint16_t *x, int64_t M, int64_t K, int64_t ldx,
 void launch_requant_transpose(const uint8_t *codes_row, const uint8_t *sf_row, int64_t M, int64_t K, bool sr,
                               uint64_t seed, uint32_t stream_id, uint8_t *codes_col, uint8_t *sf_col,
                               int num_sms, cudaStream_t s);
+void launch_quant_s2f6(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, bool rht, uint32_t mask, int8_t *codes,
+                       uint8_t *sf, int num_sms, cudaStream_t s);
+void launch_combine_s2f6(const int8_t *codes, const uint8_t *sf, int64_t K, const int32_t *off, const int32_t *rows,
+                         const float *weights, int64_t T, uint32_t mask, uint16_t *out, int64_t ldo, int num_sms,
+                         cudaStream_t s);
 void launch_rht(const uint16_t *x, uint16_t *y, int64_t M, int64_t K, int64_t ldx, int64_t ldy, uint32_t mask,
                 int num_sms, cudaStream_t s);
 

@@ -240,6 +240,36 @@ BSQ_API int bsq_quant_mxfp4(const void *x_bf16, int64_t M, int64_t K, int64_t ld
 BSQ_API int bsq_rht(const void *x_bf16, void *y_bf16, int64_t M, int64_t K, int64_t ldx, int64_t ldy,
             uint16_t rht_sign_mask, void *stream);
 
+/* Block-scaled S2F6 for the MoE combine exchange ("Thinking Machines ...",
+ * section "Why communication became the next bottleneck": expert outputs
+ * are rotated by a random Hadamard transform and sent in block-scaled S2F6,
+ * an 8-bit fixed-point format, at 8.25 bits per value).  S2F6 is read here
+ * as two's-complement fixed point with six fraction bits: code q in
+ * [-128, 127] stands for q / 64.  Per row, after the 16-point RHT along K
+ * when rht_enable != 0 (as bsq_rht, in fp32): each block of 32 has one
+ * E8M0 scale code E + 127 with E = clamp(floor(log2 block_amax), -127, 127)
+ * (an all-zero block: code 0 and zero codes), and q = nearest-even integer
+ * of x * 2^(6 - E), clamped to [-128, 127].  codes [M][K] int8 (row stride
+ * K), sf [M][K/32] bytes row-major.  K % 32 == 0; x and codes 16-byte
+ * aligned, ldx % 8 == 0. */
+BSQ_API int bsq_quant_s2f6(const void *x_bf16, int64_t M, int64_t K, int64_t ldx, int rht_enable,
+                           uint16_t rht_sign_mask, int8_t *codes_dev, uint8_t *sf_dev, void *stream);
+
+/* The S2F6 receiver (same page and section: the receiver reconstructs and
+ * combines the values, then reverses the transform).  For token t, the rows
+ * rows_dev[token_offsets_dev[t] .. token_offsets_dev[t+1]) of the S2F6
+ * matrix (codes [R][K], sf [R][K/32] as bsq_quant_s2f6 writes them) are
+ * decoded (q / 64 * 2^E, exact) and summed in list order with the weights
+ * weights_dev[j] (fp32: one rounding per product and per addition); each
+ * group of 16 of the sum is then rotated back, x = 1/4 * D * H16 * acc (the
+ * inverse of bsq_rht's transform with the same sign mask), and rounded to
+ * bf16: out [T][K] with leading dimension ldo.  token_offsets_dev is int32
+ * [T+1], rows_dev int32 and weights_dev fp32 of its last value's length.
+ * K % 32 == 0; codes and out 16-byte aligned, ldo % 8 == 0. */
+BSQ_API int bsq_combine_s2f6(const int8_t *codes_dev, const uint8_t *sf_dev, int64_t K,
+                             const int32_t *token_offsets_dev, const int32_t *rows_dev, const float *weights_dev,
+                             int64_t T, uint16_t rht_sign_mask, void *out_bf16_dev, int64_t ldo, void *stream);
+
 /* Dequantize -> transpose -> requantize ("Thinking Machines ...", section
  * "A precision choice for each stage"): the row-wise MXFP8 tensor (codes
  * [M][K], swizzled sf for M x K/32) is decoded exactly (E4M3 x 2^E, fp32),

@@ -733,6 +733,110 @@ int ora_requant_nvfp4_mxfp8_rows(const uint8_t *codes, const uint8_t *sf, float 
 }
 
 /* ------------------------------------------------------------------------ */
+/* S2F6 combine compression -- [TML] "Why communication became the next     */
+/* bottleneck": the combined MoE outputs are rotated by a random Hadamard   */
+/* transform, sent in block-scaled S2F6 ("an 8-bit fixed-point format") at  */
+/* 8.25 bits per value, and the receiver reconstructs and combines them,     */
+/* then reverses the transform.                                               */
+/* R34: S2F6 is two's-complement fixed point with two integer bits (the     */
+/* sign among them) and six fraction bits: code q in [-128, 127], value     */
+/* q / 64.  R35: 32 consecutive values share one E8M0 scale (8 + 8/32 =     */
+/* 8.25 bits): E = floor(log2 block_amax) clamped to [-127, 127], so that   */
+/* block_amax / 2^E lies in [1, 2); q = nearest-even integer of            */
+/* x * 2^(6 - E) (exact scaling), clamped to [-128, 127]; an all-zero block  */
+/* has scale code 0 and zero codes.  The transform is the 16-point RHT of    */
+/* R14 applied first (binary32).                                             */
+/* ------------------------------------------------------------------------ */
+
+static int8_t s2f6_round(float s)
+{
+    float r = rintf(s); /* the default rounding mode: nearest, ties to even */
+    if (r > 127.0f)
+        r = 127.0f;
+    if (r < -128.0f)
+        r = -128.0f;
+    return (int8_t)r;
+}
+
+int ora_quant_s2f6(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, int rht, uint16_t mask,
+                   int8_t *codes, uint8_t *sf)
+{
+    if (K % 32)
+        return 1;
+    float *row = (float *)malloc(sizeof(float) * (size_t)K);
+    for (int64_t m = 0; m < M; m++) {
+        load_row(x, ldx, m, K, rht, mask, row);
+        for (int64_t b = 0; b < K / 32; b++) {
+            float bamax = 0.0f;
+            for (int i = 0; i < 32; i++)
+                if (fabsf(row[b * 32 + i]) > bamax)
+                    bamax = fabsf(row[b * 32 + i]);
+            if (bamax == 0.0f) {
+                sf[m * (K / 32) + b] = 0;
+                for (int i = 0; i < 32; i++)
+                    codes[m * K + b * 32 + i] = 0;
+                continue;
+            }
+            int e2;
+            frexpf(bamax, &e2);
+            int E = e2 - 1;
+            if (E < -127)
+                E = -127;
+            if (E > 127)
+                E = 127;
+            sf[m * (K / 32) + b] = (uint8_t)(E + 127);
+            for (int i = 0; i < 32; i++)
+                codes[m * K + b * 32 + i] = s2f6_round(ldexpf(row[b * 32 + i], 6 - E));
+        }
+    }
+    free(row);
+    return 0;
+}
+
+/* R36, the receiver: token t's output is the sum, over the rows listed for
+ * it (rows[off[t]] .. rows[off[t+1]-1], in that order), of weight * value
+ * (binary32: each value q / 64 * 2^E is exact, each product and each
+ * addition one RN operation), then the inverse transform of each group of
+ * 16: x = 1/4 * D * H16 * acc (butterflies of stride 1, 2, 4, 8, RN; the
+ * quarter and the signs exact), rounded once to bf16 (nearest-even). */
+int ora_combine_s2f6(const int8_t *codes, const uint8_t *sf, int64_t K, const int32_t *off,
+                     const int32_t *rows, const float *weights, int64_t T, uint16_t mask, uint16_t *out)
+{
+    if (K % 32)
+        return 1;
+    float *acc = (float *)malloc(sizeof(float) * (size_t)K);
+    for (int64_t t = 0; t < T; t++) {
+        for (int64_t k = 0; k < K; k++)
+            acc[k] = 0.0f;
+        for (int32_t j = off[t]; j < off[t + 1]; j++) {
+            const int64_t r = rows[j];
+            for (int64_t k = 0; k < K; k++) {
+                float v = ldexpf((float)codes[r * K + k], (int)sf[r * (K / 32) + k / 32] - 127 - 6);
+                acc[k] = acc[k] + weights[j] * v;
+            }
+        }
+        for (int64_t g = 0; g < K; g += 16) {
+            float u[16];
+            for (int i = 0; i < 16; i++)
+                u[i] = acc[g + i];
+            for (int h = 1; h < 16; h <<= 1)
+                for (int base = 0; base < 16; base += 2 * h)
+                    for (int i = base; i < base + h; i++) {
+                        float a = u[i], b = u[i + h];
+                        u[i] = a + b;
+                        u[i + h] = a - b;
+                    }
+            for (int i = 0; i < 16; i++) {
+                float y = 0.25f * u[i];
+                out[t * K + g + i] = ora_f32_to_bf16(((mask >> i) & 1) ? -y : y);
+            }
+        }
+    }
+    free(acc);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
 /* Scale-factor layout for the tensor-core MMA -- [MX] "Hardware and         */
 /* kernels": a block-scaled GEMM needs a particular scale-factor memory      */
 /* layout; the pages do not give it.  R23 (Blackwell block-scaled MMA        */

@@ -38,6 +38,7 @@ def build(force: bool = False) -> str:
 
 
 _u8p = np.ctypeslib.ndpointer(np.uint8, flags="C_CONTIGUOUS")
+_i8p = np.ctypeslib.ndpointer(np.int8, flags="C_CONTIGUOUS")
 _u16p = np.ctypeslib.ndpointer(np.uint16, flags="C_CONTIGUOUS")
 _i32p = np.ctypeslib.ndpointer(np.int32, flags="C_CONTIGUOUS")
 _i64p = np.ctypeslib.ndpointer(np.int64, flags="C_CONTIGUOUS")
@@ -92,6 +93,8 @@ def lib():
                                                          C.c_uint32, _i64, _i64, _u8p, _u8p]),
                 "ora_requant_nvfp4_mxfp8_rows": (C.c_int, [_u8p, _u8p, C.c_float, _i64, _i64, C.c_int, C.c_uint64,
                                                            C.c_uint32, _i64, _i64, _u8p, _u8p]),
+                "ora_quant_s2f6": (C.c_int, [_u16p, _i64, _i64, _i64, C.c_int, C.c_uint16, _i8p, _u8p]),
+                "ora_combine_s2f6": (C.c_int, [_i8p, _u8p, _i64, _i32p, _i32p, _f32p, _i64, C.c_uint16, _u16p]),
                 "ora_sf_swizzled_bytes": (_i64, [_i64, _i64]),
                 "ora_sf_offset": (_i64, [_i64, _i64, _i64]),
                 "ora_sf_swizzle": (None, [_u8p, _i64, _i64, _u8p]),
@@ -383,6 +386,45 @@ def requant_nvfp4_mxfp8(codes, sf, s_g, sr=True, seed=0, stream_id=1, threads=1)
 
     _run_bands(band, C, threads)
     return cc, sc
+
+
+def quant_s2f6(x, rht_mask=None, threads=1):
+    """RHT (optional) + block-scaled S2F6 (ora_quant_s2f6).  Returns (codes
+    [M, K] int8, sf [M, K/32] E8M0 codes)."""
+    x = _c(x, np.uint16)
+    M, K = x.shape
+    codes = np.zeros((M, K), np.int8)
+    sf = np.zeros((M, K // 32), np.uint8)
+    L = lib()
+
+    def band(r0, r1):
+        if L.ora_quant_s2f6(x[r0:r1], r1 - r0, K, K, int(rht_mask is not None), int(rht_mask or 0), codes[r0:r1],
+                            sf[r0:r1]):
+            raise ValueError("K must be a multiple of 32")
+
+    _run_bands(band, M, threads)
+    return codes, sf
+
+
+def combine_s2f6(codes, sf, token_offsets, rows, weights, mask, threads=1):
+    """Weighted sum per token of S2F6 rows, inverse RHT, bf16 (ora_combine_s2f6).
+    Returns bf16 bits [T, K]; threads > 1 splits the tokens into bands."""
+    codes = _c(codes, np.int8)
+    sf = _c(sf, np.uint8)
+    off = _c(token_offsets, np.int32)
+    rows = _c(rows, np.int32)
+    weights = _c(weights, np.float32)
+    T, K = off.shape[0] - 1, codes.shape[1]
+    out = np.zeros((T, K), np.uint16)
+    L = lib()
+
+    def band(t0, t1):
+        if L.ora_combine_s2f6(codes, sf, K, np.ascontiguousarray(off[t0:t1 + 1]), rows, weights, t1 - t0, int(mask),
+                              out[t0:t1]):
+            raise ValueError("K must be a multiple of 32")
+
+    _run_bands(band, T, threads)
+    return out
 
 
 # ---------------------------------------------------------------- layout

@@ -913,6 +913,12 @@ def test_threaded_oracle_equals_serial_byte_for_byte(ora):
     same(ora.quant_mxfp4(xa, sr=True, seed=3, threads=T), ora.quant_mxfp4(xa, sr=True, seed=3))
     cm, sm = ora.quant_mxfp8(xa, sr=True, seed=1)
     same(ora.requant_transpose(cm, sm, seed=1, threads=T), ora.requant_transpose(cm, sm, seed=1))
+    same(ora.quant_s2f6(xa, rht_mask=mask, threads=T), ora.quant_s2f6(xa, rht_mask=mask))
+    cs, ss = ora.quant_s2f6(xa)
+    off = np.array([0, 3, 3, 10, 288], np.int32)
+    rows = np.random.default_rng(3).permutation(288).astype(np.int32)
+    wts = np.random.default_rng(4).random(288).astype(np.float32)
+    same([ora.combine_s2f6(cs, ss, off, rows, wts, mask, threads=T)], [ora.combine_s2f6(cs, ss, off, rows, wts, mask)])
     q = ora.quant_nvfp4(xa)
     same([ora.dequant(ora.NVFP4, *q, threads=T)], [ora.dequant(ora.NVFP4, *q)])
 
@@ -988,3 +994,93 @@ def test_requant_nvfp4_mxfp8_rne_nearest_and_sr_unbiased(ora):
     ok = (scaled <= 448).reshape(128, 64)          # values past 448 saturate: no unbiasedness there
     assert ok.mean() > 0.9
     assert (np.abs(mean - deq)[ok] <= 5 * se[ok] + 1e-12).all()
+
+
+# --------------------------------------------------------------------- S2F6 combine compression
+def test_s2f6_bits_per_value_match_pages(ora):
+    """TML page "Why communication became the next bottleneck": 8.25 bits
+    per value for block-scaled S2F6 (8-bit codes, one 8-bit scale per 32)."""
+    rows = {r[0]: r for r in golden_rows("bits_per_value.txt")}
+    x = W.bf16_bits(W.nvfp4_linear_small(M=64, N=16, K=256)[0])
+    c, s = ora.quant_s2f6(x)
+    assert (c.nbytes + s.nbytes) * 8 / x.size == float(rows["s2f6"][4])
+
+
+def test_s2f6_scale_rule_and_nearest_even_codes(ora):
+    """R34/R35: E = floor(log2 block_amax) (math.frexp, a library routine),
+    every code is numpy's nearest-even integer of x * 2^(6 - E), clamped to
+    the int8 range."""
+    x = W.bf16_bits(W.mxfp8_requant(M=32, K=256, seed=8))
+    c, s = ora.quant_s2f6(x)
+    xf = (x.astype(np.uint32) << 16).view(np.float32).astype(np.float64).reshape(32, 8, 32)
+    bamax = np.abs(xf).max(-1)
+    for i in range(32):
+        for j in range(8):
+            assert int(s[i, j]) == math.frexp(float(bamax[i, j]))[1] - 1 + 127
+    want = np.clip(np.rint(xf * (2.0 ** (6 - (s.astype(np.float64) - 127)))[..., None]), -128, 127)
+    assert np.array_equal(c.reshape(32, 8, 32).astype(np.float64), want)
+
+
+def test_s2f6_round_trip_on_representable_blocks(ora):
+    """Blocks built as q / 64 * 2^E (q in the int8 range, one |q| >= 64 per
+    block so that E is the block's exponent) come back exactly."""
+    rng = np.random.default_rng(4)
+    R, K = 16, 128
+    E = rng.integers(-20, 20, size=(R, K // 32))
+    q = rng.integers(-127, 128, size=(R, K))              # -128 (= -2) would lift the block exponent
+    for r in range(R):
+        for b in range(K // 32):
+            q[r, b * 32 + rng.integers(0, 32)] = rng.choice([64, 100, 127, -127, -90])
+    v = q / 64.0 * np.repeat(2.0 ** E, 32, axis=1)
+    xb = torch.from_numpy(v.astype(np.float32)).to(torch.bfloat16)
+    assert np.array_equal(xb.float().numpy().astype(np.float64), v)
+    c, s = ora.quant_s2f6(W.bf16_bits(xb))
+    assert np.array_equal(c, q.astype(np.int8)) and np.array_equal(s, (E + 127).astype(np.uint8))
+
+
+def test_s2f6_combine_undoes_the_rotation(ora):
+    """The receiver reverses the transform (TML page): a tensor whose RHT
+    output is exactly representable in S2F6 comes back bit for bit after
+    quantize (with the RHT) and combine (one row per token, weight 1)."""
+    from scipy.linalg import hadamard
+    rng = np.random.default_rng(6)
+    mask = 0xA53C
+    T, K = 8, 64
+    D = np.array([-1.0 if (mask >> i) & 1 else 1.0 for i in range(16)])
+    H = hadamard(16).astype(np.float64)
+    y = rng.integers(-16, 17, size=(T, K)) / 4.0             # the rotated values, small quarters
+    y[:, ::32] = 4.0                                        # each block's exponent fixed at 2
+    x = np.zeros_like(y)
+    for g in range(0, K, 16):
+        x[:, g:g + 16] = (0.25 * (H @ y[:, g:g + 16].T)).T * D   # x = 1/4 D H y
+    xb = torch.from_numpy(x.astype(np.float32)).to(torch.bfloat16)
+    assert np.array_equal(xb.float().numpy().astype(np.float64), x)
+    c, s = ora.quant_s2f6(W.bf16_bits(xb), rht_mask=mask)
+    off = np.arange(T + 1, dtype=np.int32)
+    out = ora.combine_s2f6(c, s, off, np.arange(T, dtype=np.int32), np.ones(T, np.float32), mask)
+    assert np.array_equal(out, W.bf16_bits(xb))
+
+
+def test_s2f6_combine_weighted_sum(ora):
+    """Each token sums its rows times their weights, then the inverse
+    rotation 1/4 D H (scipy's Hadamard matrix, binary64): the bf16 result is
+    that sum to within one bf16 rounding plus binary32 summation error."""
+    from scipy.linalg import hadamard
+    rng = np.random.default_rng(7)
+    mask = 0x1E2D
+    R, K = 6, 96
+    c = rng.integers(-128, 128, size=(R, K)).astype(np.int8)
+    s = rng.integers(120, 130, size=(R, K // 32)).astype(np.uint8)
+    off = np.array([0, 2, 3, 6], np.int32)
+    rows = np.array([4, 1, 0, 5, 2, 3], np.int32)
+    w = rng.random(6).astype(np.float32)
+    out = ora.combine_s2f6(c, s, off, rows, w, mask)
+    got = (out.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    v = c.astype(np.float64) / 64 * np.repeat(2.0 ** (s.astype(np.float64) - 127), 32, axis=1)
+    D = np.array([-1.0 if (mask >> i) & 1 else 1.0 for i in range(16)])
+    H = hadamard(16).astype(np.float64)
+    for t in range(3):
+        acc = sum(float(w[j]) * v[rows[j]] for j in range(off[t], off[t + 1]))
+        want = np.concatenate([0.25 * D * (H @ acc[g:g + 16]) for g in range(0, K, 16)])
+        scale = np.concatenate([0.25 * (np.abs(H) @ np.abs(acc[g:g + 16])) for g in range(0, K, 16)])
+        assert (np.abs(got[t] - want) <= 2.0 ** -8 * np.abs(want) + 1e-6 * scale + 1e-30).all()

@@ -55,6 +55,9 @@ _SIGS = {
                                              _i64, _vp, C.c_int, _vp, _vp, _vp, _vp, _i64, _vp]),
     "bsq_quant_s2f6": (C.c_int, [_vp, _i64, _i64, _i64, C.c_int, C.c_uint16, _vp, _vp, _vp]),
     "bsq_combine_s2f6": (C.c_int, [_vp, _vp, _i64, _vp, _vp, _vp, _i64, C.c_uint16, _vp, _i64, _vp]),
+    "bsq_gather_rows": (C.c_int, [_vp, _i64, _vp, _i64, _vp, _vp]),
+    "bsq_sf_to_rows": (C.c_int, [_vp, _i64, _i64, _vp, _vp]),
+    "bsq_sf_from_rows": (C.c_int, [_vp, _i64, _i64, C.c_int, _vp, _vp, _vp, _vp]),
     "bsq_check": (C.c_int, [_vp]),
     "bsq_debug_timeout_probe": (C.c_int, [C.c_uint64, _vp]),
     "bsq_debug_kernel_choice": (C.c_int, [C.c_int, C.c_int]),
@@ -214,3 +217,17 @@ def bsq_combine_s2f6(codes, sf, K, token_offsets, rows, weights, T, rht_sign_mas
     return _check("bsq_combine_s2f6", lib().bsq_combine_s2f6(_p(codes), _p(sf), K, _p(token_offsets), _p(rows),
                                                              _p(weights), T, rht_sign_mask, _p(out), ldo,
                                                              _stream(stream)))
+
+
+def bsq_gather_rows(src, row_bytes, index, R, dst, stream=None):
+    return _check("bsq_gather_rows", lib().bsq_gather_rows(_p(src), row_bytes, _p(index), R, _p(dst),
+                                                           _stream(stream)))
+
+
+def bsq_sf_to_rows(sf, rows, nblk, out, stream=None):
+    return _check("bsq_sf_to_rows", lib().bsq_sf_to_rows(_p(sf), rows, nblk, _p(out), _stream(stream)))
+
+
+def bsq_sf_from_rows(rows_in, rows, nblk, G, row_offsets, sf_row_offsets, sf, stream=None):
+    return _check("bsq_sf_from_rows", lib().bsq_sf_from_rows(_p(rows_in), rows, nblk, G, _p(row_offsets),
+                                                             _p(sf_row_offsets), _p(sf), _stream(stream)))

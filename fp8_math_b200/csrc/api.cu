@@ -351,6 +351,35 @@ int bsq_combine_s2f6(const int8_t *codes, const uint8_t *sf, int64_t K, const in
     return launch_status();
 }
 
+int bsq_gather_rows(const void *src, int64_t row_bytes, const int32_t *index, int64_t R, void *dst, void *stream) {
+    if (!src || !dst || R < 0 || row_bytes < 0 || row_bytes % 16 || (R > 0 && !index)) return BSQ_ERR_INVALID;
+    if (!aligned16(src) || !aligned16(dst) || (reinterpret_cast<uintptr_t>(index) & 3u)) return BSQ_ERR_ALIGN;
+    DeviceState *d;
+    if (int st = device_state(&d)) return st;
+    if (R == 0 || row_bytes == 0) return BSQ_OK;
+    bsq::launch_gather_rows(src, row_bytes, index, R, dst, d->num_sms, static_cast<cudaStream_t>(stream));
+    return launch_status();
+}
+
+int bsq_sf_to_rows(const uint8_t *sf, int64_t rows, int64_t nblk, uint8_t *out, void *stream) {
+    if (!sf || !out || rows < 0 || nblk < 0) return BSQ_ERR_INVALID;
+    DeviceState *d;
+    if (int st = device_state(&d)) return st;
+    if (rows == 0 || nblk == 0) return BSQ_OK;
+    bsq::launch_sf_to_rows(sf, rows, nblk, out, d->num_sms, static_cast<cudaStream_t>(stream));
+    return launch_status();
+}
+
+int bsq_sf_from_rows(const uint8_t *in, int64_t rows, int64_t nblk, int G, const int32_t *row_off,
+                     const int32_t *sf_row_off, uint8_t *sf, void *stream) {
+    if (!in || !sf || rows < 0 || nblk < 0 || G < 0 || (G > 0 && (!row_off || !sf_row_off))) return BSQ_ERR_INVALID;
+    DeviceState *d;
+    if (int st = device_state(&d)) return st;
+    if (rows == 0 || nblk == 0) return BSQ_OK;
+    bsq::launch_sf_from_rows(in, rows, nblk, G, row_off, sf_row_off, sf, d->num_sms, static_cast<cudaStream_t>(stream));
+    return launch_status();
+}
+
 int bsq_rht(const void *x, void *y, int64_t M, int64_t K, int64_t ldx, int64_t ldy, uint16_t mask, void *stream) {
     if (!x || !y || M < 0 || K < 0 || K % 16 || ldx < K || ldy < K) return BSQ_ERR_INVALID;
     if (!aligned16(x) || !aligned16(y) || ldx % 8 || ldy % 8) return BSQ_ERR_ALIGN;

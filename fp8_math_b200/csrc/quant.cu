@@ -1847,6 +1847,44 @@ __global__ void __launch_bounds__(256) combine_s2f6_kernel(const int8_t *__restr
     }
 }
 
+// ===================================================================== exchange layouts
+// Byte-moving kernels for the expert-parallel exchange: rows gathered by an
+// index (16-byte pieces), and scale factors between the MMA's swizzled
+// layout and plain rows of nblk bytes (the transport form).
+__global__ void __launch_bounds__(256) gather_rows_kernel(const uint4 *__restrict__ src, int64_t row_vec,
+                                                          const int32_t *__restrict__ index, int64_t R,
+                                                          uint4 *__restrict__ dst) {
+    const int64_t n = R * row_vec;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t r = i / row_vec, v = i - r * row_vec;
+        dst[i] = __ldg(src + (int64_t)__ldg(index + r) * row_vec + v);
+    }
+}
+
+__global__ void __launch_bounds__(256) sf_to_rows_kernel(const uint8_t *__restrict__ sf, int64_t rows, int64_t nblk,
+                                                         uint8_t *__restrict__ out) {
+    const int64_t n = rows * nblk;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t r = i / nblk, b = i - r * nblk;
+        out[i] = __ldg(sf + sf_offset(r, b, nblk));
+    }
+}
+
+// Rows of scale bytes into the swizzled layout; with groups, output row r
+// of group e goes to SF row r - row_off[e] + sf_row_off[e] (rows outside
+// every group are skipped).
+__global__ void __launch_bounds__(256) sf_from_rows_kernel(const uint8_t *__restrict__ in, int64_t rows, int64_t nblk,
+                                                           int G, const int32_t *__restrict__ row_off,
+                                                           const int32_t *__restrict__ sf_off,
+                                                           uint8_t *__restrict__ sf) {
+    const int64_t n = rows * nblk;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t r = i / nblk, b = i - r * nblk;
+        const int64_t sr = G > 0 ? grouped_sf_row(r, G, row_off, sf_off) : r;
+        if (sr >= 0) sf[sf_offset(sr, b, nblk)] = __ldg(in + i);
+    }
+}
+
 // ===================================================================== RHT
 __global__ void __launch_bounds__(256) rht_kernel(const uint16_t *__restrict__ x, uint16_t *y, int64_t M,
                                                   int64_t K, int64_t ldx, int64_t ldy, uint32_t mask, RowMap map) {
@@ -2225,6 +2263,22 @@ void launch_combine_s2f6(const int8_t *codes, const uint8_t *sf, int64_t K, cons
                          cudaStream_t s) {
     const int grid = grid_for(T * (K >> 4), 256, num_sms * 8);
     combine_s2f6_kernel<<<grid, 256, 0, s>>>(codes, sf, K, off, rows, weights, T, mask, out, ldo);
+}
+
+void launch_gather_rows(const void *src, int64_t row_bytes, const int32_t *index, int64_t R, void *dst, int num_sms,
+                        cudaStream_t s) {
+    const int64_t vec = row_bytes / 16;
+    gather_rows_kernel<<<grid_for(R * vec, 256, num_sms * 8), 256, 0, s>>>(static_cast<const uint4 *>(src), vec, index,
+                                                                          R, static_cast<uint4 *>(dst));
+}
+
+void launch_sf_to_rows(const uint8_t *sf, int64_t rows, int64_t nblk, uint8_t *out, int num_sms, cudaStream_t s) {
+    sf_to_rows_kernel<<<grid_for(rows * nblk, 256, num_sms * 8), 256, 0, s>>>(sf, rows, nblk, out);
+}
+
+void launch_sf_from_rows(const uint8_t *in, int64_t rows, int64_t nblk, int G, const int32_t *row_off,
+                         const int32_t *sf_off, uint8_t *sf, int num_sms, cudaStream_t s) {
+    sf_from_rows_kernel<<<grid_for(rows * nblk, 256, num_sms * 8), 256, 0, s>>>(in, rows, nblk, G, row_off, sf_off, sf);
 }
 
 void launch_rht(const uint16_t *x, uint16_t *y, int64_t M, int64_t K, int64_t ldx, int64_t ldy, uint32_t mask,

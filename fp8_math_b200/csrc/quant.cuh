@@ -61,6 +61,11 @@ void launch_quant_s2f6(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, boo
 void launch_combine_s2f6(const int8_t *codes, const uint8_t *sf, int64_t K, const int32_t *off, const int32_t *rows,
                          const float *weights, int64_t T, uint32_t mask, uint16_t *out, int64_t ldo, int num_sms,
                          cudaStream_t s);
+void launch_gather_rows(const void *src, int64_t row_bytes, const int32_t *index, int64_t R, void *dst, int num_sms,
+                        cudaStream_t s);
+void launch_sf_to_rows(const uint8_t *sf, int64_t rows, int64_t nblk, uint8_t *out, int num_sms, cudaStream_t s);
+void launch_sf_from_rows(const uint8_t *in, int64_t rows, int64_t nblk, int G, const int32_t *row_off,
+                         const int32_t *sf_off, uint8_t *sf, int num_sms, cudaStream_t s);
 void launch_rht(const uint16_t *x, uint16_t *y, int64_t M, int64_t K, int64_t ldx, int64_t ldy, uint32_t mask,
                 int num_sms, cudaStream_t s);
 

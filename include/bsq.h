@@ -270,6 +270,25 @@ BSQ_API int bsq_combine_s2f6(const int8_t *codes_dev, const uint8_t *sf_dev, int
                              const int32_t *token_offsets_dev, const int32_t *rows_dev, const float *weights_dev,
                              int64_t T, uint16_t rht_sign_mask, void *out_bf16_dev, int64_t ldo, void *stream);
 
+/* Byte movers for the expert-parallel exchange (the pages describe the
+ * dispatch of NVFP4 rows to the GPUs holding the experts and the combine
+ * back, "Thinking Machines ...", section "Why communication became the next
+ * bottleneck"; these calls do no arithmetic).
+ * bsq_gather_rows: dst row r = src row index_dev[r], rows of row_bytes
+ * bytes (a multiple of 16); src and dst 16-byte aligned.
+ * bsq_sf_to_rows: a swizzled scale-factor buffer (rows x nblk blocks, as
+ * the quantizers write it) to plain rows of nblk bytes.
+ * bsq_sf_from_rows: plain rows back into the swizzled layout; with G > 0,
+ * row r of group e (device int32 offsets as for bsq_quant_nvfp4) goes to SF
+ * row r - row_offsets[e] + sf_row_offsets[e] (the grouped GEMM's layout).
+ * Padding bytes of the swizzled buffer are not written. */
+BSQ_API int bsq_gather_rows(const void *src_dev, int64_t row_bytes, const int32_t *index_dev, int64_t R,
+                            void *dst_dev, void *stream);
+BSQ_API int bsq_sf_to_rows(const uint8_t *sf_dev, int64_t rows, int64_t nblk, uint8_t *rows_out_dev, void *stream);
+BSQ_API int bsq_sf_from_rows(const uint8_t *rows_in_dev, int64_t rows, int64_t nblk, int G,
+                             const int32_t *row_offsets_dev, const int32_t *sf_row_offsets_dev, uint8_t *sf_dev,
+                             void *stream);
+
 /* Dequantize -> transpose -> requantize ("Thinking Machines ...", section
  * "A precision choice for each stage"): the row-wise MXFP8 tensor (codes
  * [M][K], swizzled sf for M x K/32) is decoded exactly (E4M3 x 2^E, fp32),

@@ -369,6 +369,7 @@ def measure_rows(hbm, fp4_peak, fp8_peak, reps=10, only=None):
             nbytes=N4 * K4 // 2 + N4 * K4 // 16 + 64 * K4 // 2 + 64 * K4 // 16 + 64 * N4 * 2)
         del Cr, qar, qwr, W4, qwc
     if wants("a4 NVFP4 Four Over Six quantize (gathered, expert groups)", "a9 grouped NVFP4 GEMM up", "a9 grouped NVFP4 GEMM down",
+             "a4 NVFP4 Four Over Six quantize, each token once then moved to its routed rows",
              "a9+a4 grouped up GEMM, then amax + 4/6 quantize of H (two kernels)",
              "f1 grouped up GEMM with the 4/6 NVFP4 quantize in its epilogue (next row)"):
         # -- MoE forward, 16384 tokens, 64 experts, top-8 (gathered 4/6 quantize, grouped up and down)
@@ -384,6 +385,14 @@ def measure_rows(hbm, fp4_peak, fp8_peak, reps=10, only=None):
         row("a4 NVFP4 Four Over Six quantize (gathered, expert groups)", "X 16384x4096 -> 131072 routed rows",
             lambda: api.quant_nvfp4(Xd, four_over_six=True, row_index=ri, groups=(offs, sfo, sf_rows), out=qx),
             nbytes=Mt * H3 * (2 + 2 + 0.5 + 1 / 16))
+
+        ws = torch.empty(bsq.bsq_quant_nvfp4_gather_workspace(T3, H3), dtype=torch.uint8, device=dev)
+        row("a4 NVFP4 Four Over Six quantize, each token once then moved to its routed rows",
+            "X 16384x4096 -> 131072 routed rows",
+            lambda: api.quant_nvfp4_gather(Xd, ri, four_over_six=True, groups=(offs, sfo, sf_rows), out=qx,
+                                           workspace=ws),
+            nbytes=T3 * H3 * 2 + Mt * H3 * (0.5 + 1 / 16))
+        del ws
 
         def experts(Wx):
             E, N, K = Wx.shape

@@ -200,3 +200,28 @@ def combine_s2f6(codes, sf, token_offsets, rows, weights, rht_mask, out=None):
     y = torch.empty(T, K, dtype=torch.bfloat16, device=codes.device) if out is None else out
     bsq.bsq_combine_s2f6(codes, sf, K, token_offsets, rows, weights, T, rht_mask, y, _ld(y))
     return y
+
+
+def quant_nvfp4_gather(x, row_index, four_over_six=False, rht_mask=None, groups=None, amax_in=None, out=None,
+                       workspace=None):
+    """bsq_quant_nvfp4 of the rows x[row_index] (same bytes), computed by
+    quantizing each source row once.  Returns (codes, sf, global_scale)."""
+    T, K = x.shape
+    R = row_index.shape[0]
+    G, ro, so = 0, None, None
+    sf_rows = R
+    if groups is not None:
+        ro, so, sf_rows = groups
+        G = ro.shape[0] - 1
+    if out is None:
+        codes = torch.empty(R, K // 2, dtype=torch.uint8, device=x.device)
+        sf = torch.zeros(sf_bytes(sf_rows, K // 16), dtype=torch.uint8, device=x.device)
+        gs = torch.empty(1, dtype=torch.float32, device=x.device)
+    else:
+        codes, sf, gs = out
+    nbytes = bsq.bsq_quant_nvfp4_gather_workspace(T, K)
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=x.device)
+    bsq.bsq_quant_nvfp4_gather(x, T, K, _ld(x), row_index, R, four_over_six, rht_mask is not None, rht_mask or 0, G,
+                               ro, so, amax_in, gs, codes, sf, workspace, workspace.numel())
+    return codes, sf, gs

@@ -58,6 +58,9 @@ _SIGS = {
     "bsq_gather_rows": (C.c_int, [_vp, _i64, _vp, _i64, _vp, _vp]),
     "bsq_sf_to_rows": (C.c_int, [_vp, _i64, _i64, _vp, _vp]),
     "bsq_sf_from_rows": (C.c_int, [_vp, _i64, _i64, C.c_int, _vp, _vp, _vp, _vp]),
+    "bsq_quant_nvfp4_gather_workspace": (C.c_size_t, [_i64, _i64]),
+    "bsq_quant_nvfp4_gather": (C.c_int, [_vp, _i64, _i64, _i64, _vp, _i64, C.c_int, C.c_int, C.c_uint16, C.c_int,
+                                         _vp, _vp, _vp, _vp, _vp, _vp, _vp, C.c_size_t, _vp]),
     "bsq_check": (C.c_int, [_vp]),
     "bsq_debug_timeout_probe": (C.c_int, [C.c_uint64, _vp]),
     "bsq_debug_kernel_choice": (C.c_int, [C.c_int, C.c_int]),
@@ -231,3 +234,15 @@ def bsq_sf_to_rows(sf, rows, nblk, out, stream=None):
 def bsq_sf_from_rows(rows_in, rows, nblk, G, row_offsets, sf_row_offsets, sf, stream=None):
     return _check("bsq_sf_from_rows", lib().bsq_sf_from_rows(_p(rows_in), rows, nblk, G, _p(row_offsets),
                                                              _p(sf_row_offsets), _p(sf), _stream(stream)))
+
+
+def bsq_quant_nvfp4_gather_workspace(T, K):
+    return int(lib().bsq_quant_nvfp4_gather_workspace(T, K))
+
+
+def bsq_quant_nvfp4_gather(x, T, K, ldx, row_index, M, four_over_six, rht_enable, rht_sign_mask, G, row_offsets,
+                           sf_row_offsets, amax_in, global_scale, codes, sf, workspace, workspace_bytes, stream=None):
+    return _check("bsq_quant_nvfp4_gather", lib().bsq_quant_nvfp4_gather(
+        _p(x), T, K, ldx, _p(row_index), M, int(four_over_six), int(rht_enable), rht_sign_mask, G, _p(row_offsets),
+        _p(sf_row_offsets), _p(amax_in), _p(global_scale), _p(codes), _p(sf), _p(workspace), workspace_bytes,
+        _stream(stream)))

@@ -222,6 +222,61 @@ int bsq_quant_nvfp4(const void *x, int64_t M, int64_t K, int64_t ldx, int block_
     return launch_status();
 }
 
+// Workspace of bsq_quant_nvfp4_gather: 256 bytes (counter, amax bits), the
+// per-row maxima, the source rows' codes and their swizzled scales.
+static int64_t gather_ws_rowmax(int64_t) { return 256; }
+static int64_t gather_ws_codes(int64_t T) { return (256 + 4 * T + 255) / 256 * 256; }
+static int64_t gather_ws_sf(int64_t T, int64_t K) { return gather_ws_codes(T) + (T * (K / 2) + 255) / 256 * 256; }
+
+size_t bsq_quant_nvfp4_gather_workspace(int64_t T, int64_t K) {
+    if (T < 0 || K < 0 || K % 16) return 0;
+    return (size_t)gather_ws_sf(T, K) + bsq_sf_bytes(T, K / 16);
+}
+
+int bsq_quant_nvfp4_gather(const void *x, int64_t T, int64_t K, int64_t ldx, const int32_t *row_index, int64_t M,
+                           int four_over_six, int rht_enable, uint16_t mask, int G, const int32_t *row_off,
+                           const int32_t *sf_off, const float *amax_in, float *gs, uint8_t *codes, uint8_t *sf,
+                           void *workspace, size_t workspace_bytes, void *stream) {
+    if (!x || !row_index || !gs || !codes || !sf || !workspace || T < 0 || M < 0 || K < 0 || K % 64 || ldx < K ||
+        G < 0 || (G > 0 && (!row_off || !sf_off)))
+        return BSQ_ERR_INVALID;
+    if (workspace_bytes < bsq_quant_nvfp4_gather_workspace(T, K)) return BSQ_ERR_INVALID;
+    if (!aligned16(x) || !aligned16(codes) || !aligned16(sf) || ldx % 8 || (reinterpret_cast<uintptr_t>(gs) & 3u) ||
+        (reinterpret_cast<uintptr_t>(workspace) & 255u) || (amax_in && (reinterpret_cast<uintptr_t>(amax_in) & 3u)))
+        return BSQ_ERR_ALIGN;
+    DeviceState *d;
+    if (int st = device_state(&d)) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const uint16_t *xx = static_cast<const uint16_t *>(x);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    unsigned int *scratch = reinterpret_cast<unsigned int *>(ws);
+    float *rowmax = reinterpret_cast<float *>(ws + gather_ws_rowmax(T));
+    uint8_t *codes_src = ws + gather_ws_codes(T);
+    uint8_t *sf_src = ws + gather_ws_sf(T, K);
+    if (M == 0 || K == 0 || T == 0) {
+        if (cudaMemsetAsync(gs, 0, sizeof(float), s) != cudaSuccess) return BSQ_ERR_CUDA;
+        bsq::launch_finalize_global_scale(gs, s);
+        return launch_status();
+    }
+    if (amax_in == nullptr) {
+        if (cudaMemsetAsync(scratch, 0, 8, s) != cudaSuccess) return BSQ_ERR_CUDA;
+        bsq::launch_row_absmax(xx, T, K, ldx, rht_enable != 0, mask, rowmax, d->num_sms, s);
+        bsq::launch_gathered_max(rowmax, row_index, M, scratch + 1, scratch, gs, d->num_sms, s);
+        bsq::launch_quant_nvfp4(xx, T, K, ldx, false, four_over_six != 0, rht_enable != 0, mask, nullptr, 0, nullptr,
+                                nullptr, gs, false, gs, false, codes_src, sf_src, d->num_sms, s);
+    } else if (amax_in == gs) {
+        bsq::launch_quant_nvfp4(xx, T, K, ldx, false, four_over_six != 0, rht_enable != 0, mask, nullptr, 0, nullptr,
+                                nullptr, gs, true, gs, false, codes_src, sf_src, d->num_sms, s);
+        bsq::launch_finalize_global_scale(gs, s);
+    } else {
+        bsq::launch_quant_nvfp4(xx, T, K, ldx, false, four_over_six != 0, rht_enable != 0, mask, nullptr, 0, nullptr,
+                                nullptr, amax_in, true, gs, true, codes_src, sf_src, d->num_sms, s);
+    }
+    bsq::launch_gather_rows(codes_src, K / 2, row_index, M, codes, d->num_sms, s);
+    bsq::launch_gather_sf(sf_src, K / 16, row_index, M, G, row_off, sf_off, sf, d->num_sms, s);
+    return launch_status();
+}
+
 int bsq_quant_nvfp4_sr(const void *x, int64_t M, int64_t K, int64_t ldx, int block_2d, int rht_enable, uint16_t mask,
                        const int32_t *row_index, const float *amax_in, float *gs, uint64_t seed, uint32_t stream_id,
                        uint8_t *codes, uint8_t *sf, void *stream) {

@@ -1885,6 +1885,66 @@ __global__ void __launch_bounds__(256) sf_from_rows_kernel(const uint8_t *__rest
     }
 }
 
+// ===================================================================== NVFP4 of gathered rows, by source row
+// When the rows to quantize are gathered with repeats (MoE routing sends
+// every token to k experts), each output row's codes and scales depend only
+// on its source row and s_g.  So the source rows are quantized once and the
+// results gathered: a per-row maximum of the source (one warp per row), the
+// maximum over the gathered rows (-> s_g), the quantization of the source
+// rows, then the code rows and scale words moved to the output.
+
+// rowmax[r] = max |x[r][:]| (after the RHT when enabled): one warp per row.
+template <bool RHT>
+__global__ void __launch_bounds__(256) row_absmax_kernel(const uint16_t *__restrict__ x, int64_t T, int64_t K,
+                                                         int64_t ldx, uint32_t mask, float *__restrict__ rowmax) {
+    uint32_t sw[8];
+    rht_sign_words(mask, sw);
+    const int lane = threadIdx.x & 31;
+    const int64_t KB = K >> 4;
+    const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    for (int64_t r = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; r < T; r += nw) {
+        float m = 0.0f;
+        for (int64_t kb = lane; kb < KB; kb += 32) {
+            uint32_t w[8];
+            load_words16(x + r * ldx + kb * 16, w);
+            m = fmaxf(m, block_absmax<RHT>(w, sw));
+        }
+#pragma unroll
+        for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+        if (lane == 0) rowmax[r] = m;
+    }
+}
+
+// max over i < M of rowmax[row_index[i]] into *amax_bits; the last CTA
+// writes s_g to *gs_out.
+__global__ void __launch_bounds__(256) gathered_max_kernel(const float *__restrict__ rowmax,
+                                                           const int32_t *__restrict__ row_index, int64_t M,
+                                                           unsigned int *amax_bits, unsigned int *counter,
+                                                           float *gs_out) {
+    float m = 0.0f;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < M; i += (int64_t)gridDim.x * blockDim.x)
+        m = fmaxf(m, __ldg(rowmax + __ldg(row_index + i)));
+    block_reduce_atomic_max(m, amax_bits, counter, gs_out);
+}
+
+// Scale words of gathered rows: output row i (SF row through the groups, as
+// the quantizer maps it) takes source row row_index[i]'s words.
+__global__ void __launch_bounds__(256) gather_sf_kernel(const uint8_t *__restrict__ sf_src, int64_t nblk,
+                                                        const int32_t *__restrict__ row_index, int64_t M, int G,
+                                                        const int32_t *__restrict__ row_off,
+                                                        const int32_t *__restrict__ sf_off, uint8_t *__restrict__ sf) {
+    const int64_t nw4 = nblk >> 2;
+    const int64_t n = M * nw4;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t r = i / nw4, b4 = i - r * nw4;
+        const int64_t dst_row = G > 0 ? grouped_sf_row(r, G, row_off, sf_off) : r;
+        if (dst_row < 0) continue;
+        const int64_t src_row = __ldg(row_index + r);
+        *reinterpret_cast<uint32_t *>(sf + sf_word_offset(dst_row, b4, nblk)) =
+            __ldg(reinterpret_cast<const uint32_t *>(sf_src + sf_word_offset(src_row, b4, nblk)));
+    }
+}
+
 // ===================================================================== RHT
 __global__ void __launch_bounds__(256) rht_kernel(const uint16_t *__restrict__ x, uint16_t *y, int64_t M,
                                                   int64_t K, int64_t ldx, int64_t ldy, uint32_t mask, RowMap map) {
@@ -2279,6 +2339,24 @@ void launch_sf_to_rows(const uint8_t *sf, int64_t rows, int64_t nblk, uint8_t *o
 void launch_sf_from_rows(const uint8_t *in, int64_t rows, int64_t nblk, int G, const int32_t *row_off,
                          const int32_t *sf_off, uint8_t *sf, int num_sms, cudaStream_t s) {
     sf_from_rows_kernel<<<grid_for(rows * nblk, 256, num_sms * 8), 256, 0, s>>>(in, rows, nblk, G, row_off, sf_off, sf);
+}
+
+void launch_row_absmax(const uint16_t *x, int64_t T, int64_t K, int64_t ldx, bool rht, uint32_t mask, float *rowmax,
+                       int num_sms, cudaStream_t s) {
+    const int grid = grid_for(T, 8, num_sms * 8);
+    if (rht) row_absmax_kernel<true><<<grid, 256, 0, s>>>(x, T, K, ldx, mask, rowmax);
+    else row_absmax_kernel<false><<<grid, 256, 0, s>>>(x, T, K, ldx, mask, rowmax);
+}
+
+void launch_gathered_max(const float *rowmax, const int32_t *row_index, int64_t M, unsigned int *amax_bits,
+                         unsigned int *counter, float *gs_out, int num_sms, cudaStream_t s) {
+    gathered_max_kernel<<<grid_for(M, 256 * 8, num_sms), 256, 0, s>>>(rowmax, row_index, M, amax_bits, counter, gs_out);
+}
+
+void launch_gather_sf(const uint8_t *sf_src, int64_t nblk, const int32_t *row_index, int64_t M, int G,
+                      const int32_t *row_off, const int32_t *sf_off, uint8_t *sf, int num_sms, cudaStream_t s) {
+    gather_sf_kernel<<<grid_for(M * (nblk >> 2), 256, num_sms * 8), 256, 0, s>>>(sf_src, nblk, row_index, M, G, row_off,
+                                                                                 sf_off, sf);
 }
 
 void launch_rht(const uint16_t *x, uint16_t *y, int64_t M, int64_t K, int64_t ldx, int64_t ldy, uint32_t mask,

@@ -66,6 +66,12 @@ void launch_gather_rows(const void *src, int64_t row_bytes, const int32_t *index
 void launch_sf_to_rows(const uint8_t *sf, int64_t rows, int64_t nblk, uint8_t *out, int num_sms, cudaStream_t s);
 void launch_sf_from_rows(const uint8_t *in, int64_t rows, int64_t nblk, int G, const int32_t *row_off,
                          const int32_t *sf_off, uint8_t *sf, int num_sms, cudaStream_t s);
+void launch_row_absmax(const uint16_t *x, int64_t T, int64_t K, int64_t ldx, bool rht, uint32_t mask, float *rowmax,
+                       int num_sms, cudaStream_t s);
+void launch_gathered_max(const float *rowmax, const int32_t *row_index, int64_t M, unsigned int *amax_bits,
+                         unsigned int *counter, float *gs_out, int num_sms, cudaStream_t s);
+void launch_gather_sf(const uint8_t *sf_src, int64_t nblk, const int32_t *row_index, int64_t M, int G,
+                      const int32_t *row_off, const int32_t *sf_off, uint8_t *sf, int num_sms, cudaStream_t s);
 void launch_rht(const uint16_t *x, uint16_t *y, int64_t M, int64_t K, int64_t ldx, int64_t ldy, uint32_t mask,
                 int num_sms, cudaStream_t s);
 

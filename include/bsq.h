@@ -151,6 +151,26 @@ BSQ_API int bsq_quant_nvfp4(const void *x_bf16, int64_t M, int64_t K, int64_t ld
                     const float *amax_in_dev, float *global_scale_dev,
                     uint8_t *codes_dev, uint8_t *sf_dev, void *stream);
 
+/* NVFP4 quantize of gathered rows, for gathers that repeat rows (MoE
+ * routing sends each token to several experts).  The result is byte for
+ * byte that of bsq_quant_nvfp4 with the same row_index (1x16 blocks,
+ * optional Four Over Six and RHT, expert groups, amax_in semantics): output
+ * row i is the quantization of source row row_index[i] under the global
+ * scale of the gathered rows' amax.  Since a row's codes and scales depend
+ * only on its source row and s_g, the T source rows (x is [T][K]) are
+ * quantized once into the caller's workspace and then moved to the output
+ * rows.  workspace: device memory of at least
+ * bsq_quant_nvfp4_gather_workspace(T, K) bytes, 256-byte aligned, owned by
+ * the caller (its contents are scratch); every row_index value must be in
+ * [0, T).  K % 64 == 0. */
+BSQ_API size_t bsq_quant_nvfp4_gather_workspace(int64_t T, int64_t K);
+BSQ_API int bsq_quant_nvfp4_gather(const void *x_bf16, int64_t T, int64_t K, int64_t ldx,
+                                   const int32_t *row_index_dev, int64_t M, int four_over_six, int rht_enable,
+                                   uint16_t rht_sign_mask, int G, const int32_t *row_offsets_dev,
+                                   const int32_t *sf_row_offsets_dev, const float *amax_in_dev,
+                                   float *global_scale_dev, uint8_t *codes_dev, uint8_t *sf_dev, void *workspace_dev,
+                                   size_t workspace_bytes, void *stream);
+
 /* NVFP4 quantize with stochastic rounding of the elements ("Microscaling
  * ...", section "NVFP4": the NVFP4 pretraining recipe rounds gradients
  * stochastically).  s_g, the block scales (1x16, or 16x16 with block_2d)

@@ -307,6 +307,11 @@ def test_moe_forward_chain_full(ora, T):
     cx, sx, gx = api.quant_nvfp4(dev(moe.X), four_over_six=True, row_index=ri_d, groups=(offs_d, sfo_d, sf_rows))
     assert bsq.bsq_check() == bsq.BSQ_OK
     assert_quant_full(ora, cx, sx, qx, sf_rows, H // 16, "X gathered 4/6", sf_row_of=sf_row_of, gs_dev=gx)
+    # the same bytes by quantizing each token once and moving its rows
+    cg, sg_, gg = api.quant_nvfp4_gather(dev(moe.X), ri_d, four_over_six=True, groups=(offs_d, sfo_d, sf_rows))
+    assert bsq.bsq_check() == bsq.BSQ_OK
+    assert torch.equal(cg, cx) and torch.equal(sg_, sx) and gg.item() == gx.item()
+    del cg, sg_, gg
     up_dev = _experts_device(ora, qup, F, H)
     dn_dev = _experts_device(ora, qdn, H, F)
     for e in (0, E // 2, E - 1):   # the device's own weight quantization gives the same bytes

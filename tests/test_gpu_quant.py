@@ -246,6 +246,31 @@ def test_nvfp4_moe_gather_groups_parity(ora):
                  groups=(moe.row_offsets, moe.sf_row_offsets), what="moe gather")
 
 
+@pytest.mark.parametrize("fos,rht,given", [(True, None, False), (False, 0x9A3C, False), (True, 0x0F1E, True)])
+def test_nvfp4_gather_by_source_rows(ora, fos, rht, given):
+    """bsq_quant_nvfp4_gather (each source row quantized once, the results
+    moved to the gathered rows) gives the oracle's bytes for the gathered
+    rows, and the same bytes as bsq_quant_nvfp4 with the row index."""
+    moe = W.moe_forward(T=512, H=256, E=8, F=128, weights=False)
+    X = moe.X
+    ri, offs, sfo = moe.row_index, moe.row_offsets, moe.sf_row_offsets
+    K = X.shape[1]
+    groups = (dev(torch.from_numpy(offs)), dev(torch.from_numpy(sfo)), int(sfo[-1]))
+    am_val = float(ora.amax(bits(X), rht_mask=rht, row_index=ri)) * 1.25 if given else None
+    am = None if am_val is None else dev(torch.tensor([am_val], dtype=torch.float32))
+    xd, rid = dev(X), dev(torch.from_numpy(ri))
+    c, s_, g = api.quant_nvfp4_gather(xd, rid, four_over_six=fos, rht_mask=rht, groups=groups, amax_in=am)
+    c2, s2, g2 = api.quant_nvfp4(xd, four_over_six=fos, rht_mask=rht, row_index=rid, groups=groups, amax_in=am)
+    assert bsq.bsq_check() == 0
+    assert torch.equal(c, c2) and torch.equal(s_, s2) and g.item() == g2.item()
+    oc, osf, og = ora.quant_nvfp4(bits(X), four_over_six=fos, rht_mask=rht, row_index=ri, amax_in=am_val)
+    assert np.float32(g.item()) == np.float32(og)
+    assert_codes_equal(host_u8(c), oc, "gather codes")
+    can = ora.sf_unswizzle(host_u8(s_), int(sfo[-1]), K // 16)
+    for e in range(len(offs) - 1):
+        assert_codes_equal(can[sfo[e]:sfo[e] + offs[e + 1] - offs[e]], osf[offs[e]:offs[e + 1]], f"gather sf {e}")
+
+
 def test_amax_parity(ora):
     x = edge_tensor(96, 160, seed=11)
     xd = dev(x)

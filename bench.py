@@ -641,6 +641,8 @@ def main():
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline_line()
 
+    clk_sum = clk.summary()
+    mhz = clk_sum.get("sm_mhz")
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
@@ -659,6 +661,12 @@ def main():
                                         f"of {src}"},
             "breakdown": {
                 "gemm_ms": g_ms, "gemm_tflops": gemm_tflops, "gemm_frac_of_9pf": gemm_tflops / 9000.0,
+                # the GEMM's time in SM cycles at the median sampled clock, and its
+                # rate scaled to the maximum clock (random FP4 data draws the clock
+                # down under the power limit; the MMA rate per cycle is unchanged)
+                "gemm_mcycles_at_median_clock": (g_ms * 1e-3 * mhz * 1e6 / 1e6) if mhz else None,
+                "gemm_tflops_at_max_clock": (gemm_tflops * clk_sum["sm_max_mhz"] / mhz)
+                if mhz and clk_sum.get("sm_max_mhz") else None,
                 "quant_A_ms": statistics.mean(qa_ms), "quant_A_gbs": qa_gbs,
                 "quant_W_ms": statistics.mean(qw_ms), "quant_W_gbs": qw_gbs,
                 "quant_frac_of_hbm": {"A": qa_gbs / hbm, "W": qw_gbs / hbm, "hbm_gbs": hbm, "source": src},
@@ -667,7 +675,7 @@ def main():
                     "h2d_bytes_per_step": (M + N) * K * 2, "d2h_bytes_per_step": M * N * 2,
                     "ms_per_step": e2e_ms},
             "gpu_launches": launches_per_step * args.steps,
-            "clocks": clk.summary(),
+            "clocks": clk_sum,
             "cpu_baseline": cpu,
             "rows": rows,
         }

@@ -208,8 +208,11 @@ def reference_arm(args, rank):
 # ---------------------------------------------------------------------- per-row measurements
 def measure_rows(hbm, fp4_peak, fp8_peak, reps=10, only=None):
     """Times every step of the hot path on its own workload at full size
-    (CUDA events around each call, L2 flushed before each rep by writing a
-    256 MiB buffer, median of `reps`).  Returns a list of dicts; a row that
+    (CUDA events around each call, median of `reps`).  Before each rep L2 is
+    flushed by writing a 256 MiB buffer and then reading another one: L2 is
+    write-back, so after the write alone up to 126 MB of dirty lines would be
+    written back to HBM inside the timed call; the read replaces them by
+    clean lines outside the timing.  Returns a list of dicts; a row that
     fails records its error instead of stopping the bench."""
     import torch
 
@@ -218,6 +221,7 @@ def measure_rows(hbm, fp4_peak, fp8_peak, reps=10, only=None):
 
     dev = torch.device("cuda")
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush_r = torch.ones(64 << 20, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
 
     def timed(fn):
@@ -226,6 +230,7 @@ def measure_rows(hbm, fp4_peak, fp8_peak, reps=10, only=None):
         ts = []
         for _ in range(reps):
             flush.zero_()
+            flush_r.sum()
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
             fn()
@@ -431,7 +436,7 @@ def measure_rows(hbm, fp4_peak, fp8_peak, reps=10, only=None):
         row("a9 grouped NVFP4 GEMM down", f"{Mt} routed rows x {H3} x {F3}, 64 experts",
             lambda: api.grouped_gemm(0, offs, sfo, qh[0], qh[1], dn[0], dn[1], Mt, H3, F3, gsA=qh[2], gsB=dn[2],
                                      out=Cdn), flops=2 * Mt * H3 * F3, peak_kind="fp4")
-    del flush
+    del flush, flush_r
     return rows
 
 

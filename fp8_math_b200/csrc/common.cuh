@@ -118,6 +118,21 @@ BSQ_DEV void e2m1x8_to_f32(uint32_t w, float v[8]) {
     }
 }
 
+// The two E2M1 codes in the low byte of w (element 0 in the low nibble) ->
+// fp32, exactly, as e2m1x8_to_f32 does.
+BSQ_DEV void e2m1x2_to_f32(uint32_t w, float &lo, float &hi) {
+    uint32_t h;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "mov.b32 {b0, b1, b2, b3}, %1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t}"
+        : "=r"(h)
+        : "r"(w));
+    __half_raw l, u;
+    l.x = (unsigned short)(h & 0xFFFFu);
+    u.x = (unsigned short)(h >> 16);
+    lo = __half2float(__half(l));
+    hi = __half2float(__half(u));
+}
 
 // floor(log2 a) for a finite a > 0 (normal or subnormal binary32).
 BSQ_DEV int floor_log2(float a) {

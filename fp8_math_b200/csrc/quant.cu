@@ -872,6 +872,32 @@ __device__ __noinline__ uint2 mx_sr8_float(float s0, float s1, float s2, float s
     return make_uint2(c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24), c[4] | (c[5] << 8) | (c[6] << 16) | (c[7] << 24));
 }
 
+// The same with zeros allowed (a zero never rounds: its code is the sign);
+// the float form runs only when some nonzero value lies below 2^-6.  Inline
+// for inputs where zeros are common (decoded 4-bit data), and out of line as
+// the fallback of mx_sr8.
+BSQ_DEV uint2 mx_sr8_z(const float s[8], uint4 rnd) {
+    const uint32_t w[4] = {rnd.x, rnd.y, rnd.z, rnd.w};
+    uint32_t b[8];
+    bool slow = false;
+#pragma unroll
+    for (int i = 0; i < 8; i++) {
+        const uint32_t a = __float_as_uint(fminf(fabsf(s[i]), 448.0f));
+        slow |= a - 1u < 0x3C7FFFFFu;  // 0 < a < 2^-6
+        const uint32_t p = __byte_perm(w[i >> 1], 0u, (i & 1) ? 0x4324u : 0x4104u);
+        const uint32_t t = (a << 4) + 0x40FFFFF0u - p;
+        b[i] = (a ? t : 0u) | (__float_as_uint(s[i]) & 0x80000000u);
+    }
+    if (slow) return mx_sr8_float(s[0], s[1], s[2], s[3], s[4], s[5], s[6], s[7], rnd);
+    return make_uint2(__byte_perm(__byte_perm(b[0], b[1], 0x0073u), __byte_perm(b[2], b[3], 0x7300u), 0x7610u),
+                      __byte_perm(__byte_perm(b[4], b[5], 0x0073u), __byte_perm(b[6], b[7], 0x7300u), 0x7610u));
+}
+__device__ __noinline__ uint2 mx_sr8_zeros(float s0, float s1, float s2, float s3, float s4, float s5, float s6,
+                                           float s7, uint4 rnd) {
+    const float s[8] = {s0, s1, s2, s3, s4, s5, s6, s7};
+    return mx_sr8_z(s, rnd);
+}
+
 BSQ_DEV uint2 mx_sr8(const float s[8], uint4 rnd) {
     const uint32_t w[4] = {rnd.x, rnd.y, rnd.z, rnd.w};
     uint32_t b[8];
@@ -884,7 +910,7 @@ BSQ_DEV uint2 mx_sr8(const float s[8], uint4 rnd) {
         const uint32_t t = (a << 4) + 0x40FFFFF0u - p;  // 0xFFFFF0 - (120 << 27) mod 2^32
         b[i] = t | (__float_as_uint(s[i]) & 0x80000000u);
     }
-    if (slow) return mx_sr8_float(s[0], s[1], s[2], s[3], s[4], s[5], s[6], s[7], rnd);
+    if (slow) return mx_sr8_zeros(s[0], s[1], s[2], s[3], s[4], s[5], s[6], s[7], rnd);
     return make_uint2(__byte_perm(__byte_perm(b[0], b[1], 0x0073u), __byte_perm(b[2], b[3], 0x7300u), 0x7610u),
                       __byte_perm(__byte_perm(b[4], b[5], 0x0073u), __byte_perm(b[6], b[7], 0x7300u), 0x7610u));
 }
@@ -894,15 +920,17 @@ BSQ_DEV uint4 mx_draws(uint64_t chunk, const PhiloxKeys &keys, uint32_t stream_i
 }
 
 // True when stochastic rounding of the 8 scaled values cannot depend on the
-// draws: each one is an E4M3 value of the normal range or above 448 (its low
-// 20 bits are zero, so frac = 0 and it never rounds up), as every E4M3 input
-// rescaled by a power of two is unless it falls below 2^-6.
+// draws: each one is zero or an E4M3 value of the normal range or above 448
+// (its low 20 bits are zero, so frac = 0 and it never rounds up), as every
+// E4M3 input rescaled by a power of two is unless it falls below 2^-6.  Such
+// a chunk's codes are its nearest-even codes (exact values, saturated above
+// 448 as stochastic rounding saturates them).
 BSQ_DEV bool mx_sr8_drawless(const float s[8]) {
     bool ok = true;
 #pragma unroll
     for (int i = 0; i < 8; i++) {
         const uint32_t a = __float_as_uint(fminf(fabsf(s[i]), 448.0f));
-        ok &= ((a & 0xFFFFFu) == 0u) & (a >= 0x3C800000u);
+        ok &= ((a & 0xFFFFFu) == 0u) & ((a >= 0x3C800000u) | (a == 0u));
     }
     return ok;
 }
@@ -921,17 +949,19 @@ __device__ __noinline__ uint2 mx_sr8_drawn(float s0, float s1, float s2, float s
 // of the chunk's first element divided by 8: the Philox counter of SR.  With
 // EXACT_IN (inputs that are E4M3 values times a power of two) the Philox call
 // runs only for chunks whose rounding can depend on it.
-template <bool SR, bool EXACT_IN = false>
+template <bool SR, bool EXACT_IN = false, bool ZEROS = false>
 BSQ_DEV uint2 mx_encode8(const float v[8], bool zero, uint32_t sb, uint64_t chunk, const PhiloxKeys &keys,
                          uint32_t stream_id) {
     float s[8];
     mx_scale8(v, mx_inv_scale(sb), s);
     uint2 q;
     if (SR) {
-        if (!EXACT_IN)
+        if (ZEROS)
+            q = mx_sr8_z(s, mx_draws(chunk, keys, stream_id));
+        else if (!EXACT_IN)
             q = mx_sr8(s, mx_draws(chunk, keys, stream_id));
         else if (mx_sr8_drawless(s))
-            q = mx_sr8(s, make_uint4(0u, 0u, 0u, 0u));
+            q = mx_rne8(s);
         else
             q = mx_sr8_drawn(s[0], s[1], s[2], s[3], s[4], s[5], s[6], s[7], chunk, keys, stream_id);
     } else {
@@ -979,8 +1009,40 @@ BSQ_DEV uint32_t mx_scale_code_bf16(uint32_t m) { return (uint32_t)max((int)(m >
 // (s + 15 - (r16 >> 12) - (120 << 7)) >> 4 is then the E4M3 magnitude code
 // (exponent - 120 and three mantissa bits).  Shifted left by 4, each lane's
 // code sits in its upper byte with bit 7 clear, where the bf16 sign bit is
-// or-ed in.  A chunk holding some s < 2^-6 (E4M3 subnormals, zeros) runs
-// the fp32 form on all eight values.
+// or-ed in.  A chunk holding some s < 2^-6 is redone with zeros allowed: a
+// zero input lane (which never rounds) is computed as s = 2^-6 so that no
+// borrow crosses into the other lane, and its code masked to the sign; only
+// a chunk with some nonzero input below 2^-6 (E4M3 subnormals, or a product
+// that underflowed) runs the fp32 form on all eight values.
+// The fallback of mx_sr8_bf16 for a chunk that failed its fast check (out of
+// line: the unrolled callers stay small).
+__device__ __noinline__ uint2 mx_sr8_bf16_slow(uint4 pv, uint4 av, uint32_t sb, uint4 rnd) {
+    const uint32_t p[4] = {pv.x, pv.y, pv.z, pv.w}, a[4] = {av.x, av.y, av.z, av.w};
+    const uint32_t inv2 = ((254u - sb) << 7) * 0x10001u;
+    const uint32_t w[4] = {rnd.x, rnd.y, rnd.z, rnd.w};
+    uint32_t mn = 0xFFFFFFFFu, u[4];
+#pragma unroll
+    for (int k = 0; k < 4; k++) {
+        const uint32_t s0 = u16x2_min(bf16x2_mul(a[k], inv2), 0x43E043E0u);
+        const uint32_t nz = __vcmpne2(a[k], 0u);         // 0xFFFF in each nonzero input lane
+        const uint32_t s = s0 | (~nz & 0x3C803C80u);
+        mn = u16x2_min(mn, s);
+        const uint32_t r = (~w[k] >> 12) & 0x000F000Fu;
+        u[k] = (((s + r - 0x3C003C00u) << 4) & nz) | (p[k] & 0x80008000u);
+    }
+    if (min(mn & 0xFFFFu, mn >> 16) < 0x3C80u) {
+        float v[8], sc[8];
+#pragma unroll
+        for (int k = 0; k < 4; k++) {
+            v[2 * k] = bf16_lo(p[k]);
+            v[2 * k + 1] = bf16_hi(p[k]);
+        }
+        mx_scale8(v, mx_inv_scale(sb), sc);
+        return mx_sr8_float(sc[0], sc[1], sc[2], sc[3], sc[4], sc[5], sc[6], sc[7], rnd);
+    }
+    return make_uint2(__byte_perm(u[0], u[1], 0x7531u), __byte_perm(u[2], u[3], 0x7531u));
+}
+
 BSQ_DEV uint2 mx_sr8_bf16(const uint32_t p[4], const uint32_t a[4], uint32_t sb, uint4 rnd) {
     const uint32_t inv2 = ((254u - sb) << 7) * 0x10001u;  // 2^-E in both bf16 lanes
     const uint32_t w[4] = {rnd.x, rnd.y, rnd.z, rnd.w};
@@ -992,16 +1054,8 @@ BSQ_DEV uint2 mx_sr8_bf16(const uint32_t p[4], const uint32_t a[4], uint32_t sb,
         const uint32_t r = (~w[k] >> 12) & 0x000F000Fu;  // 15 - (r16 >> 12), both lanes
         u[k] = ((s + r - 0x3C003C00u) << 4) | (p[k] & 0x80008000u);
     }
-    if (min(mn & 0xFFFFu, mn >> 16) < 0x3C80u) {  // 2^-6
-        float v[8], s[8];
-#pragma unroll
-        for (int k = 0; k < 4; k++) {
-            v[2 * k] = bf16_lo(p[k]);
-            v[2 * k + 1] = bf16_hi(p[k]);
-        }
-        mx_scale8(v, mx_inv_scale(sb), s);
-        return mx_sr8_float(s[0], s[1], s[2], s[3], s[4], s[5], s[6], s[7], rnd);
-    }
+    if (min(mn & 0xFFFFu, mn >> 16) < 0x3C80u)  // 2^-6
+        return mx_sr8_bf16_slow(make_uint4(p[0], p[1], p[2], p[3]), make_uint4(a[0], a[1], a[2], a[3]), sb, rnd);
     return make_uint2(__byte_perm(u[0], u[1], 0x7531u), __byte_perm(u[2], u[3], 0x7531u));
 }
 // Row-wise: one thread per 8 elements, 4 lanes per block of 32.
@@ -1163,22 +1217,21 @@ __global__ void __launch_bounds__(256) quant_mxfp8_row_span_kernel(
 }
 
 // Column-wise (output [K, M] = quantization of the transpose, blocks of 32
-// along M), from bf16 or from row-wise MXFP8 (dequantized exactly).  A warp
-// covers 32 input rows x 64 input columns with no shared memory: lane
-// l = 4 kg + mg loads the 8 x 8 piece of rows 8 mg .. 8 mg + 7 and columns
-// 8 kg .. 8 kg + 7 (each warp-wide load reads 128 contiguous bytes of four
-// rows), which holds, per column, one output chunk of 8 consecutive m; the
-// four lanes with the same kg share that column's block of 32 (two-step
-// shuffle max).  Warp tiles run m-fastest, so consecutive warps write
-// adjacent 32-byte pieces of each output row.
-template <bool FROM_MX, bool SR>
+// along M) from bf16.  A warp covers 32 input rows x 64 input columns with
+// no shared memory: lane l = 4 kg + mg loads the 8 x 8 piece of rows
+// 8 mg .. 8 mg + 7 and columns 8 kg .. 8 kg + 7 (each warp-wide load reads
+// 128 contiguous bytes of four rows), which holds, per column, one output
+// chunk of 8 consecutive m; the four lanes with the same kg share that
+// column's block of 32 (two-step shuffle max).  Warp tiles run m-fastest, so
+// consecutive warps write adjacent 32-byte pieces of each output row.
+template <bool SR>
 __global__ void __launch_bounds__(256) quant_mxfp8_col_kernel(
-    const void *__restrict__ xin, const uint8_t *__restrict__ sf_in, int64_t M, int64_t K, int64_t ldx,
-    uint32_t ntile, DivU32 div_mt, const __grid_constant__ PhiloxKeys keys, uint32_t stream_id,
-    uint8_t *__restrict__ codes, uint8_t *__restrict__ sf) {
+    const uint16_t *__restrict__ xin, int64_t M, int64_t K, int64_t ldx, uint32_t ntile, DivU32 div_mt,
+    const __grid_constant__ PhiloxKeys keys, uint32_t stream_id, uint8_t *__restrict__ codes,
+    uint8_t *__restrict__ sf) {
     const int lane = threadIdx.x & 31, kg = lane >> 2, mg = lane & 3;
     const uint32_t mt_n = (uint32_t)(M >> 5);
-    const int64_t MB = M >> 5, KBin = K >> 5;
+    const int64_t MB = M >> 5;
     const uint32_t nwarps = (gridDim.x * blockDim.x) >> 5;
     for (uint32_t t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < ntile; t += nwarps) {
         const uint32_t kt = divu32(t, div_mt), mt = t - kt * mt_n;
@@ -1186,28 +1239,19 @@ __global__ void __launch_bounds__(256) quant_mxfp8_col_kernel(
         const bool kvalid = k0 < K;  // K % 8 == 0: a lane's 8 columns are all in or all out
         // w[i][p]: columns 2p, 2p + 1 of row m0 + i (low half: the even column)
         uint32_t w[8][4];
-        float sc[8];
-        if (!FROM_MX) {
-            const uint16_t *x = static_cast<const uint16_t *>(xin) + m0 * ldx + k0;
+        const uint16_t *x = xin + m0 * ldx + k0;
 #pragma unroll
-            for (int i = 0; i < 8; i++) {
-                const uint4 r = kvalid ? __ldg(reinterpret_cast<const uint4 *>(x + i * ldx)) : make_uint4(0, 0, 0, 0);
-                w[i][0] = r.x; w[i][1] = r.y; w[i][2] = r.z; w[i][3] = r.w;
-            }
-        } else {
-            const uint8_t *x = static_cast<const uint8_t *>(xin) + m0 * ldx + k0;
-#pragma unroll
-            for (int i = 0; i < 8; i++) {
-                const uint2 r = kvalid ? __ldg(reinterpret_cast<const uint2 *>(x + i * ldx)) : make_uint2(0, 0);
-                w[i][0] = r.x; w[i][1] = r.y;
-                sc[i] = kvalid ? exp2i((int)__ldg(sf_in + sf_offset(m0 + i, k0 >> 5, KBin)) - 127) : 0.0f;
-            }
+        for (int i = 0; i < 8; i++) {
+            const uint4 r = kvalid ? __ldg(reinterpret_cast<const uint4 *>(x + i * ldx)) : make_uint4(0, 0, 0, 0);
+            w[i][0] = r.x; w[i][1] = r.y; w[i][2] = r.z; w[i][3] = r.w;
         }
-        float odd[8];  // E4M3 input: column j + 1, decoded with column j
 #pragma unroll
         for (int j = 0; j < 8; j++) {
             const int64_t k = k0 + j;
-            if (!FROM_MX && SR) {
+            uint2 q;
+            uint32_t sb;
+            bool zero;
+            if (SR) {
                 // rows 2i, 2i + 1 of column j as one bf16 pair
                 uint32_t p[4], a[4];
 #pragma unroll
@@ -1216,36 +1260,22 @@ __global__ void __launch_bounds__(256) quant_mxfp8_col_kernel(
                 uint32_t m = bf16_chunk_absmax(p, a);
                 m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
                 m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
-                const uint32_t sb = mx_scale_code_bf16(m);
-                uint2 q = mx_sr8_bf16(p, a, sb, mx_draws((uint64_t)(k * M + m0) >> 3, keys, stream_id));
-                if (m == 0u) q = make_uint2(0u, 0u);
-                if (kvalid) {
-                    *reinterpret_cast<uint2 *>(codes + k * M + m0) = q;
-                    if (mg == 0) sf[sf_offset(k, m0 >> 5, MB)] = (uint8_t)sb;
-                }
-                continue;
-            }
-            float v[8];
+                sb = mx_scale_code_bf16(m);
+                q = mx_sr8_bf16(p, a, sb, mx_draws((uint64_t)(k * M + m0) >> 3, keys, stream_id));
+                zero = m == 0u;
+            } else {
+                float v[8];
 #pragma unroll
-            for (int i = 0; i < 8; i++) {
-                if (!FROM_MX) {
-                    v[i] = (j & 1) ? bf16_hi(w[i][j >> 1]) : bf16_lo(w[i][j >> 1]);
-                } else if ((j & 1) == 0) {
-                    float e0, e1;
-                    e4m3x2_to_f32(w[i][j >> 2] >> (8 * (j & 3)), e0, e1);
-                    v[i] = __fmul_rn(e0, sc[i]);
-                    odd[i] = __fmul_rn(e1, sc[i]);
-                } else {
-                    v[i] = odd[i];
-                }
+                for (int i = 0; i < 8; i++) v[i] = (j & 1) ? bf16_hi(w[i][j >> 1]) : bf16_lo(w[i][j >> 1]);
+                float m = fmax3(fmax3(fabsf(v[0]), fabsf(v[1]), fabsf(v[2])),
+                                fmax3(fabsf(v[3]), fabsf(v[4]), fabsf(v[5])), fmaxf(fabsf(v[6]), fabsf(v[7])));
+                m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+                m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+                sb = mx_scale_code(m);
+                q = mx_encode8<false>(v, false, sb, 0, keys, 0u);
+                zero = m == 0.0f;
             }
-            float m = fmax3(fmax3(fabsf(v[0]), fabsf(v[1]), fabsf(v[2])), fmax3(fabsf(v[3]), fabsf(v[4]), fabsf(v[5])),
-                            fmaxf(fabsf(v[6]), fabsf(v[7])));
-            m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
-            m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
-            const uint32_t sb = mx_scale_code(m);
-            const uint2 q =
-                mx_encode8<SR, FROM_MX>(v, m == 0.0f, sb, (uint64_t)(k * M + m0) >> 3, keys, stream_id);
+            if (zero) q = make_uint2(0u, 0u);
             if (kvalid) {
                 *reinterpret_cast<uint2 *>(codes + k * M + m0) = q;
                 if (mg == 0) sf[sf_offset(k, m0 >> 5, MB)] = (uint8_t)sb;
@@ -1254,22 +1284,14 @@ __global__ void __launch_bounds__(256) quant_mxfp8_col_kernel(
     }
 }
 
-// Dequantize -> transpose -> requantize of a row-wise MXFP8 tensor in
-// integer arithmetic.  The column kernel's warp tile: lane l = 4 kg + mg
-// holds rows 8 mg .. 8 mg + 7 and columns 8 kg .. 8 kg + 7 (one 8-byte code
-// load and one E8M0 byte per row: the 8 columns sit in one input block).  A
-// normal E4M3 code c (exponent field e >= 1) in a row with scale code f
-// decodes to the binary32 whose bits are (c & 0x7F) << 20 plus (f - 7) << 23
-// (exponent e + f - 7 + 127 - 127, mantissa the code's three bits), exact
-// whenever that exponent field stays in 1..254.  The block maximum is then
-// an unsigned maximum of bits, the new scale code max(field - 8, 0) (as for
-// bf16 input), and the rescaled value's bits one subtraction of the new
-// exponent: with three mantissa bits it is an E4M3 value whenever its field
-// is at least 121 (2^-6), so its code is the bits >> 20 less 120 << 3
-// (saturated at 0x7E = 448) for nearest-even and stochastic rounding alike
-// (a representable value never rounds).  A chunk holding an E4M3 subnormal
-// input, a row scale outside 7..246, or a value that lands below 2^-6 takes
-// the exact binary32 path (decode, then the general encode).
+// Dequantize -> transpose -> requantize of a row-wise MXFP8 tensor.  The
+// column kernel's warp tile: lane l = 4 kg + mg holds rows 8 mg .. 8 mg + 7
+// and columns 8 kg .. 8 kg + 7 (one 8-byte code load and one E8M0 byte per
+// row: the 8 columns sit in one input block).  Each value is decoded exactly
+// (E4M3 -> f16 -> fp32, times its power-of-two row scale) and requantized
+// with the column block's scale; a chunk whose rescaled values are all E4M3
+// values (the common case: an E4M3 value times a power of two) needs no
+// rounding and takes the nearest-even conversion without drawing.
 template <bool SR>
 __global__ void __launch_bounds__(256) requant_transpose_kernel(
     const uint8_t *__restrict__ codes_in, const uint8_t *__restrict__ sf_in, int64_t M, int64_t K, uint32_t ntile,
@@ -1283,65 +1305,39 @@ __global__ void __launch_bounds__(256) requant_transpose_kernel(
         const uint32_t kt = divu32(t, div_mt), mt = t - kt * mt_n;
         const int64_t m0 = (int64_t)mt * 32 + mg * 8, k0 = (int64_t)kt * 64 + kg * 8;
         const bool kvalid = k0 < K;  // K % 32 == 0: a lane's 8 columns are all in or all out
-        uint32_t w[8][2], fsc[8];
-        bool rows_ok = true;
+        uint32_t w[8][2];
+        float sc[8];
 #pragma unroll
         for (int i = 0; i < 8; i++) {
             const uint2 r = kvalid ? __ldg(reinterpret_cast<const uint2 *>(codes_in + (m0 + i) * K + k0)) : make_uint2(0, 0);
             w[i][0] = r.x;
             w[i][1] = r.y;
-            fsc[i] = kvalid ? __ldg(sf_in + sf_offset(m0 + i, k0 >> 5, KB)) : 127u;
-            rows_ok &= (fsc[i] >= 7u) & (fsc[i] <= 246u);
+            sc[i] = kvalid ? exp2i((int)__ldg(sf_in + sf_offset(m0 + i, k0 >> 5, KB)) - 127) : 0.0f;
         }
+        float odd[8];  // column j + 1, decoded with column j
 #pragma unroll
         for (int j = 0; j < 8; j++) {
             const int64_t k = k0 + j;
-            uint32_t bits[8], sgn[8];
-            bool fast = rows_ok;
+            float v[8];
 #pragma unroll
             for (int i = 0; i < 8; i++) {
-                const uint32_t c = (w[i][j >> 2] >> (8 * (j & 3))) & 0xFFu;
-                const uint32_t mag = c & 0x7Fu;
-                sgn[i] = c & 0x80u;
-                fast &= (mag >= 8u) | (mag == 0u);
-                bits[i] = mag >= 8u ? (mag << 20) + ((fsc[i] - 7u) << 23) : 0u;
-            }
-            if (!fast) {
-                // exact binary32 decode of every element of the chunk
-#pragma unroll
-                for (int i = 0; i < 8; i++) {
-                    const uint32_t c = (w[i][j >> 2] >> (8 * (j & 3))) & 0x7Fu;
-                    bits[i] = __float_as_uint(__fmul_rn(e4m3_to_f32(c), exp2i((int)fsc[i] - 127)));
+                if ((j & 1) == 0) {
+                    float e0, e1;
+                    e4m3x2_to_f32(w[i][j >> 2] >> (8 * (j & 3)), e0, e1);
+                    v[i] = __fmul_rn(e0, sc[i]);
+                    odd[i] = __fmul_rn(e1, sc[i]);
+                } else {
+                    v[i] = odd[i];
                 }
             }
-            uint32_t m = max(max(max(bits[0], bits[1]), max(bits[2], bits[3])),
-                             max(max(bits[4], bits[5]), max(bits[6], bits[7])));
-            m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
-            m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
-            const uint32_t sb = (uint32_t)max((int)(m >> 23) - 8, 0);
-            const uint32_t down = (sb - 127u) << 23;  // subtracting it divides by 2^(sb - 127)
-            uint32_t q[8];
-            bool exact = fast;
-#pragma unroll
-            for (int i = 0; i < 8; i++) {
-                const uint32_t sbits = bits[i] - down;   // meaningful when the new field is >= 121
-                exact &= (bits[i] == 0u) | ((int)(bits[i] >> 23) - (int)sb + 127 >= 121);
-                q[i] = bits[i] ? (min((sbits >> 20) - 960u, 0x7Eu) | sgn[i]) : sgn[i];
-            }
-            uint2 out;
-            if (m == 0u) {
-                out = make_uint2(0u, 0u);
-            } else if (exact) {
-                out = make_uint2(q[0] | (q[1] << 8) | (q[2] << 16) | (q[3] << 24),
-                                 q[4] | (q[5] << 8) | (q[6] << 16) | (q[7] << 24));
-            } else {
-                float v[8];
-#pragma unroll
-                for (int i = 0; i < 8; i++) v[i] = __uint_as_float(bits[i] | (sgn[i] << 24));
-                out = mx_encode8<SR, true>(v, false, sb, (uint64_t)(k * M + m0) >> 3, keys, stream_id);
-            }
+            float m = fmax3(fmax3(fabsf(v[0]), fabsf(v[1]), fabsf(v[2])), fmax3(fabsf(v[3]), fabsf(v[4]), fabsf(v[5])),
+                            fmaxf(fabsf(v[6]), fabsf(v[7])));
+            m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+            m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+            const uint32_t sb = mx_scale_code(m);
+            const uint2 q = mx_encode8<SR, true>(v, m == 0.0f, sb, (uint64_t)(k * M + m0) >> 3, keys, stream_id);
             if (kvalid) {
-                *reinterpret_cast<uint2 *>(codes + k * M + m0) = out;
+                *reinterpret_cast<uint2 *>(codes + k * M + m0) = q;
                 if (mg == 0) sf[sf_offset(k, m0 >> 5, MB)] = (uint8_t)sb;
             }
         }
@@ -1467,33 +1463,39 @@ __global__ void __launch_bounds__(256) requant_nvfp4_mxfp8_kernel(
         const uint32_t kt = divu32(t, div_mt), mt = t - kt * mt_n;
         const int64_t m0 = (int64_t)mt * 32 + mg * 8, k0 = (int64_t)kt * 64 + kg * 8;
         const bool kvalid = k0 < C;  // C % 16 == 0: a lane's 8 columns are all in or all out
-        float v[8][8];               // v[i][j]: row m0 + i, column k0 + j
+        uint32_t w[8];               // w[i]: the 8 codes of row m0 + i
+        float sbv[8];                // its block scale
 #pragma unroll
         for (int i = 0; i < 8; i++) {
-            const uint32_t w = kvalid ? __ldg(reinterpret_cast<const uint32_t *>(codes_in + (m0 + i) * (C >> 1) + (k0 >> 1)))
-                                      : 0u;
-            const float sbv = kvalid ? e4m3_to_f32(__ldg(sf_in + sf_offset(m0 + i, k0 >> 4, CB16))) : 0.0f;
-            float e[8];
-            e2m1x8_to_f32(w, e);
-#pragma unroll
-            for (int j = 0; j < 8; j++) v[i][j] = __fmul_rn(__fmul_rn(e[j], sbv), s_g);
+            w[i] = kvalid ? __ldg(reinterpret_cast<const uint32_t *>(codes_in + (m0 + i) * (C >> 1) + (k0 >> 1))) : 0u;
+            sbv[i] = kvalid ? e4m3_to_f32(__ldg(sf_in + sf_offset(m0 + i, k0 >> 4, CB16))) : 0.0f;
         }
-#pragma unroll
-        for (int j = 0; j < 8; j++) {
+        auto column = [&](int j, const float (&c)[8]) {
             const int64_t k = k0 + j;
-            float c[8];
-#pragma unroll
-            for (int i = 0; i < 8; i++) c[i] = v[i][j];
             float m = fmax3(fmax3(fabsf(c[0]), fabsf(c[1]), fabsf(c[2])), fmax3(fabsf(c[3]), fabsf(c[4]), fabsf(c[5])),
                             fmaxf(fabsf(c[6]), fabsf(c[7])));
             m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
             m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
             const uint32_t sb = mx_scale_code(m);
-            const uint2 q = mx_encode8<SR>(c, m == 0.0f, sb, (uint64_t)(k * R + m0) >> 3, keys, stream_id);
+            const uint2 q = mx_encode8<SR, false, true>(c, m == 0.0f, sb, (uint64_t)(k * R + m0) >> 3, keys, stream_id);
             if (kvalid) {
                 *reinterpret_cast<uint2 *>(codes + k * R + m0) = q;
                 if (mg == 0) sf[sf_offset(k, m0 >> 5, RB)] = (uint8_t)sb;
             }
+        };
+        // columns 2 jj and 2 jj + 1 (byte jj of every row), decoded as needed
+#pragma unroll
+        for (int jj = 0; jj < 4; jj++) {
+            float ce[8], co[8];
+#pragma unroll
+            for (int i = 0; i < 8; i++) {
+                float lo, hi;
+                e2m1x2_to_f32(w[i] >> (8 * jj), lo, hi);
+                ce[i] = __fmul_rn(__fmul_rn(lo, sbv[i]), s_g);
+                co[i] = __fmul_rn(__fmul_rn(hi, sbv[i]), s_g);
+            }
+            column(2 * jj, ce);
+            column(2 * jj + 1, co);
         }
     }
 }
@@ -2210,13 +2212,11 @@ void launch_quant_mxfp8(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, bo
     const uint32_t ntile = (uint32_t)((M >> 5) * ((K + 63) >> 6));
     const DivU32 dmt = divu32_for((uint32_t)(M >> 5));
     if (sr) {
-        const int grid = grid_for(ntile, 8, resident_ctas<quant_mxfp8_col_kernel<false, true>>(num_sms));
-        quant_mxfp8_col_kernel<false, true><<<grid, 256, 0, s>>>(x, nullptr, M, K, ldx, ntile, dmt, keys,
-                                                                 stream_id, codes, sf);
+        const int grid = grid_for(ntile, 8, resident_ctas<quant_mxfp8_col_kernel<true>>(num_sms));
+        quant_mxfp8_col_kernel<true><<<grid, 256, 0, s>>>(x, M, K, ldx, ntile, dmt, keys, stream_id, codes, sf);
     } else {
-        const int grid = grid_for(ntile, 8, resident_ctas<quant_mxfp8_col_kernel<false, false>>(num_sms));
-        quant_mxfp8_col_kernel<false, false><<<grid, 256, 0, s>>>(x, nullptr, M, K, ldx, ntile, dmt, keys,
-                                                                  stream_id, codes, sf);
+        const int grid = grid_for(ntile, 8, resident_ctas<quant_mxfp8_col_kernel<false>>(num_sms));
+        quant_mxfp8_col_kernel<false><<<grid, 256, 0, s>>>(x, M, K, ldx, ntile, dmt, keys, stream_id, codes, sf);
     }
 }
 

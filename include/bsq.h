@@ -74,7 +74,8 @@ enum {
     BSQ_KNOB_FUSED_QUANT = 0, /* 1/-1: amax + 16x16 quantize in one cooperative launch; 0: two passes */
     BSQ_KNOB_GEMM_PAIR = 1,   /* -1: automatic; 0: single-CTA GEMM; 1: CTA-pair GEMM where it applies */
     BSQ_KNOB_GEMM_BN = 2,     /* -1: automatic; 128 or 256 (bf16 output): the single-CTA GEMM's N tile */
-    BSQ_KNOB_STREAM_QUANT = 3 /* 1/-1: bulk-copy streaming amax / NVFP4 kernels for contiguous tensors; 0: off */
+    BSQ_KNOB_STREAM_QUANT = 3 /* -1: bulk-copy streaming NVFP4 kernels for contiguous 16x16 tensors; 1: for every
+                                 contiguous amax / NVFP4 call; 0: never */
 };
 
 /* Human-readable name of a status code (static string). */

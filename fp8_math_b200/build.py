@@ -25,7 +25,7 @@ SOURCES = {
     "gemm.cu": [],
     "api.cu": [],
 }
-HEADERS = ["common.cuh", "nvfp4.cuh", "quant.cuh", "gemm.cuh", "sm100.cuh"]
+HEADERS = ["common.cuh", "devcache.h", "nvfp4.cuh", "quant.cuh", "gemm.cuh", "sm100.cuh"]
 
 
 def _mtime(p):

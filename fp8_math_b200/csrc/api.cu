@@ -60,7 +60,7 @@ void philox_host(uint32_t c[4], uint32_t k0, uint32_t k1) {
 }
 
 // Kernel-selection overrides (bsq_debug_kernel_choice): -1 = automatic.
-std::atomic<int> g_knob[4] = {{-1}, {-1}, {-1}, {-1}};
+std::atomic<int> g_knob[5] = {{-1}, {-1}, {-1}, {-1}, {-1}};
 
 }  // namespace
 
@@ -79,6 +79,9 @@ int bsq_debug_kernel_choice(int knob, int value) {
             break;
         case BSQ_KNOB_GEMM_BN:
             if (value != -1 && value != 128 && value != 256) return BSQ_ERR_INVALID;
+            break;
+        case BSQ_KNOB_GEMM_SPLITK:
+            if (value != -1 && value != 1 && value != 2 && value != 4 && value != 8) return BSQ_ERR_INVALID;
             break;
         default:
             return BSQ_ERR_INVALID;

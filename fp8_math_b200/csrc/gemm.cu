@@ -25,6 +25,7 @@
 #include <mutex>
 
 #include "common.cuh"
+#include "devcache.h"
 #include "gemm.cuh"
 #include "nvfp4.cuh"
 #include "sm100.cuh"
@@ -81,7 +82,7 @@ struct FmtTraits<BSQ_MXFP8> {
     static constexpr uint32_t kIdescFmt = (0u << 7) | (0u << 10) | (1u << 23);  // E4M3 x E4M3, UE8M0
 };
 
-template <int FMT, int BN>
+template <int FMT, int BN, int MAXNS = 8>
 struct Cfg {
     using T = FmtTraits<FMT>;
     static constexpr int kBM = 128;
@@ -91,7 +92,8 @@ struct Cfg {
     static constexpr int kSfaBytes = T::kAtomsPerKt * 512;
     static constexpr int kSfbBytes = kNbAtomTiles * kSfaBytes;
     static constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
-    static constexpr int kStages = (220 * 1024) / kStageBytes > 8 ? 8 : (220 * 1024) / kStageBytes;
+    static constexpr int kFit = (220 * 1024) / kStageBytes;
+    static constexpr int kStages = kFit > MAXNS ? MAXNS : kFit;
     static constexpr int kSmemBytes = kStages * kStageBytes + 1024;  // + alignment slack
     // TMEM scale-factor slots: NVFP4 copies one slot per MMA (4 SFA columns
     // + 4 per 128 rows of B), MXFP8 one slot per k-tile (its atoms cover the
@@ -143,11 +145,17 @@ BSQ_DEV TileInfo tile_info(int64_t t, int64_t m_tiles, const GemmParams &p, cons
     return ti;
 }
 
-template <int FMT, int BN, int ACC, bool OUT_BF16, bool SWAP, bool GROUPED>
-__global__ void __launch_bounds__(320, 1)
+template <int FMT, int BN, int ACC, bool OUT_BF16, bool SWAP, bool GROUPED, int SPLITK = 1>
+__global__ void __launch_bounds__(320, SPLITK == 1 ? 1 : 2)
     gemm_bs_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const GemmParams p) {
-    using C_ = Cfg<FMT, BN>;
+    // SPLITK > 1: a cluster of SPLITK CTAs computes one tile, CTA r over the
+    // r-th of SPLITK equal runs of k-tiles; the partial sums meet in the
+    // rank-0 CTA (distributed shared memory) in rank order.  Three stages
+    // (86 KB) and 256 TMEM columns per CTA, so that two CTAs share an SM.
+    static_assert(SPLITK == 1 || (SWAP && BN == 64 && !GROUPED), "split-K: the skinny swap-AB tile only");
+    using C_ = Cfg<FMT, BN, SPLITK == 1 ? 8 : 3>;
+    constexpr int kTmemCols = SPLITK == 1 ? 512 : 256;
     using T = typename C_::T;
     constexpr int NS = C_::kStages;
     extern __shared__ uint8_t smem_raw[];
@@ -213,7 +221,7 @@ __global__ void __launch_bounds__(320, 1)
         }
     }
     if (warp == 1) {
-        tmem_alloc(smem_u32(&tmem_base_slot), 512);
+        tmem_alloc(smem_u32(&tmem_base_slot), kTmemCols);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -223,7 +231,18 @@ __global__ void __launch_bounds__(320, 1)
     if (GROUPED) total_tiles = tile_start[p.G];
 
     constexpr int SF_TMEM0 = ACC * BN;  // first TMEM column of the scale-factor slots
-    static_assert(ACC * BN + C_::kSlots * C_::kSlotCols <= 512, "TMEM budget");
+    static_assert(ACC * BN + C_::kSlots * C_::kSlotCols <= kTmemCols, "TMEM budget");
+    // this CTA's tiles and k-tiles (split-K: one tile per cluster, launched as
+    // tiles x SPLITK CTAs)
+    const uint32_t crank = SPLITK > 1 ? cluster_ctarank() : 0u;
+    const int64_t t_first = blockIdx.x / SPLITK, t_step = gridDim.x / SPLITK;
+    const int64_t kt_begin = k_tiles * crank / SPLITK, kt_end = k_tiles * (crank + 1) / SPLITK;
+
+    // split-K: what an epilogue thread carries from its drain to the reduction
+    uint32_t sk_part[SPLITK > 1 ? 32 : 1];
+    bool sk_have = false, sk_row_ok = false;
+    int64_t sk_ar = 0, sk_nb0 = 0;
+    float sk_alpha = 1.0f;
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
@@ -231,13 +250,13 @@ __global__ void __launch_bounds__(320, 1)
             int s = 0;
             uint32_t ph = 0, armed = 0, armed_par = 0;
             bool ok = true;
-            for (int64_t t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+            for (int64_t t = t_first; t < total_tiles && ok; t += t_step) {
                 TileInfo ti = tile_info<GROUPED>(t, m_tiles, p, tile_start, offs);
                 const int64_t nb0 = ti.n0 * BN;
                 const int64_t b_row0 = (int64_t)ti.group * p.NB + nb0;
                 const uint8_t *sfa_tile = p.sfA + (ti.sfa_row0 / 128) * KBT * 512;
                 const uint8_t *sfb_base = p.sfB + (int64_t)ti.group * p.sfB_group_bytes;
-                for (int64_t kt = 0; kt < k_tiles; kt++) {
+                for (int64_t kt = kt_begin; kt < kt_end; kt++) {
                     if (!mbar_wait(smem_u32(&empty_bar[s]), ph ^ 1u, &abort_flag, p.err, 1, kTimeoutNs)) {
                         ok = false;
                         break;
@@ -293,7 +312,7 @@ __global__ void __launch_bounds__(320, 1)
             bool issued = false;
             uint32_t ktc = 0;  // k-tiles issued: selects the scale slots
             int64_t it = 0;
-            for (int64_t t = blockIdx.x; t < total_tiles && ok; t += gridDim.x, it++) {
+            for (int64_t t = t_first; t < total_tiles && ok; t += t_step, it++) {
                 const int a = (int)(it % ACC);
                 const uint32_t aph = (uint32_t)((it / ACC) & 1);
                 if (!mbar_wait(smem_u32(&acce_bar[a]), aph ^ 1u, &abort_flag, p.err, 3, kTimeoutNs)) {
@@ -302,7 +321,7 @@ __global__ void __launch_bounds__(320, 1)
                 }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(a * BN);
-                for (int64_t kt = 0; kt < k_tiles; kt++, ktc++) {
+                for (int64_t kt = kt_begin; kt < kt_end; kt++, ktc++) {
                     if (!mbar_test_wait(smem_u32(&full_bar[s]), ph) &&
                         !mbar_wait(smem_u32(&full_bar[s]), ph, &abort_flag, p.err, 4, kTimeoutNs)) {
                         ok = false;
@@ -326,7 +345,7 @@ __global__ void __launch_bounds__(320, 1)
                             for (int r = 0; r < C_::kNbAtomTiles; r++)
                                 tmem_cp_sf_atom(slot + 4 + 4 * r, desc_pack(sfb_lo + kSfbTileLo * r + kSfAtomLo * j, kSfHi));
                             mma_nvfp4(d_tmem, desc_pack(a_lo + 2 * j, kOpHi), desc_pack(b_lo + 2 * j, kOpHi), idesc, slot,
-                                      slot + 4, (kt > 0 || j > 0) ? 1u : 0u);
+                                      slot + 4, (kt > kt_begin || j > 0) ? 1u : 0u);
                         };
                         if (full_kt) {
 #pragma unroll
@@ -352,7 +371,7 @@ __global__ void __launch_bounds__(320, 1)
                             const uint32_t id = 2u * (uint32_t)(j & 1), a = (uint32_t)(j >> 1);
                             mma_mxfp4(d_tmem, desc_pack(a_lo + 2 * j, kOpHi), desc_pack(b_lo + 2 * j, kOpHi),
                                       idesc | (id << 29) | (id << 4), (slot + 4 * a) | (id << 30),
-                                      (slot + kSfb0 + kSfbA * a) | (id << 30), (kt > 0 || j > 0) ? 1u : 0u);
+                                      (slot + kSfb0 + kSfbA * a) | (id << 30), (kt > kt_begin || j > 0) ? 1u : 0u);
                         };
                         if (full_kt) {
 #pragma unroll
@@ -372,7 +391,7 @@ __global__ void __launch_bounds__(320, 1)
                         auto issue = [&](int j) {
                             mma_mxfp8(d_tmem, desc_pack(a_lo + 2 * j, kOpHi), desc_pack(b_lo + 2 * j, kOpHi),
                                       idesc | ((uint32_t)j << 29) | ((uint32_t)j << 4), slot | ((uint32_t)j << 30),
-                                      (slot + 4) | ((uint32_t)j << 30), (kt > 0 || j > 0) ? 1u : 0u);
+                                      (slot + 4) | ((uint32_t)j << 30), (kt > kt_begin || j > 0) ? 1u : 0u);
                         };
                         if (full_kt) {
 #pragma unroll
@@ -405,7 +424,7 @@ __global__ void __launch_bounds__(320, 1)
         constexpr int HC = BN / 2;          // columns per warp
         const int row = 32 * q + lane;
         int64_t it = 0;
-        for (int64_t t = blockIdx.x; t < total_tiles; t += gridDim.x, it++) {
+        for (int64_t t = t_first; t < total_tiles; t += t_step, it++) {
             TileInfo ti = tile_info<GROUPED>(t, m_tiles, p, tile_start, offs);
             const int a = (int)(it % ACC);
             const uint32_t aph = (uint32_t)((it / ACC) & 1);
@@ -422,7 +441,28 @@ __global__ void __launch_bounds__(320, 1)
             const int64_t nb0 = ti.n0 * BN + half * HC;   // first column of this warp
             const int64_t n_lim = p.n_lim;
             const uint32_t tbase = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(a * BN + half * HC);
-            if (OUT_BF16 && ACC == 1) {
+            if constexpr (SPLITK > 1) {
+                // this CTA's partial sums (HC = 32 columns of one row), kept for the reduction
+                if (kt_begin < kt_end) {
+                    tmem_ld32(tbase, sk_part);
+                    tmem_ld_wait();
+                    tc_fence_before();
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 32; c++) sk_part[c] = 0u;  // no k-tile in this CTA's run
+                }
+                if (crank != 0) {
+                    float *red = reinterpret_cast<float *>(sA);  // the stages are no longer read
+#pragma unroll
+                    for (int c = 0; c < 32; c++) red[(half * HC + c) * 128 + row] = __uint_as_float(sk_part[c]);
+                }
+                sk_have = true;
+                sk_ar = ar;
+                sk_row_ok = row_ok;
+                sk_nb0 = nb0;
+                sk_alpha = alpha;
+                continue;
+            } else if (OUT_BF16 && ACC == 1) {
                 // drain this warp's columns into registers (two loads per wait),
                 // release the accumulator, then store
                 uint32_t pk[HC / 2];
@@ -534,11 +574,44 @@ __global__ void __launch_bounds__(320, 1)
             }
         }
     }
+    if constexpr (SPLITK > 1) {
+        // every thread of the cluster passes both barriers: the partials are
+        // in shared memory after the first, read by rank 0 before the second
+        __syncthreads();
+        cluster_sync();
+        if (crank == 0 && sk_have && sk_row_ok) {
+            const uint32_t red0 = smem_u32(sA);
+            const int half = (warp - 2) >> 2;
+            const int row = 32 * (warp & 3) + lane;
+            float v[32];
+#pragma unroll
+            for (int c = 0; c < 32; c++) v[c] = __uint_as_float(sk_part[c]);
+#pragma unroll 1
+            for (int r = 1; r < SPLITK; r++) {
+                const uint32_t peer = mapa(red0, (uint32_t)r);
+#pragma unroll
+                for (int c = 0; c < 32; c++)
+                    v[c] = __fadd_rn(v[c], ld_shared_cluster_f32(peer + 4u * (uint32_t)((half * 32 + c) * 128 + row)));
+            }
+            const int64_t n_lim = p.n_lim;
+#pragma unroll
+            for (int c = 0; c < 32; c++) {
+                const int64_t n = sk_nb0 + c;
+                if (n < n_lim) {
+                    const float y = __fmul_rn(sk_alpha, v[c]);
+                    if (OUT_BF16) static_cast<__nv_bfloat16 *>(p.C)[n * p.ldc + sk_ar] = __float2bfloat16_rn(y);
+                    else static_cast<float *>(p.C)[n * p.ldc + sk_ar] = y;
+                }
+            }
+        }
+        __syncwarp();
+        cluster_sync();
+    }
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, 512);
+        tmem_dealloc(tmem_base, kTmemCols);
     }
 }
 
@@ -1130,26 +1203,19 @@ void launch_timeout_probe(uint64_t timeout_ns, unsigned int *err, cudaStream_t s
 
 // ============================================================ host side
 // The dynamic shared-memory limit of a kernel is a per-device attribute:
-// set it once per (kernel, device), under a lock, and remember the outcome.
+// set it once per (kernel, device), under a lock; a success is remembered.
 int smem_attr_once(const void *kern, int bytes) {
-    struct Entry {
-        const void *kern;
-        int dev;
-        int status;
-    };
-    static std::mutex mu;
-    static Entry done[256];
-    static int ndone = 0;
+    static PerDeviceMemo<1024> done;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return BSQ_ERR_CUDA;
-    std::lock_guard<std::mutex> lk(mu);
-    for (int i = 0; i < ndone; i++)
-        if (done[i].kern == kern && done[i].dev == dev) return done[i].status;
-    const int st = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess
+    return done.get(
+        kern, dev,
+        [&] {
+            return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess
                        ? BSQ_OK
                        : BSQ_ERR_CUDA;
-    if (st == BSQ_OK && ndone < 256) done[ndone++] = {kern, dev, st};
-    return st;
+        },
+        [](int st) { return st == BSQ_OK; });
 }
 
 namespace {
@@ -1245,6 +1311,28 @@ int run(const CUtensorMap &ta, const CUtensorMap &tb, const GemmParams &p, int g
     return cudaGetLastError() == cudaSuccess ? BSQ_OK : BSQ_ERR_CUDA;
 }
 
+// The swap-AB kernel split over K: clusters of S CTAs, one tile per cluster.
+template <int FMT, bool OUT_BF16, int S>
+int run_splitk(const CUtensorMap &ta, const CUtensorMap &tb, const GemmParams &p, int64_t tiles, cudaStream_t s) {
+    using C_ = Cfg<FMT, 64, 3>;
+    auto kern = gemm_bs_kernel<FMT, 64, 2, OUT_BF16, true, false, S>;
+    if (smem_attr_once(reinterpret_cast<const void *>(kern), C_::kSmemBytes) != BSQ_OK) return BSQ_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(tiles * S), 1, 1);
+    cfg.blockDim = dim3(C_::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = C_::kSmemBytes;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = S;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, ta, tb, p) != cudaSuccess) return BSQ_ERR_CUDA;
+    return cudaGetLastError() == cudaSuccess ? BSQ_OK : BSQ_ERR_CUDA;
+}
+
 template <int FMT>
 int dispatch(const GemmArgs &g, cudaStream_t s) {
     using T = FmtTraits<FMT>;
@@ -1329,6 +1417,18 @@ int dispatch(const GemmArgs &g, cudaStream_t s) {
     else tiles = (MA / 128 + g.G) * ((NB + bn - 1) / bn);
     const int grid = (int)(tiles < g.num_sms ? (tiles < 1 ? 1 : tiles) : g.num_sms);
     if (swap) {
+        // Split K when the tiles leave SMs idle: two split-K CTAs share an SM
+        // (3 stages, 256 TMEM columns each), so S = 2, 4 or 8 is taken as
+        // long as tiles x S fits twice the SM count and every CTA keeps at
+        // least two k-tiles.  BSQ_KNOB_GEMM_SPLITK forces S (1: off).
+        const int64_t k_tiles = (g.K + T::kBkElems - 1) / T::kBkElems;
+        int S = 1;
+        while (S < 8 && tiles * (2 * S) <= 2LL * g.num_sms && k_tiles >= 2 * (2 * S)) S *= 2;
+        if (const int v = kernel_choice(BSQ_KNOB_GEMM_SPLITK); v > 0) S = v;
+        while (S > 1 && S > k_tiles) S /= 2;
+        if (S == 2) return g.out_bf16 ? run_splitk<FMT, true, 2>(ta, tb, p, tiles, s) : run_splitk<FMT, false, 2>(ta, tb, p, tiles, s);
+        if (S == 4) return g.out_bf16 ? run_splitk<FMT, true, 4>(ta, tb, p, tiles, s) : run_splitk<FMT, false, 4>(ta, tb, p, tiles, s);
+        if (S == 8) return g.out_bf16 ? run_splitk<FMT, true, 8>(ta, tb, p, tiles, s) : run_splitk<FMT, false, 8>(ta, tb, p, tiles, s);
         if (g.out_bf16) return run<FMT, 64, 2, true, true, false>(ta, tb, p, grid, s);
         return run<FMT, 64, 2, false, true, false>(ta, tb, p, grid, s);
     }

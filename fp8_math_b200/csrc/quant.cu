@@ -7,9 +7,9 @@
 // All of them stream bf16/fp8 from HBM with 16-byte vector loads, reduce the
 // block amax with warp shuffles, and write packed codes plus scale factors
 // directly in the swizzled layout the block-scaled MMA reads.
-#include <atomic>
 
 #include "common.cuh"
+#include "devcache.h"
 #include "nvfp4.cuh"
 #include "quant.cuh"
 #include "sm100.cuh"
@@ -1986,21 +1986,24 @@ static int grid_for(int64_t work_items, int per_block, int max_ctas) {
 
 // CTAs of `kernel` (256 threads, static shared memory only) that fit on the
 // device at once: the grid of the persistent streaming kernels is one full
-// wave, so no partial last wave leaves SMs idle.  Cached per kernel and
-// device (atomics, so concurrent first calls from several host threads are
-// defined; they compute the same value).
+// wave, so no partial last wave leaves SMs idle.  Kept per kernel and device.
+PerDeviceMemo<1024> g_occupancy;
+
+static int current_device() {
+    int dev = 0;
+    return cudaGetDevice(&dev) == cudaSuccess && dev >= 0 ? dev : 0;
+}
+
 template <auto Kern>
 static int resident_ctas(int num_sms) {
-    constexpr int kDevs = 64;
-    static std::atomic<int> per_sm[kDevs];
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kDevs) dev = 0;
-    int n = per_sm[dev].load(std::memory_order_relaxed);
-    if (n == 0) {
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, Kern, 256, 0) != cudaSuccess || n < 1) n = 1;
-        per_sm[dev].store(n, std::memory_order_relaxed);
-    }
-    return n * num_sms;
+    const int n = g_occupancy.get(
+        reinterpret_cast<const void *>(Kern), current_device(),
+        [] {
+            int v = 0;
+            return cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, Kern, 256, 0) == cudaSuccess ? v : 0;
+        },
+        [](int v) { return v >= 1; });
+    return (n < 1 ? 1 : n) * num_sms;
 }
 
 void launch_amax(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, bool rht, uint32_t mask,
@@ -2106,18 +2109,16 @@ int launch_quant_nvfp4_fused(const uint16_t *x, int64_t M, int64_t K, bool rht, 
 // included), per kernel and device.
 template <auto Kern>
 static int resident_stream(int num_sms) {
-    constexpr int kDevs = 64;
-    static std::atomic<int> per_sm[kDevs];
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kDevs) dev = 0;
-    int n = per_sm[dev].load(std::memory_order_relaxed);
-    if (n == 0) {
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, Kern, nvs::kThreads, nvs::kSmemBytes) != cudaSuccess ||
-            n < 1)
-            n = 1;
-        per_sm[dev].store(n, std::memory_order_relaxed);
-    }
-    return n * num_sms;
+    const int n = g_occupancy.get(
+        reinterpret_cast<const void *>(Kern), current_device(),
+        [] {
+            int v = 0;
+            return cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, Kern, nvs::kThreads, nvs::kSmemBytes) == cudaSuccess
+                       ? v
+                       : 0;
+        },
+        [](int v) { return v >= 1; });
+    return (n < 1 ? 1 : n) * num_sms;
 }
 
 template <int MODE, bool RHT, bool TWO_D>

@@ -74,8 +74,9 @@ enum {
     BSQ_KNOB_FUSED_QUANT = 0, /* 1/-1: amax + 16x16 quantize in one cooperative launch; 0: two passes */
     BSQ_KNOB_GEMM_PAIR = 1,   /* -1: automatic; 0: single-CTA GEMM; 1: CTA-pair GEMM where it applies */
     BSQ_KNOB_GEMM_BN = 2,     /* -1: automatic; 128 or 256 (bf16 output): the single-CTA GEMM's N tile */
-    BSQ_KNOB_STREAM_QUANT = 3 /* -1: bulk-copy streaming NVFP4 kernels for contiguous 16x16 tensors; 1: for every
-                                 contiguous amax / NVFP4 call; 0: never */
+    BSQ_KNOB_STREAM_QUANT = 3, /* -1: bulk-copy streaming NVFP4 kernels for contiguous 16x16 tensors; 1: for every
+                                  contiguous amax / NVFP4 call; 0: never */
+    BSQ_KNOB_GEMM_SPLITK = 4   /* -1: automatic; 1: off; 2, 4 or 8: the skinny (M <= 64) GEMM's K split */
 };
 
 /* Human-readable name of a status code (static string). */

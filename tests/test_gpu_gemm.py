@@ -77,6 +77,27 @@ def test_gemm_full_compare(ora, knobs, pair, fmt, M, N, K, out):
     assert_gemm_close(Cg, Cr, Ra, out == torch.bfloat16, f"gemm pair={pair} fmt={fmt} {M}x{N}x{K}")
 
 
+# the skinny (swap-AB) GEMM split over K: clusters of S CTAs, partial sums
+# added in the rank-0 CTA; S = 1 is the unsplit kernel, -1 the automatic
+# choice.  K runs that do not divide evenly (K / 256 = 7, 9), more CTAs than
+# k-tiles (clamped), several W tiles, ragged token and W-row counts.
+@pytest.mark.parametrize("split", [-1, 1, 2, 4, 8])
+@pytest.mark.parametrize("fmt", [NV, MX, MX4])
+@pytest.mark.parametrize("M,N,K,out", [
+    (64, 1024, 2048, torch.bfloat16),
+    (37, 400, 1792, torch.float32),
+    (8, 256, 2304, torch.bfloat16),
+    (64, 384, 512, torch.float32),
+])
+def test_gemm_splitk_compare(ora, knobs, split, fmt, M, N, K, out):
+    knobs(bsq.BSQ_KNOB_GEMM_SPLITK, split)
+    A, Bm = W.nvfp4_linear_small(M=M, N=N, K=K, seed=M * 5 + N + K)
+    qa, qb = oracle_operands(ora, fmt, A, Bm)
+    Cg = run_gemm(ora, fmt, qa, qb, M, N, K, out)
+    Cr, Ra = ora.gemm_f64(ora.dequant(fmt, *qa), ora.dequant(fmt, *qb))
+    assert_gemm_close(Cg, Cr, Ra, out == torch.bfloat16, f"split-K {split} fmt={fmt} {M}x{N}x{K}")
+
+
 def test_gemm_small_linear_workload_exact_inputs(ora):
     """NVFP4 linear, 128x256 (1x16) times 256x256 (16x16), fp32 output."""
     A, Wt = W.nvfp4_linear_small()

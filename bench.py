@@ -207,13 +207,16 @@ def reference_arm(args, rank):
 
 # ---------------------------------------------------------------------- per-row measurements
 def measure_rows(hbm, fp4_peak, fp8_peak, reps=10, only=None):
-    """Times every step of the hot path on its own workload at full size
-    (CUDA events around each call, median of `reps`).  Before each rep L2 is
-    flushed by writing a 256 MiB buffer and then reading another one: L2 is
-    write-back, so after the write alone up to 126 MB of dirty lines would be
-    written back to HBM inside the timed call; the read replaces them by
-    clean lines outside the timing.  Returns a list of dicts; a row that
-    fails records its error instead of stopping the bench."""
+    """Times every step of the hot path on its own workload at full size.
+    Each call runs on a cold L2: before it, L2 is flushed by writing a 256 MiB
+    buffer and then reading another one (L2 is write-back, so after the write
+    alone up to 126 MB of dirty lines would be written back inside the timed
+    call; the read replaces them by clean lines).  The CUDA event clock here
+    ticks in steps of about 2 us, too coarse for one short call, so a row's
+    time is a difference of two event-timed batches on the stream: `reps`
+    times (flush, call) minus `reps` times (flush), divided by `reps`, each
+    batch the median of three.  Returns a list of dicts; a row that fails
+    records its error instead of stopping the bench."""
     import torch
 
     from fp8_math_b200 import api, bsq
@@ -224,22 +227,28 @@ def measure_rows(hbm, fp4_peak, fp8_peak, reps=10, only=None):
     flush_r = torch.ones(64 << 20, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
 
+    def batch(fn, n):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n):
+            flush.zero_()
+            flush_r.sum()
+            if fn is not None:
+                fn()
+        e1.record(stream)
+        e1.synchronize()
+        return e0.elapsed_time(e1) * 1e3
+
     def timed(fn):
         for _ in range(3):
             fn()
-        ts = []
-        for _ in range(reps):
-            flush.zero_()
-            flush_r.sum()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            fn()
-            e1.record(stream)
-            e1.synchronize()
-            ts.append(e0.elapsed_time(e1) * 1e3)
+        with_fn, without = [], []
+        for _ in range(3):
+            with_fn.append(batch(fn, reps))
+            without.append(batch(None, reps))
         if bsq.bsq_check() != bsq.BSQ_OK:
             raise RuntimeError("device error")
-        return statistics.median(ts)
+        return max(statistics.median(with_fn) - statistics.median(without), 0.0) / reps
 
     rows = []
 
@@ -524,13 +533,15 @@ def main():
 
     # ---- per-kernel breakdown (events on the launching stream)
     def time_fn(fn, reps):
-        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
-        for e0, e1 in evs:
-            e0.record(stream)
+        # one event pair around `reps` back-to-back calls (the event clock
+        # ticks in ~2 us steps, too coarse for one call)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
             fn()
-            e1.record(stream)
+        e1.record(stream)
         torch.cuda.synchronize()
-        return [e0.elapsed_time(e1) for e0, e1 in evs]
+        return [e0.elapsed_time(e1) / reps]
 
     # ---- the timed region
     if world > 1:

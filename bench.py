@@ -256,11 +256,25 @@ def measure_rows(hbm, fp4_peak, fp8_peak, reps=10, only=None):
         """Whether any of these rows is selected (inputs are built only then)."""
         return only is None or any(only in n for n in names)
 
-    def row(name, workload, fn, nbytes=None, flops=None, peak_kind=None):
+    def looped(fn, n=50):
+        # n back-to-back calls between one event pair, no flush: the time per
+        # call of a loop, host launch overhead included when it is the bound
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n):
+            fn()
+        e1.record(stream)
+        e1.synchronize()
+        return e0.elapsed_time(e1) * 1e3 / n
+
+    def row(name, workload, fn, nbytes=None, flops=None, peak_kind=None, loop=False):
         if only and only not in name:
             return
         try:
-            us = timed(fn)
+            us = looped(fn) if loop else timed(fn)
             r = {"row": name, "workload": workload, "us": round(us, 2)}
             if flops is not None:
                 peak = fp4_peak if peak_kind == "fp4" else fp8_peak
@@ -305,7 +319,7 @@ def measure_rows(hbm, fp4_peak, fp8_peak, reps=10, only=None):
             lambda: api.gemm(0, qa[0], qa[1], qw[0], qw[1], M2, N2, K2, gsA=qa[2], gsB=qw[2], out=C2),
             flops=2 * M2 * N2 * K2, peak_kind="fp4")
         del y, C2
-    if wants("a2+a3+a8 small linear step (latency)"):
+    if wants("a2+a3+a8 small linear step (latency)", "a2+a3+a8 small linear step as one CUDA graph (latency)"):
         # -- the small NVFP4 linear, A 128x256, W 256x256 (latency)
         As, Ws = W.nvfp4_linear_small()
         As, Ws = As.to(dev), Ws.to(dev)
@@ -318,6 +332,25 @@ def measure_rows(hbm, fp4_peak, fp8_peak, reps=10, only=None):
             api.gemm(0, qas[0], qas[1], qws[0], qws[1], 128, 256, 256, gsA=qas[2], gsB=qws[2], out=Cs)
         row("a2+a3+a8 small linear step (latency)", "A 128x256, W 256x256, fp32 out", small_step,
             nbytes=(128 + 256) * 256 * 2)
+        if wants("a2+a3+a8 small linear step as one CUDA graph (latency)"):
+            # the same five launches captured once and replayed as one graph
+            side = torch.cuda.Stream()
+            side.wait_stream(stream)
+            with torch.cuda.stream(side):
+                small_step()
+            stream.wait_stream(side)
+            torch.cuda.synchronize()
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                small_step()
+            row("a2+a3+a8 small linear step as one CUDA graph (latency)", "A 128x256, W 256x256, fp32 out",
+                graph.replay, nbytes=(128 + 256) * 256 * 2)
+            # in a loop the host's launch work sets the pace of the eager calls
+            row("a2+a3+a8 small linear step as one CUDA graph (latency), 50 in a loop",
+                "A 128x256, W 256x256, fp32 out; per step", graph.replay, nbytes=(128 + 256) * 256 * 2, loop=True)
+            row("a2+a3+a8 small linear step (latency), 50 eager calls in a loop", "A 128x256, W 256x256, fp32 out; per step",
+                small_step, nbytes=(128 + 256) * 256 * 2, loop=True)
+            del graph
     if wants("a6 MXFP8 row quantize RNE", "a6 MXFP8 row quantize SR (Philox)", "a7 requant-transpose SR",
              "f3 MXFP4 quantize RNE (next row)", "f3 MXFP4 quantize SR (next row)"):
         # -- MXFP8 4096x4096 Student-t: RNE and SR, requant-transpose

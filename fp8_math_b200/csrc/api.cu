@@ -138,8 +138,15 @@ int bsq_amax(const void *x, int64_t M, int64_t K, int64_t ldx, int rht_enable, u
 
 // The fused amax + quantize kernel can be switched off
 // (bsq_debug_kernel_choice(BSQ_KNOB_FUSED_QUANT, 0)) for tuning and for
-// tests of the two-pass path.
-static bool fused_enabled() { return bsq::kernel_choice(BSQ_KNOB_FUSED_QUANT) != 0; }
+// tests of the two-pass path.  It is a cooperative launch with a grid
+// barrier; while the stream is being captured into a CUDA graph the two
+// passes are launched instead (same bytes), so that a graph holds only
+// ordinary kernel nodes.
+static bool fused_enabled(cudaStream_t s) {
+    cudaStreamCaptureStatus st = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(s, &st) == cudaSuccess && st != cudaStreamCaptureStatusNone) return false;
+    return bsq::kernel_choice(BSQ_KNOB_FUSED_QUANT) != 0;
+}
 // The bulk-copy streaming kernels for contiguous tensors: by default for
 // 16x16 blocks only (on 14336x4096 with the RHT they measure 71.7 us against
 // 75.8 for the register-streaming fused kernel; on 8192x4096 with 1x16
@@ -182,7 +189,7 @@ int bsq_quant_nvfp4(const void *x, int64_t M, int64_t K, int64_t ldx, int block_
         if (streamable) {
             unsigned int *scratch = reinterpret_cast<unsigned int *>(codes);
             int rc;
-            if (fused_enabled()) {
+            if (fused_enabled(s)) {
                 // amax and quantize in one cooperative launch
                 rc = bsq::launch_nvfp4_stream(2, xx, M, K, block_2d != 0, rht_enable != 0, mask, scratch, scratch + 1,
                                               nullptr, false, gs, codes, sf, d->err, d->num_sms, s);
@@ -200,7 +207,7 @@ int bsq_quant_nvfp4(const void *x, int64_t M, int64_t K, int64_t ldx, int block_
         // on 8192x4096, where the fused kernel's lower occupancy outweighs the
         // L2 reuse; 16x16 tensors gain: 70.9 vs 74.5 us on 14336x4096)
         (void)KB;
-        const bool fusable = !row_index && G == 0 && ldx == K && !four_over_six && block_2d && fused_enabled();
+        const bool fusable = !row_index && G == 0 && ldx == K && !four_over_six && block_2d && fused_enabled(s);
         if (fusable) {
             // amax and quantize in one cooperative kernel
             if (bsq::launch_quant_nvfp4_fused(xx, M, K, rht_enable != 0, mask, gs, codes, sf, d->err, d->num_sms,

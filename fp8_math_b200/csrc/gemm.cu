@@ -239,9 +239,8 @@ __global__ void __launch_bounds__(320, SPLITK == 1 ? 1 : 2)
     const int64_t kt_begin = k_tiles * crank / SPLITK, kt_end = k_tiles * (crank + 1) / SPLITK;
 
     // split-K: what an epilogue thread carries from its drain to the reduction
-    uint32_t sk_part[SPLITK > 1 ? 32 : 1];
-    bool sk_have = false, sk_row_ok = false;
-    int64_t sk_ar = 0, sk_nb0 = 0;
+    bool sk_have = false;
+    int64_t sk_a_row0 = 0, sk_m_lim = 0, sk_n0 = 0;
     float sk_alpha = 1.0f;
 
     if (warp == 0) {
@@ -442,25 +441,28 @@ __global__ void __launch_bounds__(320, SPLITK == 1 ? 1 : 2)
             const int64_t n_lim = p.n_lim;
             const uint32_t tbase = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(a * BN + half * HC);
             if constexpr (SPLITK > 1) {
-                // this CTA's partial sums (HC = 32 columns of one row), kept for the reduction
+                // this CTA's partial sums (HC = 32 columns of one row) into its
+                // shared memory, column-major [64][128]: the stages are no longer read
+                uint32_t part[32];
                 if (kt_begin < kt_end) {
-                    tmem_ld32(tbase, sk_part);
+                    tmem_ld32(tbase, part);
                     tmem_ld_wait();
                     tc_fence_before();
                 } else {
 #pragma unroll
-                    for (int c = 0; c < 32; c++) sk_part[c] = 0u;  // no k-tile in this CTA's run
+                    for (int c = 0; c < 32; c++) part[c] = 0u;  // no k-tile in this CTA's run
                 }
-                if (crank != 0) {
-                    float *red = reinterpret_cast<float *>(sA);  // the stages are no longer read
+                float *red = reinterpret_cast<float *>(sA);
 #pragma unroll
-                    for (int c = 0; c < 32; c++) red[(half * HC + c) * 128 + row] = __uint_as_float(sk_part[c]);
-                }
+                for (int c = 0; c < 32; c++) red[(half * HC + c) * 128 + row] = __uint_as_float(part[c]);
                 sk_have = true;
-                sk_ar = ar;
-                sk_row_ok = row_ok;
-                sk_nb0 = nb0;
+                sk_a_row0 = ti.a_row0;
+                sk_m_lim = ti.m_lim;
+                sk_n0 = ti.n0 * BN;
                 sk_alpha = alpha;
+                (void)row_ok;
+                (void)nb0;
+                (void)n_lim;
                 continue;
             } else if (OUT_BF16 && ACC == 1) {
                 // drain this warp's columns into registers (two loads per wait),
@@ -579,32 +581,42 @@ __global__ void __launch_bounds__(320, SPLITK == 1 ? 1 : 2)
         // in shared memory after the first, read by rank 0 before the second
         __syncthreads();
         cluster_sync();
-        if (crank == 0 && sk_have && sk_row_ok) {
+        if (sk_have) {
+            // CTA r reduces rows [r R, r R + R) of the tile, R = 128 / SPLITK:
+            // element e of its slice is column e / R, row r R + e % R (consecutive
+            // threads on consecutive rows: conflict-free shared reads, adjacent
+            // output addresses).  Each thread's 32 / SPLITK elements: all
+            // 32 partials are loaded first (independent remote loads in flight
+            // together), then added in rank order 0, 1, ...
+            constexpr int R = 128 / SPLITK, PER = 32 / SPLITK;
+            const int t = threadIdx.x - 64;  // the 256 epilogue threads
             const uint32_t red0 = smem_u32(sA);
-            const int half = (warp - 2) >> 2;
-            const int row = 32 * (warp & 3) + lane;
-            float v[32];
+            uint32_t base[SPLITK];
 #pragma unroll
-            for (int c = 0; c < 32; c++) v[c] = __uint_as_float(sk_part[c]);
-#pragma unroll 1
-            for (int r = 1; r < SPLITK; r++) {
-                const uint32_t peer = mapa(red0, (uint32_t)r);
+            for (int r = 0; r < SPLITK; r++) base[r] = mapa(red0, (uint32_t)r);
+            float v[SPLITK][PER];
 #pragma unroll
-                for (int c = 0; c < 32; c++)
-                    v[c] = __fadd_rn(v[c], ld_shared_cluster_f32(peer + 4u * (uint32_t)((half * 32 + c) * 128 + row)));
+            for (int i = 0; i < PER; i++) {
+                const int e = t + 256 * i, col = e / R, row = (int)crank * R + e % R;
+#pragma unroll
+                for (int r = 0; r < SPLITK; r++) v[r][i] = ld_shared_cluster_f32_nv(base[r] + 4u * (uint32_t)(col * 128 + row));
             }
             const int64_t n_lim = p.n_lim;
 #pragma unroll
-            for (int c = 0; c < 32; c++) {
-                const int64_t n = sk_nb0 + c;
-                if (n < n_lim) {
-                    const float y = __fmul_rn(sk_alpha, v[c]);
-                    if (OUT_BF16) static_cast<__nv_bfloat16 *>(p.C)[n * p.ldc + sk_ar] = __float2bfloat16_rn(y);
-                    else static_cast<float *>(p.C)[n * p.ldc + sk_ar] = y;
+            for (int i = 0; i < PER; i++) {
+                const int e = t + 256 * i, col = e / R, row = (int)crank * R + e % R;
+                float sum = v[0][i];
+#pragma unroll
+                for (int r = 1; r < SPLITK; r++) sum = __fadd_rn(sum, v[r][i]);
+                const int64_t ar = sk_a_row0 + row, n = sk_n0 + col;
+                if (ar < sk_m_lim && n < n_lim) {
+                    const float y = __fmul_rn(sk_alpha, sum);
+                    if (OUT_BF16) static_cast<__nv_bfloat16 *>(p.C)[n * p.ldc + ar] = __float2bfloat16_rn(y);
+                    else static_cast<float *>(p.C)[n * p.ldc + ar] = y;
                 }
             }
         }
-        __syncwarp();
+        __syncthreads();
         cluster_sync();
     }
     tc_fence_before();

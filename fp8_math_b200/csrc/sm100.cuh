@@ -298,10 +298,12 @@ BSQ_DEV uint32_t mapa(uint32_t saddr, uint32_t rank) {
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
     return r;
 }
-// 32-bit load from a shared::cluster address (another CTA's shared memory)
-BSQ_DEV float ld_shared_cluster_f32(uint32_t caddr) {
+// 32-bit load from a shared::cluster address (another CTA's shared memory),
+// for data published before a cluster barrier: a plain load the compiler may
+// schedule freely after that barrier, so that many are in flight at once
+BSQ_DEV float ld_shared_cluster_f32_nv(uint32_t caddr) {
     float v;
-    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(caddr) : "memory");
+    asm("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(caddr));
     return v;
 }
 BSQ_DEV void mbar_arrive_cluster(uint32_t remote_bar) {

@@ -39,6 +39,14 @@
  *  - Behaviour is selected by the arguments alone; the library reads no
  *    environment variable.  bsq_debug_kernel_choice() can force one of two
  *    equivalent kernels for tests and tuning (results are identical).
+ *  - CUDA graphs: the quantize and GEMM entry points may be called on a
+ *    stream under capture once the same calls have run once outside capture
+ *    on that device (the first call creates the per-device error word and
+ *    sets kernel attributes).  Under capture an amax + quantize pair is
+ *    recorded as two ordinary kernels instead of one cooperative launch;
+ *    the bytes are the same.  The GEMM's tensor maps are encoded at call
+ *    time from the pointers given, so a replayed graph uses those buffers.
+ *    bsq_check() synchronizes and may not be called under capture.
  */
 #ifndef BSQ_H
 #define BSQ_H

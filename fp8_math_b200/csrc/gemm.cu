@@ -53,6 +53,7 @@ struct GemmParams {
     const float *q_sg;    // the global scale the output is quantized with
     unsigned int *q_amax; // atomicMax of the bits of max |bf16 output| (NULL: not kept)
     int q_fos;            // Four Over Six block scales
+    int c_tma;            // skinny bf16 output through shared memory and one TMA tile store
 };
 
 template <int FMT>
@@ -94,7 +95,10 @@ struct Cfg {
     static constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
     static constexpr int kFit = (220 * 1024) / kStageBytes;
     static constexpr int kStages = kFit > MAXNS ? MAXNS : kFit;
-    static constexpr int kSmemBytes = kStages * kStageBytes + 1024;  // + alignment slack
+    // skinny (BN = 64) bf16 output staged for one TMA tile store: 64 x 128
+    static constexpr int kStagingOff = kStages * kStageBytes;
+    static constexpr int kStagingBytes = BN == 64 ? 64 * 128 * 2 : 0;
+    static constexpr int kSmemBytes = kStagingOff + kStagingBytes + 1024;  // + alignment slack
     // TMEM scale-factor slots: NVFP4 copies one slot per MMA (4 SFA columns
     // + 4 per 128 rows of B), MXFP8 one slot per k-tile (its atoms cover the
     // 4 MMAs of the k-tile, selected by the scale-factor id)
@@ -104,7 +108,8 @@ struct Cfg {
     static constexpr int kSlots = (FMT == BSQ_NVFP4) ? 16 : 8;
     static constexpr int kMmaPerKt = T::kBkElems / T::kMmaK;  // 4
     static constexpr int kEpiWarps = 8;
-    static constexpr int kThreads = 32 * (2 + kEpiWarps);
+    // two more warps: the scale copiers of the skinny NVFP4 kernel (idle elsewhere)
+    static constexpr int kThreads = 32 * (2 + kEpiWarps + 2);
 };
 
 // Tile -> (group, m tile, n tile) for the persistent loop.
@@ -146,9 +151,9 @@ BSQ_DEV TileInfo tile_info(int64_t t, int64_t m_tiles, const GemmParams &p, cons
 }
 
 template <int FMT, int BN, int ACC, bool OUT_BF16, bool SWAP, bool GROUPED, int SPLITK = 1>
-__global__ void __launch_bounds__(320, SPLITK == 1 ? 1 : 2)
+__global__ void __launch_bounds__(384, SPLITK == 1 ? 1 : 2)
     gemm_bs_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const GemmParams p) {
+                   const __grid_constant__ CUtensorMap tmC, const GemmParams p) {
     // SPLITK > 1: a cluster of SPLITK CTAs computes one tile, CTA r over the
     // r-th of SPLITK equal runs of k-tiles; the partial sums meet in the
     // rank-0 CTA (distributed shared memory) in rank order.  Three stages
@@ -158,8 +163,17 @@ __global__ void __launch_bounds__(320, SPLITK == 1 ? 1 : 2)
     constexpr int kTmemCols = SPLITK == 1 ? 512 : 256;
     using T = typename C_::T;
     constexpr int NS = C_::kStages;
+    // Skinny NVFP4 (swap-AB): the tiny MMAs leave the MMA thread bound by its
+    // own tcgen05 issue (8 scale copies + 4 MMAs + a commit per k-tile), so two
+    // copier threads (warps 10 and 11) copy the SFA and SFB atoms of each
+    // stage into that stage's own TMEM slots and commit to sfa_bar / sfb_bar;
+    // the MMA thread issues only MMAs.  A stage's slots are free whenever its
+    // smem is: the producer refills a stage only after its MMAs completed.
+    constexpr bool COPIERS = FMT == BSQ_NVFP4 && SWAP;
     extern __shared__ uint8_t smem_raw[];
     __shared__ __align__(8) uint64_t full_bar[NS], empty_bar[NS], accf_bar[ACC], acce_bar[ACC], drain_bar;
+    __shared__ __align__(8) uint64_t sfa_bar[COPIERS ? NS : 1], sfb_bar[COPIERS ? NS : 1];
+    __shared__ __align__(8) uint64_t stg_full, stg_free;  // skinny bf16 output staging (p.c_tma)
     __shared__ uint32_t tmem_base_slot;
     __shared__ volatile int abort_flag;
     __shared__ int tile_start[GROUPED ? 1025 : 1];
@@ -187,6 +201,13 @@ __global__ void __launch_bounds__(320, SPLITK == 1 ? 1 : 2)
             mbar_init(smem_u32(&acce_bar[i]), C_::kEpiWarps);
         }
         mbar_init(smem_u32(&drain_bar), 1);
+        mbar_init(smem_u32(&stg_full), C_::kEpiWarps);
+        mbar_init(smem_u32(&stg_free), 1);
+        if (COPIERS)
+            for (int i = 0; i < NS; i++) {
+                mbar_init(smem_u32(&sfa_bar[i]), 1);
+                mbar_init(smem_u32(&sfb_bar[i]), 1);
+            }
         abort_flag = 0;
         fence_barrier_init();
     }
@@ -232,6 +253,7 @@ __global__ void __launch_bounds__(320, SPLITK == 1 ? 1 : 2)
 
     constexpr int SF_TMEM0 = ACC * BN;  // first TMEM column of the scale-factor slots
     static_assert(ACC * BN + C_::kSlots * C_::kSlotCols <= kTmemCols, "TMEM budget");
+    static_assert(!COPIERS || ACC * BN + NS * C_::kMmaPerKt * C_::kSlotCols <= kTmemCols, "TMEM budget (copiers)");
     // this CTA's tiles and k-tiles (split-K: one tile per cluster, launched as
     // tiles x SPLITK CTAs)
     const uint32_t crank = SPLITK > 1 ? cluster_ctarank() : 0u;
@@ -326,6 +348,15 @@ __global__ void __launch_bounds__(320, SPLITK == 1 ? 1 : 2)
                         ok = false;
                         break;
                     }
+                    if constexpr (COPIERS) {  // this stage's scale atoms are in its TMEM slots
+                        if (!(mbar_test_wait(smem_u32(&sfa_bar[s]), ph) ||
+                              mbar_wait(smem_u32(&sfa_bar[s]), ph, &abort_flag, p.err, 9, kTimeoutNs)) ||
+                            !(mbar_test_wait(smem_u32(&sfb_bar[s]), ph) ||
+                              mbar_wait(smem_u32(&sfb_bar[s]), ph, &abort_flag, p.err, 10, kTimeoutNs))) {
+                            ok = false;
+                            break;
+                        }
+                    }
                     tc_fence_after();
                     const uint32_t a_lo = a_lo0 + (uint32_t)s * (C_::kABytes >> 4);
                     const uint32_t b_lo = b_lo0 + (uint32_t)s * (C_::kBBytes >> 4);
@@ -336,13 +367,18 @@ __global__ void __launch_bounds__(320, SPLITK == 1 ? 1 : 2)
                     const int nmma = full_kt ? C_::kMmaPerKt : (int)(krem / T::kMmaK);
                     if (FMT == BSQ_NVFP4) {
                         // four slots per k-tile, one per MMA: its SFA atom, then one atom per 128 rows of B
-                        const uint32_t slot0 = sf_t0 + (ktc & (C_::kSlots / 4 - 1)) * (4 * C_::kSlotCols);
+                        // (with copiers: the stage's own slots, already filled)
+                        const uint32_t slot0 = COPIERS ? sf_t0 + (uint32_t)s * (4 * C_::kSlotCols)
+                                                       : sf_t0 + (ktc & (C_::kSlots / 4 - 1)) * (4 * C_::kSlotCols);
                         auto issue = [&](int j) {
                             const uint32_t slot = slot0 + (uint32_t)j * C_::kSlotCols;
-                            tmem_cp_sf_atom(slot, desc_pack(sfa_lo + kSfAtomLo * j, kSfHi));
+                            if constexpr (!COPIERS) {
+                                tmem_cp_sf_atom(slot, desc_pack(sfa_lo + kSfAtomLo * j, kSfHi));
 #pragma unroll
-                            for (int r = 0; r < C_::kNbAtomTiles; r++)
-                                tmem_cp_sf_atom(slot + 4 + 4 * r, desc_pack(sfb_lo + kSfbTileLo * r + kSfAtomLo * j, kSfHi));
+                                for (int r = 0; r < C_::kNbAtomTiles; r++)
+                                    tmem_cp_sf_atom(slot + 4 + 4 * r,
+                                                    desc_pack(sfb_lo + kSfbTileLo * r + kSfAtomLo * j, kSfHi));
+                            }
                             mma_nvfp4(d_tmem, desc_pack(a_lo + 2 * j, kOpHi), desc_pack(b_lo + 2 * j, kOpHi), idesc, slot,
                                       slot + 4, (kt > kt_begin || j > 0) ? 1u : 0u);
                         };
@@ -416,7 +452,7 @@ __global__ void __launch_bounds__(320, SPLITK == 1 ? 1 : 2)
                 mbar_wait(smem_u32(&drain_bar), 0, &never, p.err, 5, kTimeoutNs);
             }
         }
-    } else {
+    } else if (warp < 2 + C_::kEpiWarps) {
         // ------------------------------------------------------------ epilogue
         const int q = warp & 3;             // TMEM lane quarter this warp may access
         const int half = (warp - 2) >> 2;   // which half of the tile's columns
@@ -460,6 +496,40 @@ __global__ void __launch_bounds__(320, SPLITK == 1 ? 1 : 2)
                 sk_m_lim = ti.m_lim;
                 sk_n0 = ti.n0 * BN;
                 sk_alpha = alpha;
+                (void)row_ok;
+                (void)nb0;
+                (void)n_lim;
+                continue;
+            } else if (SWAP && OUT_BF16 && SPLITK == 1 && p.c_tma) {
+                // the tile as bf16 into the staging buffer [64 tokens][128 W rows],
+                // written out by one TMA tile store (clipped at C's edges)
+                uint32_t r[32];
+                tmem_ld32(tbase, r);
+                tmem_ld_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&acce_bar[a]));
+                // the previous tile's store has finished reading the buffer
+                if (it > 0 &&
+                    !mbar_wait(smem_u32(&stg_free), (uint32_t)((it - 1) & 1), &abort_flag, p.err, 13, kTimeoutNs))
+                    break;
+                uint16_t *stg = reinterpret_cast<uint16_t *>(smem + C_::kStagingOff);
+#pragma unroll
+                for (int j = 0; j < 32; j++) {
+                    const __nv_bfloat16 h = __float2bfloat16_rn(__fmul_rn(alpha, __uint_as_float(r[j])));
+                    stg[(half * HC + j) * 128 + row] = *reinterpret_cast<const uint16_t *>(&h);
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&stg_full));
+                if (threadIdx.x == 64) {
+                    if (mbar_wait(smem_u32(&stg_full), (uint32_t)(it & 1), &abort_flag, p.err, 14, kTimeoutNs)) {
+                        tma_store_2d(&tmC, smem_u32(stg), (int32_t)ti.a_row0, (int32_t)(ti.n0 * BN));
+                        bulk_commit();
+                        bulk_wait_read<0>();
+                    }
+                    mbar_arrive(smem_u32(&stg_free));
+                }
                 (void)row_ok;
                 (void)nb0;
                 (void)n_lim;
@@ -573,6 +643,64 @@ __global__ void __launch_bounds__(320, SPLITK == 1 ? 1 : 2)
                             }
                     }
                 }
+            }
+        }
+        // every TMA store of the staged tiles has completed before the CTA exits
+        if (SWAP && OUT_BF16 && SPLITK == 1 && p.c_tma && threadIdx.x == 64) bulk_wait<0>();
+    } else if constexpr (COPIERS) {
+        // ------------------------------------------------------------ scale copiers
+        // warp 10: SFA atoms, warp 11: SFB atoms; each walks the same tiles and
+        // k-tiles as the MMA thread, waits for the stage's data, copies the
+        // atoms of its MMAs into the stage's slots and commits to its barrier
+        if (lane == 0) {
+            const bool sfa_side = warp == 2 + C_::kEpiWarps;
+            constexpr uint32_t kSfHi = smem_desc_hi(128, 0);   // scale atoms: 32 rows of 16 bytes
+            constexpr uint32_t kSfAtomLo = 512 >> 4;
+            constexpr uint32_t kSfbTileLo = C_::kSfaBytes >> 4;
+            const uint32_t sfa_lo0 = smem_desc_lo(smem_u32(sSFA), 0), sfb_lo0 = smem_desc_lo(smem_u32(sSFB), 0);
+            const uint32_t sf_t0 = tmem_base + SF_TMEM0;
+            uint64_t *bars = sfa_side ? sfa_bar : sfb_bar;
+            int s = 0;
+            uint32_t ph = 0;
+            int last = -1;
+            uint32_t last_ph = 0;
+            bool ok = true;
+            for (int64_t t = t_first; t < total_tiles && ok; t += t_step) {
+                for (int64_t kt = kt_begin; kt < kt_end; kt++) {
+                    if (!mbar_test_wait(smem_u32(&full_bar[s]), ph) &&
+                        !mbar_wait(smem_u32(&full_bar[s]), ph, &abort_flag, p.err, 11, kTimeoutNs)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const int64_t krem = p.K - kt * T::kBkElems;
+                    const int nmma = krem >= T::kBkElems ? C_::kMmaPerKt : (int)(krem / T::kMmaK);
+                    const uint32_t slot0 = sf_t0 + (uint32_t)s * (4 * C_::kSlotCols);
+                    if (sfa_side) {
+                        const uint32_t lo = sfa_lo0 + (uint32_t)s * (C_::kSfaBytes >> 4);
+                        for (int j = 0; j < nmma; j++)
+                            tmem_cp_sf_atom(slot0 + (uint32_t)j * C_::kSlotCols, desc_pack(lo + kSfAtomLo * j, kSfHi));
+                    } else {
+                        const uint32_t lo = sfb_lo0 + (uint32_t)s * (C_::kSfbBytes >> 4);
+                        for (int j = 0; j < nmma; j++)
+#pragma unroll
+                            for (int r = 0; r < C_::kNbAtomTiles; r++)
+                                tmem_cp_sf_atom(slot0 + (uint32_t)j * C_::kSlotCols + 4 + 4 * r,
+                                                desc_pack(lo + kSfbTileLo * r + kSfAtomLo * j, kSfHi));
+                    }
+                    tc_commit(smem_u32(&bars[s]));
+                    last = s;
+                    last_ph = ph;
+                    if (++s == NS) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
+                }
+            }
+            // this thread's copies have executed before the CTA frees TMEM
+            if (last >= 0) {
+                volatile int never = 0;
+                mbar_wait(smem_u32(&bars[last]), last_ph, &never, p.err, 12, kTimeoutNs);
             }
         }
     }
@@ -1292,6 +1420,20 @@ bool make_c_tmap(CUtensorMap *m, void *C, bool bf16, int64_t n_cols, int64_t row
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// bf16 C [rows][ld] seen as (n_cols x rows) tiles of box_cols x box_rows,
+// no swizzle (the staging tile is plain row-major)
+bool make_c_tmap_box(CUtensorMap *m, void *C, int64_t n_cols, int64_t rows, int64_t ldc, int box_cols, int box_rows) {
+    EncodeFn enc = get_encode();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)n_cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)(ldc * 2)};
+    cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1u, 1u};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, C, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+           CUDA_SUCCESS;
+}
+
 template <int FMT, bool OUT_BF16, bool GROUPED, bool QOUT = false>
 int run_pair(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &tsa, const CUtensorMap &tsb,
              const CUtensorMap &tc, const GemmParams &p, int pairs, cudaStream_t s) {
@@ -1315,11 +1457,12 @@ int run_pair(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &ts
 }
 
 template <int FMT, int BN, int ACC, bool OUT_BF16, bool SWAP, bool GROUPED>
-int run(const CUtensorMap &ta, const CUtensorMap &tb, const GemmParams &p, int grid, cudaStream_t s) {
+int run(const CUtensorMap &ta, const CUtensorMap &tb, const GemmParams &p, int grid, cudaStream_t s,
+        const CUtensorMap *tc = nullptr) {
     using C_ = Cfg<FMT, BN>;
     auto kern = gemm_bs_kernel<FMT, BN, ACC, OUT_BF16, SWAP, GROUPED>;
     if (smem_attr_once(reinterpret_cast<const void *>(kern), C_::kSmemBytes) != BSQ_OK) return BSQ_ERR_CUDA;
-    kern<<<grid, C_::kThreads, C_::kSmemBytes, s>>>(ta, tb, p);
+    kern<<<grid, C_::kThreads, C_::kSmemBytes, s>>>(ta, tb, tc ? *tc : ta, p);
     return cudaGetLastError() == cudaSuccess ? BSQ_OK : BSQ_ERR_CUDA;
 }
 
@@ -1341,7 +1484,7 @@ int run_splitk(const CUtensorMap &ta, const CUtensorMap &tb, const GemmParams &p
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, kern, ta, tb, p) != cudaSuccess) return BSQ_ERR_CUDA;
+    if (cudaLaunchKernelEx(&cfg, kern, ta, tb, ta, p) != cudaSuccess) return BSQ_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? BSQ_OK : BSQ_ERR_CUDA;
 }
 
@@ -1432,16 +1575,29 @@ int dispatch(const GemmArgs &g, cudaStream_t s) {
         // Split K when the tiles leave SMs idle: two split-K CTAs share an SM
         // (3 stages, 256 TMEM columns each), so S = 2, 4 or 8 is taken as
         // long as tiles x S fits twice the SM count and every CTA keeps at
-        // least two k-tiles.  BSQ_KNOB_GEMM_SPLITK forces S (1: off).
+        // least two k-tiles.  Not for NVFP4, whose unsplit kernel has the
+        // scale-copier threads: on 64x14336x4096 it measures 15.9 us against
+        // 16.7 split in two (MXFP4: 18.3 unsplit, 16.0 split).
+        // BSQ_KNOB_GEMM_SPLITK forces S (1: off).
         const int64_t k_tiles = (g.K + T::kBkElems - 1) / T::kBkElems;
         int S = 1;
-        while (S < 8 && tiles * (2 * S) <= 2LL * g.num_sms && k_tiles >= 2 * (2 * S)) S *= 2;
+        while (FMT != BSQ_NVFP4 && S < 8 && tiles * (2 * S) <= 2LL * g.num_sms && k_tiles >= 2 * (2 * S)) S *= 2;
         if (const int v = kernel_choice(BSQ_KNOB_GEMM_SPLITK); v > 0) S = v;
         while (S > 1 && S > k_tiles) S /= 2;
         if (S == 2) return g.out_bf16 ? run_splitk<FMT, true, 2>(ta, tb, p, tiles, s) : run_splitk<FMT, false, 2>(ta, tb, p, tiles, s);
         if (S == 4) return g.out_bf16 ? run_splitk<FMT, true, 4>(ta, tb, p, tiles, s) : run_splitk<FMT, false, 4>(ta, tb, p, tiles, s);
         if (S == 8) return g.out_bf16 ? run_splitk<FMT, true, 8>(ta, tb, p, tiles, s) : run_splitk<FMT, false, 8>(ta, tb, p, tiles, s);
-        if (g.out_bf16) return run<FMT, 64, 2, true, true, false>(ta, tb, p, grid, s);
+        if (g.out_bf16) {
+            // the bf16 tile goes out as one TMA store ([tokens][W rows] of C)
+            // when C's base and row stride suit TMA
+            CUtensorMap tc;
+            if ((reinterpret_cast<uintptr_t>(g.C) % 16) == 0 && (g.ldc * 2) % 16 == 0 &&
+                make_c_tmap_box(&tc, g.C, MA, NB, g.ldc, 128, 64)) {
+                p.c_tma = 1;
+                return run<FMT, 64, 2, true, true, false>(ta, tb, p, grid, s, &tc);
+            }
+            return run<FMT, 64, 2, true, true, false>(ta, tb, p, grid, s);
+        }
         return run<FMT, 64, 2, false, true, false>(ta, tb, p, grid, s);
     }
     if (grouped) {

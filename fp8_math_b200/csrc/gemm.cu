@@ -463,14 +463,14 @@ __global__ void __launch_bounds__(384, SPLITK == 1 ? 1 : 2)
             TileInfo ti = tile_info<GROUPED>(t, m_tiles, p, tile_start, offs);
             const int a = (int)(it % ACC);
             const uint32_t aph = (uint32_t)((it / ACC) & 1);
-            if (!mbar_wait(smem_u32(&accf_bar[a]), aph, &abort_flag, p.err, 6, kTimeoutNs)) break;
-            tc_fence_after();
-            float alpha = 1.0f;
+            float alpha = 1.0f;  // read before the wait: off the drain's critical path
             if (FMT == BSQ_NVFP4) {
                 const float ga = p.gsA ? __ldg(p.gsA) : 1.0f;
                 const float gb = p.gsB ? __ldg(p.gsB + ti.group) : 1.0f;
                 alpha = __fmul_rn(ga, gb);
             }
+            if (!mbar_wait(smem_u32(&accf_bar[a]), aph, &abort_flag, p.err, 6, kTimeoutNs)) break;
+            tc_fence_after();
             const int64_t ar = ti.a_row0 + row;           // operand-A row of this thread
             const bool row_ok = ar < ti.m_lim;
             const int64_t nb0 = ti.n0 * BN + half * HC;   // first column of this warp
@@ -1169,14 +1169,14 @@ __global__ void __launch_bounds__(448, 1)
             int64_t a_row0, sfa_row0, m_lim, nt;
             int group;
             info(t, a_row0, sfa_row0, m_lim, nt, group);
-            if (!mbar_wait(smem_u32(&accf_bar), (uint32_t)(it & 1), &abort_flag, p.err, 6, kTimeoutNs)) break;
-            tc_fence_after();
-            float alpha = 1.0f;
+            float alpha = 1.0f;  // read before the wait: off the drain's critical path
             if (FMT == BSQ_NVFP4) {
                 const float ga = p.gsA ? __ldg(p.gsA) : 1.0f;
                 const float gb = p.gsB ? __ldg(p.gsB + group) : 1.0f;
                 alpha = __fmul_rn(ga, gb);
             }
+            if (!mbar_wait(smem_u32(&accf_bar), (uint32_t)(it & 1), &abort_flag, p.err, 6, kTimeoutNs)) break;
+            tc_fence_after();
             const int64_t row0 = a_row0 + 32 * q;  // first row of this warp's boxes
             const int64_t ar = row0 + lane;
             const bool row_ok = ar < m_lim;
@@ -1189,15 +1189,23 @@ __global__ void __launch_bounds__(448, 1)
                 // release the accumulator before any store
                 uint32_t pk[HC / 2];
 #pragma unroll
-                for (int c = 0; c < HC / 32; c++) {
-                    uint32_t r0[32];
+                for (int c = 0; c < HC / 32; c += 2) {
+                    // two 32-column loads in flight per wait
+                    uint32_t r0[32], r1[32];
                     tmem_ld32(tbase + 32 * c, r0);
+                    tmem_ld32(tbase + 32 * c + 32, r1);
                     tmem_ld_wait();
 #pragma unroll
                     for (int j = 0; j < 16; j++) {
                         __nv_bfloat162 h = __floats2bfloat162_rn(__fmul_rn(alpha, __uint_as_float(r0[2 * j])),
                                                                  __fmul_rn(alpha, __uint_as_float(r0[2 * j + 1])));
                         pk[16 * c + j] = *reinterpret_cast<uint32_t *>(&h);
+                    }
+#pragma unroll
+                    for (int j = 0; j < 16; j++) {
+                        __nv_bfloat162 h = __floats2bfloat162_rn(__fmul_rn(alpha, __uint_as_float(r1[2 * j])),
+                                                                 __fmul_rn(alpha, __uint_as_float(r1[2 * j + 1])));
+                        pk[16 * c + 16 + j] = *reinterpret_cast<uint32_t *>(&h);
                     }
                 }
                 tc_fence_before();

@@ -21,7 +21,8 @@ BSQ_OK, BSQ_ERR_INVALID, BSQ_ERR_ALIGN, BSQ_ERR_UNSUPPORTED, BSQ_ERR_CUDA, BSQ_E
 BSQ_RNE, BSQ_SR = 0, 1
 BSQ_NVFP4, BSQ_MXFP8, BSQ_MXFP4 = 0, 1, 2
 BSQ_OUT_F32, BSQ_OUT_BF16 = 0, 1
-BSQ_KNOB_FUSED_QUANT, BSQ_KNOB_GEMM_PAIR, BSQ_KNOB_GEMM_BN, BSQ_KNOB_STREAM_QUANT, BSQ_KNOB_GEMM_SPLITK = 0, 1, 2, 3, 4
+(BSQ_KNOB_FUSED_QUANT, BSQ_KNOB_GEMM_PAIR, BSQ_KNOB_GEMM_BN, BSQ_KNOB_STREAM_QUANT, BSQ_KNOB_GEMM_SPLITK,
+ BSQ_KNOB_LAUNCH_OVERLAP) = 0, 1, 2, 3, 4, 5
 
 _lock = threading.Lock()
 _lib = None

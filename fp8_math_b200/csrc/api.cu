@@ -60,7 +60,7 @@ void philox_host(uint32_t c[4], uint32_t k0, uint32_t k1) {
 }
 
 // Kernel-selection overrides (bsq_debug_kernel_choice): -1 = automatic.
-std::atomic<int> g_knob[5] = {{-1}, {-1}, {-1}, {-1}, {-1}};
+std::atomic<int> g_knob[6] = {{-1}, {-1}, {-1}, {-1}, {-1}, {-1}};
 
 }  // namespace
 
@@ -75,6 +75,7 @@ int bsq_debug_kernel_choice(int knob, int value) {
         case BSQ_KNOB_FUSED_QUANT:
         case BSQ_KNOB_GEMM_PAIR:
         case BSQ_KNOB_STREAM_QUANT:
+        case BSQ_KNOB_LAUNCH_OVERLAP:
             if (value < -1 || value > 1) return BSQ_ERR_INVALID;
             break;
         case BSQ_KNOB_GEMM_BN:

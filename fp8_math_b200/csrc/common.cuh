@@ -14,6 +14,40 @@
 
 namespace bsq {
 
+// ---------------------------------------------------------------- launch overlap
+// Programmatic dependent launch.  A kernel launched by launch_dependent() may
+// be scheduled while the kernel before it in the stream is still running.
+// Every such kernel calls grid_dependency_wait() before its first access to
+// global memory: the call returns once the previous kernel has completed and
+// its writes are visible, so results are those of plain stream order and
+// only the launch latency overlaps.  grid_dependents_launch() lets the next
+// kernel be scheduled as soon as every CTA of this one has called it (or has
+// exited).  Outside such launches both are no-ops.
+BSQ_DEV void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+BSQ_DEV void grid_dependents_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// Current value of a kernel-selection override (BSQ_KNOB_*; -1 = automatic).
+int kernel_choice(int knob);
+
+// kern<<<grid, block, smem, s>>>(args...), marked for programmatic dependent
+// launch unless BSQ_KNOB_LAUNCH_OVERLAP is 0.  kern must call
+// grid_dependency_wait() before it touches global memory.
+template <class... P, class... A>
+cudaError_t launch_dependent(void (*kern)(P...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                             A &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = kernel_choice(BSQ_KNOB_LAUNCH_OVERLAP) != 0 ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kern, static_cast<A &&>(args)...);
+}
+
 // ---------------------------------------------------------------- error word
 // One 32-bit word per device: bit 0 set by a bounded wait that ran out, bits
 // 8..15 hold the site id of the first such wait.
@@ -294,16 +328,53 @@ BSQ_DEV void rht16_u_words(const uint32_t w_in[8], const uint32_t sw[8], f32x2 P
         }
     }
 }
-BSQ_DEV void pairs_scale(f32x2 P[8], float c) {
-    const f32x2 C = f2_pack(c, c);
-#pragma unroll
-    for (int k = 0; k < 8; k++) P[k] = f2_mul(P[k], C);
-}
 // three-input max (sm_100)
 BSQ_DEV float fmax3(float a, float b, float c) {
     float r;
     asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
     return r;
+}
+// max |u| over the 16 outputs of rht16_u_words, without forming them: the
+// last butterfly (stride 8) maps each pair (a, b) to RN(a + b) and RN(a - b),
+// and max(|RN(a + b)|, |RN(a - b)|) = RN(|a| + |b|) -- one of a + b, a - b
+// has magnitude |a| + |b| exactly, the other no more, and RN is symmetric
+// and monotone.  (A NaN pair contributes NaN either way, which the maxima
+// below skip as the per-output maxima do.)
+BSQ_DEV float rht16_u_absmax(const uint32_t w_in[8], const uint32_t sw[8]) {
+    f32x2 P[8];
+#pragma unroll
+    for (int k = 0; k < 8; k++) {
+        const uint32_t w = w_in[k] ^ sw[k];
+        const float a = bf16_lo(w), b = bf16_hi(w);
+        P[k] = f2_pack(__fadd_rn(a, b), __fsub_rn(a, b));
+    }
+#pragma unroll
+    for (int h = 1; h < 4; h <<= 1) {  // strides 2 and 4 as pair strides 1 and 2
+#pragma unroll
+        for (int base = 0; base < 8; base += 2 * h) {
+#pragma unroll
+            for (int k = base; k < base + h; k++) {
+                const f32x2 a = P[k], b = P[k + h];
+                P[k] = f2_add(a, b);
+                P[k + h] = f2_sub(a, b);
+            }
+        }
+    }
+    float s[8];
+#pragma unroll
+    for (int k = 0; k < 4; k++) {
+        float a0, a1, b0, b1;
+        f2_unpack(P[k], a0, a1);
+        f2_unpack(P[k + 4], b0, b1);
+        s[2 * k] = __fadd_rn(fabsf(a0), fabsf(b0));
+        s[2 * k + 1] = __fadd_rn(fabsf(a1), fabsf(b1));
+    }
+    return fmax3(fmax3(s[0], s[1], s[2]), fmax3(s[3], s[4], s[5]), fmax3(s[6], s[7], 0.0f));
+}
+BSQ_DEV void pairs_scale(f32x2 P[8], float c) {
+    const f32x2 C = f2_pack(c, c);
+#pragma unroll
+    for (int k = 0; k < 8; k++) P[k] = f2_mul(P[k], C);
 }
 // max |v| over 8 pairs, as a tree of three-input maxima
 BSQ_DEV float pairs_absmax3(const f32x2 P[8]) {

@@ -159,6 +159,8 @@ __global__ void __launch_bounds__(384, SPLITK == 1 ? 1 : 2)
     // rank-0 CTA (distributed shared memory) in rank order.  Three stages
     // (86 KB) and 256 TMEM columns per CTA, so that two CTAs share an SM.
     static_assert(SPLITK == 1 || (SWAP && BN == 64 && !GROUPED), "split-K: the skinny swap-AB tile only");
+    grid_dependency_wait();
+    grid_dependents_launch();
     using C_ = Cfg<FMT, BN, SPLITK == 1 ? 8 : 3>;
     constexpr int kTmemCols = SPLITK == 1 ? 512 : 256;
     using T = typename C_::T;
@@ -825,6 +827,8 @@ __global__ void __launch_bounds__(448, 1)
                     const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
                     const __grid_constant__ CUtensorMap tmC, const GemmParams p) {
     static_assert(!QOUT || OUT_BF16, "the quantizing epilogue quantizes the bf16 output");
+    grid_dependency_wait();
+    grid_dependents_launch();
     using C_ = Cfg2<FMT, GROUPED>;
     using T = typename C_::T;
     constexpr int NS = C_::kStages;
@@ -1453,13 +1457,15 @@ int run_pair(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &ts
     cfg.blockDim = dim3(C_::kThreads, 1, 1);
     cfg.dynamicSmemBytes = C_::kSmemBytes;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // the kernel waits first (grid_dependency_wait)
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = kernel_choice(BSQ_KNOB_LAUNCH_OVERLAP) != 0 ? 2 : 1;
     if (cudaLaunchKernelEx(&cfg, kern, ta, tb, tsa, tsb, tc, p) != cudaSuccess) return BSQ_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? BSQ_OK : BSQ_ERR_CUDA;
 }
@@ -1470,7 +1476,8 @@ int run(const CUtensorMap &ta, const CUtensorMap &tb, const GemmParams &p, int g
     using C_ = Cfg<FMT, BN>;
     auto kern = gemm_bs_kernel<FMT, BN, ACC, OUT_BF16, SWAP, GROUPED>;
     if (smem_attr_once(reinterpret_cast<const void *>(kern), C_::kSmemBytes) != BSQ_OK) return BSQ_ERR_CUDA;
-    kern<<<grid, C_::kThreads, C_::kSmemBytes, s>>>(ta, tb, tc ? *tc : ta, p);
+    if (launch_dependent(kern, grid, C_::kThreads, C_::kSmemBytes, s, ta, tb, tc ? *tc : ta, p) != cudaSuccess)
+        return BSQ_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? BSQ_OK : BSQ_ERR_CUDA;
 }
 
@@ -1485,13 +1492,15 @@ int run_splitk(const CUtensorMap &ta, const CUtensorMap &tb, const GemmParams &p
     cfg.blockDim = dim3(C_::kThreads, 1, 1);
     cfg.dynamicSmemBytes = C_::kSmemBytes;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = S;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // the kernel waits first (grid_dependency_wait)
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = kernel_choice(BSQ_KNOB_LAUNCH_OVERLAP) != 0 ? 2 : 1;
     if (cudaLaunchKernelEx(&cfg, kern, ta, tb, ta, p) != cudaSuccess) return BSQ_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? BSQ_OK : BSQ_ERR_CUDA;
 }

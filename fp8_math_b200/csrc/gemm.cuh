@@ -27,8 +27,6 @@ struct GemmArgs {
 };
 
 int launch_gemm(const GemmArgs &g, cudaStream_t s);
-// Current value of a kernel-selection override (BSQ_KNOB_*; -1 = automatic).
-int kernel_choice(int knob);
 void launch_timeout_probe(uint64_t timeout_ns, unsigned int *err, cudaStream_t s);
 
 }  // namespace bsq

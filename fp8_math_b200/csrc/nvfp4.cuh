@@ -19,11 +19,10 @@ BSQ_DEV float global_scale_of(float amax) { return amax == 0.0f ? 1.0f : __fdiv_
 // applied once, to the maximum.
 template <bool RHT>
 BSQ_DEV float block_absmax(const uint32_t w[8], const uint32_t sw[8]) {
+    if (RHT) return __fmul_rn(rht16_u_absmax(w, sw), 0.25f);
     f32x2 P[8];
-    if (RHT) rht16_u_words(w, sw, P);
-    else words_to_pairs(w, P);
-    const float m = pairs_absmax3(P);
-    return RHT ? __fmul_rn(m, 0.25f) : m;
+    words_to_pairs(w, P);
+    return pairs_absmax3(P);
 }
 
 // Per-CTA tables and constants of one tensor's global scale s_g.  For every

@@ -90,6 +90,8 @@ template <bool RHT>
 __global__ void __launch_bounds__(256) amax_flat_kernel(const uint16_t *__restrict__ x, int64_t nblk, uint32_t mask,
                                                         unsigned int *amax_bits, unsigned int *counter,
                                                         float *gs_out) {
+    grid_dependency_wait();
+    grid_dependents_launch();
     uint32_t sw[8];
     rht_sign_words(mask, sw);
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
@@ -228,6 +230,8 @@ template <bool RHT, bool FOS>
 __global__ void __launch_bounds__(256) quant_nvfp4_1d_flat_kernel(
     const uint16_t *__restrict__ x, int64_t nblk, int kb_shift, uint32_t mask, const float *scale_src,
     int src_is_amax, float *gs_out, int write_gs, uint8_t *__restrict__ codes, uint8_t *__restrict__ sf) {
+    grid_dependency_wait();
+    grid_dependents_launch();
     __shared__ float den_tab[128], rcp_tab[128];
     const float s_g = src_is_amax ? global_scale_of(*scale_src) : *scale_src;
     if (write_gs && blockIdx.x == 0 && threadIdx.x == 0) *gs_out = s_g;
@@ -267,6 +271,8 @@ template <bool RHT>
 __global__ void __launch_bounds__(256) quant_nvfp4_2d_kernel(
     const uint16_t *__restrict__ x, int64_t M, int64_t K, int64_t ldx, uint32_t mask, const float *scale_src,
     int src_is_amax, float *gs_out, int write_gs, uint8_t *__restrict__ codes, uint8_t *__restrict__ sf) {
+    grid_dependency_wait();
+    grid_dependents_launch();
     __shared__ float den_tab[128], rcp_tab[128];
     const float s_g = src_is_amax ? global_scale_of(*scale_src) : *scale_src;
     if (write_gs && blockIdx.x == 0 && threadIdx.x == 0) *gs_out = s_g;
@@ -547,6 +553,8 @@ __global__ void __launch_bounds__(nvs::kThreads, 2) quant_nvfp4_stream_kernel(
     unsigned int *amax_bits, const float *scale_src, int src_is_amax, float *gs_out, uint8_t *__restrict__ codes,
     uint8_t *__restrict__ sf, unsigned int *err) {
     using namespace sm100;
+    grid_dependency_wait();
+    grid_dependents_launch();
     extern __shared__ __align__(128) uint8_t ring[];
     __shared__ __align__(8) uint64_t full_bar[nvs::kStages], empty_bar[nvs::kStages];
     __shared__ float den_tab[128], rcp_tab[128];
@@ -2013,10 +2021,10 @@ void launch_amax(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, bool rht,
         const int64_t nblk = M * (K >> 4);
         if (rht) {
             const int grid = grid_for(nblk, 4 * 256, resident_ctas<amax_flat_kernel<true>>(num_sms));
-            amax_flat_kernel<true><<<grid, 256, 0, s>>>(x, nblk, mask, amax_bits, counter, gs_out);
+            launch_dependent(amax_flat_kernel<true>, grid, 256, 0, s, x, nblk, mask, amax_bits, counter, gs_out);
         } else {
             const int grid = grid_for(nblk, 4 * 256, resident_ctas<amax_flat_kernel<false>>(num_sms));
-            amax_flat_kernel<false><<<grid, 256, 0, s>>>(x, nblk, mask, amax_bits, counter, gs_out);
+            launch_dependent(amax_flat_kernel<false>, grid, 256, 0, s, x, nblk, mask, amax_bits, counter, gs_out);
         }
         return;
     }
@@ -2060,10 +2068,10 @@ void launch_quant_nvfp4(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, bo
         int kb_shift = 0;
         while ((int64_t(1) << kb_shift) < KB) kb_shift++;
         const int64_t nblk = M * KB;
-#define BSQ_NVF(R, F)                                                                                          \
-    quant_nvfp4_1d_flat_kernel<R, F><<<grid_for(nblk, 2 * 256, resident_ctas<quant_nvfp4_1d_flat_kernel<R, F>>( \
-                                                                             num_sms)),                        \
-                                       256, 0, s>>>(x, nblk, kb_shift, mask, scale_src, sa, gs_out, wg, codes, sf)
+#define BSQ_NVF(R, F)                                                                                           \
+    launch_dependent(quant_nvfp4_1d_flat_kernel<R, F>,                                                         \
+                     grid_for(nblk, 2 * 256, resident_ctas<quant_nvfp4_1d_flat_kernel<R, F>>(num_sms)), 256, 0, s, \
+                     x, nblk, kb_shift, mask, scale_src, sa, gs_out, wg, codes, sf)
         if (rht) { if (fos) BSQ_NVF(true, true); else BSQ_NVF(true, false); }
         else { if (fos) BSQ_NVF(false, true); else BSQ_NVF(false, false); }
 #undef BSQ_NVF
@@ -2141,8 +2149,9 @@ static int launch_stream_t(const uint16_t *x, int64_t M, int64_t K, uint32_t mas
                    ? 0
                    : 1;
     }
-    kern<<<grid, nvs::kThreads, nvs::kSmemBytes, s>>>(x, M, K, div_kb, mask, counter, amax_bits, scale_src,
-                                                      src_is_amax, gs_out, codes, sf, err);
+    if (launch_dependent(kern, grid, nvs::kThreads, nvs::kSmemBytes, s, x, M, K, div_kb, mask, counter, amax_bits,
+                         scale_src, src_is_amax, gs_out, codes, sf, err) != cudaSuccess)
+        return 1;
     return cudaGetLastError() == cudaSuccess ? 0 : 1;
 }
 

@@ -84,7 +84,10 @@ enum {
     BSQ_KNOB_GEMM_BN = 2,     /* -1: automatic; 128 or 256 (bf16 output): the single-CTA GEMM's N tile */
     BSQ_KNOB_STREAM_QUANT = 3, /* -1: bulk-copy streaming NVFP4 kernels for contiguous 16x16 tensors; 1: for every
                                   contiguous amax / NVFP4 call; 0: never */
-    BSQ_KNOB_GEMM_SPLITK = 4   /* -1: automatic; 1: off; 2, 4 or 8: the skinny (M <= 64) GEMM's K split */
+    BSQ_KNOB_GEMM_SPLITK = 4,  /* -1: automatic; 1: off; 2, 4 or 8: the skinny (M <= 64) GEMM's K split */
+    BSQ_KNOB_LAUNCH_OVERLAP = 5 /* 1/-1: the GEMMs and the linear step's quantize kernels are launched for
+                                   programmatic dependent launch (scheduled while the previous kernel in the
+                                   stream finishes; each waits for it before touching memory); 0: plain launches */
 };
 
 /* Human-readable name of a status code (static string). */

@@ -109,7 +109,9 @@ def test_kernel_choice_knobs_validate(lib):
     assert L.bsq_debug_kernel_choice(lib.BSQ_KNOB_FUSED_QUANT, 2) == lib.BSQ_ERR_INVALID
     assert L.bsq_debug_kernel_choice(lib.BSQ_KNOB_GEMM_BN, 64) == lib.BSQ_ERR_INVALID
     assert L.bsq_debug_kernel_choice(lib.BSQ_KNOB_GEMM_SPLITK, 3) == lib.BSQ_ERR_INVALID
-    for knob, value in [(lib.BSQ_KNOB_FUSED_QUANT, 0), (lib.BSQ_KNOB_GEMM_PAIR, 1), (lib.BSQ_KNOB_GEMM_BN, 256)]:
+    assert L.bsq_debug_kernel_choice(lib.BSQ_KNOB_LAUNCH_OVERLAP, 2) == lib.BSQ_ERR_INVALID
+    for knob, value in [(lib.BSQ_KNOB_FUSED_QUANT, 0), (lib.BSQ_KNOB_GEMM_PAIR, 1), (lib.BSQ_KNOB_GEMM_BN, 256),
+                        (lib.BSQ_KNOB_LAUNCH_OVERLAP, 0)]:
         assert L.bsq_debug_kernel_choice(knob, value) == lib.BSQ_OK
         assert L.bsq_debug_kernel_choice(knob, -1) == lib.BSQ_OK
 

@@ -703,7 +703,8 @@ def main():
             "roofline": {"bound": "tensor", "achieved": gemm_tflops, "peak": fp4_peak, "unit": "TFLOP/s",
                          "frac": gemm_tflops / fp4_peak,
                          "traffic": ncu_traffic("gemm_pair_nvfp4_8192x14336x4096.md",
-                                                ["fp8_math_b200/csrc/gemm.cu", "fp8_math_b200/csrc/sm100.cuh"]),
+                                                ["fp8_math_b200/csrc/gemm.cu", "fp8_math_b200/csrc/sm100.cuh",
+                                                 "fp8_math_b200/csrc/common.cuh", "fp8_math_b200/csrc/nvfp4.cuh"]),
                          "algorithmic_bytes": (M * K + N * K) // 2 + (M + N) * (K // 16) + M * N * 2,
                          "kernel": "gemm_bs2_kernel (NVFP4 8192x14336x4096, CTA pairs)",
                          "peak_source": f"{src} bf16 burst {bf16} x {NOMINAL_FP4_OVER_BF16} (nominal FP4/BF16), "

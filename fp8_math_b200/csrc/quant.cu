@@ -85,22 +85,26 @@ __global__ void __launch_bounds__(256) amax_kernel(const uint16_t *__restrict__ 
 }
 
 // Contiguous tensor as a flat sequence of 16-element blocks; four blocks per
-// thread in flight (all loads issued before any is reduced).
-template <bool RHT>
-__global__ void __launch_bounds__(256) amax_flat_kernel(const uint16_t *__restrict__ x, int64_t nblk, uint32_t mask,
+// thread in flight (all loads issued before any is reduced).  I is the block
+// index type: uint32_t when the block count and the loop's overshoot fit
+// (below 2^31 blocks), which keeps the index arithmetic to single 32-bit
+// instructions; int64_t otherwise.
+template <bool RHT, typename I>
+__global__ void __launch_bounds__(256) amax_flat_kernel(const uint16_t *__restrict__ x, int64_t nblk64, uint32_t mask,
                                                         unsigned int *amax_bits, unsigned int *counter,
                                                         float *gs_out) {
     grid_dependency_wait();
     grid_dependents_launch();
     uint32_t sw[8];
     rht_sign_words(mask, sw);
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    const I nblk = (I)nblk64;
+    const I stride = (I)gridDim.x * (I)blockDim.x;
     float m = 0.0f;
-    for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < nblk; b += 4 * stride) {
+    for (I b = (I)blockIdx.x * (I)blockDim.x + (I)threadIdx.x; b < nblk; b += 4 * stride) {
         uint32_t w[4][8];
 #pragma unroll
         for (int i = 0; i < 4; i++)
-            if (b + i * stride < nblk) load_words16(x + (b + i * stride) * 16, w[i]);
+            if (b + i * stride < nblk) load_words16(x + (size_t)(b + i * stride) * 16, w[i]);
 #pragma unroll
         for (int i = 0; i < 4; i++)
             if (b + i * stride < nblk) m = fmaxf(m, block_absmax<RHT>(w[i], sw));
@@ -226,9 +230,9 @@ __global__ void __launch_bounds__(256) quant_nvfp4_1d_kernel(
 // row holds a power-of-two number of blocks (>= 4): a flat sequence of
 // blocks, two per thread in flight.  Lanes 4j..4j+3 hold four consecutive
 // blocks of one row, so the scale bytes pack into one word.
-template <bool RHT, bool FOS>
+template <bool RHT, bool FOS, typename I>
 __global__ void __launch_bounds__(256) quant_nvfp4_1d_flat_kernel(
-    const uint16_t *__restrict__ x, int64_t nblk, int kb_shift, uint32_t mask, const float *scale_src,
+    const uint16_t *__restrict__ x, int64_t nblk64, int kb_shift, uint32_t mask, const float *scale_src,
     int src_is_amax, float *gs_out, int write_gs, uint8_t *__restrict__ codes, uint8_t *__restrict__ sf) {
     grid_dependency_wait();
     grid_dependents_launch();
@@ -238,26 +242,42 @@ __global__ void __launch_bounds__(256) quant_nvfp4_1d_flat_kernel(
     const NvScale c = nv_scale_setup(s_g, den_tab, rcp_tab);
     uint32_t sw[8];
     rht_sign_words(mask, sw);
-    const int64_t KB = int64_t(1) << kb_shift;
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    // I: the block index type (uint32_t below 2^31 blocks, as for amax_flat_kernel)
+    const I nblk = (I)nblk64;
+    const I KB = I(1) << kb_shift;
+    const I bt = (KB + 3) >> 2;  // 4-block groups per row (the scale layout's atom columns)
+    const I stride = (I)gridDim.x * (I)blockDim.x;
     // the loop bound is rounded to whole warps so that shuffles see all lanes
-    const int64_t nwarp_blk = (nblk + 31) & ~int64_t(31);
-    for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b - (threadIdx.x & 31) < nwarp_blk;
+    const I nwarp_blk = (nblk + 31) & ~I(31);
+    // scale bytes of lanes 4j..4j+3 (blocks 4i..4i+3 of one row) as one word
+    // at the swizzled offset of (row, block group)
+    auto store_sf4 = [&](bool valid, uint32_t sb, I b) {
+        const uint32_t b1 = __shfl_down_sync(0xFFFFFFFFu, sb, 1);
+        const uint32_t b2 = __shfl_down_sync(0xFFFFFFFFu, sb, 2);
+        const uint32_t b3 = __shfl_down_sync(0xFFFFFFFFu, sb, 3);
+        if (valid && (threadIdx.x & 3) == 0) {
+            const I r = b >> kb_shift, b4 = (b & (KB - 1)) >> 2;
+            const I off = (((r >> 7) * bt + b4) << 9) + ((r & 31) << 4) + (((r >> 5) & 3) << 2);
+            *reinterpret_cast<uint32_t *>(sf + (size_t)off) =
+                (sb & 0xFFu) | ((b1 & 0xFFu) << 8) | ((b2 & 0xFFu) << 16) | ((b3 & 0xFFu) << 24);
+        }
+    };
+    for (I b = (I)blockIdx.x * (I)blockDim.x + (I)threadIdx.x; b - (I)(threadIdx.x & 31) < nwarp_blk;
          b += 2 * stride) {
-        const int64_t b1 = b + stride;
+        const I b1 = b + stride;
         const bool v0 = b < nblk, v1 = b1 < nblk;
         uint32_t w0[8], w1[8];
-        load_words16(x + (v0 ? b : 0) * 16, w0);
-        load_words16(x + (v1 ? b1 : 0) * 16, w1);
+        load_words16(x + (size_t)(v0 ? b : 0) * 16, w0);
+        load_words16(x + (size_t)(v1 ? b1 : 0) * 16, w1);
         uint32_t sb0, sb1;
         uint2 cd0, cd1;
         nv_block_1d<RHT, FOS>(w0, sw, c, den_tab, rcp_tab, sb0, cd0);
-        if (v0) *reinterpret_cast<uint2 *>(codes + b * 8) = cd0;
-        store_sf(sf, v0, sb0, b >> kb_shift, b & (KB - 1), KB, true);
+        if (v0) *reinterpret_cast<uint2 *>(codes + (size_t)b * 8) = cd0;
+        store_sf4(v0, sb0, b);
         if (__any_sync(0xFFFFFFFFu, v1)) {
             nv_block_1d<RHT, FOS>(w1, sw, c, den_tab, rcp_tab, sb1, cd1);
-            if (v1) *reinterpret_cast<uint2 *>(codes + b1 * 8) = cd1;
-            store_sf(sf, v1, sb1, b1 >> kb_shift, b1 & (KB - 1), KB, true);
+            if (v1) *reinterpret_cast<uint2 *>(codes + (size_t)b1 * 8) = cd1;
+            store_sf4(v1, sb1, b1);
         }
     }
 }
@@ -2019,13 +2039,15 @@ void launch_amax(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, bool rht,
                  int num_sms, cudaStream_t s) {
     if (!row_index && ldx == K) {
         const int64_t nblk = M * (K >> 4);
-        if (rht) {
-            const int grid = grid_for(nblk, 4 * 256, resident_ctas<amax_flat_kernel<true>>(num_sms));
-            launch_dependent(amax_flat_kernel<true>, grid, 256, 0, s, x, nblk, mask, amax_bits, counter, gs_out);
+#define BSQ_AMF(R, I)                                                                              \
+    launch_dependent(amax_flat_kernel<R, I>, grid_for(nblk, 4 * 256, resident_ctas<amax_flat_kernel<R, I>>(num_sms)), \
+                     256, 0, s, x, nblk, mask, amax_bits, counter, gs_out)
+        if (nblk < (int64_t(1) << 31)) {
+            if (rht) BSQ_AMF(true, uint32_t); else BSQ_AMF(false, uint32_t);
         } else {
-            const int grid = grid_for(nblk, 4 * 256, resident_ctas<amax_flat_kernel<false>>(num_sms));
-            launch_dependent(amax_flat_kernel<false>, grid, 256, 0, s, x, nblk, mask, amax_bits, counter, gs_out);
+            if (rht) BSQ_AMF(true, int64_t); else BSQ_AMF(false, int64_t);
         }
+#undef BSQ_AMF
         return;
     }
     RowMap map{lpr_shift_for(K >> 4)};
@@ -2068,12 +2090,17 @@ void launch_quant_nvfp4(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, bo
         int kb_shift = 0;
         while ((int64_t(1) << kb_shift) < KB) kb_shift++;
         const int64_t nblk = M * KB;
-#define BSQ_NVF(R, F)                                                                                           \
-    launch_dependent(quant_nvfp4_1d_flat_kernel<R, F>,                                                         \
-                     grid_for(nblk, 2 * 256, resident_ctas<quant_nvfp4_1d_flat_kernel<R, F>>(num_sms)), 256, 0, s, \
-                     x, nblk, kb_shift, mask, scale_src, sa, gs_out, wg, codes, sf)
-        if (rht) { if (fos) BSQ_NVF(true, true); else BSQ_NVF(true, false); }
-        else { if (fos) BSQ_NVF(false, true); else BSQ_NVF(false, false); }
+#define BSQ_NVF(R, F, I)                                                                                        \
+    launch_dependent(quant_nvfp4_1d_flat_kernel<R, F, I>,                                                      \
+                     grid_for(nblk, 2 * 256, resident_ctas<quant_nvfp4_1d_flat_kernel<R, F, I>>(num_sms)), 256, 0, \
+                     s, x, nblk, kb_shift, mask, scale_src, sa, gs_out, wg, codes, sf)
+        if (nblk < (int64_t(1) << 31)) {
+            if (rht) { if (fos) BSQ_NVF(true, true, uint32_t); else BSQ_NVF(true, false, uint32_t); }
+            else { if (fos) BSQ_NVF(false, true, uint32_t); else BSQ_NVF(false, false, uint32_t); }
+        } else {
+            if (rht) { if (fos) BSQ_NVF(true, true, int64_t); else BSQ_NVF(true, false, int64_t); }
+            else { if (fos) BSQ_NVF(false, true, int64_t); else BSQ_NVF(false, false, int64_t); }
+        }
 #undef BSQ_NVF
         return;
     }

@@ -569,7 +569,8 @@ BSQ_DEV NvChunks nv_chunks(int64_t M, int64_t K) {
 
 template <int MODE, bool RHT, bool TWO_D>
 __global__ void __launch_bounds__(nvs::kThreads, 2) quant_nvfp4_stream_kernel(
-    const uint16_t *__restrict__ x, int64_t M, int64_t K, DivU32 div_kb, uint32_t mask, unsigned int *counter,
+    const uint16_t *__restrict__ x, int64_t M, int64_t K, DivU32 div_kb, DivU32 div_span, uint32_t mask,
+    unsigned int *counter,
     unsigned int *amax_bits, const float *scale_src, int src_is_amax, float *gs_out, uint8_t *__restrict__ codes,
     uint8_t *__restrict__ sf, unsigned int *err) {
     using namespace sm100;
@@ -621,8 +622,9 @@ __global__ void __launch_bounds__(nvs::kThreads, 2) quant_nvfp4_stream_kernel(
                     bulk_load(smem_u32(dst), x + b0 * 16, (uint32_t)(nb * 32), fb);
                 }
             } else {
-                const int64_t rg = c / g.nspan, sp = c - rg * g.nspan;
-                const int64_t k0 = sp << 9;
+                // chunk counts stay below 2^32 on this path (stream_ok): 32-bit division
+                const uint32_t rg = divu32((uint32_t)c, div_span), sp = (uint32_t)c - rg * (uint32_t)g.nspan;
+                const int64_t k0 = (int64_t)sp << 9;
                 const int64_t cols = (K - k0) < 512 ? (K - k0) : 512;
                 if (lane == 0) mbar_arrive_expect_tx(fb, (uint32_t)(16 * cols * 2));
                 __syncwarp();
@@ -702,7 +704,7 @@ __global__ void __launch_bounds__(nvs::kThreads, 2) quant_nvfp4_stream_kernel(
                 if (t < nb) m = fmaxf(m, block_absmax<RHT>(w0, sw));
                 if (t + 256 < nb) m = fmaxf(m, block_absmax<RHT>(w1, sw));
             } else {
-                const int64_t sp = c % g.nspan;
+                const uint32_t sp = (uint32_t)c - divu32((uint32_t)c, div_span) * (uint32_t)g.nspan;
                 const int64_t nb = (K - (sp << 9)) >> 4;
                 const int row = t & 15, b0 = 2 * (t >> 4);
                 uint32_t w0[8], w1[8];
@@ -795,11 +797,12 @@ __global__ void __launch_bounds__(nvs::kThreads, 2) quant_nvfp4_stream_kernel(
                 store_sf(sf, v, sb, row, b - row * g.KB, g.KB, true);
             }
         } else {
-            const int64_t rg = c / g.nspan, sp = c - rg * g.nspan;
-            const int64_t nb = (K - (sp << 9)) >> 4;      // blocks in this span (multiple of 4)
+            // 32-bit chunk, row and block indices (M * K / 16 < 2^32 on this path)
+            const uint32_t rg = divu32((uint32_t)c, div_span), sp = (uint32_t)c - rg * (uint32_t)g.nspan;
+            const int64_t nb = (K - ((int64_t)sp << 9)) >> 4;  // blocks in this span (multiple of 4)
             const int row = t & 15, bp = t >> 4;
-            const int64_t grow = rg * 16 + row;
-            const int64_t kb0 = (sp << 5) + 2 * bp;        // first block of this thread
+            const uint32_t grow = rg * 16 + row;
+            const uint32_t kb0 = (sp << 5) + 2 * bp;          // first block of this thread
             const bool v = 2 * bp < nb;                    // both blocks valid (nb is even)
             uint32_t w[2][8];
             words_2d(st, row, v ? 2 * bp : 0, w[0]);
@@ -823,12 +826,17 @@ __global__ void __launch_bounds__(nvs::kThreads, 2) quant_nvfp4_stream_kernel(
             if (MODE == nvs::FUSED && v && grow == 0 && kb0 == 0 && !wait_counter(counter, all_read, err, 35))
                 cd[0] = make_uint2(0u, 0u);
             if (v)
-                *reinterpret_cast<uint4 *>(codes + grow * (K >> 1) + kb0 * 8) =
+                *reinterpret_cast<uint4 *>(codes + (size_t)grow * (uint32_t)(K >> 1) + kb0 * 8) =
                     make_uint4(cd[0].x, cd[0].y, cd[1].x, cd[1].y);
-            // lanes l and l + 16 hold blocks 4i .. 4i + 3 of one row: one word
+            // lanes l and l + 16 hold blocks 4i .. 4i + 3 of one row: one word,
+            // at the swizzled offset of (row, 4-block group) (sf_word_offset in
+            // 32-bit arithmetic: the scale buffer holds fewer than 2^32 bytes)
             const uint32_t other = __shfl_down_sync(0xFFFFFFFFu, sbw, 16);
-            if (v && lane < 16)
-                *reinterpret_cast<uint32_t *>(sf + sf_word_offset(grow, kb0 >> 2, g.KB)) = sbw | (other << 16);
+            if (v && lane < 16) {
+                const uint32_t bt = (uint32_t)((g.KB + 3) >> 2);
+                const uint32_t off = (((grow >> 7) * bt + (kb0 >> 2)) << 9) + ((grow & 31) << 4) + (((grow >> 5) & 3) << 2);
+                *reinterpret_cast<uint32_t *>(sf + off) = sbw | (other << 16);
+            }
         }
     }
 }
@@ -2166,18 +2174,20 @@ static int launch_stream_t(const uint16_t *x, int64_t M, int64_t K, uint32_t mas
     const int64_t chunks = TWO_D ? (M >> 4) * ((K + 511) >> 9) : (M * KB + 511) >> 9;
     const int grid = grid_for(chunks, 1, resident_stream<quant_nvfp4_stream_kernel<MODE, RHT, TWO_D>>(num_sms));
     DivU32 div_kb = divu32_for((uint32_t)KB);
+    DivU32 div_span = divu32_for((uint32_t)((K + 511) >> 9));
     if (MODE == nvs::FUSED) {
-        void *args[] = {(void *)&x,        (void *)&M,         (void *)&K,         (void *)&div_kb,
-                        (void *)&mask,     (void *)&counter,   (void *)&amax_bits, (void *)&scale_src,
-                        (void *)&src_is_amax, (void *)&gs_out, (void *)&codes,     (void *)&sf,
-                        (void *)&err};
+        // one pointer per kernel parameter, in the kernel's order
+        void *args[] = {(void *)&x,         (void *)&M,           (void *)&K,      (void *)&div_kb,
+                        (void *)&div_span,  (void *)&mask,        (void *)&counter, (void *)&amax_bits,
+                        (void *)&scale_src, (void *)&src_is_amax, (void *)&gs_out, (void *)&codes,
+                        (void *)&sf,        (void *)&err};
         return cudaLaunchCooperativeKernel(reinterpret_cast<const void *>(kern), dim3(grid), dim3(nvs::kThreads), args,
                                            nvs::kSmemBytes, s) == cudaSuccess
                    ? 0
                    : 1;
     }
-    if (launch_dependent(kern, grid, nvs::kThreads, nvs::kSmemBytes, s, x, M, K, div_kb, mask, counter, amax_bits,
-                         scale_src, src_is_amax, gs_out, codes, sf, err) != cudaSuccess)
+    if (launch_dependent(kern, grid, nvs::kThreads, nvs::kSmemBytes, s, x, M, K, div_kb, div_span, mask, counter,
+                         amax_bits, scale_src, src_is_amax, gs_out, codes, sf, err) != cudaSuccess)
         return 1;
     return cudaGetLastError() == cudaSuccess ? 0 : 1;
 }

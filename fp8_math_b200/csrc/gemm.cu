@@ -344,7 +344,11 @@ __global__ void __launch_bounds__(384, SPLITK == 1 ? 1 : 2)
                 }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(a * BN);
-                for (int64_t kt = kt_begin; kt < kt_end; kt++, ktc++) {
+                // 32-bit k-tile bookkeeping (on the MMA thread's critical path)
+                const uint32_t kt_lo = (uint32_t)kt_begin, kt_hi = (uint32_t)kt_end;
+                const uint32_t kt_full = (uint32_t)(p.K / T::kBkElems);
+                const int nmma_tail = (int)((p.K % T::kBkElems) / T::kMmaK);
+                for (uint32_t kt = kt_lo; kt < kt_hi; kt++, ktc++) {
                     if (!mbar_test_wait(smem_u32(&full_bar[s]), ph) &&
                         !mbar_wait(smem_u32(&full_bar[s]), ph, &abort_flag, p.err, 4, kTimeoutNs)) {
                         ok = false;
@@ -364,9 +368,8 @@ __global__ void __launch_bounds__(384, SPLITK == 1 ? 1 : 2)
                     const uint32_t b_lo = b_lo0 + (uint32_t)s * (C_::kBBytes >> 4);
                     const uint32_t sfa_lo = sfa_lo0 + (uint32_t)s * (C_::kSfaBytes >> 4);
                     const uint32_t sfb_lo = sfb_lo0 + (uint32_t)s * (C_::kSfbBytes >> 4);
-                    const int64_t krem = p.K - kt * T::kBkElems;
-                    const bool full_kt = krem >= T::kBkElems;
-                    const int nmma = full_kt ? C_::kMmaPerKt : (int)(krem / T::kMmaK);
+                    const bool full_kt = kt < kt_full;
+                    const int nmma = full_kt ? C_::kMmaPerKt : nmma_tail;
                     if (FMT == BSQ_NVFP4) {
                         // four slots per k-tile, one per MMA: its SFA atom, then one atom per 128 rows of B
                         // (with copiers: the stage's own slots, already filled)
@@ -382,7 +385,7 @@ __global__ void __launch_bounds__(384, SPLITK == 1 ? 1 : 2)
                                                     desc_pack(sfb_lo + kSfbTileLo * r + kSfAtomLo * j, kSfHi));
                             }
                             mma_nvfp4(d_tmem, desc_pack(a_lo + 2 * j, kOpHi), desc_pack(b_lo + 2 * j, kOpHi), idesc, slot,
-                                      slot + 4, (kt > kt_begin || j > 0) ? 1u : 0u);
+                                      slot + 4, (kt > kt_lo || j > 0) ? 1u : 0u);
                         };
                         if (full_kt) {
 #pragma unroll
@@ -408,7 +411,7 @@ __global__ void __launch_bounds__(384, SPLITK == 1 ? 1 : 2)
                             const uint32_t id = 2u * (uint32_t)(j & 1), a = (uint32_t)(j >> 1);
                             mma_mxfp4(d_tmem, desc_pack(a_lo + 2 * j, kOpHi), desc_pack(b_lo + 2 * j, kOpHi),
                                       idesc | (id << 29) | (id << 4), (slot + 4 * a) | (id << 30),
-                                      (slot + kSfb0 + kSfbA * a) | (id << 30), (kt > kt_begin || j > 0) ? 1u : 0u);
+                                      (slot + kSfb0 + kSfbA * a) | (id << 30), (kt > kt_lo || j > 0) ? 1u : 0u);
                         };
                         if (full_kt) {
 #pragma unroll
@@ -428,7 +431,7 @@ __global__ void __launch_bounds__(384, SPLITK == 1 ? 1 : 2)
                         auto issue = [&](int j) {
                             mma_mxfp8(d_tmem, desc_pack(a_lo + 2 * j, kOpHi), desc_pack(b_lo + 2 * j, kOpHi),
                                       idesc | ((uint32_t)j << 29) | ((uint32_t)j << 4), slot | ((uint32_t)j << 30),
-                                      (slot + 4) | ((uint32_t)j << 30), (kt > kt_begin || j > 0) ? 1u : 0u);
+                                      (slot + 4) | ((uint32_t)j << 30), (kt > kt_lo || j > 0) ? 1u : 0u);
                         };
                         if (full_kt) {
 #pragma unroll

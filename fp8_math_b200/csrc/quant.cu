@@ -774,8 +774,10 @@ __global__ void __launch_bounds__(nvs::kThreads, 2) quant_nvfp4_stream_kernel(
         if (!st) break;
         const int64_t c = chunk_of(j);
         if (!TWO_D) {
-            const int64_t b0 = c << 9;
-            const int64_t nb = g.nblk - b0;
+            // 32-bit block indices (M * K / 16 < 2^32 on this path)
+            const uint32_t b0 = (uint32_t)c << 9;
+            const int64_t nb = g.nblk - (int64_t)b0;
+            const uint32_t kb32 = (uint32_t)g.KB, bt = (kb32 + 3) >> 2;
             uint32_t w0[8], w1[8];
             words_1d(st, t, w0);   // slots past the tensor's end hold stale bytes: never stored
             words_1d(st, t + 256, w1);
@@ -784,7 +786,7 @@ __global__ void __launch_bounds__(nvs::kThreads, 2) quant_nvfp4_stream_kernel(
             for (int h = 0; h < 2; h++) {
                 const int slot = t + 256 * h;
                 const bool v = slot < nb;
-                const int64_t b = b0 + slot;
+                const uint32_t b = b0 + slot;
                 uint32_t sb;
                 uint2 cd;
                 nv_block_1d<RHT, false>(h ? w1 : w0, sw, cs, den_tab, rcp_tab, sb, cd);
@@ -792,9 +794,18 @@ __global__ void __launch_bounds__(nvs::kThreads, 2) quant_nvfp4_stream_kernel(
                 // once every CTA has read the amax
                 if (MODE == nvs::FUSED && v && b == 0 && !wait_counter(counter, all_read, err, 34))
                     cd = make_uint2(0u, 0u);
-                if (v) *reinterpret_cast<uint2 *>(codes + b * 8) = cd;
-                const int64_t row = divu32((uint32_t)b, div_kb);
-                store_sf(sf, v, sb, row, b - row * g.KB, g.KB, true);
+                if (v) *reinterpret_cast<uint2 *>(codes + (size_t)b * 8) = cd;
+                // lanes 4j..4j+3 hold blocks 4i..4i+3 of one row (K % 64 == 0):
+                // one scale word at the swizzled offset of (row, 4-block group)
+                const uint32_t b1 = __shfl_down_sync(0xFFFFFFFFu, sb, 1);
+                const uint32_t b2 = __shfl_down_sync(0xFFFFFFFFu, sb, 2);
+                const uint32_t b3 = __shfl_down_sync(0xFFFFFFFFu, sb, 3);
+                if (v && (lane & 3) == 0) {
+                    const uint32_t r = divu32(b, div_kb), b4 = (b - r * kb32) >> 2;
+                    const uint32_t off = (((r >> 7) * bt + b4) << 9) + ((r & 31) << 4) + (((r >> 5) & 3) << 2);
+                    *reinterpret_cast<uint32_t *>(sf + off) =
+                        (sb & 0xFFu) | ((b1 & 0xFFu) << 8) | ((b2 & 0xFFu) << 16) | ((b3 & 0xFFu) << 24);
+                }
             }
         } else {
             // 32-bit chunk, row and block indices (M * K / 16 < 2^32 on this path)

@@ -73,6 +73,28 @@ def test_nvfp4_1d_parity(ora, M, K):
     _nvfp4_check(ora, x, what=f"nvfp4 1d {M}x{K}")
 
 
+@pytest.mark.parametrize("rht", [None, 0x5A5A])
+@pytest.mark.parametrize("fos", [False, True])
+def test_nvfp4_input_16_byte_aligned(ora, rht, fos):
+    """A contiguous input that starts 16 bytes past a 32-byte boundary (the
+    least alignment the boundary accepts) goes through the flat amax and 1x16
+    kernels like an aligned one, and the result is the oracle's."""
+    M, K = 64, 512
+    x = edge_tensor(M, K, seed=77)
+    buf = torch.zeros(M * K + 8, dtype=torch.bfloat16, device="cuda")
+    xd = buf[8:].view(M, K)
+    xd.copy_(dev(x))
+    assert xd.data_ptr() % 32 == 16
+    codes, sf, gs = api.quant_nvfp4(xd, four_over_six=fos, rht_mask=rht)
+    a = api.amax(xd, rht_mask=rht)
+    assert bsq.bsq_check() == 0
+    oc, osf, og = ora.quant_nvfp4(bits(x), four_over_six=fos, rht_mask=rht)
+    assert np.float32(gs.item()) == np.float32(og)
+    assert np.float32(a.item()) == np.float32(ora.amax(bits(x), rht_mask=rht))
+    assert_codes_equal(host_u8(codes), oc, "codes (16-byte aligned input)")
+    assert_codes_equal(sf_canonical(ora, sf, M, K // 16), osf, "sf (16-byte aligned input)")
+
+
 @pytest.mark.parametrize("block_2d", [False, True])
 def test_nvfp4_two_pass_path(ora, knobs, block_2d):
     """The separate amax and quantize kernels (what gathered, grouped and 4/6

@@ -159,8 +159,6 @@ __global__ void __launch_bounds__(384, SPLITK == 1 ? 1 : 2)
     // rank-0 CTA (distributed shared memory) in rank order.  Three stages
     // (86 KB) and 256 TMEM columns per CTA, so that two CTAs share an SM.
     static_assert(SPLITK == 1 || (SWAP && BN == 64 && !GROUPED), "split-K: the skinny swap-AB tile only");
-    grid_dependency_wait();
-    grid_dependents_launch();
     using C_ = Cfg<FMT, BN, SPLITK == 1 ? 8 : 3>;
     constexpr int kTmemCols = SPLITK == 1 ? 512 : 256;
     using T = typename C_::T;
@@ -217,6 +215,15 @@ __global__ void __launch_bounds__(384, SPLITK == 1 ? 1 : 2)
         prefetch_tmap(&tmA);
         prefetch_tmap(&tmB);
     }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(&tmem_base_slot), kTmemCols);
+        tmem_relinquish();
+    }
+    // The set-up above touches no global memory, so it overlaps the previous
+    // kernel under launch overlap; from here on the previous kernel has
+    // completed and its writes are visible.
+    grid_dependency_wait();
+    grid_dependents_launch();
     // grouped: per-group tile prefix (one warp, 32 groups per step)
     int64_t total_tiles = m_tiles * n_tiles;
     if (GROUPED) {
@@ -242,10 +249,6 @@ __global__ void __launch_bounds__(384, SPLITK == 1 ? 1 : 2)
             }
             if (lane == 0) tile_start[p.G] = carry;
         }
-    }
-    if (warp == 1) {
-        tmem_alloc(smem_u32(&tmem_base_slot), kTmemCols);
-        tmem_relinquish();
     }
     tc_fence_before();
     __syncthreads();
@@ -833,6 +836,8 @@ __global__ void __launch_bounds__(448, 1)
                     const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
                     const __grid_constant__ CUtensorMap tmC, const GemmParams p) {
     static_assert(!QOUT || OUT_BF16, "the quantizing epilogue quantizes the bf16 output");
+    // the previous kernel in the stream has completed before anything here
+    // (waiting after the set-up, as the single-CTA kernel does, measured slower)
     grid_dependency_wait();
     grid_dependents_launch();
     using C_ = Cfg2<FMT, GROUPED>;
@@ -1488,7 +1493,8 @@ int run_pair(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &ts
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
-    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // the kernel waits first (grid_dependency_wait)
+    // the kernel waits for the previous one (grid_dependency_wait) before any global access
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = kernel_choice(BSQ_KNOB_LAUNCH_OVERLAP) != 0 ? 2 : 1;
@@ -1523,7 +1529,8 @@ int run_splitk(const CUtensorMap &ta, const CUtensorMap &tb, const GemmParams &p
     attr[0].val.clusterDim.x = S;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
-    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // the kernel waits first (grid_dependency_wait)
+    // the kernel waits for the previous one (grid_dependency_wait) before any global access
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = kernel_choice(BSQ_KNOB_LAUNCH_OVERLAP) != 0 ? 2 : 1;

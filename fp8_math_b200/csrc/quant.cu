@@ -584,9 +584,10 @@ __global__ void __launch_bounds__(nvs::kThreads, 2) quant_nvfp4_stream_kernel(
     __shared__ int ok_sh;
     const NvChunks g = nv_chunks<TWO_D>(M, K);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    // chunks of this CTA: c = blockIdx.x + i * gridDim.x, i < my
-    const int64_t my = blockIdx.x < g.count ? (g.count - 1 - blockIdx.x) / gridDim.x + 1 : 0;
-    const int64_t total = (MODE == nvs::FUSED ? 2 : 1) * my;  // stage fills in this CTA's sequence
+    // chunks of this CTA: c = blockIdx.x + i * gridDim.x, i < my (32-bit
+    // counters: fewer than 2^32 chunks on this path)
+    const uint32_t my = blockIdx.x < g.count ? (uint32_t)(g.count - 1 - blockIdx.x) / gridDim.x + 1 : 0u;
+    const uint32_t total = (MODE == nvs::FUSED ? 2u : 1u) * my;  // stage fills in this CTA's sequence
     if (threadIdx.x == 0) {
         for (int i = 0; i < nvs::kStages; i++) {
             mbar_init(smem_u32(&full_bar[i]), 1);
@@ -597,15 +598,15 @@ __global__ void __launch_bounds__(nvs::kThreads, 2) quant_nvfp4_stream_kernel(
     }
     __syncthreads();
     // j-th fill of the sequence -> chunk index (FUSED: forward, then reverse)
-    auto chunk_of = [&](int64_t j) -> int64_t {
-        const int64_t i = (MODE == nvs::FUSED && j >= my) ? (2 * my - 1 - j) : j;
+    auto chunk_of = [&](uint32_t j) -> uint32_t {
+        const uint32_t i = (MODE == nvs::FUSED && j >= my) ? (2 * my - 1 - j) : j;
         return blockIdx.x + i * gridDim.x;
     };
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         uint32_t armed = 0, armed_par = 0;
-        for (int64_t j = 0; j < total; j++) {
+        for (uint32_t j = 0; j < total; j++) {
             const int s = (int)(j % nvs::kStages);
             const uint32_t ph = (uint32_t)((j / nvs::kStages) & 1);
             bool ok = true;
@@ -650,16 +651,16 @@ __global__ void __launch_bounds__(nvs::kThreads, 2) quant_nvfp4_stream_kernel(
     const int t = threadIdx.x - 32;  // 0..255
     uint32_t sw[8];
     rht_sign_words(mask, sw);
-    int64_t j = 0;
+    uint32_t j = 0;
     // waits for fill j; false when the CTA gives up
-    auto acquire = [&](int64_t jj) -> const uint8_t * {
+    auto acquire = [&](uint32_t jj) -> const uint8_t * {
         const int s = (int)(jj % nvs::kStages);
         const uint32_t ph = (uint32_t)((jj / nvs::kStages) & 1);
         const bool ok = mbar_wait(smem_u32(&full_bar[s]), ph, &abort_flag, err, 32, nvs::kTimeoutNs);
         if (!__all_sync(0xFFFFFFFFu, ok)) return nullptr;
         return ring + s * nvs::kStageBytes;
     };
-    auto release = [&](int64_t jj) {
+    auto release = [&](uint32_t jj) {
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&empty_bar[jj % nvs::kStages]));
     };
@@ -768,7 +769,7 @@ __global__ void __launch_bounds__(nvs::kThreads, 2) quant_nvfp4_stream_kernel(
     const unsigned int all_read = 2u * gridDim.x;
 
     // ---- quantize this CTA's chunks (FUSED: in reverse order)
-    const int64_t jend = (MODE == nvs::FUSED) ? 2 * my : my;
+    const uint32_t jend = (MODE == nvs::FUSED) ? 2 * my : my;
     for (; j < jend && alive; j++) {
         const uint8_t *st = acquire(j);
         if (!st) break;

@@ -1272,7 +1272,9 @@ __global__ void __launch_bounds__(256) quant_mxfp8_row_span_kernel(
 // chunk of 8 consecutive m; the four lanes with the same kg share that
 // column's block of 32 (two-step shuffle max).  Warp tiles run m-fastest, so
 // consecutive warps write adjacent 32-byte pieces of each output row.
-template <bool SR>
+// I: the output index type (uint32_t when M * K < 2^31: the code offset,
+// the Philox counter and the scale offset in single 32-bit instructions).
+template <bool SR, typename I>
 __global__ void __launch_bounds__(256) quant_mxfp8_col_kernel(
     const uint16_t *__restrict__ xin, int64_t M, int64_t K, int64_t ldx, uint32_t ntile, DivU32 div_mt,
     const __grid_constant__ PhiloxKeys keys, uint32_t stream_id, uint8_t *__restrict__ codes,
@@ -1295,7 +1297,8 @@ __global__ void __launch_bounds__(256) quant_mxfp8_col_kernel(
         }
 #pragma unroll
         for (int j = 0; j < 8; j++) {
-            const int64_t k = k0 + j;
+            const I k = (I)k0 + (I)j;
+            const I o = k * (I)M + (I)m0;  // output offset of this chunk
             uint2 q;
             uint32_t sb;
             bool zero;
@@ -1309,7 +1312,7 @@ __global__ void __launch_bounds__(256) quant_mxfp8_col_kernel(
                 m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
                 m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
                 sb = mx_scale_code_bf16(m);
-                q = mx_sr8_bf16(p, a, sb, mx_draws((uint64_t)(k * M + m0) >> 3, keys, stream_id));
+                q = mx_sr8_bf16(p, a, sb, mx_draws((uint64_t)(o >> 3), keys, stream_id));
                 zero = m == 0u;
             } else {
                 float v[8];
@@ -1325,8 +1328,13 @@ __global__ void __launch_bounds__(256) quant_mxfp8_col_kernel(
             }
             if (zero) q = make_uint2(0u, 0u);
             if (kvalid) {
-                *reinterpret_cast<uint2 *>(codes + k * M + m0) = q;
-                if (mg == 0) sf[sf_offset(k, m0 >> 5, MB)] = (uint8_t)sb;
+                *reinterpret_cast<uint2 *>(codes + (size_t)o) = q;
+                if (mg == 0) {
+                    // sf_offset(k, m0 / 32, MB) in the index type
+                    const I b = (I)(m0 >> 5), bt = ((I)MB + 3) >> 2;
+                    const I so = (((k >> 7) * bt + (b >> 2)) << 9) + ((k & 31) << 4) + (((k >> 5) & 3) << 2) + (b & 3);
+                    sf[(size_t)so] = (uint8_t)sb;
+                }
             }
         }
     }
@@ -2271,11 +2279,13 @@ void launch_quant_mxfp8(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, bo
     const uint32_t ntile = (uint32_t)((M >> 5) * ((K + 63) >> 6));
     const DivU32 dmt = divu32_for((uint32_t)(M >> 5));
     if (sr) {
-        const int grid = grid_for(ntile, 8, resident_ctas<quant_mxfp8_col_kernel<true>>(num_sms));
-        quant_mxfp8_col_kernel<true><<<grid, 256, 0, s>>>(x, M, K, ldx, ntile, dmt, keys, stream_id, codes, sf);
+#define BSQ_MXC(S, I)                                                                                        \
+    quant_mxfp8_col_kernel<S, I><<<grid_for(ntile, 8, resident_ctas<quant_mxfp8_col_kernel<S, I>>(num_sms)), 256, 0, \
+                                   s>>>(x, M, K, ldx, ntile, dmt, keys, stream_id, codes, sf)
+        if (M * K < (int64_t(1) << 31)) BSQ_MXC(true, uint32_t); else BSQ_MXC(true, int64_t);
     } else {
-        const int grid = grid_for(ntile, 8, resident_ctas<quant_mxfp8_col_kernel<false>>(num_sms));
-        quant_mxfp8_col_kernel<false><<<grid, 256, 0, s>>>(x, M, K, ldx, ntile, dmt, keys, stream_id, codes, sf);
+        if (M * K < (int64_t(1) << 31)) BSQ_MXC(false, uint32_t); else BSQ_MXC(false, int64_t);
+#undef BSQ_MXC
     }
 }
 

@@ -399,6 +399,13 @@ BSQ_DEV int64_t sf_offset(int64_t r, int64_t b, int64_t nblk) {
     int64_t bt = (nblk + 3) >> 2;
     return (((r >> 7) * bt + (b >> 2)) << 9) + ((r & 31) << 4) + (((r >> 5) & 3) << 2) + (b & 3);
 }
+// sf_offset in the index type I: uint32_t where the scale buffer holds fewer
+// than 2^31 bytes, so that the offset takes single 32-bit instructions.
+template <typename I>
+BSQ_DEV I sf_offset_t(I r, I b, I nblk) {
+    const I bt = (nblk + 3) >> 2;
+    return (((r >> 7) * bt + (b >> 2)) << 9) + ((r & 31) << 4) + (((r >> 5) & 3) << 2) + (b & 3);
+}
 // Offset of the 4-byte word holding blocks 4j..4j+3 of row r.
 BSQ_DEV int64_t sf_word_offset(int64_t r, int64_t b4, int64_t nblk) {
     int64_t bt = (nblk + 3) >> 2;

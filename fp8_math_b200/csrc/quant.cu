@@ -1348,7 +1348,9 @@ __global__ void __launch_bounds__(256) quant_mxfp8_col_kernel(
 // with the column block's scale; a chunk whose rescaled values are all E4M3
 // values (the common case: an E4M3 value times a power of two) needs no
 // rounding and takes the nearest-even conversion without drawing.
-template <bool SR>
+// I: the index type of offsets and Philox counters (uint32_t when the
+// tensor has fewer than 2^31 elements: single 32-bit instructions).
+template <bool SR, typename I>
 __global__ void __launch_bounds__(256) requant_transpose_kernel(
     const uint8_t *__restrict__ codes_in, const uint8_t *__restrict__ sf_in, int64_t M, int64_t K, uint32_t ntile,
     DivU32 div_mt, const __grid_constant__ PhiloxKeys keys, uint32_t stream_id, uint8_t *__restrict__ codes,
@@ -1365,15 +1367,16 @@ __global__ void __launch_bounds__(256) requant_transpose_kernel(
         float sc[8];
 #pragma unroll
         for (int i = 0; i < 8; i++) {
-            const uint2 r = kvalid ? __ldg(reinterpret_cast<const uint2 *>(codes_in + (m0 + i) * K + k0)) : make_uint2(0, 0);
+            const uint2 r = kvalid ? __ldg(reinterpret_cast<const uint2 *>(codes_in + (size_t)((I)(m0 + i) * (I)K + (I)k0))) : make_uint2(0, 0);
             w[i][0] = r.x;
             w[i][1] = r.y;
-            sc[i] = kvalid ? exp2i((int)__ldg(sf_in + sf_offset(m0 + i, k0 >> 5, KB)) - 127) : 0.0f;
+            sc[i] = kvalid ? exp2i((int)__ldg(sf_in + (size_t)sf_offset_t<I>((I)(m0 + i), (I)(k0 >> 5), (I)KB)) - 127) : 0.0f;
         }
         float odd[8];  // column j + 1, decoded with column j
 #pragma unroll
         for (int j = 0; j < 8; j++) {
-            const int64_t k = k0 + j;
+            const I k = (I)k0 + (I)j;
+            const I o = k * (I)M + (I)m0;  // output offset of this chunk
             float v[8];
 #pragma unroll
             for (int i = 0; i < 8; i++) {
@@ -1391,10 +1394,10 @@ __global__ void __launch_bounds__(256) requant_transpose_kernel(
             m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
             m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
             const uint32_t sb = mx_scale_code(m);
-            const uint2 q = mx_encode8<SR, true>(v, m == 0.0f, sb, (uint64_t)(k * M + m0) >> 3, keys, stream_id);
+            const uint2 q = mx_encode8<SR, true>(v, m == 0.0f, sb, (uint64_t)(o >> 3), keys, stream_id);
             if (kvalid) {
-                *reinterpret_cast<uint2 *>(codes + k * M + m0) = q;
-                if (mg == 0) sf[sf_offset(k, m0 >> 5, MB)] = (uint8_t)sb;
+                *reinterpret_cast<uint2 *>(codes + (size_t)o) = q;
+                if (mg == 0) sf[(size_t)sf_offset_t<I>(k, (I)(m0 >> 5), (I)MB)] = (uint8_t)sb;
             }
         }
     }
@@ -1408,7 +1411,9 @@ __global__ void __launch_bounds__(256) requant_transpose_kernel(
 // hold one row block of 32, reduced with shuffles over lane bits 2 and 3.
 // Row output: codes_r [M][K], SR draws of row * K + col with stream_r;
 // column output: codes_c [K][M], draws of k * M + m with stream_c.
-template <bool SR>
+// I: the index type of offsets and Philox counters (uint32_t when the
+// tensor has fewer than 2^31 elements: single 32-bit instructions).
+template <bool SR, typename I>
 __global__ void __launch_bounds__(256) quant_mxfp8_rowcol_kernel(
     const uint16_t *__restrict__ x, int64_t M, int64_t K, int64_t ldx, uint32_t ntile, DivU32 div_mt,
     const __grid_constant__ PhiloxKeys keys, uint32_t stream_r, uint32_t stream_c, uint8_t *__restrict__ codes_r,
@@ -1431,7 +1436,8 @@ __global__ void __launch_bounds__(256) quant_mxfp8_rowcol_kernel(
         // ---- row-wise: row m0 + i, columns k0 .. k0 + 7
 #pragma unroll
         for (int i = 0; i < 8; i++) {
-            const int64_t row = m0 + i;
+            const I row = (I)m0 + (I)i;
+            const I orow = row * (I)K + (I)k0;  // row-wise output offset
             uint32_t sb;
             uint2 q;
             if (SR) {
@@ -1440,7 +1446,7 @@ __global__ void __launch_bounds__(256) quant_mxfp8_rowcol_kernel(
                 m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 4));
                 m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 8));
                 sb = mx_scale_code_bf16(m);
-                q = mx_sr8_bf16(w[i], a, sb, mx_draws((uint64_t)(row * K + k0) >> 3, keys, stream_r));
+                q = mx_sr8_bf16(w[i], a, sb, mx_draws((uint64_t)(orow >> 3), keys, stream_r));
                 if (m == 0u) q = make_uint2(0u, 0u);
             } else {
                 float v[8];
@@ -1457,14 +1463,15 @@ __global__ void __launch_bounds__(256) quant_mxfp8_rowcol_kernel(
                 q = mx_encode8<false>(v, m == 0.0f, sb, 0, keys, 0u);
             }
             if (kvalid) {
-                *reinterpret_cast<uint2 *>(codes_r + row * K + k0) = q;
-                if ((kg & 3) == 0) sf_r[sf_offset(row, k0 >> 5, KB)] = (uint8_t)sb;
+                *reinterpret_cast<uint2 *>(codes_r + (size_t)orow) = q;
+                if ((kg & 3) == 0) sf_r[(size_t)sf_offset_t<I>(row, (I)(k0 >> 5), (I)KB)] = (uint8_t)sb;
             }
         }
         // ---- column-wise: column k0 + j, rows m0 .. m0 + 7
 #pragma unroll
         for (int j = 0; j < 8; j++) {
-            const int64_t k = k0 + j;
+            const I k = (I)k0 + (I)j;
+            const I o = k * (I)M + (I)m0;  // column-wise output offset
             uint32_t sb;
             uint2 q;
             if (SR) {
@@ -1476,7 +1483,7 @@ __global__ void __launch_bounds__(256) quant_mxfp8_rowcol_kernel(
                 m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
                 m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
                 sb = mx_scale_code_bf16(m);
-                q = mx_sr8_bf16(p, a, sb, mx_draws((uint64_t)(k * M + m0) >> 3, keys, stream_c));
+                q = mx_sr8_bf16(p, a, sb, mx_draws((uint64_t)(o >> 3), keys, stream_c));
                 if (m == 0u) q = make_uint2(0u, 0u);
             } else {
                 float v[8];
@@ -1490,8 +1497,8 @@ __global__ void __launch_bounds__(256) quant_mxfp8_rowcol_kernel(
                 q = mx_encode8<false>(v, m == 0.0f, sb, 0, keys, 0u);
             }
             if (kvalid) {
-                *reinterpret_cast<uint2 *>(codes_c + k * M + m0) = q;
-                if (mg == 0) sf_c[sf_offset(k, m0 >> 5, MB)] = (uint8_t)sb;
+                *reinterpret_cast<uint2 *>(codes_c + (size_t)o) = q;
+                if (mg == 0) sf_c[(size_t)sf_offset_t<I>(k, (I)(m0 >> 5), (I)MB)] = (uint8_t)sb;
             }
         }
     }
@@ -1505,7 +1512,9 @@ __global__ void __launch_bounds__(256) quant_mxfp8_rowcol_kernel(
 // and columns 8 kg .. 8 kg + 7 (one 32-bit code load and one scale byte per
 // row: the 8 columns sit in one 16-block); the four lanes of a kg share the
 // output block of column 8 kg + j.
-template <bool SR>
+// I: the index type of offsets and Philox counters (uint32_t when the
+// tensor has fewer than 2^31 elements: single 32-bit instructions).
+template <bool SR, typename I>
 __global__ void __launch_bounds__(256) requant_nvfp4_mxfp8_kernel(
     const uint8_t *__restrict__ codes_in, const uint8_t *__restrict__ sf_in, const float *gs, int64_t R, int64_t C,
     uint32_t ntile, DivU32 div_mt, const __grid_constant__ PhiloxKeys keys, uint32_t stream_id,
@@ -1523,20 +1532,21 @@ __global__ void __launch_bounds__(256) requant_nvfp4_mxfp8_kernel(
         float sbv[8];                // its block scale
 #pragma unroll
         for (int i = 0; i < 8; i++) {
-            w[i] = kvalid ? __ldg(reinterpret_cast<const uint32_t *>(codes_in + (m0 + i) * (C >> 1) + (k0 >> 1))) : 0u;
-            sbv[i] = kvalid ? e4m3_to_f32(__ldg(sf_in + sf_offset(m0 + i, k0 >> 4, CB16))) : 0.0f;
+            w[i] = kvalid ? __ldg(reinterpret_cast<const uint32_t *>(codes_in + (size_t)((I)(m0 + i) * (I)(C >> 1) + (I)(k0 >> 1)))) : 0u;
+            sbv[i] = kvalid ? e4m3_to_f32(__ldg(sf_in + (size_t)sf_offset_t<I>((I)(m0 + i), (I)(k0 >> 4), (I)CB16))) : 0.0f;
         }
         auto column = [&](int j, const float (&c)[8]) {
-            const int64_t k = k0 + j;
+            const I k = (I)k0 + (I)j;
+            const I o = k * (I)R + (I)m0;  // output offset of this chunk
             float m = fmax3(fmax3(fabsf(c[0]), fabsf(c[1]), fabsf(c[2])), fmax3(fabsf(c[3]), fabsf(c[4]), fabsf(c[5])),
                             fmaxf(fabsf(c[6]), fabsf(c[7])));
             m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
             m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
             const uint32_t sb = mx_scale_code(m);
-            const uint2 q = mx_encode8<SR, false, true>(c, m == 0.0f, sb, (uint64_t)(k * R + m0) >> 3, keys, stream_id);
+            const uint2 q = mx_encode8<SR, false, true>(c, m == 0.0f, sb, (uint64_t)(o >> 3), keys, stream_id);
             if (kvalid) {
-                *reinterpret_cast<uint2 *>(codes + k * R + m0) = q;
-                if (mg == 0) sf[sf_offset(k, m0 >> 5, RB)] = (uint8_t)sb;
+                *reinterpret_cast<uint2 *>(codes + (size_t)o) = q;
+                if (mg == 0) sf[(size_t)sf_offset_t<I>(k, (I)(m0 >> 5), (I)RB)] = (uint8_t)sb;
             }
         };
         // columns 2 jj and 2 jj + 1 (byte jj of every row), decoded as needed
@@ -2295,15 +2305,13 @@ void launch_requant_transpose(const uint8_t *codes_row, const uint8_t *sf_row, i
     const PhiloxKeys keys = philox_keys((uint32_t)seed, (uint32_t)(seed >> 32));
     const uint32_t ntile = (uint32_t)((M >> 5) * ((K + 63) >> 6));
     const DivU32 dmt = divu32_for((uint32_t)(M >> 5));
-    if (sr) {
-        const int grid = grid_for(ntile, 8, resident_ctas<requant_transpose_kernel<true>>(num_sms));
-        requant_transpose_kernel<true><<<grid, 256, 0, s>>>(codes_row, sf_row, M, K, ntile, dmt, keys, stream_id,
-                                                            codes_col, sf_col);
-    } else {
-        const int grid = grid_for(ntile, 8, resident_ctas<requant_transpose_kernel<false>>(num_sms));
-        requant_transpose_kernel<false><<<grid, 256, 0, s>>>(codes_row, sf_row, M, K, ntile, dmt, keys, stream_id,
-                                                             codes_col, sf_col);
-    }
+#define BSQ_RQT(S, I)                                                                                        \
+    requant_transpose_kernel<S, I><<<grid_for(ntile, 8, resident_ctas<requant_transpose_kernel<S, I>>(num_sms)), 256, \
+                                     0, s>>>(codes_row, sf_row, M, K, ntile, dmt, keys, stream_id, codes_col, sf_col)
+    const bool i32 = M * K < (int64_t(1) << 31);
+    if (sr) { if (i32) BSQ_RQT(true, uint32_t); else BSQ_RQT(true, int64_t); }
+    else { if (i32) BSQ_RQT(false, uint32_t); else BSQ_RQT(false, int64_t); }
+#undef BSQ_RQT
 }
 
 void launch_quant_mxfp8_rowcol(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, bool sr, uint64_t seed,
@@ -2312,15 +2320,14 @@ void launch_quant_mxfp8_rowcol(const uint16_t *x, int64_t M, int64_t K, int64_t 
     const PhiloxKeys keys = philox_keys((uint32_t)seed, (uint32_t)(seed >> 32));
     const uint32_t ntile = (uint32_t)((M >> 5) * ((K + 63) >> 6));
     const DivU32 dmt = divu32_for((uint32_t)(M >> 5));
-    if (sr) {
-        const int grid = grid_for(ntile, 8, resident_ctas<quant_mxfp8_rowcol_kernel<true>>(num_sms));
-        quant_mxfp8_rowcol_kernel<true><<<grid, 256, 0, s>>>(x, M, K, ldx, ntile, dmt, keys, stream_r, stream_c,
-                                                             codes_r, sf_r, codes_c, sf_c);
-    } else {
-        const int grid = grid_for(ntile, 8, resident_ctas<quant_mxfp8_rowcol_kernel<false>>(num_sms));
-        quant_mxfp8_rowcol_kernel<false><<<grid, 256, 0, s>>>(x, M, K, ldx, ntile, dmt, keys, stream_r, stream_c,
-                                                              codes_r, sf_r, codes_c, sf_c);
-    }
+#define BSQ_RC(S, I)                                                                                          \
+    quant_mxfp8_rowcol_kernel<S, I><<<grid_for(ntile, 8, resident_ctas<quant_mxfp8_rowcol_kernel<S, I>>(num_sms)),  \
+                                      256, 0, s>>>(x, M, K, ldx, ntile, dmt, keys, stream_r, stream_c, codes_r, sf_r, \
+                                                   codes_c, sf_c)
+    const bool i32 = M * K < (int64_t(1) << 31);
+    if (sr) { if (i32) BSQ_RC(true, uint32_t); else BSQ_RC(true, int64_t); }
+    else { if (i32) BSQ_RC(false, uint32_t); else BSQ_RC(false, int64_t); }
+#undef BSQ_RC
 }
 
 void launch_requant_nvfp4_mxfp8(const uint8_t *codes_in, const uint8_t *sf_in, const float *gs, int64_t R, int64_t C,
@@ -2329,15 +2336,13 @@ void launch_requant_nvfp4_mxfp8(const uint8_t *codes_in, const uint8_t *sf_in, c
     const PhiloxKeys keys = philox_keys((uint32_t)seed, (uint32_t)(seed >> 32));
     const uint32_t ntile = (uint32_t)((R >> 5) * ((C + 63) >> 6));
     const DivU32 dmt = divu32_for((uint32_t)(R >> 5));
-    if (sr) {
-        const int grid = grid_for(ntile, 8, resident_ctas<requant_nvfp4_mxfp8_kernel<true>>(num_sms));
-        requant_nvfp4_mxfp8_kernel<true><<<grid, 256, 0, s>>>(codes_in, sf_in, gs, R, C, ntile, dmt, keys, stream_id,
-                                                              codes, sf);
-    } else {
-        const int grid = grid_for(ntile, 8, resident_ctas<requant_nvfp4_mxfp8_kernel<false>>(num_sms));
-        requant_nvfp4_mxfp8_kernel<false><<<grid, 256, 0, s>>>(codes_in, sf_in, gs, R, C, ntile, dmt, keys,
-                                                               stream_id, codes, sf);
-    }
+#define BSQ_RQ4(S, I)                                                                                         \
+    requant_nvfp4_mxfp8_kernel<S, I><<<grid_for(ntile, 8, resident_ctas<requant_nvfp4_mxfp8_kernel<S, I>>(num_sms)), \
+                                       256, 0, s>>>(codes_in, sf_in, gs, R, C, ntile, dmt, keys, stream_id, codes, sf)
+    const bool i32 = R * C < (int64_t(1) << 31);
+    if (sr) { if (i32) BSQ_RQ4(true, uint32_t); else BSQ_RQ4(true, int64_t); }
+    else { if (i32) BSQ_RQ4(false, uint32_t); else BSQ_RQ4(false, int64_t); }
+#undef BSQ_RQ4
 }
 
 void launch_quant_mxfp4(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, bool sr, uint64_t seed,

@@ -406,6 +406,11 @@ BSQ_DEV I sf_offset_t(I r, I b, I nblk) {
     const I bt = (nblk + 3) >> 2;
     return (((r >> 7) * bt + (b >> 2)) << 9) + ((r & 31) << 4) + (((r >> 5) & 3) << 2) + (b & 3);
 }
+template <typename I>
+BSQ_DEV I sf_word_offset_t(I r, I b4, I nblk) {
+    const I bt = (nblk + 3) >> 2;
+    return (((r >> 7) * bt + b4) << 9) + ((r & 31) << 4) + (((r >> 5) & 3) << 2);
+}
 // Offset of the 4-byte word holding blocks 4j..4j+3 of row r.
 BSQ_DEV int64_t sf_word_offset(int64_t r, int64_t b4, int64_t nblk) {
     int64_t bt = (nblk + 3) >> 2;

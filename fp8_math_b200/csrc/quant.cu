@@ -1107,7 +1107,9 @@ BSQ_DEV uint2 mx_sr8_bf16(const uint32_t p[4], const uint32_t a[4], uint32_t sb,
     return make_uint2(__byte_perm(u[0], u[1], 0x7531u), __byte_perm(u[2], u[3], 0x7531u));
 }
 // Row-wise: one thread per 8 elements, 4 lanes per block of 32.
-template <bool SR>
+// I: the index type of the per-chunk offsets and Philox counters (uint32_t
+// when M * ldx < 2^31: single 32-bit instructions).
+template <bool SR, typename I>
 __global__ void __launch_bounds__(256) quant_mxfp8_row_kernel(
     const uint16_t *__restrict__ x, int64_t M, int64_t K, int64_t ldx, const __grid_constant__ PhiloxKeys keys,
     uint32_t stream_id, uint8_t *__restrict__ codes, uint8_t *__restrict__ sf, RowMap map) {
@@ -1126,7 +1128,7 @@ __global__ void __launch_bounds__(256) quant_mxfp8_row_kernel(
             const bool valid = row_ok && c8 < K8;
             const int64_t cc = c8 < K8 ? c8 : K8 - 1;
             float v[8];
-            load8_bf16(x + rr * ldx + cc * 8, v);
+            load8_bf16(x + (size_t)((I)rr * (I)ldx + (I)cc * 8), v);
             float m = 0.0f;
 #pragma unroll
             for (int i = 0; i < 8; i++) m = fmaxf(m, fabsf(v[i]));
@@ -1134,9 +1136,10 @@ __global__ void __launch_bounds__(256) quant_mxfp8_row_kernel(
             m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
             const bool zero = (m == 0.0f);
             const uint32_t sb = mx_scale_code(m);
-            const uint64_t chunk = (uint64_t)(rr * K + cc * 8) >> 3;
+            const I o = (I)rr * (I)K + (I)cc * 8;  // output offset of this chunk
+            const uint64_t chunk = (uint64_t)(o >> 3);
             uint2 q = mx_encode8<SR>(v, zero, sb, chunk, keys, stream_id);
-            if (valid) *reinterpret_cast<uint2 *>(codes + rr * K + cc * 8) = q;
+            if (valid) *reinterpret_cast<uint2 *>(codes + (size_t)o) = q;
             // scale byte: lanes 4j hold block j; 4 blocks (16 lanes) per word
             const int64_t kb = cc >> 2;
             if (pack4) {
@@ -1144,10 +1147,10 @@ __global__ void __launch_bounds__(256) quant_mxfp8_row_kernel(
                 uint32_t b2 = __shfl_down_sync(0xFFFFFFFFu, sb, 8);
                 uint32_t b3 = __shfl_down_sync(0xFFFFFFFFu, sb, 12);
                 if (valid && (lane & 15) == 0)
-                    *reinterpret_cast<uint32_t *>(sf + sf_word_offset(rr, kb >> 2, KB)) =
+                    *reinterpret_cast<uint32_t *>(sf + (size_t)sf_word_offset_t<I>((I)rr, (I)(kb >> 2), (I)KB)) =
                         sb | (b1 << 8) | (b2 << 16) | (b3 << 24);
             } else if (valid && (lane & 3) == 0) {
-                sf[sf_offset(rr, kb, KB)] = (uint8_t)sb;
+                sf[(size_t)sf_offset_t<I>((I)rr, (I)kb, (I)KB)] = (uint8_t)sb;
             }
         }
     }
@@ -1628,7 +1631,9 @@ BSQ_DEV uint32_t mx4_encode8(const float v[8], bool zero, uint32_t sb, uint64_t 
 // shuffles for the block maximum), rows mapped to lanes as in the MXFP8 row
 // kernel; one 32-bit code store per chunk, the scale bytes of 4 blocks
 // packed into one 32-bit store when a row holds a multiple of 4 blocks.
-template <bool SR>
+// I: the index type of the per-chunk offsets and Philox counters (uint32_t
+// when M * ldx < 2^31: single 32-bit instructions).
+template <bool SR, typename I>
 __global__ void __launch_bounds__(256) quant_mxfp4_row_kernel(
     const uint16_t *__restrict__ x, int64_t M, int64_t K, int64_t ldx, const __grid_constant__ PhiloxKeys keys,
     uint32_t stream_id, uint8_t *__restrict__ codes, uint8_t *__restrict__ sf, RowMap map) {
@@ -1647,24 +1652,25 @@ __global__ void __launch_bounds__(256) quant_mxfp4_row_kernel(
             const bool valid = row_ok && c8 < K8;
             const int64_t cc = c8 < K8 ? c8 : K8 - 1;
             float v[8];
-            load8_bf16(x + rr * ldx + cc * 8, v);
+            load8_bf16(x + (size_t)((I)rr * (I)ldx + (I)cc * 8), v);
             float m = fmax3(fmax3(fabsf(v[0]), fabsf(v[1]), fabsf(v[2])), fmax3(fabsf(v[3]), fabsf(v[4]), fabsf(v[5])),
                             fmaxf(fabsf(v[6]), fabsf(v[7])));
             m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
             m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
             const uint32_t sb = mx4_scale_code(m);
-            const uint32_t q = mx4_encode8<SR>(v, m == 0.0f, sb, (uint64_t)(rr * K + cc * 8) >> 3, keys, stream_id);
-            if (valid) *reinterpret_cast<uint32_t *>(codes + rr * (K >> 1) + cc * 4) = q;
+            const I o = (I)rr * (I)K + (I)cc * 8;  // element offset of this chunk
+            const uint32_t q = mx4_encode8<SR>(v, m == 0.0f, sb, (uint64_t)(o >> 3), keys, stream_id);
+            if (valid) *reinterpret_cast<uint32_t *>(codes + (size_t)(o >> 1)) = q;
             const int64_t kb = cc >> 2;
             if (pack4) {
                 const uint32_t b1 = __shfl_down_sync(0xFFFFFFFFu, sb, 4);
                 const uint32_t b2 = __shfl_down_sync(0xFFFFFFFFu, sb, 8);
                 const uint32_t b3 = __shfl_down_sync(0xFFFFFFFFu, sb, 12);
                 if (valid && (lane & 15) == 0)
-                    *reinterpret_cast<uint32_t *>(sf + sf_word_offset(rr, kb >> 2, KB)) =
+                    *reinterpret_cast<uint32_t *>(sf + (size_t)sf_word_offset_t<I>((I)rr, (I)(kb >> 2), (I)KB)) =
                         sb | (b1 << 8) | (b2 << 16) | (b3 << 24);
             } else if (valid && (lane & 3) == 0) {
-                sf[sf_offset(rr, kb, KB)] = (uint8_t)sb;
+                sf[(size_t)sf_offset_t<I>((I)rr, (I)kb, (I)KB)] = (uint8_t)sb;
             }
         }
     }
@@ -2282,8 +2288,14 @@ void launch_quant_mxfp8(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, bo
         RowMap map{lpr_shift_for(K >> 3)};
         if (map.lpr_shift < 2) map.lpr_shift = 2;  // 4 lanes per block of 32
         const int grid = grid_for(M, 256 >> map.lpr_shift, num_sms * 8);
-        if (sr) quant_mxfp8_row_kernel<true><<<grid, 256, 0, s>>>(x, M, K, ldx, keys, stream_id, codes, sf, map);
-        else quant_mxfp8_row_kernel<false><<<grid, 256, 0, s>>>(x, M, K, ldx, keys, stream_id, codes, sf, map);
+        const bool i32 = M * ldx < (int64_t(1) << 31);
+        if (sr) {
+            if (i32) quant_mxfp8_row_kernel<true, uint32_t><<<grid, 256, 0, s>>>(x, M, K, ldx, keys, stream_id, codes, sf, map);
+            else quant_mxfp8_row_kernel<true, int64_t><<<grid, 256, 0, s>>>(x, M, K, ldx, keys, stream_id, codes, sf, map);
+        } else {
+            if (i32) quant_mxfp8_row_kernel<false, uint32_t><<<grid, 256, 0, s>>>(x, M, K, ldx, keys, stream_id, codes, sf, map);
+            else quant_mxfp8_row_kernel<false, int64_t><<<grid, 256, 0, s>>>(x, M, K, ldx, keys, stream_id, codes, sf, map);
+        }
         return;
     }
     const uint32_t ntile = (uint32_t)((M >> 5) * ((K + 63) >> 6));
@@ -2351,8 +2363,14 @@ void launch_quant_mxfp4(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, bo
     RowMap map{lpr_shift_for(K >> 3)};
     if (map.lpr_shift < 2) map.lpr_shift = 2;  // 4 lanes per block of 32
     const int grid = grid_for(M, 256 >> map.lpr_shift, num_sms * 8);
-    if (sr) quant_mxfp4_row_kernel<true><<<grid, 256, 0, s>>>(x, M, K, ldx, keys, stream_id, codes, sf, map);
-    else quant_mxfp4_row_kernel<false><<<grid, 256, 0, s>>>(x, M, K, ldx, keys, stream_id, codes, sf, map);
+    const bool i32 = M * ldx < (int64_t(1) << 31);
+    if (sr) {
+        if (i32) quant_mxfp4_row_kernel<true, uint32_t><<<grid, 256, 0, s>>>(x, M, K, ldx, keys, stream_id, codes, sf, map);
+        else quant_mxfp4_row_kernel<true, int64_t><<<grid, 256, 0, s>>>(x, M, K, ldx, keys, stream_id, codes, sf, map);
+    } else {
+        if (i32) quant_mxfp4_row_kernel<false, uint32_t><<<grid, 256, 0, s>>>(x, M, K, ldx, keys, stream_id, codes, sf, map);
+        else quant_mxfp4_row_kernel<false, int64_t><<<grid, 256, 0, s>>>(x, M, K, ldx, keys, stream_id, codes, sf, map);
+    }
 }
 
 void launch_quant_nvfp4_sr(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, bool block_2d, bool rht,

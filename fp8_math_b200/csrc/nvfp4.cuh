@@ -147,4 +147,21 @@ BSQ_DEV void store_sf(uint8_t *sf, bool valid, uint32_t sb, int64_t sf_row, int6
     }
 }
 
+// store_sf with the offset in the index type I (uint32_t where the scale
+// buffer holds fewer than 2^31 bytes); sf_row is read only when valid.
+template <typename I>
+BSQ_DEV void store_sf_t(uint8_t *sf, bool valid, uint32_t sb, I sf_row, I kb, I KB, bool pack4) {
+    if (pack4) {
+        uint32_t b1 = __shfl_down_sync(0xFFFFFFFFu, sb, 1);
+        uint32_t b2 = __shfl_down_sync(0xFFFFFFFFu, sb, 2);
+        uint32_t b3 = __shfl_down_sync(0xFFFFFFFFu, sb, 3);
+        if (valid && (threadIdx.x & 3) == 0) {
+            uint32_t w = (sb & 0xFFu) | ((b1 & 0xFFu) << 8) | ((b2 & 0xFFu) << 16) | ((b3 & 0xFFu) << 24);
+            *reinterpret_cast<uint32_t *>(sf + (size_t)sf_word_offset_t<I>(sf_row, kb >> 2, KB)) = w;
+        }
+    } else if (valid) {
+        sf[(size_t)sf_offset_t<I>(sf_row, kb, KB)] = (uint8_t)sb;
+    }
+}
+
 }  // namespace bsq

@@ -187,7 +187,9 @@ BSQ_DEV int64_t grouped_sf_row(int64_t row, int G, const int32_t *__restrict__ o
 // 1x16 blocks, rows (gathered, grouped): one thread per block of 16 (two
 // 16-byte loads, one 8-byte code store).  Loops are warp-uniform so that
 // shuffles see all lanes.
-template <bool RHT, bool FOS, bool GATHER, bool GROUPED>
+// I: the index type of the per-block offsets (uint32_t when the output holds
+// fewer than 2^31 elements; a source row's start stays 64-bit).
+template <bool RHT, bool FOS, bool GATHER, bool GROUPED, typename I>
 __global__ void __launch_bounds__(256) quant_nvfp4_1d_kernel(
     const uint16_t *__restrict__ x, int64_t M, int64_t K, int64_t ldx, uint32_t mask,
     const int32_t *__restrict__ row_index, int G, const int32_t *__restrict__ row_off,
@@ -216,12 +218,12 @@ __global__ void __launch_bounds__(256) quant_nvfp4_1d_kernel(
             const bool valid = row_ok && kb < KB;
             const int64_t kk = kb < KB ? kb : KB - 1;
             uint32_t w[8];
-            load_words16(rp + kk * 16, w);
+            load_words16(rp + (size_t)((I)kk * 16), w);
             uint32_t sb;
             uint2 cd;
             nv_block_1d<RHT, FOS>(w, sw, c, den_tab, rcp_tab, sb, cd);
-            if (valid) *reinterpret_cast<uint2 *>(codes + rr * (K >> 1) + kb * 8) = cd;
-            store_sf(sf, valid && sf_row >= 0, sb, sf_row, kb, KB, pack4);
+            if (valid) *reinterpret_cast<uint2 *>(codes + (size_t)((I)rr * (I)(K >> 1) + (I)kb * 8)) = cd;
+            store_sf_t<I>(sf, valid && sf_row >= 0, sb, (I)(sf_row >= 0 ? sf_row : 0), (I)kb, (I)KB, pack4);
         }
     }
 }
@@ -1709,7 +1711,9 @@ BSQ_DEV uint2 nv_codes_sr(const f32x2 P[8], float r, uint64_t idx0, const Philox
 
 // 1x16 blocks, rows (optionally gathered): one thread per block, rows mapped
 // to lanes as in quant_nvfp4_1d_kernel.
-template <bool RHT, bool GATHER>
+// I: the index type of the per-block offsets and Philox counters (uint32_t
+// when the output holds fewer than 2^31 elements).
+template <bool RHT, bool GATHER, typename I>
 __global__ void __launch_bounds__(256) quant_nvfp4_sr_1d_kernel(
     const uint16_t *__restrict__ x, int64_t M, int64_t K, int64_t ldx, uint32_t mask,
     const int32_t *__restrict__ row_index, const float *scale_src, int src_is_amax, float *gs_out, int write_gs,
@@ -1737,16 +1741,16 @@ __global__ void __launch_bounds__(256) quant_nvfp4_sr_1d_kernel(
             const bool valid = row_ok && kb < KB;
             const int64_t kk = kb < KB ? kb : KB - 1;
             uint32_t w[8];
-            load_words16(rp + kk * 16, w);
+            load_words16(rp + (size_t)((I)kk * 16), w);
             f32x2 P[8];
             if (RHT) rht16_u_words(w, sw, P);
             else words_to_pairs(w, P);
             const float mu = pairs_absmax3(P);
             const uint32_t sb = nv_scale_code(RHT ? __fmul_rn(mu, 0.25f) : mu, 6.0f, c.c6, c);
-            const uint2 cd = sb ? nv_codes_sr<RHT>(P, rcp_tab[sb], (uint64_t)(rr * K + kk * 16), keys, stream_id)
+            const uint2 cd = sb ? nv_codes_sr<RHT>(P, rcp_tab[sb], (uint64_t)((I)rr * (I)K + (I)kk * 16), keys, stream_id)
                                 : make_uint2(0u, 0u);
-            if (valid) *reinterpret_cast<uint2 *>(codes + rr * (K >> 1) + kb * 8) = cd;
-            store_sf(sf, valid, sb, rr, kb, KB, pack4);
+            if (valid) *reinterpret_cast<uint2 *>(codes + (size_t)((I)rr * (I)(K >> 1) + (I)kb * 8)) = cd;
+            store_sf_t<I>(sf, valid, sb, (I)rr, (I)kb, (I)KB, pack4);
         }
     }
 }
@@ -2151,9 +2155,16 @@ void launch_quant_nvfp4(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, bo
     RowMap map{lpr_shift_for(K >> 4)};
     const int grid = grid_for(M, 256 >> map.lpr_shift, num_sms * 8);
     const bool gather = row_index != nullptr, grouped = G > 0;
-#define BSQ_NV1(R, F, GA, GR)                                                                            \
-    quant_nvfp4_1d_kernel<R, F, GA, GR><<<grid, 256, 0, s>>>(x, M, K, ldx, mask, row_index, G, row_off, \
-                                                            sf_off, scale_src, sa, gs_out, wg, codes, sf, map)
+    const bool i32 = M * K < (int64_t(1) << 31);
+#define BSQ_NV1(R, F, GA, GR)                                                                                  \
+    do {                                                                                                       \
+        if (i32)                                                                                               \
+            quant_nvfp4_1d_kernel<R, F, GA, GR, uint32_t><<<grid, 256, 0, s>>>(                                \
+                x, M, K, ldx, mask, row_index, G, row_off, sf_off, scale_src, sa, gs_out, wg, codes, sf, map);    \
+        else                                                                                                   \
+            quant_nvfp4_1d_kernel<R, F, GA, GR, int64_t><<<grid, 256, 0, s>>>(                                 \
+                x, M, K, ldx, mask, row_index, G, row_off, sf_off, scale_src, sa, gs_out, wg, codes, sf, map);    \
+    } while (0)
 #define BSQ_NV1_G(R, F)                                 \
     do {                                                \
         if (gather) {                                   \
@@ -2394,11 +2405,17 @@ void launch_quant_nvfp4_sr(const uint16_t *x, int64_t M, int64_t K, int64_t ldx,
     }
     RowMap map{lpr_shift_for(K >> 4)};
     const int grid = grid_for(M, 256 >> map.lpr_shift, num_sms * 8);
-#define BSQ_NVSR(R, GA)                                                                                       \
-    quant_nvfp4_sr_1d_kernel<R, GA><<<grid, 256, 0, s>>>(x, M, K, ldx, mask, row_index, scale_src, sa, gs_out, wg, \
-                                                         keys, stream_id, codes, sf, map)
-    if (rht) { if (row_index) BSQ_NVSR(true, true); else BSQ_NVSR(true, false); }
-    else { if (row_index) BSQ_NVSR(false, true); else BSQ_NVSR(false, false); }
+#define BSQ_NVSR(R, GA, I)                                                                                     \
+    quant_nvfp4_sr_1d_kernel<R, GA, I><<<grid, 256, 0, s>>>(x, M, K, ldx, mask, row_index, scale_src, sa, gs_out, wg, \
+                                                            keys, stream_id, codes, sf, map)
+    // 32-bit offsets within a row and over the output (the source row's start stays 64-bit)
+    if (M * K < (int64_t(1) << 31)) {
+        if (rht) { if (row_index) BSQ_NVSR(true, true, uint32_t); else BSQ_NVSR(true, false, uint32_t); }
+        else { if (row_index) BSQ_NVSR(false, true, uint32_t); else BSQ_NVSR(false, false, uint32_t); }
+    } else {
+        if (rht) { if (row_index) BSQ_NVSR(true, true, int64_t); else BSQ_NVSR(true, false, int64_t); }
+        else { if (row_index) BSQ_NVSR(false, true, int64_t); else BSQ_NVSR(false, false, int64_t); }
+    }
 #undef BSQ_NVSR
 }
 

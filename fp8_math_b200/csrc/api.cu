@@ -259,6 +259,7 @@ int bsq_quant_nvfp4_gather(const void *x, int64_t T, int64_t K, int64_t ldx, con
         G < 0 || (G > 0 && (!row_off || !sf_off)))
         return BSQ_ERR_INVALID;
     if (workspace_bytes < bsq_quant_nvfp4_gather_workspace(T, K)) return BSQ_ERR_INVALID;
+    if (G > 1024) return BSQ_ERR_UNSUPPORTED;  // the scale mover keeps the offsets in shared memory
     if (!aligned16(x) || !aligned16(codes) || !aligned16(sf) || ldx % 8 || (reinterpret_cast<uintptr_t>(gs) & 3u) ||
         (reinterpret_cast<uintptr_t>(workspace) & 255u) || (amax_in && (reinterpret_cast<uintptr_t>(amax_in) & 3u)))
         return BSQ_ERR_ALIGN;

@@ -1932,10 +1932,21 @@ __global__ void __launch_bounds__(256) combine_s2f6_kernel(const int8_t *__restr
 __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4 *__restrict__ src, int64_t row_vec,
                                                           const int32_t *__restrict__ index, int64_t R,
                                                           uint4 *__restrict__ dst) {
-    const int64_t n = R * row_vec;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t r = i / row_vec, v = i - r * row_vec;
-        dst[i] = __ldg(src + (int64_t)__ldg(index + r) * row_vec + v);
+    // one warp per destination row; four 16-byte loads in flight per lane
+    const int lane = threadIdx.x & 31;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    for (int64_t row = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; row < R; row += nwarps) {
+        const uint4 *s = src + (int64_t)__ldg(index + row) * row_vec;
+        uint4 *d = dst + row * row_vec;
+        int64_t v = lane;
+        for (; v + 96 < row_vec; v += 128) {
+            const uint4 a = __ldg(s + v), b = __ldg(s + v + 32), c = __ldg(s + v + 64), e = __ldg(s + v + 96);
+            d[v] = a;
+            d[v + 32] = b;
+            d[v + 64] = c;
+            d[v + 96] = e;
+        }
+        for (; v < row_vec; v += 32) d[v] = __ldg(s + v);
     }
 }
 
@@ -2008,18 +2019,52 @@ __global__ void __launch_bounds__(256) gathered_max_kernel(const float *__restri
 // Scale words of gathered rows: output row i (SF row through the groups, as
 // the quantizer maps it) takes source row row_index[i]'s words.
 __global__ void __launch_bounds__(256) gather_sf_kernel(const uint8_t *__restrict__ sf_src, int64_t nblk,
-                                                        const int32_t *__restrict__ row_index, int64_t M, int G,
-                                                        const int32_t *__restrict__ row_off,
+                                                        DivU32 div_nw4, const int32_t *__restrict__ row_index,
+                                                        int64_t M, int G, const int32_t *__restrict__ row_off,
                                                         const int32_t *__restrict__ sf_off, uint8_t *__restrict__ sf) {
-    const int64_t nw4 = nblk >> 2;
-    const int64_t n = M * nw4;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t r = i / nw4, b4 = i - r * nw4;
-        const int64_t dst_row = G > 0 ? grouped_sf_row(r, G, row_off, sf_off) : r;
-        if (dst_row < 0) continue;
-        const int64_t src_row = __ldg(row_index + r);
-        *reinterpret_cast<uint32_t *>(sf + sf_word_offset(dst_row, b4, nblk)) =
-            __ldg(reinterpret_cast<const uint32_t *>(sf_src + sf_word_offset(src_row, b4, nblk)));
+    // The destination is written one 512-byte atom (128 rows x one 4-block
+    // group) per 128 threads: thread t writes the atom's word t, which holds
+    // tile row (t >> 2) + 32 (t & 3) (the swizzle puts row r's word at
+    // 16 (r % 32) + 4 ((r / 32) % 4)), so an atom's stores are one contiguous
+    // run.  With groups, destination row d of group e (sf_off[e] <= d <
+    // sf_off[e] + rows of e) holds routed row d - sf_off[e] + row_off[e]; the
+    // padding rows of a group's last tile are not written.
+    __shared__ int32_t s_off[1025], s_sfo[1025];
+    if (G > 0) {
+        for (int i = threadIdx.x; i <= G; i += blockDim.x) {
+            s_off[i] = __ldg(row_off + i);
+            s_sfo[i] = __ldg(sf_off + i);
+        }
+        __syncthreads();
+    }
+    const uint32_t nw4 = (uint32_t)(nblk >> 2);
+    const int64_t rows = G > 0 ? (int64_t)s_sfo[G] : M;
+    const uint32_t atoms = (uint32_t)((rows + 127) >> 7) * nw4;
+    const uint32_t t = threadIdx.x & 127;
+    const uint32_t rl = (t >> 2) + 32 * (t & 3);
+    for (uint32_t a = blockIdx.x * 2 + (threadIdx.x >> 7); a < atoms; a += gridDim.x * 2) {
+        const uint32_t tile = divu32(a, div_nw4), b4 = a - tile * nw4;
+        const int64_t dr = (int64_t)tile * 128 + rl;
+        int64_t r = dr;
+        bool valid = dr < M;
+        if (G > 0) {
+            valid = dr >= s_sfo[0];
+            if (valid) {
+                int lo = 0, hi = G;  // s_sfo[lo] <= dr < s_sfo[hi]: the last group starting at or before dr
+                while (hi - lo > 1) {
+                    const int mid = (lo + hi) >> 1;
+                    if (s_sfo[mid] <= dr) lo = mid; else hi = mid;
+                }
+                const int64_t in_grp = dr - s_sfo[lo];
+                valid = in_grp < (int64_t)(s_off[lo + 1] - s_off[lo]);
+                r = s_off[lo] + in_grp;
+            }
+        }
+        if (valid) {
+            const int64_t src_row = __ldg(row_index + r);
+            *reinterpret_cast<uint32_t *>(sf + ((size_t)a << 9) + 4 * t) =
+                __ldg(reinterpret_cast<const uint32_t *>(sf_src + sf_word_offset(src_row, b4, nblk)));
+        }
     }
 }
 
@@ -2437,8 +2482,8 @@ void launch_combine_s2f6(const int8_t *codes, const uint8_t *sf, int64_t K, cons
 void launch_gather_rows(const void *src, int64_t row_bytes, const int32_t *index, int64_t R, void *dst, int num_sms,
                         cudaStream_t s) {
     const int64_t vec = row_bytes / 16;
-    gather_rows_kernel<<<grid_for(R * vec, 256, num_sms * 8), 256, 0, s>>>(static_cast<const uint4 *>(src), vec, index,
-                                                                          R, static_cast<uint4 *>(dst));
+    gather_rows_kernel<<<grid_for(R, 8, num_sms * 8), 256, 0, s>>>(static_cast<const uint4 *>(src), vec, index, R,
+                                                                    static_cast<uint4 *>(dst));
 }
 
 void launch_sf_to_rows(const uint8_t *sf, int64_t rows, int64_t nblk, uint8_t *out, int num_sms, cudaStream_t s) {
@@ -2464,8 +2509,10 @@ void launch_gathered_max(const float *rowmax, const int32_t *row_index, int64_t 
 
 void launch_gather_sf(const uint8_t *sf_src, int64_t nblk, const int32_t *row_index, int64_t M, int G,
                       const int32_t *row_off, const int32_t *sf_off, uint8_t *sf, int num_sms, cudaStream_t s) {
-    gather_sf_kernel<<<grid_for(M * (nblk >> 2), 256, num_sms * 8), 256, 0, s>>>(sf_src, nblk, row_index, M, G, row_off,
-                                                                                 sf_off, sf);
+    // destination rows: M, or with groups at most M + 128 G (each group padded to 128 rows)
+    const int64_t atoms = ((M + 128 * (int64_t)G + 127) >> 7) * (nblk >> 2);
+    gather_sf_kernel<<<grid_for(atoms, 2, num_sms * 8), 256, 0, s>>>(sf_src, nblk, divu32_for((uint32_t)(nblk >> 2)),
+                                                                      row_index, M, G, row_off, sf_off, sf);
 }
 
 void launch_rht(const uint16_t *x, uint16_t *y, int64_t M, int64_t K, int64_t ldx, int64_t ldy, uint32_t mask,

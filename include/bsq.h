@@ -175,7 +175,7 @@ BSQ_API int bsq_quant_nvfp4(const void *x_bf16, int64_t M, int64_t K, int64_t ld
  * rows.  workspace: device memory of at least
  * bsq_quant_nvfp4_gather_workspace(T, K) bytes, 256-byte aligned, owned by
  * the caller (its contents are scratch); every row_index value must be in
- * [0, T).  K % 64 == 0. */
+ * [0, T).  K % 64 == 0.  G <= 1024 (BSQ_ERR_UNSUPPORTED above). */
 BSQ_API size_t bsq_quant_nvfp4_gather_workspace(int64_t T, int64_t K);
 BSQ_API int bsq_quant_nvfp4_gather(const void *x_bf16, int64_t T, int64_t K, int64_t ldx,
                                    const int32_t *row_index_dev, int64_t M, int four_over_six, int rht_enable,

@@ -116,6 +116,18 @@ def test_kernel_choice_knobs_validate(lib):
         assert L.bsq_debug_kernel_choice(knob, -1) == lib.BSQ_OK
 
 
+def test_gathered_quantize_bounds_the_group_count(lib):
+    """bsq_quant_nvfp4_gather moves scale words with the group offsets held in
+    shared memory (at most 1024 groups): more is refused on the host, before
+    any CUDA call.  The pointers are placeholders that are never dereferenced."""
+    L = lib.lib()
+    p = 256
+    ws = lib.bsq_quant_nvfp4_gather_workspace(4, 64)
+    args = lambda G: (p, 4, 64, 64, p, 4, 0, 0, 0, G, p, p, None, p, p, p, p, ws, None)
+    assert L.bsq_quant_nvfp4_gather(*args(1025)) == lib.BSQ_ERR_UNSUPPORTED
+    assert L.bsq_quant_nvfp4_gather(*args(-1)) == lib.BSQ_ERR_INVALID
+
+
 def test_noalloc_rejects_requests_beyond_its_scratch(lib):
     """The no-allocation entry point holds one partial maximum per 65536
     elements in a 4096-word array (one word is the counter): 4095 CTAs are

@@ -2019,16 +2019,18 @@ __global__ void __launch_bounds__(256) gathered_max_kernel(const float *__restri
 // Scale words of gathered rows: output row i (SF row through the groups, as
 // the quantizer maps it) takes source row row_index[i]'s words.
 __global__ void __launch_bounds__(256) gather_sf_kernel(const uint8_t *__restrict__ sf_src, int64_t nblk,
-                                                        DivU32 div_nw4, const int32_t *__restrict__ row_index,
+                                                        DivU32 div_ng, const int32_t *__restrict__ row_index,
                                                         int64_t M, int G, const int32_t *__restrict__ row_off,
                                                         const int32_t *__restrict__ sf_off, uint8_t *__restrict__ sf) {
-    // The destination is written one 512-byte atom (128 rows x one 4-block
-    // group) per 128 threads: thread t writes the atom's word t, which holds
-    // tile row (t >> 2) + 32 (t & 3) (the swizzle puts row r's word at
-    // 16 (r % 32) + 4 ((r / 32) % 4)), so an atom's stores are one contiguous
-    // run.  With groups, destination row d of group e (sf_off[e] <= d <
-    // sf_off[e] + rows of e) holds routed row d - sf_off[e] + row_off[e]; the
-    // padding rows of a group's last tile are not written.
+    // The destination is written in units of four 512-byte atoms (128 rows x
+    // four 4-block groups) per 128 threads: thread t writes word t of each of
+    // the unit's atoms, which holds tile row (t >> 2) + 32 (t & 3) (the
+    // swizzle puts row r's word at 16 (r % 32) + 4 ((r / 32) % 4)), so each
+    // atom's stores are one contiguous run, and the thread's four source
+    // words (one row, four groups) are loaded together.  With groups,
+    // destination row d of group e (sf_off[e] <= d < sf_off[e] + rows of e)
+    // holds routed row d - sf_off[e] + row_off[e]; the padding rows of a
+    // group's last tile are not written.
     __shared__ int32_t s_off[1025], s_sfo[1025];
     if (G > 0) {
         for (int i = threadIdx.x; i <= G; i += blockDim.x) {
@@ -2037,13 +2039,13 @@ __global__ void __launch_bounds__(256) gather_sf_kernel(const uint8_t *__restric
         }
         __syncthreads();
     }
-    const uint32_t nw4 = (uint32_t)(nblk >> 2);
+    const uint32_t nw4 = (uint32_t)(nblk >> 2), ng = (nw4 + 3) >> 2;  // 4-block groups, units per tile
     const int64_t rows = G > 0 ? (int64_t)s_sfo[G] : M;
-    const uint32_t atoms = (uint32_t)((rows + 127) >> 7) * nw4;
+    const uint32_t units = (uint32_t)((rows + 127) >> 7) * ng;
     const uint32_t t = threadIdx.x & 127;
     const uint32_t rl = (t >> 2) + 32 * (t & 3);
-    for (uint32_t a = blockIdx.x * 2 + (threadIdx.x >> 7); a < atoms; a += gridDim.x * 2) {
-        const uint32_t tile = divu32(a, div_nw4), b4 = a - tile * nw4;
+    for (uint32_t u = blockIdx.x * 2 + (threadIdx.x >> 7); u < units; u += gridDim.x * 2) {
+        const uint32_t tile = divu32(u, div_ng), b40 = (u - tile * ng) * 4;
         const int64_t dr = (int64_t)tile * 128 + rl;
         int64_t r = dr;
         bool valid = dr < M;
@@ -2062,8 +2064,16 @@ __global__ void __launch_bounds__(256) gather_sf_kernel(const uint8_t *__restric
         }
         if (valid) {
             const int64_t src_row = __ldg(row_index + r);
-            *reinterpret_cast<uint32_t *>(sf + ((size_t)a << 9) + 4 * t) =
-                __ldg(reinterpret_cast<const uint32_t *>(sf_src + sf_word_offset(src_row, b4, nblk)));
+            const uint8_t *src = sf_src + sf_word_offset(src_row, b40, nblk);  // group b40; b40 + i is 512 i further
+            uint8_t *dst = sf + (((size_t)tile * nw4 + b40) << 9) + 4 * t;
+            const uint32_t n = nw4 - b40 < 4 ? nw4 - b40 : 4;
+            uint32_t w[4];
+#pragma unroll
+            for (int i = 0; i < 4; i++)
+                if ((uint32_t)i < n) w[i] = __ldg(reinterpret_cast<const uint32_t *>(src + 512 * i));
+#pragma unroll
+            for (int i = 0; i < 4; i++)
+                if ((uint32_t)i < n) *reinterpret_cast<uint32_t *>(dst + 512 * i) = w[i];
         }
     }
 }
@@ -2510,9 +2520,10 @@ void launch_gathered_max(const float *rowmax, const int32_t *row_index, int64_t 
 void launch_gather_sf(const uint8_t *sf_src, int64_t nblk, const int32_t *row_index, int64_t M, int G,
                       const int32_t *row_off, const int32_t *sf_off, uint8_t *sf, int num_sms, cudaStream_t s) {
     // destination rows: M, or with groups at most M + 128 G (each group padded to 128 rows)
-    const int64_t atoms = ((M + 128 * (int64_t)G + 127) >> 7) * (nblk >> 2);
-    gather_sf_kernel<<<grid_for(atoms, 2, num_sms * 8), 256, 0, s>>>(sf_src, nblk, divu32_for((uint32_t)(nblk >> 2)),
-                                                                      row_index, M, G, row_off, sf_off, sf);
+    const int64_t ng = ((nblk >> 2) + 3) >> 2;
+    const int64_t units = ((M + 128 * (int64_t)G + 127) >> 7) * ng;
+    gather_sf_kernel<<<grid_for(units, 2, num_sms * 8), 256, 0, s>>>(sf_src, nblk, divu32_for((uint32_t)ng), row_index,
+                                                                      M, G, row_off, sf_off, sf);
 }
 
 void launch_rht(const uint16_t *x, uint16_t *y, int64_t M, int64_t K, int64_t ldx, int64_t ldy, uint32_t mask,

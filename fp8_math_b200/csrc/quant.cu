@@ -1678,6 +1678,52 @@ __global__ void __launch_bounds__(256) quant_mxfp4_row_kernel(
     }
 }
 
+// Row-wise MXFP4 for a contiguous tensor whose rows hold a multiple of 1024
+// elements: the MXFP8 span kernel's mapping (a warp per 1024-element span of
+// one row, lane l loads the 8-element chunks l, l + 32, l + 64, l + 96, four
+// 16-byte loads in flight; lanes 4j .. 4j + 3 share a block of 32), with one
+// 32-bit code store per chunk.  The SR draw index of a chunk is its flat
+// position, as in quant_mxfp4_row_kernel.
+template <bool SR>
+__global__ void __launch_bounds__(256) quant_mxfp4_row_span_kernel(
+    const uint16_t *__restrict__ x, uint32_t nspan, int64_t K, DivU32 div_spr, const __grid_constant__ PhiloxKeys keys,
+    uint32_t stream_id, uint8_t *__restrict__ codes, uint8_t *__restrict__ sf) {
+    const int lane = threadIdx.x & 31;
+    const uint32_t spr = (uint32_t)(K >> 10);  // spans per row
+    const int64_t KB = K >> 5;
+    const uint32_t nwarps = (gridDim.x * blockDim.x) >> 5;
+    const bool sf_lane = (lane & 3) == 0;
+    for (uint32_t sp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; sp < nspan; sp += nwarps) {
+        const int64_t e0 = (int64_t)sp << 10;
+        const uint4 *src = reinterpret_cast<const uint4 *>(x + e0) + lane;
+        uint4 raw[4];
+#pragma unroll
+        for (int h = 0; h < 4; h++) raw[h] = __ldg(src + 32 * h);
+        const uint32_t row = divu32(sp, div_spr), seg = sp - row * spr;
+        // scale byte of block 32 seg + 8 h + lane / 4: word 8 seg + 2 h + lane / 16 of the row
+        uint8_t *sfp = sf + sf_word_offset(row, (int64_t)seg * 8 + (lane >> 4), KB) + ((lane >> 2) & 3);
+        uint32_t *dst = reinterpret_cast<uint32_t *>(codes + (e0 >> 1)) + lane;
+        const uint64_t chunk0 = ((uint64_t)sp << 7) + lane;
+#pragma unroll
+        for (int h = 0; h < 4; h++) {
+            const uint32_t w[4] = {raw[h].x, raw[h].y, raw[h].z, raw[h].w};
+            float v[8];
+#pragma unroll
+            for (int i = 0; i < 4; i++) {
+                v[2 * i] = bf16_lo(w[i]);
+                v[2 * i + 1] = bf16_hi(w[i]);
+            }
+            float m = fmax3(fmax3(fabsf(v[0]), fabsf(v[1]), fabsf(v[2])), fmax3(fabsf(v[3]), fabsf(v[4]), fabsf(v[5])),
+                            fmaxf(fabsf(v[6]), fabsf(v[7])));
+            m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+            m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+            const uint32_t sb = mx4_scale_code(m);
+            dst[32 * h] = mx4_encode8<SR>(v, m == 0.0f, sb, chunk0 + 32 * h, keys, stream_id);
+            if (sf_lane) sfp[h * 1024] = (uint8_t)sb;
+        }
+    }
+}
+
 // ===================================================================== NVFP4, stochastic rounding
 // NVFP4 with the elements rounded stochastically: block scales and s_g as
 // in the nearest-even kernels above; each element q = y * r (y = RN(u / 4)
@@ -2426,6 +2472,18 @@ void launch_requant_nvfp4_mxfp8(const uint8_t *codes_in, const uint8_t *sf_in, c
 void launch_quant_mxfp4(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, bool sr, uint64_t seed,
                         uint32_t stream_id, uint8_t *codes, uint8_t *sf, int num_sms, cudaStream_t s) {
     const PhiloxKeys keys = philox_keys((uint32_t)seed, (uint32_t)(seed >> 32));
+    if (ldx == K && K % 1024 == 0 && M * (K >> 10) < (int64_t(1) << 31)) {
+        const uint32_t nspan = (uint32_t)(M * (K >> 10));
+        const DivU32 dspr = divu32_for((uint32_t)(K >> 10));
+        if (sr) {
+            const int grid = grid_for(nspan, 8, resident_ctas<quant_mxfp4_row_span_kernel<true>>(num_sms));
+            quant_mxfp4_row_span_kernel<true><<<grid, 256, 0, s>>>(x, nspan, K, dspr, keys, stream_id, codes, sf);
+        } else {
+            const int grid = grid_for(nspan, 8, resident_ctas<quant_mxfp4_row_span_kernel<false>>(num_sms));
+            quant_mxfp4_row_span_kernel<false><<<grid, 256, 0, s>>>(x, nspan, K, dspr, keys, stream_id, codes, sf);
+        }
+        return;
+    }
     RowMap map{lpr_shift_for(K >> 3)};
     if (map.lpr_shift < 2) map.lpr_shift = 2;  // 4 lanes per block of 32
     const int grid = grid_for(M, 256 >> map.lpr_shift, num_sms * 8);

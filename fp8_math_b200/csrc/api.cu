@@ -437,6 +437,7 @@ int bsq_gather_rows(const void *src, int64_t row_bytes, const int32_t *index, in
 
 int bsq_sf_to_rows(const uint8_t *sf, int64_t rows, int64_t nblk, uint8_t *out, void *stream) {
     if (!sf || !out || rows < 0 || nblk < 0) return BSQ_ERR_INVALID;
+    if (rows * nblk >= (int64_t(1) << 31)) return BSQ_ERR_UNSUPPORTED;  // 32-bit indexing
     DeviceState *d;
     if (int st = device_state(&d)) return st;
     if (rows == 0 || nblk == 0) return BSQ_OK;
@@ -447,6 +448,7 @@ int bsq_sf_to_rows(const uint8_t *sf, int64_t rows, int64_t nblk, uint8_t *out, 
 int bsq_sf_from_rows(const uint8_t *in, int64_t rows, int64_t nblk, int G, const int32_t *row_off,
                      const int32_t *sf_row_off, uint8_t *sf, void *stream) {
     if (!in || !sf || rows < 0 || nblk < 0 || G < 0 || (G > 0 && (!row_off || !sf_row_off))) return BSQ_ERR_INVALID;
+    if (rows * nblk >= (int64_t(1) << 31)) return BSQ_ERR_UNSUPPORTED;  // 32-bit indexing
     DeviceState *d;
     if (int st = device_state(&d)) return st;
     if (rows == 0 || nblk == 0) return BSQ_OK;

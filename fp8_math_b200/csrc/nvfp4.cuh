@@ -132,23 +132,9 @@ BSQ_DEV void nv_block_1d(const uint32_t w[8], const uint32_t sw[8], const NvScal
 
 // Writes the scale byte of a unit: packs 4 consecutive blocks into one word
 // when the row's block count is a multiple of 4 (lanes 4j..4j+3 hold blocks
-// 4i..4i+3 of one row), else stores the byte.
-BSQ_DEV void store_sf(uint8_t *sf, bool valid, uint32_t sb, int64_t sf_row, int64_t kb, int64_t KB, bool pack4) {
-    if (pack4) {
-        uint32_t b1 = __shfl_down_sync(0xFFFFFFFFu, sb, 1);
-        uint32_t b2 = __shfl_down_sync(0xFFFFFFFFu, sb, 2);
-        uint32_t b3 = __shfl_down_sync(0xFFFFFFFFu, sb, 3);
-        if (valid && (threadIdx.x & 3) == 0) {
-            uint32_t w = (sb & 0xFFu) | ((b1 & 0xFFu) << 8) | ((b2 & 0xFFu) << 16) | ((b3 & 0xFFu) << 24);
-            *reinterpret_cast<uint32_t *>(sf + sf_word_offset(sf_row, kb >> 2, KB)) = w;
-        }
-    } else if (valid) {
-        sf[sf_offset(sf_row, kb, KB)] = (uint8_t)sb;
-    }
-}
-
-// store_sf with the offset in the index type I (uint32_t where the scale
-// buffer holds fewer than 2^31 bytes); sf_row is read only when valid.
+// 4i..4i+3 of one row), else stores the byte.  The offset is computed in the
+// index type I (uint32_t where the scale buffer holds fewer than 2^31 bytes);
+// sf_row is read only when valid.
 template <typename I>
 BSQ_DEV void store_sf_t(uint8_t *sf, bool valid, uint32_t sb, I sf_row, I kb, I KB, bool pack4) {
     if (pack4) {

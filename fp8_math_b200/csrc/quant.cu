@@ -1996,11 +1996,13 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4 *__restric
     }
 }
 
+// (i = r nblk + b: the row by a precomputed multiply-shift divider, 32-bit
+// indices: the entry points accept rows * nblk < 2^31 only)
 __global__ void __launch_bounds__(256) sf_to_rows_kernel(const uint8_t *__restrict__ sf, int64_t rows, int64_t nblk,
-                                                         uint8_t *__restrict__ out) {
-    const int64_t n = rows * nblk;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t r = i / nblk, b = i - r * nblk;
+                                                         DivU32 div_nblk, uint8_t *__restrict__ out) {
+    const uint32_t n = (uint32_t)(rows * nblk), nb = (uint32_t)nblk;
+    for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
+        const uint32_t r = divu32(i, div_nblk), b = i - r * nb;
         out[i] = __ldg(sf + sf_offset(r, b, nblk));
     }
 }
@@ -2009,13 +2011,13 @@ __global__ void __launch_bounds__(256) sf_to_rows_kernel(const uint8_t *__restri
 // of group e goes to SF row r - row_off[e] + sf_row_off[e] (rows outside
 // every group are skipped).
 __global__ void __launch_bounds__(256) sf_from_rows_kernel(const uint8_t *__restrict__ in, int64_t rows, int64_t nblk,
-                                                           int G, const int32_t *__restrict__ row_off,
+                                                           DivU32 div_nblk, int G, const int32_t *__restrict__ row_off,
                                                            const int32_t *__restrict__ sf_off,
                                                            uint8_t *__restrict__ sf) {
-    const int64_t n = rows * nblk;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t r = i / nblk, b = i - r * nblk;
-        const int64_t sr = G > 0 ? grouped_sf_row(r, G, row_off, sf_off) : r;
+    const uint32_t n = (uint32_t)(rows * nblk), nb = (uint32_t)nblk;
+    for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
+        const uint32_t r = divu32(i, div_nblk), b = i - r * nb;
+        const int64_t sr = G > 0 ? grouped_sf_row(r, G, row_off, sf_off) : (int64_t)r;
         if (sr >= 0) sf[sf_offset(sr, b, nblk)] = __ldg(in + i);
     }
 }
@@ -2555,12 +2557,14 @@ void launch_gather_rows(const void *src, int64_t row_bytes, const int32_t *index
 }
 
 void launch_sf_to_rows(const uint8_t *sf, int64_t rows, int64_t nblk, uint8_t *out, int num_sms, cudaStream_t s) {
-    sf_to_rows_kernel<<<grid_for(rows * nblk, 256, num_sms * 8), 256, 0, s>>>(sf, rows, nblk, out);
+    sf_to_rows_kernel<<<grid_for(rows * nblk, 256, num_sms * 8), 256, 0, s>>>(sf, rows, nblk,
+                                                                             divu32_for((uint32_t)nblk), out);
 }
 
 void launch_sf_from_rows(const uint8_t *in, int64_t rows, int64_t nblk, int G, const int32_t *row_off,
                          const int32_t *sf_off, uint8_t *sf, int num_sms, cudaStream_t s) {
-    sf_from_rows_kernel<<<grid_for(rows * nblk, 256, num_sms * 8), 256, 0, s>>>(in, rows, nblk, G, row_off, sf_off, sf);
+    sf_from_rows_kernel<<<grid_for(rows * nblk, 256, num_sms * 8), 256, 0, s>>>(
+        in, rows, nblk, divu32_for((uint32_t)nblk), G, row_off, sf_off, sf);
 }
 
 void launch_row_absmax(const uint16_t *x, int64_t T, int64_t K, int64_t ldx, bool rht, uint32_t mask, float *rowmax,

@@ -314,7 +314,8 @@ BSQ_API int bsq_combine_s2f6(const int8_t *codes_dev, const uint8_t *sf_dev, int
  * bsq_sf_from_rows: plain rows back into the swizzled layout; with G > 0,
  * row r of group e (device int32 offsets as for bsq_quant_nvfp4) goes to SF
  * row r - row_offsets[e] + sf_row_offsets[e] (the grouped GEMM's layout).
- * Padding bytes of the swizzled buffer are not written. */
+ * Padding bytes of the swizzled buffer are not written.  Both take
+ * rows * nblk < 2^31 (BSQ_ERR_UNSUPPORTED above). */
 BSQ_API int bsq_gather_rows(const void *src_dev, int64_t row_bytes, const int32_t *index_dev, int64_t R,
                             void *dst_dev, void *stream);
 BSQ_API int bsq_sf_to_rows(const uint8_t *sf_dev, int64_t rows, int64_t nblk, uint8_t *rows_out_dev, void *stream);

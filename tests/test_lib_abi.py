@@ -128,6 +128,16 @@ def test_gathered_quantize_bounds_the_group_count(lib):
     assert L.bsq_quant_nvfp4_gather(*args(-1)) == lib.BSQ_ERR_INVALID
 
 
+def test_scale_row_movers_bound_their_size(lib):
+    """bsq_sf_to_rows / bsq_sf_from_rows index with 32-bit arithmetic and
+    refuse rows * nblk >= 2^31 on the host, before any CUDA call (the
+    pointers are placeholders that are never dereferenced)."""
+    L = lib.lib()
+    assert L.bsq_sf_to_rows(256, 1 << 20, 1 << 11, 256, None) == lib.BSQ_ERR_UNSUPPORTED
+    assert L.bsq_sf_from_rows(256, 1 << 20, 1 << 11, 0, None, None, 256, None) == lib.BSQ_ERR_UNSUPPORTED
+    assert L.bsq_sf_to_rows(256, -1, 4, 256, None) == lib.BSQ_ERR_INVALID
+
+
 def test_noalloc_rejects_requests_beyond_its_scratch(lib):
     """The no-allocation entry point holds one partial maximum per 65536
     elements in a 4096-word array (one word is the counter): 4095 CTAs are
